@@ -1,0 +1,218 @@
+"""CPU oracle for exact softmax attention (forward and backward) in fp64.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and
+the CPU-baseline leg of ``bench.py`` may import this package.  It shares no
+code with the GPU library (no common kernels, headers, helpers or constants)
+and never imports it.
+
+The arithmetic lives in ``oracle.c`` (plain C, fp64, one thread per
+independent head); this module compiles it with gcc on first use and wraps
+it for numpy arrays.  Every function follows the plain definition of
+attention given on the pages ("flash attention io aware", section "The
+Memory Bandwidth Bottleneck", steps 1-3: S = QK^T, P = softmax(S), O = PV),
+with the softmax statistics kept as one natural-log logsumexp per row
+("FlashAttention" glossary, recomputation paragraph: the backward pass keeps
+only the normalisation statistics).  The backward formulas are the calculus
+of softmax; ``oracle.c`` writes them out in its header.
+
+Parity status of each function (what pins it, see tests/test_oracle_pins.py):
+  fwd, fwd_rows          closed forms (Q = 0, one-hot keys, causal row 0),
+                         hand-derived golden values, torch fp64 SDPA,
+                         brute-force Python loops
+  fwd_online             equal to the two-pass form within 1e-12 (fp64)
+  bwd, bwd_rows,         central finite differences of the forward,
+  bwd_cols               closed forms at Q = 0, torch fp64 autograd,
+                         gradient invariants, hand-derived golden values
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+SOURCE = os.path.join(_HERE, "oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_default = None
+
+_i64 = ctypes.c_int64
+_dp = ctypes.POINTER(ctypes.c_double)
+_ip = ctypes.POINTER(ctypes.c_int64)
+
+
+def build(force: bool = False, src: str = SOURCE, out: str = _LIB_PATH) -> str:
+    """Compile ``src`` (default oracle.c) into the shared library ``out`` (gcc -O2, no fast-math)."""
+    if force or not os.path.exists(out) or os.path.getmtime(out) < os.path.getmtime(src):
+        tmp = out + f".tmp{os.getpid()}"
+        cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-pthread", src, "-o", tmp, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, out)
+    return out
+
+
+def _f64(a) -> np.ndarray:
+    """Exact upcast of an array (numpy or torch CPU tensor) to contiguous fp64."""
+    if hasattr(a, "detach"):
+        a = a.detach().cpu().double().numpy()
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(_dp)
+
+
+def _dims(q, k):
+    B, Hq, N, d = q.shape
+    Bk, Hkv, Nk, dk = k.shape
+    if (Bk, Nk, dk) != (B, N, d) or Hq % Hkv:
+        raise ValueError(f"incompatible shapes q{q.shape} k{k.shape}")
+    return B, Hq, Hkv, N, d
+
+
+class Oracle:
+    """numpy-facing wrapper of one compiled copy of the oracle library."""
+
+    def __init__(self, lib_path: str):
+        lib = ctypes.CDLL(lib_path)
+        common = [_i64, _i64, _i64, _i64, _i64, ctypes.c_double, ctypes.c_int]
+        lib.oracle_fwd.argtypes = [_dp, _dp, _dp, _dp, _dp] + common + [ctypes.c_int]
+        lib.oracle_fwd_rows.argtypes = [_dp, _dp, _dp, _ip, _i64, _dp, _dp] + common + [ctypes.c_int]
+        lib.oracle_fwd_online.argtypes = [_dp, _dp, _dp, _dp, _dp] + common + [_i64, ctypes.c_int]
+        lib.oracle_bwd.argtypes = [_dp, _dp, _dp, _dp, _dp, _dp, _dp] + common + [ctypes.c_int]
+        lib.oracle_bwd_rows.argtypes = [_dp, _dp, _dp, _dp, _ip, _i64, _dp] + common + [ctypes.c_int]
+        lib.oracle_bwd_cols.argtypes = ([_dp, _dp, _dp, _dp, _i64, _i64, _ip, _i64, _dp, _dp]
+                                        + common + [ctypes.c_int])
+        lib.oracle_num_threads.argtypes = [ctypes.c_int]
+        for f in ("oracle_fwd", "oracle_fwd_rows", "oracle_fwd_online", "oracle_bwd",
+                  "oracle_bwd_rows", "oracle_bwd_cols", "oracle_num_threads"):
+            getattr(lib, f).restype = ctypes.c_int
+        self.lib = lib
+
+    def num_threads(self, nthreads: int = 0) -> int:
+        """Threads the oracle uses for ``nthreads`` (<= 0: every online core)."""
+        return self.lib.oracle_num_threads(nthreads)
+
+    def fwd(self, q, k, v, scale: float, causal: bool, nthreads: int = 0):
+        """O [B,Hq,N,d] and lse [B,Hq,N] (natural log), materialising N x N per head."""
+        q, k, v = _f64(q), _f64(k), _f64(v)
+        B, Hq, Hkv, N, d = _dims(q, k)
+        o = np.zeros((B, Hq, N, d))
+        lse = np.zeros((B, Hq, N))
+        rc = self.lib.oracle_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                                 B, Hq, Hkv, N, d, float(scale), int(causal), nthreads)
+        if rc:
+            raise ValueError(f"oracle_fwd rejected its arguments ({rc})")
+        return o, lse
+
+    def fwd_rows(self, q, k, v, rows, scale: float, causal: bool, nthreads: int = 0):
+        """O and lse of the query rows ``rows`` of every head: [B,Hq,R,d], [B,Hq,R]."""
+        q, k, v = _f64(q), _f64(k), _f64(v)
+        B, Hq, Hkv, N, d = _dims(q, k)
+        rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+        R = rows.size
+        o = np.zeros((B, Hq, R, d))
+        lse = np.zeros((B, Hq, R))
+        rc = self.lib.oracle_fwd_rows(_ptr(q), _ptr(k), _ptr(v), rows.ctypes.data_as(_ip), R,
+                                      _ptr(o), _ptr(lse), B, Hq, Hkv, N, d, float(scale),
+                                      int(causal), nthreads)
+        if rc:
+            raise ValueError(f"oracle_fwd_rows rejected its arguments ({rc})")
+        return o, lse
+
+    def fwd_online(self, q, k, v, scale: float, causal: bool, block: int = 128, nthreads: int = 0):
+        """O and lse by the one-pass blocked online softmax (not the definition)."""
+        q, k, v = _f64(q), _f64(k), _f64(v)
+        B, Hq, Hkv, N, d = _dims(q, k)
+        o = np.zeros((B, Hq, N, d))
+        lse = np.zeros((B, Hq, N))
+        rc = self.lib.oracle_fwd_online(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                                        B, Hq, Hkv, N, d, float(scale), int(causal), int(block),
+                                        nthreads)
+        if rc:
+            raise ValueError(f"oracle_fwd_online rejected its arguments ({rc})")
+        return o, lse
+
+    def bwd(self, q, k, v, dout, scale: float, causal: bool, nthreads: int = 0):
+        """dQ [B,Hq,N,d], dK, dV [B,Hkv,N,d] (dK, dV summed over each query group)."""
+        q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
+        B, Hq, Hkv, N, d = _dims(q, k)
+        dq = np.zeros((B, Hq, N, d))
+        dk = np.zeros((B, Hkv, N, d))
+        dv = np.zeros((B, Hkv, N, d))
+        rc = self.lib.oracle_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(dq), _ptr(dk),
+                                 _ptr(dv), B, Hq, Hkv, N, d, float(scale), int(causal), nthreads)
+        if rc:
+            raise ValueError(f"oracle_bwd rejected its arguments ({rc})")
+        return dq, dk, dv
+
+    def bwd_rows(self, q, k, v, dout, rows, scale: float, causal: bool, nthreads: int = 0):
+        """dQ of the query rows ``rows`` of every head: [B,Hq,R,d]."""
+        q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
+        B, Hq, Hkv, N, d = _dims(q, k)
+        rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+        R = rows.size
+        dq = np.zeros((B, Hq, R, d))
+        rc = self.lib.oracle_bwd_rows(_ptr(q), _ptr(k), _ptr(v), _ptr(dout),
+                                      rows.ctypes.data_as(_ip), R, _ptr(dq),
+                                      B, Hq, Hkv, N, d, float(scale), int(causal), nthreads)
+        if rc:
+            raise ValueError(f"oracle_bwd_rows rejected its arguments ({rc})")
+        return dq
+
+    def bwd_cols(self, q, k, v, dout, b: int, hkv: int, cols, scale: float, causal: bool,
+                 nthreads: int = 0):
+        """dK and dV of key rows ``cols`` of kv head (b, hkv): [C,d] each."""
+        q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
+        B, Hq, Hkv, N, d = _dims(q, k)
+        cols = np.ascontiguousarray(np.asarray(cols, dtype=np.int64))
+        C = cols.size
+        dk = np.zeros((C, d))
+        dv = np.zeros((C, d))
+        rc = self.lib.oracle_bwd_cols(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), int(b), int(hkv),
+                                      cols.ctypes.data_as(_ip), C, _ptr(dk), _ptr(dv),
+                                      B, Hq, Hkv, N, d, float(scale), int(causal), nthreads)
+        if rc:
+            raise ValueError(f"oracle_bwd_cols rejected its arguments ({rc})")
+        return dk, dv
+
+
+def default() -> Oracle:
+    """The oracle compiled from oracle.c (built on first use)."""
+    global _default
+    with _lock:
+        if _default is None:
+            _default = Oracle(build())
+    return _default
+
+
+def num_threads(nthreads: int = 0) -> int:
+    return default().num_threads(nthreads)
+
+
+def fwd(*a, **kw):
+    return default().fwd(*a, **kw)
+
+
+def fwd_rows(*a, **kw):
+    return default().fwd_rows(*a, **kw)
+
+
+def fwd_online(*a, **kw):
+    return default().fwd_online(*a, **kw)
+
+
+def bwd(*a, **kw):
+    return default().bwd(*a, **kw)
+
+
+def bwd_rows(*a, **kw):
+    return default().bwd_rows(*a, **kw)
+
+
+def bwd_cols(*a, **kw):
+    return default().bwd_cols(*a, **kw)

@@ -1,0 +1,531 @@
+/*
+ * CPU oracle for exact softmax attention, forward and backward, in fp64.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the CPU
+ * baseline leg of the benchmark load this file's library.  The GPU library
+ * shares no code with it and never calls it.
+ *
+ * What it computes (the plain definition, no blocking, no fusion):
+ *   the pages define attention as S = QK^T, P = softmax(S) row by row,
+ *   O = PV ("flash attention io aware", section "The Memory Bandwidth
+ *   Bottleneck", steps 1-3), and say the tiled method reaches exactly this
+ *   result ("FlashAttention" glossary, online-softmax paragraph: output
+ *   identical to the two-pass version).  The statistics kept for the
+ *   backward pass are the running max m and sum l ("FlashAttention"
+ *   glossary, recomputation paragraph); they are stored here as one
+ *   logsumexp per row, lse = m + ln(l), natural log.
+ *
+ *   For batch b, query head h, kv head g = h / (Hq / Hkv) (contiguous groups,
+ *   "Flash Attention" glossary, grouped-query attention paragraph):
+ *     s_ij  = scale * sum_c q_ic k_jc,   s_ij = -inf for j > i when causal
+ *     m_i   = max_j s_ij                                (pass 1)
+ *     l_i   = sum_j exp(s_ij - m_i)                     (pass 2)
+ *     P_ij  = exp(s_ij - m_i) / l_i
+ *     O_i   = sum_j P_ij v_j
+ *     lse_i = m_i + ln(l_i)
+ *
+ *   Backward (the pages print no formula; this is the calculus of
+ *   y = softmax(x) applied to the definition above, summed over the query
+ *   heads of a group for dK and dV):
+ *     dV_j  = sum_i P_ij dO_i
+ *     dP_ij = dO_i . v_j
+ *     D_i   = sum_j P_ij dP_ij
+ *     dS_ij = P_ij (dP_ij - D_i)
+ *     dQ_i  = scale * sum_j dS_ij k_j
+ *     dK_j  = scale * sum_i dS_ij q_i
+ *
+ * Layouts: all arrays are dense row-major fp64.
+ *   q, o, dout, dq : [B][Hq][N][d]
+ *   k, v, dk, dv   : [B][Hkv][N][d]
+ *   lse            : [B][Hq][N]
+ *
+ * Threads: work items are independent (one head, or one kv head with its
+ * query group), handed out through an atomic counter; nthreads <= 0 means
+ * every online core.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#include <unistd.h>
+
+typedef int64_t i64;
+
+/* ------------------------------------------------------------------------ */
+/* a minimal thread pool: run fn(ctx, item) for item in [0, n_items)          */
+
+typedef void (*item_fn)(void *ctx, i64 item);
+
+typedef struct {
+    item_fn fn;
+    void *ctx;
+    i64 n_items;
+    i64 next; /* accessed with __atomic builtins */
+} pool_t;
+
+static void *pool_worker(void *arg) {
+    pool_t *p = (pool_t *)arg;
+    for (;;) {
+        i64 it = __atomic_fetch_add(&p->next, 1, __ATOMIC_RELAXED);
+        if (it >= p->n_items) break;
+        p->fn(p->ctx, it);
+    }
+    return NULL;
+}
+
+static int resolve_threads(int nthreads) {
+    if (nthreads > 0) return nthreads;
+    long n = sysconf(_SC_NPROCESSORS_ONLN);
+    return n > 0 ? (int)n : 1;
+}
+
+static void run_pool(item_fn fn, void *ctx, i64 n_items, int nthreads) {
+    pool_t p = {fn, ctx, n_items, 0};
+    int nt = resolve_threads(nthreads);
+    if (nt > n_items) nt = (int)(n_items > 0 ? n_items : 1);
+    if (nt <= 1) {
+        pool_worker(&p);
+        return;
+    }
+    pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)nt);
+    for (int t = 0; t < nt; ++t) pthread_create(&th[t], NULL, pool_worker, &p);
+    for (int t = 0; t < nt; ++t) pthread_join(th[t], NULL);
+    free(th);
+}
+
+int oracle_num_threads(int nthreads) { return resolve_threads(nthreads); }
+
+/* ------------------------------------------------------------------------ */
+/* shared problem description                                                */
+
+typedef struct {
+    const double *q, *k, *v, *dout;
+    double *o, *lse, *dq, *dk, *dv;
+    i64 B, Hq, Hkv, N, d;
+    double scale;
+    int causal;
+    /* row / column subsets */
+    const i64 *rows;
+    i64 nrows;
+    i64 b_sel, hkv_sel;
+    /* online-softmax block size */
+    i64 block;
+} prob_t;
+
+static const double *head_ptr(const double *base, i64 b, i64 h, i64 H, i64 N, i64 d) {
+    return base + ((b * H + h) * N) * d;
+}
+
+static double dot(const double *a, const double *b, i64 d) {
+    double s = 0.0;
+    for (i64 c = 0; c < d; ++c) s += a[c] * b[c];
+    return s;
+}
+
+/* Scores of one query row against every key: s[j] = scale * q_i . k_j, with
+ * -inf for masked keys.  Returns the number of unmasked keys. */
+static i64 score_row(const prob_t *P, const double *qi, const double *kh, i64 i, double *s) {
+    i64 n_valid = 0;
+    for (i64 j = 0; j < P->N; ++j) {
+        if (P->causal && j > i) {
+            s[j] = -INFINITY;
+        } else {
+            s[j] = P->scale * dot(qi, kh + j * P->d, P->d);
+            ++n_valid;
+        }
+    }
+    return n_valid;
+}
+
+/* Two-pass softmax of one row in place: s -> P.  Writes m and l. */
+static void softmax_row_two_pass(double *s, i64 N, double *m_out, double *l_out) {
+    double m = -INFINITY;
+    for (i64 j = 0; j < N; ++j)
+        if (s[j] > m) m = s[j]; /* pass 1: max */
+    double l = 0.0;
+    for (i64 j = 0; j < N; ++j) l += exp(s[j] - m); /* pass 2: sum */
+    for (i64 j = 0; j < N; ++j) s[j] = exp(s[j] - m) / l;
+    *m_out = m;
+    *l_out = l;
+}
+
+/* ------------------------------------------------------------------------ */
+/* forward, full: materialises the N x N matrix of one head                  */
+
+static void fwd_full_item(void *ctx, i64 item) {
+    const prob_t *P = (const prob_t *)ctx;
+    const i64 N = P->N, d = P->d, group = P->Hq / P->Hkv;
+    const i64 b = item / P->Hq, h = item % P->Hq, g = h / group;
+    const double *qh = head_ptr(P->q, b, h, P->Hq, N, d);
+    const double *kh = head_ptr(P->k, b, g, P->Hkv, N, d);
+    const double *vh = head_ptr(P->v, b, g, P->Hkv, N, d);
+    double *oh = P->o + ((b * P->Hq + h) * N) * d;
+    double *lseh = P->lse + (b * P->Hq + h) * N;
+
+    double *S = (double *)malloc(sizeof(double) * (size_t)(N * N));
+    for (i64 i = 0; i < N; ++i) score_row(P, qh + i * d, kh, i, S + i * N);
+    for (i64 i = 0; i < N; ++i) {
+        double m, l;
+        softmax_row_two_pass(S + i * N, N, &m, &l);
+        lseh[i] = m + log(l);
+    }
+    /* O = P V */
+    for (i64 i = 0; i < N; ++i) {
+        double *oi = oh + i * d;
+        for (i64 c = 0; c < d; ++c) oi[c] = 0.0;
+        for (i64 j = 0; j < N; ++j) {
+            const double p = S[i * N + j];
+            const double *vj = vh + j * d;
+            for (i64 c = 0; c < d; ++c) oi[c] += p * vj[c];
+        }
+    }
+    free(S);
+}
+
+int oracle_fwd(const double *q, const double *k, const double *v, double *o, double *lse,
+               i64 B, i64 Hq, i64 Hkv, i64 N, i64 d, double scale, int causal, int nthreads) {
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || N < 0 || d <= 0 || Hq % Hkv) return 1;
+    prob_t P = {0};
+    P.q = q; P.k = k; P.v = v; P.o = o; P.lse = lse;
+    P.B = B; P.Hq = Hq; P.Hkv = Hkv; P.N = N; P.d = d; P.scale = scale; P.causal = causal;
+    if (N > 0) run_pool(fwd_full_item, &P, B * Hq, nthreads);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* forward, selected query rows of every head (row-streamed form of the same
+ * formulas: each output row depends on its own query row only)              */
+
+static void fwd_rows_item(void *ctx, i64 item) {
+    const prob_t *P = (const prob_t *)ctx;
+    const i64 N = P->N, d = P->d, group = P->Hq / P->Hkv;
+    const i64 bh = item / P->nrows, r = item % P->nrows;
+    const i64 b = bh / P->Hq, h = bh % P->Hq, g = h / group;
+    const i64 i = P->rows[r];
+    const double *qi = head_ptr(P->q, b, h, P->Hq, N, d) + i * d;
+    const double *kh = head_ptr(P->k, b, g, P->Hkv, N, d);
+    const double *vh = head_ptr(P->v, b, g, P->Hkv, N, d);
+    double *oi = P->o + (bh * P->nrows + r) * d;
+
+    double *s = (double *)malloc(sizeof(double) * (size_t)N);
+    score_row(P, qi, kh, i, s);
+    double m, l;
+    softmax_row_two_pass(s, N, &m, &l);
+    P->lse[bh * P->nrows + r] = m + log(l);
+    for (i64 c = 0; c < d; ++c) oi[c] = 0.0;
+    for (i64 j = 0; j < N; ++j) {
+        const double *vj = vh + j * d;
+        for (i64 c = 0; c < d; ++c) oi[c] += s[j] * vj[c];
+    }
+    free(s);
+}
+
+/* o_rows: [B][Hq][nrows][d], lse_rows: [B][Hq][nrows] */
+int oracle_fwd_rows(const double *q, const double *k, const double *v, const i64 *rows, i64 nrows,
+                    double *o_rows, double *lse_rows, i64 B, i64 Hq, i64 Hkv, i64 N, i64 d,
+                    double scale, int causal, int nthreads) {
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || N < 0 || d <= 0 || Hq % Hkv || nrows < 0) return 1;
+    for (i64 r = 0; r < nrows; ++r)
+        if (rows[r] < 0 || rows[r] >= N) return 2;
+    prob_t P = {0};
+    P.q = q; P.k = k; P.v = v; P.o = o_rows; P.lse = lse_rows; P.rows = rows; P.nrows = nrows;
+    P.B = B; P.Hq = Hq; P.Hkv = Hkv; P.N = N; P.d = d; P.scale = scale; P.causal = causal;
+    if (nrows > 0) run_pool(fwd_rows_item, &P, B * Hq * nrows, nthreads);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* forward by the online (one-pass, blocked) softmax, the method the pages
+ * describe: keep a running max m and running sum l, and rescale the partial
+ * sums when the max grows ("FlashAttention" glossary, online-softmax
+ * paragraph; "flash attention io aware", section "Online Softmax").  This is
+ * NOT the definition; it exists so a test can check, in fp64, that the
+ * one-pass recurrence reaches the two-pass result.                          */
+
+static void fwd_online_item(void *ctx, i64 item) {
+    const prob_t *P = (const prob_t *)ctx;
+    const i64 N = P->N, d = P->d, group = P->Hq / P->Hkv, Bc = P->block;
+    const i64 b = item / P->Hq, h = item % P->Hq, g = h / group;
+    const double *qh = head_ptr(P->q, b, h, P->Hq, N, d);
+    const double *kh = head_ptr(P->k, b, g, P->Hkv, N, d);
+    const double *vh = head_ptr(P->v, b, g, P->Hkv, N, d);
+    double *oh = P->o + ((b * P->Hq + h) * N) * d;
+    double *lseh = P->lse + (b * P->Hq + h) * N;
+    double *s = (double *)malloc(sizeof(double) * (size_t)Bc);
+
+    for (i64 i = 0; i < N; ++i) {
+        double m = -INFINITY, l = 0.0;
+        double *acc = oh + i * d;
+        for (i64 c = 0; c < d; ++c) acc[c] = 0.0;
+        for (i64 j0 = 0; j0 < N; j0 += Bc) {
+            const i64 nb = (j0 + Bc <= N) ? Bc : N - j0;
+            double mb = -INFINITY;
+            for (i64 t = 0; t < nb; ++t) {
+                const i64 j = j0 + t;
+                s[t] = (P->causal && j > i) ? -INFINITY : P->scale * dot(qh + i * d, kh + j * d, d);
+                if (s[t] > mb) mb = s[t];
+            }
+            if (mb == -INFINITY) continue; /* block fully masked */
+            const double m_new = mb > m ? mb : m;
+            const double corr = exp(m - m_new); /* 0 when m = -inf */
+            l *= corr;
+            for (i64 c = 0; c < d; ++c) acc[c] *= corr;
+            for (i64 t = 0; t < nb; ++t) {
+                const double p = exp(s[t] - m_new);
+                l += p;
+                const double *vj = vh + (j0 + t) * d;
+                for (i64 c = 0; c < d; ++c) acc[c] += p * vj[c];
+            }
+            m = m_new;
+        }
+        for (i64 c = 0; c < d; ++c) acc[c] /= l;
+        lseh[i] = m + log(l);
+    }
+    free(s);
+}
+
+int oracle_fwd_online(const double *q, const double *k, const double *v, double *o, double *lse,
+                      i64 B, i64 Hq, i64 Hkv, i64 N, i64 d, double scale, int causal, i64 block,
+                      int nthreads) {
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || N < 0 || d <= 0 || Hq % Hkv || block <= 0) return 1;
+    prob_t P = {0};
+    P.q = q; P.k = k; P.v = v; P.o = o; P.lse = lse; P.block = block;
+    P.B = B; P.Hq = Hq; P.Hkv = Hkv; P.N = N; P.d = d; P.scale = scale; P.causal = causal;
+    if (N > 0) run_pool(fwd_online_item, &P, B * Hq, nthreads);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* backward, full: one work item = one kv head and all query heads of its
+ * group, so that dK and dV are summed without sharing between threads.      */
+
+static void bwd_full_item(void *ctx, i64 item) {
+    const prob_t *P = (const prob_t *)ctx;
+    const i64 N = P->N, d = P->d, group = P->Hq / P->Hkv;
+    const i64 b = item / P->Hkv, g = item % P->Hkv;
+    const double *kh = head_ptr(P->k, b, g, P->Hkv, N, d);
+    const double *vh = head_ptr(P->v, b, g, P->Hkv, N, d);
+    double *dkh = P->dk + ((b * P->Hkv + g) * N) * d;
+    double *dvh = P->dv + ((b * P->Hkv + g) * N) * d;
+    memset(dkh, 0, sizeof(double) * (size_t)(N * d));
+    memset(dvh, 0, sizeof(double) * (size_t)(N * d));
+
+    double *Pm = (double *)malloc(sizeof(double) * (size_t)(N * N));
+    double *dP = (double *)malloc(sizeof(double) * (size_t)(N * N));
+    for (i64 h = g * group; h < (g + 1) * group; ++h) {
+        const double *qh = head_ptr(P->q, b, h, P->Hq, N, d);
+        const double *doh = head_ptr(P->dout, b, h, P->Hq, N, d);
+        double *dqh = P->dq + ((b * P->Hq + h) * N) * d;
+        /* recompute P from the definition */
+        for (i64 i = 0; i < N; ++i) {
+            double m, l;
+            score_row(P, qh + i * d, kh, i, Pm + i * N);
+            softmax_row_two_pass(Pm + i * N, N, &m, &l);
+        }
+        /* dP = dO V^T */
+        for (i64 i = 0; i < N; ++i)
+            for (i64 j = 0; j < N; ++j) dP[i * N + j] = dot(doh + i * d, vh + j * d, d);
+        /* dS = P o (dP - D), D_i = sum_j P_ij dP_ij; stored in place of dP */
+        for (i64 i = 0; i < N; ++i) {
+            double D = 0.0;
+            for (i64 j = 0; j < N; ++j) D += Pm[i * N + j] * dP[i * N + j];
+            for (i64 j = 0; j < N; ++j) dP[i * N + j] = Pm[i * N + j] * (dP[i * N + j] - D);
+        }
+        /* dQ = scale dS K ; dK += scale dS^T Q ; dV += P^T dO */
+        for (i64 i = 0; i < N; ++i) {
+            double *dqi = dqh + i * d;
+            for (i64 c = 0; c < d; ++c) dqi[c] = 0.0;
+            for (i64 j = 0; j < N; ++j) {
+                const double ds = dP[i * N + j], p = Pm[i * N + j];
+                const double *kj = kh + j * d;
+                const double *qi = qh + i * d;
+                const double *doi = doh + i * d;
+                double *dkj = dkh + j * d;
+                double *dvj = dvh + j * d;
+                for (i64 c = 0; c < d; ++c) {
+                    dqi[c] += P->scale * ds * kj[c];
+                    dkj[c] += P->scale * ds * qi[c];
+                    dvj[c] += p * doi[c];
+                }
+            }
+        }
+    }
+    free(Pm);
+    free(dP);
+}
+
+int oracle_bwd(const double *q, const double *k, const double *v, const double *dout, double *dq,
+               double *dk, double *dv, i64 B, i64 Hq, i64 Hkv, i64 N, i64 d, double scale,
+               int causal, int nthreads) {
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || N < 0 || d <= 0 || Hq % Hkv) return 1;
+    prob_t P = {0};
+    P.q = q; P.k = k; P.v = v; P.dout = dout; P.dq = dq; P.dk = dk; P.dv = dv;
+    P.B = B; P.Hq = Hq; P.Hkv = Hkv; P.N = N; P.d = d; P.scale = scale; P.causal = causal;
+    if (N > 0) run_pool(bwd_full_item, &P, B * Hkv, nthreads);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* backward, dQ of selected query rows of every head.  dQ_i depends on query
+ * row i only: P_i. and dP_i. over all keys, D_i from the same row.           */
+
+static void bwd_rows_item(void *ctx, i64 item) {
+    const prob_t *P = (const prob_t *)ctx;
+    const i64 N = P->N, d = P->d, group = P->Hq / P->Hkv;
+    const i64 bh = item / P->nrows, r = item % P->nrows;
+    const i64 b = bh / P->Hq, h = bh % P->Hq, g = h / group;
+    const i64 i = P->rows[r];
+    const double *qi = head_ptr(P->q, b, h, P->Hq, N, d) + i * d;
+    const double *doi = head_ptr(P->dout, b, h, P->Hq, N, d) + i * d;
+    const double *kh = head_ptr(P->k, b, g, P->Hkv, N, d);
+    const double *vh = head_ptr(P->v, b, g, P->Hkv, N, d);
+    double *dqi = P->dq + (bh * P->nrows + r) * d;
+
+    double *p = (double *)malloc(sizeof(double) * (size_t)N);
+    double *dp = (double *)malloc(sizeof(double) * (size_t)N);
+    double m, l;
+    score_row(P, qi, kh, i, p);
+    softmax_row_two_pass(p, N, &m, &l);
+    double D = 0.0;
+    for (i64 j = 0; j < N; ++j) {
+        dp[j] = dot(doi, vh + j * d, d);
+        D += p[j] * dp[j];
+    }
+    for (i64 c = 0; c < d; ++c) dqi[c] = 0.0;
+    for (i64 j = 0; j < N; ++j) {
+        const double ds = p[j] * (dp[j] - D);
+        if (ds == 0.0) continue;
+        const double *kj = kh + j * d;
+        for (i64 c = 0; c < d; ++c) dqi[c] += P->scale * ds * kj[c];
+    }
+    free(p);
+    free(dp);
+}
+
+/* dq_rows: [B][Hq][nrows][d] */
+int oracle_bwd_rows(const double *q, const double *k, const double *v, const double *dout,
+                    const i64 *rows, i64 nrows, double *dq_rows, i64 B, i64 Hq, i64 Hkv, i64 N,
+                    i64 d, double scale, int causal, int nthreads) {
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || N < 0 || d <= 0 || Hq % Hkv || nrows < 0) return 1;
+    for (i64 r = 0; r < nrows; ++r)
+        if (rows[r] < 0 || rows[r] >= N) return 2;
+    prob_t P = {0};
+    P.q = q; P.k = k; P.v = v; P.dout = dout; P.dq = dq_rows; P.rows = rows; P.nrows = nrows;
+    P.B = B; P.Hq = Hq; P.Hkv = Hkv; P.N = N; P.d = d; P.scale = scale; P.causal = causal;
+    if (nrows > 0) run_pool(bwd_rows_item, &P, B * Hq * nrows, nthreads);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* backward, dK and dV of selected key rows of one kv head (b_sel, hkv_sel).
+ * dK_j and dV_j need P_ij over every query row i of every head in the group,
+ * so the per-row statistics (m_i, l_i) and D_i are computed first for every
+ * row (one O(N^2 d) pass per head); then each selected column is summed.
+ * With a causal mask only rows i >= min(selected j) contribute, so the
+ * statistics are computed for those rows only.                              */
+
+typedef struct {
+    const prob_t *P;
+    i64 h;          /* query head being processed */
+    i64 i_lo;       /* first query row that can contribute */
+    double *m, *l;  /* [N] per-row max and sum */
+    double *D;      /* [N] per-row D_i */
+} colstat_t;
+
+static void col_stats_item(void *ctx, i64 item) {
+    colstat_t *C = (colstat_t *)ctx;
+    const prob_t *P = C->P;
+    const i64 N = P->N, d = P->d, g = P->hkv_sel, b = P->b_sel, h = C->h;
+    const i64 i = C->i_lo + item;
+    const double *qi = head_ptr(P->q, b, h, P->Hq, N, d) + i * d;
+    const double *doi = head_ptr(P->dout, b, h, P->Hq, N, d) + i * d;
+    const double *kh = head_ptr(P->k, b, g, P->Hkv, N, d);
+    const double *vh = head_ptr(P->v, b, g, P->Hkv, N, d);
+    double *p = (double *)malloc(sizeof(double) * (size_t)N);
+    double m, l;
+    score_row(P, qi, kh, i, p);
+    softmax_row_two_pass(p, N, &m, &l);
+    double D = 0.0;
+    for (i64 j = 0; j < N; ++j)
+        if (p[j] != 0.0) D += p[j] * dot(doi, vh + j * d, d);
+    C->m[i] = m;
+    C->l[i] = l;
+    C->D[i] = D;
+    free(p);
+}
+
+typedef struct {
+    const prob_t *P;
+    const colstat_t *stats; /* one per group head */
+    i64 group;
+} colsum_t;
+
+static void col_sum_item(void *ctx, i64 r) {
+    const colsum_t *C = (const colsum_t *)ctx;
+    const prob_t *P = C->P;
+    const i64 N = P->N, d = P->d, g = P->hkv_sel, b = P->b_sel;
+    const i64 j = P->rows[r];
+    const double *kj = head_ptr(P->k, b, g, P->Hkv, N, d) + j * d;
+    const double *vj = head_ptr(P->v, b, g, P->Hkv, N, d) + j * d;
+    double *dkj = P->dk + r * d;
+    double *dvj = P->dv + r * d;
+    for (i64 c = 0; c < d; ++c) dkj[c] = dvj[c] = 0.0;
+    for (i64 t = 0; t < C->group; ++t) {
+        const colstat_t *S = &C->stats[t];
+        const double *qh = head_ptr(P->q, b, S->h, P->Hq, N, d);
+        const double *doh = head_ptr(P->dout, b, S->h, P->Hq, N, d);
+        for (i64 i = S->i_lo; i < N; ++i) {
+            if (P->causal && j > i) continue;
+            const double s = P->scale * dot(qh + i * d, kj, d);
+            const double p = exp(s - S->m[i]) / S->l[i];
+            const double dp = dot(doh + i * d, vj, d);
+            const double ds = p * (dp - S->D[i]);
+            for (i64 c = 0; c < d; ++c) {
+                dvj[c] += p * doh[i * d + c];
+                dkj[c] += P->scale * ds * qh[i * d + c];
+            }
+        }
+    }
+}
+
+/* dk_cols, dv_cols: [ncols][d] for kv rows cols[] of kv head (b_sel, hkv_sel) */
+int oracle_bwd_cols(const double *q, const double *k, const double *v, const double *dout,
+                    i64 b_sel, i64 hkv_sel, const i64 *cols, i64 ncols, double *dk_cols,
+                    double *dv_cols, i64 B, i64 Hq, i64 Hkv, i64 N, i64 d, double scale,
+                    int causal, int nthreads) {
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || N < 0 || d <= 0 || Hq % Hkv || ncols < 0) return 1;
+    if (b_sel < 0 || b_sel >= B || hkv_sel < 0 || hkv_sel >= Hkv) return 2;
+    i64 j_min = N;
+    for (i64 r = 0; r < ncols; ++r) {
+        if (cols[r] < 0 || cols[r] >= N) return 2;
+        if (cols[r] < j_min) j_min = cols[r];
+    }
+    if (ncols == 0) return 0;
+    const i64 group = Hq / Hkv;
+    prob_t P = {0};
+    P.q = q; P.k = k; P.v = v; P.dout = dout; P.dk = dk_cols; P.dv = dv_cols;
+    P.rows = cols; P.nrows = ncols; P.b_sel = b_sel; P.hkv_sel = hkv_sel;
+    P.B = B; P.Hq = Hq; P.Hkv = Hkv; P.N = N; P.d = d; P.scale = scale; P.causal = causal;
+
+    const i64 i_lo = causal ? j_min : 0;
+    colstat_t *stats = (colstat_t *)calloc((size_t)group, sizeof(colstat_t));
+    for (i64 t = 0; t < group; ++t) {
+        stats[t].P = &P;
+        stats[t].h = hkv_sel * group + t;
+        stats[t].i_lo = i_lo;
+        stats[t].m = (double *)malloc(sizeof(double) * (size_t)N);
+        stats[t].l = (double *)malloc(sizeof(double) * (size_t)N);
+        stats[t].D = (double *)malloc(sizeof(double) * (size_t)N);
+        run_pool(col_stats_item, &stats[t], N - i_lo, nthreads);
+    }
+    colsum_t C = {&P, stats, group};
+    run_pool(col_sum_item, &C, ncols, nthreads);
+    for (i64 t = 0; t < group; ++t) {
+        free(stats[t].m);
+        free(stats[t].l);
+        free(stats[t].D);
+    }
+    free(stats);
+    return 0;
+}

@@ -1,0 +1,292 @@
+"""Pins of the CPU oracle against facts that do not come from the oracle.
+
+Each ``pin_*`` takes an ``oracle.Oracle`` instance and raises AssertionError
+when the oracle disagrees with a closed form, a hand-derived value, a library
+routine, a finite difference or an invariant of the mathematics.  They are
+collected here so that the same list can be run against the real oracle
+(tests/test_oracle_pins.py) and against copies with a planted mistake
+(tests/test_oracle_mutants.py), which must each fail at least one pin.
+"""
+
+from __future__ import annotations
+
+import json
+import math
+import os
+
+import numpy as np
+import torch
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+def _rand(seed, B=1, Hq=2, Hkv=2, N=8, d=4):
+    r = _rng(seed)
+    q = r.standard_normal((B, Hq, N, d))
+    k = r.standard_normal((B, Hkv, N, d))
+    v = r.standard_normal((B, Hkv, N, d))
+    do = r.standard_normal((B, Hq, N, d))
+    return q, k, v, do
+
+
+def _close(a, b, tol, what):
+    a, b = np.asarray(a, dtype=np.float64), np.asarray(b, dtype=np.float64)
+    err = float(np.max(np.abs(a - b))) if a.size else 0.0
+    assert a.shape == b.shape, f"{what}: shape {a.shape} vs {b.shape}"
+    assert err <= tol, f"{what}: max abs err {err:.3e} > {tol:.1e}"
+
+
+# ---------------------------------------------------------------- forward pins
+
+def pin_q_zero_noncausal(orc):
+    """Q = 0: every score is 0, P is uniform, O_i = mean_j V_j, lse_i = ln N."""
+    _, k, v, _ = _rand(1, Hq=2, Hkv=2, N=12, d=5)
+    q = np.zeros((1, 2, 12, 5))
+    o, lse = orc.fwd(q, k, v, 0.37, False)
+    _close(o, np.broadcast_to(v.mean(axis=2, keepdims=True), o.shape), 1e-13, "O at Q=0")
+    _close(lse, np.full(lse.shape, math.log(12)), 1e-13, "lse at Q=0")
+
+
+def pin_q_zero_causal(orc):
+    """Q = 0, causal: O_i = mean_{j<=i} V_j, lse_i = ln(i + 1)."""
+    _, k, v, _ = _rand(2, Hq=1, Hkv=1, N=10, d=3)
+    q = np.zeros((1, 1, 10, 3))
+    o, lse = orc.fwd(q, k, v, 0.5, True)
+    prefix = np.cumsum(v[0, 0], axis=0) / np.arange(1, 11)[:, None]
+    _close(o[0, 0], prefix, 1e-13, "causal O at Q=0")
+    _close(lse[0, 0], np.log(np.arange(1, 11)), 1e-13, "causal lse at Q=0")
+
+
+def pin_one_hot(orc):
+    """q_i = c e_t, k_{j*} = e_t, every other key 0: scores are (scale c) at j* and
+    0 elsewhere, so O_i = (e^{sc} V_j* + sum_{j != j*} V_j) / (e^{sc} + N - 1) and
+    lse_i = ln(e^{sc} + N - 1); for large c, O_i -> V_j*."""
+    N, d, t, js, c, scale = 9, 4, 2, 6, 40.0, 0.5
+    q = np.zeros((1, 1, N, d)); q[..., t] = c
+    k = np.zeros((1, 1, N, d)); k[0, 0, js, t] = 1.0
+    v = _rng(3).standard_normal((1, 1, N, d))
+    o, lse = orc.fwd(q, k, v, scale, False)
+    e = math.exp(scale * c)
+    want = (e * v[0, 0, js] + (v[0, 0].sum(axis=0) - v[0, 0, js])) / (e + N - 1)
+    _close(o[0, 0], np.broadcast_to(want, (N, d)), 1e-12, "one-hot O")
+    _close(lse[0, 0], np.full(N, math.log(e + N - 1)), 1e-12, "one-hot lse")
+    _close(o[0, 0], np.broadcast_to(v[0, 0, js], (N, d)), 1e-6, "one-hot selects V[j*]")
+
+
+def pin_causal_row0(orc):
+    """Causal row 0 sees key 0 only: O_0 = V_0, lse_0 = scale q_0 . k_0."""
+    q, k, v, _ = _rand(4, Hq=4, Hkv=2, N=7, d=6)
+    o, lse = orc.fwd(q, k, v, 0.41, True)
+    for h in range(4):
+        g = h // 2
+        _close(o[0, h, 0], v[0, g, 0], 1e-14, "causal O_0")
+        _close(lse[0, h, 0], 0.41 * q[0, h, 0] @ k[0, g, 0], 1e-14, "causal lse_0")
+
+
+def pin_rows_sum_to_one(orc):
+    """sum_j P_ij = 1: with V = 1 every output is 1, causal or not."""
+    q, k, _, _ = _rand(5, Hq=2, Hkv=1, N=11, d=4)
+    v = np.ones((1, 1, 11, 4))
+    for causal in (False, True):
+        o, _ = orc.fwd(q * 3, k, v, 0.8, causal)
+        _close(o, np.ones_like(o), 1e-14, f"rows of P sum to 1 (causal={causal})")
+
+
+def pin_key_shift(orc):
+    """K -> K + 1 c^T shifts row i of the scores by scale q_i . c: P and O are
+    unchanged and lse_i moves by exactly that amount."""
+    q, k, v, _ = _rand(6, Hq=2, Hkv=2, N=9, d=3)
+    c = np.array([0.7, -1.3, 2.1])
+    for causal in (False, True):
+        o1, l1 = orc.fwd(q, k, v, 0.6, causal)
+        o2, l2 = orc.fwd(q, k + c, v, 0.6, causal)
+        _close(o2, o1, 1e-12, "O invariant to key shift")
+        _close(l2 - l1, 0.6 * q @ c, 1e-12, "lse shift")
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        g = json.load(f)
+
+    def val(x):
+        if isinstance(x, (int, float)):
+            return float(x)
+        consts = {"ln3": math.log(3), "ln4": math.log(4), "ln2": math.log(2),
+                  "0.75ln3": 0.75 * math.log(3)}
+        return consts[x]
+
+    s = g["shape"]
+    B, Hq, Hkv, N, d = s["B"], s["Hq"], s["Hkv"], s["N"], s["d"]
+    arr = lambda x, H: np.array([val(t) for t in x]).reshape(B, H, N, d)
+    q, k, v, do = arr(g["q"], Hq), arr(g["k"], Hkv), arr(g["v"], Hkv), arr(g["dout"], Hq)
+    return g, q, k, v, do, val
+
+
+def pin_golden(orc):
+    """Hand-derived two-token examples (tests/golden/*.json)."""
+    for name in ("two_token_mha.json", "two_token_gqa.json"):
+        g, q, k, v, do, val = _golden(name)
+        for case, want in g["cases"].items():
+            causal = case == "causal"
+            o, lse = orc.fwd(q, k, v, g["scale"], causal)
+            dq, dk, dv = orc.bwd(q, k, v, do, g["scale"], causal)
+            _close(o.ravel(), [val(x) for x in want["o"]], 1e-13, f"{name} {case} O")
+            _close(lse.ravel(), [val(x) for x in want["lse"]], 1e-13, f"{name} {case} lse")
+            _close(dq.ravel(), [val(x) for x in want["dq"]], 1e-13, f"{name} {case} dQ")
+            _close(dk.ravel(), [val(x) for x in want["dk"]], 1e-13, f"{name} {case} dK")
+            _close(dv.ravel(), [val(x) for x in want["dv"]], 1e-13, f"{name} {case} dV")
+
+
+def pin_brute_force_python(orc):
+    """Forward by pure-Python loops (math.exp, two explicit passes) on tiny inputs."""
+    B, Hq, Hkv, N, d = 1, 4, 2, 5, 3
+    q, k, v, _ = _rand(7, B, Hq, Hkv, N, d)
+    scale = 0.9
+    for causal in (False, True):
+        o, lse = orc.fwd(q, k, v, scale, causal)
+        for h in range(Hq):
+            g = h // (Hq // Hkv)
+            for i in range(N):
+                js = [j for j in range(N) if not (causal and j > i)]
+                s = {j: scale * sum(q[0, h, i, c] * k[0, g, j, c] for c in range(d)) for j in js}
+                m = max(s.values())
+                z = sum(math.exp(s[j] - m) for j in js)
+                for c in range(d):
+                    want = sum(math.exp(s[j] - m) / z * v[0, g, j, c] for j in js)
+                    assert abs(o[0, h, i, c] - want) < 1e-13, ("brute O", h, i, c)
+                assert abs(lse[0, h, i] - (m + math.log(z))) < 1e-13, ("brute lse", h, i)
+
+
+def _torch_ref(q, k, v, do, scale, causal):
+    """torch fp64 SDPA (CPU math path) + autograd; lse by torch.logsumexp."""
+    tq, tk, tv = (torch.tensor(x, dtype=torch.float64, requires_grad=True) for x in (q, k, v))
+    Hq, Hkv = q.shape[1], k.shape[1]
+    o = torch.nn.functional.scaled_dot_product_attention(
+        tq, tk, tv, is_causal=causal, scale=scale, enable_gqa=Hq != Hkv)
+    o.backward(torch.tensor(do, dtype=torch.float64))
+    with torch.no_grad():
+        kk = tk.repeat_interleave(Hq // Hkv, dim=1)
+        s = scale * tq @ kk.transpose(-1, -2)
+        if causal:
+            n = s.shape[-1]
+            s = s.masked_fill(torch.ones(n, n, dtype=torch.bool).triu(1), float("-inf"))
+        lse = torch.logsumexp(s, dim=-1)
+    return (o.detach().numpy(), lse.numpy(), tq.grad.numpy(), tk.grad.numpy(), tv.grad.numpy())
+
+
+def pin_torch_sdpa(orc):
+    """Library special case: torch fp64 scaled_dot_product_attention and autograd,
+    MHA and GQA, causal and not."""
+    for (Hq, Hkv, N, d, seed) in ((2, 2, 64, 16, 8), (4, 2, 33, 8, 9), (4, 1, 20, 8, 10)):
+        q, k, v, do = _rand(seed, 1, Hq, Hkv, N, d)
+        scale = 1.0 / math.sqrt(d)
+        for causal in (False, True):
+            o, lse = orc.fwd(q, k, v, scale, causal)
+            dq, dk, dv = orc.bwd(q, k, v, do, scale, causal)
+            ro, rl, rdq, rdk, rdv = _torch_ref(q, k, v, do, scale, causal)
+            tag = f"Hq{Hq} Hkv{Hkv} N{N} causal={causal}"
+            _close(o, ro, 1e-12, f"torch O {tag}")
+            _close(lse, rl, 1e-12, f"torch lse {tag}")
+            _close(dq, rdq, 1e-11, f"torch dQ {tag}")
+            _close(dk, rdk, 1e-11, f"torch dK {tag}")
+            _close(dv, rdv, 1e-11, f"torch dV {tag}")
+
+
+# --------------------------------------------------------------- backward pins
+
+def pin_finite_differences(orc):
+    """Central differences (h = 1e-6) of L = sum(dO * O) against dQ, dK, dV."""
+    h = 1e-6
+    for (Hq, Hkv, N, d, causal, seed) in ((1, 1, 6, 3, False, 11), (2, 1, 5, 4, True, 12),
+                                          (2, 2, 7, 2, True, 13)):
+        q, k, v, do = _rand(seed, 1, Hq, Hkv, N, d)
+        scale = 0.7
+        dq, dk, dv = orc.bwd(q, k, v, do, scale, causal)
+
+        def loss(args):
+            o, _ = orc.fwd(args[0], args[1], args[2], scale, causal)
+            return float(np.sum(do * o))
+
+        for slot, (name, g) in enumerate((("q", dq), ("k", dk), ("v", dv))):
+            x = (q, k, v)[slot]
+            num = np.zeros_like(x)
+            for idx in np.ndindex(x.shape):
+                plus, minus = [q, k, v], [q, k, v]
+                plus[slot], minus[slot] = x.copy(), x.copy()
+                plus[slot][idx] += h
+                minus[slot][idx] -= h
+                num[idx] = (loss(plus) - loss(minus)) / (2 * h)
+            rel = np.linalg.norm(num - g) / max(np.linalg.norm(num), 1e-30)
+            assert rel <= 1e-6, f"finite differences d{name} (Hq{Hq} Hkv{Hkv} causal={causal}): rel {rel:.2e}"
+
+
+def pin_q_zero_backward(orc):
+    """Q = 0, non-causal: dK = 0 exactly, dV_j = mean_i dO_i,
+    dQ_i = scale (1/N) sum_j (dO_i . (v_j - vbar)) k_j."""
+    _, k, v, do = _rand(14, 1, 2, 2, 10, 4)
+    q = np.zeros_like(do)
+    scale = 0.3
+    dq, dk, dv = orc.bwd(q, k, v, do, scale, False)
+    _close(dk, np.zeros_like(dk), 0.0, "dK at Q=0")
+    _close(dv, np.broadcast_to(do.mean(axis=2, keepdims=True), dv.shape), 1e-14, "dV at Q=0")
+    vbar = v.mean(axis=2, keepdims=True)
+    coef = np.einsum("bhic,bhjc->bhij", do, v - vbar)
+    want = scale / 10 * np.einsum("bhij,bhjc->bhic", coef, k)
+    _close(dq, want, 1e-13, "dQ at Q=0")
+
+
+def pin_gradient_invariants(orc):
+    """(i) sum_j dK_j = 0 per kv head; (ii) sum_j dV_j = sum over the group of
+    sum_i dO_i; (iii) <Q, dQ> = <K, dK> per kv group."""
+    for causal in (False, True):
+        q, k, v, do = _rand(15, 2, 4, 2, 13, 5)
+        dq, dk, dv = orc.bwd(q, k, v, do, 0.45, causal)
+        _close(dk.sum(axis=2), np.zeros((2, 2, 5)), 1e-12, "sum_j dK_j")
+        grp = do.reshape(2, 2, 2, 13, 5).sum(axis=(2, 3))
+        _close(dv.sum(axis=2), grp, 1e-12, "sum_j dV_j")
+        qdq = (q * dq).reshape(2, 2, 2, 13, 5).sum(axis=(2, 3, 4))
+        kdk = (k * dk).sum(axis=(2, 3))
+        _close(qdq, kdk, 1e-12, "<Q,dQ> = <K,dK>")
+
+
+def pin_subsets_match_full(orc):
+    """Row- and column-subset forms equal the full forms on the same inputs."""
+    q, k, v, do = _rand(16, 2, 4, 2, 40, 8)
+    rows = np.array([0, 3, 17, 39])
+    cols = np.array([1, 20, 38])
+    for causal in (False, True):
+        o, lse = orc.fwd(q, k, v, 0.35, causal)
+        dq, dk, dv = orc.bwd(q, k, v, do, 0.35, causal)
+        o_r, lse_r = orc.fwd_rows(q, k, v, rows, 0.35, causal)
+        _close(o_r, o[:, :, rows], 1e-13, "fwd_rows O")
+        _close(lse_r, lse[:, :, rows], 1e-13, "fwd_rows lse")
+        _close(orc.bwd_rows(q, k, v, do, rows, 0.35, causal), dq[:, :, rows], 1e-12, "bwd_rows dQ")
+        for (b, g) in ((0, 1), (1, 0)):
+            dkc, dvc = orc.bwd_cols(q, k, v, do, b, g, cols, 0.35, causal)
+            _close(dkc, dk[b, g, cols], 1e-12, "bwd_cols dK")
+            _close(dvc, dv[b, g, cols], 1e-12, "bwd_cols dV")
+
+
+def pin_online_equals_two_pass(orc):
+    """The one-pass blocked recurrence reaches the two-pass result (fp64, 1e-12),
+    for block sizes that divide N and that leave a ragged last block."""
+    q, k, v, _ = _rand(17, 1, 2, 1, 70, 8)
+    q = q * 4  # wide score range: the running max moves many times along a row
+    for causal in (False, True):
+        o, lse = orc.fwd(q, k, v, 0.5, causal)
+        for block in (1, 7, 16, 128):
+            o2, lse2 = orc.fwd_online(q, k, v, 0.5, causal, block=block)
+            _close(o2, o, 1e-12, f"online O (block {block})")
+            _close(lse2, lse, 1e-12, f"online lse (block {block})")
+
+
+ALL_PINS = [
+    pin_q_zero_noncausal, pin_q_zero_causal, pin_one_hot, pin_causal_row0,
+    pin_rows_sum_to_one, pin_key_shift, pin_golden, pin_brute_force_python,
+    pin_torch_sdpa, pin_finite_differences, pin_q_zero_backward,
+    pin_gradient_invariants, pin_subsets_match_full, pin_online_equals_two_pass,
+]

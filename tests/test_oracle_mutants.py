@@ -1,0 +1,47 @@
+"""Plant a plausible mistake in a copy of the oracle (on the CPU) and check
+that at least one pin catches it: the pins must be able to tell a wrong
+oracle from a right one, or they pin nothing."""
+
+import os
+
+import pytest
+
+import oracle
+import oracle_pins
+
+# (name, text in oracle.c, replacement): a dropped term, a wrong sign, a wrong
+# index, a transposed operand, a wrong head mapping, a missing rescale ...
+MUTANTS = [
+    ("lse_drops_log_l", "lseh[i] = m + log(l);", "lseh[i] = m;"),
+    ("causal_mask_off_by_one", "(P->causal && j > i)", "(P->causal && j >= i)"),
+    ("softmax_max_not_subtracted", "s[j] = exp(s[j] - m) / l;", "s[j] = exp(s[j]) / l;"),
+    ("dS_wrong_sign", "Pm[i * N + j] * (dP[i * N + j] - D)", "Pm[i * N + j] * (D - dP[i * N + j])"),
+    ("dP_transposed", "dP[i * N + j] = dot(doh + i * d, vh + j * d, d);",
+     "dP[i * N + j] = dot(doh + j * d, vh + i * d, d);"),
+    ("dQ_missing_scale", "dqi[c] += P->scale * ds * kj[c];", "dqi[c] += ds * kj[c];"),
+    ("gqa_interleaved_heads", "g = h / group;", "g = h % P->Hkv;"),
+    ("D_without_P", "D += Pm[i * N + j] * dP[i * N + j];", "D += dP[i * N + j];"),
+    ("dV_from_dS", "dvj[c] += p * doi[c];", "dvj[c] += ds * doi[c];"),
+    ("dK_from_k", "dkj[c] += P->scale * ds * qi[c];", "dkj[c] += P->scale * ds * kj[c];"),
+    ("online_no_rescale", "acc[c] *= corr;", "acc[c] *= 1.0;"),
+    ("rows_D_from_wrong_row", "dp[j] = dot(doi, vh + j * d, d);", "dp[j] = dot(qi, vh + j * d, d);"),
+    ("cols_missing_group_sum", "for (i64 t = 0; t < C->group; ++t) {", "for (i64 t = 0; t < 1; ++t) {"),
+]
+
+
+@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_pins_catch_planted_mistake(tmp_path, name, old, new):
+    src = open(oracle.SOURCE).read()
+    assert old in src, f"mutation site for {name} not found in oracle.c"
+    mutant_src = tmp_path / "oracle_mutant.c"
+    mutant_src.write_text(src.replace(old, new))
+    lib = oracle.build(force=True, src=str(mutant_src), out=str(tmp_path / f"lib_{name}.so"))
+    orc = oracle.Oracle(lib)
+    caught = []
+    for pin in oracle_pins.ALL_PINS:
+        try:
+            pin(orc)
+        except (AssertionError, ValueError, FloatingPointError) as e:
+            caught.append((pin.__name__, str(e)[:80]))
+            break
+    assert caught, f"no pin caught the planted mistake {name}"
