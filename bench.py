@@ -1,0 +1,363 @@
+#!/usr/bin/env python
+"""Throughput of exact attention forward + backward on B200, one JSON line.
+
+One step = the whole hot path once over one batch: fa_fwd (O, lse) then
+fa_bwd (dQ, dK, dV) on the 4K-token MHA workload (B=4, Hq=Hkv=32, N=4096,
+d=128, causal, bf16) unless --workload names another.  FLOPs follow the
+stated convention: forward 4*B*Hq*N^2*d, halved when causal; backward 2.5x
+forward.  ``value`` is whole-job TFLOPS (all ranks); every rank runs its own
+replica (the path has no exchange step), so scaling is weak.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py --impl reference ...   # the CPU oracle arm
+
+Timing: W untimed steps, then K steps between a barrier + synchronize on both
+sides, CUDA events on the launching stream, max over ranks.  The inputs
+(Q, K, V, dO: 512 MiB for the default workload) are larger than L2.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from exact_io_aware_bwd_b200 import binding  # noqa: E402
+from exact_io_aware_bwd_b200.build import build  # noqa: E402
+from exact_io_aware_bwd_b200.workloads import WORKLOADS  # noqa: E402
+
+METRIC = "attention fwd+bwd TFLOPS/GPU at N=4K–64K, d=128, and % of B200 bf16 peak"
+UNIT = "TFLOPS"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return p, "measured"
+    except Exception:
+        return FALLBACK_PEAKS, "fallback"
+
+
+def workload_desc(w, causal):
+    return (f"{w.name}: B={w.B} Hq={w.Hq} Hkv={w.Hkv} N={w.N} d={w.d} "
+            f"{'causal' if causal else 'non-causal'} {str(w.dtype).replace('torch.', '')}")
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples of this GPU's clocks and throttle reasons."""
+
+    FIELDS = ("pci.bus_id,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device):
+        p = torch.cuda.get_device_properties(device)
+        self.bus = f"{p.pci_bus_id:02X}:{p.pci_device_id:02X}"
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            import tempfile
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 8:
+                continue
+            bus = parts[0].upper()
+            if self.bus not in bus and len({r[0] for r in rows} | {bus}) > 1:
+                continue
+            rows.append(parts)
+        os.unlink(self.path)
+        mine = [r for r in rows if self.bus in r[0].upper()] or rows
+        if not mine:
+            return None
+        sm = [float(r[1]) for r in mine if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in mine if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in mine for i in range(4) if r[4 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(mine)}
+
+
+# ---------------------------------------------------------------- our arm
+
+def run_ours(args, w, causal, rank, world, device):
+    torch.cuda.set_device(device)
+    build()
+    binding.load()
+    B, Hq, Hkv, N, d = w.B, w.Hq, w.Hkv, w.N, w.d
+    g = torch.Generator(device=device).manual_seed(w.seed + 1000 * rank)
+    mk = lambda H, s: (torch.randn((B, H, N, d), generator=g, device=device, dtype=torch.float32) * s).to(w.dtype)
+    q, k, v, do = mk(Hq, w.sigma_qk), mk(Hkv, w.sigma_qk), mk(Hkv, w.sigma_vdo), mk(Hq, w.sigma_vdo)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, N), device=device, dtype=torch.float32)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(binding.fa_bwd_workspace_bytes(B, Hq, Hkv, N, d), device=device, dtype=torch.uint8)
+    scale = w.scale
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        binding.fa_fwd(q, k, v, o, lse, scale, causal, stream)
+        binding.fa_bwd(q, k, v, o, do, lse, dq, dk, dv, scale, causal, ws, stream)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    assert binding.fa_get_device_status(stream) == binding.FA_OK
+
+    # per-step events around the whole step and around each kernel of interest
+    K = args.steps
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    fwd_ev = [(ev(), ev()) for _ in range(K)]
+    bwd_ev = [(ev(), ev()) for _ in range(K)]
+    for a, b in fwd_ev + bwd_ev:  # materialise the handles
+        a.record(stream)
+        b.record(stream)
+    t0, t1 = ev(), ev()
+    clocks = ClockSampler(device) if rank == 0 else None
+    if clocks:
+        clocks.start()
+        time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize(device)
+    t0.record(stream)
+    for i in range(K):
+        binding.fa_set_profile_events(binding.KERNEL_FWD, *fwd_ev[i])
+        binding.fa_set_profile_events(binding.KERNEL_BWD_MAIN, *bwd_ev[i])
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize(device)
+    barrier()
+    binding.fa_set_profile_events(binding.KERNEL_FWD, None, None)
+    binding.fa_set_profile_events(binding.KERNEL_BWD_MAIN, None, None)
+    clk = clocks.stop() if clocks else None
+    status = binding.fa_get_device_status(stream)
+    assert status == binding.FA_OK, binding.fa_status_string(status)
+
+    ms_total = t0.elapsed_time(t1)
+    fwd_ms = statistics.mean(a.elapsed_time(b) for a, b in fwd_ev)
+    bwd_main_ms = statistics.mean(a.elapsed_time(b) for a, b in bwd_ev)
+    if world > 1:
+        t = torch.tensor([ms_total], device=device, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms_total = float(t.item())
+    ms_step = ms_total / K
+    f_fwd, f_bwd = w.flops_fwd(causal), w.flops_bwd(causal)
+    value = world * (f_fwd + f_bwd) / (ms_step * 1e-3) / 1e12
+
+    # end to end through the C ABI with host buffers: pinned host inputs are
+    # copied in, the step runs, the results are copied back, every step
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv, hdo = (t.cpu().pin_memory() for t in (q, k, v, do))
+        ho, hlse, hdq, hdk, hdv = (torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+                                   for t in (o, lse, dq, dk, dv))
+        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdo))
+        d2h = sum(t.numel() * t.element_size() for t in (ho, hlse, hdq, hdk, hdv))
+
+        def e2e_step():
+            for dst, src in ((q, hq), (k, hk), (v, hv), (do, hdo)):
+                dst.copy_(src, non_blocking=True)
+            step()
+            for dst, src in ((ho, o), (hlse, lse), (hdq, dq), (hdk, dk), (hdv, dv)):
+                dst.copy_(src, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize(device)
+        Ke = max(3, min(K, 10))
+        e0, e1 = ev(), ev()
+        barrier()
+        torch.cuda.synchronize(device)
+        e0.record(stream)
+        for _ in range(Ke):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        barrier()
+        ems = e0.elapsed_time(e1) / Ke
+        if world > 1:
+            t = torch.tensor([ems], device=device, dtype=torch.float64)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            ems = float(t.item())
+        e2e = {"value": world * (f_fwd + f_bwd) / (ems * 1e-3) / 1e12, "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ems}
+
+    pk, pk_kind = peaks()
+    peak = pk["bf16_tflops"]
+    bwd_tflops_main = f_bwd / (bwd_main_ms * 1e-3) / 1e12
+    fwd_tflops = f_fwd / (fwd_ms * 1e-3) / 1e12
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": str(w.dtype).replace("torch.", ""),
+        "data": "synthetic: seeded normals (per-rank CUDA generator) with the workload's shapes and sigmas",
+        "config": {"workload": workload_desc(w, causal), "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv,
+                   "seq_len": w.N, "head_dim": w.d, "causal": causal,
+                   "parallelism": f"replicas x{world} (no exchange)",
+                   "l2": "inputs larger than L2 (no flush)",
+                   "flops_per_step": f_fwd + f_bwd},
+        "pct_of_peak": round(100 * value / world / peak, 2),
+        "fwd_ms": round(fwd_ms, 4), "fwd_tflops": round(fwd_tflops, 2),
+        "fwd_pct_of_peak": round(100 * fwd_tflops / peak, 2),
+        "bwd_main_ms": round(bwd_main_ms, 4), "bwd_main_tflops": round(bwd_tflops_main, 2),
+        "bwd_ms": round(ms_step - fwd_ms, 4),
+        "bwd_tflops": round(f_bwd / ((ms_step - fwd_ms) * 1e-3) / 1e12, 2),
+        "bwd_pct_of_peak": round(100 * f_bwd / ((ms_step - fwd_ms) * 1e-3) / 1e12 / peak, 2),
+        "roofline": {"kernel": "fa_bwd_kernel (main backward pass)", "bound": "tensor",
+                     "achieved": round(bwd_tflops_main, 2), "peak": peak, "unit": "TFLOP/s",
+                     "frac": round(bwd_tflops_main / peak, 4), "peak_kind": f"{pk_kind} bf16 burst",
+                     "traffic": None,
+                     "algorithmic": "2.5 x 4*B*Hq*N^2*d (/2 causal) FLOPs per launch"},
+        "gpu_launches": 4 * K,
+        "clocks": clk,
+        "e2e": e2e,
+    }
+    return line
+
+
+# ---------------------------------------------------------------- CPU oracle
+
+def oracle_sample(w, causal, seconds, rows_hint=None):
+    """Times the fp64 oracle (forward rows + dQ rows) on seeded query rows of
+    one head of the workload; returns (TFLOPS-equivalent, rows, s, threads).
+    Each row carries its share of the workload's conventional FLOPs."""
+    import oracle
+    from exact_io_aware_bwd_b200.workloads import make_inputs
+    g = torch.Generator().manual_seed(w.seed + 3)
+    per_row = (w.flops_fwd(causal) + w.flops_bwd(causal)) / (w.B * w.Hq * w.N)
+    heads_max = min(w.B * w.Hq, 64)
+    q, k, v, do = make_inputs(w, shape_override=(1, heads_max, heads_max, w.N, w.d))
+
+    def run(nrows):
+        # nrows query rows in total: the same seeded rows in each of H heads
+        H = min(heads_max, max(1, -(-nrows // w.N)))
+        per_head = min(w.N, max(1, nrows // H))
+        rows = torch.sort(torch.randperm(w.N, generator=g)[:per_head]).values.numpy()
+        t = time.perf_counter()
+        oracle.fwd_rows(q[:, :H], k[:, :H], v[:, :H], rows, w.scale, causal)
+        oracle.bwd_rows(q[:, :H], k[:, :H], v[:, :H], do[:, :H], rows, w.scale, causal)
+        return time.perf_counter() - t, H * per_head
+
+    threads = oracle.num_threads()
+    if rows_hint is None:
+        probe = max(threads, 8)
+        dt, n = run(probe)
+        rows_hint = max(1, min(heads_max * w.N, int(n * seconds / max(dt, 1e-6))))
+    dt, n = run(rows_hint)
+    return per_row * n / dt / 1e12, n, dt, threads
+
+
+def run_reference(args, w, causal):
+    """The oracle arm: each step is a bounded sample of the same workload."""
+    budget = 150.0
+    per_step = max(0.2, min(10.0, budget / max(1, args.steps + args.warmup)))
+    _, rows, dt, threads = oracle_sample(w, causal, per_step)
+    vals = []
+    for i in range(args.warmup + args.steps):
+        v, _, dt, _ = oracle_sample(w, causal, per_step, rows_hint=rows)
+        if i >= args.warmup:
+            vals.append((v, dt))
+    value = statistics.mean(v for v, _ in vals)
+    ms = 1e3 * statistics.mean(dt for _, dt in vals)
+    sample = (f"{rows} seeded query rows per step (forward O/lse rows + dQ rows, fp64), "
+              f"{workload_desc(w, causal)}")
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 2),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": workload_desc(w, causal)},
+        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+# ---------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="mha4k", choices=sorted(WORKLOADS))
+    ap.add_argument("--noncausal", action="store_true", help="non-causal variant of the workload")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    assert args.warmup >= 0 and args.steps >= 1
+
+    w = WORKLOADS[args.workload]
+    causal = (not args.noncausal) and (True in w.causal_modes)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, w, causal)), flush=True)
+        return
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py: no CUDA device; the product path has no CPU fallback")
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(device)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=device)
+    try:
+        line = run_ours(args, w, causal, rank, world, device)
+        if rank == 0 and not args.no_cpu_baseline:
+            v, rows, dt, threads = oracle_sample(w, causal, args.cpu_seconds)
+            line["cpu_baseline"] = {
+                "value": round(v, 6), "unit": UNIT, "cores": threads, "kind": "oracle",
+                "sample": f"{rows} seeded query rows, forward O/lse rows + dQ rows in fp64, "
+                          f"{dt:.1f} s; each row counted at its share of the workload's FLOPs"}
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,170 @@
+"""ctypes binding of libfa_b200.so: the C ABI of include/fa.h, one Python
+function per entry point with the same name, plus two conveniences that
+allocate outputs with PyTorch.  Argument marshalling only: every step of the
+computation runs in the library's CUDA kernels.  There is no fallback: if the
+library cannot be loaded, every call raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import threading
+
+import torch
+
+from .build import LIB_PATH
+
+FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_MISALIGNED, FA_ERR_CUDA, FA_ERR_TIMEOUT = range(6)
+FA_BF16, FA_FP16 = 0, 1
+
+_DTYPES = {torch.bfloat16: FA_BF16, torch.float16: FA_FP16}
+
+_lock = threading.Lock()
+_lib = None
+
+
+class FaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {fa_status_string(status)} (status {status})")
+
+
+def library_path() -> str:
+    return os.environ.get("FA_B200_LIB", LIB_PATH)
+
+
+def load():
+    """Load libfa_b200.so (built in-tree by build.build()); raise if absent."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            path = library_path()
+            if not os.path.exists(path):
+                raise RuntimeError(
+                    f"{path} is missing: build it with exact_io_aware_bwd_b200.build.build() "
+                    "(there is no fallback implementation)")
+            lib = ctypes.CDLL(path)
+            vp, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+            lib.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp]
+            lib.fa_fwd.restype = i
+            lib.fa_bwd_workspace_bytes.argtypes = [i, i, i, i, i]
+            lib.fa_bwd_workspace_bytes.restype = ctypes.c_size_t
+            lib.fa_bwd.argtypes = ([vp] * 9 + [i, i, i, i, i, f, i, i, vp, ctypes.c_size_t, vp])
+            lib.fa_bwd.restype = i
+            lib.fa_get_device_status.argtypes = [vp]
+            lib.fa_get_device_status.restype = i
+            lib.fa_peek_device_status_word.argtypes = [vp]
+            lib.fa_peek_device_status_word.restype = ctypes.c_uint32
+            lib.fa_selftest_wait_timeout.argtypes = [ctypes.c_uint64, vp]
+            lib.fa_selftest_wait_timeout.restype = i
+            lib.fa_set_profile_events.argtypes = [i, vp, vp]
+            lib.fa_set_profile_events.restype = i
+            lib.fa_status_string.argtypes = [i]
+            lib.fa_status_string.restype = ctypes.c_char_p
+            _lib = lib
+    return _lib
+
+
+def _stream(stream):
+    if stream is None:
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return ctypes.c_void_p(t)
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _check(status: int, where: str):
+    if status != FA_OK:
+        raise FaError(status, where)
+
+
+def _dims(q, k):
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    return B, Hq, Hkv, N, d
+
+
+def fa_status_string(status: int) -> str:
+    return load().fa_status_string(int(status)).decode()
+
+
+def fa_fwd(q, k, v, o, lse, scale: float, causal: bool, stream=None) -> None:
+    """O and lse (natural log) of exact attention into the given tensors.
+    q [B,Hq,N,d], k/v [B,Hkv,N,d] (bf16 or fp16, contiguous, on the GPU)."""
+    B, Hq, Hkv, N, d = _dims(q, k)
+    st = load().fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, N, d,
+                       float(scale), int(bool(causal)), _DTYPES[q.dtype], _stream(stream))
+    _check(st, "fa_fwd")
+
+
+def fa_bwd_workspace_bytes(B: int, Hq: int, Hkv: int, N: int, d: int) -> int:
+    return int(load().fa_bwd_workspace_bytes(B, Hq, Hkv, N, d))
+
+
+def fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, scale: float, causal: bool, workspace,
+           stream=None) -> None:
+    """dQ, dK, dV into the given tensors; workspace: a uint8 GPU tensor of at
+    least fa_bwd_workspace_bytes(...) bytes."""
+    B, Hq, Hkv, N, d = _dims(q, k)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = load().fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq),
+                       _ptr(dk), _ptr(dv), B, Hq, Hkv, N, d, float(scale), int(bool(causal)),
+                       _DTYPES[q.dtype], _ptr(workspace), ws_bytes, _stream(stream))
+    _check(st, "fa_bwd")
+
+
+def fa_get_device_status(stream=None) -> int:
+    return int(load().fa_get_device_status(_stream(stream)))
+
+
+def fa_peek_device_status_word(stream=None) -> int:
+    return int(load().fa_peek_device_status_word(_stream(stream)))
+
+
+def fa_selftest_wait_timeout(limit_ns: int, stream=None) -> int:
+    return int(load().fa_selftest_wait_timeout(int(limit_ns), _stream(stream)))
+
+
+KERNEL_FWD, KERNEL_BWD_MAIN = 1, 3
+
+
+def fa_set_profile_events(kernel_id: int, start=None, stop=None) -> None:
+    """Bracket every launch of a kernel with two CUDA events (torch.cuda.Event
+    objects that have been recorded once, or raw handles); None clears."""
+    h = lambda e: None if e is None else ctypes.c_void_p(e.cuda_event if hasattr(e, "cuda_event") else int(e))
+    _check(load().fa_set_profile_events(int(kernel_id), h(start), h(stop)), "fa_set_profile_events")
+
+
+# ------------------------------------------------------------ conveniences
+
+def attention_fwd(q, k, v, scale: float | None = None, causal: bool = False, stream=None):
+    """Allocates O and lse with PyTorch and runs fa_fwd; returns (O, lse)."""
+    B, Hq, Hkv, N, d = _dims(q, k)
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, N), device=q.device, dtype=torch.float32)
+    fa_fwd(q, k, v, o, lse, scale, causal, stream)
+    return o, lse
+
+
+def attention_bwd(q, k, v, o, dout, lse, scale: float | None = None, causal: bool = False,
+                  workspace=None, stream=None):
+    """Allocates dQ, dK, dV (and the workspace if not given) and runs fa_bwd."""
+    B, Hq, Hkv, N, d = _dims(q, k)
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    if workspace is None:
+        workspace = torch.empty(max(fa_bwd_workspace_bytes(B, Hq, Hkv, N, d), 16),
+                                device=q.device, dtype=torch.uint8)
+    fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, scale, causal, workspace, stream)
+    return dq, dk, dv

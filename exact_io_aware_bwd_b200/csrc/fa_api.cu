@@ -1,0 +1,330 @@
+// Host side of libfa_b200.so: argument checks, TMA tensor maps and kernel
+// launches behind the C ABI declared in include/fa.h.  The whole library is
+// this one translation unit (the kernels are included below).
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <algorithm>
+#include <mutex>
+
+#include "fa.h"
+#include "sm100.cuh"
+#include "fa_fwd.cuh"
+#include "fa_bwd.cuh"
+
+namespace {
+
+using fa::FwdLayout;
+using fa::FwdParams;
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  return g_encode;
+}
+
+// 3-D tiled map over a dense [outer][rows][cols] tensor (cols contiguous),
+// copied in boxes of box_rows x box_cols with 128-byte swizzle.  Out-of-range
+// rows read as zero and are skipped on stores.
+bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esize, uint64_t cols,
+              uint64_t rows, uint64_t outer, uint32_t box_cols, uint32_t box_rows) {
+  auto enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {cols, rows, outer};
+  cuuint64_t strides[2] = {cols * esize, cols * rows * esize};
+  cuuint32_t box[3] = {box_cols, box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Events bracketing the launches of one kernel (see fa_set_profile_events).
+cudaEvent_t g_prof_start[8] = {nullptr};
+cudaEvent_t g_prof_stop[8] = {nullptr};
+
+void prof_begin(int id, cudaStream_t st) {
+  if (g_prof_start[id]) cudaEventRecord(g_prof_start[id], st);
+}
+void prof_end(int id, cudaStream_t st) {
+  if (g_prof_stop[id]) cudaEventRecord(g_prof_stop[id], st);
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Device must be sm_100 (B200 class); checked once per device.
+fa_status_t check_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
+  static int ok_dev[64] = {0};  // 0 unknown, 1 ok, 2 not ok
+  if (dev < 0 || dev >= 64) return FA_ERR_UNSUPPORTED;
+  if (ok_dev[dev] == 0) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+      return FA_ERR_CUDA;
+    ok_dev[dev] = (major == 10 && minor == 0) ? 1 : 2;
+  }
+  return ok_dev[dev] == 1 ? FA_OK : FA_ERR_UNSUPPORTED;
+}
+
+// Checks shared by fa_fwd and fa_bwd.  Sets *empty for a problem with no work.
+fa_status_t check_common(int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+                         fa_dtype_t dtype, bool* empty) {
+  if (B < 0 || N < 0 || Hq <= 0 || Hkv <= 0) return FA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return FA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  if (dtype != FA_BF16 && dtype != FA_FP16) return FA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  // sizes the kernels index with 32-bit block counts and TMA coordinates
+  const int64_t tiles = (static_cast<int64_t>(N) + 127) / 128;
+  if (static_cast<int64_t>(B) * Hq * tiles > INT32_MAX) return FA_ERR_UNSUPPORTED;
+  *empty = (B == 0 || N == 0);
+  return FA_OK;
+}
+
+// Opt a kernel into `smem` bytes of dynamic shared memory (once per kernel).
+template <typename K>
+fa_status_t opt_in_smem(K kernel, int smem) {
+  static std::mutex mu;
+  static const void* done[64];
+  static int n_done = 0;
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < n_done; ++i)
+    if (done[i] == reinterpret_cast<const void*>(kernel)) return FA_OK;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return FA_ERR_CUDA;
+  if (n_done < 64) done[n_done++] = reinterpret_cast<const void*>(kernel);
+  return FA_OK;
+}
+
+template <int HD, bool BF, bool CA>
+fa_status_t launch_fwd(const FwdParams& prm, cudaStream_t st) {
+  auto kern = fa::fa_fwd_kernel<HD, BF, CA>;
+  const int smem = FwdLayout<HD>::kDynSmem;
+  fa_status_t s = opt_in_smem(kern, smem);
+  if (s != FA_OK) return s;
+  const int grid = prm.n_qtiles * prm.BH;
+  prof_begin(fa::kKernFwd, st);
+  kern<<<grid, fa::kFwdThreads, smem, st>>>(prm);
+  const bool ok = cudaGetLastError() == cudaSuccess;
+  prof_end(fa::kKernFwd, st);
+  return ok ? FA_OK : FA_ERR_CUDA;
+}
+
+template <int HD, bool BF>
+fa_status_t launch_fwd_c(const FwdParams& prm, int causal, cudaStream_t st) {
+  return causal ? launch_fwd<HD, BF, true>(prm, st) : launch_fwd<HD, BF, false>(prm, st);
+}
+
+template <int HD, bool BF, bool CA>
+fa_status_t launch_bwd_main(const fa::BwdParams& prm, int grid, cudaStream_t st) {
+  auto kern = fa::fa_bwd_kernel<HD, BF, CA>;
+  const int smem = fa::BwdLayout<HD>::kDynSmem;
+  fa_status_t s = opt_in_smem(kern, smem);
+  if (s != FA_OK) return s;
+  prof_begin(fa::kKernBwd, st);
+  kern<<<grid, fa::kBwdThreads, smem, st>>>(prm);
+  const bool ok = cudaGetLastError() == cudaSuccess;
+  prof_end(fa::kKernBwd, st);
+  return ok ? FA_OK : FA_ERR_CUDA;
+}
+
+template <int HD, bool BF>
+fa_status_t bwd_run(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                    const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N,
+                    float scale, int causal, void* workspace, cudaStream_t st) {
+  const int64_t Np = fa::bwd_padded_rows(N);
+  const int64_t BHq = static_cast<int64_t>(B) * Hq, BHkv = static_cast<int64_t>(B) * Hkv;
+  float* Dvec = static_cast<float*>(workspace);
+  float* lse2 = Dvec + BHq * Np;
+  float* dqacc = lse2 + BHq * Np;
+
+  // 1. D, lse2, zeroed accumulator
+  const int64_t rows = BHq * Np;
+  fa::fa_bwd_pre_kernel<HD, BF><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(
+      o, dout, lse, Dvec, lse2, dqacc, N, static_cast<int>(Np), rows);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+
+  // 2. main pass
+  const CUtensorMapDataType dt = BF ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  fa::BwdParams prm;
+  std::memset(&prm, 0, sizeof(prm));
+  if (!make_map(&prm.tm_q, q, dt, 2, HD, N, BHq, 64, 64) ||
+      !make_map(&prm.tm_do, dout, dt, 2, HD, N, BHq, 64, 64) ||
+      !make_map(&prm.tm_k, k, dt, 2, HD, N, BHkv, 64, 128) ||
+      !make_map(&prm.tm_v, v, dt, 2, HD, N, BHkv, 64, 128) ||
+      !make_map(&prm.tm_dqacc, dqacc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, HD, Np, BHq, 32, 32))
+    return FA_ERR_CUDA;
+  prm.lse2 = lse2;
+  prm.Dvec = Dvec;
+  prm.dk = dk;
+  prm.dv = dv;
+  prm.N = N;
+  prm.Np = static_cast<int>(Np);
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  prm.group = Hq / Hkv;
+  prm.n_ktiles = (N + 127) / 128;
+  prm.n_qtiles = (N + 63) / 64;
+  prm.BHkv = static_cast<int>(BHkv);
+  prm.scale = scale;
+  prm.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  const int grid = prm.n_ktiles * prm.BHkv;
+  fa_status_t s = causal ? launch_bwd_main<HD, BF, true>(prm, grid, st)
+                         : launch_bwd_main<HD, BF, false>(prm, grid, st);
+  if (s != FA_OK) return s;
+
+  // 3. dQ = scale * accumulator
+  const int64_t total_vec = BHq * N * (HD / 8);
+  const int64_t blocks = std::min<int64_t>((total_vec + 255) / 256, 148 * 16);
+  fa::fa_bwd_post_kernel<HD, BF><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+      dqacc, dq, N, static_cast<int>(Np), total_vec, scale);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+fa_status_t fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                   int Hq, int Hkv, int N, int d, float scale, int causal, fa_dtype_t dtype,
+                   void* stream) {
+  bool empty = false;
+  fa_status_t s = check_common(B, Hq, Hkv, N, d, scale, causal, dtype, &empty);
+  if (s != FA_OK) return s;
+  if (empty) return FA_OK;
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return FA_ERR_MISALIGNED;
+  if ((s = check_device()) != FA_OK) return s;
+
+  const bool bf = dtype == FA_BF16;
+  const CUtensorMapDataType dt = bf ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  FwdParams prm;
+  std::memset(&prm, 0, sizeof(prm));
+  const uint64_t BHq = static_cast<uint64_t>(B) * Hq, BHkv = static_cast<uint64_t>(B) * Hkv;
+  if (!make_map(&prm.tm_q, q, dt, 2, d, N, BHq, 64, 128) ||
+      !make_map(&prm.tm_k, k, dt, 2, d, N, BHkv, 64, 128) ||
+      !make_map(&prm.tm_v, v, dt, 2, d, N, BHkv, 64, 128) ||
+      !make_map(&prm.tm_o, o, dt, 2, d, N, BHq, 64, 128))
+    return FA_ERR_CUDA;
+  prm.lse = lse;
+  prm.N = N;
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  prm.group = Hq / Hkv;
+  prm.BH = static_cast<int>(BHq);
+  prm.n_qtiles = (N + 127) / 128;
+  prm.n_ktiles = (N + 127) / 128;
+  prm.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (d == 128) return bf ? launch_fwd_c<128, true>(prm, causal, st) : launch_fwd_c<128, false>(prm, causal, st);
+  return bf ? launch_fwd_c<64, true>(prm, causal, st) : launch_fwd_c<64, false>(prm, causal, st);
+}
+
+size_t fa_bwd_workspace_bytes(int B, int Hq, int Hkv, int N, int d) {
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || N <= 0 || d <= 0) return 0;
+  return fa::bwd_workspace_bytes(B, Hq, N, d);
+}
+
+fa_status_t fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                   const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N,
+                   int d, float scale, int causal, fa_dtype_t dtype, void* workspace,
+                   size_t workspace_bytes, void* stream) {
+  bool empty = false;
+  fa_status_t s = check_common(B, Hq, Hkv, N, d, scale, causal, dtype, &empty);
+  if (s != FA_OK) return s;
+  if (empty) return FA_OK;
+  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv || !workspace)
+    return FA_ERR_INVALID_ARG;
+  if (workspace_bytes < fa::bwd_workspace_bytes(B, Hq, N, d)) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
+      !aligned16(lse) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
+      !aligned16(workspace))
+    return FA_ERR_MISALIGNED;
+  if ((s = check_device()) != FA_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const bool bf = dtype == FA_BF16;
+  if (d == 128)
+    return bf ? bwd_run<128, true>(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, N, scale, causal, workspace, st)
+              : bwd_run<128, false>(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, N, scale, causal, workspace, st);
+  return bf ? bwd_run<64, true>(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, N, scale, causal, workspace, st)
+            : bwd_run<64, false>(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, N, scale, causal, workspace, st);
+}
+
+fa_status_t fa_get_device_status(void* stream) {
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return FA_ERR_CUDA;
+  uint32_t word = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&word, fa::g_device_status, sizeof(word)) != cudaSuccess)
+    return FA_ERR_CUDA;
+  if (word == 0) return FA_OK;
+  if (cudaMemcpyToSymbol(fa::g_device_status, &zero, sizeof(zero)) != cudaSuccess)
+    return FA_ERR_CUDA;
+  const uint32_t code = word & 0xFFu;
+  return code == fa::kStatusTimeout ? FA_ERR_TIMEOUT : FA_ERR_CUDA;
+}
+
+uint32_t fa_peek_device_status_word(void* stream) {
+  cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+  uint32_t word = 0;
+  cudaMemcpyFromSymbol(&word, fa::g_device_status, sizeof(word));
+  return word;
+}
+
+fa_status_t fa_selftest_wait_timeout(uint64_t limit_ns, void* stream) {
+  fa_status_t s = check_device();
+  if (s != FA_OK) return s;
+  if (limit_ns == 0 || limit_ns > 10ull * 1000 * 1000 * 1000) return FA_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // clear any earlier status, shorten the limit, run, restore
+  if ((s = fa_get_device_status(stream)) == FA_ERR_CUDA) return s;
+  const uint64_t dflt = 2000000000ull;
+  if (cudaMemcpyToSymbolAsync(fa::g_wait_limit_ns, &limit_ns, sizeof(limit_ns), 0,
+                              cudaMemcpyHostToDevice, st) != cudaSuccess)
+    return FA_ERR_CUDA;
+  fa::wait_timeout_selftest_kernel<<<1, 32, 0, st>>>();
+  const bool launched = cudaGetLastError() == cudaSuccess;
+  cudaMemcpyToSymbolAsync(fa::g_wait_limit_ns, &dflt, sizeof(dflt), 0, cudaMemcpyHostToDevice, st);
+  if (!launched) return FA_ERR_CUDA;
+  return fa_get_device_status(stream);
+}
+
+fa_status_t fa_set_profile_events(int kernel_id, void* start, void* stop) {
+  if (kernel_id != static_cast<int>(fa::kKernFwd) && kernel_id != static_cast<int>(fa::kKernBwd))
+    return FA_ERR_INVALID_ARG;
+  if ((start == nullptr) != (stop == nullptr)) return FA_ERR_INVALID_ARG;
+  g_prof_start[kernel_id] = reinterpret_cast<cudaEvent_t>(start);
+  g_prof_stop[kernel_id] = reinterpret_cast<cudaEvent_t>(stop);
+  return FA_OK;
+}
+
+const char* fa_status_string(fa_status_t status) {
+  switch (status) {
+    case FA_OK: return "ok";
+    case FA_ERR_INVALID_ARG: return "invalid argument";
+    case FA_ERR_UNSUPPORTED: return "unsupported configuration or device";
+    case FA_ERR_MISALIGNED: return "tensor pointer not 16-byte aligned";
+    case FA_ERR_CUDA: return "CUDA error";
+    case FA_ERR_TIMEOUT: return "device-side barrier wait timed out";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

@@ -1,0 +1,547 @@
+// Backward pass of exact attention on sm_100a, by recomputation.
+//
+// The pages keep only the softmax statistics from the forward pass and
+// recompute the scores on chip in the backward pass ("FlashAttention"
+// glossary, recomputation paragraph), and let one thread block own a block of
+// keys so that dK and dV need no atomics ("FlashAttention" glossary,
+// FlashAttention-2 list, backward-pass item).  The gradient formulas are the
+// calculus of softmax (the pages print none):
+//   P_ij  = exp(scale s_ij - lse_i)            (recomputed, s = q.k)
+//   dV_j  = sum_i P_ij dO_i
+//   dP_ij = dO_i . v_j
+//   D_i   = sum_j P_ij dP_ij = dO_i . O_i
+//   dS_ij = P_ij (dP_ij - D_i)
+//   dQ_i  = scale sum_j dS_ij k_j,   dK_j = scale sum_i dS_ij q_i
+//
+// Three kernels:
+//   bwd_pre   one warp per query row: D_i = dO_i . O_i, lse2_i = lse_i log2(e)
+//             (+inf for padding rows, which makes their P exactly 0), and a
+//             zeroed fp32 dQ accumulator row.
+//   bwd_main  one thread block per (128-row key block j, kv head): K_j, V_j
+//             stay in shared memory; the block walks every query head of the
+//             group and every 64-row query block i (causal: i >= the
+//             diagonal).  Per step, all products on the tensor cores with
+//             fp32 accumulators in tensor memory:
+//               S^T  = K_j Q_i^T        (128 x 64)
+//               dP^T = V_j dO_i^T       (128 x 64)
+//               softmax warps: P^T, dS^T = P^T o (dP^T - D)
+//               dQ_i^T = K_j^T dS^T     (d x 64) -> TMA reduce-add (fp32) into
+//                                        the dQ accumulator in L2
+//               dV  += P^T dO_i         (P^T read from tensor memory)
+//               dK  += dS^T Q_i
+//             dK, dV stay in tensor memory for the whole walk and are written
+//             once at the end: no atomics on them.
+//   bwd_post  dQ = scale * accumulator, converted to the I/O dtype.
+//
+// Warp roles of bwd_main (448 threads):
+//   warps 0-7   softmax-gradient: warp w owns key rows 32(w%4)..+31 (tensor
+//               memory lanes) and query columns 32(w/4)..+31 of each step.
+//   warps 8-11  dQ drain (lane = feature index of dQ^T) and, at the end, the
+//               dK / dV epilogue (lane = key row).
+//   warp 12     TMA producer.     warp 13     MMA issuer (one thread).
+// Tensor memory: dV [0,128), dK [128,256), and two step buffers b = 0, 1:
+// S^T at 256+128b (64 columns; P^T is written over it as 16-bit pairs, each
+// warp half over its own columns) and dP^T at 256+128b+64 (dQ^T is written
+// over it once the softmax warps have read dP^T).  The step buffers let the
+// tensor cores compute step t+1's S^T / dP^T while the softmax warps work on
+// step t.
+#pragma once
+
+#include <type_traits>
+
+#include "sm100.cuh"
+
+namespace fa {
+
+constexpr uint32_t kKernBwdPre = 2;
+constexpr uint32_t kKernBwd = 3;
+constexpr uint32_t kKernBwdPost = 4;
+constexpr uint32_t kKernSelftest = 9;
+
+__host__ __device__ inline int64_t bwd_padded_rows(int N) { return (static_cast<int64_t>(N) + 127) / 128 * 128; }
+
+inline size_t bwd_workspace_bytes(int B, int Hq, int N, int d) {
+  const int64_t rows = static_cast<int64_t>(B) * Hq * bwd_padded_rows(N);
+  return static_cast<size_t>(rows) * 4u * static_cast<size_t>(2 + d);
+}
+
+// ---------------------------------------------------------------------------
+// bwd_pre
+
+template <int HD, bool BF16>
+__global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const void* __restrict__ o_,
+                                                         const void* __restrict__ do_,
+                                                         const float* __restrict__ lse,
+                                                         float* __restrict__ Dvec,
+                                                         float* __restrict__ lse2,
+                                                         float* __restrict__ dqacc, int N, int Np,
+                                                         int64_t total_rows) {
+  using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= total_rows) return;
+  const int64_t bh = row / Np;
+  const int n = static_cast<int>(row % Np);
+  constexpr int kPer = HD / 32;  // elements per lane: 2 or 4
+  float acc = 0.f;
+  if (n < N) {
+    const int64_t base = (bh * N + n) * HD + lane * kPer;
+    const T* o = reinterpret_cast<const T*>(o_) + base;
+    const T* d = reinterpret_cast<const T*>(do_) + base;
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) acc += static_cast<float>(o[e]) * static_cast<float>(d[e]);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if (lane == 0) {
+    Dvec[row] = acc;
+    lse2[row] = n < N ? lse[bh * N + n] * 1.4426950408889634f : INFINITY;
+  }
+  float* z = dqacc + row * HD + lane * kPer;
+#pragma unroll
+  for (int e = 0; e < kPer; ++e) z[e] = 0.f;
+}
+
+// ---------------------------------------------------------------------------
+// bwd_main
+
+struct BwdParams {
+  CUtensorMap tm_q;      // [B*Hq][N][d], box 64 cols x 64 rows
+  CUtensorMap tm_do;     // [B*Hq][N][d], box 64 x 64
+  CUtensorMap tm_k;      // [B*Hkv][N][d], box 64 x 128
+  CUtensorMap tm_v;      // [B*Hkv][N][d], box 64 x 128
+  CUtensorMap tm_dqacc;  // fp32 [B*Hq][Np][d], box 32 cols x 32 rows (reduce-add)
+  const float* lse2;     // [B*Hq][Np]
+  const float* Dvec;     // [B*Hq][Np]
+  void* dk;              // [B*Hkv][N][d]
+  void* dv;
+  int N, Np, Hq, Hkv, group, n_ktiles, n_qtiles, BHkv;
+  float scale_log2, scale;
+};
+
+template <int HD>
+struct BwdLayout {
+  static constexpr int kStages = 3;                     // Q / dO / lse2 / D ring
+  static constexpr int kChunks = HD / 64;
+  static constexpr int kKVBox = 128 * 128;              // 128 rows x 64 cols x 2 B
+  static constexpr int kQBox = 64 * 128;                // 64 rows x 64 cols x 2 B
+  static constexpr int kKVTile = kChunks * kKVBox;
+  static constexpr int kQTile = kChunks * kQBox;
+  static constexpr int kDsBytes = 128 * 128;            // dS^T: 128 key rows x 64 query cols x 2 B
+  static constexpr int kDqHalf = 32 * HD * 4;           // 32 query rows x d fp32
+  static constexpr int kOffK = 0;
+  static constexpr int kOffV = kOffK + kKVTile;
+  static constexpr int kOffQ = kOffV + kKVTile;
+  static constexpr int kOffDO = kOffQ + kStages * kQTile;
+  static constexpr int kOffDS = kOffDO + kStages * kQTile;
+  static constexpr int kOffDQ = kOffDS + 2 * kDsBytes;
+  static constexpr int kOffLse = kOffDQ + 2 * kDqHalf;
+  static constexpr int kOffD = kOffLse + kStages * 256;
+  static constexpr int kOffBar = kOffD + kStages * 256;
+  // kv_full, q_full[S], q_empty[S], s_full[2], dp_full[2], ds_full[2], pt_free[2],
+  // dq_full[2], dq_drained[2], ds_free[2], acc_done, done
+  static constexpr int kNumBars = 1 + 2 * kStages + 7 * 2 + 2;
+  static constexpr int kOffTmemPtr = kOffBar + kNumBars * 8;
+  static constexpr int kOffAbort = kOffTmemPtr + 4;
+  static constexpr int kSmemBytes = kOffAbort + 4;
+  static constexpr int kDynSmem = kSmemBytes + 1024;
+  static_assert(kDynSmem <= 232448, "shared memory budget");
+};
+
+constexpr int kBwdThreads = 448;
+
+template <int HD, bool BF16, bool CAUSAL>
+__global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_constant__ BwdParams p) {
+  using L = BwdLayout<HD>;
+  using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                           ~static_cast<uintptr_t>(1023));
+  uint8_t* sK = sm + L::kOffK;
+  uint8_t* sV = sm + L::kOffV;
+  uint8_t* sQ = sm + L::kOffQ;
+  uint8_t* sDO = sm + L::kOffDO;
+  uint8_t* sDS = sm + L::kOffDS;
+  uint8_t* sDQ = sm + L::kOffDQ;
+  float* sLse = reinterpret_cast<float*>(sm + L::kOffLse);
+  float* sD = reinterpret_cast<float*>(sm + L::kOffD);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::kOffBar);
+  uint64_t* kv_full = bars;
+  uint64_t* q_full = kv_full + 1;
+  uint64_t* q_empty = q_full + L::kStages;
+  uint64_t* s_full = q_empty + L::kStages;
+  uint64_t* dp_full = s_full + 2;
+  uint64_t* ds_full = dp_full + 2;
+  uint64_t* pt_free = ds_full + 2;
+  uint64_t* dq_full = pt_free + 2;
+  uint64_t* dq_drained = dq_full + 2;
+  uint64_t* ds_free = dq_drained + 2;
+  uint64_t* acc_done = ds_free + 2;
+  uint64_t* done_bar = acc_done + 1;
+  uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(sm + L::kOffTmemPtr);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::kOffAbort);
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+
+  // Work item: key blocks nearest the start first (under a causal mask they
+  // see the most query blocks).
+  const int item = blockIdx.x;
+  const int jt = item / p.BHkv;     // key block (128 rows)
+  const int kvh = item % p.BHkv;    // b * Hkv + g
+  const int b = kvh / p.Hkv;
+  const int g = kvh % p.Hkv;
+  const int kv0 = jt * 128;
+  const int i0 = CAUSAL ? 2 * jt : 0;       // first query block (64 rows) that sees key block jt
+  const int nq = p.n_qtiles - i0;            // query blocks per head
+  const int T_steps = p.group * nq;
+  constexpr int kDrainThreads = HD == 128 ? 128 : 64;
+
+  if (tid == 0) {
+    mbar_init(kv_full, 1);
+    for (int s = 0; s < L::kStages; ++s) {
+      mbar_init(&q_full[s], 1);
+      mbar_init(&q_empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&dp_full[i], 1);
+      mbar_init(&ds_full[i], 256);
+      mbar_init(&pt_free[i], 1);
+      mbar_init(&dq_full[i], 1);
+      mbar_init(&dq_drained[i], kDrainThreads);
+      mbar_init(&ds_free[i], 1);
+    }
+    mbar_init(acc_done, 1);
+    mbar_init(done_bar, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 13) {
+    tmem_alloc(tmem_ptr, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_ptr;
+  const uint32_t tm_dV = tmem;
+  const uint32_t tm_dK = tmem + 128;
+  auto tm_S = [&](int buf) { return tmem + 256 + 128 * buf; };
+  auto tm_dP = [&](int buf) { return tmem + 256 + 128 * buf + 64; };
+  // step t -> (query head, query block)
+  auto step_bh = [&](int t) { return b * p.Hq + g * p.group + t / nq; };
+  auto step_qt = [&](int t) { return i0 + t % nq; };
+
+  if (warp == 12) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tensormap(&p.tm_q);
+      prefetch_tensormap(&p.tm_do);
+      prefetch_tensormap(&p.tm_k);
+      prefetch_tensormap(&p.tm_v);
+      mbar_expect_tx(kv_full, 2 * L::kKVTile);
+      for (int c = 0; c < L::kChunks; ++c) {
+        tma_load_3d(sK + c * L::kKVBox, &p.tm_k, kv_full, c * 64, kv0, kvh);
+        tma_load_3d(sV + c * L::kKVBox, &p.tm_v, kv_full, c * 64, kv0, kvh);
+      }
+      for (int t = 0; t < T_steps; ++t) {
+        const int s = t % L::kStages;
+        if (t >= L::kStages &&
+            !mbar_wait(&q_empty[s], ((t / L::kStages) - 1) & 1, abort_flag, kKernBwd, 12, 0))
+          break;
+        const int bh = step_bh(t), qt = step_qt(t);
+        mbar_expect_tx(&q_full[s], 2 * L::kQTile + 512);
+        for (int c = 0; c < L::kChunks; ++c) {
+          tma_load_3d(sQ + s * L::kQTile + c * L::kQBox, &p.tm_q, &q_full[s], c * 64, qt * 64, bh);
+          tma_load_3d(sDO + s * L::kQTile + c * L::kQBox, &p.tm_do, &q_full[s], c * 64, qt * 64,
+                      bh);
+        }
+        const int64_t row0 = static_cast<int64_t>(bh) * p.Np + qt * 64;
+        bulk_load(sLse + s * 64, p.lse2 + row0, 256, &q_full[s]);
+        bulk_load(sD + s * 64, p.Dvec + row0, 256, &q_full[s]);
+      }
+    }
+  } else if (warp == 13) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t kIdS = idesc_f16(BF16, 128, 64, false, false);    // S^T, dP^T
+      constexpr uint32_t kIdDQ = idesc_f16(BF16, 128, 64, true, true);     // dQ^T = K^T dS^T
+      constexpr uint32_t kIdAcc = idesc_f16(BF16, 128, HD, false, true);   // dV, dK
+      const uint32_t kb = smem_u32(sK), vb = smem_u32(sV), dsb = smem_u32(sDS);
+      bool ok = mbar_wait(kv_full, 0, abort_flag, kKernBwd, 13, 0);
+      tc_fence_after();
+      auto issue_s = [&](int t) -> bool {
+        const int s = t % L::kStages;
+        if (!mbar_wait(&q_full[s], (t / L::kStages) & 1, abort_flag, kKernBwd, 13, 1)) return false;
+        tc_fence_after();
+        const uint32_t qb = smem_u32(sQ + s * L::kQTile);
+#pragma unroll
+        for (int k = 0; k < HD / 16; ++k)
+          umma_ss(tm_S(t & 1),
+                  sdesc_sw128(kb + (k >> 2) * L::kKVBox + (k & 3) * 32, 16, 1024),
+                  sdesc_sw128(qb + (k >> 2) * L::kQBox + (k & 3) * 32, 16, 1024), kIdS, k > 0);
+        umma_commit(&s_full[t & 1]);
+        return true;
+      };
+      auto issue_dp = [&](int t) {
+        const int s = t % L::kStages;
+        const uint32_t ob = smem_u32(sDO + s * L::kQTile);
+#pragma unroll
+        for (int k = 0; k < HD / 16; ++k)
+          umma_ss(tm_dP(t & 1),
+                  sdesc_sw128(vb + (k >> 2) * L::kKVBox + (k & 3) * 32, 16, 1024),
+                  sdesc_sw128(ob + (k >> 2) * L::kQBox + (k & 3) * 32, 16, 1024), kIdS, k > 0);
+        umma_commit(&dp_full[t & 1]);
+      };
+      for (int t = 0; ok && t < 2 && t < T_steps; ++t) {
+        ok = issue_s(t);
+        if (ok) issue_dp(t);
+      }
+      for (int t = 0; ok && t < T_steps; ++t) {
+        const int buf = t & 1, s = t % L::kStages;
+        if (!mbar_wait(&ds_full[buf], (t >> 1) & 1, abort_flag, kKernBwd, 13, 2)) break;
+        tc_fence_after();
+        const uint32_t qb = smem_u32(sQ + s * L::kQTile);
+        const uint32_t ob = smem_u32(sDO + s * L::kQTile);
+        const uint32_t db = dsb + buf * L::kDsBytes;
+        // dQ^T (d x 64) = K^T dS^T over the 128 keys, into the dP^T columns.
+        // K^T is K read MN-major; its second 64-feature half sits kKVBox bytes
+        // further (for d = 64 that is V: rows 64..127 of the product are
+        // unused).
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          umma_ss(tm_dP(buf), sdesc_sw128(kb + k * 2048, L::kKVBox, 1024),
+                  sdesc_sw128(db + k * 2048, 8192, 1024), kIdDQ, k > 0);
+        umma_commit(&dq_full[buf]);
+        // dV += P^T dO: P^T from tensor memory (each 32-query half of it sits
+        // at the start of its own 32-column group), dO read MN-major.
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          umma_ts(tm_dV, tm_S(buf) + (k >> 1) * 32 + (k & 1) * 8,
+                  sdesc_sw128(ob + k * 2048, L::kQBox, 1024), kIdAcc, (t > 0 || k > 0) ? 1u : 0u);
+        umma_commit(&pt_free[buf]);
+        // dK += dS^T Q: dS^T K-major from shared memory, Q read MN-major.
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          umma_ss(tm_dK, sdesc_sw128(db + k * 32, 16, 1024),
+                  sdesc_sw128(qb + k * 2048, L::kQBox, 1024), kIdAcc, (t > 0 || k > 0) ? 1u : 0u);
+        umma_commit(&ds_free[buf]);
+        umma_commit(&q_empty[s]);
+        if (t + 2 < T_steps) {
+          // S^T_{t+2} overwrites P^T_t: wait for dV_t; dP^T_{t+2} overwrites
+          // dQ^T_t: wait for the drain warps to have read it.
+          if (!mbar_wait(&pt_free[buf], (t >> 1) & 1, abort_flag, kKernBwd, 13, 3)) break;
+          tc_fence_after();
+          if (!issue_s(t + 2)) break;
+          if (!mbar_wait(&dq_drained[buf], (t >> 1) & 1, abort_flag, kKernBwd, 13, 4)) break;
+          tc_fence_after();
+          issue_dp(t + 2);
+        }
+      }
+      umma_commit(acc_done);
+      umma_commit(done_bar);
+      mbar_wait(done_bar, 0, abort_flag, kKernBwd, 13, 5);
+    }
+  } else if (warp < 8) {
+    // ------------------------------------------------------------ softmax gradient
+    const int quarter = warp & 3, half = warp >> 2;
+    const int r = quarter * 32 + lane;                 // key row within the block
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const int kv_row = kv0 + r;
+    const bool row_valid = kv_row < p.N;
+    const float c_log2 = p.scale_log2;
+    for (int t = 0; t < T_steps; ++t) {
+      const int buf = t & 1, s = t % L::kStages;
+      const int q_first = step_qt(t) * 64 + half * 32;  // first query of this thread's columns
+      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[buf], (t >> 1) & 1, abort_flag, kKernBwd, 0, 0)))
+        break;
+      tc_fence_after();
+      uint32_t v[32];
+      tmem_ld32(tm_S(buf) + lane_off + half * 32, v);
+      const float4* lse4 = reinterpret_cast<const float4*>(sLse + s * 64 + half * 32);
+      float pr[32];
+      tmem_ld_wait();
+#pragma unroll
+      for (int c4 = 0; c4 < 8; ++c4) {
+        const float4 l4 = lse4[c4];
+        pr[4 * c4 + 0] = ex2_approx(fmaf(__uint_as_float(v[4 * c4 + 0]), c_log2, -l4.x));
+        pr[4 * c4 + 1] = ex2_approx(fmaf(__uint_as_float(v[4 * c4 + 1]), c_log2, -l4.y));
+        pr[4 * c4 + 2] = ex2_approx(fmaf(__uint_as_float(v[4 * c4 + 2]), c_log2, -l4.z));
+        pr[4 * c4 + 3] = ex2_approx(fmaf(__uint_as_float(v[4 * c4 + 3]), c_log2, -l4.w));
+      }
+      // causal: key kv_row is hidden from queries before it; padding keys
+      // (kv_row >= N) carry no probability
+      if (!row_valid) {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) pr[c] = 0.f;
+      } else if (CAUSAL && q_first < kv_row) {
+#pragma unroll
+        for (int c = 0; c < 32; ++c)
+          if (q_first + c < kv_row) pr[c] = 0.f;
+      }
+      uint32_t pk[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) pk[i] = pack2<BF16>(pr[2 * i], pr[2 * i + 1]);
+      tmem_st16(tm_S(buf) + lane_off + half * 32, pk);
+      if (!__all_sync(0xffffffffu, mbar_wait(&dp_full[buf], (t >> 1) & 1, abort_flag, kKernBwd, 0, 1)))
+        break;
+      tc_fence_after();
+      tmem_ld32(tm_dP(buf) + lane_off + half * 32, v);
+      const float4* d4 = reinterpret_cast<const float4*>(sD + s * 64 + half * 32);
+      tmem_ld_wait();
+#pragma unroll
+      for (int c4 = 0; c4 < 8; ++c4) {
+        const float4 dd = d4[c4];
+        pr[4 * c4 + 0] *= __uint_as_float(v[4 * c4 + 0]) - dd.x;
+        pr[4 * c4 + 1] *= __uint_as_float(v[4 * c4 + 1]) - dd.y;
+        pr[4 * c4 + 2] *= __uint_as_float(v[4 * c4 + 2]) - dd.z;
+        pr[4 * c4 + 3] *= __uint_as_float(v[4 * c4 + 3]) - dd.w;
+      }
+#pragma unroll
+      for (int i = 0; i < 16; ++i) pk[i] = pack2<BF16>(pr[2 * i], pr[2 * i + 1]);
+      // dS^T buffer `buf` is free once dK_{t-2} (its last reader) has completed
+      if (t >= 2 &&
+          !__all_sync(0xffffffffu, mbar_wait(&ds_free[buf], ((t >> 1) - 1) & 1, abort_flag, kKernBwd, 0, 2)))
+        break;
+      uint8_t* row_base = sDS + buf * L::kDsBytes + r * 128;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int chunk = (half * 4 + u) ^ (r & 7);
+        *reinterpret_cast<uint4*>(row_base + chunk * 16) =
+            make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+      }
+      fence_proxy_async_smem();
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&ds_full[buf]);
+    }
+  } else {
+    // ------------------------------------------------------------ dQ drain, dK/dV epilogue
+    // Each drain warp owns 32 features of dQ^T (one 128-byte column box of
+    // the staging tile) and issues its own TMA reduce-adds, so the drain
+    // needs no barrier across warps.
+    const int dw = warp - 8;                           // 0..3 == lane quarter
+    const uint32_t lane_off = static_cast<uint32_t>(dw * 32) << 16;
+    const bool drains = dw * 32 < HD;                  // warp holds real dQ^T rows
+    int groups = 0;                                    // bulk groups committed by lane 0
+    for (int t = 0; drains && t < T_steps; ++t) {
+      const int buf = t & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(&dq_full[buf], (t >> 1) & 1, abort_flag, kKernBwd, 8, 0)))
+        break;
+      tc_fence_after();
+      uint32_t v0[32], v1[32];
+      tmem_ld32(tm_dP(buf) + lane_off, v0);
+      tmem_ld32(tm_dP(buf) + lane_off + 32, v1);
+      tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(&dq_drained[buf]);
+      const int bh = step_bh(t), qt = step_qt(t);
+      // two halves of 32 query rows; this warp's box is 32 rows x 32 fp32,
+      // 128-byte swizzled, reduce-added into the accumulator by TMA
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        uint8_t* box = sDQ + hh * L::kDqHalf + dw * 4096;
+        if (lane == 0 && groups >= 1) bulk_wait_group_read1();  // box hh free again
+        __syncwarp();
+        const uint32_t* vv = hh ? v1 : v0;
+        uint8_t* col_base = box + (lane & 3) * 4;
+#pragma unroll
+        for (int q = 0; q < 32; ++q) {
+          const int chunk = (lane >> 2) ^ (q & 7);
+          *reinterpret_cast<uint32_t*>(col_base + q * 128 + chunk * 16) = vv[q];
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && !*abort_flag) {
+          tma_reduce_add_3d(&p.tm_dqacc, box, dw * 32, qt * 64 + hh * 32, bh);
+          bulk_commit_group();
+          ++groups;
+        }
+      }
+    }
+    if (lane == 0) bulk_wait_group0();
+    // epilogue: dV, dK (times scale) rows -> I/O dtype, written once
+    if (__all_sync(0xffffffffu, mbar_wait(acc_done, 0, abort_flag, kKernBwd, 8, 1))) {
+      tc_fence_after();
+      const int r = dw * 32 + lane;
+      const int kv_row = kv0 + r;
+      const size_t row_off = (static_cast<size_t>(kvh) * p.N + kv_row) * HD;
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+        const uint32_t src = (which ? tm_dK : tm_dV) + lane_off;
+        const float mul = which ? p.scale : 1.0f;
+        T* dst = reinterpret_cast<T*>(which ? p.dk : p.dv) + row_off;
+#pragma unroll
+        for (int c = 0; c < HD; c += 32) {
+          uint32_t v[32];
+          tmem_ld32(src + c, v);
+          tmem_ld_wait();
+          if (kv_row < p.N) {
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              uint4 w;
+              w.x = pack2<BF16>(__uint_as_float(v[8 * u + 0]) * mul, __uint_as_float(v[8 * u + 1]) * mul);
+              w.y = pack2<BF16>(__uint_as_float(v[8 * u + 2]) * mul, __uint_as_float(v[8 * u + 3]) * mul);
+              w.z = pack2<BF16>(__uint_as_float(v[8 * u + 4]) * mul, __uint_as_float(v[8 * u + 5]) * mul);
+              w.w = pack2<BF16>(__uint_as_float(v[8 * u + 6]) * mul, __uint_as_float(v[8 * u + 7]) * mul);
+              *reinterpret_cast<uint4*>(dst + c + 8 * u) = w;
+            }
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 13) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// bwd_post: dQ = scale * accumulator -> I/O dtype (8 elements per thread)
+
+template <int HD, bool BF16>
+__global__ void __launch_bounds__(256) fa_bwd_post_kernel(const float* __restrict__ dqacc,
+                                                          void* __restrict__ dq_, int N, int Np,
+                                                          int64_t total_vec, float scale) {
+  using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
+  constexpr int kVecPerRow = HD / 8;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total_vec;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t row = i / kVecPerRow;  // row of the [B*Hq][N] output
+    const int cv = static_cast<int>(i % kVecPerRow);
+    const int64_t bh = row / N;
+    const int64_t n = row % N;
+    const float4* src = reinterpret_cast<const float4*>(dqacc + (bh * Np + n) * HD + cv * 8);
+    const float4 a = src[0], c = src[1];
+    uint4 w;
+    w.x = pack2<BF16>(a.x * scale, a.y * scale);
+    w.y = pack2<BF16>(a.z * scale, a.w * scale);
+    w.z = pack2<BF16>(c.x * scale, c.y * scale);
+    w.w = pack2<BF16>(c.z * scale, c.w * scale);
+    reinterpret_cast<uint4*>(reinterpret_cast<T*>(dq_) + row * HD)[cv] = w;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// failure-path self test: one barrier that nobody signals
+
+__global__ void wait_timeout_selftest_kernel() {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, kKernSelftest, 0, 0);
+  __syncthreads();
+}
+
+}  // namespace fa

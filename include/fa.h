@@ -1,0 +1,144 @@
+/*
+ * fa.h - C ABI of the B200 (sm_100a) exact-attention library libfa_b200.so.
+ *
+ * The library computes exact softmax attention and its gradient, tiled so
+ * that the N x N score matrix never reaches device memory:
+ *
+ *   forward   O = softmax(scale * Q K^T + causal mask) V, plus one logsumexp
+ *             per query row.  The pages define attention as S = QK^T,
+ *             P = softmax(S), O = PV ("flash attention io aware", section
+ *             "The Memory Bandwidth Bottleneck") and the method as tiles of
+ *             Q, K, V streamed through on-chip memory with a running max and
+ *             sum, writing only O back ("FlashAttention" glossary, opening
+ *             list and online-softmax paragraph; same page, section
+ *             "Flash Attention Algorithm", step 4).
+ *   backward  dQ, dK, dV from Q, K, V, O, dO and the logsumexp alone: the
+ *             scores are recomputed on chip instead of being stored
+ *             ("FlashAttention" glossary, recomputation paragraph).  dK and
+ *             dV are owned by one thread block per key block and written
+ *             once, with no atomics ("FlashAttention" glossary,
+ *             FlashAttention-2 list, backward-pass item).
+ *
+ * Conventions shared by every entry point
+ *   - Tensors are dense, row-major, in device memory owned by the caller:
+ *       q, o, dout, dq : [B][Hq][N][d]
+ *       k, v, dk, dv   : [B][Hkv][N][d]
+ *       lse            : [B][Hq][N] fp32, natural log:
+ *                        lse_i = ln sum_j exp(scale * q_i . k_j) over unmasked j
+ *   - Grouped-query attention: Hq % Hkv == 0 and query head h reads key/value
+ *     head h / (Hq / Hkv) ("Flash Attention" glossary of inferensys,
+ *     grouped-query attention paragraph; Hkv == Hq is plain multi-head,
+ *     Hkv == 1 multi-query).  dK and dV sum over each group.
+ *   - causal != 0 masks key j for query i when j > i.
+ *   - q, k, v, dout share one dtype (bf16 or fp16); o, dq, dk, dv are written
+ *     in it.  Arithmetic: tensor-core products of the I/O dtype with fp32
+ *     accumulation; softmax statistics in fp32.
+ *   - d must be 64 or 128; N may be any size >= 0 (a ragged last tile is
+ *     masked); B == 0 or N == 0 is an empty problem and returns FA_OK at once.
+ *   - scale must be finite and > 0 (usually 1/sqrt(d)).
+ *   - Every tensor pointer must be 16-byte aligned (TMA requirement).
+ *   - stream is a cudaStream_t (NULL: the legacy default stream).  All work is
+ *     enqueued asynchronously on it; the call returns without waiting.
+ *   - Argument errors are returned before anything is launched.  Errors
+ *     inside a kernel (a barrier wait that ran out, see fa_get_device_status)
+ *     are recorded on the device; no call aborts the process and there is no
+ *     CPU fallback.
+ *   - The library never allocates device memory.  Its only state is one
+ *     status word per device and a cache of kernel attributes.
+ */
+#ifndef FA_B200_H
+#define FA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FA_OK = 0,
+    FA_ERR_INVALID_ARG = 1,  /* null pointer, negative size, Hq % Hkv != 0, bad scale, small workspace */
+    FA_ERR_UNSUPPORTED = 2,  /* d not in {64, 128}, dtype not bf16/fp16, no sm_100 device */
+    FA_ERR_MISALIGNED = 3,   /* a tensor pointer is not 16-byte aligned */
+    FA_ERR_CUDA = 4,         /* a CUDA runtime or driver call failed */
+    FA_ERR_TIMEOUT = 5       /* a kernel's bounded barrier wait ran out (device-side) */
+} fa_status_t;
+
+typedef enum { FA_BF16 = 0, FA_FP16 = 1 } fa_dtype_t;
+
+/*
+ * Forward pass.  Writes o [B][Hq][N][d] and lse [B][Hq][N].
+ * Reads q, k, v only; o and lse may not alias the inputs.
+ */
+fa_status_t fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                   int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+                   fa_dtype_t dtype, void* stream);
+
+/*
+ * Bytes of device scratch that fa_bwd needs for these sizes (0 for an empty
+ * problem).  Linear in N: two fp32 values per query row (D_i = dO_i . O_i and
+ * the logsumexp in base 2) plus an fp32 dQ accumulator [B][Hq][Np][d], with N
+ * rounded up to a multiple of 128 (Np).
+ */
+size_t fa_bwd_workspace_bytes(int B, int Hq, int Hkv, int N, int d);
+
+/*
+ * Backward pass: given dout = dL/dO, writes dq, dk, dv.  o and lse must be
+ * the forward outputs for the same q, k, v, scale and causal flag.  The
+ * scores and probabilities are recomputed from q, k and lse.  workspace is
+ * caller-owned device memory of at least fa_bwd_workspace_bytes(...) bytes,
+ * 16-byte aligned; its contents on entry do not matter and on exit are
+ * unspecified.  Three kernels run on `stream` in order: a row pass (D and the
+ * zeroed dQ accumulator), the main pass (one thread block per key block of
+ * 128 rows and key/value head: dK, dV in tensor memory, dQ added into the
+ * accumulator), and a pass that scales and converts dQ.
+ */
+fa_status_t fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                   const float* lse, void* dq, void* dk, void* dv,
+                   int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+                   fa_dtype_t dtype, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Synchronises `stream`, then returns and clears the first device-side error
+ * any kernel of this library recorded on the current device since the last
+ * call: FA_OK, or FA_ERR_TIMEOUT when a bounded barrier wait ran out (the
+ * kernel then skipped its remaining work and its outputs are undefined).
+ * Returns FA_ERR_CUDA when the stream itself reports an error.
+ */
+fa_status_t fa_get_device_status(void* stream);
+
+/*
+ * Raw form of the last recorded device status word (0 = none), for
+ * diagnostics: bits 0-7 status, 8-15 kernel id, 16-23 warp role, 24-31 wait
+ * site.  Does not clear it.  Synchronises `stream`.
+ */
+uint32_t fa_peek_device_status_word(void* stream);
+
+/*
+ * Self-test of the failure path: launches one thread block that waits on a
+ * barrier nobody signals, with the wait limit set to limit_ns nanoseconds,
+ * then restores the default limit (2 s) and returns what
+ * fa_get_device_status reports (FA_ERR_TIMEOUT when the bounded wait works).
+ * No fault, trap or hang is involved.
+ */
+fa_status_t fa_selftest_wait_timeout(uint64_t limit_ns, void* stream);
+
+/*
+ * Profiling hook: while set, every launch of kernel `kernel_id` (1: the
+ * forward kernel of fa_fwd, 3: the main kernel of fa_bwd) is bracketed by
+ * cudaEventRecord(start) / cudaEventRecord(stop) on the stream it is launched
+ * on.  start and stop are cudaEvent_t handles created by the caller; pass
+ * NULL for both to clear.  Process-wide, not synchronised with concurrent
+ * calls: set it only from the thread that launches.
+ */
+fa_status_t fa_set_profile_events(int kernel_id, void* start, void* stop);
+
+/* Static English description of a status code. */
+const char* fa_status_string(fa_status_t status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_B200_H */

@@ -1,0 +1,155 @@
+"""Helpers of the GPU parity tests: run the CUDA path through the C ABI and
+compare it with the fp64 oracle on the same (rounded) inputs.
+
+Tolerances are those stated for this path: max |dO| <= 1e-2, max |dlse| <= 1e-3,
+relative Frobenius error <= 2e-2 on dQ, dK, dV.  An output element of O whose
+error is above 1e-2 passes only if the error is explained by the rounding of
+O to the I/O dtype (at most half an ulp of the output plus 5e-3); such
+elements are counted and reported, never silently absorbed."""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import torch
+
+import oracle
+from exact_io_aware_bwd_b200 import binding
+
+TOL_O = 1e-2
+TOL_LSE = 1e-3
+TOL_GRAD = 2e-2
+
+
+def run_gpu(q, k, v, do, scale, causal):
+    """Forward + backward on cuda:0 through the C ABI; returns CPU tensors."""
+    dev = "cuda:0"
+    qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, do))
+    o, lse = binding.attention_fwd(qd, kd, vd, scale, causal)
+    dq, dk, dv = binding.attention_bwd(qd, kd, vd, o, dod, lse, scale, causal)
+    status = binding.fa_get_device_status()
+    assert status == binding.FA_OK, binding.fa_status_string(status)
+    return {n: t.cpu() for n, t in dict(o=o, lse=lse, dq=dq, dk=dk, dv=dv).items()}
+
+
+def _np(t):
+    return t.double().numpy() if hasattr(t, "double") else np.asarray(t, dtype=np.float64)
+
+
+def check_o(o_gpu, o_ref, dtype, o_absv=None, what="O"):
+    """max |O_gpu - O_ref| <= 1e-2.  An element above it passes only if the
+    rounding of the tensor-core operands and of the output explains it:
+    |err| <= u * sum_j p_ij |v_jc| + half an ulp of O + 1e-3, where u is the
+    unit roundoff of the I/O dtype (P is rounded to it before the P V
+    product) and ``o_absv`` is the oracle's output with |V| in place of V,
+    i.e. sum_j p_ij |v_jc|.  Such elements are counted in the report."""
+    g, r = _np(o_gpu), _np(o_ref)
+    err = np.abs(g - r)
+    mant = 8 if dtype == torch.bfloat16 else 11
+    u = 2.0 ** -mant
+    ar = np.maximum(np.abs(r), 1e-30)
+    half_ulp = 0.5 * np.exp2(np.floor(np.log2(ar)) - (mant - 1))
+    over = err > TOL_O
+    bound = half_ulp + 1e-3 + (u * _np(o_absv) if o_absv is not None else 0.0)
+    explained = err <= bound
+    bad = over & ~explained
+    info = dict(max_err=float(err.max(initial=0.0)),
+                n_over_tol_explained_by_rounding=int((over & explained).sum()))
+    assert not bad.any(), f"{what}: {int(bad.sum())} elements beyond tolerance, {info}"
+    return info
+
+
+def check_lse(lse_gpu, lse_ref, what="lse"):
+    err = float(np.abs(_np(lse_gpu) - _np(lse_ref)).max(initial=0.0))
+    assert err <= TOL_LSE, f"{what}: max abs err {err:.3e} > {TOL_LSE}"
+    return err
+
+
+def rel_frob(g, r):
+    g, r = _np(g), _np(r)
+    den = np.linalg.norm(r)
+    return float(np.linalg.norm(g - r) / den) if den > 0 else float(np.linalg.norm(g))
+
+
+def check_grad(g, r, what):
+    e = rel_frob(g, r)
+    assert e <= TOL_GRAD, f"{what}: relative Frobenius error {e:.3e} > {TOL_GRAD}"
+    return e
+
+
+def check_full(q, k, v, do, scale, causal, out):
+    """Every output element against the full oracle."""
+    o_r, lse_r = oracle.fwd(q, k, v, scale, causal)
+    o_abs, _ = oracle.fwd(q, k, v.abs(), scale, causal)
+    dq_r, dk_r, dv_r = oracle.bwd(q, k, v, do, scale, causal)
+    rep = dict(o=check_o(out["o"], o_r, q.dtype, o_abs), lse=check_lse(out["lse"], lse_r))
+    rep.update(dq=check_grad(out["dq"], dq_r, "dQ"), dk=check_grad(out["dk"], dk_r, "dK"),
+               dv=check_grad(out["dv"], dv_r, "dV"))
+    return rep
+
+
+def check_rows(q, k, v, do, scale, causal, out, rows):
+    """O, lse, dQ of the given query rows of every head, one kv group at a time."""
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    G = Hq // Hkv
+    rows = np.asarray(rows, dtype=np.int64)
+    o_g, lse_g, dq_g, o_r, lse_r, dq_r, o_a = [], [], [], [], [], [], []
+    for b in range(B):
+        for g in range(Hkv):
+            hs = slice(g * G, (g + 1) * G)
+            qq, kk, vv, dd = q[b:b + 1, hs], k[b:b + 1, g:g + 1], v[b:b + 1, g:g + 1], do[b:b + 1, hs]
+            o1, l1 = oracle.fwd_rows(qq, kk, vv, rows, scale, causal)
+            oa, _ = oracle.fwd_rows(qq, kk, vv.abs(), rows, scale, causal)
+            dq1 = oracle.bwd_rows(qq, kk, vv, dd, rows, scale, causal)
+            o_r.append(o1); lse_r.append(l1); dq_r.append(dq1); o_a.append(oa)
+            o_g.append(_np(out["o"][b:b + 1, hs][:, :, rows]))
+            lse_g.append(_np(out["lse"][b:b + 1, hs][:, :, rows]))
+            dq_g.append(_np(out["dq"][b:b + 1, hs][:, :, rows]))
+    cat = lambda xs: np.concatenate([x.reshape(-1) for x in xs])
+    rep = dict(o=check_o(cat(o_g), cat(o_r), q.dtype, cat(o_a)), lse=check_lse(cat(lse_g), cat(lse_r)),
+               dq=check_grad(cat(dq_g), cat(dq_r), "dQ rows"))
+    return rep
+
+
+def check_cols(q, k, v, do, scale, causal, out, col_sets):
+    """dK, dV of selected key rows of selected kv heads."""
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    G = Hq // Hkv
+    dk_g, dv_g, dk_r, dv_r = [], [], [], []
+    for (b, g, cols) in col_sets:
+        cols = np.asarray(cols, dtype=np.int64)
+        hs = slice(g * G, (g + 1) * G)
+        dk1, dv1 = oracle.bwd_cols(q[b:b + 1, hs], k[b:b + 1, g:g + 1], v[b:b + 1, g:g + 1],
+                                   do[b:b + 1, hs], 0, 0, cols, scale, causal)
+        dk_r.append(dk1); dv_r.append(dv1)
+        dk_g.append(_np(out["dk"][b, g][cols])); dv_g.append(_np(out["dv"][b, g][cols]))
+    cat = lambda xs: np.concatenate([x.reshape(-1) for x in xs])
+    return dict(dk=check_grad(cat(dk_g), cat(dk_r), "dK cols"),
+                dv=check_grad(cat(dv_g), cat(dv_r), "dV cols"))
+
+
+def check_invariants(q, k, do, out, tol=1e-2):
+    """Properties that hold at any size: (i) sum_j dK_j = 0 per kv head;
+    (ii) sum_j dV_j = sum over the group of sum_i dO_i; (iii) <Q,dQ> = <K,dK>
+    per kv group.  Each is checked relative to the summed magnitudes."""
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    G = Hq // Hkv
+    dev = "cuda:0"
+    f = lambda t: t.to(dev).double()
+    dk, dv, dq = f(out["dk"]), f(out["dv"]), f(out["dq"])
+    qd, kd, dod = f(q), f(k), f(do)
+    r1 = (dk.sum(2).abs() / dk.abs().sum(2).clamp_min(1e-30)).max().item()
+    grp = dod.reshape(B, Hkv, G, N, d).sum((2, 3))
+    r2 = ((dv.sum(2) - grp).abs() / dod.abs().reshape(B, Hkv, G, N, d).sum((2, 3)).clamp_min(1e-30)).max().item()
+    qdq = (qd * dq).reshape(B, Hkv, G, N, d).sum((2, 3, 4))
+    kdk = (kd * dk).sum((2, 3))
+    mag = (qd * dq).abs().reshape(B, Hkv, G, N, d).sum((2, 3, 4)) + (kd * dk).abs().sum((2, 3))
+    r3 = ((qdq - kdk).abs() / mag.clamp_min(1e-30)).max().item()
+    assert r1 <= tol, f"sum_j dK_j relative {r1:.3e}"
+    assert r2 <= tol, f"sum_j dV_j relative {r2:.3e}"
+    assert r3 <= tol, f"<Q,dQ> vs <K,dK> relative {r3:.3e}"
+    return dict(sum_dk=r1, sum_dv=r2, qdq_kdk=r3)

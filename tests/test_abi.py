@@ -1,0 +1,113 @@
+"""The C ABI of libfa_b200.so without a GPU: every symbol include/fa.h
+declares is exported, and argument errors come back as status codes before
+anything touches a device."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from exact_io_aware_bwd_b200 import binding
+from exact_io_aware_bwd_b200.build import INCLUDE, build
+
+HEADER = os.path.join(INCLUDE, "fa.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build()
+    return binding.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z_0-9]*\s*\**\s+\**\s*(fa_[a-z_0-9]+)\s*\(",
+                       text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ("fa_fwd", "fa_bwd", "fa_bwd_workspace_bytes", "fa_get_device_status",
+              "fa_status_string"):
+        assert n in names, names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), f"{name} declared in fa.h but not exported"
+
+
+def test_status_strings(lib):
+    for s in range(6):
+        assert binding.fa_status_string(s)
+    assert "unknown" in binding.fa_status_string(99)
+
+
+FAKE = 1 << 20  # a 16-byte-aligned non-null pointer value; never dereferenced
+
+
+def fwd_raw(lib, B=1, Hq=2, Hkv=2, N=128, d=64, scale=0.125, causal=0, dtype=0, ptrs=None):
+    p = ptrs or [FAKE] * 5
+    return lib.fa_fwd(*[ctypes.c_void_p(x) for x in p], B, Hq, Hkv, N, d, scale, causal, dtype, None)
+
+
+def bwd_raw(lib, B=1, Hq=2, Hkv=2, N=128, d=64, scale=0.125, causal=0, dtype=0, ptrs=None,
+            ws_bytes=None):
+    p = ptrs or [FAKE] * 10
+    ws = binding.fa_bwd_workspace_bytes(B, Hq, Hkv, N, d) if ws_bytes is None else ws_bytes
+    vp = [ctypes.c_void_p(x) for x in p]
+    return lib.fa_bwd(*vp[:9], B, Hq, Hkv, N, d, scale, causal, dtype, vp[9], ws, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(Hq=3, Hkv=2), binding.FA_ERR_INVALID_ARG),
+    (dict(Hq=0), binding.FA_ERR_INVALID_ARG),
+    (dict(Hkv=0), binding.FA_ERR_INVALID_ARG),
+    (dict(B=-1), binding.FA_ERR_INVALID_ARG),
+    (dict(N=-5), binding.FA_ERR_INVALID_ARG),
+    (dict(scale=0.0), binding.FA_ERR_INVALID_ARG),
+    (dict(scale=-1.0), binding.FA_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), binding.FA_ERR_INVALID_ARG),
+    (dict(scale=float("inf")), binding.FA_ERR_INVALID_ARG),
+    (dict(causal=2), binding.FA_ERR_INVALID_ARG),
+    (dict(d=96), binding.FA_ERR_UNSUPPORTED),
+    (dict(d=256), binding.FA_ERR_UNSUPPORTED),
+    (dict(dtype=7), binding.FA_ERR_UNSUPPORTED),
+    (dict(ptrs=[FAKE, 0, FAKE, FAKE, FAKE]), binding.FA_ERR_INVALID_ARG),
+    (dict(ptrs=[FAKE, FAKE + 8, FAKE, FAKE, FAKE]), binding.FA_ERR_MISALIGNED),
+])
+def test_fwd_argument_errors(lib, kw, status):
+    assert fwd_raw(lib, **kw) == status
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(Hq=4, Hkv=3), binding.FA_ERR_INVALID_ARG),
+    (dict(d=32), binding.FA_ERR_UNSUPPORTED),
+    (dict(ws_bytes=100), binding.FA_ERR_INVALID_ARG),
+    (dict(ptrs=[FAKE] * 9 + [0]), binding.FA_ERR_INVALID_ARG),
+    (dict(ptrs=[FAKE] * 6 + [FAKE + 4] + [FAKE] * 3), binding.FA_ERR_MISALIGNED),
+])
+def test_bwd_argument_errors(lib, kw, status):
+    assert bwd_raw(lib, **kw) == status
+
+
+def test_empty_problems_are_no_ops(lib):
+    # B == 0 or N == 0: nothing to compute, nothing launched, even with null pointers
+    assert fwd_raw(lib, B=0, ptrs=[0] * 5) == binding.FA_OK
+    assert fwd_raw(lib, N=0, ptrs=[0] * 5) == binding.FA_OK
+    assert bwd_raw(lib, N=0, ptrs=[0] * 10, ws_bytes=0) == binding.FA_OK
+    assert binding.fa_bwd_workspace_bytes(1, 2, 2, 0, 64) == 0
+
+
+def test_workspace_is_linear_in_n():
+    # two fp32 row statistics + an fp32 dQ accumulator per (padded) query row
+    for d in (64, 128):
+        sizes = [binding.fa_bwd_workspace_bytes(1, 16, 16, n, d) for n in (4096, 8192, 16384, 32768, 65536)]
+        for a, b in zip(sizes, sizes[1:]):
+            assert b == 2 * a
+        assert sizes[0] == 16 * 4096 * 4 * (2 + d)
+    # padding to a multiple of 128 rows
+    assert binding.fa_bwd_workspace_bytes(1, 1, 1, 129, 64) == 256 * 4 * 66
