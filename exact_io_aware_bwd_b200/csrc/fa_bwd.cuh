@@ -185,11 +185,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
   const int warp = tid >> 5;
   const int lane = tid & 31;
 
-  // Work item: key blocks nearest the start first (under a causal mask they
-  // see the most query blocks).
+  // Work item, head-major: the blocks running at the same time mostly share
+  // a kv head, so its Q, dO and dQ accumulator stay in L2; inside a head the
+  // key blocks nearest the start go first (under a causal mask they see the
+  // most query blocks).
   const int item = blockIdx.x;
-  const int jt = item / p.BHkv;     // key block (128 rows)
-  const int kvh = item % p.BHkv;    // b * Hkv + g
+  const int kvh = item / p.n_ktiles;  // b * Hkv + g
+  const int jt = item % p.n_ktiles;   // key block (128 rows)
   const int b = kvh / p.Hkv;
   const int g = kvh % p.Hkv;
   const int kv0 = jt * 128;

@@ -91,10 +91,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
   const int warp = tid >> 5;
   const int lane = tid & 31;
 
-  // Work item: largest query blocks first (the causal ones do the most work).
+  // Work item, head-major: the blocks running at the same time mostly share
+  // a head, so its K and V stay in L2; inside a head the largest query
+  // blocks (the most key blocks under a causal mask) go first.
   const int item = blockIdx.x;
-  const int qt = p.n_qtiles - 1 - item / p.BH;
-  const int bh = item % p.BH;
+  const int bh = item / p.n_qtiles;
+  const int qt = p.n_qtiles - 1 - item % p.n_qtiles;
   const int h = bh % p.Hq;
   const int b = bh / p.Hq;
   const int kvh = b * p.Hkv + h / p.group;
