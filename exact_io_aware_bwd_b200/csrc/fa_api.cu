@@ -119,7 +119,7 @@ fa_status_t launch_fwd(const FwdParams& prm, cudaStream_t st) {
   const int smem = FwdLayout<HD>::kDynSmem;
   fa_status_t s = opt_in_smem(kern, smem);
   if (s != FA_OK) return s;
-  const int grid = prm.n_qtiles * prm.BH;
+  const int grid = prm.n_pairs * prm.BH;
   prof_begin(fa::kKernFwd, st);
   kern<<<grid, fa::kFwdThreads, smem, st>>>(prm);
   const bool ok = cudaGetLastError() == cudaSuccess;
@@ -168,11 +168,11 @@ fa_status_t bwd_run(const void* q, const void* k, const void* v, const void* o, 
   if (!make_map(&prm.tm_q, q, dt, 2, HD, N, BHq, 64, 64) ||
       !make_map(&prm.tm_do, dout, dt, 2, HD, N, BHq, 64, 64) ||
       !make_map(&prm.tm_k, k, dt, 2, HD, N, BHkv, 64, 128) ||
-      !make_map(&prm.tm_v, v, dt, 2, HD, N, BHkv, 64, 128) ||
-      !make_map(&prm.tm_dqacc, dqacc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, HD, Np, BHq, 32, 32))
+      !make_map(&prm.tm_v, v, dt, 2, HD, N, BHkv, 64, 128))
     return FA_ERR_CUDA;
   prm.lse2 = lse2;
   prm.Dvec = Dvec;
+  prm.dqacc = dqacc;
   prm.dk = dk;
   prm.dv = dv;
   prm.N = N;
@@ -230,7 +230,7 @@ fa_status_t fa_fwd(const void* q, const void* k, const void* v, void* o, float* 
   prm.Hkv = Hkv;
   prm.group = Hq / Hkv;
   prm.BH = static_cast<int>(BHq);
-  prm.n_qtiles = (N + 127) / 128;
+  prm.n_pairs = (N + 255) / 256;
   prm.n_ktiles = (N + 127) / 128;
   prm.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);

@@ -110,9 +110,9 @@ struct BwdParams {
   CUtensorMap tm_do;     // [B*Hq][N][d], box 64 x 64
   CUtensorMap tm_k;      // [B*Hkv][N][d], box 64 x 128
   CUtensorMap tm_v;      // [B*Hkv][N][d], box 64 x 128
-  CUtensorMap tm_dqacc;  // fp32 [B*Hq][Np][d], box 32 cols x 32 rows (reduce-add)
   const float* lse2;     // [B*Hq][Np]
   const float* Dvec;     // [B*Hq][Np]
+  float* dqacc;          // [B*Hq][Np][d] fp32 accumulator
   void* dk;              // [B*Hkv][N][d]
   void* dv;
   int N, Np, Hq, Hkv, group, n_ktiles, n_qtiles, BHkv;
@@ -121,21 +121,19 @@ struct BwdParams {
 
 template <int HD>
 struct BwdLayout {
-  static constexpr int kStages = 3;                     // Q / dO / lse2 / D ring
+  static constexpr int kStages = 4;                     // Q / dO / lse2 / D ring
   static constexpr int kChunks = HD / 64;
   static constexpr int kKVBox = 128 * 128;              // 128 rows x 64 cols x 2 B
   static constexpr int kQBox = 64 * 128;                // 64 rows x 64 cols x 2 B
   static constexpr int kKVTile = kChunks * kKVBox;
   static constexpr int kQTile = kChunks * kQBox;
   static constexpr int kDsBytes = 128 * 128;            // dS^T: 128 key rows x 64 query cols x 2 B
-  static constexpr int kDqHalf = 32 * HD * 4;           // 32 query rows x d fp32
   static constexpr int kOffK = 0;
   static constexpr int kOffV = kOffK + kKVTile;
   static constexpr int kOffQ = kOffV + kKVTile;
   static constexpr int kOffDO = kOffQ + kStages * kQTile;
   static constexpr int kOffDS = kOffDO + kStages * kQTile;
-  static constexpr int kOffDQ = kOffDS + 2 * kDsBytes;
-  static constexpr int kOffLse = kOffDQ + 2 * kDqHalf;
+  static constexpr int kOffLse = kOffDS + 2 * kDsBytes;
   static constexpr int kOffD = kOffLse + kStages * 256;
   static constexpr int kOffBar = kOffD + kStages * 256;
   // kv_full, q_full[S], q_empty[S], s_full[2], dp_full[2], ds_full[2], pt_free[2],
@@ -144,7 +142,11 @@ struct BwdLayout {
   static constexpr int kOffTmemPtr = kOffBar + kNumBars * 8;
   static constexpr int kOffAbort = kOffTmemPtr + 4;
   static constexpr int kSmemBytes = kOffAbort + 4;
-  static constexpr int kDynSmem = kSmemBytes + 1024;
+  // Tiles must sit on 1024-byte boundaries (128-byte swizzle atoms).  The
+  // dynamic shared memory of a block without static shared memory starts on
+  // such a boundary on sm_100; the d = 64 layout keeps spare bytes for
+  // re-alignment anyway, the d = 128 layout has none to spare and checks.
+  static constexpr int kDynSmem = kSmemBytes + (232448 - kSmemBytes >= 1024 ? 1024 : 0);
   static_assert(kDynSmem <= 232448, "shared memory budget");
 };
 
@@ -162,7 +164,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
   uint8_t* sQ = sm + L::kOffQ;
   uint8_t* sDO = sm + L::kOffDO;
   uint8_t* sDS = sm + L::kOffDS;
-  uint8_t* sDQ = sm + L::kOffDQ;
   float* sLse = reinterpret_cast<float*>(sm + L::kOffLse);
   float* sD = reinterpret_cast<float*>(sm + L::kOffD);
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::kOffBar);
@@ -184,6 +185,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
+  if (sm + L::kSmemBytes > smem_raw + L::kDynSmem) {  // no room to re-align: refuse
+    if (tid == 0) record_error(kStatusSmemAlign, kKernBwd, 0, 0);
+    return;
+  }
 
   // Work item, head-major: the blocks running at the same time mostly share
   // a kv head, so its Q, dO and dQ accumulator stay in L2; inside a head the
@@ -421,13 +426,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
     }
   } else {
     // ------------------------------------------------------------ dQ drain, dK/dV epilogue
-    // Each drain warp owns 32 features of dQ^T (one 128-byte column box of
-    // the staging tile) and issues its own TMA reduce-adds, so the drain
-    // needs no barrier across warps.
+    // Lane f of drain warp w holds feature f = 32w + lane of dQ^T: 64 query
+    // values.  They are added into the fp32 accumulator straight from
+    // registers; for a fixed query the 32 lanes of a warp touch 128
+    // consecutive bytes, so every reduction is one coalesced request.
     const int dw = warp - 8;                           // 0..3 == lane quarter
     const uint32_t lane_off = static_cast<uint32_t>(dw * 32) << 16;
     const bool drains = dw * 32 < HD;                  // warp holds real dQ^T rows
-    int groups = 0;                                    // bulk groups committed by lane 0
     for (int t = 0; drains && t < T_steps; ++t) {
       const int buf = t & 1;
       if (!__all_sync(0xffffffffu, mbar_wait(&dq_full[buf], (t >> 1) & 1, abort_flag, kKernBwd, 8, 0)))
@@ -440,30 +445,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
       tc_fence_before();
       mbar_arrive(&dq_drained[buf]);
       const int bh = step_bh(t), qt = step_qt(t);
-      // two halves of 32 query rows; this warp's box is 32 rows x 32 fp32,
-      // 128-byte swizzled, reduce-added into the accumulator by TMA
+      float* dst = p.dqacc + (static_cast<size_t>(bh) * p.Np + qt * 64) * HD + dw * 32 + lane;
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        uint8_t* box = sDQ + hh * L::kDqHalf + dw * 4096;
-        if (lane == 0 && groups >= 1) bulk_wait_group_read1();  // box hh free again
-        __syncwarp();
-        const uint32_t* vv = hh ? v1 : v0;
-        uint8_t* col_base = box + (lane & 3) * 4;
+      for (int q = 0; q < 32; ++q) atomicAdd(dst + q * HD, __uint_as_float(v0[q]));
 #pragma unroll
-        for (int q = 0; q < 32; ++q) {
-          const int chunk = (lane >> 2) ^ (q & 7);
-          *reinterpret_cast<uint32_t*>(col_base + q * 128 + chunk * 16) = vv[q];
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0 && !*abort_flag) {
-          tma_reduce_add_3d(&p.tm_dqacc, box, dw * 32, qt * 64 + hh * 32, bh);
-          bulk_commit_group();
-          ++groups;
-        }
-      }
+      for (int q = 0; q < 32; ++q) atomicAdd(dst + (32 + q) * HD, __uint_as_float(v1[q]));
     }
-    if (lane == 0) bulk_wait_group0();
     // epilogue: dV, dK (times scale) rows -> I/O dtype, written once
     if (__all_sync(0xffffffffu, mbar_wait(acc_done, 0, abort_flag, kKernBwd, 8, 1))) {
       tc_fence_after();

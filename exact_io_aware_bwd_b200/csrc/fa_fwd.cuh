@@ -1,10 +1,10 @@
 // Forward pass of exact attention on sm_100a: one thread block per
-// (batch, query head, 128-row query block).
+// (batch, query head, pair of 128-row query blocks).
 //
 // Method (pages: "FlashAttention" glossary, opening list and online-softmax
 // paragraph; "flash attention io aware", sections "Flash Attention
-// Algorithm" and "Online Softmax"): the query block stays on chip while the
-// key/value blocks of its head stream through a shared-memory ring; each
+// Algorithm" and "Online Softmax"): the query blocks stay on chip while the
+// key/value blocks of their head stream through a shared-memory ring; each
 // score block S_j = Q K_j^T lives only in tensor memory; a running row max m
 // and row sum l are kept and the partial output is rescaled when the max
 // grows; only O and one logsumexp per row are written back.  Queries are the
@@ -12,26 +12,29 @@
 // glossary of inferensys ("for each query block, iterate over key-value
 // blocks"); the other order on the chipfoundry page reaches the same result.
 //
-// Warp roles (192 threads):
-//   warps 0-3  softmax: thread r owns query row r of the block and tensor
-//              memory lane r.  Reads S_j, applies mask and scale, updates
-//              (m, l), writes P_j (16-bit) back over S_j, rescales O when
-//              needed, and finally normalises O, stores it (via TMA) and lse.
-//   warp 4     TMA producer: Q once, then K_0, K_1, V_0, K_2, V_1, ... in the
-//              order the MMA warp consumes them, through an NSLOT ring.
-//   warp 5     MMA issuer (one thread): S_{j+1} = Q K_{j+1}^T into the other
-//              score buffer while the softmax warps work on S_j, then
-//              O += P_j V_j with P_j read from tensor memory.
+// Two query blocks per thread block, each with its own softmax warpgroup, so
+// that the tensor cores work on one block while the softmax warps work on the
+// other (the B200 form of the "two sets of registers" alternation the
+// FlashAttention glossary names for Hopper).  Warp roles (320 threads):
+//   warps 0-3 / 4-7  softmax of query block 0 / 1: thread r owns row r of its
+//              block and tensor-memory lane r.  Reads S_j, masks, scales,
+//              updates (m, l), writes P_j (16-bit) over S_j, rescales O when
+//              needed, and at the end normalises O, stores it (TMA) and lse.
+//   warp 8     MMA issuer (one thread): S_t,j = Q_t K_j^T and O_t += P_t,j V_j
+//              for t = 0, 1, staggered as S0_j+1, O1 += P1_j V_j, S1_j+1,
+//              O0 += P0_j+1 V_j+1, ... so that one block's softmax overlaps the
+//              other block's products.  S_t,j+1 overwrites P_t,j, so it is
+//              issued only once O_t += P_t,j V_j has completed.
+//   warp 9     TMA producer: Q0, Q1 once, then K_0, V_0, K_1, V_1, ... through
+//              a ring of kSlots tiles.
+// Tensor memory (512 columns x 128 lanes x 32 bit): S0 [0,128), S1 [128,256),
+// O0 [256, 256+d), O1 [384, 384+d); P_t packs into the first 64 columns of S_t.
 //
-// Tensor memory (512 columns x 128 lanes x 32 bit): score buffers at columns
-// [0,128) and [128,256) (P_j aliases the first 64 columns of its buffer as
-// packed 16-bit pairs), O at [256, 256 + d).
-//
-// Running max: the max used for the exponentials (m_ref) is only moved when
-// a row's max exceeds it by more than 8 (in log2 units), so that O and l are
-// rescaled rarely; P = 2^(s - m_ref) <= 2^8 stays well inside bf16/fp16 range.
-// O and l always share the same m_ref, so O / l is exact (the reference point
-// of a softmax is arbitrary).
+// Running max: the max used for the exponentials (m_ref) moves only when a
+// row's max exceeds it by more than 8 (log2 units), so O and l are rescaled
+// rarely; P = 2^(s - m_ref) <= 2^8 stays well inside bf16/fp16 range.  O and
+// l always share one m_ref, so O / l is exact (a softmax's reference point is
+// arbitrary).
 #pragma once
 
 #include "sm100.cuh"
@@ -44,7 +47,7 @@ struct FwdParams {
   CUtensorMap tm_v;
   CUtensorMap tm_o;  // [B*Hq][N][d] (store)
   float* lse;        // [B*Hq][N]
-  int N, Hq, Hkv, group, BH, n_qtiles, n_ktiles;
+  int N, Hq, Hkv, group, BH, n_pairs, n_ktiles;
   float scale_log2;  // scale * log2(e)
 };
 
@@ -53,19 +56,20 @@ struct FwdLayout {
   static constexpr int kBoxBytes = 128 * 128;        // 128 rows x 64 columns x 2 B
   static constexpr int kChunks = HD / 64;            // 64-column boxes per tile
   static constexpr int kTileBytes = 128 * HD * 2;    // one 128-row tile
-  static constexpr int kSlots = HD == 128 ? 6 : 8;   // K/V ring depth
-  static constexpr int kOffQ = 0;
-  static constexpr int kOffRing = kTileBytes;
+  static constexpr int kSlots = HD == 128 ? 5 : 8;   // K/V ring depth
+  static constexpr int kOffQ = 0;                    // two query tiles
+  static constexpr int kOffRing = 2 * kTileBytes;
   static constexpr int kOffBar = kOffRing + kSlots * kTileBytes;
-  // barriers: q_full, slot_full[kSlots], slot_empty[kSlots], s_full[2], p_full[2], pv_done, done
-  static constexpr int kNumBars = 1 + 2 * kSlots + 2 + 2 + 1 + 1;
+  // barriers: q_full, slot_full[kSlots], slot_empty[kSlots], s_full[2], p_full[2], pv_done[2], done
+  static constexpr int kNumBars = 1 + 2 * kSlots + 6 + 1;
   static constexpr int kOffTmemPtr = kOffBar + kNumBars * 8;
   static constexpr int kOffAbort = kOffTmemPtr + 4;
   static constexpr int kSmemBytes = kOffAbort + 4;
   static constexpr int kDynSmem = kSmemBytes + 1024;  // slack for 1024-byte alignment
+  static_assert(kDynSmem <= 232448, "shared memory budget");
 };
 
-constexpr int kFwdThreads = 192;
+constexpr int kFwdThreads = 320;
 constexpr uint32_t kKernFwd = 1;
 
 template <int HD, bool BF16, bool CAUSAL>
@@ -83,7 +87,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
   uint64_t* s_full = slot_empty + L::kSlots;
   uint64_t* p_full = s_full + 2;
   uint64_t* pv_done = p_full + 2;
-  uint64_t* done_bar = pv_done + 1;
+  uint64_t* done_bar = pv_done + 2;
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(sm + L::kOffTmemPtr);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::kOffAbort);
 
@@ -92,15 +96,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
   const int lane = tid & 31;
 
   // Work item, head-major: the blocks running at the same time mostly share
-  // a head, so its K and V stay in L2; inside a head the largest query
-  // blocks (the most key blocks under a causal mask) go first.
+  // a head, so its K and V stay in L2; inside a head the query pairs with the
+  // most key blocks (under a causal mask) go first.
   const int item = blockIdx.x;
-  const int bh = item / p.n_qtiles;
-  const int qt = p.n_qtiles - 1 - item % p.n_qtiles;
+  const int bh = item / p.n_pairs;
+  const int pair = p.n_pairs - 1 - item % p.n_pairs;
   const int h = bh % p.Hq;
   const int b = bh / p.Hq;
   const int kvh = b * p.Hkv + h / p.group;
-  const int n_kv = CAUSAL ? min(qt + 1, p.n_ktiles) : p.n_ktiles;
+  // key blocks seen by query block t (t = 0, 1) of the pair
+  const int n_kv0 = CAUSAL ? min(2 * pair + 1, p.n_ktiles) : p.n_ktiles;
+  const int n_kv1 = CAUSAL ? min(2 * pair + 2, p.n_ktiles) : p.n_ktiles;
 
   if (tid == 0) {
     mbar_init(q_full, 1);
@@ -111,13 +117,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&p_full[i], 128);
+      mbar_init(&pv_done[i], 1);
     }
-    mbar_init(pv_done, 1);
     mbar_init(done_bar, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == 8) {
     tmem_alloc(tmem_ptr, 512);
     tmem_relinquish();
   }
@@ -125,201 +131,237 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_ptr;
-  const uint32_t tm_S0 = tmem;        // score buffer 0, columns [0, 128)
-  const uint32_t tm_O = tmem + 256;   // output accumulator
 
-  if (warp == 4) {
+  if (warp == 9) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       prefetch_tensormap(&p.tm_q);
       prefetch_tensormap(&p.tm_k);
       prefetch_tensormap(&p.tm_v);
-      mbar_expect_tx(q_full, L::kTileBytes);
-      for (int c = 0; c < L::kChunks; ++c)
-        tma_load_3d(sQ + c * L::kBoxBytes, &p.tm_q, q_full, c * 64, qt * 128, bh);
-      int t = 0;
+      mbar_expect_tx(q_full, 2 * L::kTileBytes);
+      for (int t = 0; t < 2; ++t)
+        for (int c = 0; c < L::kChunks; ++c)
+          tma_load_3d(sQ + t * L::kTileBytes + c * L::kBoxBytes, &p.tm_q, q_full, c * 64,
+                      (2 * pair + t) * 128, bh);
+      int n = 0;
       auto load = [&](const CUtensorMap* map, int tile) -> bool {
-        const int s = t % L::kSlots;
-        if (t >= L::kSlots &&
-            !mbar_wait(&slot_empty[s], ((t / L::kSlots) - 1) & 1, abort_flag, kKernFwd, 4, 0))
+        const int s = n % L::kSlots;
+        if (n >= L::kSlots &&
+            !mbar_wait(&slot_empty[s], ((n / L::kSlots) - 1) & 1, abort_flag, kKernFwd, 9, 0))
           return false;
         mbar_expect_tx(&slot_full[s], L::kTileBytes);
         uint8_t* dst = sRing + s * L::kTileBytes;
         for (int c = 0; c < L::kChunks; ++c)
           tma_load_3d(dst + c * L::kBoxBytes, map, &slot_full[s], c * 64, tile * 128, kvh);
-        ++t;
+        ++n;
         return true;
       };
-      // consumption order of the MMA warp: K0, then (K_{j+1}, V_j) for each j
-      bool ok = load(&p.tm_k, 0);
-      for (int j = 0; ok && j < n_kv; ++j) {
-        if (j + 1 < n_kv) ok = load(&p.tm_k, j + 1);
+      bool ok = true;
+      for (int j = 0; ok && j < n_kv1; ++j) {
+        ok = load(&p.tm_k, j);
         if (ok) ok = load(&p.tm_v, j);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == 8) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t kIdS = idesc_f16(BF16, 128, 128, false, false);
       constexpr uint32_t kIdPV = idesc_f16(BF16, 128, HD, false, true);
-      int t = 0;
-      bool ok = mbar_wait(q_full, 0, abort_flag, kKernFwd, 5, 0);
+      const uint32_t q_base = smem_u32(sQ);
+      int n = 0;
+      bool ok = mbar_wait(q_full, 0, abort_flag, kKernFwd, 8, 0);
       auto take = [&](int& slot) -> bool {
-        slot = t % L::kSlots;
-        if (!mbar_wait(&slot_full[slot], (t / L::kSlots) & 1, abort_flag, kKernFwd, 5, 1))
+        slot = n % L::kSlots;
+        if (!mbar_wait(&slot_full[slot], (n / L::kSlots) & 1, abort_flag, kKernFwd, 8, 1))
           return false;
         tc_fence_after();
-        ++t;
+        ++n;
         return true;
       };
-      auto issue_s = [&](int j, int slot) {
-        const uint32_t kb = smem_u32(sRing + slot * L::kTileBytes);
-        const uint32_t qb = smem_u32(sQ);
-        const uint32_t d_tm = tm_S0 + (j & 1) * 128;
+      // Staggered order: S0_0 S1_0 PV0_0 | S0_1 PV1_0 S1_1 PV0_1 | S0_2 PV1_1 ...
+      // so that one block's softmax runs while the tensor cores work on the
+      // other block.  K_j and V_j are taken in load order (K0 V0 K1 V1 ...).
+      auto issue_s = [&](int t, uint32_t kb) {
+        const uint32_t qb = q_base + t * L::kTileBytes;
 #pragma unroll
         for (int k = 0; k < HD / 16; ++k) {
           const uint32_t off = (k >> 2) * L::kBoxBytes + (k & 3) * 32;
-          umma_ss(d_tm, sdesc_sw128(qb + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024), kIdS,
-                  k > 0);
+          umma_ss(tmem + t * 128, sdesc_sw128(qb + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024),
+                  kIdS, k > 0);
         }
-        umma_commit(&s_full[j & 1]);
-        umma_commit(&slot_empty[slot]);
+        umma_commit(&s_full[t]);
       };
-      int slot = 0;
-      if (ok && n_kv > 0) {
-        ok = take(slot);
-        if (ok) issue_s(0, slot);
-      }
-      for (int j = 0; ok && j < n_kv; ++j) {
-        if (j + 1 < n_kv) {
-          // buffer (j+1)&1 still holds P_{j-1} until PV_{j-1} has completed
-          if (j >= 1) ok = mbar_wait(pv_done, (j - 1) & 1, abort_flag, kKernFwd, 5, 2);
-          if (ok) ok = take(slot);
-          if (!ok) break;
-          issue_s(j + 1, slot);
-        }
-        if (!mbar_wait(&p_full[j & 1], (j >> 1) & 1, abort_flag, kKernFwd, 5, 3)) break;
+      auto issue_pv = [&](int t, int j, uint32_t vb) -> bool {
+        if (!mbar_wait(&p_full[t], j & 1, abort_flag, kKernFwd, 8, 3)) return false;
         tc_fence_after();
-        if (!take(slot)) break;
-        const uint32_t vb = smem_u32(sRing + slot * L::kTileBytes);
-        const uint32_t p_tm = tm_S0 + (j & 1) * 128;
 #pragma unroll
         for (int k = 0; k < 8; ++k)
-          umma_ts(tm_O, p_tm + k * 8, sdesc_sw128(vb + k * 2048, L::kBoxBytes, 1024), kIdPV,
-                  (j > 0 || k > 0) ? 1u : 0u);
-        umma_commit(&slot_empty[slot]);
-        umma_commit(pv_done);
+          umma_ts(tmem + 256 + t * 128, tmem + t * 128 + k * 8,
+                  sdesc_sw128(vb + k * 2048, L::kBoxBytes, 1024), kIdPV, (j > 0 || k > 0) ? 1u : 0u);
+        umma_commit(&pv_done[t]);
+        return true;
+      };
+      // S_t,j+1 overwrites P_t,j: wait until O_t += P_t,j V_j has completed
+      auto wait_pv = [&](int t, int j) -> bool {
+        if (!mbar_wait(&pv_done[t], j & 1, abort_flag, kKernFwd, 8, 2)) return false;
+        tc_fence_after();
+        return true;
+      };
+      int kslot = 0, vslot = 0;
+      if (ok) ok = take(kslot);
+      if (ok) {
+        const uint32_t kb = smem_u32(sRing + kslot * L::kTileBytes);
+        if (n_kv0 > 0) issue_s(0, kb);
+        issue_s(1, kb);
+        umma_commit(&slot_empty[kslot]);
+        ok = take(vslot);
+      }
+      if (ok && n_kv0 > 0) ok = issue_pv(0, 0, smem_u32(sRing + vslot * L::kTileBytes));
+      for (int j = 0; ok && j < n_kv1; ++j) {
+        const bool next1 = j + 1 < n_kv1, next0 = j + 1 < n_kv0;
+        uint32_t kb = 0;
+        if (next1) {
+          if (!(ok = take(kslot))) break;
+          kb = smem_u32(sRing + kslot * L::kTileBytes);
+        }
+        if (next0) {
+          if (!(ok = wait_pv(0, j))) break;
+          issue_s(0, kb);
+        }
+        if (!(ok = issue_pv(1, j, smem_u32(sRing + vslot * L::kTileBytes)))) break;
+        umma_commit(&slot_empty[vslot]);  // V_j: read by both PV_j
+        if (next1) {
+          if (!(ok = wait_pv(1, j))) break;
+          issue_s(1, kb);
+          umma_commit(&slot_empty[kslot]);  // K_j+1: read by both S_j+1
+          if (!(ok = take(vslot))) break;
+        }
+        if (next0 && !(ok = issue_pv(0, j + 1, smem_u32(sRing + vslot * L::kTileBytes)))) break;
       }
       // Everything issued has completed once done_bar flips (also on abort).
       umma_commit(done_bar);
-      mbar_wait(done_bar, 0, abort_flag, kKernFwd, 5, 4);
+      mbar_wait(done_bar, 0, abort_flag, kKernFwd, 8, 4);
     }
   } else {
     // ------------------------------------------------------------ softmax
-    const int r = tid;  // query row within the block == TMEM lane
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-    const int q_row = qt * 128 + r;
+    const int t = warp >> 2;                 // query block of this warpgroup
+    const int r = tid & 127;                 // row within the block == TMEM lane
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tm_S = tmem + t * 128 + lane_off;
+    const uint32_t tm_O = tmem + 256 + t * 128 + lane_off;
+    const int qtile = 2 * pair + t;
+    const int q_row = qtile * 128 + r;
+    const int n_kv = t ? n_kv1 : n_kv0;
     const float c_log2 = p.scale_log2;
+    const uint64_t c2 = f2pack(c_log2, c_log2);
     float m_ref = -INFINITY;  // in log2 units of the scaled scores
     float l_sum = 0.f;
     bool ok = true;
     // Waits are made warp-uniform: tcgen05.ld/st are warp-collective, so a
     // warp either goes on together or leaves together (on abort).
     for (int j = 0; j < n_kv; ++j) {
-      const int buf = j & 1;
-      if (!__all_sync(0xffffffffu,
-                      mbar_wait(&s_full[buf], (j >> 1) & 1, abort_flag, kKernFwd, 0, 0))) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[t], j & 1, abort_flag, kKernFwd, t, 0))) {
         ok = false;
         break;
       }
       tc_fence_after();
       uint32_t s[128];
-      const uint32_t s_tm = tm_S0 + buf * 128 + lane_off;
-      tmem_ld32(s_tm + 0, s);
-      tmem_ld32(s_tm + 32, s + 32);
-      tmem_ld32(s_tm + 64, s + 64);
-      tmem_ld32(s_tm + 96, s + 96);
+      tmem_ld32(tm_S + 0, s);
+      tmem_ld32(tm_S + 32, s + 32);
+      tmem_ld32(tm_S + 64, s + 64);
+      tmem_ld32(tm_S + 96, s + 96);
       tmem_ld_wait();
       // mask: keys past the end of the sequence, and keys after the query
       // inside the diagonal block of a causal problem
       const int kv0 = j * 128;
-      const bool diag = CAUSAL && (j == qt);
+      const bool diag = CAUSAL && (j == qtile);
       if (diag || kv0 + 128 > p.N) {
         const int lim = min(diag ? r : 127, p.N - 1 - kv0);  // last visible column
 #pragma unroll
         for (int c = 0; c < 128; ++c)
           if (c > lim) s[c] = __float_as_uint(-INFINITY);
       }
-      // row max with four independent chains (shorter dependency)
-      float mx4[4] = {__uint_as_float(s[0]), __uint_as_float(s[1]), __uint_as_float(s[2]),
-                      __uint_as_float(s[3])};
+      // row max, four independent chains of three-input max
+      float mx[4] = {__uint_as_float(s[0]), __uint_as_float(s[1]), __uint_as_float(s[2]),
+                     __uint_as_float(s[3])};
 #pragma unroll
-      for (int c = 4; c < 128; ++c) mx4[c & 3] = fmaxf(mx4[c & 3], __uint_as_float(s[c]));
-      const float m_new = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * c_log2;
+      for (int c = 4; c < 128; c += 8) {
+        mx[0] = max3f(mx[0], __uint_as_float(s[c + 0]), __uint_as_float(s[c + 1]));
+        mx[1] = max3f(mx[1], __uint_as_float(s[c + 2]), __uint_as_float(s[c + 3]));
+        mx[2] = max3f(mx[2], __uint_as_float(s[c + 4]), __uint_as_float(s[c + 5]));
+        mx[3] = max3f(mx[3], __uint_as_float(s[c + 6]), __uint_as_float(s[c + 7]));
+      }
+      const float m_new = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * c_log2;
       if (j == 0) {
         m_ref = m_new;
       } else if (__any_sync(0xffffffffu, m_new > m_ref + 8.0f)) {
-        // Move the reference max of every row of this warp (tcgen05.ld/st
-        // are warp-wide), rescaling O and l; O is stable once PV_{j-1} is done.
-        if (!__all_sync(0xffffffffu,
-                        mbar_wait(pv_done, (j - 1) & 1, abort_flag, kKernFwd, 0, 1))) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
+        // Move the reference max of every row of this warp (tcgen05.ld/st are
+        // warp-wide), rescaling O and l.  O_t is stable: S_t,j was issued
+        // only after O_t += P_t,j-1 V_j-1 had completed.
         const float m_upd = fmaxf(m_ref, m_new);
         const float corr = ex2_approx(m_ref - m_upd);
+        const uint64_t corr2 = f2pack(corr, corr);
         m_ref = m_upd;
         l_sum *= corr;
-#pragma unroll
-        for (int c = 0; c < HD; c += 32) {
-          uint32_t o[32];
-          tmem_ld32(tm_O + lane_off + c, o);
+#pragma unroll 1
+        for (int c = 0; c < HD; c += 16) {
+          uint32_t o[16];
+          tmem_ld16(tm_O + c, o);
           tmem_ld_wait();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * corr);
-          tmem_st32(tm_O + lane_off + c, o);
+          for (int i = 0; i < 16; i += 2) {
+            const uint64_t v = mul2(f2pack(__uint_as_float(o[i]), __uint_as_float(o[i + 1])), corr2);
+            o[i] = __float_as_uint(f2lo(v));
+            o[i + 1] = __float_as_uint(f2hi(v));
+          }
+          tmem_st16(tm_O + c, o);
         }
       }
-      const float neg_m = -m_ref;
-      float ls4[4] = {0.f, 0.f, 0.f, 0.f};
+      // P = 2^(s c - m_ref), packed to 16 bits over the first 64 columns of S
+      const uint64_t nm2 = f2pack(-m_ref, -m_ref);
+      uint64_t acc[4] = {0, 0, 0, 0};
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t pk[32];
+      for (int q4 = 0; q4 < 4; ++q4) {
+        uint32_t pk[16];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float p0 = ex2_approx(fmaf(__uint_as_float(s[half * 64 + 2 * i]), c_log2, neg_m));
-          const float p1 =
-              ex2_approx(fmaf(__uint_as_float(s[half * 64 + 2 * i + 1]), c_log2, neg_m));
-          ls4[i & 3] += p0 + p1;
-          pk[i] = pack2<BF16>(p0, p1);
+        for (int i = 0; i < 16; ++i) {
+          const int c = q4 * 32 + 2 * i;
+          const uint64_t x = fma2(f2pack(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), c2, nm2);
+          const uint64_t pp = f2pack(ex2_approx(f2lo(x)), ex2_approx(f2hi(x)));
+          acc[i & 3] = add2(acc[i & 3], pp);
+          pk[i] = pack2<BF16>(f2lo(pp), f2hi(pp));
         }
-        tmem_st32(tm_S0 + buf * 128 + lane_off + half * 32, pk);
+        tmem_st16(tm_S + q4 * 16, pk);
       }
-      l_sum += (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]);
+      const uint64_t a01 = add2(acc[0], acc[1]), a23 = add2(acc[2], acc[3]);
+      const uint64_t a = add2(a01, a23);
+      l_sum += f2lo(a) + f2hi(a);
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&p_full[buf]);
+      mbar_arrive(&p_full[t]);
     }
-    // epilogue: O / l -> 16-bit, staged in the (now idle) Q tile, TMA store
+    // epilogue: O / l -> 16-bit, staged in this block's (now idle) Q tile, TMA store
+    uint8_t* sQt = sQ + t * L::kTileBytes;
     bool ep_ok = ok && n_kv > 0;
-    if (ep_ok) ep_ok = mbar_wait(pv_done, (n_kv - 1) & 1, abort_flag, kKernFwd, 0, 2);
+    if (ep_ok) ep_ok = mbar_wait(&pv_done[t], (n_kv - 1) & 1, abort_flag, kKernFwd, t, 2);
     ep_ok = __all_sync(0xffffffffu, ep_ok);
     if (ep_ok) {
       tc_fence_after();
       const float inv_l = 1.0f / l_sum;
+      const uint64_t inv2 = f2pack(inv_l, inv_l);
 #pragma unroll
       for (int c = 0; c < HD; c += 32) {
         uint32_t o[32];
-        tmem_ld32(tm_O + lane_off + c, o);
+        tmem_ld32(tm_O + c, o);
         tmem_ld_wait();
         uint32_t pk[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          pk[i] = pack2<BF16>(__uint_as_float(o[2 * i]) * inv_l,
-                              __uint_as_float(o[2 * i + 1]) * inv_l);
+        for (int i = 0; i < 16; ++i) {
+          const uint64_t v = mul2(f2pack(__uint_as_float(o[2 * i]), __uint_as_float(o[2 * i + 1])), inv2);
+          pk[i] = pack2<BF16>(f2lo(v), f2hi(v));
+        }
         // columns c..c+31 = 4 chunks of 16 B in box c/64, logical chunk (c%64)/8 + u
-        uint8_t* row_base = sQ + (c / 64) * L::kBoxBytes + r * 128;
+        uint8_t* row_base = sQt + (c / 64) * L::kBoxBytes + r * 128;
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           const int chunk = ((c % 64) / 8 + u) ^ (r & 7);
@@ -331,11 +373,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
         p.lse[static_cast<size_t>(bh) * p.N + q_row] = (m_ref + __log2f(l_sum)) * 0.69314718055994531f;
       fence_proxy_async_smem();
     }
-    // every softmax thread reaches this barrier, whatever happened above
-    named_barrier_sync(1, 128);
-    if (tid == 0 && !*abort_flag) {
+    // every thread of the warpgroup reaches this barrier, whatever happened above
+    named_barrier_sync(1 + t, 128);
+    if (r == 0 && !*abort_flag) {
       for (int c = 0; c < L::kChunks; ++c)
-        tma_store_3d(&p.tm_o, sQ + c * L::kBoxBytes, c * 64, qt * 128, bh);
+        tma_store_3d(&p.tm_o, sQt + c * L::kBoxBytes, c * 64, qtile * 128, bh);
       bulk_commit_group();
       bulk_wait_group_read0();
     }
@@ -343,7 +385,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 8) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
