@@ -136,9 +136,9 @@ struct BwdLayout {
   static constexpr int kOffLse = kOffDS + 2 * kDsBytes;
   static constexpr int kOffD = kOffLse + kStages * 256;
   static constexpr int kOffBar = kOffD + kStages * 256;
-  // kv_full, q_full[S], q_empty[S], s_full[2], dp_full[2], ds_full[2], pt_free[2],
-  // dq_full[2], dq_drained[2], ds_free[2], acc_done, done
-  static constexpr int kNumBars = 1 + 2 * kStages + 7 * 2 + 2;
+  // kv_full, q_full[S], step_done[S], sdp_full[2], ds_full[2], dq_full[2],
+  // dq_drained[2], acc_done, done
+  static constexpr int kNumBars = 1 + 2 * kStages + 4 * 2 + 2;
   static constexpr int kOffTmemPtr = kOffBar + kNumBars * 8;
   static constexpr int kOffAbort = kOffTmemPtr + 4;
   static constexpr int kSmemBytes = kOffAbort + 4;
@@ -169,15 +169,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::kOffBar);
   uint64_t* kv_full = bars;
   uint64_t* q_full = kv_full + 1;
-  uint64_t* q_empty = q_full + L::kStages;
-  uint64_t* s_full = q_empty + L::kStages;
-  uint64_t* dp_full = s_full + 2;
-  uint64_t* ds_full = dp_full + 2;
-  uint64_t* pt_free = ds_full + 2;
-  uint64_t* dq_full = pt_free + 2;
+  // step_done[s]: every MMA of the step held in stage s has completed, so
+  // the stage may be refilled and the step's dS^T buffer rewritten
+  uint64_t* step_done = q_full + L::kStages;
+  uint64_t* sdp_full = step_done + L::kStages;  // S^T and dP^T of a step buffer ready
+  uint64_t* ds_full = sdp_full + 2;
+  uint64_t* dq_full = ds_full + 2;
   uint64_t* dq_drained = dq_full + 2;
-  uint64_t* ds_free = dq_drained + 2;
-  uint64_t* acc_done = ds_free + 2;
+  uint64_t* acc_done = dq_drained + 2;
   uint64_t* done_bar = acc_done + 1;
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(sm + L::kOffTmemPtr);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::kOffAbort);
@@ -209,16 +208,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
     mbar_init(kv_full, 1);
     for (int s = 0; s < L::kStages; ++s) {
       mbar_init(&q_full[s], 1);
-      mbar_init(&q_empty[s], 1);
+      mbar_init(&step_done[s], 1);
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&s_full[i], 1);
-      mbar_init(&dp_full[i], 1);
+      mbar_init(&sdp_full[i], 1);
       mbar_init(&ds_full[i], 256);
-      mbar_init(&pt_free[i], 1);
       mbar_init(&dq_full[i], 1);
       mbar_init(&dq_drained[i], kDrainThreads);
-      mbar_init(&ds_free[i], 1);
     }
     mbar_init(acc_done, 1);
     mbar_init(done_bar, 1);
@@ -256,7 +252,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
       for (int t = 0; t < T_steps; ++t) {
         const int s = t % L::kStages;
         if (t >= L::kStages &&
-            !mbar_wait(&q_empty[s], ((t / L::kStages) - 1) & 1, abort_flag, kKernBwd, 12, 0))
+            !mbar_wait(&step_done[s], ((t / L::kStages) - 1) & 1, abort_flag, kKernBwd, 12, 0))
           break;
         const int bh = step_bh(t), qt = step_qt(t);
         mbar_expect_tx(&q_full[s], 2 * L::kQTile + 512);
@@ -289,7 +285,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
           umma_ss(tm_S(t & 1),
                   sdesc_sw128(kb + (k >> 2) * L::kKVBox + (k & 3) * 32, 16, 1024),
                   sdesc_sw128(qb + (k >> 2) * L::kQBox + (k & 3) * 32, 16, 1024), kIdS, k > 0);
-        umma_commit(&s_full[t & 1]);
         return true;
       };
       auto issue_dp = [&](int t) {
@@ -300,7 +295,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
           umma_ss(tm_dP(t & 1),
                   sdesc_sw128(vb + (k >> 2) * L::kKVBox + (k & 3) * 32, 16, 1024),
                   sdesc_sw128(ob + (k >> 2) * L::kQBox + (k & 3) * 32, 16, 1024), kIdS, k > 0);
-        umma_commit(&dp_full[t & 1]);
+        umma_commit(&sdp_full[t & 1]);
       };
       for (int t = 0; ok && t < 2 && t < T_steps; ++t) {
         ok = issue_s(t);
@@ -328,19 +323,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
         for (int k = 0; k < 4; ++k)
           umma_ts(tm_dV, tm_S(buf) + (k >> 1) * 32 + (k & 1) * 8,
                   sdesc_sw128(ob + k * 2048, L::kQBox, 1024), kIdAcc, (t > 0 || k > 0) ? 1u : 0u);
-        umma_commit(&pt_free[buf]);
         // dK += dS^T Q: dS^T K-major from shared memory, Q read MN-major.
 #pragma unroll
         for (int k = 0; k < 4; ++k)
           umma_ss(tm_dK, sdesc_sw128(db + k * 32, 16, 1024),
                   sdesc_sw128(qb + k * 2048, L::kQBox, 1024), kIdAcc, (t > 0 || k > 0) ? 1u : 0u);
-        umma_commit(&ds_free[buf]);
-        umma_commit(&q_empty[s]);
+        umma_commit(&step_done[s]);
         if (t + 2 < T_steps) {
-          // S^T_{t+2} overwrites P^T_t: wait for dV_t; dP^T_{t+2} overwrites
-          // dQ^T_t: wait for the drain warps to have read it.
-          if (!mbar_wait(&pt_free[buf], (t >> 1) & 1, abort_flag, kKernBwd, 13, 3)) break;
-          tc_fence_after();
+          // S^T_{t+2} overwrites P^T_t, which dV_t (issued just before by this
+          // thread) reads: the tensor core runs one thread's MMAs in issue
+          // order, reading an MMA's operands before a later MMA writes its
+          // result, so no wait is needed (a wait for an MMA's completion
+          // costs several hundred idle tensor-core cycles on B200).
+          // dP^T_{t+2} overwrites dQ^T_t: wait for the drain warps to read it.
           if (!issue_s(t + 2)) break;
           if (!mbar_wait(&dq_drained[buf], (t >> 1) & 1, abort_flag, kKernBwd, 13, 4)) break;
           tc_fence_after();
@@ -362,7 +357,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
     for (int t = 0; t < T_steps; ++t) {
       const int buf = t & 1, s = t % L::kStages;
       const int q_first = step_qt(t) * 64 + half * 32;  // first query of this thread's columns
-      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[buf], (t >> 1) & 1, abort_flag, kKernBwd, 0, 0)))
+      if (!__all_sync(0xffffffffu, mbar_wait(&sdp_full[buf], (t >> 1) & 1, abort_flag, kKernBwd, 0, 0)))
         break;
       tc_fence_after();
       uint32_t v[32];
@@ -392,9 +387,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
 #pragma unroll
       for (int i = 0; i < 16; ++i) pk[i] = pack2<BF16>(pr[2 * i], pr[2 * i + 1]);
       tmem_st16(tm_S(buf) + lane_off + half * 32, pk);
-      if (!__all_sync(0xffffffffu, mbar_wait(&dp_full[buf], (t >> 1) & 1, abort_flag, kKernBwd, 0, 1)))
-        break;
-      tc_fence_after();
       tmem_ld32(tm_dP(buf) + lane_off + half * 32, v);
       const float4* d4 = reinterpret_cast<const float4*>(sD + s * 64 + half * 32);
       tmem_ld_wait();
@@ -408,9 +400,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
       }
 #pragma unroll
       for (int i = 0; i < 16; ++i) pk[i] = pack2<BF16>(pr[2 * i], pr[2 * i + 1]);
-      // dS^T buffer `buf` is free once dK_{t-2} (its last reader) has completed
-      if (t >= 2 &&
-          !__all_sync(0xffffffffu, mbar_wait(&ds_free[buf], ((t >> 1) - 1) & 1, abort_flag, kKernBwd, 0, 2)))
+      // dS^T buffer `buf` is free once step t-2 (dK_{t-2} its last reader) is done
+      if (t >= 2 && !__all_sync(0xffffffffu, mbar_wait(&step_done[(t - 2) % L::kStages],
+                                                       ((t - 2) / L::kStages) & 1, abort_flag,
+                                                       kKernBwd, 0, 2)))
         break;
       uint8_t* row_base = sDS + buf * L::kDsBytes + r * 128;
 #pragma unroll

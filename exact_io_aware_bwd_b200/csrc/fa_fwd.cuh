@@ -23,8 +23,7 @@
 //   warp 8     MMA issuer (one thread): S_t,j = Q_t K_j^T and O_t += P_t,j V_j
 //              for t = 0, 1, staggered as S0_j+1, O1 += P1_j V_j, S1_j+1,
 //              O0 += P0_j+1 V_j+1, ... so that one block's softmax overlaps the
-//              other block's products.  S_t,j+1 overwrites P_t,j, so it is
-//              issued only once O_t += P_t,j V_j has completed.
+//              other block's products.
 //   warp 9     TMA producer: Q0, Q1 once, then K_0, V_0, K_1, V_1, ... through
 //              a ring of kSlots tiles.
 // Tensor memory (512 columns x 128 lanes x 32 bit): S0 [0,128), S1 [128,256),
@@ -181,6 +180,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
       // Staggered order: S0_0 S1_0 PV0_0 | S0_1 PV1_0 S1_1 PV0_1 | S0_2 PV1_1 ...
       // so that one block's softmax runs while the tensor cores work on the
       // other block.  K_j and V_j are taken in load order (K0 V0 K1 V1 ...).
+      // S_t,j+1 is written over the tensor memory that O_t += P_t,j V_j reads
+      // P_t,j from, and is issued right after it by this same thread: the
+      // tensor core runs the MMAs of one thread in issue order, reading an
+      // MMA's operands before a later MMA writes its result, so no wait is
+      // put between them (waiting for an MMA's completion before issuing the
+      // next costs several hundred cycles of idle tensor core on B200).
       auto issue_s = [&](int t, uint32_t kb) {
         const uint32_t qb = q_base + t * L::kTileBytes;
 #pragma unroll
@@ -201,12 +206,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
         umma_commit(&pv_done[t]);
         return true;
       };
-      // S_t,j+1 overwrites P_t,j: wait until O_t += P_t,j V_j has completed
-      auto wait_pv = [&](int t, int j) -> bool {
-        if (!mbar_wait(&pv_done[t], j & 1, abort_flag, kKernFwd, 8, 2)) return false;
-        tc_fence_after();
-        return true;
-      };
       int kslot = 0, vslot = 0;
       if (ok) ok = take(kslot);
       if (ok) {
@@ -224,14 +223,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
           if (!(ok = take(kslot))) break;
           kb = smem_u32(sRing + kslot * L::kTileBytes);
         }
-        if (next0) {
-          if (!(ok = wait_pv(0, j))) break;
-          issue_s(0, kb);
-        }
+        if (next0) issue_s(0, kb);
         if (!(ok = issue_pv(1, j, smem_u32(sRing + vslot * L::kTileBytes)))) break;
         umma_commit(&slot_empty[vslot]);  // V_j: read by both PV_j
         if (next1) {
-          if (!(ok = wait_pv(1, j))) break;
           issue_s(1, kb);
           umma_commit(&slot_empty[kslot]);  // K_j+1: read by both S_j+1
           if (!(ok = take(vslot))) break;
@@ -296,8 +291,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
         m_ref = m_new;
       } else if (__any_sync(0xffffffffu, m_new > m_ref + 8.0f)) {
         // Move the reference max of every row of this warp (tcgen05.ld/st are
-        // warp-wide), rescaling O and l.  O_t is stable: S_t,j was issued
-        // only after O_t += P_t,j-1 V_j-1 had completed.
+        // warp-wide), rescaling O and l, once O_t += P_t,j-1 V_j-1 is done.
+        if (!__all_sync(0xffffffffu, mbar_wait(&pv_done[t], (j - 1) & 1, abort_flag, kKernFwd, t, 1))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
         const float m_upd = fmaxf(m_ref, m_new);
         const float corr = ex2_approx(m_ref - m_upd);
         const uint64_t corr2 = f2pack(corr, corr);
