@@ -276,16 +276,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
         for (int c = 0; c < 128; ++c)
           if (c > lim) s[c] = __float_as_uint(-INFINITY);
       }
-      // row max, four independent chains of three-input max
-      float mx[4] = {__uint_as_float(s[0]), __uint_as_float(s[1]), __uint_as_float(s[2]),
-                     __uint_as_float(s[3])};
+      // row max, eight independent chains
+      float mx[8];
 #pragma unroll
-      for (int c = 4; c < 128; c += 8) {
-        mx[0] = max3f(mx[0], __uint_as_float(s[c + 0]), __uint_as_float(s[c + 1]));
-        mx[1] = max3f(mx[1], __uint_as_float(s[c + 2]), __uint_as_float(s[c + 3]));
-        mx[2] = max3f(mx[2], __uint_as_float(s[c + 4]), __uint_as_float(s[c + 5]));
-        mx[3] = max3f(mx[3], __uint_as_float(s[c + 6]), __uint_as_float(s[c + 7]));
-      }
+      for (int i = 0; i < 8; ++i) mx[i] = __uint_as_float(s[i]);
+#pragma unroll
+      for (int c = 8; c < 128; ++c) mx[c & 7] = fmaxf(mx[c & 7], __uint_as_float(s[c]));
+#pragma unroll
+      for (int i = 0; i < 4; ++i) mx[i] = fmaxf(mx[i], mx[i + 4]);
       const float m_new = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * c_log2;
       if (j == 0) {
         m_ref = m_new;

@@ -74,6 +74,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Same, but the thread may be suspended in hardware for up to `hint_ns`
+// until the phase completes, instead of returning at once (no polling
+// traffic on shared memory while it waits).
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity,
+                                                    uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Waits for the phase of `bar` with the given parity to complete.  Gives up
 // after g_wait_limit_ns (or at once when *abort is set by another thread of
 // the CTA), records a timeout in g_device_status, raises *abort and returns
@@ -84,10 +100,11 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   const uint64_t limit = g_wait_limit_ns;
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
+  for (;;) {
+    // sleep in hardware until the phase flips, at most 0.2 ms per round
+    if (mbar_try_wait_sleep(bar, parity, 200000u)) return true;
     if (*abort) return false;
-    if ((it & 63u) == 0 && globaltimer_ns() - t0 > limit) {
+    if (globaltimer_ns() - t0 > limit) {
       record_error(kStatusTimeout, kernel, role, site);
       *abort = 1;
       return false;
