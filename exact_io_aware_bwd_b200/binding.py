@@ -168,3 +168,22 @@ def attention_bwd(q, k, v, o, dout, lse, scale: float | None = None, causal: boo
                                 device=q.device, dtype=torch.uint8)
     fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, scale, causal, workspace, stream)
     return dq, dk, dv
+
+
+def fa_bwd_noalloc(q, k, v, o, dout, lse, dq, dk, dv, scale: float, causal: bool,
+                   stream=None) -> None:
+    """fa_bwd without a workspace: for callers that cannot allocate device
+    memory.  Uses the library's fixed scratch array (FA_BWD_NOALLOC_SCRATCH_BYTES
+    per device); raises FaError(FA_ERR_UNSUPPORTED) for problems that need more.
+    Calls on one device share that array, so order them on one stream."""
+    lib = load()
+    fn = lib.fa_bwd_noalloc
+    if fn.argtypes is None:
+        vp, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+        fn.argtypes = [vp] * 9 + [i, i, i, i, i, f, i, i, vp]
+        fn.restype = i
+    B, Hq, Hkv, N, d = _dims(q, k)
+    st = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
+            _ptr(dv), B, Hq, Hkv, N, d, float(scale), int(bool(causal)), _DTYPES[q.dtype],
+            _stream(stream))
+    _check(st, "fa_bwd_noalloc")

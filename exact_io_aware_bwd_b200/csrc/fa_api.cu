@@ -315,6 +315,57 @@ fa_status_t fa_set_profile_events(int kernel_id, void* start, void* stop) {
   return FA_OK;
 }
 
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Fixed scratch for fa_bwd_noalloc: reserved in the device memory of every GPU
+// that loads this library, for the life of the process.  Host code must not
+// pass `g_bwd_noalloc_scratch` itself to a kernel (on the host the name is
+// only a stand-in); its device address is looked up once per device with
+// cudaGetSymbolAddress.
+static __device__ __align__(256) unsigned char g_bwd_noalloc_scratch[FA_BWD_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[64] = {nullptr};
+
+// Device address of the scratch array on the current device (looked up on
+// the first call per device).
+fa_status_t noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return FA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_bwd_noalloc_scratch) != cudaSuccess || p == nullptr)
+      return FA_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return FA_OK;
+}
+}  // namespace
+
+extern "C" {
+
+fa_status_t fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                           const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                           int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+                           fa_dtype_t dtype, void* stream) {
+  bool empty = false;
+  fa_status_t s = check_common(B, Hq, Hkv, N, d, scale, causal, dtype, &empty);
+  if (s != FA_OK) return s;
+  if (empty) return FA_OK;
+  const size_t need = fa::bwd_workspace_bytes(B, Hq, N, d);
+  if (need > FA_BWD_NOALLOC_SCRATCH_BYTES) return FA_ERR_UNSUPPORTED;
+  if ((s = check_device()) != FA_OK) return s;
+  void* scratch = nullptr;
+  if ((s = noalloc_scratch(&scratch)) != FA_OK) return s;
+  return fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, N, d, scale, causal, dtype,
+                scratch, FA_BWD_NOALLOC_SCRATCH_BYTES, stream);
+}
+
 const char* fa_status_string(fa_status_t status) {
   switch (status) {
     case FA_OK: return "ok";

@@ -134,6 +134,41 @@ fa_status_t fa_selftest_wait_timeout(uint64_t limit_ns, void* stream);
  */
 fa_status_t fa_set_profile_events(int kernel_id, void* start, void* stop);
 
+/*
+ * Backward pass for callers that cannot allocate device memory.
+ *
+ * fa_bwd needs a caller-provided workspace.  Some callers cannot obtain one:
+ * code that runs where cudaMalloc is not allowed or not wanted (a host
+ * callback or plugin that only receives raw tensor pointers from a host
+ * framework, a real-time loop that forbids allocation after start-up, or a
+ * runtime whose memory is owned by another allocator).  This entry point
+ * takes the same tensors as fa_bwd but no workspace: it uses a fixed scratch
+ * array of FA_BWD_NOALLOC_SCRATCH_BYTES bytes that the library reserves in
+ * device memory of every GPU that loads it, kept until the process exits.
+ * The pages describe no counterpart; this is an interface convenience.
+ *
+ * - Size limit: the problem must satisfy
+ *     fa_bwd_workspace_bytes(B, Hq, Hkv, N, d) <= FA_BWD_NOALLOC_SCRATCH_BYTES,
+ *   otherwise FA_ERR_UNSUPPORTED is returned and nothing is launched.
+ * - The first call on a device looks up the array's device address (once
+ *   per device, with that device current); make that first call before any
+ *   stream capture.  Later calls do no set-up.
+ * - No allocation of any kind: no cudaMalloc / cudaFree, no library routine
+ *   that allocates.
+ * - Every call on a device shares the one array.  Calls whose kernels
+ *   overlap on the GPU (different streams, or different host threads without
+ *   ordering) race on it and give wrong results: order them on one stream.
+ *   The array keeps the last call's contents; each call clears what it needs
+ *   zeroed (the dQ accumulator) and overwrites the rest before reading it.
+ * - Everything else (arguments, layouts, errors, asynchrony) is as fa_bwd.
+ */
+#define FA_BWD_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
+
+fa_status_t fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                           const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                           int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+                           fa_dtype_t dtype, void* stream);
+
 /* Static English description of a status code. */
 const char* fa_status_string(fa_status_t status);
 
