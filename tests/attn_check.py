@@ -28,8 +28,9 @@ def run_gpu(q, k, v, do, scale, causal):
     qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, do))
     o, lse = binding.attention_fwd(qd, kd, vd, scale, causal)
     dq, dk, dv = binding.attention_bwd(qd, kd, vd, o, dod, lse, scale, causal)
+    word = binding.fa_peek_device_status_word()
     status = binding.fa_get_device_status()
-    assert status == binding.FA_OK, binding.fa_status_string(status)
+    assert status == binding.FA_OK, f"{binding.fa_status_string(status)} (status word {word:#010x})"
     return {n: t.cpu() for n, t in dict(o=o, lse=lse, dq=dq, dk=dk, dv=dv).items()}
 
 
