@@ -61,6 +61,8 @@ def load():
             lib.fa_selftest_wait_timeout.restype = i
             lib.fa_set_profile_events.argtypes = [i, vp, vp]
             lib.fa_set_profile_events.restype = i
+            lib.fa_set_bwd_max_blocks.argtypes = [i]
+            lib.fa_set_bwd_max_blocks.restype = i
             lib.fa_status_string.argtypes = [i]
             lib.fa_status_string.restype = ctypes.c_char_p
             _lib = lib
@@ -143,6 +145,11 @@ def fa_set_profile_events(kernel_id: int, start=None, stop=None) -> None:
     objects that have been recorded once, or raw handles); None clears."""
     h = lambda e: None if e is None else ctypes.c_void_p(e.cuda_event if hasattr(e, "cuda_event") else int(e))
     _check(load().fa_set_profile_events(int(kernel_id), h(start), h(stop)), "fa_set_profile_events")
+
+
+def fa_set_bwd_max_blocks(max_blocks: int) -> None:
+    """Cap the persistent blocks of the backward main pass (0: one per SM)."""
+    _check(load().fa_set_bwd_max_blocks(int(max_blocks)), "fa_set_bwd_max_blocks")
 
 
 # ------------------------------------------------------------ conveniences

@@ -9,6 +9,7 @@
 #include <cstdint>
 #include <cstring>
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 
 #include "fa.h"
@@ -64,6 +65,9 @@ void prof_end(int id, cudaStream_t st) {
   if (g_prof_stop[id]) cudaEventRecord(g_prof_stop[id], st);
 }
 
+// Cap on the persistent blocks of the backward main pass (0: one per SM).
+std::atomic<int> g_bwd_max_blocks{0};
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // Device must be sm_100 (B200 class); checked once per device.
@@ -80,6 +84,19 @@ fa_status_t check_device() {
     ok_dev[dev] = (major == 10 && minor == 0) ? 1 : 2;
   }
   return ok_dev[dev] == 1 ? FA_OK : FA_ERR_UNSUPPORTED;
+}
+
+// Number of SMs of the current device (cached per device); 0 on error.
+int sm_count() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  static int n_sm[64] = {0};
+  if (n_sm[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    n_sm[dev] = n;
+  }
+  return n_sm[dev];
 }
 
 // Checks shared by fa_fwd and fa_bwd.  Sets *empty for a problem with no work.
@@ -154,11 +171,12 @@ fa_status_t bwd_run(const void* q, const void* k, const void* v, const void* o, 
   float* Dvec = static_cast<float*>(workspace);
   float* lse2 = Dvec + BHq * Np;
   float* dqacc = lse2 + BHq * Np;
-
-  // 1. D, lse2, zeroed accumulator
   const int64_t rows = BHq * Np;
+  unsigned* work_counter = reinterpret_cast<unsigned*>(dqacc + rows * HD);
+
+  // 1. D, lse2, zeroed accumulator and work counter
   fa::fa_bwd_pre_kernel<HD, BF><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(
-      o, dout, lse, Dvec, lse2, dqacc, N, static_cast<int>(Np), rows);
+      o, dout, lse, Dvec, lse2, dqacc, work_counter, N, static_cast<int>(Np), rows);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
 
   // 2. main pass
@@ -175,6 +193,7 @@ fa_status_t bwd_run(const void* q, const void* k, const void* v, const void* o, 
   prm.dqacc = dqacc;
   prm.dk = dk;
   prm.dv = dv;
+  prm.work_counter = work_counter;
   prm.N = N;
   prm.Np = static_cast<int>(Np);
   prm.Hq = Hq;
@@ -185,7 +204,11 @@ fa_status_t bwd_run(const void* q, const void* k, const void* v, const void* o, 
   prm.BHkv = static_cast<int>(BHkv);
   prm.scale = scale;
   prm.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
-  const int grid = prm.n_ktiles * prm.BHkv;
+  prm.n_items = prm.n_ktiles * prm.BHkv;
+  int n_sm = 0;
+  if ((n_sm = sm_count()) <= 0) return FA_ERR_CUDA;
+  const int cap = g_bwd_max_blocks.load();
+  const int grid = std::min(prm.n_items, cap > 0 ? std::min(cap, n_sm) : n_sm);  // persistent
   fa_status_t s = causal ? launch_bwd_main<HD, BF, true>(prm, grid, st)
                          : launch_bwd_main<HD, BF, false>(prm, grid, st);
   if (s != FA_OK) return s;
@@ -312,6 +335,12 @@ fa_status_t fa_set_profile_events(int kernel_id, void* start, void* stop) {
   if ((start == nullptr) != (stop == nullptr)) return FA_ERR_INVALID_ARG;
   g_prof_start[kernel_id] = reinterpret_cast<cudaEvent_t>(start);
   g_prof_stop[kernel_id] = reinterpret_cast<cudaEvent_t>(stop);
+  return FA_OK;
+}
+
+fa_status_t fa_set_bwd_max_blocks(int max_blocks) {
+  if (max_blocks < 0) return FA_ERR_INVALID_ARG;
+  g_bwd_max_blocks.store(max_blocks);
   return FA_OK;
 }
 

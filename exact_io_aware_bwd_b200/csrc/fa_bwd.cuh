@@ -17,11 +17,14 @@
 //   bwd_pre   one warp per query row: D_i = dO_i . O_i, lse2_i = lse_i log2(e)
 //             (+inf for padding rows, which makes their P exactly 0), and a
 //             zeroed fp32 dQ accumulator row.
-//   bwd_main  one thread block per (128-row key block j, kv head): K_j, V_j
-//             stay in shared memory; the block walks every query head of the
-//             group and every 64-row query block i (causal: i >= the
-//             diagonal).  Per step, all products on the tensor cores with
-//             fp32 accumulators in tensor memory:
+//   bwd_main  persistent: one thread block per SM takes work items (128-row
+//             key block j, kv head) one after another from a counter in the
+//             workspace, head-major and, within a head, the key blocks with
+//             the most query blocks first.  For an item, K_j and V_j stay in
+//             shared memory; the block walks every query head of the group
+//             and every 64-row query block i (causal: i >= the diagonal).
+//             Per step, all products on the tensor cores with fp32
+//             accumulators in tensor memory:
 //               S^T  = K_j Q_i^T        (128 x 64)
 //               dP^T = V_j dO_i^T       (128 x 64)
 //               softmax warps: P^T, dS^T = P^T o (dP^T - D)
@@ -30,15 +33,21 @@
 //               dV  += P^T dO_i         (P^T read from tensor memory)
 //               dK  += dS^T Q_i
 //             dK, dV stay in tensor memory for the whole walk and are written
-//             once at the end: no atomics on them.
+//             once at the end: no atomics on them.  The steps of consecutive
+//             items run through the same rings without a break: the next
+//             item's Q / dO loads start while the last steps of the previous
+//             one run, and its dK / dV are written out while the next item's
+//             first steps run.
 //   bwd_post  dQ = scale * accumulator, converted to the I/O dtype.
 //
 // Warp roles of bwd_main (448 threads):
 //   warps 0-7   softmax-gradient: warp w owns key rows 32(w%4)..+31 (tensor
 //               memory lanes) and query columns 32(w/4)..+31 of each step.
-//   warps 8-11  dQ drain (lane = feature index of dQ^T) and, at the end, the
-//               dK / dV epilogue (lane = key row).
-//   warp 12     TMA producer.     warp 13     MMA issuer (one thread).
+//   warps 8-11  dQ drain (lane = feature index of dQ^T) and, after each
+//               item, the dK / dV epilogue (lane = key row).
+//   warp 12     TMA producer; it also claims the work items and passes them
+//               to the other roles through a small ring in shared memory.
+//   warp 13     MMA issuer (one thread).
 // Tensor memory: dV [0,128), dK [128,256), and two step buffers b = 0, 1:
 // S^T at 256+128b (64 columns; P^T is written over it as 16-bit pairs, each
 // warp half over its own columns) and dP^T at 256+128b+64 (dQ^T is written
@@ -60,9 +69,13 @@ constexpr uint32_t kKernSelftest = 9;
 
 __host__ __device__ inline int64_t bwd_padded_rows(int N) { return (static_cast<int64_t>(N) + 127) / 128 * 128; }
 
+// Workspace: D [rows], lse2 [rows], dQ accumulator [rows][d] (fp32), then
+// 256 bytes holding the work-item counter of bwd_main.
+constexpr size_t kBwdWorkspaceTail = 256;
+
 inline size_t bwd_workspace_bytes(int B, int Hq, int N, int d) {
   const int64_t rows = static_cast<int64_t>(B) * Hq * bwd_padded_rows(N);
-  return static_cast<size_t>(rows) * 4u * static_cast<size_t>(2 + d);
+  return static_cast<size_t>(rows) * 4u * static_cast<size_t>(2 + d) + kBwdWorkspaceTail;
 }
 
 // ---------------------------------------------------------------------------
@@ -74,11 +87,13 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const void* __restrict_
                                                          const float* __restrict__ lse,
                                                          float* __restrict__ Dvec,
                                                          float* __restrict__ lse2,
-                                                         float* __restrict__ dqacc, int N, int Np,
-                                                         int64_t total_rows) {
+                                                         float* __restrict__ dqacc,
+                                                         unsigned* __restrict__ work_counter, int N,
+                                                         int Np, int64_t total_rows) {
   using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
+  if (blockIdx.x == 0 && threadIdx.x == 0) *work_counter = 0u;
   if (row >= total_rows) return;
   const int64_t bh = row / Np;
   const int n = static_cast<int>(row % Np);
@@ -115,7 +130,8 @@ struct BwdParams {
   float* dqacc;          // [B*Hq][Np][d] fp32 accumulator
   void* dk;              // [B*Hkv][N][d]
   void* dv;
-  int N, Np, Hq, Hkv, group, n_ktiles, n_qtiles, BHkv;
+  unsigned* work_counter;  // next work item (zeroed by bwd_pre)
+  int N, Np, Hq, Hkv, group, n_ktiles, n_qtiles, BHkv, n_items;
   float scale_log2, scale;
 };
 
@@ -136,10 +152,12 @@ struct BwdLayout {
   static constexpr int kOffLse = kOffDS + 2 * kDsBytes;
   static constexpr int kOffD = kOffLse + kStages * 256;
   static constexpr int kOffBar = kOffD + kStages * 256;
+  static constexpr int kSched = 4;                      // work-item ring slots
   // kv_full, q_full[S], step_done[S], sdp_full[2], ds_full[2], dq_full[2],
-  // dq_drained[2], acc_done, done
-  static constexpr int kNumBars = 1 + 2 * kStages + 4 * 2 + 2;
-  static constexpr int kOffTmemPtr = kOffBar + kNumBars * 8;
+  // dq_drained[2], acc_done, acc_free, done, sched_full[4], sched_empty[4]
+  static constexpr int kNumBars = 1 + 2 * kStages + 4 * 2 + 3 + 2 * kSched;
+  static constexpr int kOffSched = kOffBar + kNumBars * 8;
+  static constexpr int kOffTmemPtr = kOffSched + kSched * 4;
   static constexpr int kOffAbort = kOffTmemPtr + 4;
   static constexpr int kSmemBytes = kOffAbort + 4;
   // Tiles must sit on 1024-byte boundaries (128-byte swizzle atoms).  The
@@ -149,6 +167,30 @@ struct BwdLayout {
   static constexpr int kDynSmem = kSmemBytes + (232448 - kSmemBytes >= 1024 ? 1024 : 0);
   static_assert(kDynSmem <= 232448, "shared memory budget");
 };
+
+// One work item of bwd_main: key block jt (128 rows) of kv head kvh.
+struct BwdItem {
+  int kvh;  // b * Hkv + kv head
+  int kv0;  // first key row
+  int i0;   // first query block (64 rows) that sees the key block
+  int nq;   // query blocks per query head
+  int T;    // steps: group * nq
+  int bh0;  // first query head of the group (b * Hq + g * group)
+};
+
+template <bool CAUSAL>
+__device__ __forceinline__ BwdItem bwd_item(const BwdParams& p, int item) {
+  BwdItem it;
+  it.kvh = item / p.n_ktiles;
+  const int jt = item % p.n_ktiles;
+  const int b = it.kvh / p.Hkv, g = it.kvh % p.Hkv;
+  it.kv0 = jt * 128;
+  it.i0 = CAUSAL ? 2 * jt : 0;
+  it.nq = p.n_qtiles - it.i0;
+  it.T = p.group * it.nq;
+  it.bh0 = b * p.Hq + g * p.group;
+  return it;
+}
 
 constexpr int kBwdThreads = 448;
 
@@ -176,8 +218,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
   uint64_t* ds_full = sdp_full + 2;
   uint64_t* dq_full = ds_full + 2;
   uint64_t* dq_drained = dq_full + 2;
-  uint64_t* acc_done = dq_drained + 2;
-  uint64_t* done_bar = acc_done + 1;
+  uint64_t* acc_done = dq_drained + 2;  // every MMA of an item has completed
+  uint64_t* acc_free = acc_done + 1;    // the epilogue has read an item's dK, dV
+  uint64_t* done_bar = acc_free + 1;
+  uint64_t* sched_full = done_bar + 1;
+  uint64_t* sched_empty = sched_full + L::kSched;
+  volatile int* sched_item = reinterpret_cast<volatile int*>(sm + L::kOffSched);
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(sm + L::kOffTmemPtr);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::kOffAbort);
 
@@ -188,21 +234,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
     if (tid == 0) record_error(kStatusSmemAlign, kKernBwd, 0, 0);
     return;
   }
-
-  // Work item, head-major: the blocks running at the same time mostly share
-  // a kv head, so its Q, dO and dQ accumulator stay in L2; inside a head the
-  // key blocks nearest the start go first (under a causal mask they see the
-  // most query blocks).
-  const int item = blockIdx.x;
-  const int kvh = item / p.n_ktiles;  // b * Hkv + g
-  const int jt = item % p.n_ktiles;   // key block (128 rows)
-  const int b = kvh / p.Hkv;
-  const int g = kvh % p.Hkv;
-  const int kv0 = jt * 128;
-  const int i0 = CAUSAL ? 2 * jt : 0;       // first query block (64 rows) that sees key block jt
-  const int nq = p.n_qtiles - i0;            // query blocks per head
-  const int T_steps = p.group * nq;
   constexpr int kDrainThreads = HD == 128 ? 128 : 64;
+  constexpr int kSchedReaders = 1 + 8 + 4;  // MMA thread, softmax warps, drain warps
 
   if (tid == 0) {
     mbar_init(kv_full, 1);
@@ -217,7 +250,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
       mbar_init(&dq_drained[i], kDrainThreads);
     }
     mbar_init(acc_done, 1);
+    mbar_init(acc_free, 128);
     mbar_init(done_bar, 1);
+    for (int i = 0; i < L::kSched; ++i) {
+      mbar_init(&sched_full[i], 1);
+      mbar_init(&sched_empty[i], kSchedReaders);
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -233,10 +271,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
   const uint32_t tm_dK = tmem + 128;
   auto tm_S = [&](int buf) { return tmem + 256 + 128 * buf; };
   auto tm_dP = [&](int buf) { return tmem + 256 + 128 * buf + 64; };
-  // step t -> (query head, query block)
-  auto step_bh = [&](int t) { return b * p.Hq + g * p.group + t / nq; };
-  auto step_qt = [&](int t) { return i0 + t % nq; };
 
+  // Reads the n-th work item from the ring (one warp, or the MMA thread
+  // alone with `whole_warp` false); -1 ends the walk, -2 reports an abort.
+  auto sched_read = [&](int n, bool whole_warp, uint32_t role) -> int {
+    const int slot = n % L::kSched;
+    const bool ok = mbar_wait(&sched_full[slot], (n / L::kSched) & 1, abort_flag, kKernBwd, role, 6);
+    if (whole_warp ? !__all_sync(0xffffffffu, ok) : !ok) return -2;
+    const int item = sched_item[slot];
+    if (whole_warp) __syncwarp();
+    if (!whole_warp || lane == 0) mbar_arrive(&sched_empty[slot]);
+    return item;
+  };
+
+  // Steps are numbered across the items a block takes (g); the Q / dO ring
+  // stage is g % kStages, the tensor-memory step buffer g & 1.
   if (warp == 12) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -244,26 +293,52 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
       prefetch_tensormap(&p.tm_do);
       prefetch_tensormap(&p.tm_k);
       prefetch_tensormap(&p.tm_v);
-      mbar_expect_tx(kv_full, 2 * L::kKVTile);
-      for (int c = 0; c < L::kChunks; ++c) {
-        tma_load_3d(sK + c * L::kKVBox, &p.tm_k, kv_full, c * 64, kv0, kvh);
-        tma_load_3d(sV + c * L::kKVBox, &p.tm_v, kv_full, c * 64, kv0, kvh);
-      }
-      for (int t = 0; t < T_steps; ++t) {
-        const int s = t % L::kStages;
-        if (t >= L::kStages &&
-            !mbar_wait(&step_done[s], ((t / L::kStages) - 1) & 1, abort_flag, kKernBwd, 12, 0))
+      int gt = 0;
+      for (int n = 0;; ++n) {
+        const int slot = n % L::kSched;
+        if (n >= L::kSched &&
+            !mbar_wait(&sched_empty[slot], ((n / L::kSched) - 1) & 1, abort_flag, kKernBwd, 12, 1))
           break;
-        const int bh = step_bh(t), qt = step_qt(t);
-        mbar_expect_tx(&q_full[s], 2 * L::kQTile + 512);
+        int item = static_cast<int>(atomicAdd(p.work_counter, 1u));
+        if (item >= p.n_items) item = -1;
+        sched_item[slot] = item;
+        mbar_arrive(&sched_full[slot]);
+        if (item < 0) break;
+        const BwdItem it = bwd_item<CAUSAL>(p, item);
+        auto load_step = [&](int t) -> bool {
+          const int g = gt + t, s = g % L::kStages;
+          if (g >= L::kStages &&
+              !mbar_wait(&step_done[s], ((g / L::kStages) - 1) & 1, abort_flag, kKernBwd, 12, 0))
+            return false;
+          const int bh = it.bh0 + t / it.nq, qt = it.i0 + t % it.nq;
+          mbar_expect_tx(&q_full[s], 2 * L::kQTile + 512);
+          for (int c = 0; c < L::kChunks; ++c) {
+            tma_load_3d(sQ + s * L::kQTile + c * L::kQBox, &p.tm_q, &q_full[s], c * 64, qt * 64, bh);
+            tma_load_3d(sDO + s * L::kQTile + c * L::kQBox, &p.tm_do, &q_full[s], c * 64, qt * 64,
+                        bh);
+          }
+          const int64_t row0 = static_cast<int64_t>(bh) * p.Np + qt * 64;
+          bulk_load(sLse + s * 64, p.lse2 + row0, 256, &q_full[s]);
+          bulk_load(sD + s * 64, p.Dvec + row0, 256, &q_full[s]);
+          return true;
+        };
+        // Q / dO of the first steps may land while the previous item is
+        // still running; K and V only once its MMAs (the last readers of
+        // sK and sV) have completed.
+        const int early = it.T < L::kStages ? it.T : L::kStages;
+        bool ok = true;
+        int t = 0;
+        for (; ok && t < early; ++t) ok = load_step(t);
+        if (ok && n > 0) ok = mbar_wait(acc_done, (n - 1) & 1, abort_flag, kKernBwd, 12, 2);
+        if (!ok) break;
+        mbar_expect_tx(kv_full, 2 * L::kKVTile);
         for (int c = 0; c < L::kChunks; ++c) {
-          tma_load_3d(sQ + s * L::kQTile + c * L::kQBox, &p.tm_q, &q_full[s], c * 64, qt * 64, bh);
-          tma_load_3d(sDO + s * L::kQTile + c * L::kQBox, &p.tm_do, &q_full[s], c * 64, qt * 64,
-                      bh);
+          tma_load_3d(sK + c * L::kKVBox, &p.tm_k, kv_full, c * 64, it.kv0, it.kvh);
+          tma_load_3d(sV + c * L::kKVBox, &p.tm_v, kv_full, c * 64, it.kv0, it.kvh);
         }
-        const int64_t row0 = static_cast<int64_t>(bh) * p.Np + qt * 64;
-        bulk_load(sLse + s * 64, p.lse2 + row0, 256, &q_full[s]);
-        bulk_load(sD + s * 64, p.Dvec + row0, 256, &q_full[s]);
+        for (; ok && t < it.T; ++t) ok = load_step(t);
+        if (!ok) break;
+        gt += it.T;
       }
     }
   } else if (warp == 13) {
@@ -273,149 +348,199 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
       constexpr uint32_t kIdDQ = idesc_f16(BF16, 128, 64, true, true);     // dQ^T = K^T dS^T
       constexpr uint32_t kIdAcc = idesc_f16(BF16, 128, HD, false, true);   // dV, dK
       const uint32_t kb = smem_u32(sK), vb = smem_u32(sV), dsb = smem_u32(sDS);
-      bool ok = mbar_wait(kv_full, 0, abort_flag, kKernBwd, 13, 0);
-      tc_fence_after();
-      auto issue_s = [&](int t) -> bool {
-        const int s = t % L::kStages;
-        if (!mbar_wait(&q_full[s], (t / L::kStages) & 1, abort_flag, kKernBwd, 13, 1)) return false;
+      auto issue_s = [&](int g) -> bool {
+        const int s = g % L::kStages;
+        if (!mbar_wait(&q_full[s], (g / L::kStages) & 1, abort_flag, kKernBwd, 13, 1)) return false;
         tc_fence_after();
         const uint32_t qb = smem_u32(sQ + s * L::kQTile);
 #pragma unroll
         for (int k = 0; k < HD / 16; ++k)
-          umma_ss(tm_S(t & 1),
+          umma_ss(tm_S(g & 1),
                   sdesc_sw128(kb + (k >> 2) * L::kKVBox + (k & 3) * 32, 16, 1024),
                   sdesc_sw128(qb + (k >> 2) * L::kQBox + (k & 3) * 32, 16, 1024), kIdS, k > 0);
         return true;
       };
-      auto issue_dp = [&](int t) {
-        const int s = t % L::kStages;
+      auto issue_dp = [&](int g) {
+        const int s = g % L::kStages;
         const uint32_t ob = smem_u32(sDO + s * L::kQTile);
 #pragma unroll
         for (int k = 0; k < HD / 16; ++k)
-          umma_ss(tm_dP(t & 1),
+          umma_ss(tm_dP(g & 1),
                   sdesc_sw128(vb + (k >> 2) * L::kKVBox + (k & 3) * 32, 16, 1024),
                   sdesc_sw128(ob + (k >> 2) * L::kQBox + (k & 3) * 32, 16, 1024), kIdS, k > 0);
-        umma_commit(&sdp_full[t & 1]);
+        umma_commit(&sdp_full[g & 1]);
       };
-      for (int t = 0; ok && t < 2 && t < T_steps; ++t) {
-        ok = issue_s(t);
-        if (ok) issue_dp(t);
-      }
-      for (int t = 0; ok && t < T_steps; ++t) {
-        const int buf = t & 1, s = t % L::kStages;
-        if (!mbar_wait(&ds_full[buf], (t >> 1) & 1, abort_flag, kKernBwd, 13, 2)) break;
+      int gt = 0;
+      bool ok = true;
+      for (int n = 0; ok; ++n) {
+        const int item = sched_read(n, false, 13);
+        if (item < 0) break;
+        const BwdItem it = bwd_item<CAUSAL>(p, item);
+        if (!mbar_wait(kv_full, n & 1, abort_flag, kKernBwd, 13, 0)) break;
         tc_fence_after();
-        const uint32_t qb = smem_u32(sQ + s * L::kQTile);
-        const uint32_t ob = smem_u32(sDO + s * L::kQTile);
-        const uint32_t db = dsb + buf * L::kDsBytes;
-        // dQ^T (d x 64) = K^T dS^T over the 128 keys, into the dP^T columns.
-        // K^T is K read MN-major; its second 64-feature half sits kKVBox bytes
-        // further (for d = 64 that is V: rows 64..127 of the product are
-        // unused).
-#pragma unroll
-        for (int k = 0; k < 8; ++k)
-          umma_ss(tm_dP(buf), sdesc_sw128(kb + k * 2048, L::kKVBox, 1024),
-                  sdesc_sw128(db + k * 2048, 8192, 1024), kIdDQ, k > 0);
-        umma_commit(&dq_full[buf]);
-        // dV += P^T dO: P^T from tensor memory (each 32-query half of it sits
-        // at the start of its own 32-column group), dO read MN-major.
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-          umma_ts(tm_dV, tm_S(buf) + (k >> 1) * 32 + (k & 1) * 8,
-                  sdesc_sw128(ob + k * 2048, L::kQBox, 1024), kIdAcc, (t > 0 || k > 0) ? 1u : 0u);
-        // dK += dS^T Q: dS^T K-major from shared memory, Q read MN-major.
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-          umma_ss(tm_dK, sdesc_sw128(db + k * 32, 16, 1024),
-                  sdesc_sw128(qb + k * 2048, L::kQBox, 1024), kIdAcc, (t > 0 || k > 0) ? 1u : 0u);
-        umma_commit(&step_done[s]);
-        if (t + 2 < T_steps) {
-          // S^T_{t+2} overwrites P^T_t, which dV_t (issued just before by this
-          // thread) reads: the tensor core runs one thread's MMAs in issue
-          // order, reading an MMA's operands before a later MMA writes its
-          // result, so no wait is needed (a wait for an MMA's completion
-          // costs several hundred idle tensor-core cycles on B200).
-          // dP^T_{t+2} overwrites dQ^T_t: wait for the drain warps to read it.
-          if (!issue_s(t + 2)) break;
-          if (!mbar_wait(&dq_drained[buf], (t >> 1) & 1, abort_flag, kKernBwd, 13, 4)) break;
-          tc_fence_after();
-          issue_dp(t + 2);
+        // S^T, dP^T of the item's first two steps.  dP^T of step g lands on
+        // the columns that held dQ^T of step g-2 (the previous item's): wait
+        // for its drain.
+        for (int t = 0; ok && t < 2 && t < it.T; ++t) {
+          const int g = gt + t;
+          ok = issue_s(g);
+          if (ok && g >= 2) {
+            ok = mbar_wait(&dq_drained[g & 1], ((g - 2) >> 1) & 1, abort_flag, kKernBwd, 13, 4);
+            tc_fence_after();
+          }
+          if (ok) issue_dp(g);
         }
+        for (int t = 0; ok && t < it.T; ++t) {
+          const int g = gt + t, buf = g & 1, s = g % L::kStages;
+          if (!mbar_wait(&ds_full[buf], (g >> 1) & 1, abort_flag, kKernBwd, 13, 2)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t qb = smem_u32(sQ + s * L::kQTile);
+          const uint32_t ob = smem_u32(sDO + s * L::kQTile);
+          const uint32_t db = dsb + buf * L::kDsBytes;
+          // dQ^T (d x 64) = K^T dS^T over the 128 keys, into the dP^T columns.
+          // K^T is K read MN-major; its second 64-feature half sits kKVBox
+          // bytes further (for d = 64 that is V: rows 64..127 of the product
+          // are unused).
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            umma_ss(tm_dP(buf), sdesc_sw128(kb + k * 2048, L::kKVBox, 1024),
+                    sdesc_sw128(db + k * 2048, 8192, 1024), kIdDQ, k > 0);
+          umma_commit(&dq_full[buf]);
+          if (t == 0 && n > 0) {
+            // this item's dV, dK start afresh in the accumulators that the
+            // epilogue of the previous item reads
+            if (!mbar_wait(acc_free, (n - 1) & 1, abort_flag, kKernBwd, 13, 7)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+          }
+          // dV += P^T dO: P^T from tensor memory (each 32-query half of it
+          // sits at the start of its own 32-column group), dO read MN-major.
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            umma_ts(tm_dV, tm_S(buf) + (k >> 1) * 32 + (k & 1) * 8,
+                    sdesc_sw128(ob + k * 2048, L::kQBox, 1024), kIdAcc, (t > 0 || k > 0) ? 1u : 0u);
+          // dK += dS^T Q: dS^T K-major from shared memory, Q read MN-major.
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            umma_ss(tm_dK, sdesc_sw128(db + k * 32, 16, 1024),
+                    sdesc_sw128(qb + k * 2048, L::kQBox, 1024), kIdAcc, (t > 0 || k > 0) ? 1u : 0u);
+          umma_commit(&step_done[s]);
+          if (t + 2 < it.T) {
+            // S^T_{g+2} overwrites P^T_g, which dV_g (issued just before by
+            // this thread) reads: the tensor core runs one thread's MMAs in
+            // issue order, reading an MMA's operands before a later MMA
+            // writes its result, so no wait is needed (a wait for an MMA's
+            // completion costs several hundred idle tensor-core cycles on
+            // B200).  dP^T_{g+2} overwrites dQ^T_g: wait for the drain warps
+            // to read it.
+            if (!issue_s(g + 2)) {
+              ok = false;
+              break;
+            }
+            if (!mbar_wait(&dq_drained[buf], (g >> 1) & 1, abort_flag, kKernBwd, 13, 4)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_dp(g + 2);
+          }
+        }
+        if (!ok) break;
+        umma_commit(acc_done);
+        gt += it.T;
       }
-      umma_commit(acc_done);
+      // every MMA this thread issued completes before tensor memory is freed
       umma_commit(done_bar);
-      mbar_wait(done_bar, 0, abort_flag, kKernBwd, 13, 5);
+      mbar_wait_drain(done_bar, 0, kKernBwd, 13, 5);
     }
   } else if (warp < 8) {
     // ------------------------------------------------------------ softmax gradient
     const int quarter = warp & 3, half = warp >> 2;
     const int r = quarter * 32 + lane;                 // key row within the block
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    const int kv_row = kv0 + r;
-    const bool row_valid = kv_row < p.N;
     const float c_log2 = p.scale_log2;
-    for (int t = 0; t < T_steps; ++t) {
-      const int buf = t & 1, s = t % L::kStages;
-      const int q_first = step_qt(t) * 64 + half * 32;  // first query of this thread's columns
-      if (!__all_sync(0xffffffffu, mbar_wait(&sdp_full[buf], (t >> 1) & 1, abort_flag, kKernBwd, 0, 0)))
-        break;
-      tc_fence_after();
-      uint32_t v[32];
-      tmem_ld32(tm_S(buf) + lane_off + half * 32, v);
-      const float4* lse4 = reinterpret_cast<const float4*>(sLse + s * 64 + half * 32);
-      float pr[32];
-      tmem_ld_wait();
+    int gt = 0;
+    for (int n = 0;; ++n) {
+      const int item = sched_read(n, true, 0);
+      if (item < 0) break;
+      const BwdItem it = bwd_item<CAUSAL>(p, item);
+      const int kv_row = it.kv0 + r;
+      const bool row_valid = kv_row < p.N;
+      bool ok = true;
+      for (int t = 0; t < it.T; ++t) {
+        const int g = gt + t, buf = g & 1, s = g % L::kStages;
+        const int q_first = (it.i0 + t % it.nq) * 64 + half * 32;  // first query of this thread's columns
+        if (!__all_sync(0xffffffffu, mbar_wait(&sdp_full[buf], (g >> 1) & 1, abort_flag, kKernBwd, 0, 0))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint32_t v[32];
+        tmem_ld32(tm_S(buf) + lane_off + half * 32, v);
+        const float4* lse4 = reinterpret_cast<const float4*>(sLse + s * 64 + half * 32);
+        float pr[32];
+        tmem_ld_wait();
 #pragma unroll
-      for (int c4 = 0; c4 < 8; ++c4) {
-        const float4 l4 = lse4[c4];
-        pr[4 * c4 + 0] = ex2_approx(fmaf(__uint_as_float(v[4 * c4 + 0]), c_log2, -l4.x));
-        pr[4 * c4 + 1] = ex2_approx(fmaf(__uint_as_float(v[4 * c4 + 1]), c_log2, -l4.y));
-        pr[4 * c4 + 2] = ex2_approx(fmaf(__uint_as_float(v[4 * c4 + 2]), c_log2, -l4.z));
-        pr[4 * c4 + 3] = ex2_approx(fmaf(__uint_as_float(v[4 * c4 + 3]), c_log2, -l4.w));
+        for (int c4 = 0; c4 < 8; ++c4) {
+          const float4 l4 = lse4[c4];
+          pr[4 * c4 + 0] = ex2_approx(fmaf(__uint_as_float(v[4 * c4 + 0]), c_log2, -l4.x));
+          pr[4 * c4 + 1] = ex2_approx(fmaf(__uint_as_float(v[4 * c4 + 1]), c_log2, -l4.y));
+          pr[4 * c4 + 2] = ex2_approx(fmaf(__uint_as_float(v[4 * c4 + 2]), c_log2, -l4.z));
+          pr[4 * c4 + 3] = ex2_approx(fmaf(__uint_as_float(v[4 * c4 + 3]), c_log2, -l4.w));
+        }
+        // causal: key kv_row is hidden from queries before it; padding keys
+        // (kv_row >= N) carry no probability
+        if (!row_valid) {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) pr[c] = 0.f;
+        } else if (CAUSAL && q_first < kv_row) {
+#pragma unroll
+          for (int c = 0; c < 32; ++c)
+            if (q_first + c < kv_row) pr[c] = 0.f;
+        }
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) pk[i] = pack2<BF16>(pr[2 * i], pr[2 * i + 1]);
+        tmem_st16(tm_S(buf) + lane_off + half * 32, pk);
+        tmem_ld32(tm_dP(buf) + lane_off + half * 32, v);
+        const float4* d4 = reinterpret_cast<const float4*>(sD + s * 64 + half * 32);
+        tmem_ld_wait();
+#pragma unroll
+        for (int c4 = 0; c4 < 8; ++c4) {
+          const float4 dd = d4[c4];
+          pr[4 * c4 + 0] *= __uint_as_float(v[4 * c4 + 0]) - dd.x;
+          pr[4 * c4 + 1] *= __uint_as_float(v[4 * c4 + 1]) - dd.y;
+          pr[4 * c4 + 2] *= __uint_as_float(v[4 * c4 + 2]) - dd.z;
+          pr[4 * c4 + 3] *= __uint_as_float(v[4 * c4 + 3]) - dd.w;
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i) pk[i] = pack2<BF16>(pr[2 * i], pr[2 * i + 1]);
+        // dS^T buffer `buf` is free once step g-2 (dK_{g-2} its last reader) is done
+        if (g >= 2 && !__all_sync(0xffffffffu, mbar_wait(&step_done[(g - 2) % L::kStages],
+                                                         ((g - 2) / L::kStages) & 1, abort_flag,
+                                                         kKernBwd, 0, 2))) {
+          ok = false;
+          break;
+        }
+        uint8_t* row_base = sDS + buf * L::kDsBytes + r * 128;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int chunk = (half * 4 + u) ^ (r & 7);
+          *reinterpret_cast<uint4*>(row_base + chunk * 16) =
+              make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+        }
+        fence_proxy_async_smem();
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&ds_full[buf]);
       }
-      // causal: key kv_row is hidden from queries before it; padding keys
-      // (kv_row >= N) carry no probability
-      if (!row_valid) {
-#pragma unroll
-        for (int c = 0; c < 32; ++c) pr[c] = 0.f;
-      } else if (CAUSAL && q_first < kv_row) {
-#pragma unroll
-        for (int c = 0; c < 32; ++c)
-          if (q_first + c < kv_row) pr[c] = 0.f;
-      }
-      uint32_t pk[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) pk[i] = pack2<BF16>(pr[2 * i], pr[2 * i + 1]);
-      tmem_st16(tm_S(buf) + lane_off + half * 32, pk);
-      tmem_ld32(tm_dP(buf) + lane_off + half * 32, v);
-      const float4* d4 = reinterpret_cast<const float4*>(sD + s * 64 + half * 32);
-      tmem_ld_wait();
-#pragma unroll
-      for (int c4 = 0; c4 < 8; ++c4) {
-        const float4 dd = d4[c4];
-        pr[4 * c4 + 0] *= __uint_as_float(v[4 * c4 + 0]) - dd.x;
-        pr[4 * c4 + 1] *= __uint_as_float(v[4 * c4 + 1]) - dd.y;
-        pr[4 * c4 + 2] *= __uint_as_float(v[4 * c4 + 2]) - dd.z;
-        pr[4 * c4 + 3] *= __uint_as_float(v[4 * c4 + 3]) - dd.w;
-      }
-#pragma unroll
-      for (int i = 0; i < 16; ++i) pk[i] = pack2<BF16>(pr[2 * i], pr[2 * i + 1]);
-      // dS^T buffer `buf` is free once step t-2 (dK_{t-2} its last reader) is done
-      if (t >= 2 && !__all_sync(0xffffffffu, mbar_wait(&step_done[(t - 2) % L::kStages],
-                                                       ((t - 2) / L::kStages) & 1, abort_flag,
-                                                       kKernBwd, 0, 2)))
-        break;
-      uint8_t* row_base = sDS + buf * L::kDsBytes + r * 128;
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int chunk = (half * 4 + u) ^ (r & 7);
-        *reinterpret_cast<uint4*>(row_base + chunk * 16) =
-            make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
-      }
-      fence_proxy_async_smem();
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(&ds_full[buf]);
+      if (!ok) break;
+      gt += it.T;
     }
   } else {
     // ------------------------------------------------------------ dQ drain, dK/dV epilogue
@@ -426,30 +551,40 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
     const int dw = warp - 8;                           // 0..3 == lane quarter
     const uint32_t lane_off = static_cast<uint32_t>(dw * 32) << 16;
     const bool drains = dw * 32 < HD;                  // warp holds real dQ^T rows
-    for (int t = 0; drains && t < T_steps; ++t) {
-      const int buf = t & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(&dq_full[buf], (t >> 1) & 1, abort_flag, kKernBwd, 8, 0)))
-        break;
-      tc_fence_after();
-      uint32_t v0[32], v1[32];
-      tmem_ld32(tm_dP(buf) + lane_off, v0);
-      tmem_ld32(tm_dP(buf) + lane_off + 32, v1);
-      tmem_ld_wait();
-      tc_fence_before();
-      mbar_arrive(&dq_drained[buf]);
-      const int bh = step_bh(t), qt = step_qt(t);
-      float* dst = p.dqacc + (static_cast<size_t>(bh) * p.Np + qt * 64) * HD + dw * 32 + lane;
+    int gt = 0;
+    for (int n = 0;; ++n) {
+      const int item = sched_read(n, true, 8);
+      if (item < 0) break;
+      const BwdItem it = bwd_item<CAUSAL>(p, item);
+      bool ok = true;
+      for (int t = 0; drains && t < it.T; ++t) {
+        const int g = gt + t, buf = g & 1;
+        if (!__all_sync(0xffffffffu, mbar_wait(&dq_full[buf], (g >> 1) & 1, abort_flag, kKernBwd, 8, 0))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint32_t v0[32], v1[32];
+        tmem_ld32(tm_dP(buf) + lane_off, v0);
+        tmem_ld32(tm_dP(buf) + lane_off + 32, v1);
+        tmem_ld_wait();
+        tc_fence_before();
+        mbar_arrive(&dq_drained[buf]);
+        const int bh = it.bh0 + t / it.nq, qt = it.i0 + t % it.nq;
+        float* dst = p.dqacc + (static_cast<size_t>(bh) * p.Np + qt * 64) * HD + dw * 32 + lane;
 #pragma unroll
-      for (int q = 0; q < 32; ++q) atomicAdd(dst + q * HD, __uint_as_float(v0[q]));
+        for (int q = 0; q < 32; ++q) atomicAdd(dst + q * HD, __uint_as_float(v0[q]));
 #pragma unroll
-      for (int q = 0; q < 32; ++q) atomicAdd(dst + (32 + q) * HD, __uint_as_float(v1[q]));
-    }
-    // epilogue: dV, dK (times scale) rows -> I/O dtype, written once
-    if (__all_sync(0xffffffffu, mbar_wait(acc_done, 0, abort_flag, kKernBwd, 8, 1))) {
+        for (int q = 0; q < 32; ++q) atomicAdd(dst + (32 + q) * HD, __uint_as_float(v1[q]));
+      }
+      if (!ok) break;
+      gt += it.T;
+      // epilogue: dV, dK (times scale) rows -> I/O dtype, written once
+      if (!__all_sync(0xffffffffu, mbar_wait(acc_done, n & 1, abort_flag, kKernBwd, 8, 1))) break;
       tc_fence_after();
       const int r = dw * 32 + lane;
-      const int kv_row = kv0 + r;
-      const size_t row_off = (static_cast<size_t>(kvh) * p.N + kv_row) * HD;
+      const int kv_row = it.kv0 + r;
+      const size_t row_off = (static_cast<size_t>(it.kvh) * p.N + kv_row) * HD;
 #pragma unroll
       for (int which = 0; which < 2; ++which) {
         const uint32_t src = (which ? tm_dK : tm_dV) + lane_off;
@@ -473,6 +608,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
           }
         }
       }
+      tc_fence_before();
+      mbar_arrive(acc_free);
     }
   }
 

@@ -112,6 +112,23 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// For a thread that must see its own asynchronous work complete before the
+// block frees what that work touches (tensor memory): waits regardless of the
+// abort flag, still at most g_wait_limit_ns.
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, uint32_t kernel,
+                                                uint32_t role, uint32_t site) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  const uint64_t limit = g_wait_limit_ns;
+  for (;;) {
+    if (mbar_try_wait_sleep(bar, parity, 200000u)) return true;
+    if (globaltimer_ns() - t0 > limit) {
+      record_error(kStatusTimeout, kernel, role, site);
+      return false;
+    }
+  }
+}
+
 // ----------------------------------------------------------------------------
 // TMA (tensor-map) and bulk copies
 

@@ -79,7 +79,8 @@ fa_status_t fa_fwd(const void* q, const void* k, const void* v, void* o, float* 
  * Bytes of device scratch that fa_bwd needs for these sizes (0 for an empty
  * problem).  Linear in N: two fp32 values per query row (D_i = dO_i . O_i and
  * the logsumexp in base 2) plus an fp32 dQ accumulator [B][Hq][Np][d], with N
- * rounded up to a multiple of 128 (Np).
+ * rounded up to a multiple of 128 (Np), plus 256 bytes (the main pass's
+ * work-item counter).
  */
 size_t fa_bwd_workspace_bytes(int B, int Hq, int Hkv, int N, int d);
 
@@ -90,9 +91,10 @@ size_t fa_bwd_workspace_bytes(int B, int Hq, int Hkv, int N, int d);
  * caller-owned device memory of at least fa_bwd_workspace_bytes(...) bytes,
  * 16-byte aligned; its contents on entry do not matter and on exit are
  * unspecified.  Three kernels run on `stream` in order: a row pass (D and the
- * zeroed dQ accumulator), the main pass (one thread block per key block of
- * 128 rows and key/value head: dK, dV in tensor memory, dQ added into the
- * accumulator), and a pass that scales and converts dQ.
+ * zeroed dQ accumulator), the main pass (persistent, one thread block per
+ * SM, each taking work items = (key block of 128 rows, key/value head) in
+ * turn: dK, dV in tensor memory, dQ added into the accumulator), and a pass
+ * that scales and converts dQ.
  */
 fa_status_t fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
                    const float* lse, void* dq, void* dk, void* dv,
@@ -133,6 +135,16 @@ fa_status_t fa_selftest_wait_timeout(uint64_t limit_ns, void* stream);
  * calls: set it only from the thread that launches.
  */
 fa_status_t fa_set_profile_events(int kernel_id, void* start, void* stop);
+
+/*
+ * Caps the number of thread blocks of fa_bwd's main pass, which otherwise
+ * runs one persistent block per SM; each block then takes more work items in
+ * turn.  0 restores the default.  Results do not depend on the cap (beyond
+ * the order of the fp32 dQ additions); it exists to exercise and measure the
+ * hand-over between work items on small problems.  Process-wide; negative
+ * values return FA_ERR_INVALID_ARG.
+ */
+fa_status_t fa_set_bwd_max_blocks(int max_blocks);
 
 /*
  * Backward pass for callers that cannot allocate device memory.

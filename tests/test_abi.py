@@ -103,11 +103,20 @@ def test_empty_problems_are_no_ops(lib):
 
 
 def test_workspace_is_linear_in_n():
-    # two fp32 row statistics + an fp32 dQ accumulator per (padded) query row
+    # two fp32 row statistics + an fp32 dQ accumulator per (padded) query row,
+    # plus a fixed 256-byte tail (the main pass's work-item counter)
+    tail = 256
     for d in (64, 128):
-        sizes = [binding.fa_bwd_workspace_bytes(1, 16, 16, n, d) for n in (4096, 8192, 16384, 32768, 65536)]
+        sizes = [binding.fa_bwd_workspace_bytes(1, 16, 16, n, d) - tail
+                 for n in (4096, 8192, 16384, 32768, 65536)]
         for a, b in zip(sizes, sizes[1:]):
             assert b == 2 * a
         assert sizes[0] == 16 * 4096 * 4 * (2 + d)
     # padding to a multiple of 128 rows
-    assert binding.fa_bwd_workspace_bytes(1, 1, 1, 129, 64) == 256 * 4 * 66
+    assert binding.fa_bwd_workspace_bytes(1, 1, 1, 129, 64) == 256 * 4 * 66 + tail
+
+
+def test_bwd_max_blocks_setting(lib):
+    assert lib.fa_set_bwd_max_blocks(-1) == binding.FA_ERR_INVALID_ARG
+    assert lib.fa_set_bwd_max_blocks(3) == binding.FA_OK
+    assert lib.fa_set_bwd_max_blocks(0) == binding.FA_OK

@@ -59,6 +59,32 @@ def test_parity_full(shape, dtype, causal):
     print(shape, dtype, causal, rep)
 
 
+PERSISTENT_CASES = [
+    # (B, Hq, Hkv, N, d), dtype, causal, blocks: few persistent blocks, so each
+    # takes many work items in turn, including causal items of a single step
+    ((2, 3, 3, 130, 64), torch.bfloat16, True, 1),
+    ((2, 3, 3, 130, 64), torch.float16, False, 2),
+    ((1, 8, 2, 333, 128), torch.bfloat16, True, 1),
+    ((1, 8, 2, 333, 128), torch.bfloat16, True, 3),
+    ((2, 4, 4, 640, 128), torch.float16, True, 5),
+    ((1, 6, 1, 260, 128), torch.bfloat16, False, 2),
+]
+
+
+@pytest.mark.parametrize("shape,dtype,causal,blocks", PERSISTENT_CASES,
+                         ids=[f"{'x'.join(map(str, s))}-{str(t)[6:]}-{'c' if c else 'nc'}-b{n}"
+                              for s, t, c, n in PERSISTENT_CASES])
+def test_parity_persistent_handover(shape, dtype, causal, blocks):
+    q, k, v, do = _inputs(shape, dtype, seed=3 * sum(shape) + blocks)
+    scale = 1.0 / math.sqrt(shape[-1])
+    binding.fa_set_bwd_max_blocks(blocks)
+    try:
+        out = ac.run_gpu(q, k, v, do, scale, causal)
+    finally:
+        binding.fa_set_bwd_max_blocks(0)
+    ac.check_full(q, k, v, do, scale, causal, out)
+
+
 def test_parity_wide_logits_fp16():
     # the fp16 recipe with Q, K ~ N(0, 3^2): the running max moves many times
     q, k, v, do = _inputs((1, 2, 2, 640, 128), torch.float16, seed=99, sigma_qk=3.0)
