@@ -47,7 +47,8 @@
 //               item, the dK / dV epilogue (lane = key row).
 //   warp 12     TMA producer; it also claims the work items and passes them
 //               to the other roles through a small ring in shared memory.
-//   warp 13     MMA issuer (one thread).
+//   warp 13     MMA issuer (the whole warp runs the loop, one elected lane
+//               issues).
 // Tensor memory: dV [0,128), dK [128,256), and two step buffers b = 0, 1:
 // S^T at 256+128b (64 columns; P^T is written over it as 16-bit pairs, each
 // warp half over its own columns) and dP^T at 256+128b+64 (dQ^T is written
@@ -235,7 +236,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
     return;
   }
   constexpr int kDrainThreads = HD == 128 ? 128 : 64;
-  constexpr int kSchedReaders = 1 + 8 + 4;  // MMA thread, softmax warps, drain warps
+  constexpr int kSchedReaders = 1 + 8 + 4;  // MMA warp, softmax warps, drain warps
 
   if (tid == 0) {
     mbar_init(kv_full, 1);
@@ -272,8 +273,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
   auto tm_S = [&](int buf) { return tmem + 256 + 128 * buf; };
   auto tm_dP = [&](int buf) { return tmem + 256 + 128 * buf + 64; };
 
-  // Reads the n-th work item from the ring (one warp, or the MMA thread
-  // alone with `whole_warp` false); -1 ends the walk, -2 reports an abort.
+  // Reads the n-th work item from the ring (a whole warp, or one thread with
+  // `whole_warp` false); -1 ends the walk, -2 reports an abort.
   auto sched_read = [&](int n, bool whole_warp, uint32_t role) -> int {
     const int slot = n % L::kSched;
     const bool ok = mbar_wait(&sched_full[slot], (n / L::kSched) & 1, abort_flag, kKernBwd, role, 6);
@@ -343,121 +344,129 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
     }
   } else if (warp == 13) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t kIdS = idesc_f16(BF16, 128, 64, false, false);    // S^T, dP^T
-      constexpr uint32_t kIdDQ = idesc_f16(BF16, 128, 64, true, true);     // dQ^T = K^T dS^T
-      constexpr uint32_t kIdAcc = idesc_f16(BF16, 128, HD, false, true);   // dV, dK
-      const uint32_t kb = smem_u32(sK), vb = smem_u32(sV), dsb = smem_u32(sDS);
-      auto issue_s = [&](int g) -> bool {
-        const int s = g % L::kStages;
-        if (!mbar_wait(&q_full[s], (g / L::kStages) & 1, abort_flag, kKernBwd, 13, 1)) return false;
-        tc_fence_after();
-        const uint32_t qb = smem_u32(sQ + s * L::kQTile);
+    // The whole warp runs this loop with warp-uniform values; one elected
+    // lane issues each MMA and commit.  Descriptors are formed once and
+    // moved by constant offsets.
+    constexpr uint32_t kIdS = idesc_f16(BF16, 128, 64, false, false);    // S^T, dP^T
+    constexpr uint32_t kIdDQ = idesc_f16(BF16, 128, 64, true, true);     // dQ^T = K^T dS^T
+    constexpr uint32_t kIdAcc = idesc_f16(BF16, 128, HD, false, true);   // dV, dK
+    const uint32_t dsb = smem_u32(sDS);
+    const uint64_t dK_k = sdesc_sw128(smem_u32(sK), 16, 1024);           // K, K-major
+    const uint64_t dV_k = sdesc_sw128(smem_u32(sV), 16, 1024);           // V, K-major
+    const uint64_t dK_mn = sdesc_sw128(smem_u32(sK), L::kKVBox, 1024);   // K^T, MN-major
+    const uint64_t dQ_k = sdesc_sw128(smem_u32(sQ), 16, 1024);           // Q stage 0, K-major
+    const uint64_t dQ_mn = sdesc_sw128(smem_u32(sQ), L::kQBox, 1024);    // Q stage 0, MN-major
+    const uint64_t dO_k = sdesc_sw128(smem_u32(sDO), 16, 1024);
+    const uint64_t dO_mn = sdesc_sw128(smem_u32(sDO), L::kQBox, 1024);
+    const uint64_t dS_mn = sdesc_sw128(dsb, 8192, 1024);                 // dS^T buffer 0, MN-major
+    const uint64_t dS_k = sdesc_sw128(dsb, 16, 1024);                    // dS^T buffer 0, K-major
+    auto wait_all = [&](uint64_t* bar, uint32_t parity, uint32_t site) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, kKernBwd, 13, site));
+    };
+    auto issue_s = [&](int g) -> bool {
+      const int s = g % L::kStages;
+      if (!wait_all(&q_full[s], (g / L::kStages) & 1, 1)) return false;
+      tc_fence_after();
+      const uint32_t qs = s * L::kQTile;
 #pragma unroll
-        for (int k = 0; k < HD / 16; ++k)
-          umma_ss(tm_S(g & 1),
-                  sdesc_sw128(kb + (k >> 2) * L::kKVBox + (k & 3) * 32, 16, 1024),
-                  sdesc_sw128(qb + (k >> 2) * L::kQBox + (k & 3) * 32, 16, 1024), kIdS, k > 0);
-        return true;
-      };
-      auto issue_dp = [&](int g) {
-        const int s = g % L::kStages;
-        const uint32_t ob = smem_u32(sDO + s * L::kQTile);
+      for (int k = 0; k < HD / 16; ++k)
+        umma_ss_w(tm_S(g & 1), sdesc_add(dK_k, (k >> 2) * L::kKVBox + (k & 3) * 32),
+                  sdesc_add(dQ_k, qs + (k >> 2) * L::kQBox + (k & 3) * 32), kIdS, k > 0);
+      return true;
+    };
+    auto issue_dp = [&](int g) {
+      const uint32_t os = (g % L::kStages) * L::kQTile;
 #pragma unroll
-        for (int k = 0; k < HD / 16; ++k)
-          umma_ss(tm_dP(g & 1),
-                  sdesc_sw128(vb + (k >> 2) * L::kKVBox + (k & 3) * 32, 16, 1024),
-                  sdesc_sw128(ob + (k >> 2) * L::kQBox + (k & 3) * 32, 16, 1024), kIdS, k > 0);
-        umma_commit(&sdp_full[g & 1]);
-      };
-      int gt = 0;
-      bool ok = true;
-      for (int n = 0; ok; ++n) {
-        const int item = sched_read(n, false, 13);
-        if (item < 0) break;
-        const BwdItem it = bwd_item<CAUSAL>(p, item);
-        if (!mbar_wait(kv_full, n & 1, abort_flag, kKernBwd, 13, 0)) break;
-        tc_fence_after();
-        // S^T, dP^T of the item's first two steps.  dP^T of step g lands on
-        // the columns that held dQ^T of step g-2 (the previous item's): wait
-        // for its drain.
-        for (int t = 0; ok && t < 2 && t < it.T; ++t) {
-          const int g = gt + t;
-          ok = issue_s(g);
-          if (ok && g >= 2) {
-            ok = mbar_wait(&dq_drained[g & 1], ((g - 2) >> 1) & 1, abort_flag, kKernBwd, 13, 4);
-            tc_fence_after();
-          }
-          if (ok) issue_dp(g);
+      for (int k = 0; k < HD / 16; ++k)
+        umma_ss_w(tm_dP(g & 1), sdesc_add(dV_k, (k >> 2) * L::kKVBox + (k & 3) * 32),
+                  sdesc_add(dO_k, os + (k >> 2) * L::kQBox + (k & 3) * 32), kIdS, k > 0);
+      umma_commit_w(&sdp_full[g & 1]);
+    };
+    int gt = 0;
+    bool ok = true;
+    for (int n = 0; ok; ++n) {
+      const int item = sched_read(n, true, 13);
+      if (item < 0) break;
+      const BwdItem it = bwd_item<CAUSAL>(p, item);
+      if (!wait_all(kv_full, n & 1, 0)) break;
+      tc_fence_after();
+      // S^T, dP^T of the item's first two steps.  dP^T of step g lands on
+      // the columns that held dQ^T of step g-2 (the previous item's): wait
+      // for its drain.
+      for (int t = 0; ok && t < 2 && t < it.T; ++t) {
+        const int g = gt + t;
+        ok = issue_s(g);
+        if (ok && g >= 2) {
+          ok = wait_all(&dq_drained[g & 1], ((g - 2) >> 1) & 1, 4);
+          tc_fence_after();
         }
-        for (int t = 0; ok && t < it.T; ++t) {
-          const int g = gt + t, buf = g & 1, s = g % L::kStages;
-          if (!mbar_wait(&ds_full[buf], (g >> 1) & 1, abort_flag, kKernBwd, 13, 2)) {
+        if (ok) issue_dp(g);
+      }
+      for (int t = 0; ok && t < it.T; ++t) {
+        const int g = gt + t, buf = g & 1, s = g % L::kStages;
+        if (!wait_all(&ds_full[buf], (g >> 1) & 1, 2)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t qs = s * L::kQTile;
+        const uint32_t ds = buf * L::kDsBytes;
+        // dQ^T (d x 64) = K^T dS^T over the 128 keys, into the dP^T columns.
+        // K^T is K read MN-major; its second 64-feature half sits kKVBox
+        // bytes further (for d = 64 that is V: rows 64..127 of the product
+        // are unused).
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          umma_ss_w(tm_dP(buf), sdesc_add(dK_mn, k * 2048), sdesc_add(dS_mn, ds + k * 2048), kIdDQ,
+                    k > 0);
+        umma_commit_w(&dq_full[buf]);
+        if (t == 0 && n > 0) {
+          // this item's dV, dK start afresh in the accumulators that the
+          // epilogue of the previous item reads
+          if (!wait_all(acc_free, (n - 1) & 1, 7)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t qb = smem_u32(sQ + s * L::kQTile);
-          const uint32_t ob = smem_u32(sDO + s * L::kQTile);
-          const uint32_t db = dsb + buf * L::kDsBytes;
-          // dQ^T (d x 64) = K^T dS^T over the 128 keys, into the dP^T columns.
-          // K^T is K read MN-major; its second 64-feature half sits kKVBox
-          // bytes further (for d = 64 that is V: rows 64..127 of the product
-          // are unused).
-#pragma unroll
-          for (int k = 0; k < 8; ++k)
-            umma_ss(tm_dP(buf), sdesc_sw128(kb + k * 2048, L::kKVBox, 1024),
-                    sdesc_sw128(db + k * 2048, 8192, 1024), kIdDQ, k > 0);
-          umma_commit(&dq_full[buf]);
-          if (t == 0 && n > 0) {
-            // this item's dV, dK start afresh in the accumulators that the
-            // epilogue of the previous item reads
-            if (!mbar_wait(acc_free, (n - 1) & 1, abort_flag, kKernBwd, 13, 7)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-          }
-          // dV += P^T dO: P^T from tensor memory (each 32-query half of it
-          // sits at the start of its own 32-column group), dO read MN-major.
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            umma_ts(tm_dV, tm_S(buf) + (k >> 1) * 32 + (k & 1) * 8,
-                    sdesc_sw128(ob + k * 2048, L::kQBox, 1024), kIdAcc, (t > 0 || k > 0) ? 1u : 0u);
-          // dK += dS^T Q: dS^T K-major from shared memory, Q read MN-major.
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            umma_ss(tm_dK, sdesc_sw128(db + k * 32, 16, 1024),
-                    sdesc_sw128(qb + k * 2048, L::kQBox, 1024), kIdAcc, (t > 0 || k > 0) ? 1u : 0u);
-          umma_commit(&step_done[s]);
-          if (t + 2 < it.T) {
-            // S^T_{g+2} overwrites P^T_g, which dV_g (issued just before by
-            // this thread) reads: the tensor core runs one thread's MMAs in
-            // issue order, reading an MMA's operands before a later MMA
-            // writes its result, so no wait is needed (a wait for an MMA's
-            // completion costs several hundred idle tensor-core cycles on
-            // B200).  dP^T_{g+2} overwrites dQ^T_g: wait for the drain warps
-            // to read it.
-            if (!issue_s(g + 2)) {
-              ok = false;
-              break;
-            }
-            if (!mbar_wait(&dq_drained[buf], (g >> 1) & 1, abort_flag, kKernBwd, 13, 4)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            issue_dp(g + 2);
-          }
         }
-        if (!ok) break;
-        umma_commit(acc_done);
-        gt += it.T;
+        // dV += P^T dO: P^T from tensor memory (each 32-query half of it sits
+        // at the start of its own 32-column group), dO read MN-major.
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          umma_ts_w(tm_dV, tm_S(buf) + (k >> 1) * 32 + (k & 1) * 8, sdesc_add(dO_mn, qs + k * 2048),
+                    kIdAcc, (t > 0 || k > 0) ? 1u : 0u);
+        // dK += dS^T Q: dS^T K-major from shared memory, Q read MN-major.
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          umma_ss_w(tm_dK, sdesc_add(dS_k, ds + k * 32), sdesc_add(dQ_mn, qs + k * 2048), kIdAcc,
+                    (t > 0 || k > 0) ? 1u : 0u);
+        umma_commit_w(&step_done[s]);
+        if (t + 2 < it.T) {
+          // S^T_{g+2} overwrites P^T_g, which dV_g (issued just before by
+          // this warp) reads: the tensor core runs one thread's MMAs in issue
+          // order, reading an MMA's operands before a later MMA writes its
+          // result, so no wait is needed (a wait for an MMA's completion
+          // costs several hundred idle tensor-core cycles on B200).
+          // dP^T_{g+2} overwrites dQ^T_g: wait for the drain warps to read it.
+          if (!issue_s(g + 2)) {
+            ok = false;
+            break;
+          }
+          if (!wait_all(&dq_drained[buf], (g >> 1) & 1, 4)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          issue_dp(g + 2);
+        }
       }
-      // every MMA this thread issued completes before tensor memory is freed
-      umma_commit(done_bar);
-      mbar_wait_drain(done_bar, 0, kKernBwd, 13, 5);
+      if (!ok) break;
+      umma_commit_w(acc_done);
+      gt += it.T;
     }
+    // every MMA this warp issued completes before tensor memory is freed
+    umma_commit_w(done_bar);
+    mbar_wait_drain(done_bar, 0, kKernBwd, 13, 5);
   } else if (warp < 8) {
     // ------------------------------------------------------------ softmax gradient
     const int quarter = warp & 3, half = warp >> 2;

@@ -20,7 +20,8 @@
 //              block and tensor-memory lane r.  Reads S_j, masks, scales,
 //              updates (m, l), writes P_j (16-bit) over S_j, rescales O when
 //              needed, and at the end normalises O, stores it (TMA) and lse.
-//   warp 8     MMA issuer (one thread): S_t,j = Q_t K_j^T and O_t += P_t,j V_j
+//   warp 8     MMA issuer (whole warp, one elected lane issues): S_t,j = Q_t K_j^T
+//              and O_t += P_t,j V_j
 //              for t = 0, 1, staggered as S0_j+1, O1 += P1_j V_j, S1_j+1,
 //              O0 += P0_j+1 V_j+1, ... so that one block's softmax overlaps the
 //              other block's products.
@@ -163,80 +164,80 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
     }
   } else if (warp == 8) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t kIdS = idesc_f16(BF16, 128, 128, false, false);
-      constexpr uint32_t kIdPV = idesc_f16(BF16, 128, HD, false, true);
-      const uint32_t q_base = smem_u32(sQ);
-      int n = 0;
-      bool ok = mbar_wait(q_full, 0, abort_flag, kKernFwd, 8, 0);
-      auto take = [&](int& slot) -> bool {
-        slot = n % L::kSlots;
-        if (!mbar_wait(&slot_full[slot], (n / L::kSlots) & 1, abort_flag, kKernFwd, 8, 1))
-          return false;
-        tc_fence_after();
-        ++n;
-        return true;
-      };
-      // Staggered order: S0_0 S1_0 PV0_0 | S0_1 PV1_0 S1_1 PV0_1 | S0_2 PV1_1 ...
-      // so that one block's softmax runs while the tensor cores work on the
-      // other block.  K_j and V_j are taken in load order (K0 V0 K1 V1 ...).
-      // S_t,j+1 is written over the tensor memory that O_t += P_t,j V_j reads
-      // P_t,j from, and is issued right after it by this same thread: the
-      // tensor core runs the MMAs of one thread in issue order, reading an
-      // MMA's operands before a later MMA writes its result, so no wait is
-      // put between them (waiting for an MMA's completion before issuing the
-      // next costs several hundred cycles of idle tensor core on B200).
-      auto issue_s = [&](int t, uint32_t kb) {
-        const uint32_t qb = q_base + t * L::kTileBytes;
+    // The whole warp runs this loop with warp-uniform values; one elected
+    // lane issues each MMA and commit.  Descriptors are formed once and
+    // moved by constant offsets.
+    constexpr uint32_t kIdS = idesc_f16(BF16, 128, 128, false, false);
+    constexpr uint32_t kIdPV = idesc_f16(BF16, 128, HD, false, true);
+    const uint64_t dQ_k = sdesc_sw128(smem_u32(sQ), 16, 1024);           // Q tile 0, K-major
+    const uint64_t dR_k = sdesc_sw128(smem_u32(sRing), 16, 1024);        // ring slot 0, K-major
+    const uint64_t dR_mn = sdesc_sw128(smem_u32(sRing), L::kBoxBytes, 1024);  // ring slot 0, MN-major
+    auto wait_all = [&](uint64_t* bar, uint32_t parity, uint32_t site) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, kKernFwd, 8, site));
+    };
+    int n = 0;
+    bool ok = wait_all(q_full, 0, 0);
+    auto take = [&](int& slot) -> bool {
+      slot = n % L::kSlots;
+      if (!wait_all(&slot_full[slot], (n / L::kSlots) & 1, 1)) return false;
+      tc_fence_after();
+      ++n;
+      return true;
+    };
+    // Staggered order: S0_0 S1_0 PV0_0 | S0_1 PV1_0 S1_1 PV0_1 | S0_2 PV1_1 ...
+    // so that one block's softmax runs while the tensor cores work on the
+    // other block.  K_j and V_j are taken in load order (K0 V0 K1 V1 ...).
+    // S_t,j+1 is written over the tensor memory that O_t += P_t,j V_j reads
+    // P_t,j from, and is issued right after it by this same warp: the tensor
+    // core runs the MMAs of one thread in issue order, reading an MMA's
+    // operands before a later MMA writes its result, so no wait is put
+    // between them (waiting for an MMA's completion before issuing the next
+    // costs several hundred cycles of idle tensor core on B200).
+    auto issue_s = [&](int t, int kslot) {
+      const uint32_t qo = t * L::kTileBytes, ko = kslot * L::kTileBytes;
 #pragma unroll
-        for (int k = 0; k < HD / 16; ++k) {
-          const uint32_t off = (k >> 2) * L::kBoxBytes + (k & 3) * 32;
-          umma_ss(tmem + t * 128, sdesc_sw128(qb + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024),
-                  kIdS, k > 0);
-        }
-        umma_commit(&s_full[t]);
-      };
-      auto issue_pv = [&](int t, int j, uint32_t vb) -> bool {
-        if (!mbar_wait(&p_full[t], j & 1, abort_flag, kKernFwd, 8, 3)) return false;
-        tc_fence_after();
+      for (int k = 0; k < HD / 16; ++k) {
+        const uint32_t off = (k >> 2) * L::kBoxBytes + (k & 3) * 32;
+        umma_ss_w(tmem + t * 128, sdesc_add(dQ_k, qo + off), sdesc_add(dR_k, ko + off), kIdS, k > 0);
+      }
+      umma_commit_w(&s_full[t]);
+    };
+    auto issue_pv = [&](int t, int j, int vslot) -> bool {
+      if (!wait_all(&p_full[t], j & 1, 3)) return false;
+      tc_fence_after();
+      const uint32_t vo = vslot * L::kTileBytes;
 #pragma unroll
-        for (int k = 0; k < 8; ++k)
-          umma_ts(tmem + 256 + t * 128, tmem + t * 128 + k * 8,
-                  sdesc_sw128(vb + k * 2048, L::kBoxBytes, 1024), kIdPV, (j > 0 || k > 0) ? 1u : 0u);
-        umma_commit(&pv_done[t]);
-        return true;
-      };
-      int kslot = 0, vslot = 0;
-      if (ok) ok = take(kslot);
-      if (ok) {
-        const uint32_t kb = smem_u32(sRing + kslot * L::kTileBytes);
-        if (n_kv0 > 0) issue_s(0, kb);
-        issue_s(1, kb);
-        umma_commit(&slot_empty[kslot]);
-        ok = take(vslot);
-      }
-      if (ok && n_kv0 > 0) ok = issue_pv(0, 0, smem_u32(sRing + vslot * L::kTileBytes));
-      for (int j = 0; ok && j < n_kv1; ++j) {
-        const bool next1 = j + 1 < n_kv1, next0 = j + 1 < n_kv0;
-        uint32_t kb = 0;
-        if (next1) {
-          if (!(ok = take(kslot))) break;
-          kb = smem_u32(sRing + kslot * L::kTileBytes);
-        }
-        if (next0) issue_s(0, kb);
-        if (!(ok = issue_pv(1, j, smem_u32(sRing + vslot * L::kTileBytes)))) break;
-        umma_commit(&slot_empty[vslot]);  // V_j: read by both PV_j
-        if (next1) {
-          issue_s(1, kb);
-          umma_commit(&slot_empty[kslot]);  // K_j+1: read by both S_j+1
-          if (!(ok = take(vslot))) break;
-        }
-        if (next0 && !(ok = issue_pv(0, j + 1, smem_u32(sRing + vslot * L::kTileBytes)))) break;
-      }
-      // Everything issued has completed once done_bar flips (also on abort).
-      umma_commit(done_bar);
-      mbar_wait(done_bar, 0, abort_flag, kKernFwd, 8, 4);
+      for (int k = 0; k < 8; ++k)
+        umma_ts_w(tmem + 256 + t * 128, tmem + t * 128 + k * 8, sdesc_add(dR_mn, vo + k * 2048),
+                  kIdPV, (j > 0 || k > 0) ? 1u : 0u);
+      umma_commit_w(&pv_done[t]);
+      return true;
+    };
+    int kslot = 0, vslot = 0;
+    if (ok) ok = take(kslot);
+    if (ok) {
+      if (n_kv0 > 0) issue_s(0, kslot);
+      issue_s(1, kslot);
+      umma_commit_w(&slot_empty[kslot]);
+      ok = take(vslot);
     }
+    if (ok && n_kv0 > 0) ok = issue_pv(0, 0, vslot);
+    for (int j = 0; ok && j < n_kv1; ++j) {
+      const bool next1 = j + 1 < n_kv1, next0 = j + 1 < n_kv0;
+      if (next1 && !(ok = take(kslot))) break;
+      if (next0) issue_s(0, kslot);
+      if (!(ok = issue_pv(1, j, vslot))) break;
+      umma_commit_w(&slot_empty[vslot]);  // V_j: read by both PV_j
+      if (next1) {
+        issue_s(1, kslot);
+        umma_commit_w(&slot_empty[kslot]);  // K_j+1: read by both S_j+1
+        if (!(ok = take(vslot))) break;
+      }
+      if (next0 && !(ok = issue_pv(0, j + 1, vslot))) break;
+    }
+    // every MMA this warp issued completes before tensor memory is freed
+    umma_commit_w(done_bar);
+    mbar_wait_drain(done_bar, 0, kKernFwd, 8, 4);
   } else {
     // ------------------------------------------------------------ softmax
     const int t = warp >> 2;                 // query block of this warpgroup
