@@ -205,6 +205,15 @@ fa_status_t bwd_run(const void* q, const void* k, const void* v, const void* o, 
   prm.scale = scale;
   prm.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   prm.n_items = prm.n_ktiles * prm.BHkv;
+  {
+    // kv heads per chunk of the item order: Q, dO (group query heads), K, V
+    // and the fp32 dQ accumulator of a chunk stay within about 48 MB of L2
+    const double head_bytes = static_cast<double>(prm.group) * N * HD * 2.0 * 2.0 +
+                              static_cast<double>(prm.group) * Np * HD * 4.0 +
+                              static_cast<double>(N) * HD * 2.0 * 2.0;
+    const double c = std::floor(48.0 * 1024.0 * 1024.0 / head_bytes);
+    prm.chunk_heads = static_cast<int>(std::max(1.0, std::min(c, static_cast<double>(prm.BHkv))));
+  }
   int n_sm = 0;
   if ((n_sm = sm_count()) <= 0) return FA_ERR_CUDA;
   const int cap = g_bwd_max_blocks.load();

@@ -133,6 +133,7 @@ struct BwdParams {
   void* dv;
   unsigned* work_counter;  // next work item (zeroed by bwd_pre)
   int N, Np, Hq, Hkv, group, n_ktiles, n_qtiles, BHkv, n_items;
+  int chunk_heads;         // kv heads per chunk of the item order
   float scale_log2, scale;
 };
 
@@ -179,11 +180,22 @@ struct BwdItem {
   int bh0;  // first query head of the group (b * Hq + g * group)
 };
 
+// Item order: kv heads are taken in chunks of chunk_heads (as many as keep
+// their Q, dO, K, V and dQ accumulator within part of L2); inside a chunk the
+// key blocks go in order (under a causal mask the first ones see the most
+// query blocks), each across the chunk's heads.  The blocks running at one
+// time then share few heads, and the items claimed last are short ones, so
+// the blocks finish close together.
 template <bool CAUSAL>
 __device__ __forceinline__ BwdItem bwd_item(const BwdParams& p, int item) {
   BwdItem it;
-  it.kvh = item / p.n_ktiles;
-  const int jt = item % p.n_ktiles;
+  const int per_chunk = p.chunk_heads * p.n_ktiles;
+  const int chunk = item / per_chunk;
+  const int r = item - chunk * per_chunk;
+  const int h0 = chunk * p.chunk_heads;
+  const int nh = p.BHkv - h0 < p.chunk_heads ? p.BHkv - h0 : p.chunk_heads;
+  it.kvh = h0 + r % nh;
+  const int jt = r / nh;
   const int b = it.kvh / p.Hkv, g = it.kvh % p.Hkv;
   it.kv0 = jt * 128;
   it.i0 = CAUSAL ? 2 * jt : 0;
@@ -469,6 +481,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
     mbar_wait_drain(done_bar, 0, kKernBwd, 13, 5);
   } else if (warp < 8) {
     // ------------------------------------------------------------ softmax gradient
+    // Every step is shared by the eight warps: warp w takes key rows
+    // 32(w%4)..+31 and query columns 32(w/4)..+31.
     const int quarter = warp & 3, half = warp >> 2;
     const int r = quarter * 32 + lane;                 // key row within the block
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
@@ -483,65 +497,71 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
       bool ok = true;
       for (int t = 0; t < it.T; ++t) {
         const int g = gt + t, buf = g & 1, s = g % L::kStages;
-        const int q_first = (it.i0 + t % it.nq) * 64 + half * 32;  // first query of this thread's columns
+        const int q_step = (it.i0 + t % it.nq) * 64;   // first query of the step
         if (!__all_sync(0xffffffffu, mbar_wait(&sdp_full[buf], (g >> 1) & 1, abort_flag, kKernBwd, 0, 0))) {
           ok = false;
           break;
         }
         tc_fence_after();
-        uint32_t v[32];
-        tmem_ld32(tm_S(buf) + lane_off + half * 32, v);
-        const float4* lse4 = reinterpret_cast<const float4*>(sLse + s * 64 + half * 32);
-        float pr[32];
-        tmem_ld_wait();
+        // Two passes of 16 query columns keep the live registers low (no
+        // spills).  P^T of columns 16u..16u+15 is packed into the 8
+        // tensor-memory columns at 32(u/2) + 8(u%2) of the S^T buffer, where
+        // the dV product reads it; they held S^T of columns 32(u/2) + 8(u%2)
+        // .. +7, which this warp read in this pass or the one before it.
 #pragma unroll
-        for (int c4 = 0; c4 < 8; ++c4) {
-          const float4 l4 = lse4[c4];
-          pr[4 * c4 + 0] = ex2_approx(fmaf(__uint_as_float(v[4 * c4 + 0]), c_log2, -l4.x));
-          pr[4 * c4 + 1] = ex2_approx(fmaf(__uint_as_float(v[4 * c4 + 1]), c_log2, -l4.y));
-          pr[4 * c4 + 2] = ex2_approx(fmaf(__uint_as_float(v[4 * c4 + 2]), c_log2, -l4.z));
-          pr[4 * c4 + 3] = ex2_approx(fmaf(__uint_as_float(v[4 * c4 + 3]), c_log2, -l4.w));
-        }
-        // causal: key kv_row is hidden from queries before it; padding keys
-        // (kv_row >= N) carry no probability
-        if (!row_valid) {
+        for (int qq = 2 * half; qq < 2 * half + 2; ++qq) {
+          const int q_first = q_step + qq * 16;          // first query of these 16 columns
+          uint32_t v[16];
+          tmem_ld16(tm_S(buf) + lane_off + qq * 16, v);
+          const float4* lse4 = reinterpret_cast<const float4*>(sLse + s * 64 + qq * 16);
+          const float4* d4 = reinterpret_cast<const float4*>(sD + s * 64 + qq * 16);
+          float pr[16];
+          tmem_ld_wait();
 #pragma unroll
-          for (int c = 0; c < 32; ++c) pr[c] = 0.f;
-        } else if (CAUSAL && q_first < kv_row) {
+          for (int c4 = 0; c4 < 4; ++c4) {
+            const float4 l4 = lse4[c4];
+            pr[4 * c4 + 0] = ex2_approx(fmaf(__uint_as_float(v[4 * c4 + 0]), c_log2, -l4.x));
+            pr[4 * c4 + 1] = ex2_approx(fmaf(__uint_as_float(v[4 * c4 + 1]), c_log2, -l4.y));
+            pr[4 * c4 + 2] = ex2_approx(fmaf(__uint_as_float(v[4 * c4 + 2]), c_log2, -l4.z));
+            pr[4 * c4 + 3] = ex2_approx(fmaf(__uint_as_float(v[4 * c4 + 3]), c_log2, -l4.w));
+          }
+          // causal: key kv_row is hidden from queries before it; padding keys
+          // (kv_row >= N) carry no probability
+          if (!row_valid) {
 #pragma unroll
-          for (int c = 0; c < 32; ++c)
-            if (q_first + c < kv_row) pr[c] = 0.f;
-        }
-        uint32_t pk[16];
+            for (int c = 0; c < 16; ++c) pr[c] = 0.f;
+          } else if (CAUSAL && q_first < kv_row) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) pk[i] = pack2<BF16>(pr[2 * i], pr[2 * i + 1]);
-        tmem_st16(tm_S(buf) + lane_off + half * 32, pk);
-        tmem_ld32(tm_dP(buf) + lane_off + half * 32, v);
-        const float4* d4 = reinterpret_cast<const float4*>(sD + s * 64 + half * 32);
-        tmem_ld_wait();
+            for (int c = 0; c < 16; ++c)
+              if (q_first + c < kv_row) pr[c] = 0.f;
+          }
+          uint32_t pk[8];
 #pragma unroll
-        for (int c4 = 0; c4 < 8; ++c4) {
-          const float4 dd = d4[c4];
-          pr[4 * c4 + 0] *= __uint_as_float(v[4 * c4 + 0]) - dd.x;
-          pr[4 * c4 + 1] *= __uint_as_float(v[4 * c4 + 1]) - dd.y;
-          pr[4 * c4 + 2] *= __uint_as_float(v[4 * c4 + 2]) - dd.z;
-          pr[4 * c4 + 3] *= __uint_as_float(v[4 * c4 + 3]) - dd.w;
-        }
+          for (int i = 0; i < 8; ++i) pk[i] = pack2<BF16>(pr[2 * i], pr[2 * i + 1]);
+          tmem_st8(tm_S(buf) + lane_off + (qq >> 1) * 32 + (qq & 1) * 8, pk);
+          tmem_ld16(tm_dP(buf) + lane_off + qq * 16, v);
+          tmem_ld_wait();
 #pragma unroll
-        for (int i = 0; i < 16; ++i) pk[i] = pack2<BF16>(pr[2 * i], pr[2 * i + 1]);
-        // dS^T buffer `buf` is free once step g-2 (dK_{g-2} its last reader) is done
-        if (g >= 2 && !__all_sync(0xffffffffu, mbar_wait(&step_done[(g - 2) % L::kStages],
-                                                         ((g - 2) / L::kStages) & 1, abort_flag,
-                                                         kKernBwd, 0, 2))) {
-          ok = false;
-          break;
-        }
-        uint8_t* row_base = sDS + buf * L::kDsBytes + r * 128;
+          for (int c4 = 0; c4 < 4; ++c4) {
+            const float4 dd = d4[c4];
+            pr[4 * c4 + 0] *= __uint_as_float(v[4 * c4 + 0]) - dd.x;
+            pr[4 * c4 + 1] *= __uint_as_float(v[4 * c4 + 1]) - dd.y;
+            pr[4 * c4 + 2] *= __uint_as_float(v[4 * c4 + 2]) - dd.z;
+            pr[4 * c4 + 3] *= __uint_as_float(v[4 * c4 + 3]) - dd.w;
+          }
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int chunk = (half * 4 + u) ^ (r & 7);
-          *reinterpret_cast<uint4*>(row_base + chunk * 16) =
-              make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+          for (int i = 0; i < 8; ++i) pk[i] = pack2<BF16>(pr[2 * i], pr[2 * i + 1]);
+          // dS^T buffer `buf` was last read by dQ_{g-2} and dK_{g-2}.  Both
+          // were issued before dP_g, and the commit that completed sdp_full
+          // for step g above arrives only once every MMA issued before it has
+          // completed: the buffer is free.
+          uint8_t* row_base = sDS + buf * L::kDsBytes + r * 128;
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int chunk = (qq * 2 + u) ^ (r & 7);
+            *reinterpret_cast<uint4*>(row_base + chunk * 16) =
+                make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+          }
         }
         fence_proxy_async_smem();
         tmem_st_wait();
