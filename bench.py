@@ -135,12 +135,31 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- our arm
 
+def max_over_ranks(x, world, device):
+    """The largest value of x over the ranks (one all-reduce; x itself when alone)."""
+    if world <= 1:
+        return x
+    t = torch.tensor([x], device=device, dtype=torch.float64)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(world, flops_per_replica_step, ms_per_step):
+    """Whole-job throughput: every rank runs one replica of the step."""
+    return world * flops_per_replica_step / (ms_per_step * 1e-3) / 1e12
+
+
+def rank_seed(w, rank):
+    """Seed of a rank's synthetic inputs (replicas draw different data)."""
+    return w.seed + 1000 * rank
+
+
 def run_ours(args, w, causal, rank, world, device):
     torch.cuda.set_device(device)
     build()
     binding.load()
     B, Hq, Hkv, N, d = w.B, w.Hq, w.Hkv, w.N, w.d
-    g = torch.Generator(device=device).manual_seed(w.seed + 1000 * rank)
+    g = torch.Generator(device=device).manual_seed(rank_seed(w, rank))
     mk = lambda H, s: (torch.randn((B, H, N, d), generator=g, device=device, dtype=torch.float32) * s).to(w.dtype)
     q, k, v, do = mk(Hq, w.sigma_qk), mk(Hkv, w.sigma_qk), mk(Hkv, w.sigma_vdo), mk(Hq, w.sigma_vdo)
     o = torch.empty_like(q)
@@ -195,13 +214,10 @@ def run_ours(args, w, causal, rank, world, device):
     ms_total = t0.elapsed_time(t1)
     fwd_ms = statistics.mean(a.elapsed_time(b) for a, b in fwd_ev)
     bwd_main_ms = statistics.mean(a.elapsed_time(b) for a, b in bwd_ev)
-    if world > 1:
-        t = torch.tensor([ms_total], device=device, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = max_over_ranks(ms_total, world, device)
     ms_step = ms_total / K
     f_fwd, f_bwd = w.flops_fwd(causal), w.flops_bwd(causal)
-    value = world * (f_fwd + f_bwd) / (ms_step * 1e-3) / 1e12
+    value = job_tflops(world, f_fwd + f_bwd, ms_step)
 
     # end to end through the C ABI with host buffers: pinned host inputs are
     # copied in, the step runs, the results are copied back, every step
@@ -232,12 +248,8 @@ def run_ours(args, w, causal, rank, world, device):
         e1.record(stream)
         torch.cuda.synchronize(device)
         barrier()
-        ems = e0.elapsed_time(e1) / Ke
-        if world > 1:
-            t = torch.tensor([ems], device=device, dtype=torch.float64)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            ems = float(t.item())
-        e2e = {"value": world * (f_fwd + f_bwd) / (ems * 1e-3) / 1e12, "unit": UNIT,
+        ems = max_over_ranks(e0.elapsed_time(e1) / Ke, world, device)
+        e2e = {"value": job_tflops(world, f_fwd + f_bwd, ems), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ems}
 
     pk, pk_kind = peaks()
