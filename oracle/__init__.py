@@ -79,7 +79,7 @@ class Oracle:
 
     def __init__(self, lib_path: str):
         lib = ctypes.CDLL(lib_path)
-        common = [_i64, _i64, _i64, _i64, _i64, ctypes.c_double, ctypes.c_int]
+        common = [_i64, _i64, _i64, _i64, _i64, ctypes.c_double, ctypes.c_int, _i64]  # .., causal, window
         lib.oracle_fwd.argtypes = [_dp, _dp, _dp, _dp, _dp] + common + [ctypes.c_int]
         lib.oracle_fwd_rows.argtypes = [_dp, _dp, _dp, _ip, _i64, _dp, _dp] + common + [ctypes.c_int]
         lib.oracle_fwd_online.argtypes = [_dp, _dp, _dp, _dp, _dp] + common + [_i64, ctypes.c_int]
@@ -97,19 +97,20 @@ class Oracle:
         """Threads the oracle uses for ``nthreads`` (<= 0: every online core)."""
         return self.lib.oracle_num_threads(nthreads)
 
-    def fwd(self, q, k, v, scale: float, causal: bool, nthreads: int = 0):
+    def fwd(self, q, k, v, scale: float, causal: bool, nthreads: int = 0, *, window: int = 0):
         """O [B,Hq,N,d] and lse [B,Hq,N] (natural log), materialising N x N per head."""
         q, k, v = _f64(q), _f64(k), _f64(v)
         B, Hq, Hkv, N, d = _dims(q, k)
         o = np.zeros((B, Hq, N, d))
         lse = np.zeros((B, Hq, N))
         rc = self.lib.oracle_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
-                                 B, Hq, Hkv, N, d, float(scale), int(causal), nthreads)
+                                 B, Hq, Hkv, N, d, float(scale), int(causal), int(window), nthreads)
         if rc:
             raise ValueError(f"oracle_fwd rejected its arguments ({rc})")
         return o, lse
 
-    def fwd_rows(self, q, k, v, rows, scale: float, causal: bool, nthreads: int = 0):
+    def fwd_rows(self, q, k, v, rows, scale: float, causal: bool, nthreads: int = 0, *,
+                 window: int = 0):
         """O and lse of the query rows ``rows`` of every head: [B,Hq,R,d], [B,Hq,R]."""
         q, k, v = _f64(q), _f64(k), _f64(v)
         B, Hq, Hkv, N, d = _dims(q, k)
@@ -119,25 +120,26 @@ class Oracle:
         lse = np.zeros((B, Hq, R))
         rc = self.lib.oracle_fwd_rows(_ptr(q), _ptr(k), _ptr(v), rows.ctypes.data_as(_ip), R,
                                       _ptr(o), _ptr(lse), B, Hq, Hkv, N, d, float(scale),
-                                      int(causal), nthreads)
+                                      int(causal), int(window), nthreads)
         if rc:
             raise ValueError(f"oracle_fwd_rows rejected its arguments ({rc})")
         return o, lse
 
-    def fwd_online(self, q, k, v, scale: float, causal: bool, block: int = 128, nthreads: int = 0):
+    def fwd_online(self, q, k, v, scale: float, causal: bool, block: int = 128, nthreads: int = 0,
+                   *, window: int = 0):
         """O and lse by the one-pass blocked online softmax (not the definition)."""
         q, k, v = _f64(q), _f64(k), _f64(v)
         B, Hq, Hkv, N, d = _dims(q, k)
         o = np.zeros((B, Hq, N, d))
         lse = np.zeros((B, Hq, N))
         rc = self.lib.oracle_fwd_online(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
-                                        B, Hq, Hkv, N, d, float(scale), int(causal), int(block),
+                                        B, Hq, Hkv, N, d, float(scale), int(causal), int(window), int(block),
                                         nthreads)
         if rc:
             raise ValueError(f"oracle_fwd_online rejected its arguments ({rc})")
         return o, lse
 
-    def bwd(self, q, k, v, dout, scale: float, causal: bool, nthreads: int = 0):
+    def bwd(self, q, k, v, dout, scale: float, causal: bool, nthreads: int = 0, *, window: int = 0):
         """dQ [B,Hq,N,d], dK, dV [B,Hkv,N,d] (dK, dV summed over each query group)."""
         q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
         B, Hq, Hkv, N, d = _dims(q, k)
@@ -145,12 +147,13 @@ class Oracle:
         dk = np.zeros((B, Hkv, N, d))
         dv = np.zeros((B, Hkv, N, d))
         rc = self.lib.oracle_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(dq), _ptr(dk),
-                                 _ptr(dv), B, Hq, Hkv, N, d, float(scale), int(causal), nthreads)
+                                 _ptr(dv), B, Hq, Hkv, N, d, float(scale), int(causal), int(window), nthreads)
         if rc:
             raise ValueError(f"oracle_bwd rejected its arguments ({rc})")
         return dq, dk, dv
 
-    def bwd_rows(self, q, k, v, dout, rows, scale: float, causal: bool, nthreads: int = 0):
+    def bwd_rows(self, q, k, v, dout, rows, scale: float, causal: bool, nthreads: int = 0, *,
+                 window: int = 0):
         """dQ of the query rows ``rows`` of every head: [B,Hq,R,d]."""
         q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
         B, Hq, Hkv, N, d = _dims(q, k)
@@ -159,13 +162,13 @@ class Oracle:
         dq = np.zeros((B, Hq, R, d))
         rc = self.lib.oracle_bwd_rows(_ptr(q), _ptr(k), _ptr(v), _ptr(dout),
                                       rows.ctypes.data_as(_ip), R, _ptr(dq),
-                                      B, Hq, Hkv, N, d, float(scale), int(causal), nthreads)
+                                      B, Hq, Hkv, N, d, float(scale), int(causal), int(window), nthreads)
         if rc:
             raise ValueError(f"oracle_bwd_rows rejected its arguments ({rc})")
         return dq
 
     def bwd_cols(self, q, k, v, dout, b: int, hkv: int, cols, scale: float, causal: bool,
-                 nthreads: int = 0):
+                 nthreads: int = 0, *, window: int = 0):
         """dK and dV of key rows ``cols`` of kv head (b, hkv): [C,d] each."""
         q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
         B, Hq, Hkv, N, d = _dims(q, k)
@@ -175,7 +178,7 @@ class Oracle:
         dv = np.zeros((C, d))
         rc = self.lib.oracle_bwd_cols(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), int(b), int(hkv),
                                       cols.ctypes.data_as(_ip), C, _ptr(dk), _ptr(dv),
-                                      B, Hq, Hkv, N, d, float(scale), int(causal), nthreads)
+                                      B, Hq, Hkv, N, d, float(scale), int(causal), int(window), nthreads)
         if rc:
             raise ValueError(f"oracle_bwd_cols rejected its arguments ({rc})")
         return dk, dv

@@ -17,7 +17,11 @@
  *
  *   For batch b, query head h, kv head g = h / (Hq / Hkv) (contiguous groups,
  *   "Flash Attention" glossary, grouped-query attention paragraph):
- *     s_ij  = scale * sum_c q_ic k_jc,   s_ij = -inf for j > i when causal
+ *     s_ij  = scale * sum_c q_ic k_jc,   s_ij = -inf for j > i when causal,
+ *             and, with a sliding window of W keys, -inf for j <= i - W
+ *             (query i sees keys i-W+1 .. i: the banded pattern is the
+ *             plainest instance of the block-sparse attention that the
+ *             "FlashAttention" glossary's block-sparse entry describes)
  *     m_i   = max_j s_ij                                (pass 1)
  *     l_i   = sum_j exp(s_ij - m_i)                     (pass 2)
  *     P_ij  = exp(s_ij - m_i) / l_i
@@ -105,6 +109,7 @@ typedef struct {
     i64 B, Hq, Hkv, N, d;
     double scale;
     int causal;
+    i64 window; /* 0: no window; W > 0: key j hidden from query i when j <= i - W */
     /* row / column subsets */
     const i64 *rows;
     i64 nrows;
@@ -123,12 +128,18 @@ static double dot(const double *a, const double *b, i64 d) {
     return s;
 }
 
+/* Key j is hidden from query i: after it under a causal mask, or W or more
+ * keys before it under a sliding window of W keys. */
+static int hidden(const prob_t *P, i64 i, i64 j) {
+    return (P->causal && j > i) || (P->window > 0 && j <= i - P->window);
+}
+
 /* Scores of one query row against every key: s[j] = scale * q_i . k_j, with
  * -inf for masked keys.  Returns the number of unmasked keys. */
 static i64 score_row(const prob_t *P, const double *qi, const double *kh, i64 i, double *s) {
     i64 n_valid = 0;
     for (i64 j = 0; j < P->N; ++j) {
-        if (P->causal && j > i) {
+        if (hidden(P, i, j)) {
             s[j] = -INFINITY;
         } else {
             s[j] = P->scale * dot(qi, kh + j * P->d, P->d);
@@ -184,9 +195,11 @@ static void fwd_full_item(void *ctx, i64 item) {
 }
 
 int oracle_fwd(const double *q, const double *k, const double *v, double *o, double *lse,
-               i64 B, i64 Hq, i64 Hkv, i64 N, i64 d, double scale, int causal, int nthreads) {
-    if (B < 0 || Hq <= 0 || Hkv <= 0 || N < 0 || d <= 0 || Hq % Hkv) return 1;
+               i64 B, i64 Hq, i64 Hkv, i64 N, i64 d, double scale, int causal, i64 window,
+               int nthreads) {
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || N < 0 || d <= 0 || Hq % Hkv || window < 0) return 1;
     prob_t P = {0};
+    P.window = window;
     P.q = q; P.k = k; P.v = v; P.o = o; P.lse = lse;
     P.B = B; P.Hq = Hq; P.Hkv = Hkv; P.N = N; P.d = d; P.scale = scale; P.causal = causal;
     if (N > 0) run_pool(fwd_full_item, &P, B * Hq, nthreads);
@@ -224,11 +237,13 @@ static void fwd_rows_item(void *ctx, i64 item) {
 /* o_rows: [B][Hq][nrows][d], lse_rows: [B][Hq][nrows] */
 int oracle_fwd_rows(const double *q, const double *k, const double *v, const i64 *rows, i64 nrows,
                     double *o_rows, double *lse_rows, i64 B, i64 Hq, i64 Hkv, i64 N, i64 d,
-                    double scale, int causal, int nthreads) {
-    if (B < 0 || Hq <= 0 || Hkv <= 0 || N < 0 || d <= 0 || Hq % Hkv || nrows < 0) return 1;
+                    double scale, int causal, i64 window, int nthreads) {
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || N < 0 || d <= 0 || Hq % Hkv || nrows < 0 || window < 0)
+        return 1;
     for (i64 r = 0; r < nrows; ++r)
         if (rows[r] < 0 || rows[r] >= N) return 2;
     prob_t P = {0};
+    P.window = window;
     P.q = q; P.k = k; P.v = v; P.o = o_rows; P.lse = lse_rows; P.rows = rows; P.nrows = nrows;
     P.B = B; P.Hq = Hq; P.Hkv = Hkv; P.N = N; P.d = d; P.scale = scale; P.causal = causal;
     if (nrows > 0) run_pool(fwd_rows_item, &P, B * Hq * nrows, nthreads);
@@ -263,7 +278,7 @@ static void fwd_online_item(void *ctx, i64 item) {
             double mb = -INFINITY;
             for (i64 t = 0; t < nb; ++t) {
                 const i64 j = j0 + t;
-                s[t] = (P->causal && j > i) ? -INFINITY : P->scale * dot(qh + i * d, kh + j * d, d);
+                s[t] = hidden(P, i, j) ? -INFINITY : P->scale * dot(qh + i * d, kh + j * d, d);
                 if (s[t] > mb) mb = s[t];
             }
             if (mb == -INFINITY) continue; /* block fully masked */
@@ -286,10 +301,12 @@ static void fwd_online_item(void *ctx, i64 item) {
 }
 
 int oracle_fwd_online(const double *q, const double *k, const double *v, double *o, double *lse,
-                      i64 B, i64 Hq, i64 Hkv, i64 N, i64 d, double scale, int causal, i64 block,
-                      int nthreads) {
-    if (B < 0 || Hq <= 0 || Hkv <= 0 || N < 0 || d <= 0 || Hq % Hkv || block <= 0) return 1;
+                      i64 B, i64 Hq, i64 Hkv, i64 N, i64 d, double scale, int causal, i64 window,
+                      i64 block, int nthreads) {
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || N < 0 || d <= 0 || Hq % Hkv || block <= 0 || window < 0)
+        return 1;
     prob_t P = {0};
+    P.window = window;
     P.q = q; P.k = k; P.v = v; P.o = o; P.lse = lse; P.block = block;
     P.B = B; P.Hq = Hq; P.Hkv = Hkv; P.N = N; P.d = d; P.scale = scale; P.causal = causal;
     if (N > 0) run_pool(fwd_online_item, &P, B * Hq, nthreads);
@@ -357,9 +374,10 @@ static void bwd_full_item(void *ctx, i64 item) {
 
 int oracle_bwd(const double *q, const double *k, const double *v, const double *dout, double *dq,
                double *dk, double *dv, i64 B, i64 Hq, i64 Hkv, i64 N, i64 d, double scale,
-               int causal, int nthreads) {
-    if (B < 0 || Hq <= 0 || Hkv <= 0 || N < 0 || d <= 0 || Hq % Hkv) return 1;
+               int causal, i64 window, int nthreads) {
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || N < 0 || d <= 0 || Hq % Hkv || window < 0) return 1;
     prob_t P = {0};
+    P.window = window;
     P.q = q; P.k = k; P.v = v; P.dout = dout; P.dq = dq; P.dk = dk; P.dv = dv;
     P.B = B; P.Hq = Hq; P.Hkv = Hkv; P.N = N; P.d = d; P.scale = scale; P.causal = causal;
     if (N > 0) run_pool(bwd_full_item, &P, B * Hkv, nthreads);
@@ -406,11 +424,13 @@ static void bwd_rows_item(void *ctx, i64 item) {
 /* dq_rows: [B][Hq][nrows][d] */
 int oracle_bwd_rows(const double *q, const double *k, const double *v, const double *dout,
                     const i64 *rows, i64 nrows, double *dq_rows, i64 B, i64 Hq, i64 Hkv, i64 N,
-                    i64 d, double scale, int causal, int nthreads) {
-    if (B < 0 || Hq <= 0 || Hkv <= 0 || N < 0 || d <= 0 || Hq % Hkv || nrows < 0) return 1;
+                    i64 d, double scale, int causal, i64 window, int nthreads) {
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || N < 0 || d <= 0 || Hq % Hkv || nrows < 0 || window < 0)
+        return 1;
     for (i64 r = 0; r < nrows; ++r)
         if (rows[r] < 0 || rows[r] >= N) return 2;
     prob_t P = {0};
+    P.window = window;
     P.q = q; P.k = k; P.v = v; P.dout = dout; P.dq = dq_rows; P.rows = rows; P.nrows = nrows;
     P.B = B; P.Hq = Hq; P.Hkv = Hkv; P.N = N; P.d = d; P.scale = scale; P.causal = causal;
     if (nrows > 0) run_pool(bwd_rows_item, &P, B * Hq * nrows, nthreads);
@@ -476,7 +496,7 @@ static void col_sum_item(void *ctx, i64 r) {
         const double *qh = head_ptr(P->q, b, S->h, P->Hq, N, d);
         const double *doh = head_ptr(P->dout, b, S->h, P->Hq, N, d);
         for (i64 i = S->i_lo; i < N; ++i) {
-            if (P->causal && j > i) continue;
+            if (hidden(P, i, j)) continue;
             const double s = P->scale * dot(qh + i * d, kj, d);
             const double p = exp(s - S->m[i]) / S->l[i];
             const double dp = dot(doh + i * d, vj, d);
@@ -493,8 +513,9 @@ static void col_sum_item(void *ctx, i64 r) {
 int oracle_bwd_cols(const double *q, const double *k, const double *v, const double *dout,
                     i64 b_sel, i64 hkv_sel, const i64 *cols, i64 ncols, double *dk_cols,
                     double *dv_cols, i64 B, i64 Hq, i64 Hkv, i64 N, i64 d, double scale,
-                    int causal, int nthreads) {
-    if (B < 0 || Hq <= 0 || Hkv <= 0 || N < 0 || d <= 0 || Hq % Hkv || ncols < 0) return 1;
+                    int causal, i64 window, int nthreads) {
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || N < 0 || d <= 0 || Hq % Hkv || ncols < 0 || window < 0)
+        return 1;
     if (b_sel < 0 || b_sel >= B || hkv_sel < 0 || hkv_sel >= Hkv) return 2;
     i64 j_min = N;
     for (i64 r = 0; r < ncols; ++r) {
@@ -505,7 +526,7 @@ int oracle_bwd_cols(const double *q, const double *k, const double *v, const dou
     const i64 group = Hq / Hkv;
     prob_t P = {0};
     P.q = q; P.k = k; P.v = v; P.dout = dout; P.dk = dk_cols; P.dv = dv_cols;
-    P.rows = cols; P.nrows = ncols; P.b_sel = b_sel; P.hkv_sel = hkv_sel;
+    P.rows = cols; P.nrows = ncols; P.b_sel = b_sel; P.hkv_sel = hkv_sel; P.window = window;
     P.B = B; P.Hq = Hq; P.Hkv = Hkv; P.N = N; P.d = d; P.scale = scale; P.causal = causal;
 
     const i64 i_lo = causal ? j_min : 0;

@@ -284,9 +284,128 @@ def pin_online_equals_two_pass(orc):
             _close(lse2, lse, 1e-12, f"online lse (block {block})")
 
 
+# ----------------------------------------------------- sliding-window pins
+# Causal sliding window of W keys: query i sees keys max(0, i-W+1) .. i.
+
+def pin_window_closed_forms(orc):
+    """W = 1: each query sees only its own key, O_i = V_i, lse_i = s_ii.
+    Q = 0: O_i = mean of V over the window, lse_i = ln(min(i+1, W)).
+    W >= N: the plain causal result."""
+    q, k, v, _ = _rand(18, 1, 2, 2, 21, 6)
+    o, lse = orc.fwd(q, k, v, 0.4, True, window=1)
+    _close(o, v, 1e-15, "O with W=1")
+    _close(lse, 0.4 * np.einsum("bhic,bhic->bhi", q, k), 1e-14, "lse with W=1")
+    z = np.zeros_like(q)
+    for W in (2, 5, 8):
+        o, lse = orc.fwd(z, k, v, 0.4, True, window=W)
+        want = np.stack([v[:, :, max(0, i - W + 1):i + 1].mean(axis=2) for i in range(21)], axis=2)
+        _close(o, want, 1e-14, f"O at Q=0, W={W}")
+        _close(lse, np.broadcast_to(np.log(np.minimum(np.arange(1, 22), W)), lse.shape), 1e-14,
+               f"lse at Q=0, W={W}")
+    o1, l1 = orc.fwd(q, k, v, 0.4, True, window=21)
+    o2, l2 = orc.fwd(q, k, v, 0.4, True)
+    _close(o1, o2, 0.0, "W = N equals causal")
+    _close(l1, l2, 0.0, "W = N equals causal (lse)")
+
+
+def pin_window_brute_force(orc):
+    """Forward with a window by pure-Python loops over the visible keys."""
+    B, Hq, Hkv, N, d = 1, 2, 1, 9, 3
+    q, k, v, _ = _rand(19, B, Hq, Hkv, N, d)
+    for W in (2, 4):
+        o, lse = orc.fwd(q, k, v, 0.8, True, window=W)
+        for h in range(Hq):
+            for i in range(N):
+                js = range(max(0, i - W + 1), i + 1)
+                s = {j: 0.8 * sum(q[0, h, i, c] * k[0, 0, j, c] for c in range(d)) for j in js}
+                m = max(s.values())
+                z = sum(math.exp(x - m) for x in s.values())
+                for c in range(d):
+                    want = sum(math.exp(s[j] - m) / z * v[0, 0, j, c] for j in js)
+                    assert abs(o[0, h, i, c] - want) < 1e-13, ("window brute O", W, h, i, c)
+                assert abs(lse[0, h, i] - (m + math.log(z))) < 1e-13, ("window brute lse", W, h, i)
+
+
+def _torch_window_ref(q, k, v, do, scale, W):
+    """torch fp64 SDPA with an explicit boolean mask (True = visible) + autograd."""
+    tq, tk, tv = (torch.tensor(x, dtype=torch.float64, requires_grad=True) for x in (q, k, v))
+    Hq, Hkv, n = q.shape[1], k.shape[1], q.shape[2]
+    i = torch.arange(n)[:, None]
+    j = torch.arange(n)[None, :]
+    mask = (j <= i) & (j > i - W)
+    o = torch.nn.functional.scaled_dot_product_attention(
+        tq, tk, tv, attn_mask=mask, scale=scale, enable_gqa=Hq != Hkv)
+    o.backward(torch.tensor(do, dtype=torch.float64))
+    return o.detach().numpy(), tq.grad.numpy(), tk.grad.numpy(), tv.grad.numpy()
+
+
+def pin_window_torch_sdpa(orc):
+    """Library special case: torch fp64 SDPA with the window as an explicit
+    mask, forward and gradients, MHA and GQA."""
+    for (Hq, Hkv, N, d, W, seed) in ((2, 2, 40, 8, 7, 20), (4, 2, 33, 8, 16, 21), (2, 1, 25, 4, 1, 22)):
+        q, k, v, do = _rand(seed, 1, Hq, Hkv, N, d)
+        scale = 1.0 / math.sqrt(d)
+        o, _ = orc.fwd(q, k, v, scale, True, window=W)
+        dq, dk, dv = orc.bwd(q, k, v, do, scale, True, window=W)
+        ro, rdq, rdk, rdv = _torch_window_ref(q, k, v, do, scale, W)
+        tag = f"Hq{Hq} Hkv{Hkv} N{N} W{W}"
+        _close(o, ro, 1e-12, f"torch windowed O {tag}")
+        _close(dq, rdq, 1e-11, f"torch windowed dQ {tag}")
+        _close(dk, rdk, 1e-11, f"torch windowed dK {tag}")
+        _close(dv, rdv, 1e-11, f"torch windowed dV {tag}")
+
+
+def pin_window_finite_differences(orc):
+    """Central differences of L = sum(dO * O) with a window of 3 keys."""
+    h = 1e-6
+    q, k, v, do = _rand(23, 1, 2, 1, 6, 3)
+    dq, dk, dv = orc.bwd(q, k, v, do, 0.6, True, window=3)
+
+    def loss(a):
+        o, _ = orc.fwd(a[0], a[1], a[2], 0.6, True, window=3)
+        return float(np.sum(do * o))
+
+    for slot, g in enumerate((dq, dk, dv)):
+        x = (q, k, v)[slot]
+        num = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            plus, minus = [q, k, v], [q, k, v]
+            plus[slot], minus[slot] = x.copy(), x.copy()
+            plus[slot][idx] += h
+            minus[slot][idx] -= h
+            num[idx] = (loss(plus) - loss(minus)) / (2 * h)
+        rel = np.linalg.norm(num - g) / max(np.linalg.norm(num), 1e-30)
+        assert rel <= 1e-6, f"windowed finite differences slot {slot}: rel {rel:.2e}"
+
+
+def pin_window_subsets_and_online(orc):
+    """With a window, the row/column subset forms equal the full forms and the
+    blocked one-pass recurrence (fully hidden blocks skipped) equals two-pass."""
+    q, k, v, do = _rand(24, 1, 4, 2, 50, 8)
+    rows, cols = np.array([0, 9, 30, 49]), np.array([0, 13, 47])
+    for W in (5, 17):
+        o, lse = orc.fwd(q, k, v, 0.35, True, window=W)
+        dq, dk, dv = orc.bwd(q, k, v, do, 0.35, True, window=W)
+        o_r, lse_r = orc.fwd_rows(q, k, v, rows, 0.35, True, window=W)
+        _close(o_r, o[:, :, rows], 1e-13, f"windowed fwd_rows O W{W}")
+        _close(lse_r, lse[:, :, rows], 1e-13, f"windowed fwd_rows lse W{W}")
+        _close(orc.bwd_rows(q, k, v, do, rows, 0.35, True, window=W), dq[:, :, rows], 1e-12,
+               f"windowed bwd_rows W{W}")
+        dkc, dvc = orc.bwd_cols(q, k, v, do, 0, 1, cols, 0.35, True, window=W)
+        _close(dkc, dk[0, 1, cols], 1e-12, f"windowed bwd_cols dK W{W}")
+        _close(dvc, dv[0, 1, cols], 1e-12, f"windowed bwd_cols dV W{W}")
+        for block in (4, 16):
+            o2, lse2 = orc.fwd_online(q * 3, k, v, 0.35, True, block=block, window=W)
+            o3, lse3 = orc.fwd(q * 3, k, v, 0.35, True, window=W)
+            _close(o2, o3, 1e-12, f"windowed online O W{W} block {block}")
+            _close(lse2, lse3, 1e-12, f"windowed online lse W{W} block {block}")
+
+
 ALL_PINS = [
     pin_q_zero_noncausal, pin_q_zero_causal, pin_one_hot, pin_causal_row0,
     pin_rows_sum_to_one, pin_key_shift, pin_golden, pin_brute_force_python,
     pin_torch_sdpa, pin_finite_differences, pin_q_zero_backward,
     pin_gradient_invariants, pin_subsets_match_full, pin_online_equals_two_pass,
+    pin_window_closed_forms, pin_window_brute_force, pin_window_torch_sdpa,
+    pin_window_finite_differences, pin_window_subsets_and_online,
 ]

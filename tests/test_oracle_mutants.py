@@ -26,6 +26,8 @@ MUTANTS = [
     ("online_no_rescale", "acc[c] *= corr;", "acc[c] *= 1.0;"),
     ("rows_D_from_wrong_row", "dp[j] = dot(doi, vh + j * d, d);", "dp[j] = dot(qi, vh + j * d, d);"),
     ("cols_missing_group_sum", "for (i64 t = 0; t < C->group; ++t) {", "for (i64 t = 0; t < 1; ++t) {"),
+    ("window_edge_off_by_one", "j <= i - P->window", "j < i - P->window"),
+    ("window_ignored_in_columns", "            if (hidden(P, i, j)) continue;", "            if (P->causal && j > i) continue;"),
 ]
 
 
