@@ -53,6 +53,10 @@ def load():
             lib.fa_bwd_workspace_bytes.restype = ctypes.c_size_t
             lib.fa_bwd.argtypes = ([vp] * 9 + [i, i, i, i, i, f, i, i, vp, ctypes.c_size_t, vp])
             lib.fa_bwd.restype = i
+            lib.fa_fwd_window.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp]
+            lib.fa_fwd_window.restype = i
+            lib.fa_bwd_window.argtypes = ([vp] * 9 + [i, i, i, i, i, f, i, i, vp, ctypes.c_size_t, vp])
+            lib.fa_bwd_window.restype = i
             lib.fa_get_device_status.argtypes = [vp]
             lib.fa_get_device_status.restype = i
             lib.fa_peek_device_status_word.argtypes = [vp]
@@ -109,6 +113,25 @@ def fa_fwd(q, k, v, o, lse, scale: float, causal: bool, stream=None) -> None:
     _check(st, "fa_fwd")
 
 
+def fa_fwd_window(q, k, v, o, lse, scale: float, window: int, stream=None) -> None:
+    """Causal sliding-window forward: query i sees keys i-window+1 .. i."""
+    B, Hq, Hkv, N, d = _dims(q, k)
+    st = load().fa_fwd_window(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, N, d,
+                              float(scale), int(window), _DTYPES[q.dtype], _stream(stream))
+    _check(st, "fa_fwd_window")
+
+
+def fa_bwd_window(q, k, v, o, dout, lse, dq, dk, dv, scale: float, window: int, workspace,
+                  stream=None) -> None:
+    """Backward of fa_fwd_window with the same window."""
+    B, Hq, Hkv, N, d = _dims(q, k)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = load().fa_bwd_window(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq),
+                              _ptr(dk), _ptr(dv), B, Hq, Hkv, N, d, float(scale), int(window),
+                              _DTYPES[q.dtype], _ptr(workspace), ws_bytes, _stream(stream))
+    _check(st, "fa_bwd_window")
+
+
 def fa_bwd_workspace_bytes(B: int, Hq: int, Hkv: int, N: int, d: int) -> int:
     return int(load().fa_bwd_workspace_bytes(B, Hq, Hkv, N, d))
 
@@ -154,26 +177,35 @@ def fa_set_bwd_max_blocks(max_blocks: int) -> None:
 
 # ------------------------------------------------------------ conveniences
 
-def attention_fwd(q, k, v, scale: float | None = None, causal: bool = False, stream=None):
-    """Allocates O and lse with PyTorch and runs fa_fwd; returns (O, lse)."""
+def attention_fwd(q, k, v, scale: float | None = None, causal: bool = False, stream=None,
+                  window: int = 0):
+    """Allocates O and lse with PyTorch and runs fa_fwd (fa_fwd_window when
+    window > 0, which implies causal); returns (O, lse)."""
     B, Hq, Hkv, N, d = _dims(q, k)
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     o = torch.empty_like(q)
     lse = torch.empty((B, Hq, N), device=q.device, dtype=torch.float32)
-    fa_fwd(q, k, v, o, lse, scale, causal, stream)
+    if window:
+        fa_fwd_window(q, k, v, o, lse, scale, window, stream)
+    else:
+        fa_fwd(q, k, v, o, lse, scale, causal, stream)
     return o, lse
 
 
 def attention_bwd(q, k, v, o, dout, lse, scale: float | None = None, causal: bool = False,
-                  workspace=None, stream=None):
-    """Allocates dQ, dK, dV (and the workspace if not given) and runs fa_bwd."""
+                  workspace=None, stream=None, window: int = 0):
+    """Allocates dQ, dK, dV (and the workspace if not given) and runs fa_bwd
+    (fa_bwd_window when window > 0)."""
     B, Hq, Hkv, N, d = _dims(q, k)
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     if workspace is None:
         workspace = torch.empty(max(fa_bwd_workspace_bytes(B, Hq, Hkv, N, d), 16),
                                 device=q.device, dtype=torch.uint8)
-    fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, scale, causal, workspace, stream)
+    if window:
+        fa_bwd_window(q, k, v, o, dout, lse, dq, dk, dv, scale, window, workspace, stream)
+    else:
+        fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, scale, causal, workspace, stream)
     return dq, dk, dv
 
 

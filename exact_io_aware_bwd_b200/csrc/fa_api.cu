@@ -165,7 +165,7 @@ fa_status_t launch_bwd_main(const fa::BwdParams& prm, int grid, cudaStream_t st)
 template <int HD, bool BF>
 fa_status_t bwd_run(const void* q, const void* k, const void* v, const void* o, const void* dout,
                     const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N,
-                    float scale, int causal, void* workspace, cudaStream_t st) {
+                    float scale, int causal, int window, void* workspace, cudaStream_t st) {
   const int64_t Np = fa::bwd_padded_rows(N);
   const int64_t BHq = static_cast<int64_t>(B) * Hq, BHkv = static_cast<int64_t>(B) * Hkv;
   float* Dvec = static_cast<float*>(workspace);
@@ -204,6 +204,7 @@ fa_status_t bwd_run(const void* q, const void* k, const void* v, const void* o, 
   prm.BHkv = static_cast<int>(BHkv);
   prm.scale = scale;
   prm.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  prm.window = window;
   prm.n_items = prm.n_ktiles * prm.BHkv;
   {
     // kv heads per chunk of the item order: Q, dO (group query heads), K, V
@@ -234,9 +235,13 @@ fa_status_t bwd_run(const void* q, const void* k, const void* v, const void* o, 
 
 extern "C" {
 
-fa_status_t fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
-                   int Hq, int Hkv, int N, int d, float scale, int causal, fa_dtype_t dtype,
-                   void* stream) {
+}  // extern "C"
+
+namespace {
+
+fa_status_t fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                     int Hq, int Hkv, int N, int d, float scale, int causal, int window,
+                     fa_dtype_t dtype, void* stream) {
   bool empty = false;
   fa_status_t s = check_common(B, Hq, Hkv, N, d, scale, causal, dtype, &empty);
   if (s != FA_OK) return s;
@@ -265,9 +270,27 @@ fa_status_t fa_fwd(const void* q, const void* k, const void* v, void* o, float* 
   prm.n_pairs = (N + 255) / 256;
   prm.n_ktiles = (N + 127) / 128;
   prm.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  prm.window = window;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (d == 128) return bf ? launch_fwd_c<128, true>(prm, causal, st) : launch_fwd_c<128, false>(prm, causal, st);
   return bf ? launch_fwd_c<64, true>(prm, causal, st) : launch_fwd_c<64, false>(prm, causal, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+fa_status_t fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                   int Hq, int Hkv, int N, int d, float scale, int causal, fa_dtype_t dtype,
+                   void* stream) {
+  return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, causal, 0, dtype, stream);
+}
+
+fa_status_t fa_fwd_window(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                          int Hq, int Hkv, int N, int d, float scale, int window, fa_dtype_t dtype,
+                          void* stream) {
+  if (window < 1) return FA_ERR_INVALID_ARG;
+  return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, 1, window, dtype, stream);
 }
 
 size_t fa_bwd_workspace_bytes(int B, int Hq, int Hkv, int N, int d) {
@@ -275,10 +298,14 @@ size_t fa_bwd_workspace_bytes(int B, int Hq, int Hkv, int N, int d) {
   return fa::bwd_workspace_bytes(B, Hq, N, d);
 }
 
-fa_status_t fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
-                   const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N,
-                   int d, float scale, int causal, fa_dtype_t dtype, void* workspace,
-                   size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+fa_status_t bwd_impl(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                     const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N,
+                     int d, float scale, int causal, int window, fa_dtype_t dtype, void* workspace,
+                     size_t workspace_bytes, void* stream) {
   bool empty = false;
   fa_status_t s = check_common(B, Hq, Hkv, N, d, scale, causal, dtype, &empty);
   if (s != FA_OK) return s;
@@ -294,10 +321,31 @@ fa_status_t fa_bwd(const void* q, const void* k, const void* v, const void* o, c
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const bool bf = dtype == FA_BF16;
   if (d == 128)
-    return bf ? bwd_run<128, true>(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, N, scale, causal, workspace, st)
-              : bwd_run<128, false>(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, N, scale, causal, workspace, st);
-  return bf ? bwd_run<64, true>(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, N, scale, causal, workspace, st)
-            : bwd_run<64, false>(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, N, scale, causal, workspace, st);
+    return bf ? bwd_run<128, true>(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, N, scale, causal, window, workspace, st)
+              : bwd_run<128, false>(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, N, scale, causal, window, workspace, st);
+  return bf ? bwd_run<64, true>(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, N, scale, causal, window, workspace, st)
+            : bwd_run<64, false>(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, N, scale, causal, window, workspace, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+fa_status_t fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                   const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N,
+                   int d, float scale, int causal, fa_dtype_t dtype, void* workspace,
+                   size_t workspace_bytes, void* stream) {
+  return bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, N, d, scale, causal, 0, dtype,
+                  workspace, workspace_bytes, stream);
+}
+
+fa_status_t fa_bwd_window(const void* q, const void* k, const void* v, const void* o,
+                          const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
+                          int Hq, int Hkv, int N, int d, float scale, int window, fa_dtype_t dtype,
+                          void* workspace, size_t workspace_bytes, void* stream) {
+  if (window < 1) return FA_ERR_INVALID_ARG;
+  return bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, N, d, scale, 1, window, dtype,
+                  workspace, workspace_bytes, stream);
 }
 
 fa_status_t fa_get_device_status(void* stream) {

@@ -134,6 +134,7 @@ struct BwdParams {
   unsigned* work_counter;  // next work item (zeroed by bwd_pre)
   int N, Np, Hq, Hkv, group, n_ktiles, n_qtiles, BHkv, n_items;
   int chunk_heads;         // kv heads per chunk of the item order
+  int window;              // causal sliding window of this many keys; 0: none
   float scale_log2, scale;
 };
 
@@ -199,7 +200,12 @@ __device__ __forceinline__ BwdItem bwd_item(const BwdParams& p, int item) {
   const int b = it.kvh / p.Hkv, g = it.kvh % p.Hkv;
   it.kv0 = jt * 128;
   it.i0 = CAUSAL ? 2 * jt : 0;
-  it.nq = p.n_qtiles - it.i0;
+  // under a sliding window of W keys the block's keys are seen by queries
+  // up to kv0 + 127 + W - 1 only
+  const int i_end = (CAUSAL && p.window > 0)
+                        ? min(p.n_qtiles, (min(p.N - 1, it.kv0 + 126 + p.window)) / 64 + 1)
+                        : p.n_qtiles;
+  it.nq = i_end - it.i0;
   it.T = p.group * it.nq;
   it.bh0 = b * p.Hq + g * p.group;
   return it;
@@ -530,10 +536,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
           if (!row_valid) {
 #pragma unroll
             for (int c = 0; c < 16; ++c) pr[c] = 0.f;
-          } else if (CAUSAL && q_first < kv_row) {
+          } else {
+            if (CAUSAL && q_first < kv_row) {
 #pragma unroll
-            for (int c = 0; c < 16; ++c)
-              if (q_first + c < kv_row) pr[c] = 0.f;
+              for (int c = 0; c < 16; ++c)
+                if (q_first + c < kv_row) pr[c] = 0.f;
+            }
+            // sliding window: query q sees key kv_row only while q < kv_row + W
+            if (CAUSAL && p.window > 0 && q_first + 15 >= kv_row + p.window) {
+#pragma unroll
+              for (int c = 0; c < 16; ++c)
+                if (q_first + c >= kv_row + p.window) pr[c] = 0.f;
+            }
           }
           uint32_t pk[8];
 #pragma unroll

@@ -48,6 +48,7 @@ struct FwdParams {
   CUtensorMap tm_o;  // [B*Hq][N][d] (store)
   float* lse;        // [B*Hq][N]
   int N, Hq, Hkv, group, BH, n_pairs, n_ktiles;
+  int window;        // causal sliding window of this many keys (query i sees i-W+1..i); 0: none
   float scale_log2;  // scale * log2(e)
 };
 
@@ -105,8 +106,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
   const int b = bh / p.Hq;
   const int kvh = b * p.Hkv + h / p.group;
   // key blocks seen by query block t (t = 0, 1) of the pair
-  const int n_kv0 = CAUSAL ? min(2 * pair + 1, p.n_ktiles) : p.n_ktiles;
-  const int n_kv1 = CAUSAL ? min(2 * pair + 2, p.n_ktiles) : p.n_ktiles;
+  // With a sliding window the key/value stream starts at the first block the
+  // pair's first row can see; counts below are of blocks from that one on.
+  const int j_start = (CAUSAL && p.window > 0) ? max(0, 2 * pair * 128 - p.window + 1) / 128 : 0;
+  const int n_kv0 = (CAUSAL ? min(2 * pair + 1, p.n_ktiles) : p.n_ktiles) - j_start;
+  const int n_kv1 = (CAUSAL ? min(2 * pair + 2, p.n_ktiles) : p.n_ktiles) - j_start;
 
   if (tid == 0) {
     mbar_init(q_full, 1);
@@ -152,7 +156,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
         mbar_expect_tx(&slot_full[s], L::kTileBytes);
         uint8_t* dst = sRing + s * L::kTileBytes;
         for (int c = 0; c < L::kChunks; ++c)
-          tma_load_3d(dst + c * L::kBoxBytes, map, &slot_full[s], c * 64, tile * 128, kvh);
+          tma_load_3d(dst + c * L::kBoxBytes, map, &slot_full[s], c * 64, (j_start + tile) * 128, kvh);
         ++n;
         return true;
       };
@@ -269,13 +273,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
       tmem_ld_wait();
       // mask: keys past the end of the sequence, and keys after the query
       // inside the diagonal block of a causal problem
-      const int kv0 = j * 128;
-      const bool diag = CAUSAL && (j == qtile);
-      if (diag || kv0 + 128 > p.N) {
+      const int kv0 = (j_start + j) * 128;
+      const bool diag = CAUSAL && (j_start + j == qtile);
+      // sliding window: keys below q_row - W + 1 are hidden; some row of the
+      // block meets that edge in this key block
+      const bool low = CAUSAL && p.window > 0 && kv0 + p.window <= qtile * 128 + 127;
+      if (diag || low || kv0 + 128 > p.N) {
         const int lim = min(diag ? r : 127, p.N - 1 - kv0);  // last visible column
+        const int first = low ? q_row - p.window + 1 - kv0 : 0;  // first visible column
 #pragma unroll
         for (int c = 0; c < 128; ++c)
-          if (c > lim) s[c] = __float_as_uint(-INFINITY);
+          if (c > lim || c < first) s[c] = __float_as_uint(-INFINITY);
       }
       // row max, eight independent chains
       float mx[8];
@@ -297,7 +305,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
         }
         tc_fence_after();
         const float m_upd = fmaxf(m_ref, m_new);
-        const float corr = ex2_approx(m_ref - m_upd);
+        // rows still without a visible key (m_upd = -inf) keep their zeros
+        const float corr = m_upd == -INFINITY ? 1.f : ex2_approx(m_ref - m_upd);
         const uint64_t corr2 = f2pack(corr, corr);
         m_ref = m_upd;
         l_sum *= corr;
@@ -315,8 +324,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
           tmem_st16(tm_O + c, o);
         }
       }
-      // P = 2^(s c - m_ref), packed to 16 bits over the first 64 columns of S
-      const uint64_t nm2 = f2pack(-m_ref, -m_ref);
+      // P = 2^(s c - m_ref), packed to 16 bits over the first 64 columns of S.
+      // A row that has seen no visible key yet (only under a sliding window)
+      // keeps m_ref = -inf; its scores are all -inf and give P = 0 against 0.
+      const float m_use = m_ref == -INFINITY ? 0.f : m_ref;
+      const uint64_t nm2 = f2pack(-m_use, -m_use);
       uint64_t acc[4] = {0, 0, 0, 0};
 #pragma unroll
       for (int q4 = 0; q4 < 4; ++q4) {

@@ -76,6 +76,19 @@ fa_status_t fa_fwd(const void* q, const void* k, const void* v, void* o, float* 
                    fa_dtype_t dtype, void* stream);
 
 /*
+ * Causal sliding-window forward pass: query i attends to keys
+ * max(0, i - window + 1) .. i only (window >= 1 keys, itself included; a
+ * window of N or more is the plain causal pass).  This banded mask is the
+ * simplest block-sparse pattern ("FlashAttention" glossary, block-sparse
+ * entry: skip the blocks a sparsity mask hides): key blocks wholly outside
+ * the band are not read at all.  Arguments, layouts and errors as fa_fwd;
+ * window < 1 returns FA_ERR_INVALID_ARG.
+ */
+fa_status_t fa_fwd_window(const void* q, const void* k, const void* v, void* o, float* lse,
+                          int B, int Hq, int Hkv, int N, int d, float scale, int window,
+                          fa_dtype_t dtype, void* stream);
+
+/*
  * Bytes of device scratch that fa_bwd needs for these sizes (0 for an empty
  * problem).  Linear in N: two fp32 values per query row (D_i = dO_i . O_i and
  * the logsumexp in base 2) plus an fp32 dQ accumulator [B][Hq][Np][d], with N
@@ -100,6 +113,17 @@ fa_status_t fa_bwd(const void* q, const void* k, const void* v, const void* o, c
                    const float* lse, void* dq, void* dk, void* dv,
                    int B, int Hq, int Hkv, int N, int d, float scale, int causal,
                    fa_dtype_t dtype, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Backward pass of fa_fwd_window (same window); o and lse must come from
+ * fa_fwd_window with the same window.  Arguments, workspace, layouts and
+ * errors as fa_bwd; window < 1 returns FA_ERR_INVALID_ARG.
+ */
+fa_status_t fa_bwd_window(const void* q, const void* k, const void* v, const void* o,
+                          const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                          int B, int Hq, int Hkv, int N, int d, float scale, int window,
+                          fa_dtype_t dtype, void* workspace, size_t workspace_bytes,
+                          void* stream);
 
 /*
  * Synchronises `stream`, then returns and clears the first device-side error

@@ -22,12 +22,13 @@ TOL_LSE = 1e-3
 TOL_GRAD = 2e-2
 
 
-def run_gpu(q, k, v, do, scale, causal):
-    """Forward + backward on cuda:0 through the C ABI; returns CPU tensors."""
+def run_gpu(q, k, v, do, scale, causal, window=0):
+    """Forward + backward on cuda:0 through the C ABI (the sliding-window entry
+    points when window > 0); returns CPU tensors."""
     dev = "cuda:0"
     qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, do))
-    o, lse = binding.attention_fwd(qd, kd, vd, scale, causal)
-    dq, dk, dv = binding.attention_bwd(qd, kd, vd, o, dod, lse, scale, causal)
+    o, lse = binding.attention_fwd(qd, kd, vd, scale, causal, window=window)
+    dq, dk, dv = binding.attention_bwd(qd, kd, vd, o, dod, lse, scale, causal, window=window)
     word = binding.fa_peek_device_status_word()
     status = binding.fa_get_device_status()
     assert status == binding.FA_OK, f"{binding.fa_status_string(status)} (status word {word:#010x})"
@@ -79,18 +80,18 @@ def check_grad(g, r, what):
     return e
 
 
-def check_full(q, k, v, do, scale, causal, out):
+def check_full(q, k, v, do, scale, causal, out, window=0):
     """Every output element against the full oracle."""
-    o_r, lse_r = oracle.fwd(q, k, v, scale, causal)
-    o_abs, _ = oracle.fwd(q, k, v.abs(), scale, causal)
-    dq_r, dk_r, dv_r = oracle.bwd(q, k, v, do, scale, causal)
+    o_r, lse_r = oracle.fwd(q, k, v, scale, causal, window=window)
+    o_abs, _ = oracle.fwd(q, k, v.abs(), scale, causal, window=window)
+    dq_r, dk_r, dv_r = oracle.bwd(q, k, v, do, scale, causal, window=window)
     rep = dict(o=check_o(out["o"], o_r, q.dtype, o_abs), lse=check_lse(out["lse"], lse_r))
     rep.update(dq=check_grad(out["dq"], dq_r, "dQ"), dk=check_grad(out["dk"], dk_r, "dK"),
                dv=check_grad(out["dv"], dv_r, "dV"))
     return rep
 
 
-def check_rows(q, k, v, do, scale, causal, out, rows):
+def check_rows(q, k, v, do, scale, causal, out, rows, window=0):
     """O, lse, dQ of the given query rows of every head, one kv group at a time."""
     B, Hq, N, d = q.shape
     Hkv = k.shape[1]
@@ -101,9 +102,9 @@ def check_rows(q, k, v, do, scale, causal, out, rows):
         for g in range(Hkv):
             hs = slice(g * G, (g + 1) * G)
             qq, kk, vv, dd = q[b:b + 1, hs], k[b:b + 1, g:g + 1], v[b:b + 1, g:g + 1], do[b:b + 1, hs]
-            o1, l1 = oracle.fwd_rows(qq, kk, vv, rows, scale, causal)
-            oa, _ = oracle.fwd_rows(qq, kk, vv.abs(), rows, scale, causal)
-            dq1 = oracle.bwd_rows(qq, kk, vv, dd, rows, scale, causal)
+            o1, l1 = oracle.fwd_rows(qq, kk, vv, rows, scale, causal, window=window)
+            oa, _ = oracle.fwd_rows(qq, kk, vv.abs(), rows, scale, causal, window=window)
+            dq1 = oracle.bwd_rows(qq, kk, vv, dd, rows, scale, causal, window=window)
             o_r.append(o1); lse_r.append(l1); dq_r.append(dq1); o_a.append(oa)
             o_g.append(_np(out["o"][b:b + 1, hs][:, :, rows]))
             lse_g.append(_np(out["lse"][b:b + 1, hs][:, :, rows]))
@@ -114,7 +115,7 @@ def check_rows(q, k, v, do, scale, causal, out, rows):
     return rep
 
 
-def check_cols(q, k, v, do, scale, causal, out, col_sets):
+def check_cols(q, k, v, do, scale, causal, out, col_sets, window=0):
     """dK, dV of selected key rows of selected kv heads."""
     B, Hq, N, d = q.shape
     Hkv = k.shape[1]
@@ -124,7 +125,7 @@ def check_cols(q, k, v, do, scale, causal, out, col_sets):
         cols = np.asarray(cols, dtype=np.int64)
         hs = slice(g * G, (g + 1) * G)
         dk1, dv1 = oracle.bwd_cols(q[b:b + 1, hs], k[b:b + 1, g:g + 1], v[b:b + 1, g:g + 1],
-                                   do[b:b + 1, hs], 0, 0, cols, scale, causal)
+                                   do[b:b + 1, hs], 0, 0, cols, scale, causal, window=window)
         dk_r.append(dk1); dv_r.append(dv1)
         dk_g.append(_np(out["dk"][b, g][cols])); dv_g.append(_np(out["dv"][b, g][cols]))
     cat = lambda xs: np.concatenate([x.reshape(-1) for x in xs])

@@ -120,3 +120,17 @@ def test_bwd_max_blocks_setting(lib):
     assert lib.fa_set_bwd_max_blocks(-1) == binding.FA_ERR_INVALID_ARG
     assert lib.fa_set_bwd_max_blocks(3) == binding.FA_OK
     assert lib.fa_set_bwd_max_blocks(0) == binding.FA_OK
+
+
+def test_window_entry_points_check_their_arguments(lib):
+    vp = ctypes.c_void_p
+    args = lambda w: [vp(FAKE)] * 5 + [1, 2, 2, 256, 64, 0.125, w, binding.FA_BF16, None]
+    assert lib.fa_fwd_window(*args(0)) == binding.FA_ERR_INVALID_ARG
+    assert lib.fa_fwd_window(*args(-3)) == binding.FA_ERR_INVALID_ARG
+    ws = binding.fa_bwd_workspace_bytes(1, 2, 2, 256, 64)
+    bargs = lambda w, d=64: ([vp(FAKE)] * 9 + [1, 2, 2, 256, d, 0.125, w, binding.FA_BF16,
+                                               vp(FAKE), ws, None])
+    assert lib.fa_bwd_window(*bargs(0)) == binding.FA_ERR_INVALID_ARG
+    assert lib.fa_bwd_window(*bargs(16, d=96)) == binding.FA_ERR_UNSUPPORTED
+    # empty problems are no-ops here too
+    assert lib.fa_fwd_window(*([vp(0)] * 5 + [0, 2, 2, 256, 64, 0.125, 8, binding.FA_BF16, None])) == binding.FA_OK

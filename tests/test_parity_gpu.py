@@ -85,6 +85,53 @@ def test_parity_persistent_handover(shape, dtype, causal, blocks):
     ac.check_full(q, k, v, do, scale, causal, out)
 
 
+WINDOW_CASES = [
+    # (B, Hq, Hkv, N, d), dtype, window: causal sliding window of `window` keys
+    ((1, 2, 2, 256, 64), torch.bfloat16, 1),
+    ((1, 2, 2, 256, 64), torch.bfloat16, 64),
+    ((1, 2, 2, 256, 64), torch.float16, 100),
+    ((1, 2, 2, 256, 64), torch.bfloat16, 300),
+    ((2, 4, 2, 333, 128), torch.bfloat16, 128),
+    ((2, 4, 2, 333, 128), torch.float16, 77),
+    ((1, 3, 1, 520, 64), torch.bfloat16, 130),
+    ((1, 8, 2, 700, 128), torch.bfloat16, 257),
+]
+
+
+@pytest.mark.parametrize("shape,dtype,window", WINDOW_CASES,
+                         ids=[f"{'x'.join(map(str, s))}-{str(t)[6:]}-w{w}" for s, t, w in WINDOW_CASES])
+def test_parity_window(shape, dtype, window):
+    q, k, v, do = _inputs(shape, dtype, seed=5 * sum(shape) + window)
+    scale = 1.0 / math.sqrt(shape[-1])
+    out = ac.run_gpu(q, k, v, do, scale, True, window=window)
+    ac.check_full(q, k, v, do, scale, True, out, window=window)
+
+
+def test_parity_window_wide_logits_and_handover():
+    # wide fp16 logits (running max moves within the window) with few
+    # persistent backward blocks taking many items each
+    q, k, v, do = _inputs((1, 4, 2, 900, 128), torch.float16, seed=123, sigma_qk=3.0)
+    binding.fa_set_bwd_max_blocks(3)
+    try:
+        out = ac.run_gpu(q, k, v, do, 1 / math.sqrt(128), True, window=300)
+    finally:
+        binding.fa_set_bwd_max_blocks(0)
+    ac.check_full(q, k, v, do, 1 / math.sqrt(128), True, out, window=300)
+
+
+def test_window_at_4k_rows_and_columns():
+    """A 4K-token MHA problem with a 1024-key window: seeded query rows and
+    key rows against the oracle, and the gradient invariants."""
+    w = WORKLOADS["mha4k"]
+    shape = (1, 8, 8, 4096, 128)
+    q, k, v, do = make_inputs(w, shape_override=shape)
+    out = ac.run_gpu(q, k, v, do, w.scale, True, window=1024)
+    rows = check_rows(w, N=4096)[::2]
+    ac.check_rows(q, k, v, do, w.scale, True, out, rows, window=1024)
+    ac.check_cols(q, k, v, do, w.scale, True, out, [(0, 3, [0, 1000, 2047, 3000, 4095])], window=1024)
+    ac.check_invariants(q, k, do, out)
+
+
 def test_parity_wide_logits_fp16():
     # the fp16 recipe with Q, K ~ N(0, 3^2): the running max moves many times
     q, k, v, do = _inputs((1, 2, 2, 640, 128), torch.float16, seed=99, sigma_qk=3.0)
