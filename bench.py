@@ -169,9 +169,15 @@ def run_ours(args, w, causal, rank, world, device):
     scale = w.scale
     stream = torch.cuda.current_stream(device)
 
+    W = args.window
+
     def step():
-        binding.fa_fwd(q, k, v, o, lse, scale, causal, stream)
-        binding.fa_bwd(q, k, v, o, do, lse, dq, dk, dv, scale, causal, ws, stream)
+        if W:
+            binding.fa_fwd_window(q, k, v, o, lse, scale, W, stream)
+            binding.fa_bwd_window(q, k, v, o, do, lse, dq, dk, dv, scale, W, ws, stream)
+        else:
+            binding.fa_fwd(q, k, v, o, lse, scale, causal, stream)
+            binding.fa_bwd(q, k, v, o, do, lse, dq, dk, dv, scale, causal, ws, stream)
 
     def barrier():
         if world > 1:
@@ -216,7 +222,7 @@ def run_ours(args, w, causal, rank, world, device):
     bwd_main_ms = statistics.mean(a.elapsed_time(b) for a, b in bwd_ev)
     ms_total = max_over_ranks(ms_total, world, device)
     ms_step = ms_total / K
-    f_fwd, f_bwd = w.flops_fwd(causal), w.flops_bwd(causal)
+    f_fwd, f_bwd = w.flops_fwd(causal, W), w.flops_bwd(causal, W)
     value = job_tflops(world, f_fwd + f_bwd, ms_step)
 
     # end to end through the C ABI with host buffers: every step copies the
@@ -244,8 +250,12 @@ def run_ours(args, w, causal, rank, world, device):
                     dst.copy_(src, non_blocking=True)
                 bq, bk, bv, bdo = b["inp"]
                 bo, blse, bdq, bdk, bdv = b["out"]
-                binding.fa_fwd(bq, bk, bv, bo, blse, scale, causal, st)
-                binding.fa_bwd(bq, bk, bv, bo, bdo, blse, bdq, bdk, bdv, scale, causal, b["ws"], st)
+                if W:
+                    binding.fa_fwd_window(bq, bk, bv, bo, blse, scale, W, st)
+                    binding.fa_bwd_window(bq, bk, bv, bo, bdo, blse, bdq, bdk, bdv, scale, W, b["ws"], st)
+                else:
+                    binding.fa_fwd(bq, bk, bv, bo, blse, scale, causal, st)
+                    binding.fa_bwd(bq, bk, bv, bo, bdo, blse, bdq, bdk, bdv, scale, causal, b["ws"], st)
                 for dst, src in zip(ho, b["out"]):
                     dst.copy_(src, non_blocking=True)
 
@@ -285,8 +295,9 @@ def run_ours(args, w, causal, rank, world, device):
         "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": str(w.dtype).replace("torch.", ""),
         "data": "synthetic: seeded normals (per-rank CUDA generator) with the workload's shapes and sigmas",
-        "config": {"workload": workload_desc(w, causal), "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv,
-                   "seq_len": w.N, "head_dim": w.d, "causal": causal,
+        "config": {"workload": workload_desc(w, causal) + (f" window={W}" if W else ""),
+                   "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv,
+                   "seq_len": w.N, "head_dim": w.d, "causal": causal, "window": W,
                    "parallelism": f"replicas x{world} (no exchange)",
                    "l2": "inputs larger than L2 (no flush)",
                    "flops_per_step": f_fwd + f_bwd},
@@ -302,7 +313,8 @@ def run_ours(args, w, causal, rank, world, device):
                      "frac": round(bwd_tflops_main / peak, 4), "peak_kind": f"{pk_kind} bf16 burst",
                      "traffic": profiled_traffic(w.name),
                      "traffic_unit": "bytes per launch (ncu)",
-                     "algorithmic": "2.5 x 4*B*Hq*N^2*d (/2 causal) FLOPs per launch"},
+                     "algorithmic": "2.5 x 4*B*Hq*N^2*d (/2 causal) FLOPs per launch"
+                                    + (" (visible pairs under the window)" if W else "")},
         "gpu_launches": 4 * K,
         "clocks": clk,
         "e2e": e2e,
@@ -388,6 +400,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="mha4k", choices=sorted(WORKLOADS))
     ap.add_argument("--noncausal", action="store_true", help="non-causal variant of the workload")
+    ap.add_argument("--window", type=int, default=0,
+                    help="causal sliding window of this many keys (0: none); FLOPs counted over visible pairs")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
@@ -396,6 +410,10 @@ def main():
 
     w = WORKLOADS[args.workload]
     causal = (not args.noncausal) and (True in w.causal_modes)
+    if args.window:
+        assert args.window > 0 and causal, "--window needs a causal workload"
+        if args.impl == "reference":
+            raise SystemExit("bench.py: the reference arm times the plain workload only (no --window)")
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -415,7 +433,7 @@ def main():
                                              device_id=device)
     try:
         line = run_ours(args, w, causal, rank, world, device)
-        if rank == 0 and not args.no_cpu_baseline:
+        if rank == 0 and not args.no_cpu_baseline and not args.window:
             v, rows, dt, threads = oracle_sample(w, causal, args.cpu_seconds)
             line["cpu_baseline"] = {
                 "value": round(v, 6), "unit": UNIT, "cores": threads, "kind": "oracle",

@@ -56,14 +56,19 @@ class Workload:
     def seed(self) -> int:
         return 1234 + 100 * self.index
 
-    def flops_fwd(self, causal: bool) -> float:
-        """Forward FLOPs by the convention 4*B*Hq*N^2*d, halved when causal."""
-        f = 4.0 * self.B * self.Hq * self.N * self.N * self.d
+    def flops_fwd(self, causal: bool, window: int = 0) -> float:
+        """Forward FLOPs by the convention 4*B*Hq*N^2*d, halved when causal.
+        With a causal sliding window of W < N keys: 4*B*Hq*d per visible
+        (query, key) pair, N*W - W(W-1)/2 pairs per head."""
+        N = self.N
+        if causal and 0 < window < N:
+            return 4.0 * self.B * self.Hq * self.d * (N * window - window * (window - 1) / 2)
+        f = 4.0 * self.B * self.Hq * N * N * self.d
         return f / 2 if causal else f
 
-    def flops_bwd(self, causal: bool) -> float:
+    def flops_bwd(self, causal: bool, window: int = 0) -> float:
         """Backward FLOPs by the convention 2.5 x forward."""
-        return 2.5 * self.flops_fwd(causal)
+        return 2.5 * self.flops_fwd(causal, window)
 
 
 WORKLOADS = {
