@@ -74,12 +74,24 @@ def _dims(q, k):
     return B, Hq, Hkv, N, d
 
 
+def _drop(dropout):
+    """(drop_t, seed_lo, seed_hi) from dropout = None or (t, seed): t the 8-bit
+    threshold (a key is dropped when its random byte is below t), seed 64-bit."""
+    if not dropout:
+        return 0, 0, 0
+    t, seed = dropout
+    seed = int(seed) & 0xFFFFFFFFFFFFFFFF
+    return int(t), seed & 0xFFFFFFFF, seed >> 32
+
+
 class Oracle:
     """numpy-facing wrapper of one compiled copy of the oracle library."""
 
     def __init__(self, lib_path: str):
         lib = ctypes.CDLL(lib_path)
-        common = [_i64, _i64, _i64, _i64, _i64, ctypes.c_double, ctypes.c_int, _i64]  # .., causal, window
+        u32 = ctypes.c_uint32
+        # B, Hq, Hkv, N, d, scale, causal, window, drop_t, seed_lo, seed_hi
+        common = [_i64, _i64, _i64, _i64, _i64, ctypes.c_double, ctypes.c_int, _i64, ctypes.c_int, u32, u32]
         lib.oracle_fwd.argtypes = [_dp, _dp, _dp, _dp, _dp] + common + [ctypes.c_int]
         lib.oracle_fwd_rows.argtypes = [_dp, _dp, _dp, _ip, _i64, _dp, _dp] + common + [ctypes.c_int]
         lib.oracle_fwd_online.argtypes = [_dp, _dp, _dp, _dp, _dp] + common + [_i64, ctypes.c_int]
@@ -88,29 +100,39 @@ class Oracle:
         lib.oracle_bwd_cols.argtypes = ([_dp, _dp, _dp, _dp, _i64, _i64, _ip, _i64, _dp, _dp]
                                         + common + [ctypes.c_int])
         lib.oracle_num_threads.argtypes = [ctypes.c_int]
+        lib.oracle_philox4x32_10.argtypes = [ctypes.POINTER(u32), ctypes.POINTER(u32), ctypes.POINTER(u32)]
+        lib.oracle_philox4x32_10.restype = None
         for f in ("oracle_fwd", "oracle_fwd_rows", "oracle_fwd_online", "oracle_bwd",
                   "oracle_bwd_rows", "oracle_bwd_cols", "oracle_num_threads"):
             getattr(lib, f).restype = ctypes.c_int
         self.lib = lib
 
+    def philox4x32_10(self, ctr, key):
+        """Philox4x32-10 of a 4-word counter and 2-word key: 4 words."""
+        c = (ctypes.c_uint32 * 4)(*[int(x) & 0xFFFFFFFF for x in ctr])
+        k = (ctypes.c_uint32 * 2)(*[int(x) & 0xFFFFFFFF for x in key])
+        o = (ctypes.c_uint32 * 4)()
+        self.lib.oracle_philox4x32_10(c, k, o)
+        return [int(x) for x in o]
+
     def num_threads(self, nthreads: int = 0) -> int:
         """Threads the oracle uses for ``nthreads`` (<= 0: every online core)."""
         return self.lib.oracle_num_threads(nthreads)
 
-    def fwd(self, q, k, v, scale: float, causal: bool, nthreads: int = 0, *, window: int = 0):
+    def fwd(self, q, k, v, scale: float, causal: bool, nthreads: int = 0, *, window: int = 0, dropout=None):
         """O [B,Hq,N,d] and lse [B,Hq,N] (natural log), materialising N x N per head."""
         q, k, v = _f64(q), _f64(k), _f64(v)
         B, Hq, Hkv, N, d = _dims(q, k)
         o = np.zeros((B, Hq, N, d))
         lse = np.zeros((B, Hq, N))
         rc = self.lib.oracle_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
-                                 B, Hq, Hkv, N, d, float(scale), int(causal), int(window), nthreads)
+                                 B, Hq, Hkv, N, d, float(scale), int(causal), int(window), *_drop(dropout), nthreads)
         if rc:
             raise ValueError(f"oracle_fwd rejected its arguments ({rc})")
         return o, lse
 
     def fwd_rows(self, q, k, v, rows, scale: float, causal: bool, nthreads: int = 0, *,
-                 window: int = 0):
+                 window: int = 0, dropout=None):
         """O and lse of the query rows ``rows`` of every head: [B,Hq,R,d], [B,Hq,R]."""
         q, k, v = _f64(q), _f64(k), _f64(v)
         B, Hq, Hkv, N, d = _dims(q, k)
@@ -120,26 +142,26 @@ class Oracle:
         lse = np.zeros((B, Hq, R))
         rc = self.lib.oracle_fwd_rows(_ptr(q), _ptr(k), _ptr(v), rows.ctypes.data_as(_ip), R,
                                       _ptr(o), _ptr(lse), B, Hq, Hkv, N, d, float(scale),
-                                      int(causal), int(window), nthreads)
+                                      int(causal), int(window), *_drop(dropout), nthreads)
         if rc:
             raise ValueError(f"oracle_fwd_rows rejected its arguments ({rc})")
         return o, lse
 
     def fwd_online(self, q, k, v, scale: float, causal: bool, block: int = 128, nthreads: int = 0,
-                   *, window: int = 0):
+                   *, window: int = 0, dropout=None):
         """O and lse by the one-pass blocked online softmax (not the definition)."""
         q, k, v = _f64(q), _f64(k), _f64(v)
         B, Hq, Hkv, N, d = _dims(q, k)
         o = np.zeros((B, Hq, N, d))
         lse = np.zeros((B, Hq, N))
         rc = self.lib.oracle_fwd_online(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
-                                        B, Hq, Hkv, N, d, float(scale), int(causal), int(window), int(block),
+                                        B, Hq, Hkv, N, d, float(scale), int(causal), int(window), *_drop(dropout), int(block),
                                         nthreads)
         if rc:
             raise ValueError(f"oracle_fwd_online rejected its arguments ({rc})")
         return o, lse
 
-    def bwd(self, q, k, v, dout, scale: float, causal: bool, nthreads: int = 0, *, window: int = 0):
+    def bwd(self, q, k, v, dout, scale: float, causal: bool, nthreads: int = 0, *, window: int = 0, dropout=None):
         """dQ [B,Hq,N,d], dK, dV [B,Hkv,N,d] (dK, dV summed over each query group)."""
         q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
         B, Hq, Hkv, N, d = _dims(q, k)
@@ -147,13 +169,13 @@ class Oracle:
         dk = np.zeros((B, Hkv, N, d))
         dv = np.zeros((B, Hkv, N, d))
         rc = self.lib.oracle_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(dq), _ptr(dk),
-                                 _ptr(dv), B, Hq, Hkv, N, d, float(scale), int(causal), int(window), nthreads)
+                                 _ptr(dv), B, Hq, Hkv, N, d, float(scale), int(causal), int(window), *_drop(dropout), nthreads)
         if rc:
             raise ValueError(f"oracle_bwd rejected its arguments ({rc})")
         return dq, dk, dv
 
     def bwd_rows(self, q, k, v, dout, rows, scale: float, causal: bool, nthreads: int = 0, *,
-                 window: int = 0):
+                 window: int = 0, dropout=None):
         """dQ of the query rows ``rows`` of every head: [B,Hq,R,d]."""
         q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
         B, Hq, Hkv, N, d = _dims(q, k)
@@ -162,13 +184,13 @@ class Oracle:
         dq = np.zeros((B, Hq, R, d))
         rc = self.lib.oracle_bwd_rows(_ptr(q), _ptr(k), _ptr(v), _ptr(dout),
                                       rows.ctypes.data_as(_ip), R, _ptr(dq),
-                                      B, Hq, Hkv, N, d, float(scale), int(causal), int(window), nthreads)
+                                      B, Hq, Hkv, N, d, float(scale), int(causal), int(window), *_drop(dropout), nthreads)
         if rc:
             raise ValueError(f"oracle_bwd_rows rejected its arguments ({rc})")
         return dq
 
     def bwd_cols(self, q, k, v, dout, b: int, hkv: int, cols, scale: float, causal: bool,
-                 nthreads: int = 0, *, window: int = 0):
+                 nthreads: int = 0, *, window: int = 0, dropout=None):
         """dK and dV of key rows ``cols`` of kv head (b, hkv): [C,d] each."""
         q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
         B, Hq, Hkv, N, d = _dims(q, k)
@@ -178,7 +200,7 @@ class Oracle:
         dv = np.zeros((C, d))
         rc = self.lib.oracle_bwd_cols(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), int(b), int(hkv),
                                       cols.ctypes.data_as(_ip), C, _ptr(dk), _ptr(dv),
-                                      B, Hq, Hkv, N, d, float(scale), int(causal), int(window), nthreads)
+                                      B, Hq, Hkv, N, d, float(scale), int(causal), int(window), *_drop(dropout), nthreads)
         if rc:
             raise ValueError(f"oracle_bwd_cols rejected its arguments ({rc})")
         return dk, dv

@@ -38,6 +38,17 @@
  *     dQ_i  = scale * sum_j dS_ij k_j
  *     dK_j  = scale * sum_i dS_ij q_i
  *
+ * Dropout (optional; the pages name dropout among the operations the kernel
+ * fuses, "Flash Attention" glossary, kernel-fusion paragraph, and give no
+ * rule): inverted dropout on the probabilities with an 8-bit threshold t,
+ *     P'_ij = P_ij * Z_ij * 256 / (256 - t),   Z_ij = [u8_ij >= t],
+ *     O_i   = sum_j P'_ij v_j           (lse_i is that of P, undropped)
+ *     dV_j  = sum_i P'_ij dO_i,  dP_ij = (dO_i . v_j) * Z_ij * 256/(256-t),
+ *     D_i, dS, dQ, dK as above with this dP (D_i = dO_i . O_i still holds).
+ * u8_ij is a byte of Philox4x32-10 (Salmon, Moraes, Dror and Shaw, "Parallel
+ * random numbers: as easy as 1, 2, 3", SC 2011) with key (seed_lo, seed_hi)
+ * and counter (j / 4, i / 4, b * Hq + h, 0): byte j % 4 of output word i % 4.
+ *
  * Layouts: all arrays are dense row-major fp64.
  *   q, o, dout, dq : [B][Hq][N][d]
  *   k, v, dk, dv   : [B][Hkv][N][d]
@@ -110,6 +121,9 @@ typedef struct {
     double scale;
     int causal;
     i64 window; /* 0: no window; W > 0: key j hidden from query i when j <= i - W */
+    /* dropout: drop_t = 0 means none */
+    int drop_t;
+    uint32_t seed_lo, seed_hi;
     /* row / column subsets */
     const i64 *rows;
     i64 nrows;
@@ -126,6 +140,45 @@ static double dot(const double *a, const double *b, i64 d) {
     double s = 0.0;
     for (i64 c = 0; c < d; ++c) s += a[c] * b[c];
     return s;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Philox4x32-10, as defined by Salmon et al. (SC 2011): ten rounds of
+ *   (hi0, lo0) = M0 * c0,  (hi1, lo1) = M1 * c2   (32 x 32 -> 64-bit products)
+ *   c = (hi1 ^ c1 ^ k0, lo1, hi0 ^ c3 ^ k1, lo0)
+ * with the key bumped by the Weyl constants (W0, W1) between rounds.        */
+
+void oracle_philox4x32_10(const uint32_t ctr_in[4], const uint32_t key_in[2], uint32_t out[4]) {
+    const uint32_t M0 = 0xD2511F53u, M1 = 0xCD9E8D57u, W0 = 0x9E3779B9u, W1 = 0xBB67AE85u;
+    uint32_t c0 = ctr_in[0], c1 = ctr_in[1], c2 = ctr_in[2], c3 = ctr_in[3];
+    uint32_t k0 = key_in[0], k1 = key_in[1];
+    for (int r = 0; r < 10; ++r) {
+        if (r > 0) {
+            k0 += W0;
+            k1 += W1;
+        }
+        const uint64_t p0 = (uint64_t)M0 * c0, p1 = (uint64_t)M1 * c2;
+        const uint32_t hi0 = (uint32_t)(p0 >> 32), lo0 = (uint32_t)p0;
+        const uint32_t hi1 = (uint32_t)(p1 >> 32), lo1 = (uint32_t)p1;
+        const uint32_t n0 = hi1 ^ c1 ^ k0, n2 = hi0 ^ c3 ^ k1;
+        c0 = n0;
+        c1 = lo1;
+        c2 = n2;
+        c3 = lo0;
+    }
+    out[0] = c0; out[1] = c1; out[2] = c2; out[3] = c3;
+}
+
+/* Dropout factor of (query head bh, query i, key j): 0 when dropped, else
+ * 256 / (256 - t).  1 when dropout is off. */
+static double drop_factor(const prob_t *P, i64 bh, i64 i, i64 j) {
+    if (P->drop_t == 0) return 1.0;
+    const uint32_t ctr[4] = {(uint32_t)(j >> 2), (uint32_t)(i >> 2), (uint32_t)bh, 0u};
+    const uint32_t key[2] = {P->seed_lo, P->seed_hi};
+    uint32_t x[4];
+    oracle_philox4x32_10(ctr, key, x);
+    const uint32_t u8 = (x[i & 3] >> (8 * (j & 3))) & 0xFFu;
+    return u8 >= (uint32_t)P->drop_t ? 256.0 / (256.0 - P->drop_t) : 0.0;
 }
 
 /* Key j is hidden from query i: after it under a causal mask, or W or more
@@ -181,12 +234,12 @@ static void fwd_full_item(void *ctx, i64 item) {
         softmax_row_two_pass(S + i * N, N, &m, &l);
         lseh[i] = m + log(l);
     }
-    /* O = P V */
+    /* O = P' V (P' = P with dropout applied) */
     for (i64 i = 0; i < N; ++i) {
         double *oi = oh + i * d;
         for (i64 c = 0; c < d; ++c) oi[c] = 0.0;
         for (i64 j = 0; j < N; ++j) {
-            const double p = S[i * N + j];
+            const double p = S[i * N + j] * drop_factor(P, b * P->Hq + h, i, j);
             const double *vj = vh + j * d;
             for (i64 c = 0; c < d; ++c) oi[c] += p * vj[c];
         }
@@ -196,10 +249,11 @@ static void fwd_full_item(void *ctx, i64 item) {
 
 int oracle_fwd(const double *q, const double *k, const double *v, double *o, double *lse,
                i64 B, i64 Hq, i64 Hkv, i64 N, i64 d, double scale, int causal, i64 window,
-               int nthreads) {
-    if (B < 0 || Hq <= 0 || Hkv <= 0 || N < 0 || d <= 0 || Hq % Hkv || window < 0) return 1;
+               int drop_t, uint32_t seed_lo, uint32_t seed_hi, int nthreads) {
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || N < 0 || d <= 0 || Hq % Hkv || window < 0 ||
+        drop_t < 0 || drop_t > 255) return 1;
     prob_t P = {0};
-    P.window = window;
+    P.window = window; P.drop_t = drop_t; P.seed_lo = seed_lo; P.seed_hi = seed_hi;
     P.q = q; P.k = k; P.v = v; P.o = o; P.lse = lse;
     P.B = B; P.Hq = Hq; P.Hkv = Hkv; P.N = N; P.d = d; P.scale = scale; P.causal = causal;
     if (N > 0) run_pool(fwd_full_item, &P, B * Hq, nthreads);
@@ -229,7 +283,8 @@ static void fwd_rows_item(void *ctx, i64 item) {
     for (i64 c = 0; c < d; ++c) oi[c] = 0.0;
     for (i64 j = 0; j < N; ++j) {
         const double *vj = vh + j * d;
-        for (i64 c = 0; c < d; ++c) oi[c] += s[j] * vj[c];
+        const double pj = s[j] * drop_factor(P, bh, i, j);
+        for (i64 c = 0; c < d; ++c) oi[c] += pj * vj[c];
     }
     free(s);
 }
@@ -237,13 +292,15 @@ static void fwd_rows_item(void *ctx, i64 item) {
 /* o_rows: [B][Hq][nrows][d], lse_rows: [B][Hq][nrows] */
 int oracle_fwd_rows(const double *q, const double *k, const double *v, const i64 *rows, i64 nrows,
                     double *o_rows, double *lse_rows, i64 B, i64 Hq, i64 Hkv, i64 N, i64 d,
-                    double scale, int causal, i64 window, int nthreads) {
-    if (B < 0 || Hq <= 0 || Hkv <= 0 || N < 0 || d <= 0 || Hq % Hkv || nrows < 0 || window < 0)
+                    double scale, int causal, i64 window, int drop_t,
+                    uint32_t seed_lo, uint32_t seed_hi, int nthreads) {
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || N < 0 || d <= 0 || Hq % Hkv || nrows < 0 || window < 0 ||
+        drop_t < 0 || drop_t > 255)
         return 1;
     for (i64 r = 0; r < nrows; ++r)
         if (rows[r] < 0 || rows[r] >= N) return 2;
     prob_t P = {0};
-    P.window = window;
+    P.window = window; P.drop_t = drop_t; P.seed_lo = seed_lo; P.seed_hi = seed_hi;
     P.q = q; P.k = k; P.v = v; P.o = o_rows; P.lse = lse_rows; P.rows = rows; P.nrows = nrows;
     P.B = B; P.Hq = Hq; P.Hkv = Hkv; P.N = N; P.d = d; P.scale = scale; P.causal = causal;
     if (nrows > 0) run_pool(fwd_rows_item, &P, B * Hq * nrows, nthreads);
@@ -289,8 +346,9 @@ static void fwd_online_item(void *ctx, i64 item) {
             for (i64 t = 0; t < nb; ++t) {
                 const double p = exp(s[t] - m_new);
                 l += p;
+                const double pd = p * drop_factor(P, b * P->Hq + h, i, j0 + t);
                 const double *vj = vh + (j0 + t) * d;
-                for (i64 c = 0; c < d; ++c) acc[c] += p * vj[c];
+                for (i64 c = 0; c < d; ++c) acc[c] += pd * vj[c];
             }
             m = m_new;
         }
@@ -302,11 +360,12 @@ static void fwd_online_item(void *ctx, i64 item) {
 
 int oracle_fwd_online(const double *q, const double *k, const double *v, double *o, double *lse,
                       i64 B, i64 Hq, i64 Hkv, i64 N, i64 d, double scale, int causal, i64 window,
-                      i64 block, int nthreads) {
-    if (B < 0 || Hq <= 0 || Hkv <= 0 || N < 0 || d <= 0 || Hq % Hkv || block <= 0 || window < 0)
+                      int drop_t, uint32_t seed_lo, uint32_t seed_hi, i64 block, int nthreads) {
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || N < 0 || d <= 0 || Hq % Hkv || block <= 0 || window < 0 ||
+        drop_t < 0 || drop_t > 255)
         return 1;
     prob_t P = {0};
-    P.window = window;
+    P.window = window; P.drop_t = drop_t; P.seed_lo = seed_lo; P.seed_hi = seed_hi;
     P.q = q; P.k = k; P.v = v; P.o = o; P.lse = lse; P.block = block;
     P.B = B; P.Hq = Hq; P.Hkv = Hkv; P.N = N; P.d = d; P.scale = scale; P.causal = causal;
     if (N > 0) run_pool(fwd_online_item, &P, B * Hq, nthreads);
@@ -340,9 +399,12 @@ static void bwd_full_item(void *ctx, i64 item) {
             score_row(P, qh + i * d, kh, i, Pm + i * N);
             softmax_row_two_pass(Pm + i * N, N, &m, &l);
         }
-        /* dP = dO V^T */
+        /* dP = dO V^T, times the dropout factor (dP of P, not of P') */
         for (i64 i = 0; i < N; ++i)
             for (i64 j = 0; j < N; ++j) dP[i * N + j] = dot(doh + i * d, vh + j * d, d);
+        if (P->drop_t)
+            for (i64 i = 0; i < N; ++i)
+                for (i64 j = 0; j < N; ++j) dP[i * N + j] *= drop_factor(P, b * P->Hq + h, i, j);
         /* dS = P o (dP - D), D_i = sum_j P_ij dP_ij; stored in place of dP */
         for (i64 i = 0; i < N; ++i) {
             double D = 0.0;
@@ -354,7 +416,8 @@ static void bwd_full_item(void *ctx, i64 item) {
             double *dqi = dqh + i * d;
             for (i64 c = 0; c < d; ++c) dqi[c] = 0.0;
             for (i64 j = 0; j < N; ++j) {
-                const double ds = dP[i * N + j], p = Pm[i * N + j];
+                const double ds = dP[i * N + j];
+                const double p = Pm[i * N + j] * drop_factor(P, b * P->Hq + h, i, j); /* P' */
                 const double *kj = kh + j * d;
                 const double *qi = qh + i * d;
                 const double *doi = doh + i * d;
@@ -374,10 +437,12 @@ static void bwd_full_item(void *ctx, i64 item) {
 
 int oracle_bwd(const double *q, const double *k, const double *v, const double *dout, double *dq,
                double *dk, double *dv, i64 B, i64 Hq, i64 Hkv, i64 N, i64 d, double scale,
-               int causal, i64 window, int nthreads) {
-    if (B < 0 || Hq <= 0 || Hkv <= 0 || N < 0 || d <= 0 || Hq % Hkv || window < 0) return 1;
+               int causal, i64 window, int drop_t, uint32_t seed_lo, uint32_t seed_hi,
+               int nthreads) {
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || N < 0 || d <= 0 || Hq % Hkv || window < 0 ||
+        drop_t < 0 || drop_t > 255) return 1;
     prob_t P = {0};
-    P.window = window;
+    P.window = window; P.drop_t = drop_t; P.seed_lo = seed_lo; P.seed_hi = seed_hi;
     P.q = q; P.k = k; P.v = v; P.dout = dout; P.dq = dq; P.dk = dk; P.dv = dv;
     P.B = B; P.Hq = Hq; P.Hkv = Hkv; P.N = N; P.d = d; P.scale = scale; P.causal = causal;
     if (N > 0) run_pool(bwd_full_item, &P, B * Hkv, nthreads);
@@ -408,6 +473,7 @@ static void bwd_rows_item(void *ctx, i64 item) {
     double D = 0.0;
     for (i64 j = 0; j < N; ++j) {
         dp[j] = dot(doi, vh + j * d, d);
+        dp[j] *= drop_factor(P, bh, i, j);
         D += p[j] * dp[j];
     }
     for (i64 c = 0; c < d; ++c) dqi[c] = 0.0;
@@ -424,13 +490,15 @@ static void bwd_rows_item(void *ctx, i64 item) {
 /* dq_rows: [B][Hq][nrows][d] */
 int oracle_bwd_rows(const double *q, const double *k, const double *v, const double *dout,
                     const i64 *rows, i64 nrows, double *dq_rows, i64 B, i64 Hq, i64 Hkv, i64 N,
-                    i64 d, double scale, int causal, i64 window, int nthreads) {
-    if (B < 0 || Hq <= 0 || Hkv <= 0 || N < 0 || d <= 0 || Hq % Hkv || nrows < 0 || window < 0)
+                    i64 d, double scale, int causal, i64 window, int drop_t,
+                    uint32_t seed_lo, uint32_t seed_hi, int nthreads) {
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || N < 0 || d <= 0 || Hq % Hkv || nrows < 0 || window < 0 ||
+        drop_t < 0 || drop_t > 255)
         return 1;
     for (i64 r = 0; r < nrows; ++r)
         if (rows[r] < 0 || rows[r] >= N) return 2;
     prob_t P = {0};
-    P.window = window;
+    P.window = window; P.drop_t = drop_t; P.seed_lo = seed_lo; P.seed_hi = seed_hi;
     P.q = q; P.k = k; P.v = v; P.dout = dout; P.dq = dq_rows; P.rows = rows; P.nrows = nrows;
     P.B = B; P.Hq = Hq; P.Hkv = Hkv; P.N = N; P.d = d; P.scale = scale; P.causal = causal;
     if (nrows > 0) run_pool(bwd_rows_item, &P, B * Hq * nrows, nthreads);
@@ -468,7 +536,7 @@ static void col_stats_item(void *ctx, i64 item) {
     softmax_row_two_pass(p, N, &m, &l);
     double D = 0.0;
     for (i64 j = 0; j < N; ++j)
-        if (p[j] != 0.0) D += p[j] * dot(doi, vh + j * d, d);
+        if (p[j] != 0.0) D += p[j] * dot(doi, vh + j * d, d) * drop_factor(P, b * P->Hq + h, i, j);
     C->m[i] = m;
     C->l[i] = l;
     C->D[i] = D;
@@ -499,10 +567,11 @@ static void col_sum_item(void *ctx, i64 r) {
             if (hidden(P, i, j)) continue;
             const double s = P->scale * dot(qh + i * d, kj, d);
             const double p = exp(s - S->m[i]) / S->l[i];
-            const double dp = dot(doh + i * d, vj, d);
+            const double f = drop_factor(P, b * P->Hq + S->h, i, j);
+            const double dp = dot(doh + i * d, vj, d) * f;
             const double ds = p * (dp - S->D[i]);
             for (i64 c = 0; c < d; ++c) {
-                dvj[c] += p * doh[i * d + c];
+                dvj[c] += p * f * doh[i * d + c];
                 dkj[c] += P->scale * ds * qh[i * d + c];
             }
         }
@@ -513,8 +582,10 @@ static void col_sum_item(void *ctx, i64 r) {
 int oracle_bwd_cols(const double *q, const double *k, const double *v, const double *dout,
                     i64 b_sel, i64 hkv_sel, const i64 *cols, i64 ncols, double *dk_cols,
                     double *dv_cols, i64 B, i64 Hq, i64 Hkv, i64 N, i64 d, double scale,
-                    int causal, i64 window, int nthreads) {
-    if (B < 0 || Hq <= 0 || Hkv <= 0 || N < 0 || d <= 0 || Hq % Hkv || ncols < 0 || window < 0)
+                    int causal, i64 window, int drop_t, uint32_t seed_lo, uint32_t seed_hi,
+               int nthreads) {
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || N < 0 || d <= 0 || Hq % Hkv || ncols < 0 || window < 0 ||
+        drop_t < 0 || drop_t > 255)
         return 1;
     if (b_sel < 0 || b_sel >= B || hkv_sel < 0 || hkv_sel >= Hkv) return 2;
     i64 j_min = N;
@@ -526,7 +597,7 @@ int oracle_bwd_cols(const double *q, const double *k, const double *v, const dou
     const i64 group = Hq / Hkv;
     prob_t P = {0};
     P.q = q; P.k = k; P.v = v; P.dout = dout; P.dk = dk_cols; P.dv = dv_cols;
-    P.rows = cols; P.nrows = ncols; P.b_sel = b_sel; P.hkv_sel = hkv_sel; P.window = window;
+    P.rows = cols; P.nrows = ncols; P.b_sel = b_sel; P.hkv_sel = hkv_sel; P.window = window; P.drop_t = drop_t; P.seed_lo = seed_lo; P.seed_hi = seed_hi;
     P.B = B; P.Hq = Hq; P.Hkv = Hkv; P.N = N; P.d = d; P.scale = scale; P.causal = causal;
 
     const i64 i_lo = causal ? j_min : 0;

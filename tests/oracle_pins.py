@@ -401,6 +401,130 @@ def pin_window_subsets_and_online(orc):
             _close(lse2, lse3, 1e-12, f"windowed online lse W{W} block {block}")
 
 
+# ------------------------------------------------------------- dropout pins
+# dropout=(t, seed): a key is dropped when its Philox byte is below t; kept
+# probabilities are scaled by 256 / (256 - t).
+
+def pin_philox_known_answers(orc):
+    """The generator reproduces the published Philox4x32-10 known-answer vectors."""
+    with open(os.path.join(GOLDEN, "philox4x32_10_kat.json")) as f:
+        kat = json.load(f)
+    for vec in kat["vectors"]:
+        got = orc.philox4x32_10([int(x, 16) for x in vec["ctr"]], [int(x, 16) for x in vec["key"]])
+        assert got == [int(x, 16) for x in vec["out"]], ("Philox KAT", vec, [hex(x) for x in got])
+
+
+def _mask(orc, bh, N, t, seed):
+    """Keep mask [N][N] of one query head from the generator, by the stated
+    counter layout (j/4, i/4, bh, 0), word i%4, byte j%4."""
+    key = [seed & 0xFFFFFFFF, seed >> 32]
+    z = np.zeros((N, N))
+    for i in range(N):
+        for j in range(N):
+            x = orc.philox4x32_10([j >> 2, i >> 2, bh, 0], key)
+            z[i, j] = ((x[i & 3] >> (8 * (j & 3))) & 0xFF) >= t
+    return z
+
+
+def pin_dropout_off_and_keep_rate(orc):
+    """t = 0 is exactly no dropout; the keep rate of t = 64 is 3/4."""
+    q, k, v, do = _rand(25, 1, 2, 1, 24, 8)
+    o0, l0 = orc.fwd(q, k, v, 0.5, True)
+    o1, l1 = orc.fwd(q, k, v, 0.5, True, dropout=(0, 99))
+    _close(o1, o0, 0.0, "dropout t=0 O")
+    _close(l1, l0, 0.0, "dropout t=0 lse")
+    g0 = orc.bwd(q, k, v, do, 0.5, True)
+    g1 = orc.bwd(q, k, v, do, 0.5, True, dropout=(0, 99))
+    for a, b_ in zip(g0, g1):
+        _close(a, b_, 0.0, "dropout t=0 gradients")
+    z = np.concatenate([_mask(orc, bh, 64, 64, 12345).ravel() for bh in range(3)])
+    assert abs(z.mean() - 0.75) < 0.01, f"keep rate {z.mean():.4f} for t=64"
+
+
+def pin_dropout_identity_readout(orc):
+    """Q = 0 (uniform P = 1/N, non-causal) and V = I: O = Z * s / N, so the
+    output is the keep mask itself, entry by entry; lse = ln N is untouched."""
+    N = d = 16
+    for (t, seed) in ((64, 7), (200, (1 << 40) + 3)):
+        q = np.zeros((1, 2, N, d))
+        k = _rand(26, 1, 2, 2, N, d)[1]
+        v = np.broadcast_to(np.eye(N)[None, None], (1, 2, N, d)).copy()
+        o, lse = orc.fwd(q, k, v, 0.3, False, dropout=(t, seed))
+        for h in range(2):
+            want = _mask(orc, h, N, t, seed) * (256.0 / (256 - t)) / N
+            _close(o[0, h], want, 1e-15, f"identity read-out t={t} head {h}")
+        _close(lse, np.full(lse.shape, math.log(N)), 1e-14, "lse with dropout")
+
+
+def pin_dropout_torch(orc):
+    """Library special case: torch fp64 attention with the keep mask applied
+    to the softmax as an explicit matrix, forward and autograd gradients."""
+    for (Hq, Hkv, N, d, causal, t, seed) in ((2, 1, 20, 8, True, 51, 5), (2, 2, 17, 4, False, 128, 6)):
+        q, k, v, do = _rand(27 + N, 1, Hq, Hkv, N, d)
+        scale = 0.6
+        z = np.stack([_mask(orc, h, N, t, seed) for h in range(Hq)]) * (256.0 / (256 - t))
+        tq, tk, tv = (torch.tensor(x, dtype=torch.float64, requires_grad=True) for x in (q, k, v))
+        kk, vv = (x.repeat_interleave(Hq // Hkv, dim=1) for x in (tk, tv))
+        s = scale * tq @ kk.transpose(-1, -2)
+        if causal:
+            s = s.masked_fill(torch.ones(N, N, dtype=torch.bool).triu(1), float("-inf"))
+        p = torch.softmax(s, dim=-1) * torch.tensor(z)[None]
+        o_t = p @ vv
+        o_t.backward(torch.tensor(do))
+        o, _ = orc.fwd(q, k, v, scale, causal, dropout=(t, seed))
+        dq, dk, dv = orc.bwd(q, k, v, do, scale, causal, dropout=(t, seed))
+        _close(o, o_t.detach().numpy(), 1e-12, "torch dropout O")
+        _close(dq, tq.grad.numpy(), 1e-11, "torch dropout dQ")
+        _close(dk, tk.grad.numpy(), 1e-11, "torch dropout dK")
+        _close(dv, tv.grad.numpy(), 1e-11, "torch dropout dV")
+
+
+def pin_dropout_finite_differences(orc):
+    """Central differences of L = sum(dO * O) under a fixed dropout mask."""
+    h = 1e-6
+    q, k, v, do = _rand(28, 1, 2, 1, 6, 3)
+    drop = (90, 77)
+    grads = orc.bwd(q, k, v, do, 0.7, True, dropout=drop)
+
+    def loss(a):
+        o, _ = orc.fwd(a[0], a[1], a[2], 0.7, True, dropout=drop)
+        return float(np.sum(do * o))
+
+    for slot, g in enumerate(grads):
+        x = (q, k, v)[slot]
+        num = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            plus, minus = [q, k, v], [q, k, v]
+            plus[slot], minus[slot] = x.copy(), x.copy()
+            plus[slot][idx] += h
+            minus[slot][idx] -= h
+            num[idx] = (loss(plus) - loss(minus)) / (2 * h)
+        rel = np.linalg.norm(num - g) / max(np.linalg.norm(num), 1e-30)
+        assert rel <= 1e-6, f"dropout finite differences slot {slot}: rel {rel:.2e}"
+
+
+def pin_dropout_subsets_and_online(orc):
+    """With dropout the row/column subset forms equal the full forms, and the
+    blocked one-pass recurrence equals two-pass."""
+    q, k, v, do = _rand(29, 2, 4, 2, 36, 8)
+    rows, cols = np.array([0, 5, 35]), np.array([2, 17, 33])
+    drop = (40, 2024)
+    for causal in (False, True):
+        o, lse = orc.fwd(q, k, v, 0.35, causal, dropout=drop)
+        dq, dk, dv = orc.bwd(q, k, v, do, 0.35, causal, dropout=drop)
+        o_r, lse_r = orc.fwd_rows(q, k, v, rows, 0.35, causal, dropout=drop)
+        _close(o_r, o[:, :, rows], 1e-13, "dropout fwd_rows O")
+        _close(lse_r, lse[:, :, rows], 1e-13, "dropout fwd_rows lse")
+        _close(orc.bwd_rows(q, k, v, do, rows, 0.35, causal, dropout=drop), dq[:, :, rows], 1e-12,
+               "dropout bwd_rows")
+        dkc, dvc = orc.bwd_cols(q, k, v, do, 1, 0, cols, 0.35, causal, dropout=drop)
+        _close(dkc, dk[1, 0, cols], 1e-12, "dropout bwd_cols dK")
+        _close(dvc, dv[1, 0, cols], 1e-12, "dropout bwd_cols dV")
+        o2, l2 = orc.fwd_online(q, k, v, 0.35, causal, block=8, dropout=drop)
+        _close(o2, o, 1e-12, "dropout online O")
+        _close(l2, lse, 1e-12, "dropout online lse")
+
+
 ALL_PINS = [
     pin_q_zero_noncausal, pin_q_zero_causal, pin_one_hot, pin_causal_row0,
     pin_rows_sum_to_one, pin_key_shift, pin_golden, pin_brute_force_python,
@@ -408,4 +532,6 @@ ALL_PINS = [
     pin_gradient_invariants, pin_subsets_match_full, pin_online_equals_two_pass,
     pin_window_closed_forms, pin_window_brute_force, pin_window_torch_sdpa,
     pin_window_finite_differences, pin_window_subsets_and_online,
+    pin_philox_known_answers, pin_dropout_off_and_keep_rate, pin_dropout_identity_readout,
+    pin_dropout_torch, pin_dropout_finite_differences, pin_dropout_subsets_and_online,
 ]
