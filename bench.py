@@ -170,9 +170,13 @@ def run_ours(args, w, causal, rank, world, device):
     stream = torch.cuda.current_stream(device)
 
     W = args.window
+    DR = (args.dropout, 0x5EED0000 + rank) if args.dropout else None
 
     def step():
-        if W:
+        if DR:
+            binding.fa_fwd_dropout(q, k, v, o, lse, scale, causal, DR[0], DR[1], stream)
+            binding.fa_bwd_dropout(q, k, v, o, do, lse, dq, dk, dv, scale, causal, DR[0], DR[1], ws, stream)
+        elif W:
             binding.fa_fwd_window(q, k, v, o, lse, scale, W, stream)
             binding.fa_bwd_window(q, k, v, o, do, lse, dq, dk, dv, scale, W, ws, stream)
         else:
@@ -250,7 +254,11 @@ def run_ours(args, w, causal, rank, world, device):
                     dst.copy_(src, non_blocking=True)
                 bq, bk, bv, bdo = b["inp"]
                 bo, blse, bdq, bdk, bdv = b["out"]
-                if W:
+                if DR:
+                    binding.fa_fwd_dropout(bq, bk, bv, bo, blse, scale, causal, DR[0], DR[1], st)
+                    binding.fa_bwd_dropout(bq, bk, bv, bo, bdo, blse, bdq, bdk, bdv, scale, causal,
+                                           DR[0], DR[1], b["ws"], st)
+                elif W:
                     binding.fa_fwd_window(bq, bk, bv, bo, blse, scale, W, st)
                     binding.fa_bwd_window(bq, bk, bv, bo, bdo, blse, bdq, bdk, bdv, scale, W, b["ws"], st)
                 else:
@@ -295,9 +303,11 @@ def run_ours(args, w, causal, rank, world, device):
         "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": str(w.dtype).replace("torch.", ""),
         "data": "synthetic: seeded normals (per-rank CUDA generator) with the workload's shapes and sigmas",
-        "config": {"workload": workload_desc(w, causal) + (f" window={W}" if W else ""),
+        "config": {"workload": workload_desc(w, causal) + (f" window={W}" if W else "")
+                   + (f" dropout={args.dropout}" if DR else ""),
                    "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv,
                    "seq_len": w.N, "head_dim": w.d, "causal": causal, "window": W,
+                   "dropout": args.dropout,
                    "parallelism": f"replicas x{world} (no exchange)",
                    "l2": "inputs larger than L2 (no flush)",
                    "flops_per_step": f_fwd + f_bwd},
@@ -400,6 +410,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="mha4k", choices=sorted(WORKLOADS))
     ap.add_argument("--noncausal", action="store_true", help="non-causal variant of the workload")
+    ap.add_argument("--dropout", type=float, default=0.0,
+                    help="dropout probability on the attention probabilities (0: none)")
     ap.add_argument("--window", type=int, default=0,
                     help="causal sliding window of this many keys (0: none); FLOPs counted over visible pairs")
     ap.add_argument("--no-e2e", action="store_true")
@@ -410,6 +422,8 @@ def main():
 
     w = WORKLOADS[args.workload]
     causal = (not args.noncausal) and (True in w.causal_modes)
+    if args.window and args.dropout:
+        raise SystemExit("bench.py: --window and --dropout are not combined")
     if args.window:
         assert args.window > 0 and causal, "--window needs a causal workload"
         if args.impl == "reference":
@@ -433,7 +447,7 @@ def main():
                                              device_id=device)
     try:
         line = run_ours(args, w, causal, rank, world, device)
-        if rank == 0 and not args.no_cpu_baseline and not args.window:
+        if rank == 0 and not args.no_cpu_baseline and not args.window and not args.dropout:
             v, rows, dt, threads = oracle_sample(w, causal, args.cpu_seconds)
             line["cpu_baseline"] = {
                 "value": round(v, 6), "unit": UNIT, "cores": threads, "kind": "oracle",

@@ -57,6 +57,12 @@ def load():
             lib.fa_fwd_window.restype = i
             lib.fa_bwd_window.argtypes = ([vp] * 9 + [i, i, i, i, i, f, i, i, vp, ctypes.c_size_t, vp])
             lib.fa_bwd_window.restype = i
+            u64 = ctypes.c_uint64
+            lib.fa_fwd_dropout.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, f, u64, i, vp]
+            lib.fa_fwd_dropout.restype = i
+            lib.fa_bwd_dropout.argtypes = ([vp] * 9 + [i, i, i, i, i, f, i, f, u64, i, vp,
+                                                       ctypes.c_size_t, vp])
+            lib.fa_bwd_dropout.restype = i
             lib.fa_get_device_status.argtypes = [vp]
             lib.fa_get_device_status.restype = i
             lib.fa_peek_device_status_word.argtypes = [vp]
@@ -132,6 +138,28 @@ def fa_bwd_window(q, k, v, o, dout, lse, dq, dk, dv, scale: float, window: int, 
     _check(st, "fa_bwd_window")
 
 
+def fa_fwd_dropout(q, k, v, o, lse, scale: float, causal: bool, p_drop: float, seed: int,
+                   stream=None) -> None:
+    """Forward with dropout on the probabilities (8-bit threshold round(256 p))."""
+    B, Hq, Hkv, N, d = _dims(q, k)
+    st = load().fa_fwd_dropout(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, N, d,
+                               float(scale), int(bool(causal)), float(p_drop),
+                               int(seed) & 0xFFFFFFFFFFFFFFFF, _DTYPES[q.dtype], _stream(stream))
+    _check(st, "fa_fwd_dropout")
+
+
+def fa_bwd_dropout(q, k, v, o, dout, lse, dq, dk, dv, scale: float, causal: bool, p_drop: float,
+                   seed: int, workspace, stream=None) -> None:
+    """Backward of fa_fwd_dropout with the same p_drop and seed."""
+    B, Hq, Hkv, N, d = _dims(q, k)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = load().fa_bwd_dropout(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq),
+                               _ptr(dk), _ptr(dv), B, Hq, Hkv, N, d, float(scale),
+                               int(bool(causal)), float(p_drop), int(seed) & 0xFFFFFFFFFFFFFFFF,
+                               _DTYPES[q.dtype], _ptr(workspace), ws_bytes, _stream(stream))
+    _check(st, "fa_bwd_dropout")
+
+
 def fa_bwd_workspace_bytes(B: int, Hq: int, Hkv: int, N: int, d: int) -> int:
     return int(load().fa_bwd_workspace_bytes(B, Hq, Hkv, N, d))
 
@@ -178,22 +206,27 @@ def fa_set_bwd_max_blocks(max_blocks: int) -> None:
 # ------------------------------------------------------------ conveniences
 
 def attention_fwd(q, k, v, scale: float | None = None, causal: bool = False, stream=None,
-                  window: int = 0):
+                  window: int = 0, dropout=None):
     """Allocates O and lse with PyTorch and runs fa_fwd (fa_fwd_window when
-    window > 0, which implies causal); returns (O, lse)."""
+    window > 0, which implies causal; fa_fwd_dropout when dropout = (p_drop,
+    seed)); returns (O, lse)."""
+    if window and dropout:
+        raise ValueError("a sliding window and dropout are not combined")
     B, Hq, Hkv, N, d = _dims(q, k)
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     o = torch.empty_like(q)
     lse = torch.empty((B, Hq, N), device=q.device, dtype=torch.float32)
     if window:
         fa_fwd_window(q, k, v, o, lse, scale, window, stream)
+    elif dropout:
+        fa_fwd_dropout(q, k, v, o, lse, scale, causal, dropout[0], dropout[1], stream)
     else:
         fa_fwd(q, k, v, o, lse, scale, causal, stream)
     return o, lse
 
 
 def attention_bwd(q, k, v, o, dout, lse, scale: float | None = None, causal: bool = False,
-                  workspace=None, stream=None, window: int = 0):
+                  workspace=None, stream=None, window: int = 0, dropout=None):
     """Allocates dQ, dK, dV (and the workspace if not given) and runs fa_bwd
     (fa_bwd_window when window > 0)."""
     B, Hq, Hkv, N, d = _dims(q, k)
@@ -204,6 +237,9 @@ def attention_bwd(q, k, v, o, dout, lse, scale: float | None = None, causal: boo
                                 device=q.device, dtype=torch.uint8)
     if window:
         fa_bwd_window(q, k, v, o, dout, lse, dq, dk, dv, scale, window, workspace, stream)
+    elif dropout:
+        fa_bwd_dropout(q, k, v, o, dout, lse, dq, dk, dv, scale, causal, dropout[0], dropout[1],
+                       workspace, stream)
     else:
         fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, scale, causal, workspace, stream)
     return dq, dk, dv

@@ -99,6 +99,16 @@ int sm_count() {
   return n_sm[dev];
 }
 
+// Dropout probability -> 8-bit threshold t = round(256 p): a key is dropped
+// when its random byte is below t.  p must be finite, 0 <= p and t <= 255.
+bool drop_threshold(float p, int* t) {
+  if (!std::isfinite(p) || p < 0.f) return false;
+  const long r = std::lround(static_cast<double>(p) * 256.0);
+  if (r > 255) return false;
+  *t = static_cast<int>(r);
+  return true;
+}
+
 // Checks shared by fa_fwd and fa_bwd.  Sets *empty for a problem with no work.
 fa_status_t check_common(int B, int Hq, int Hkv, int N, int d, float scale, int causal,
                          fa_dtype_t dtype, bool* empty) {
@@ -130,9 +140,9 @@ fa_status_t opt_in_smem(K kernel, int smem) {
   return FA_OK;
 }
 
-template <int HD, bool BF, bool CA>
+template <int HD, bool BF, bool CA, bool DR>
 fa_status_t launch_fwd(const FwdParams& prm, cudaStream_t st) {
-  auto kern = fa::fa_fwd_kernel<HD, BF, CA>;
+  auto kern = fa::fa_fwd_kernel<HD, BF, CA, DR>;
   const int smem = FwdLayout<HD>::kDynSmem;
   fa_status_t s = opt_in_smem(kern, smem);
   if (s != FA_OK) return s;
@@ -146,12 +156,14 @@ fa_status_t launch_fwd(const FwdParams& prm, cudaStream_t st) {
 
 template <int HD, bool BF>
 fa_status_t launch_fwd_c(const FwdParams& prm, int causal, cudaStream_t st) {
-  return causal ? launch_fwd<HD, BF, true>(prm, st) : launch_fwd<HD, BF, false>(prm, st);
+  if (prm.drop_t > 0)
+    return causal ? launch_fwd<HD, BF, true, true>(prm, st) : launch_fwd<HD, BF, false, true>(prm, st);
+  return causal ? launch_fwd<HD, BF, true, false>(prm, st) : launch_fwd<HD, BF, false, false>(prm, st);
 }
 
-template <int HD, bool BF, bool CA>
+template <int HD, bool BF, bool CA, bool DR>
 fa_status_t launch_bwd_main(const fa::BwdParams& prm, int grid, cudaStream_t st) {
-  auto kern = fa::fa_bwd_kernel<HD, BF, CA>;
+  auto kern = fa::fa_bwd_kernel<HD, BF, CA, DR>;
   const int smem = fa::BwdLayout<HD>::kDynSmem;
   fa_status_t s = opt_in_smem(kern, smem);
   if (s != FA_OK) return s;
@@ -165,7 +177,8 @@ fa_status_t launch_bwd_main(const fa::BwdParams& prm, int grid, cudaStream_t st)
 template <int HD, bool BF>
 fa_status_t bwd_run(const void* q, const void* k, const void* v, const void* o, const void* dout,
                     const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N,
-                    float scale, int causal, int window, void* workspace, cudaStream_t st) {
+                    float scale, int causal, int window, uint32_t drop_t, uint64_t seed,
+                    void* workspace, cudaStream_t st) {
   const int64_t Np = fa::bwd_padded_rows(N);
   const int64_t BHq = static_cast<int64_t>(B) * Hq, BHkv = static_cast<int64_t>(B) * Hkv;
   float* Dvec = static_cast<float*>(workspace);
@@ -205,6 +218,10 @@ fa_status_t bwd_run(const void* q, const void* k, const void* v, const void* o, 
   prm.scale = scale;
   prm.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   prm.window = window;
+  prm.drop_t = drop_t;
+  prm.drop_scale = drop_t ? 256.0f / static_cast<float>(256u - drop_t) : 1.0f;
+  prm.seed_lo = static_cast<uint32_t>(seed);
+  prm.seed_hi = static_cast<uint32_t>(seed >> 32);
   prm.n_items = prm.n_ktiles * prm.BHkv;
   {
     // kv heads per chunk of the item order: Q, dO (group query heads), K, V
@@ -219,8 +236,11 @@ fa_status_t bwd_run(const void* q, const void* k, const void* v, const void* o, 
   if ((n_sm = sm_count()) <= 0) return FA_ERR_CUDA;
   const int cap = g_bwd_max_blocks.load();
   const int grid = std::min(prm.n_items, cap > 0 ? std::min(cap, n_sm) : n_sm);  // persistent
-  fa_status_t s = causal ? launch_bwd_main<HD, BF, true>(prm, grid, st)
-                         : launch_bwd_main<HD, BF, false>(prm, grid, st);
+  fa_status_t s = prm.drop_t > 0
+                      ? (causal ? launch_bwd_main<HD, BF, true, true>(prm, grid, st)
+                                : launch_bwd_main<HD, BF, false, true>(prm, grid, st))
+                      : (causal ? launch_bwd_main<HD, BF, true, false>(prm, grid, st)
+                                : launch_bwd_main<HD, BF, false, false>(prm, grid, st));
   if (s != FA_OK) return s;
 
   // 3. dQ = scale * accumulator
@@ -241,7 +261,7 @@ namespace {
 
 fa_status_t fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                      int Hq, int Hkv, int N, int d, float scale, int causal, int window,
-                     fa_dtype_t dtype, void* stream) {
+                     uint32_t drop_t, uint64_t seed, fa_dtype_t dtype, void* stream) {
   bool empty = false;
   fa_status_t s = check_common(B, Hq, Hkv, N, d, scale, causal, dtype, &empty);
   if (s != FA_OK) return s;
@@ -271,6 +291,10 @@ fa_status_t fwd_impl(const void* q, const void* k, const void* v, void* o, float
   prm.n_ktiles = (N + 127) / 128;
   prm.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   prm.window = window;
+  prm.drop_t = drop_t;
+  prm.drop_scale = drop_t ? 256.0f / static_cast<float>(256u - drop_t) : 1.0f;
+  prm.seed_lo = static_cast<uint32_t>(seed);
+  prm.seed_hi = static_cast<uint32_t>(seed >> 32);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (d == 128) return bf ? launch_fwd_c<128, true>(prm, causal, st) : launch_fwd_c<128, false>(prm, causal, st);
   return bf ? launch_fwd_c<64, true>(prm, causal, st) : launch_fwd_c<64, false>(prm, causal, st);
@@ -283,14 +307,23 @@ extern "C" {
 fa_status_t fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                    int Hq, int Hkv, int N, int d, float scale, int causal, fa_dtype_t dtype,
                    void* stream) {
-  return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, causal, 0, dtype, stream);
+  return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, causal, 0, 0, 0, dtype, stream);
 }
 
 fa_status_t fa_fwd_window(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                           int Hq, int Hkv, int N, int d, float scale, int window, fa_dtype_t dtype,
                           void* stream) {
   if (window < 1) return FA_ERR_INVALID_ARG;
-  return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, 1, window, dtype, stream);
+  return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, 1, window, 0, 0, dtype, stream);
+}
+
+fa_status_t fa_fwd_dropout(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                           int Hq, int Hkv, int N, int d, float scale, int causal, float p_drop,
+                           uint64_t seed, fa_dtype_t dtype, void* stream) {
+  int t = 0;
+  if (!drop_threshold(p_drop, &t)) return FA_ERR_INVALID_ARG;
+  return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, causal, 0, static_cast<uint32_t>(t),
+                  seed, dtype, stream);
 }
 
 size_t fa_bwd_workspace_bytes(int B, int Hq, int Hkv, int N, int d) {
@@ -304,8 +337,8 @@ namespace {
 
 fa_status_t bwd_impl(const void* q, const void* k, const void* v, const void* o, const void* dout,
                      const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N,
-                     int d, float scale, int causal, int window, fa_dtype_t dtype, void* workspace,
-                     size_t workspace_bytes, void* stream) {
+                     int d, float scale, int causal, int window, uint32_t drop_t, uint64_t seed,
+                     fa_dtype_t dtype, void* workspace, size_t workspace_bytes, void* stream) {
   bool empty = false;
   fa_status_t s = check_common(B, Hq, Hkv, N, d, scale, causal, dtype, &empty);
   if (s != FA_OK) return s;
@@ -321,10 +354,10 @@ fa_status_t bwd_impl(const void* q, const void* k, const void* v, const void* o,
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const bool bf = dtype == FA_BF16;
   if (d == 128)
-    return bf ? bwd_run<128, true>(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, N, scale, causal, window, workspace, st)
-              : bwd_run<128, false>(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, N, scale, causal, window, workspace, st);
-  return bf ? bwd_run<64, true>(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, N, scale, causal, window, workspace, st)
-            : bwd_run<64, false>(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, N, scale, causal, window, workspace, st);
+    return bf ? bwd_run<128, true>(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, N, scale, causal, window, drop_t, seed, workspace, st)
+              : bwd_run<128, false>(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, N, scale, causal, window, drop_t, seed, workspace, st);
+  return bf ? bwd_run<64, true>(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, N, scale, causal, window, drop_t, seed, workspace, st)
+            : bwd_run<64, false>(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, N, scale, causal, window, drop_t, seed, workspace, st);
 }
 
 }  // namespace
@@ -335,8 +368,8 @@ fa_status_t fa_bwd(const void* q, const void* k, const void* v, const void* o, c
                    const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N,
                    int d, float scale, int causal, fa_dtype_t dtype, void* workspace,
                    size_t workspace_bytes, void* stream) {
-  return bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, N, d, scale, causal, 0, dtype,
-                  workspace, workspace_bytes, stream);
+  return bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, N, d, scale, causal, 0, 0, 0,
+                  dtype, workspace, workspace_bytes, stream);
 }
 
 fa_status_t fa_bwd_window(const void* q, const void* k, const void* v, const void* o,
@@ -344,8 +377,19 @@ fa_status_t fa_bwd_window(const void* q, const void* k, const void* v, const voi
                           int Hq, int Hkv, int N, int d, float scale, int window, fa_dtype_t dtype,
                           void* workspace, size_t workspace_bytes, void* stream) {
   if (window < 1) return FA_ERR_INVALID_ARG;
-  return bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, N, d, scale, 1, window, dtype,
-                  workspace, workspace_bytes, stream);
+  return bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, N, d, scale, 1, window, 0, 0,
+                  dtype, workspace, workspace_bytes, stream);
+}
+
+fa_status_t fa_bwd_dropout(const void* q, const void* k, const void* v, const void* o,
+                           const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
+                           int Hq, int Hkv, int N, int d, float scale, int causal, float p_drop,
+                           uint64_t seed, fa_dtype_t dtype, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+  int t = 0;
+  if (!drop_threshold(p_drop, &t)) return FA_ERR_INVALID_ARG;
+  return bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, N, d, scale, causal, 0,
+                  static_cast<uint32_t>(t), seed, dtype, workspace, workspace_bytes, stream);
 }
 
 fa_status_t fa_get_device_status(void* stream) {

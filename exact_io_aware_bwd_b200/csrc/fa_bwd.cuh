@@ -135,6 +135,9 @@ struct BwdParams {
   int N, Np, Hq, Hkv, group, n_ktiles, n_qtiles, BHkv, n_items;
   int chunk_heads;         // kv heads per chunk of the item order
   int window;              // causal sliding window of this many keys; 0: none
+  // dropout (kernel instantiated with DROP), as in the forward pass
+  uint32_t seed_lo, seed_hi, drop_t;
+  float drop_scale;
   float scale_log2, scale;
 };
 
@@ -213,7 +216,7 @@ __device__ __forceinline__ BwdItem bwd_item(const BwdParams& p, int item) {
 
 constexpr int kBwdThreads = 448;
 
-template <int HD, bool BF16, bool CAUSAL>
+template <int HD, bool BF16, bool CAUSAL, bool DROP>
 __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_constant__ BwdParams p) {
   using L = BwdLayout<HD>;
   using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
@@ -504,6 +507,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
       for (int t = 0; t < it.T; ++t) {
         const int g = gt + t, buf = g & 1, s = g % L::kStages;
         const int q_step = (it.i0 + t % it.nq) * 64;   // first query of the step
+        const int bh_step = it.bh0 + t / it.nq;          // query head of the step
         if (!__all_sync(0xffffffffu, mbar_wait(&sdp_full[buf], (g >> 1) & 1, abort_flag, kKernBwd, 0, 0))) {
           ok = false;
           break;
@@ -550,11 +554,37 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
             }
           }
           uint32_t pk[8];
+          float fd[16];  // dropout factor of each of the 16 queries (1 without dropout)
+          if constexpr (DROP) {
+            // one Philox call covers 4 queries x 4 keys: word = query % 4,
+            // byte = key % 4
 #pragma unroll
-          for (int i = 0; i < 8; ++i) pk[i] = pack2<BF16>(pr[2 * i], pr[2 * i + 1]);
+            for (int g = 0; g < 4; ++g) {
+              const uint4 rnd = philox4x32_10(
+                  make_uint4(static_cast<uint32_t>(kv_row >> 2), static_cast<uint32_t>((q_first + 4 * g) >> 2),
+                             static_cast<uint32_t>(bh_step), 0u),
+                  p.seed_lo, p.seed_hi);
+              const int sh = 8 * (kv_row & 3);
+              fd[4 * g + 0] = ((rnd.x >> sh) & 0xFFu) >= p.drop_t ? p.drop_scale : 0.f;
+              fd[4 * g + 1] = ((rnd.y >> sh) & 0xFFu) >= p.drop_t ? p.drop_scale : 0.f;
+              fd[4 * g + 2] = ((rnd.z >> sh) & 0xFFu) >= p.drop_t ? p.drop_scale : 0.f;
+              fd[4 * g + 3] = ((rnd.w >> sh) & 0xFFu) >= p.drop_t ? p.drop_scale : 0.f;
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              pk[i] = pack2<BF16>(pr[2 * i] * fd[2 * i], pr[2 * i + 1] * fd[2 * i + 1]);  // P'
+          } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) pk[i] = pack2<BF16>(pr[2 * i], pr[2 * i + 1]);
+          }
           tmem_st8(tm_S(buf) + lane_off + (qq >> 1) * 32 + (qq & 1) * 8, pk);
           tmem_ld16(tm_dP(buf) + lane_off + qq * 16, v);
           tmem_ld_wait();
+          if constexpr (DROP) {
+            // dP of P is dP' times the dropout factor
+#pragma unroll
+            for (int c = 0; c < 16; ++c) v[c] = __float_as_uint(__uint_as_float(v[c]) * fd[c]);
+          }
 #pragma unroll
           for (int c4 = 0; c4 < 4; ++c4) {
             const float4 dd = d4[c4];

@@ -49,6 +49,11 @@ struct FwdParams {
   float* lse;        // [B*Hq][N]
   int N, Hq, Hkv, group, BH, n_pairs, n_ktiles;
   int window;        // causal sliding window of this many keys (query i sees i-W+1..i); 0: none
+  // dropout (kernels instantiated with DROP): key j of query i is dropped
+  // when byte j%4 of word i%4 of Philox4x32-10((j/4, i/4, bh, 0), seed) is
+  // below drop_t; kept probabilities are scaled by drop_scale = 256/(256-t)
+  uint32_t seed_lo, seed_hi, drop_t;
+  float drop_scale;
   float scale_log2;  // scale * log2(e)
 };
 
@@ -73,7 +78,7 @@ struct FwdLayout {
 constexpr int kFwdThreads = 320;
 constexpr uint32_t kKernFwd = 1;
 
-template <int HD, bool BF16, bool CAUSAL>
+template <int HD, bool BF16, bool CAUSAL, bool DROP>
 __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_constant__ FwdParams p) {
   using L = FwdLayout<HD>;
   extern __shared__ uint8_t smem_raw[];
@@ -333,13 +338,28 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
 #pragma unroll
       for (int q4 = 0; q4 < 4; ++q4) {
         uint32_t pk[16];
+        uint32_t keep_word = 0;  // dropout bytes of 4 keys of this row
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const int c = q4 * 32 + 2 * i;
           const uint64_t x = fma2(f2pack(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), c2, nm2);
           const uint64_t pp = f2pack(ex2_approx(f2lo(x)), ex2_approx(f2hi(x)));
-          acc[i & 3] = add2(acc[i & 3], pp);
-          pk[i] = pack2<BF16>(f2lo(pp), f2hi(pp));
+          acc[i & 3] = add2(acc[i & 3], pp);  // l sums the undropped P
+          if constexpr (DROP) {
+            if ((i & 1) == 0) {
+              const uint4 rnd = philox4x32_10(
+                  make_uint4(static_cast<uint32_t>((kv0 + c) >> 2), static_cast<uint32_t>(q_row >> 2),
+                             static_cast<uint32_t>(bh), 0u),
+                  p.seed_lo, p.seed_hi);
+              keep_word = uint4_word(rnd, q_row & 3);
+            }
+            const uint32_t b0 = (keep_word >> (16 * (i & 1))) & 0xFFu;
+            const uint32_t b1 = (keep_word >> (16 * (i & 1) + 8)) & 0xFFu;
+            pk[i] = pack2<BF16>(b0 >= p.drop_t ? f2lo(pp) * p.drop_scale : 0.f,
+                                b1 >= p.drop_t ? f2hi(pp) * p.drop_scale : 0.f);
+          } else {
+            pk[i] = pack2<BF16>(f2lo(pp), f2hi(pp));
+          }
         }
         tmem_st16(tm_S + q4 * 16, pk);
       }

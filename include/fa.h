@@ -89,6 +89,23 @@ fa_status_t fa_fwd_window(const void* q, const void* k, const void* v, void* o, 
                           fa_dtype_t dtype, void* stream);
 
 /*
+ * Forward pass with dropout on the attention probabilities (the pages list
+ * dropout among the operations the attention kernel fuses: "Flash
+ * Attention" glossary, kernel-fusion paragraph; they give no rule, this is
+ * the library's): inverted dropout with an 8-bit threshold t = round(256 *
+ * p_drop): key j of query i is dropped when byte j%4 of word i%4 of
+ * Philox4x32-10(counter (j/4, i/4, b*Hq + h, 0), key (seed low 32 bits,
+ * seed high 32 bits)) is below t; kept probabilities are scaled by
+ * 256 / (256 - t), so the drop rate is exactly t/256.  lse is that of the
+ * undropped softmax.  The same (p_drop, seed) must be given to
+ * fa_bwd_dropout.  p_drop < 0, not finite, or with t > 255 returns
+ * FA_ERR_INVALID_ARG; t = 0 is the plain pass.  Otherwise as fa_fwd.
+ */
+fa_status_t fa_fwd_dropout(const void* q, const void* k, const void* v, void* o, float* lse,
+                           int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+                           float p_drop, uint64_t seed, fa_dtype_t dtype, void* stream);
+
+/*
  * Bytes of device scratch that fa_bwd needs for these sizes (0 for an empty
  * problem).  Linear in N: two fp32 values per query row (D_i = dO_i . O_i and
  * the logsumexp in base 2) plus an fp32 dQ accumulator [B][Hq][Np][d], with N
@@ -124,6 +141,16 @@ fa_status_t fa_bwd_window(const void* q, const void* k, const void* v, const voi
                           int B, int Hq, int Hkv, int N, int d, float scale, int window,
                           fa_dtype_t dtype, void* workspace, size_t workspace_bytes,
                           void* stream);
+
+/*
+ * Backward pass of fa_fwd_dropout (same p_drop and seed: the dropout mask is
+ * regenerated, not stored).  Otherwise as fa_bwd.
+ */
+fa_status_t fa_bwd_dropout(const void* q, const void* k, const void* v, const void* o,
+                           const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                           int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+                           float p_drop, uint64_t seed, fa_dtype_t dtype, void* workspace,
+                           size_t workspace_bytes, void* stream);
 
 /*
  * Synchronises `stream`, then returns and clears the first device-side error

@@ -22,13 +22,15 @@ TOL_LSE = 1e-3
 TOL_GRAD = 2e-2
 
 
-def run_gpu(q, k, v, do, scale, causal, window=0):
+def run_gpu(q, k, v, do, scale, causal, window=0, dropout=None):
     """Forward + backward on cuda:0 through the C ABI (the sliding-window entry
-    points when window > 0); returns CPU tensors."""
+    points when window > 0, the dropout ones when dropout = (p_drop, seed));
+    returns CPU tensors."""
     dev = "cuda:0"
     qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, do))
-    o, lse = binding.attention_fwd(qd, kd, vd, scale, causal, window=window)
-    dq, dk, dv = binding.attention_bwd(qd, kd, vd, o, dod, lse, scale, causal, window=window)
+    o, lse = binding.attention_fwd(qd, kd, vd, scale, causal, window=window, dropout=dropout)
+    dq, dk, dv = binding.attention_bwd(qd, kd, vd, o, dod, lse, scale, causal, window=window,
+                                       dropout=dropout)
     word = binding.fa_peek_device_status_word()
     status = binding.fa_get_device_status()
     assert status == binding.FA_OK, f"{binding.fa_status_string(status)} (status word {word:#010x})"
@@ -80,11 +82,20 @@ def check_grad(g, r, what):
     return e
 
 
-def check_full(q, k, v, do, scale, causal, out, window=0):
+def oracle_dropout(dropout):
+    """The oracle's (threshold, seed) for the library's (p_drop, seed)."""
+    if not dropout:
+        return None
+    p_drop, seed = dropout
+    return int(round(p_drop * 256)), seed
+
+
+def check_full(q, k, v, do, scale, causal, out, window=0, dropout=None):
     """Every output element against the full oracle."""
-    o_r, lse_r = oracle.fwd(q, k, v, scale, causal, window=window)
-    o_abs, _ = oracle.fwd(q, k, v.abs(), scale, causal, window=window)
-    dq_r, dk_r, dv_r = oracle.bwd(q, k, v, do, scale, causal, window=window)
+    dr = oracle_dropout(dropout)
+    o_r, lse_r = oracle.fwd(q, k, v, scale, causal, window=window, dropout=dr)
+    o_abs, _ = oracle.fwd(q, k, v.abs(), scale, causal, window=window, dropout=dr)
+    dq_r, dk_r, dv_r = oracle.bwd(q, k, v, do, scale, causal, window=window, dropout=dr)
     rep = dict(o=check_o(out["o"], o_r, q.dtype, o_abs), lse=check_lse(out["lse"], lse_r))
     rep.update(dq=check_grad(out["dq"], dq_r, "dQ"), dk=check_grad(out["dk"], dk_r, "dK"),
                dv=check_grad(out["dv"], dv_r, "dV"))

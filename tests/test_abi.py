@@ -134,3 +134,20 @@ def test_window_entry_points_check_their_arguments(lib):
     assert lib.fa_bwd_window(*bargs(16, d=96)) == binding.FA_ERR_UNSUPPORTED
     # empty problems are no-ops here too
     assert lib.fa_fwd_window(*([vp(0)] * 5 + [0, 2, 2, 256, 64, 0.125, 8, binding.FA_BF16, None])) == binding.FA_OK
+
+
+@pytest.mark.parametrize("p_drop", [-0.1, 1.0, 0.999, float("nan"), float("inf")])
+def test_dropout_entry_points_reject_bad_rates(lib, p_drop):
+    vp = ctypes.c_void_p
+    args = [vp(FAKE)] * 5 + [1, 2, 2, 256, 64, 0.125, 1, p_drop, 7, binding.FA_BF16, None]
+    assert lib.fa_fwd_dropout(*args) == binding.FA_ERR_INVALID_ARG
+    ws = binding.fa_bwd_workspace_bytes(1, 2, 2, 256, 64)
+    bargs = [vp(FAKE)] * 9 + [1, 2, 2, 256, 64, 0.125, 1, p_drop, 7, binding.FA_BF16, vp(FAKE), ws, None]
+    assert lib.fa_bwd_dropout(*bargs) == binding.FA_ERR_INVALID_ARG
+
+
+def test_dropout_entry_points_accept_good_rates_on_empty_problems(lib):
+    vp = ctypes.c_void_p
+    for p_drop in (0.0, 0.1, 0.5, 0.99):
+        args = [vp(0)] * 5 + [0, 2, 2, 256, 64, 0.125, 1, p_drop, 7, binding.FA_BF16, None]
+        assert lib.fa_fwd_dropout(*args) == binding.FA_OK

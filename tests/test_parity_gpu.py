@@ -10,6 +10,7 @@ import pytest
 import torch
 
 import attn_check as ac
+import oracle
 from exact_io_aware_bwd_b200 import binding
 from exact_io_aware_bwd_b200.build import build
 from exact_io_aware_bwd_b200.workloads import WORKLOADS, check_cols, check_rows, make_inputs
@@ -130,6 +131,48 @@ def test_window_at_4k_rows_and_columns():
     ac.check_rows(q, k, v, do, w.scale, True, out, rows, window=1024)
     ac.check_cols(q, k, v, do, w.scale, True, out, [(0, 3, [0, 1000, 2047, 3000, 4095])], window=1024)
     ac.check_invariants(q, k, do, out)
+
+
+DROPOUT_CASES = [
+    # (B, Hq, Hkv, N, d), dtype, causal, p_drop, seed
+    ((1, 2, 2, 256, 64), torch.bfloat16, False, 0.1, 1),
+    ((1, 2, 2, 256, 64), torch.bfloat16, True, 0.5, 2),
+    ((2, 4, 2, 333, 128), torch.bfloat16, True, 0.25, (1 << 40) + 17),
+    ((2, 4, 2, 333, 128), torch.float16, False, 0.2, 3),
+    ((1, 3, 1, 200, 64), torch.float16, True, 0.3, 4),
+    ((1, 8, 2, 384, 128), torch.bfloat16, True, 0.05, 5),
+]
+
+
+@pytest.mark.parametrize("shape,dtype,causal,p_drop,seed", DROPOUT_CASES,
+                         ids=[f"{'x'.join(map(str, s))}-{str(t)[6:]}-{'c' if c else 'nc'}-p{p}"
+                              for s, t, c, p, _ in DROPOUT_CASES])
+def test_parity_dropout(shape, dtype, causal, p_drop, seed):
+    q, k, v, do = _inputs(shape, dtype, seed=7 * sum(shape) + seed % 1000)
+    scale = 1.0 / math.sqrt(shape[-1])
+    out = ac.run_gpu(q, k, v, do, scale, causal, dropout=(p_drop, seed))
+    ac.check_full(q, k, v, do, scale, causal, out, dropout=(p_drop, seed))
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_dropout_mask_bit_exact(d):
+    """Q = 0 (uniform P = 1/N, non-causal) and V = I: O is the keep mask times
+    256/(256-t)/N, so every keep decision of the GPU can be read off O and
+    compared exactly with the oracle's."""
+    N, Hq, p_drop, seed = d, 3, 0.375, 987654321
+    t = round(p_drop * 256)
+    q = torch.zeros((1, Hq, N, d), dtype=torch.float16)
+    k = _inputs((1, Hq, Hq, N, d), torch.float16, seed=31)[1]
+    v = torch.eye(N, d, dtype=torch.float16).expand(1, Hq, N, d).contiguous()
+    dev = "cuda:0"
+    o, lse = binding.attention_fwd(q.to(dev), k.to(dev), v.to(dev), 0.5, False, dropout=(p_drop, seed))
+    assert binding.fa_get_device_status() == binding.FA_OK
+    level = 256.0 / (256 - t) / N
+    z_gpu = o.float().cpu().numpy() > 0.5 * level
+    o_ref, _ = oracle.fwd(q, k, v, 0.5, False, dropout=(t, seed))
+    z_ref = o_ref > 0.5 * level
+    assert (z_gpu == z_ref).all(), f"{int((z_gpu != z_ref).sum())} keep decisions differ"
+    assert abs(z_ref.mean() - (1 - t / 256)) < 0.03
 
 
 def test_parity_wide_logits_fp16():
