@@ -556,20 +556,35 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
           uint32_t pk[8];
           float fd[16];  // dropout factor of each of the 16 queries (1 without dropout)
           if constexpr (DROP) {
-            // one Philox call covers 4 queries x 4 keys: word = query % 4,
-            // byte = key % 4
+            // One Philox call covers 4 queries x 4 keys (word = query % 4,
+            // byte = key % 4).  The 4 lanes of a quad hold 4 consecutive keys:
+            // lane g of the quad draws the block of queries 4g..4g+3 of these
+            // 16 and offers each lane its byte column (that lane's key, 4
+            // queries); four rotations of a shuffle collect them.
+            const int ql = lane & 3;
+            const uint4 rnd = philox4x32_10(
+                make_uint4(static_cast<uint32_t>(kv_row >> 2), static_cast<uint32_t>((q_first + 4 * ql) >> 2),
+                           static_cast<uint32_t>(bh_step), 0u),
+                p.seed_lo, p.seed_hi);
+            uint32_t cols[4] = {0, 0, 0, 0};  // cols[g]: bytes of queries 4g..4g+3 for this key
 #pragma unroll
-            for (int g = 0; g < 4; ++g) {
-              const uint4 rnd = philox4x32_10(
-                  make_uint4(static_cast<uint32_t>(kv_row >> 2), static_cast<uint32_t>((q_first + 4 * g) >> 2),
-                             static_cast<uint32_t>(bh_step), 0u),
-                  p.seed_lo, p.seed_hi);
-              const int sh = 8 * (kv_row & 3);
-              fd[4 * g + 0] = ((rnd.x >> sh) & 0xFFu) >= p.drop_t ? p.drop_scale : 0.f;
-              fd[4 * g + 1] = ((rnd.y >> sh) & 0xFFu) >= p.drop_t ? p.drop_scale : 0.f;
-              fd[4 * g + 2] = ((rnd.z >> sh) & 0xFFu) >= p.drop_t ? p.drop_scale : 0.f;
-              fd[4 * g + 3] = ((rnd.w >> sh) & 0xFFu) >= p.drop_t ? p.drop_scale : 0.f;
+            for (int rr = 0; rr < 4; ++rr) {
+              const uint32_t b = static_cast<uint32_t>((ql - rr) & 3);  // column the reader needs
+              const uint32_t lo = __byte_perm(rnd.x, rnd.y, b | ((4u + b) << 4));
+              const uint32_t hi = __byte_perm(rnd.z, rnd.w, b | ((4u + b) << 4));
+              const uint32_t col = __byte_perm(lo, hi, 0x5410u);
+              const uint32_t got = __shfl_sync(0xffffffffu, col, (lane & ~3) | ((ql + rr) & 3));
+              const int g = (ql + rr) & 3;
+              cols[0] = g == 0 ? got : cols[0];
+              cols[1] = g == 1 ? got : cols[1];
+              cols[2] = g == 2 ? got : cols[2];
+              cols[3] = g == 3 ? got : cols[3];
             }
+#pragma unroll
+            for (int g = 0; g < 4; ++g)
+#pragma unroll
+              for (int u = 0; u < 4; ++u)
+                fd[4 * g + u] = ((cols[g] >> (8 * u)) & 0xFFu) >= p.drop_t ? p.drop_scale : 0.f;
 #pragma unroll
             for (int i = 0; i < 8; ++i)
               pk[i] = pack2<BF16>(pr[2 * i] * fd[2 * i], pr[2 * i + 1] * fd[2 * i + 1]);  // P'

@@ -338,7 +338,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
 #pragma unroll
       for (int q4 = 0; q4 < 4; ++q4) {
         uint32_t pk[16];
-        uint32_t keep_word = 0;  // dropout bytes of 4 keys of this row
+        uint32_t kw[4] = {0, 0, 0, 0};  // dropout bytes of this row: keys 4g..4g+3 of 16 in kw[g]
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const int c = q4 * 32 + 2 * i;
@@ -346,13 +346,28 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
           const uint64_t pp = f2pack(ex2_approx(f2lo(x)), ex2_approx(f2hi(x)));
           acc[i & 3] = add2(acc[i & 3], pp);  // l sums the undropped P
           if constexpr (DROP) {
-            if ((i & 1) == 0) {
+            if ((i & 7) == 0) {
+              // The 4 lanes of a quad hold 4 consecutive rows (one Philox
+              // counter row).  Lane g of the quad draws the 4x4 block of keys
+              // 4g..4g+3 of the next 16; four rotations of a shuffle give
+              // each lane its own row's word of all four blocks.
+              const int ql = lane & 3;
               const uint4 rnd = philox4x32_10(
-                  make_uint4(static_cast<uint32_t>((kv0 + c) >> 2), static_cast<uint32_t>(q_row >> 2),
+                  make_uint4(static_cast<uint32_t>((kv0 + c + 4 * ql) >> 2), static_cast<uint32_t>(q_row >> 2),
                              static_cast<uint32_t>(bh), 0u),
                   p.seed_lo, p.seed_hi);
-              keep_word = uint4_word(rnd, q_row & 3);
+#pragma unroll
+              for (int rr = 0; rr < 4; ++rr) {
+                const uint32_t got = __shfl_sync(0xffffffffu, uint4_word(rnd, (ql - rr) & 3),
+                                                 (lane & ~3) | ((ql + rr) & 3));
+                const int g = (ql + rr) & 3;
+                kw[0] = g == 0 ? got : kw[0];
+                kw[1] = g == 1 ? got : kw[1];
+                kw[2] = g == 2 ? got : kw[2];
+                kw[3] = g == 3 ? got : kw[3];
+              }
             }
+            const uint32_t keep_word = kw[(i >> 1) & 3];
             const uint32_t b0 = (keep_word >> (16 * (i & 1))) & 0xFFu;
             const uint32_t b1 = (keep_word >> (16 * (i & 1) + 8)) & 0xFFu;
             pk[i] = pack2<BF16>(b0 >= p.drop_t ? f2lo(pp) * p.drop_scale : 0.f,
