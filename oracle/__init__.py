@@ -100,6 +100,9 @@ class Oracle:
         lib.oracle_bwd_cols.argtypes = ([_dp, _dp, _dp, _dp, _i64, _i64, _ip, _i64, _dp, _dp]
                                         + common + [ctypes.c_int])
         lib.oracle_num_threads.argtypes = [ctypes.c_int]
+        lib.oracle_decode_paged.argtypes = ([_dp, _dp, _dp, _ip, _ip, _dp, _dp]
+                                            + [_i64] * 8 + [ctypes.c_double, ctypes.c_int])
+        lib.oracle_decode_paged.restype = ctypes.c_int
         lib.oracle_philox4x32_10.argtypes = [ctypes.POINTER(u32), ctypes.POINTER(u32), ctypes.POINTER(u32)]
         lib.oracle_philox4x32_10.restype = None
         for f in ("oracle_fwd", "oracle_fwd_rows", "oracle_fwd_online", "oracle_bwd",
@@ -206,6 +209,27 @@ class Oracle:
         return dk, dv
 
 
+    def decode_paged(self, q, k_cache, v_cache, block_table, seq_lens, scale: float,
+                     nthreads: int = 0):
+        """Decode over a paged cache: q [B,Hq,Nq,d], caches [pages,Hkv,P,d],
+        block_table [B,max_pages], seq_lens [B] -> O [B,Hq,Nq,d], lse [B,Hq,Nq]."""
+        q, kc, vc = _f64(q), _f64(k_cache), _f64(v_cache)
+        B, Hq, Nq, d = q.shape
+        num_pages, Hkv, P, dk = kc.shape
+        if dk != d or vc.shape != kc.shape or Hq % Hkv:
+            raise ValueError("incompatible shapes")
+        table = np.ascontiguousarray(np.asarray(block_table, dtype=np.int64).reshape(B, -1))
+        lens = np.ascontiguousarray(np.asarray(seq_lens, dtype=np.int64).reshape(B))
+        o = np.zeros((B, Hq, Nq, d))
+        lse = np.zeros((B, Hq, Nq))
+        rc = self.lib.oracle_decode_paged(_ptr(q), _ptr(kc), _ptr(vc), table.ctypes.data_as(_ip),
+                                          lens.ctypes.data_as(_ip), _ptr(o), _ptr(lse), B, Hq, Hkv,
+                                          Nq, d, P, table.shape[1], num_pages, float(scale), nthreads)
+        if rc:
+            raise ValueError(f"oracle_decode_paged rejected its arguments ({rc})")
+        return o, lse
+
+
 def default() -> Oracle:
     """The oracle compiled from oracle.c (built on first use)."""
     global _default
@@ -241,3 +265,7 @@ def bwd_rows(*a, **kw):
 
 def bwd_cols(*a, **kw):
     return default().bwd_cols(*a, **kw)
+
+
+def decode_paged(*a, **kw):
+    return default().decode_paged(*a, **kw)

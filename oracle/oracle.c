@@ -621,3 +621,71 @@ int oracle_bwd_cols(const double *q, const double *k, const double *v, const dou
     free(stats);
     return 0;
 }
+
+/* ------------------------------------------------------------------------ */
+/* Decode over a paged key/value cache (the serving workload of the pages:
+ * "Paper digest: FlashAttention", section "Limits", names decode-time
+ * attention over a KV cache; the "Flash Attention" glossary's PagedAttention
+ * entry stores that cache in fixed-size blocks found through a table).
+ * Sequence b holds seq_lens[b] = L cached tokens, its last Nq being the new
+ * queries: query t (position L - Nq + t) sees keys 0 .. L - Nq + t.  Key k of
+ * sequence b lives in physical page block_table[b][k / P], slot k % P.
+ *   q        [B][Hq][Nq][d]          o [B][Hq][Nq][d], lse [B][Hq][Nq]
+ *   k_cache  [num_pages][Hkv][P][d]  v_cache likewise
+ *   block_table [B][max_pages] (int64 here), seq_lens [B]
+ * Plain definition: gather the visible keys, two-pass softmax, O = P V.     */
+
+typedef struct {
+    const double *q, *kc, *vc;
+    const i64 *table, *lens;
+    double *o, *lse;
+    i64 B, Hq, Hkv, Nq, d, P, max_pages, num_pages;
+    double scale;
+} decode_t;
+
+static void decode_item(void *ctx, i64 item) {
+    const decode_t *D = (const decode_t *)ctx;
+    const i64 d = D->d, group = D->Hq / D->Hkv;
+    const i64 t = item % D->Nq, h = (item / D->Nq) % D->Hq, b = item / (D->Nq * D->Hq);
+    const i64 g = h / group, L = D->lens[b];
+    const i64 n_vis = L - D->Nq + t + 1; /* keys 0 .. L - Nq + t */
+    const double *qi = D->q + ((b * D->Hq + h) * D->Nq + t) * d;
+    double *oi = D->o + ((b * D->Hq + h) * D->Nq + t) * d;
+    double *s = (double *)malloc(sizeof(double) * (size_t)(n_vis > 0 ? n_vis : 1));
+    for (i64 kk = 0; kk < n_vis; ++kk) {
+        const i64 page = D->table[b * D->max_pages + kk / D->P], slot = kk % D->P;
+        const double *kr = D->kc + ((page * D->Hkv + g) * D->P + slot) * d;
+        s[kk] = D->scale * dot(qi, kr, d);
+    }
+    double m, l;
+    softmax_row_two_pass(s, n_vis, &m, &l);
+    D->lse[(b * D->Hq + h) * D->Nq + t] = m + log(l);
+    for (i64 c = 0; c < d; ++c) oi[c] = 0.0;
+    for (i64 kk = 0; kk < n_vis; ++kk) {
+        const i64 page = D->table[b * D->max_pages + kk / D->P], slot = kk % D->P;
+        const double *vr = D->vc + ((page * D->Hkv + g) * D->P + slot) * d;
+        for (i64 c = 0; c < d; ++c) oi[c] += s[kk] * vr[c];
+    }
+    free(s);
+}
+
+int oracle_decode_paged(const double *q, const double *k_cache, const double *v_cache,
+                        const i64 *block_table, const i64 *seq_lens, double *o, double *lse,
+                        i64 B, i64 Hq, i64 Hkv, i64 Nq, i64 d, i64 page_size, i64 max_pages,
+                        i64 num_pages, double scale, int nthreads) {
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || Nq <= 0 || d <= 0 || page_size <= 0 ||
+        max_pages < 0 || num_pages < 0)
+        return 1;
+    for (i64 b = 0; b < B; ++b) {
+        const i64 L = seq_lens[b];
+        if (L < Nq || L > max_pages * page_size) return 2;
+        for (i64 p = 0; p < (L + page_size - 1) / page_size; ++p) {
+            const i64 pg = block_table[b * max_pages + p];
+            if (pg < 0 || pg >= num_pages) return 2;
+        }
+    }
+    decode_t D = {q, k_cache, v_cache, block_table, seq_lens, o, lse,
+                  B, Hq, Hkv, Nq, d, page_size, max_pages, num_pages, scale};
+    if (B > 0) run_pool(decode_item, &D, B * Hq * Nq, nthreads);
+    return 0;
+}

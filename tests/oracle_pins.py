@@ -525,6 +525,70 @@ def pin_dropout_subsets_and_online(orc):
         _close(l2, lse, 1e-12, "dropout online lse")
 
 
+# -------------------------------------------------------- paged-decode pins
+
+def _paged_case(seed, B=3, Hq=4, Hkv=2, Nq=2, d=8, P=4, lens=(13, 7, 20), extra_pages=3):
+    """Contiguous K/V per sequence scattered into a shuffled page pool."""
+    r = _rng(seed)
+    max_pages = max((L + P - 1) // P for L in lens)
+    n_used = sum((L + P - 1) // P for L in lens)
+    num_pages = n_used + extra_pages
+    perm = r.permutation(num_pages)
+    kc = r.standard_normal((num_pages, Hkv, P, d))
+    vc = r.standard_normal((num_pages, Hkv, P, d))
+    table = np.full((B, max_pages), -1, dtype=np.int64)
+    k_seq, v_seq, used = [], [], 0
+    for b, L in enumerate(lens):
+        npg = (L + P - 1) // P
+        table[b, :npg] = perm[used:used + npg]
+        used += npg
+        kk = np.concatenate([kc[table[b, p]] for p in range(npg)], axis=1)[:, :L]  # [Hkv, L, d]
+        vv = np.concatenate([vc[table[b, p]] for p in range(npg)], axis=1)[:, :L]
+        k_seq.append(kk)
+        v_seq.append(vv)
+    q = r.standard_normal((B, Hq, Nq, d))
+    return q, kc, vc, table, np.array(lens), k_seq, v_seq
+
+
+def pin_decode_equals_contiguous_attention(orc):
+    """Decode over a paged cache equals the causal attention of the last Nq
+    rows of the contiguous sequence (the already-pinned row form)."""
+    q, kc, vc, table, lens, k_seq, v_seq = _paged_case(30)
+    B, Hq, Nq, d = q.shape
+    o, lse = orc.decode_paged(q, kc, vc, table, lens, 0.45)
+    for b, L in enumerate(lens):
+        qf = np.zeros((1, Hq, L, d))
+        qf[0, :, L - Nq:] = q[b]
+        rows = np.arange(L - Nq, L)
+        o_r, lse_r = orc.fwd_rows(qf, k_seq[b][None], v_seq[b][None], rows, 0.45, True)
+        _close(o[b], o_r[0], 1e-13, f"decode O seq {b}")
+        _close(lse[b], lse_r[0], 1e-13, f"decode lse seq {b}")
+
+
+def pin_decode_page_shuffle_and_q_zero(orc):
+    """Moving the pages of the pool (and the table with them) changes nothing;
+    Q = 0 gives the mean of the visible values and lse = ln(#visible)."""
+    q, kc, vc, table, lens, k_seq, v_seq = _paged_case(31, Nq=3, P=5, lens=(11, 3, 16))
+    o, lse = orc.decode_paged(q, kc, vc, table, lens, 0.6)
+    r = _rng(32)
+    perm = r.permutation(kc.shape[0])
+    inv = np.argsort(perm)
+    t2 = np.where(table >= 0, inv[np.maximum(table, 0)], -1)
+    o2, lse2 = orc.decode_paged(q, kc[perm], vc[perm], t2, lens, 0.6)
+    _close(o2, o, 0.0, "decode after moving pages")
+    _close(lse2, lse, 0.0, "decode lse after moving pages")
+    z = np.zeros_like(q)
+    oz, lz = orc.decode_paged(z, kc, vc, table, lens, 0.6)
+    B, Hq, Nq, d = q.shape
+    G = Hq // kc.shape[1]
+    for b, L in enumerate(lens):
+        for h in range(Hq):
+            for t in range(Nq):
+                n_vis = L - Nq + t + 1
+                _close(oz[b, h, t], v_seq[b][h // G, :n_vis].mean(axis=0), 1e-14, "decode O at Q=0")
+                assert abs(lz[b, h, t] - math.log(n_vis)) < 1e-14, "decode lse at Q=0"
+
+
 ALL_PINS = [
     pin_q_zero_noncausal, pin_q_zero_causal, pin_one_hot, pin_causal_row0,
     pin_rows_sum_to_one, pin_key_shift, pin_golden, pin_brute_force_python,
@@ -534,4 +598,5 @@ ALL_PINS = [
     pin_window_finite_differences, pin_window_subsets_and_online,
     pin_philox_known_answers, pin_dropout_off_and_keep_rate, pin_dropout_identity_readout,
     pin_dropout_torch, pin_dropout_finite_differences, pin_dropout_subsets_and_online,
+    pin_decode_equals_contiguous_attention, pin_decode_page_shuffle_and_q_zero,
 ]

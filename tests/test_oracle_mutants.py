@@ -28,6 +28,8 @@ MUTANTS = [
     ("cols_missing_group_sum", "for (i64 t = 0; t < C->group; ++t) {", "for (i64 t = 0; t < 1; ++t) {"),
     ("window_edge_off_by_one", "j <= i - P->window", "j < i - P->window"),
     ("philox_wrong_multiplier", "M1 = 0xCD9E8D57u", "M1 = 0xCD9E8D59u"),
+    ("decode_sees_one_key_too_few", "const i64 n_vis = L - D->Nq + t + 1;", "const i64 n_vis = L - D->Nq + t;"),
+    ("decode_slot_from_wrong_head", "((page * D->Hkv + g) * D->P + slot) * d;\n        s[kk]", "((page * D->Hkv + 0) * D->P + slot) * d;\n        s[kk]"),
     ("dropout_no_rescale", "256.0 / (256.0 - P->drop_t) : 0.0", "1.0 : 0.0"),
     ("dropout_word_byte_swapped", "(x[i & 3] >> (8 * (j & 3)))", "(x[j & 3] >> (8 * (i & 3)))"),
     ("dropout_dV_undropped_in_columns", "dvj[c] += p * f * doh[i * d + c];", "dvj[c] += p * doh[i * d + c];"),
