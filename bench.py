@@ -332,6 +332,75 @@ def run_ours(args, w, causal, rank, world, device):
     return line
 
 
+def run_decode(args, rank, world, device):
+    """Decode over a paged KV cache: B sequences of L cached tokens each, Nq
+    new query tokens, pages of 64 tokens scattered through the pool.  The
+    kernel pair is memory bound: value = cache bytes read per second."""
+    torch.cuda.set_device(device)
+    build()
+    binding.load()
+    B, Hq, Hkv, Nq, d, P, L = 32, 32, 8, 1, 128, 64, args.decode_len
+    dt = torch.bfloat16
+    npg = (L + P - 1) // P
+    num_pages = B * npg
+    g = torch.Generator(device=device).manual_seed(4321 + rank)
+    perm = torch.randperm(num_pages, generator=g, device=device).to(torch.int32)
+    table = perm.view(B, npg).contiguous()
+    lens = torch.full((B,), L, dtype=torch.int32, device=device)
+    kc = torch.randn((num_pages, Hkv, P, d), generator=g, device=device, dtype=torch.float32).to(dt)
+    vc = torch.randn((num_pages, Hkv, P, d), generator=g, device=device, dtype=torch.float32).to(dt)
+    q = torch.randn((B, Hq, Nq, d), generator=g, device=device, dtype=torch.float32).to(dt)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, Nq), device=device, dtype=torch.float32)
+    ws = torch.empty(binding.fa_decode_workspace_bytes(B, Hq, Hkv, Nq, d, npg), device=device,
+                     dtype=torch.uint8)
+    stream = torch.cuda.current_stream(device)
+    scale = 1.0 / math.sqrt(d)
+    step = lambda: binding.fa_decode_paged(q, kc, vc, table, lens, o, lse, scale, ws, stream)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    assert binding.fa_get_device_status(stream) == binding.FA_OK
+    K = args.steps
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(device) if rank == 0 else None
+    if clocks:
+        clocks.start()
+        time.sleep(0.3)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(device)
+    t0.record(stream)
+    for _ in range(K):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize(device)
+    clk = clocks.stop() if clocks else None
+    assert binding.fa_get_device_status(stream) == binding.FA_OK
+    ms = max_over_ranks(t0.elapsed_time(t1) / K, world, device)
+    cache_bytes = 2 * B * L * Hkv * d * 2                      # K and V read once
+    io_bytes = cache_bytes + 2 * q.numel() * 2 + lse.numel() * 4  # + q read, O and lse written
+    gbs = world * io_bytes / (ms * 1e-3) / 1e9
+    pk, pk_kind = peaks()
+    return {
+        "metric": "paged-KV decode: cache bytes read per second", "value": round(gbs, 1),
+        "unit": "GB/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bfloat16",
+        "data": "synthetic: seeded normals, pages of 64 tokens in a shuffled pool",
+        "config": {"workload": f"decode B={B} Hq={Hq} Hkv={Hkv} Nq={Nq} d={d} L={L} page=64",
+                   "parallelism": f"replicas x{world} (no exchange)",
+                   "l2": "cache larger than L2 (no flush)" if cache_bytes > 126e6 else "cache fits L2"},
+        "tokens_per_s": round(world * B * Nq / (ms * 1e-3), 1),
+        "roofline": {"kernel": "fa_decode_split_kernel + fa_decode_merge_kernel", "bound": "hbm",
+                     "achieved": round(gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                     "frac": round(gbs / pk["hbm_gbs"], 4), "peak_kind": f"{pk_kind} copy",
+                     "traffic": None, "algorithmic": "K and V cache read once, q read, O and lse written"},
+        "gpu_launches": 2 * K,
+        "clocks": clk,
+    }
+
+
 # ---------------------------------------------------------------- CPU oracle
 
 _ORACLE_INPUTS = {}
@@ -410,6 +479,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="mha4k", choices=sorted(WORKLOADS))
     ap.add_argument("--noncausal", action="store_true", help="non-causal variant of the workload")
+    ap.add_argument("--decode", action="store_true",
+                    help="time decode over a paged KV cache instead (B=32, Hq=32, Hkv=8, d=128)")
+    ap.add_argument("--decode-len", type=int, default=16384, help="cached tokens per sequence (--decode)")
     ap.add_argument("--dropout", type=float, default=0.0,
                     help="dropout probability on the attention probabilities (0: none)")
     ap.add_argument("--window", type=int, default=0,
@@ -446,6 +518,11 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=device)
     try:
+        if args.decode:
+            line = run_decode(args, rank, world, device)
+            if rank == 0:
+                print(json.dumps(line), flush=True)
+            return
         line = run_ours(args, w, causal, rank, world, device)
         if rank == 0 and not args.no_cpu_baseline and not args.window and not args.dropout:
             v, rows, dt, threads = oracle_sample(w, causal, args.cpu_seconds)

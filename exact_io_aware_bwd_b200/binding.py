@@ -63,6 +63,10 @@ def load():
             lib.fa_bwd_dropout.argtypes = ([vp] * 9 + [i, i, i, i, i, f, i, f, u64, i, vp,
                                                        ctypes.c_size_t, vp])
             lib.fa_bwd_dropout.restype = i
+            lib.fa_decode_workspace_bytes.argtypes = [i, i, i, i, i, i]
+            lib.fa_decode_workspace_bytes.restype = ctypes.c_size_t
+            lib.fa_decode_paged.argtypes = ([vp] * 7 + [i] * 8 + [f, i, vp, ctypes.c_size_t, vp])
+            lib.fa_decode_paged.restype = i
             lib.fa_get_device_status.argtypes = [vp]
             lib.fa_get_device_status.restype = i
             lib.fa_peek_device_status_word.argtypes = [vp]
@@ -203,7 +207,47 @@ def fa_set_bwd_max_blocks(max_blocks: int) -> None:
     _check(load().fa_set_bwd_max_blocks(int(max_blocks)), "fa_set_bwd_max_blocks")
 
 
+def fa_decode_workspace_bytes(B: int, Hq: int, Hkv: int, Nq: int, d: int, max_pages: int) -> int:
+    return int(load().fa_decode_workspace_bytes(B, Hq, Hkv, Nq, d, max_pages))
+
+
+def fa_decode_paged(q, k_cache, v_cache, block_table, seq_lens, o, lse, scale: float, workspace,
+                    stream=None) -> None:
+    """Decode over a paged cache: q [B,Hq,Nq,d]; caches [pages,Hkv,P,d];
+    block_table [B,max_pages] and seq_lens [B] int32 on the GPU."""
+    B, Hq, Nq, d = q.shape
+    num_pages, Hkv, P, dk = k_cache.shape
+    if dk != d or tuple(v_cache.shape) != tuple(k_cache.shape):
+        raise ValueError(f"incompatible shapes q{tuple(q.shape)} k_cache{tuple(k_cache.shape)}")
+    if block_table.dtype != torch.int32 or seq_lens.dtype != torch.int32:
+        raise ValueError("block_table and seq_lens must be int32")
+    for t in (q, k_cache, v_cache, block_table, seq_lens, o, lse):
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = load().fa_decode_paged(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
+                                _ptr(seq_lens), _ptr(o), _ptr(lse), B, Hq, Hkv, Nq, d, P,
+                                block_table.shape[1], num_pages, float(scale), _DTYPES[q.dtype],
+                                _ptr(workspace), ws_bytes, _stream(stream))
+    _check(st, "fa_decode_paged")
+
+
 # ------------------------------------------------------------ conveniences
+
+def attention_decode_paged(q, k_cache, v_cache, block_table, seq_lens, scale: float | None = None,
+                           stream=None):
+    """Allocates O, lse and the workspace and runs fa_decode_paged."""
+    B, Hq, Nq, d = q.shape
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, Nq), device=q.device, dtype=torch.float32)
+    ws = torch.empty(max(fa_decode_workspace_bytes(B, Hq, k_cache.shape[1], Nq, d,
+                                                   block_table.shape[1]), 16),
+                     device=q.device, dtype=torch.uint8)
+    fa_decode_paged(q, k_cache, v_cache, block_table, seq_lens, o, lse, scale, ws, stream)
+    return o, lse
+
+
 
 def attention_fwd(q, k, v, scale: float | None = None, causal: bool = False, stream=None,
                   window: int = 0, dropout=None):

@@ -16,6 +16,7 @@
 #include "sm100.cuh"
 #include "fa_fwd.cuh"
 #include "fa_bwd.cuh"
+#include "fa_decode.cuh"
 
 namespace {
 
@@ -402,7 +403,9 @@ fa_status_t fa_get_device_status(void* stream) {
   if (cudaMemcpyToSymbol(fa::g_device_status, &zero, sizeof(zero)) != cudaSuccess)
     return FA_ERR_CUDA;
   const uint32_t code = word & 0xFFu;
-  return code == fa::kStatusTimeout ? FA_ERR_TIMEOUT : FA_ERR_CUDA;
+  if (code == fa::kStatusTimeout) return FA_ERR_TIMEOUT;
+  if (code == fa::kStatusBadInput) return FA_ERR_INVALID_ARG;
+  return FA_ERR_CUDA;
 }
 
 uint32_t fa_peek_device_status_word(void* stream) {
@@ -437,6 +440,92 @@ fa_status_t fa_set_profile_events(int kernel_id, void* start, void* stop) {
   g_prof_start[kernel_id] = reinterpret_cast<cudaEvent_t>(start);
   g_prof_stop[kernel_id] = reinterpret_cast<cudaEvent_t>(stop);
   return FA_OK;
+}
+
+size_t fa_decode_workspace_bytes(int B, int Hq, int Hkv, int Nq, int d, int max_pages) {
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nq <= 0 || d <= 0 || max_pages <= 0) return 0;
+  return fa::decode_workspace_bytes(B, Hq, Hkv, Nq, d, max_pages);
+}
+
+fa_status_t fa_decode_paged(const void* q, const void* k_cache, const void* v_cache,
+                            const int* block_table, const int* seq_lens, void* o, float* lse, int B,
+                            int Hq, int Hkv, int Nq, int d, int page_size, int max_pages,
+                            int num_pages, float scale, fa_dtype_t dtype, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || Nq <= 0 || max_pages <= 0 ||
+      num_pages <= 0)
+    return FA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return FA_ERR_INVALID_ARG;
+  if (dtype != FA_BF16 && dtype != FA_FP16) return FA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (page_size != 16 && page_size != 32 && page_size != 64 && page_size != 128)
+    return FA_ERR_UNSUPPORTED;
+  if ((Hq / Hkv) * Nq > fa::kDecodeMaxRows) return FA_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(max_pages) * page_size > INT32_MAX) return FA_ERR_UNSUPPORTED;
+  if (B == 0) return FA_OK;
+  if (!q || !k_cache || !v_cache || !block_table || !seq_lens || !o || !lse || !workspace)
+    return FA_ERR_INVALID_ARG;
+  if (workspace_bytes < fa::decode_workspace_bytes(B, Hq, Hkv, Nq, d, max_pages))
+    return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) ||
+      !aligned16(workspace) || (reinterpret_cast<uintptr_t>(lse) & 3u) ||
+      (reinterpret_cast<uintptr_t>(block_table) & 3u) || (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
+    return FA_ERR_MISALIGNED;
+  fa_status_t s = check_device();
+  if (s != FA_OK) return s;
+  fa::DecodeParams prm;
+  std::memset(&prm, 0, sizeof(prm));
+  prm.q = q;
+  prm.kc = k_cache;
+  prm.vc = v_cache;
+  prm.table = block_table;
+  prm.lens = seq_lens;
+  prm.o = o;
+  prm.lse = lse;
+  prm.B = B;
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  prm.Nq = Nq;
+  prm.P = page_size;
+  prm.max_pages = max_pages;
+  prm.num_pages = num_pages;
+  prm.S = fa::decode_splits(B, Hkv, max_pages);
+  prm.pages_per_split = (max_pages + prm.S - 1) / prm.S;
+  prm.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  const int64_t rows = static_cast<int64_t>(B) * Hq * Nq;
+  prm.part_o = static_cast<float*>(workspace);
+  prm.part_ml = prm.part_o + rows * prm.S * d;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const bool bf = dtype == FA_BF16;
+  const dim3 grid(static_cast<unsigned>(prm.S), static_cast<unsigned>(Hkv), static_cast<unsigned>(B));
+  // the kernels are opted in once for the largest page size; a launch uses
+  // the bytes of its own page size
+  const int smem_max = d == 128 ? fa::DecodeLayout<128>(fa::kDecodeMaxPage).bytes
+                                : fa::DecodeLayout<64>(fa::kDecodeMaxPage).bytes;
+  auto run = [&](auto split_kern, auto merge_kern, int smem) -> fa_status_t {
+    fa_status_t r = opt_in_smem(split_kern, smem_max);
+    if (r != FA_OK) return r;
+    split_kern<<<grid, fa::kDecodeThreads, smem, st>>>(prm);
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+    merge_kern<<<static_cast<unsigned>(rows), d, 0, st>>>(prm);
+    return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+  };
+  const int R = (Hq / Hkv) * Nq;
+  const int rb = R <= 4 ? 4 : R <= 8 ? 8 : R <= 16 ? 16 : 32;
+  const int smem = d == 128 ? fa::DecodeLayout<128>(page_size).bytes : fa::DecodeLayout<64>(page_size).bytes;
+#define FA_DECODE_RUN(HD, BFV, RBV) \
+  run(fa::fa_decode_split_kernel<HD, BFV, RBV>, fa::fa_decode_merge_kernel<HD, BFV>, smem)
+#define FA_DECODE_RB(HD, BFV)                                                        \
+  (rb == 4 ? FA_DECODE_RUN(HD, BFV, 4) : rb == 8 ? FA_DECODE_RUN(HD, BFV, 8)        \
+             : rb == 16 ? FA_DECODE_RUN(HD, BFV, 16) : FA_DECODE_RUN(HD, BFV, 32))
+  fa_status_t rs;
+  if (d == 128)
+    rs = bf ? FA_DECODE_RB(128, true) : FA_DECODE_RB(128, false);
+  else
+    rs = bf ? FA_DECODE_RB(64, true) : FA_DECODE_RB(64, false);
+#undef FA_DECODE_RB
+#undef FA_DECODE_RUN
+  return rs;
 }
 
 fa_status_t fa_set_bwd_max_blocks(int max_blocks) {

@@ -153,10 +153,39 @@ fa_status_t fa_bwd_dropout(const void* q, const void* k, const void* v, const vo
                            size_t workspace_bytes, void* stream);
 
 /*
+ * Decode over a paged key/value cache ("Paper digest: FlashAttention",
+ * section "Limits": decode-time attention over a KV cache; "Flash Attention"
+ * glossary, PagedAttention entry: the cache lives in fixed-size blocks found
+ * through a table).  Sequence b holds L = seq_lens[b] cached tokens, the last
+ * Nq of which are the new queries: query t (position L - Nq + t) attends to
+ * keys 0 .. L - Nq + t.  Key k of sequence b is slot k % page_size of
+ * physical page block_table[b][k / page_size].
+ *   q        [B][Hq][Nq][d]                   o   [B][Hq][Nq][d] (same dtype)
+ *   k_cache, v_cache [num_pages][Hkv][page_size][d]   lse [B][Hq][Nq] fp32
+ *   block_table [B][max_pages] int32 (entries beyond a sequence's pages are
+ *   not read), seq_lens [B] int32; all device memory, caller-owned.
+ * The work is split along each sequence's pages and merged by logsumexp;
+ * workspace (device, 16-byte aligned) holds the partial results:
+ * fa_decode_workspace_bytes(B, Hq, Hkv, Nq, d, max_pages) bytes.
+ * Supported: d in {64, 128}, page_size in {16, 32, 64, 128},
+ * (Hq / Hkv) * Nq <= 32, bf16/fp16.  Host-side errors as fa_fwd; a
+ * seq_lens entry outside [Nq, max_pages * page_size] or a block-table
+ * entry outside [0, num_pages) is detected on the device (nothing out of
+ * range is read) and reported by fa_get_device_status as FA_ERR_INVALID_ARG.
+ */
+size_t fa_decode_workspace_bytes(int B, int Hq, int Hkv, int Nq, int d, int max_pages);
+fa_status_t fa_decode_paged(const void* q, const void* k_cache, const void* v_cache,
+                            const int* block_table, const int* seq_lens, void* o, float* lse,
+                            int B, int Hq, int Hkv, int Nq, int d, int page_size, int max_pages,
+                            int num_pages, float scale, fa_dtype_t dtype, void* workspace,
+                            size_t workspace_bytes, void* stream);
+
+/*
  * Synchronises `stream`, then returns and clears the first device-side error
  * any kernel of this library recorded on the current device since the last
  * call: FA_OK, or FA_ERR_TIMEOUT when a bounded barrier wait ran out (the
- * kernel then skipped its remaining work and its outputs are undefined).
+ * kernel then skipped its remaining work and its outputs are undefined), or
+ * FA_ERR_INVALID_ARG when fa_decode_paged met a bad table entry or length.
  * Returns FA_ERR_CUDA when the stream itself reports an error.
  */
 fa_status_t fa_get_device_status(void* stream);

@@ -151,3 +151,27 @@ def test_dropout_entry_points_accept_good_rates_on_empty_problems(lib):
     for p_drop in (0.0, 0.1, 0.5, 0.99):
         args = [vp(0)] * 5 + [0, 2, 2, 256, 64, 0.125, 1, p_drop, 7, binding.FA_BF16, None]
         assert lib.fa_fwd_dropout(*args) == binding.FA_OK
+
+
+def test_decode_argument_errors(lib):
+    vp = ctypes.c_void_p
+    ws = binding.fa_decode_workspace_bytes(2, 8, 2, 1, 128, 16)
+    assert ws > 0
+
+    def call(B=2, Hq=8, Hkv=2, Nq=1, d=128, P=64, max_pages=16, num_pages=40, scale=0.1,
+             dtype=binding.FA_BF16, ptrs=None, ws_bytes=ws):
+        p = ptrs if ptrs is not None else [FAKE] * 7
+        return lib.fa_decode_paged(*[vp(x) for x in p], B, Hq, Hkv, Nq, d, P, max_pages, num_pages,
+                                   scale, dtype, vp(FAKE), ws_bytes, None)
+
+    assert call(Hq=7) == binding.FA_ERR_INVALID_ARG
+    assert call(Nq=0) == binding.FA_ERR_INVALID_ARG
+    assert call(max_pages=0) == binding.FA_ERR_INVALID_ARG
+    assert call(scale=0.0) == binding.FA_ERR_INVALID_ARG
+    assert call(d=96) == binding.FA_ERR_UNSUPPORTED
+    assert call(P=48) == binding.FA_ERR_UNSUPPORTED
+    assert call(Hq=16, Hkv=1, Nq=4) == binding.FA_ERR_UNSUPPORTED      # 64 rows per kv head
+    assert call(ws_bytes=ws - 4) == binding.FA_ERR_INVALID_ARG
+    assert call(ptrs=[FAKE] * 6 + [0]) == binding.FA_ERR_INVALID_ARG
+    assert call(ptrs=[FAKE + 8] + [FAKE] * 6) == binding.FA_ERR_MISALIGNED
+    assert call(B=0, ptrs=[0] * 7) == binding.FA_OK

@@ -1,0 +1,87 @@
+"""Decode over a paged key/value cache on the GPU against the fp64 oracle:
+sequences of mixed lengths whose pages sit shuffled in a shared pool, MHA,
+GQA and MQA, bf16 and fp16, head dimension 64 and 128, page sizes 16-128,
+one to several new tokens; and the device-side check of bad table entries
+and lengths (reported, nothing out of range read)."""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import attn_check as ac
+import oracle
+from exact_io_aware_bwd_b200 import binding
+from exact_io_aware_bwd_b200.build import build
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def lib():
+    build()
+    binding.load()
+
+
+def make_case(seed, B, Hq, Hkv, Nq, d, P, lens, dtype, extra_pages=5):
+    g = torch.Generator("cpu").manual_seed(seed)
+    max_pages = max((L + P - 1) // P for L in lens) + 1     # a spare column, never read
+    n_used = sum((L + P - 1) // P for L in lens)
+    num_pages = n_used + extra_pages
+    perm = torch.randperm(num_pages, generator=g)
+    table = torch.full((B, max_pages), -1, dtype=torch.int32)
+    used = 0
+    for b, L in enumerate(lens):
+        npg = (L + P - 1) // P
+        table[b, :npg] = perm[used:used + npg].to(torch.int32)
+        used += npg
+    kc = torch.randn((num_pages, Hkv, P, d), generator=g).to(dtype)
+    vc = torch.randn((num_pages, Hkv, P, d), generator=g).to(dtype)
+    q = torch.randn((B, Hq, Nq, d), generator=g).to(dtype)
+    return q, kc, vc, table, torch.tensor(lens, dtype=torch.int32)
+
+
+CASES = [
+    # B, Hq, Hkv, Nq, d, P, lens, dtype
+    (3, 8, 2, 1, 128, 64, (1, 100, 1000), torch.bfloat16),
+    (2, 16, 1, 2, 128, 16, (37, 300), torch.bfloat16),          # MQA, 32 rows a kv head
+    (4, 4, 4, 1, 64, 32, (5, 64, 65, 500), torch.float16),
+    (2, 32, 8, 4, 128, 128, (129, 2048), torch.float16),       # GQA 4, 16 rows a kv head
+    (1, 8, 8, 3, 64, 128, (3,), torch.bfloat16),
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=[f"B{c[0]}-H{c[1]}/{c[2]}-Nq{c[3]}-d{c[4]}-P{c[5]}-{str(c[7])[6:]}"
+                                              for c in CASES])
+def test_decode_paged_parity(case):
+    B, Hq, Hkv, Nq, d, P, lens, dtype = case
+    q, kc, vc, table, seq_lens = make_case(sum(lens) + d + P, B, Hq, Hkv, Nq, d, P, lens, dtype)
+    scale = 1.0 / math.sqrt(d)
+    dev = "cuda:0"
+    o, lse = binding.attention_decode_paged(q.to(dev), kc.to(dev), vc.to(dev), table.to(dev),
+                                            seq_lens.to(dev), scale)
+    assert binding.fa_get_device_status() == binding.FA_OK
+    o_r, lse_r = oracle.decode_paged(q, kc, vc, table.numpy(), seq_lens.numpy(), scale)
+    o_a, _ = oracle.decode_paged(q, kc, vc.abs(), table.numpy(), seq_lens.numpy(), scale)
+    ac.check_o(o.cpu(), o_r, dtype, o_a, what="decode O")
+    ac.check_lse(lse.cpu(), lse_r, what="decode lse")
+
+
+@pytest.mark.parametrize("bad", ["page_id", "length"])
+def test_decode_bad_input_is_reported(bad):
+    q, kc, vc, table, seq_lens = make_case(9, 2, 4, 2, 1, 64, 16, (40, 20), torch.bfloat16)
+    if bad == "page_id":
+        table[1, 0] = kc.shape[0] + 3           # a page that does not exist
+    else:
+        seq_lens[0] = table.shape[1] * 16 + 1   # longer than the table can hold
+    dev = "cuda:0"
+    binding.attention_decode_paged(q.to(dev), kc.to(dev), vc.to(dev), table.to(dev), seq_lens.to(dev))
+    assert binding.fa_get_device_status() == binding.FA_ERR_INVALID_ARG
+    # the context is still usable
+    q, kc, vc, table, seq_lens = make_case(10, 1, 4, 2, 1, 64, 16, (33,), torch.bfloat16)
+    o, lse = binding.attention_decode_paged(q.to(dev), kc.to(dev), vc.to(dev), table.to(dev),
+                                            seq_lens.to(dev))
+    assert binding.fa_get_device_status() == binding.FA_OK
+    o_r, lse_r = oracle.decode_paged(q, kc, vc, table.numpy(), seq_lens.numpy(), 1 / 8)
+    ac.check_lse(lse.cpu(), lse_r, what="decode lse after an error")
