@@ -22,8 +22,9 @@
 // asynchronous 16-byte copies (cp.async), double-buffered so that the next
 // page is in flight while the current one is used; K rows are padded by 16
 // bytes so that one thread per key reads its row without bank conflicts.
-// Scores are one thread per key, the softmax update one warp per row, and
-// P V one thread per output column.
+// Scores take all 128 threads (128 / P threads per key, combined by
+// shuffles), the softmax update one warp per row, and P V one thread per
+// output column.
 #pragma once
 
 #include <type_traits>
@@ -163,16 +164,21 @@ __global__ void __launch_bounds__(kDecodeThreads) fa_decode_split_kernel(const _
     const int buf = (pg - pg0) & 1;
     const uint8_t* sK = smem + lay.off_k + buf * P * kKRow;
     const T* sV = reinterpret_cast<const T*>(smem + lay.off_v + buf * P * HD * 2);
-    // scores, one thread per key: s[r][j] = q_r . k_j (log2 units), -inf
-    // where hidden (after the query, past the sequence, or a bad page)
-    if (tid < P) {
-      const int key = pg * P + tid;
+    // scores: tpk = 128 / P threads per key, each over d / tpk features,
+    // summed across the key's threads by shuffles; s[r][j] = q_r . k_j (log2
+    // units), -inf where hidden (after the query, past the sequence, or a
+    // bad page)
+    {
+      const int tpk = kDecodeThreads / P;          // 1, 2, 4 or 8 (P = 128 .. 16)
+      const int j = tid / tpk, part = tid % tpk;   // the threads of a key are adjacent lanes
+      const int n8 = HD / 8 / tpk;                 // 16-byte chunks per thread
+      const int key = pg * P + j;
       float s[RB];
 #pragma unroll
       for (int r = 0; r < RB; ++r) s[r] = 0.f;
-      const uint8_t* kr = sK + tid * kKRow;
-#pragma unroll 4
-      for (int c8 = 0; c8 < HD / 8; ++c8) {
+      const uint8_t* kr = sK + j * kKRow;
+      for (int c = 0; c < n8; ++c) {
+        const int c8 = part * n8 + c;
         const uint4 kv = *reinterpret_cast<const uint4*>(kr + c8 * 16);
         const T* k8 = reinterpret_cast<const T*>(&kv);
         float kf[8];
@@ -188,12 +194,18 @@ __global__ void __launch_bounds__(kDecodeThreads) fa_decode_split_kernel(const _
           }
         }
       }
+      for (int off = 1; off < tpk; off <<= 1) {
 #pragma unroll
-      for (int r = 0; r < RB; ++r) {
-        if (r < R) {
-          const int t = r % p.Nq;
-          const bool vis = page_ok && key <= Lb - p.Nq + t;
-          sS[r * P + tid] = vis ? s[r] : -INFINITY;
+        for (int r = 0; r < RB; ++r) s[r] += __shfl_xor_sync(0xffffffffu, s[r], off);
+      }
+      if (part == 0) {
+#pragma unroll
+        for (int r = 0; r < RB; ++r) {
+          if (r < R) {
+            const int t = r % p.Nq;
+            const bool vis = page_ok && key <= Lb - p.Nq + t;
+            sS[r * P + j] = vis ? s[r] : -INFINITY;
+          }
         }
       }
     }
