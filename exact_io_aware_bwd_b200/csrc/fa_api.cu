@@ -75,29 +75,29 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 fa_status_t check_device() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
-  static int ok_dev[64] = {0};  // 0 unknown, 1 ok, 2 not ok
+  static std::atomic<int> ok_dev[64] = {};  // 0 unknown, 1 ok, 2 not ok (calls may race)
   if (dev < 0 || dev >= 64) return FA_ERR_UNSUPPORTED;
-  if (ok_dev[dev] == 0) {
+  if (ok_dev[dev].load() == 0) {
     int major = 0, minor = 0;
     if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
       return FA_ERR_CUDA;
-    ok_dev[dev] = (major == 10 && minor == 0) ? 1 : 2;
+    ok_dev[dev].store((major == 10 && minor == 0) ? 1 : 2);
   }
-  return ok_dev[dev] == 1 ? FA_OK : FA_ERR_UNSUPPORTED;
+  return ok_dev[dev].load() == 1 ? FA_OK : FA_ERR_UNSUPPORTED;
 }
 
 // Number of SMs of the current device (cached per device); 0 on error.
 int sm_count() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
-  static int n_sm[64] = {0};
-  if (n_sm[dev] == 0) {
+  static std::atomic<int> n_sm[64] = {};  // 0: not yet queried (calls may race)
+  if (n_sm[dev].load() == 0) {
     int n = 0;
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-    n_sm[dev] = n;
+    n_sm[dev].store(n);
   }
-  return n_sm[dev];
+  return n_sm[dev].load();
 }
 
 // Dropout probability -> 8-bit threshold t = round(256 p): a key is dropped
@@ -126,18 +126,25 @@ fa_status_t check_common(int B, int Hq, int Hkv, int N, int d, float scale, int 
   return FA_OK;
 }
 
-// Opt a kernel into `smem` bytes of dynamic shared memory (once per kernel).
+// Opt a kernel into `smem` bytes of dynamic shared memory, once per kernel
+// and device (the attribute belongs to the device's context).
 template <typename K>
 fa_status_t opt_in_smem(K kernel, int smem) {
   static std::mutex mu;
-  static const void* done[64];
+  static const void* done_fn[256];
+  static int done_dev[256];
   static int n_done = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
   std::lock_guard<std::mutex> lock(mu);
   for (int i = 0; i < n_done; ++i)
-    if (done[i] == reinterpret_cast<const void*>(kernel)) return FA_OK;
+    if (done_fn[i] == reinterpret_cast<const void*>(kernel) && done_dev[i] == dev) return FA_OK;
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return FA_ERR_CUDA;
-  if (n_done < 64) done[n_done++] = reinterpret_cast<const void*>(kernel);
+  if (n_done < 256) {
+    done_fn[n_done] = reinterpret_cast<const void*>(kernel);
+    done_dev[n_done++] = dev;
+  }
   return FA_OK;
 }
 
