@@ -175,3 +175,18 @@ def test_decode_argument_errors(lib):
     assert call(ptrs=[FAKE] * 6 + [0]) == binding.FA_ERR_INVALID_ARG
     assert call(ptrs=[FAKE + 8] + [FAKE] * 6) == binding.FA_ERR_MISALIGNED
     assert call(B=0, ptrs=[0] * 7) == binding.FA_OK
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    """No fallback: with the library absent the binding raises instead of
+    computing anything another way."""
+    import subprocess
+    import sys
+    code = ("import sys; sys.path.insert(0, %r)\n"
+            "from exact_io_aware_bwd_b200 import binding\n"
+            "try:\n    binding.load()\nexcept RuntimeError as e:\n    print('raised', e)\n"
+            % os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    env = dict(os.environ, FA_B200_LIB=str(tmp_path / "absent.so"))
+    r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0, r.stderr
+    assert "raised" in r.stdout and "no fallback" in r.stdout
