@@ -507,8 +507,8 @@ fa_status_t fa_decode_paged(const void* q, const void* k_cache, const void* v_ca
   const dim3 grid(static_cast<unsigned>(prm.S), static_cast<unsigned>(Hkv), static_cast<unsigned>(B));
   // the kernels are opted in once for the largest page size; a launch uses
   // the bytes of its own page size
-  const int smem_max = d == 128 ? fa::DecodeLayout<128>(fa::kDecodeMaxPage).bytes
-                                : fa::DecodeLayout<64>(fa::kDecodeMaxPage).bytes;
+  const int smem_max = d == 128 ? fa::DecodeLayout<128>(fa::kDecodeMaxPage, fa::kDecodeMaxRows).bytes
+                                : fa::DecodeLayout<64>(fa::kDecodeMaxPage, fa::kDecodeMaxRows).bytes;
   auto run = [&](auto split_kern, auto merge_kern, int smem) -> fa_status_t {
     fa_status_t r = opt_in_smem(split_kern, smem_max);
     if (r != FA_OK) return r;
@@ -519,7 +519,8 @@ fa_status_t fa_decode_paged(const void* q, const void* k_cache, const void* v_ca
   };
   const int R = (Hq / Hkv) * Nq;
   const int rb = R <= 4 ? 4 : R <= 8 ? 8 : R <= 16 ? 16 : 32;
-  const int smem = d == 128 ? fa::DecodeLayout<128>(page_size).bytes : fa::DecodeLayout<64>(page_size).bytes;
+  const int smem = d == 128 ? fa::DecodeLayout<128>(page_size, rb).bytes
+                            : fa::DecodeLayout<64>(page_size, rb).bytes;
 #define FA_DECODE_RUN(HD, BFV, RBV) \
   run(fa::fa_decode_split_kernel<HD, BFV, RBV>, fa::fa_decode_merge_kernel<HD, BFV>, smem)
 #define FA_DECODE_RB(HD, BFV)                                                        \

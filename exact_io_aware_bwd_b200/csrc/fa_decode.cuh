@@ -66,19 +66,21 @@ inline size_t decode_workspace_bytes(int B, int Hq, int Hkv, int Nq, int d, int 
   return static_cast<size_t>(rows) * 4u * static_cast<size_t>(d + 2);
 }
 
-// Shared memory for page size P (bytes, all offsets multiples of 16): two
-// page buffers (K padded, V), fp32 queries, fp32 scores [R][P], row state.
+// Shared memory for page size P and row bound RB (bytes, all offsets
+// multiples of 16): two page buffers (K padded, V), fp32 queries [RB][HD],
+// fp32 scores [RB][P], row state.  Sized by RB so that more blocks fit on an
+// SM when there are few rows.
 template <int HD>
 struct DecodeLayout {
   static constexpr int kKRow = HD * 2 + 16;  // padded K row, bytes
   int P, off_k, off_v, off_q, off_s, off_row, bytes;
-  __host__ __device__ explicit DecodeLayout(int page) : P(page) {
+  __host__ __device__ DecodeLayout(int page, int rb) : P(page) {
     const int kbuf = page * kKRow, vbuf = page * HD * 2;
     off_k = 0;                                   // K buffers 0, 1
     off_v = 2 * kbuf;                            // V buffers 0, 1
     off_q = off_v + 2 * vbuf;
-    off_s = off_q + kDecodeMaxRows * HD * 4;
-    off_row = off_s + kDecodeMaxRows * page * 4;
+    off_s = off_q + rb * HD * 4;
+    off_row = off_s + rb * page * 4;
     bytes = off_row + 3 * kDecodeMaxRows * 4;
   }
 };
@@ -95,7 +97,7 @@ __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_gr
 template <int HD, bool BF16, int RB>
 __global__ void __launch_bounds__(kDecodeThreads) fa_decode_split_kernel(const __grid_constant__ DecodeParams p) {
   using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
-  const DecodeLayout<HD> lay(p.P);
+  const DecodeLayout<HD> lay(p.P, RB);
   constexpr int kKRow = DecodeLayout<HD>::kKRow;
   extern __shared__ __align__(16) uint8_t smem[];
   float* sQ = reinterpret_cast<float*>(smem + lay.off_q);
