@@ -10,8 +10,8 @@
  *             "The Memory Bandwidth Bottleneck") and the method as tiles of
  *             Q, K, V streamed through on-chip memory with a running max and
  *             sum, writing only O back ("FlashAttention" glossary, opening
- *             list and online-softmax paragraph; same page, section
- *             "Flash Attention Algorithm", step 4).
+ *             list and online-softmax paragraph; "flash attention io
+ *             aware", section "Flash Attention Algorithm").
  *   backward  dQ, dK, dV from Q, K, V, O, dO and the logsumexp alone: the
  *             scores are recomputed on chip instead of being stored
  *             ("FlashAttention" glossary, recomputation paragraph).  dK and

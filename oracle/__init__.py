@@ -9,7 +9,7 @@ The arithmetic lives in ``oracle.c`` (plain C, fp64, one thread per
 independent head); this module compiles it with gcc on first use and wraps
 it for numpy arrays.  Every function follows the plain definition of
 attention given on the pages ("flash attention io aware", section "The
-Memory Bandwidth Bottleneck", steps 1-3: S = QK^T, P = softmax(S), O = PV),
+Memory Bandwidth Bottleneck": S = QK^T, P = softmax(S), O = PV),
 with the softmax statistics kept as one natural-log logsumexp per row
 ("FlashAttention" glossary, recomputation paragraph: the backward pass keeps
 only the normalisation statistics).  The backward formulas are the calculus

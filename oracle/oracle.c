@@ -8,7 +8,7 @@
  * What it computes (the plain definition, no blocking, no fusion):
  *   the pages define attention as S = QK^T, P = softmax(S) row by row,
  *   O = PV ("flash attention io aware", section "The Memory Bandwidth
- *   Bottleneck", steps 1-3), and say the tiled method reaches exactly this
+ *   Bottleneck"), and say the tiled method reaches exactly this
  *   result ("FlashAttention" glossary, online-softmax paragraph: output
  *   identical to the two-pass version).  The statistics kept for the
  *   backward pass are the running max m and sum l ("FlashAttention"
