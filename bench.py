@@ -43,9 +43,9 @@ PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of
-# the backward main kernel on the default workload, from the ncu capture
-# summarised in profiles/fa_bwd_kernel_mha4k.md, with a digest of the kernel
-# sources it was taken on: reported only while the sources are unchanged.
+# the backward main kernel on the default workload, from one ncu capture of
+# that kernel, with a digest of the kernel sources it was taken on: reported
+# only while the sources are unchanged.
 PROFILED_TRAFFIC = {"workload": "mha4k", "bytes": 1299325952, "sources_sha256_16": "9752b83a6347c5ae"}
 PROFILED_SOURCES = ("exact_io_aware_bwd_b200/csrc/fa_bwd.cuh", "exact_io_aware_bwd_b200/csrc/sm100.cuh")
 
