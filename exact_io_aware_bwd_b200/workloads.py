@@ -20,6 +20,11 @@ Recipe: a CPU ``torch.Generator`` seeded with ``1234 + 100 * index`` draws
 fp32 normals in the fixed order Q, K, V, dO; each is multiplied by its sigma
 and rounded to the I/O dtype (round to nearest even).  Row subsets for the
 large workloads come from ``randperm`` with the seed + 7.
+
+FP8 inputs (``make_fp8_inputs``) take the same fp32 draws of Q, K and V and
+quantise each tensor to E4M3 codes with one factor per tensor,
+delta = max|x| / 448 (448: the largest finite E4M3 value), code = E4M3(x / delta)
+rounded to nearest even by torch, so that the codes span the format's range.
 """
 
 from __future__ import annotations
@@ -108,6 +113,26 @@ def make_inputs(w: Workload, seed: int | None = None, device: str = "cpu",
     if device != "cpu":
         out = [t.to(device) for t in out]
     return out
+
+
+def make_fp8_inputs(w: Workload, seed: int | None = None, device: str = "cpu",
+                    shape_override: tuple | None = None):
+    """E4M3 codes of Q, K, V (uint8 tensors) and their factors (delta_q,
+    delta_k, delta_v): x is represented by delta * E4M3(code)."""
+    B, Hq, Hkv, N, d = shape_override or (w.B, w.Hq, w.Hkv, w.N, w.d)
+    g = torch.Generator("cpu").manual_seed(w.seed if seed is None else seed)
+    q = torch.randn((B, Hq, N, d), generator=g, dtype=torch.float32) * w.sigma_qk
+    k = torch.randn((B, Hkv, N, d), generator=g, dtype=torch.float32) * w.sigma_qk
+    v = torch.randn((B, Hkv, N, d), generator=g, dtype=torch.float32) * w.sigma_vdo
+    codes, factors = [], []
+    for x in (q, k, v):
+        amax = float(x.abs().max()) if x.numel() else 0.0
+        delta = torch.tensor(amax / 448.0 if amax > 0 else 1.0, dtype=torch.float32)
+        codes.append((x / delta).to(torch.float8_e4m3fn).view(torch.uint8))
+        factors.append(float(delta))
+    if device != "cpu":
+        codes = [c.to(device) for c in codes]
+    return codes, tuple(factors)
 
 
 def check_rows(w: Workload, N: int | None = None, seed: int | None = None) -> torch.Tensor:

@@ -20,6 +20,11 @@ Parity status of each function (what pins it, see tests/test_oracle_pins.py):
                          hand-derived golden values, torch fp64 SDPA,
                          brute-force Python loops
   fwd_online             equal to the two-pass form within 1e-12 (fp64)
+  e4m3_decode            every code against torch.float8_e4m3fn, values
+                         hand-derived from the format's definition
+  fwd_fp8, fwd_fp8_rows  closed form at Q = 0, torch fp64 SDPA on the
+                         dequantised values, moving a power of two between
+                         the query and key factors changes nothing
   bwd, bwd_rows,         central finite differences of the forward,
   bwd_cols               closed forms at Q = 0, torch fp64 autograd,
                          gradient invariants, hand-derived golden values
@@ -66,6 +71,20 @@ def _ptr(a: np.ndarray):
     return a.ctypes.data_as(_dp)
 
 
+def _codes(a) -> np.ndarray:
+    """8-bit codes (numpy uint8, or a torch uint8 / float8 CPU tensor) as contiguous uint8."""
+    if hasattr(a, "detach"):
+        import torch
+        a = a.detach().cpu()
+        if a.dtype != torch.uint8:
+            a = a.view(torch.uint8)
+        a = a.numpy()
+    a = np.asarray(a)
+    if a.dtype != np.uint8:
+        raise ValueError(f"expected 8-bit codes, got {a.dtype}")
+    return np.ascontiguousarray(a)
+
+
 def _dims(q, k):
     B, Hq, N, d = q.shape
     Bk, Hkv, Nk, dk = k.shape
@@ -105,6 +124,8 @@ class Oracle:
         lib.oracle_decode_paged.restype = ctypes.c_int
         lib.oracle_philox4x32_10.argtypes = [ctypes.POINTER(u32), ctypes.POINTER(u32), ctypes.POINTER(u32)]
         lib.oracle_philox4x32_10.restype = None
+        lib.oracle_e4m3_decode.argtypes = [ctypes.POINTER(ctypes.c_uint8), _i64, _dp]
+        lib.oracle_e4m3_decode.restype = None
         for f in ("oracle_fwd", "oracle_fwd_rows", "oracle_fwd_online", "oracle_bwd",
                   "oracle_bwd_rows", "oracle_bwd_cols", "oracle_num_threads"):
             getattr(lib, f).restype = ctypes.c_int
@@ -117,6 +138,28 @@ class Oracle:
         o = (ctypes.c_uint32 * 4)()
         self.lib.oracle_philox4x32_10(c, k, o)
         return [int(x) for x in o]
+
+    def e4m3_decode(self, codes) -> np.ndarray:
+        """The exact fp64 value of every E4M3 code (NaN for the NaN codes)."""
+        c = _codes(codes)
+        out = np.zeros(c.shape, dtype=np.float64)
+        self.lib.oracle_e4m3_decode(c.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)), c.size, _ptr(out))
+        return out
+
+    def _dequant(self, q8, k8, v8, descale):
+        dq, dk, dv = (float(x) for x in descale)
+        return self.e4m3_decode(q8) * dq, self.e4m3_decode(k8) * dk, self.e4m3_decode(v8) * dv
+
+    def fwd_fp8(self, q8, k8, v8, descale, scale: float, causal: bool, nthreads: int = 0):
+        """O and lse of attention on E4M3 inputs: the definition applied to
+        descale[0] * Q8, descale[1] * K8, descale[2] * V8 (exact in fp64)."""
+        q, k, v = self._dequant(q8, k8, v8, descale)
+        return self.fwd(q, k, v, scale, causal, nthreads)
+
+    def fwd_fp8_rows(self, q8, k8, v8, descale, rows, scale: float, causal: bool, nthreads: int = 0):
+        """``fwd_fp8`` for the query rows ``rows`` of every head."""
+        q, k, v = self._dequant(q8, k8, v8, descale)
+        return self.fwd_rows(q, k, v, rows, scale, causal, nthreads)
 
     def num_threads(self, nthreads: int = 0) -> int:
         """Threads the oracle uses for ``nthreads`` (<= 0: every online core)."""
@@ -269,3 +312,15 @@ def bwd_cols(*a, **kw):
 
 def decode_paged(*a, **kw):
     return default().decode_paged(*a, **kw)
+
+
+def e4m3_decode(*a, **kw):
+    return default().e4m3_decode(*a, **kw)
+
+
+def fwd_fp8(*a, **kw):
+    return default().fwd_fp8(*a, **kw)
+
+
+def fwd_fp8_rows(*a, **kw):
+    return default().fwd_fp8_rows(*a, **kw)

@@ -49,6 +49,14 @@
  * random numbers: as easy as 1, 2, 3", SC 2011) with key (seed_lo, seed_hi)
  * and counter (j / 4, i / 4, b * Hq + h, 0): byte j % 4 of output word i % 4.
  *
+ * FP8 forward (the FlashAttention-3 entry of the "FlashAttention" glossary
+ * names FP8 low-precision attention and gives no rule): Q, K and V arrive as
+ * 8-bit E4M3 codes with one fp32 dequantisation factor per tensor, and the
+ * result is the definition above applied to the dequantised values
+ * delta_q * Q8, delta_k * K8, delta_v * V8.  This file supplies the exact
+ * decode of the codes (oracle_e4m3_decode); the product delta * x of an E4M3
+ * value (4 significant bits) and an fp32 factor (24 bits) is exact in fp64.
+ *
  * Layouts: all arrays are dense row-major fp64.
  *   q, o, dout, dq : [B][Hq][N][d]
  *   k, v, dk, dv   : [B][Hkv][N][d]
@@ -66,6 +74,30 @@
 #include <unistd.h>
 
 typedef int64_t i64;
+
+/* ------------------------------------------------------------------------ */
+/* E4M3: the 8-bit float with 4 exponent and 3 fraction bits (the E4M3 format
+ * of the OCP 8-bit floating point specification, as NVIDIA's FP8 tensor cores
+ * take it).  Bit 7 is the sign; bits 6..3 hold the exponent field e with bias
+ * 7; bits 2..0 hold the fraction f.  e = 0 gives the subnormals (f / 8) * 2^-6,
+ * e = 1..15 gives (1 + f / 8) * 2^(e - 7), except that e = 15 with f = 7 is NaN.
+ * There is no infinity; the largest finite magnitude is 1.75 * 2^8 = 448.     */
+
+static double e4m3_value(uint8_t code) {
+    const int sign = code >> 7, e = (code >> 3) & 15, f = code & 7;
+    double mag;
+    if (e == 15 && f == 7)
+        return NAN;
+    if (e == 0)
+        mag = ldexp((double)f / 8.0, -6);
+    else
+        mag = ldexp(1.0 + (double)f / 8.0, e - 7);
+    return sign ? -mag : mag;
+}
+
+void oracle_e4m3_decode(const uint8_t *codes, i64 n, double *out) {
+    for (i64 i = 0; i < n; ++i) out[i] = e4m3_value(codes[i]);
+}
 
 /* ------------------------------------------------------------------------ */
 /* a minimal thread pool: run fn(ctx, item) for item in [0, n_items)          */

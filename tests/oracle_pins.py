@@ -589,6 +589,99 @@ def pin_decode_page_shuffle_and_q_zero(orc):
                 assert abs(lz[b, h, t] - math.log(n_vis)) < 1e-14, "decode lse at Q=0"
 
 
+# ------------------------------------------------------------------ FP8 pins
+
+# E4M3 values worked out by hand from the format: sign, 4-bit exponent with
+# bias 7, 3-bit fraction, subnormals (f/8)*2^-6, e=15 f=7 the only NaN.
+E4M3_HAND = {
+    0x00: 0.0, 0x01: 2.0 ** -9, 0x07: 7 * 2.0 ** -9, 0x08: 2.0 ** -6, 0x0F: 1.875 * 2.0 ** -6,
+    0x30: 0.5, 0x38: 1.0, 0x3C: 1.5, 0x40: 2.0, 0x77: 240.0, 0x7E: 448.0,
+    0x81: -(2.0 ** -9), 0xB8: -1.0, 0xFE: -448.0,
+}
+
+
+def pin_e4m3_decode(orc):
+    """Every E4M3 code decodes as torch.float8_e4m3fn does; hand values; the
+    two NaN codes; -0 keeps its sign."""
+    codes = np.arange(256, dtype=np.uint8)
+    got = orc.e4m3_decode(codes)
+    ref = torch.from_numpy(codes.copy()).view(torch.float8_e4m3fn).double().numpy()
+    assert np.array_equal(np.isnan(got), np.isnan(ref)), "E4M3 NaN codes"
+    fin = ~np.isnan(ref)
+    _close(got[fin], ref[fin], 0.0, "E4M3 decode against torch")
+    for c, val in E4M3_HAND.items():
+        assert got[c] == val, f"E4M3 code {c:#04x}: {got[c]!r} != {val!r}"
+    assert np.isnan(got[0x7F]) and np.isnan(got[0xFF]) and int(np.isnan(got).sum()) == 2
+    assert math.copysign(1.0, got[0x80]) == -1.0 and got[0x80] == 0.0, "E4M3 -0"
+
+
+def _fp8_case(seed, B=1, Hq=2, Hkv=2, N=9, d=8):
+    """Random finite E4M3 codes (NaN codes replaced) and per-tensor factors."""
+    r = _rng(seed)
+    def codes(shape):
+        c = r.integers(0, 256, size=shape, dtype=np.uint8)
+        c[(c & 0x7F) == 0x7F] = 0x38
+        return c
+    q8, k8, v8 = codes((B, Hq, N, d)), codes((B, Hkv, N, d)), codes((B, Hkv, N, d))
+    descale = (1.0 / 96.0, 1.0 / 160.0, 1.0 / 48.0)
+    return q8, k8, v8, descale
+
+
+def _torch_decode(codes):
+    return torch.from_numpy(np.ascontiguousarray(codes)).view(torch.float8_e4m3fn).double()
+
+
+def pin_fp8_q_zero(orc):
+    """Q8 = 0: O_i = delta_v * mean_j V8_j (causal: over j <= i), lse_i = ln(#keys)."""
+    _, k8, v8, ds = _fp8_case(40, N=11, d=6)
+    q8 = np.zeros((1, 2, 11, 6), dtype=np.uint8)
+    vv = _torch_decode(v8).numpy() * ds[2]
+    o, lse = orc.fwd_fp8(q8, k8, v8, ds, 0.3, False)
+    _close(o, np.broadcast_to(vv.mean(axis=2, keepdims=True), o.shape), 1e-13, "FP8 O at Q=0")
+    _close(lse, np.full(lse.shape, math.log(11)), 1e-13, "FP8 lse at Q=0")
+    o, lse = orc.fwd_fp8(q8, k8, v8, ds, 0.3, True)
+    prefix = np.cumsum(vv, axis=2) / np.arange(1, 12)[None, None, :, None]
+    _close(o, prefix, 1e-13, "FP8 causal O at Q=0")
+    _close(lse[0, 0], np.log(np.arange(1, 12)), 1e-13, "FP8 causal lse at Q=0")
+
+
+def pin_fp8_torch_sdpa(orc):
+    """FP8 forward against torch fp64 SDPA on torch's own dequantisation (GQA,
+    causal and not)."""
+    q8, k8, v8, ds = _fp8_case(41, Hq=4, Hkv=2, N=10, d=8)
+    q = _torch_decode(q8) * ds[0]
+    k = (_torch_decode(k8) * ds[1]).repeat_interleave(2, dim=1)
+    v = (_torch_decode(v8) * ds[2]).repeat_interleave(2, dim=1)
+    for causal in (False, True):
+        o, lse = orc.fwd_fp8(q8, k8, v8, ds, 0.35, causal)
+        ref = torch.nn.functional.scaled_dot_product_attention(q, k, v, is_causal=causal, scale=0.35)
+        s = (q @ k.transpose(-1, -2)) * 0.35
+        if causal:
+            s = s.masked_fill(torch.ones(10, 10, dtype=torch.bool).triu(1), float("-inf"))
+        _close(o, ref.numpy(), 1e-12, f"FP8 O vs torch (causal={causal})")
+        _close(lse, torch.logsumexp(s, dim=-1).numpy(), 1e-12, f"FP8 lse vs torch (causal={causal})")
+
+
+def pin_fp8_factor_moves(orc):
+    """A power of two moved from the query factor to the key factor changes
+    nothing; doubling the value factor doubles O and leaves lse alone; the
+    row form equals the full form."""
+    q8, k8, v8, ds = _fp8_case(42, Hq=2, Hkv=1, N=12, d=8)
+    o, lse = orc.fwd_fp8(q8, k8, v8, ds, 0.4, True)
+    o2, lse2 = orc.fwd_fp8(q8, k8, v8, (ds[0] * 4, ds[1] / 4, ds[2]), 0.4, True)
+    _close(o2, o, 0.0, "FP8 O after moving 4 from delta_q to delta_k")
+    _close(lse2, lse, 0.0, "FP8 lse after moving 4 from delta_q to delta_k")
+    o3, lse3 = orc.fwd_fp8(q8, k8, v8, (ds[0], ds[1], ds[2] * 2), 0.4, True)
+    _close(o3, 2 * o, 0.0, "FP8 O with delta_v doubled")
+    _close(lse3, lse, 0.0, "FP8 lse with delta_v doubled")
+    o4, lse4 = orc.fwd_fp8(q8, k8, v8, (ds[0] * 2, ds[1], ds[2]), 0.4, True)
+    assert float(np.max(np.abs(lse4 - lse))) > 1e-3, "FP8: delta_q must reach the scores"
+    rows = np.array([0, 5, 11])
+    o_r, lse_r = orc.fwd_fp8_rows(q8, k8, v8, ds, rows, 0.4, True)
+    _close(o_r, o[:, :, rows], 1e-13, "FP8 rows O")
+    _close(lse_r, lse[:, :, rows], 1e-13, "FP8 rows lse")
+
+
 ALL_PINS = [
     pin_q_zero_noncausal, pin_q_zero_causal, pin_one_hot, pin_causal_row0,
     pin_rows_sum_to_one, pin_key_shift, pin_golden, pin_brute_force_python,
@@ -599,4 +692,5 @@ ALL_PINS = [
     pin_philox_known_answers, pin_dropout_off_and_keep_rate, pin_dropout_identity_readout,
     pin_dropout_torch, pin_dropout_finite_differences, pin_dropout_subsets_and_online,
     pin_decode_equals_contiguous_attention, pin_decode_page_shuffle_and_q_zero,
+    pin_e4m3_decode, pin_fp8_q_zero, pin_fp8_torch_sdpa, pin_fp8_factor_moves,
 ]

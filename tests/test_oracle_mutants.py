@@ -34,6 +34,10 @@ MUTANTS = [
     ("dropout_word_byte_swapped", "(x[i & 3] >> (8 * (j & 3)))", "(x[j & 3] >> (8 * (i & 3)))"),
     ("dropout_dV_undropped_in_columns", "dvj[c] += p * f * doh[i * d + c];", "dvj[c] += p * doh[i * d + c];"),
     ("window_ignored_in_columns", "            if (hidden(P, i, j)) continue;", "            if (P->causal && j > i) continue;"),
+    ("e4m3_exponent_bias_8", "ldexp(1.0 + (double)f / 8.0, e - 7)", "ldexp(1.0 + (double)f / 8.0, e - 8)"),
+    ("e4m3_subnormal_as_normal", "mag = ldexp((double)f / 8.0, -6);", "mag = ldexp(1.0 + (double)f / 8.0, -6);"),
+    ("e4m3_no_nan_code", "if (e == 15 && f == 7)\n        return NAN;", "if (0)\n        return NAN;"),
+    ("e4m3_sign_dropped", "return sign ? -mag : mag;", "return mag;"),
 ]
 
 
@@ -49,6 +53,41 @@ def test_pins_catch_planted_mistake(tmp_path, name, old, new):
     for pin in oracle_pins.ALL_PINS:
         try:
             pin(orc)
+        except (AssertionError, ValueError, FloatingPointError) as e:
+            caught.append((pin.__name__, str(e)[:80]))
+            break
+    assert caught, f"no pin caught the planted mistake {name}"
+
+
+# Mistakes in the numpy-side wiring of the FP8 forward (the per-tensor
+# factors), planted in a subclass of the oracle.
+def _dequant_q_v_swapped(self, q8, k8, v8, descale):
+    dq, dk, dv = (float(x) for x in descale)
+    return self.e4m3_decode(q8) * dv, self.e4m3_decode(k8) * dk, self.e4m3_decode(v8) * dq
+
+
+def _dequant_no_value_factor(self, q8, k8, v8, descale):
+    dq, dk, dv = (float(x) for x in descale)
+    return self.e4m3_decode(q8) * dq, self.e4m3_decode(k8) * dk, self.e4m3_decode(v8)
+
+
+def _dequant_key_factor_twice(self, q8, k8, v8, descale):
+    dq, dk, dv = (float(x) for x in descale)
+    return self.e4m3_decode(q8) * dk, self.e4m3_decode(k8) * dk, self.e4m3_decode(v8) * dv
+
+
+PY_MUTANTS = [("fp8_q_v_factors_swapped", _dequant_q_v_swapped),
+              ("fp8_value_factor_dropped", _dequant_no_value_factor),
+              ("fp8_key_factor_for_queries", _dequant_key_factor_twice)]
+
+
+@pytest.mark.parametrize("name,dequant", PY_MUTANTS, ids=[m[0] for m in PY_MUTANTS])
+def test_pins_catch_planted_fp8_wiring_mistake(name, dequant):
+    mutant = type("MutantOracle", (oracle.Oracle,), {"_dequant": dequant})(oracle.build())
+    caught = []
+    for pin in oracle_pins.ALL_PINS:
+        try:
+            pin(mutant)
         except (AssertionError, ValueError, FloatingPointError) as e:
             caught.append((pin.__name__, str(e)[:80]))
             break
