@@ -401,6 +401,72 @@ def run_decode(args, rank, world, device):
     }
 
 
+def run_fp8(args, w, causal, rank, world, device):
+    """FP8 forward only: Q, K, V as E4M3 codes with per-tensor factors, O in
+    bf16.  FLOPs by the forward convention; roofline against the FP8 tensor
+    peak, taken as the measured bf16 peak times the nominal FP8:bf16 ratio 2."""
+    from exact_io_aware_bwd_b200.workloads import make_fp8_inputs
+    torch.cuda.set_device(device)
+    build()
+    binding.load()
+    (q8, k8, v8), descale = make_fp8_inputs(w, seed=rank_seed(w, rank))
+    q8, k8, v8 = (t.to(device) for t in (q8, k8, v8))
+    B, Hq, N, d = q8.shape
+    o = torch.empty((B, Hq, N, d), device=device, dtype=torch.bfloat16)
+    lse = torch.empty((B, Hq, N), device=device, dtype=torch.float32)
+    stream = torch.cuda.current_stream(device)
+    step = lambda: binding.fa_fwd_fp8(q8, k8, v8, o, lse, w.scale, descale, causal, stream)
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize(device)
+    assert binding.fa_get_device_status(stream) == binding.FA_OK
+    K = args.steps
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * K)]
+    for e in ev:
+        e.record(stream)  # creates the event handle the library records into
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(device) if rank == 0 else None
+    if clocks:
+        clocks.start()
+        time.sleep(0.3)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(device)
+    t0.record(stream)
+    for i in range(K):
+        binding.fa_set_profile_events(binding.KERNEL_FWD, ev[2 * i], ev[2 * i + 1])
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize(device)
+    binding.fa_set_profile_events(binding.KERNEL_FWD)
+    clk = clocks.stop() if clocks else None
+    assert binding.fa_get_device_status(stream) == binding.FA_OK
+    ms = max_over_ranks(t0.elapsed_time(t1) / K, world, device)
+    kern_ms = statistics.mean(ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(K))
+    flops = w.flops_fwd(causal)
+    value = job_tflops(world, flops, ms)
+    pk, pk_kind = peaks()
+    peak8 = 2.0 * pk["bf16_tflops"]
+    achieved = flops / (kern_ms * 1e-3) / 1e12
+    in_bytes = q8.numel() + k8.numel() + v8.numel()
+    return {
+        "metric": "FP8 attention forward TFLOPS/GPU", "value": round(value, 1), "unit": "TFLOPS",
+        "n_gpus": world, "steps": K, "warmup": max(args.warmup, 3), "ms_per_step": round(ms, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3",
+        "data": "synthetic: seeded normals quantised to E4M3 with per-tensor factors",
+        "config": {"workload": workload_desc(w, causal).replace(str(w.dtype).replace("torch.", ""),
+                                                                  "e4m3 in, bf16 out"),
+                   "parallelism": f"replicas x{world} (no exchange)",
+                   "l2": "inputs larger than L2 (no flush)" if in_bytes > 126e6 else "inputs fit L2"},
+        "roofline": {"kernel": "fa_fwd_fp8_kernel", "bound": "tensor", "achieved": round(achieved, 1),
+                     "peak": round(peak8, 1), "unit": "TFLOP/s", "frac": round(achieved / peak8, 4),
+                     "peak_kind": f"{pk_kind} bf16 burst x 2 (nominal FP8:bf16 ratio)",
+                     "traffic": None, "kernel_ms": round(kern_ms, 4)},
+        "gpu_launches": K,
+        "clocks": clk,
+    }
+
+
 # ---------------------------------------------------------------- CPU oracle
 
 _ORACLE_INPUTS = {}
@@ -482,6 +548,8 @@ def main():
     ap.add_argument("--decode", action="store_true",
                     help="time decode over a paged KV cache instead (B=32, Hq=32, Hkv=8, d=128)")
     ap.add_argument("--decode-len", type=int, default=16384, help="cached tokens per sequence (--decode)")
+    ap.add_argument("--fp8", action="store_true",
+                    help="time the FP8 forward (E4M3 Q, K, V; bf16 O) on the workload's shape")
     ap.add_argument("--dropout", type=float, default=0.0,
                     help="dropout probability on the attention probabilities (0: none)")
     ap.add_argument("--window", type=int, default=0,
@@ -518,8 +586,9 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=device)
     try:
-        if args.decode:
-            line = run_decode(args, rank, world, device)
+        if args.decode or args.fp8:
+            line = (run_decode(args, rank, world, device) if args.decode
+                    else run_fp8(args, w, causal, rank, world, device))
             if rank == 0:
                 print(json.dumps(line), flush=True)
             return

@@ -63,6 +63,8 @@ def load():
             lib.fa_bwd_dropout.argtypes = ([vp] * 9 + [i, i, i, i, i, f, i, f, u64, i, vp,
                                                        ctypes.c_size_t, vp])
             lib.fa_bwd_dropout.restype = i
+            lib.fa_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, f, f, f, i, i, vp]
+            lib.fa_fwd_fp8.restype = i
             lib.fa_decode_workspace_bytes.argtypes = [i, i, i, i, i, i]
             lib.fa_decode_workspace_bytes.restype = ctypes.c_size_t
             lib.fa_decode_paged.argtypes = ([vp] * 7 + [i] * 8 + [f, i, vp, ctypes.c_size_t, vp])
@@ -150,6 +152,32 @@ def fa_fwd_dropout(q, k, v, o, lse, scale: float, causal: bool, p_drop: float, s
                                float(scale), int(bool(causal)), float(p_drop),
                                int(seed) & 0xFFFFFFFFFFFFFFFF, _DTYPES[q.dtype], _stream(stream))
     _check(st, "fa_fwd_dropout")
+
+
+def fa_fwd_fp8(q8, k8, v8, o, lse, scale: float, descale, causal: bool, stream=None) -> None:
+    """FP8 forward: q8 [B,Hq,N,128], k8/v8 [B,Hkv,N,128] E4M3 codes (uint8 or
+    float8_e4m3fn tensors on the GPU), descale = (delta_q, delta_k, delta_v);
+    O (bf16 or fp16, its dtype picks the output type) and lse fp32."""
+    B, Hq, Hkv, N, d = _dims(q8, k8)
+    for t in (q8, k8, v8):
+        if t.element_size() != 1:
+            raise TypeError("fa_fwd_fp8 takes 8-bit E4M3 codes")
+    dq, dk, dv = (float(x) for x in descale)
+    st = load().fa_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(o), _ptr(lse), B, Hq, Hkv, N, d,
+                           float(scale), dq, dk, dv, int(bool(causal)), _DTYPES[o.dtype],
+                           _stream(stream))
+    _check(st, "fa_fwd_fp8")
+
+
+def attention_fwd_fp8(q8, k8, v8, descale, scale: float | None = None, causal: bool = False,
+                      out_dtype=torch.bfloat16, stream=None):
+    """Allocates O (out_dtype) and lse and runs fa_fwd_fp8; returns (O, lse)."""
+    B, Hq, Hkv, N, d = _dims(q8, k8)
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    o = torch.empty((B, Hq, N, d), device=q8.device, dtype=out_dtype)
+    lse = torch.empty((B, Hq, N), device=q8.device, dtype=torch.float32)
+    fa_fwd_fp8(q8, k8, v8, o, lse, scale, descale, causal, stream)
+    return o, lse
 
 
 def fa_bwd_dropout(q, k, v, o, dout, lse, dq, dk, dv, scale: float, causal: bool, p_drop: float,

@@ -15,6 +15,7 @@
 #include "fa.h"
 #include "sm100.cuh"
 #include "fa_fwd.cuh"
+#include "fa_fwd_fp8.cuh"
 #include "fa_bwd.cuh"
 #include "fa_decode.cuh"
 
@@ -167,6 +168,22 @@ fa_status_t launch_fwd_c(const FwdParams& prm, int causal, cudaStream_t st) {
   if (prm.drop_t > 0)
     return causal ? launch_fwd<HD, BF, true, true>(prm, st) : launch_fwd<HD, BF, false, true>(prm, st);
   return causal ? launch_fwd<HD, BF, true, false>(prm, st) : launch_fwd<HD, BF, false, false>(prm, st);
+}
+
+// The FP8 forward kernel; its launches are bracketed by the forward's
+// profiling events.
+template <bool OB, bool CA>
+fa_status_t launch_fwd_fp8(const fa::Fp8FwdParams& prm, cudaStream_t st) {
+  auto kern = fa::fa_fwd_fp8_kernel<OB, CA>;
+  const int smem = fa::Fp8FwdLayout::kDynSmem;
+  fa_status_t s = opt_in_smem(kern, smem);
+  if (s != FA_OK) return s;
+  const int grid = prm.n_pairs * prm.BH;
+  prof_begin(fa::kKernFwd, st);
+  kern<<<grid, fa::kFwdFp8Threads, smem, st>>>(prm);
+  const bool ok = cudaGetLastError() == cudaSuccess;
+  prof_end(fa::kKernFwd, st);
+  return ok ? FA_OK : FA_ERR_CUDA;
 }
 
 template <int HD, bool BF, bool CA, bool DR>
@@ -332,6 +349,49 @@ fa_status_t fa_fwd_dropout(const void* q, const void* k, const void* v, void* o,
   if (!drop_threshold(p_drop, &t)) return FA_ERR_INVALID_ARG;
   return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, causal, 0, static_cast<uint32_t>(t),
                   seed, dtype, stream);
+}
+
+fa_status_t fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                       int Hq, int Hkv, int N, int d, float scale, float descale_q,
+                       float descale_k, float descale_v, int causal, fa_dtype_t out_dtype,
+                       void* stream) {
+  bool empty = false;
+  fa_status_t s = check_common(B, Hq, Hkv, N, d, scale, causal, out_dtype, &empty);
+  if (s != FA_OK) return s;
+  for (float f : {descale_q, descale_k, descale_v})
+    if (!std::isfinite(f) || !(f > 0.f)) return FA_ERR_INVALID_ARG;
+  const double c = static_cast<double>(scale) * descale_q * descale_k * 1.4426950408889634;
+  if (!(c >= 1.2e-38) || c > 3.0e38) return FA_ERR_INVALID_ARG;  // a normal fp32 factor
+  if (d != 128) return FA_ERR_UNSUPPORTED;
+  if (empty) return FA_OK;
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return FA_ERR_MISALIGNED;
+  if ((s = check_device()) != FA_OK) return s;
+
+  const bool bf = out_dtype == FA_BF16;
+  const CUtensorMapDataType dt16 = bf ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  fa::Fp8FwdParams prm;
+  std::memset(&prm, 0, sizeof(prm));
+  const uint64_t BHq = static_cast<uint64_t>(B) * Hq, BHkv = static_cast<uint64_t>(B) * Hkv;
+  if (!make_map(&prm.tm_q, q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, 128, N, BHq, 128, 128) ||
+      !make_map(&prm.tm_k, k, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, 128, N, BHkv, 128, 128) ||
+      !make_map(&prm.tm_v, v, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, 128, N, BHkv, 128, 128) ||
+      !make_map(&prm.tm_o, o, dt16, 2, 128, N, BHq, 64, 128))
+    return FA_ERR_CUDA;
+  prm.lse = lse;
+  prm.N = N;
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  prm.group = Hq / Hkv;
+  prm.BH = static_cast<int>(BHq);
+  prm.n_pairs = (N + 255) / 256;
+  prm.n_ktiles = (N + 127) / 128;
+  prm.scale_log2 = static_cast<float>(c);
+  prm.delta_v = descale_v;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (causal) return bf ? launch_fwd_fp8<true, true>(prm, st) : launch_fwd_fp8<false, true>(prm, st);
+  return bf ? launch_fwd_fp8<true, false>(prm, st) : launch_fwd_fp8<false, false>(prm, st);
 }
 
 size_t fa_bwd_workspace_bytes(int B, int Hq, int Hkv, int N, int d) {

@@ -106,6 +106,30 @@ fa_status_t fa_fwd_dropout(const void* q, const void* k, const void* v, void* o,
                            float p_drop, uint64_t seed, fa_dtype_t dtype, void* stream);
 
 /*
+ * FP8 forward ("FlashAttention" glossary, FlashAttention-3 entry: attention
+ * on FP8 tensor cores; the pages give no rule, so the plainest one is taken).
+ * q [B][Hq][N][128], k and v [B][Hkv][N][128] hold 8-bit E4M3 codes (sign,
+ * 4-bit exponent with bias 7, 3-bit fraction; the value of code x times its
+ * factor is the input), one factor per tensor: descale_q, descale_k,
+ * descale_v.  Computes the forward of fa_fwd on the dequantised inputs:
+ *   s_ij = scale * descale_q * descale_k * sum_c q_ic k_jc   (masked as fa_fwd)
+ *   O_i  = descale_v * sum_j softmax(s_i.)_j v_j,   lse_i = logsumexp_j s_ij
+ * Both products run on E4M3 tensor-core operands with fp32 accumulation; the
+ * probabilities are rounded to E4M3 (relative error up to 2^-4 each) for the
+ * second product and the row sums are kept in fp32, so lse carries only the
+ * fp32 rounding of the 16-bit pass while O carries the E4M3 rounding of P.
+ * o [B][Hq][N][128] is written in out_dtype (FA_BF16 or FA_FP16); lse is fp32
+ * natural log.  Pointers are caller-owned device memory, 16-byte aligned.
+ * Errors: as fa_fwd; a factor that is not finite and > 0 (or whose product
+ * with scale overflows fp32) returns FA_ERR_INVALID_ARG; d != 128 returns
+ * FA_ERR_UNSUPPORTED.  No backward pass goes with it.
+ */
+fa_status_t fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse,
+                       int B, int Hq, int Hkv, int N, int d, float scale, float descale_q,
+                       float descale_k, float descale_v, int causal, fa_dtype_t out_dtype,
+                       void* stream);
+
+/*
  * Bytes of device scratch that fa_bwd needs for these sizes (0 for an empty
  * problem).  Linear in N: two fp32 values per query row (D_i = dO_i . O_i and
  * the logsumexp in base 2) plus an fp32 dQ accumulator [B][Hq][Np][d], with N

@@ -153,6 +153,30 @@ def test_dropout_entry_points_accept_good_rates_on_empty_problems(lib):
         assert lib.fa_fwd_dropout(*args) == binding.FA_OK
 
 
+def test_fp8_forward_argument_errors(lib):
+    vp = ctypes.c_void_p
+
+    def call(B=1, Hq=2, Hkv=2, N=256, d=128, scale=0.09, ds=(0.01, 0.02, 0.03), causal=1,
+             dtype=binding.FA_BF16, ptrs=None):
+        p = ptrs if ptrs is not None else [FAKE] * 5
+        return lib.fa_fwd_fp8(*[vp(x) for x in p], B, Hq, Hkv, N, d, scale, *ds, causal, dtype, None)
+
+    for bad in (0.0, -1.0, float("nan"), float("inf")):
+        for i in range(3):
+            ds = [0.01, 0.02, 0.03]
+            ds[i] = bad
+            assert call(ds=tuple(ds)) == binding.FA_ERR_INVALID_ARG, (i, bad)
+    assert call(ds=(1e30, 1e30, 1.0)) == binding.FA_ERR_INVALID_ARG   # scale * factors overflows
+    assert call(d=64) == binding.FA_ERR_UNSUPPORTED
+    assert call(dtype=7) == binding.FA_ERR_UNSUPPORTED
+    assert call(Hq=3) == binding.FA_ERR_INVALID_ARG
+    assert call(causal=2) == binding.FA_ERR_INVALID_ARG
+    assert call(ptrs=[FAKE] * 4 + [0]) == binding.FA_ERR_INVALID_ARG
+    assert call(ptrs=[FAKE + 8] + [FAKE] * 4) == binding.FA_ERR_MISALIGNED
+    assert call(B=0, ptrs=[0] * 5) == binding.FA_OK
+    assert call(N=0, ptrs=[0] * 5) == binding.FA_OK
+
+
 def test_decode_argument_errors(lib):
     vp = ctypes.c_void_p
     ws = binding.fa_decode_workspace_bytes(2, 8, 2, 1, 128, 16)
