@@ -46,22 +46,27 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # the backward main kernel on the default workload, from one ncu capture of
 # that kernel, with a digest of the kernel sources it was taken on: reported
 # only while the sources are unchanged.
-PROFILED_TRAFFIC = {"workload": "mha4k", "bytes": 1299325952, "sources_sha256_16": "9752b83a6347c5ae"}
-PROFILED_SOURCES = ("exact_io_aware_bwd_b200/csrc/fa_bwd.cuh", "exact_io_aware_bwd_b200/csrc/sm100.cuh")
+PROFILED_TRAFFIC = {"workload": "mha4k", "bytes": 1299325952, "sources_sha256_16": "9752b83a6347c5ae",
+                    "sources": ("exact_io_aware_bwd_b200/csrc/fa_bwd.cuh",
+                                "exact_io_aware_bwd_b200/csrc/sm100.cuh")}
+# The same for the FP8 forward kernel (one launch on the 4K-token MHA shape).
+PROFILED_TRAFFIC_FP8 = {"workload": "mha4k", "bytes": 307079936, "sources_sha256_16": "3b488718cb199377",
+                        "sources": ("exact_io_aware_bwd_b200/csrc/fa_fwd_fp8.cuh",
+                                    "exact_io_aware_bwd_b200/csrc/sm100.cuh")}
 
 
-def profiled_traffic(workload_name):
+def profiled_traffic(workload_name, spec=PROFILED_TRAFFIC):
     import hashlib
     h = hashlib.sha256()
     try:
-        for f in PROFILED_SOURCES:
+        for f in spec["sources"]:
             with open(os.path.join(ROOT, f), "rb") as fh:
                 h.update(fh.read())
     except OSError:
         return None
-    if workload_name != PROFILED_TRAFFIC["workload"] or h.hexdigest()[:16] != PROFILED_TRAFFIC["sources_sha256_16"]:
+    if workload_name != spec["workload"] or h.hexdigest()[:16] != spec["sources_sha256_16"]:
         return None
-    return PROFILED_TRAFFIC["bytes"]
+    return spec["bytes"]
 
 
 def peaks():
@@ -461,7 +466,9 @@ def run_fp8(args, w, causal, rank, world, device):
         "roofline": {"kernel": "fa_fwd_fp8_kernel", "bound": "tensor", "achieved": round(achieved, 1),
                      "peak": round(peak8, 1), "unit": "TFLOP/s", "frac": round(achieved / peak8, 4),
                      "peak_kind": f"{pk_kind} bf16 burst x 2 (nominal FP8:bf16 ratio)",
-                     "traffic": None, "kernel_ms": round(kern_ms, 4)},
+                     "traffic": profiled_traffic(w.name, PROFILED_TRAFFIC_FP8) if causal else None,
+                     "algorithmic_bytes": in_bytes + o.numel() * 2 + lse.numel() * 4,
+                     "kernel_ms": round(kern_ms, 4)},
         "gpu_launches": K,
         "clocks": clk,
     }
