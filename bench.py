@@ -50,7 +50,7 @@ PROFILED_TRAFFIC = {"workload": "mha4k", "bytes": 1299325952, "sources_sha256_16
                     "sources": ("exact_io_aware_bwd_b200/csrc/fa_bwd.cuh",
                                 "exact_io_aware_bwd_b200/csrc/sm100.cuh")}
 # The same for the FP8 forward kernel (one launch on the 4K-token MHA shape).
-PROFILED_TRAFFIC_FP8 = {"workload": "mha4k", "bytes": 307079936, "sources_sha256_16": "3b488718cb199377",
+PROFILED_TRAFFIC_FP8 = {"workload": "mha4k", "bytes": 307079936, "sources_sha256_16": "49abecf182bf2acc",
                         "sources": ("exact_io_aware_bwd_b200/csrc/fa_fwd_fp8.cuh",
                                     "exact_io_aware_bwd_b200/csrc/sm100.cuh")}
 

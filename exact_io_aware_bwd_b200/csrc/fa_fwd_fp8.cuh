@@ -2,14 +2,14 @@
 // codes with one dequantisation factor per tensor, O written in bf16 or fp16
 // and one logsumexp per row, as in the 16-bit forward.
 //
-// Method: the FlashAttention-3 entry of the "FlashAttention" glossary (and
-// the "Flash Attention" glossary's FA3 line) names FP8 low-precision tensor
-// cores for attention and gives no further rule.  The plainest reading, kept
-// here: both products run on FP8 operands with fp32 accumulation, scores
-// S = delta_q delta_k Q8 K8^T, probabilities P rounded to E4M3 for the second
-// product, O = delta_v (P V8) / l, with the running max and sum of the online
-// softmax exactly as in the 16-bit forward ("flash attention io aware",
-// section "Online Softmax").
+// Method: the FlashAttention-3 paragraph of the "FlashAttention" glossary
+// and section "Flash Attention 2 and 3" of "flash attention io aware" name
+// FP8 low-precision tensor cores for attention and give no further rule.
+// The plainest reading, kept here: both products run on FP8 operands with
+// fp32 accumulation, scores S = delta_q delta_k Q8 K8^T, probabilities P
+// rounded to E4M3 for the second product, O = delta_v (P V8) / l, with the
+// running max and sum of the online softmax exactly as in the 16-bit
+// forward ("flash attention io aware", section "Online Softmax").
 //
 // Structure (the 16-bit forward's, with 8-bit operand tiles): one thread block
 // per (batch, query head, pair of 128-row query blocks), 320 threads:

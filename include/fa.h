@@ -106,7 +106,7 @@ fa_status_t fa_fwd_dropout(const void* q, const void* k, const void* v, void* o,
                            float p_drop, uint64_t seed, fa_dtype_t dtype, void* stream);
 
 /*
- * FP8 forward ("FlashAttention" glossary, FlashAttention-3 entry: attention
+ * FP8 forward ("FlashAttention" glossary, FlashAttention-3 paragraph: attention
  * on FP8 tensor cores; the pages give no rule, so the plainest one is taken).
  * q [B][Hq][N][128], k and v [B][Hkv][N][128] hold 8-bit E4M3 codes (sign,
  * 4-bit exponent with bias 7, 3-bit fraction; the value of code x times its

@@ -49,7 +49,7 @@
  * random numbers: as easy as 1, 2, 3", SC 2011) with key (seed_lo, seed_hi)
  * and counter (j / 4, i / 4, b * Hq + h, 0): byte j % 4 of output word i % 4.
  *
- * FP8 forward (the FlashAttention-3 entry of the "FlashAttention" glossary
+ * FP8 forward (the FlashAttention-3 paragraph of the "FlashAttention" glossary
  * names FP8 low-precision attention and gives no rule): Q, K and V arrive as
  * 8-bit E4M3 codes with one fp32 dequantisation factor per tensor, and the
  * result is the definition above applied to the dequantised values
