@@ -37,3 +37,37 @@ def test_decode_workspace_bytes(B, Hq, Hkv, Nq, d, max_pages):
     S = splits(B, Hkv, max_pages)
     assert binding.fa_decode_workspace_bytes(B, Hq, Hkv, Nq, d, max_pages) == B * Hq * Nq * S * (d + 2) * 4
     assert binding.fa_decode_workspace_bytes(0, Hq, Hkv, Nq, d, max_pages) == 0
+
+
+def test_fp8_inputs_quantise_the_16bit_draws():
+    """The E4M3 inputs are the same seeded fp32 draws as the 16-bit inputs,
+    each tensor divided by max|x| / 448 and rounded to E4M3: the largest code
+    is 448 in magnitude, no code is NaN, and dequantised values are within
+    E4M3's half-ulp (2^-4 relative, 2^-10 absolute below 2^-6) of the draws."""
+    import torch
+    from exact_io_aware_bwd_b200.workloads import make_fp8_inputs, make_inputs
+    w = WORKLOADS["tiny"]
+    (q8, k8, v8), ds = make_fp8_inputs(w, seed=5, shape_override=(1, 2, 1, 40, 128))
+    g = torch.Generator("cpu").manual_seed(5)
+    draws = [torch.randn((1, 2, 40, 128), generator=g), torch.randn((1, 1, 40, 128), generator=g),
+             torch.randn((1, 1, 40, 128), generator=g)]
+    for c, delta, x in zip((q8, k8, v8), ds, draws):
+        assert c.dtype == torch.uint8 and c.shape == x.shape
+        val = c.view(torch.float8_e4m3fn).double()
+        assert not torch.isnan(val).any()
+        assert float(val.abs().max()) == 448.0
+        assert delta == float(torch.tensor(float(x.abs().max()) / 448.0, dtype=torch.float32))
+        y = x.double() / delta
+        err = (val - y).abs()
+        bound = torch.maximum(y.abs() * 2.0 ** -4, torch.full_like(y, 2.0 ** -10))
+        assert bool((err <= bound * (1 + 1e-6)).all())
+    # the same seed gives the same codes; the 16-bit inputs share the draws
+    again = make_fp8_inputs(w, seed=5, shape_override=(1, 2, 1, 40, 128))[0]
+    assert all(torch.equal(a, b) for a, b in zip((q8, k8, v8), again))
+    q16 = make_inputs(w, seed=5, shape_override=(1, 2, 1, 40, 128))[0]
+    assert torch.equal(q16, draws[0].to(w.dtype))
+
+
+def test_fp8_flops_follow_the_forward_convention():
+    w = WORKLOADS["mha4k"]
+    assert w.flops_fwd(True) == 4.0 * 4 * 32 * 4096 * 4096 * 128 / 2
