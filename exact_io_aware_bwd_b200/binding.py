@@ -107,8 +107,52 @@ def _check(status: int, where: str):
 
 
 def _dims(q, k):
+    if q.dim() != 4 or k.dim() != 4:
+        raise ValueError(f"q and k must be 4-D [B, H, N, d], got {tuple(q.shape)} and {tuple(k.shape)}")
     B, Hq, N, d = q.shape
     Hkv = k.shape[1]
+    return B, Hq, Hkv, N, d
+
+
+_E4M3 = (torch.uint8, torch.float8_e4m3fn)
+
+
+def _expect(where, *spec):
+    """Checks (name, tensor, shape, dtypes) entries before any pointer reaches
+    the library: the shape (None: any), the dtype (None: any), a dense
+    row-major layout, and one CUDA device for all.  The library reads every
+    tensor as dense rows, so a strided view would be read wrongly rather than
+    rejected there.  None and raw integer addresses pass through unchecked."""
+    spec = [(name, t, shape, dtypes) for name, t, shape, dtypes in spec
+            if t is not None and not isinstance(t, int)]
+    for name, t, shape, dtypes in spec:
+        if shape is not None and tuple(t.shape) != tuple(shape):
+            raise ValueError(f"{where}: {name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+        if dtypes is not None and t.dtype not in dtypes:
+            raise TypeError(f"{where}: {name} has dtype {t.dtype}, expected one of {list(dtypes)}")
+        if not t.is_contiguous():
+            raise ValueError(f"{where}: {name} must be contiguous")
+    dev = None
+    for name, t, _, _ in spec:
+        if not t.is_cuda:
+            raise ValueError(f"{where}: {name} must be on a CUDA device")
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError(f"{where}: all tensors must be on one device ({name} is on {t.device})")
+
+
+def _expect_attention(where, q, k, v, o, lse, dout=None, dq=None, dk=None, dv=None, workspace=None):
+    """_expect for the attention entry points; returns (B, Hq, Hkv, N, d)."""
+    B, Hq, Hkv, N, d = _dims(q, k)
+    if q.dtype not in _DTYPES:
+        raise TypeError(f"{where}: q has dtype {q.dtype}, expected bfloat16 or float16")
+    same = (q.dtype,)
+    qs, ks = (B, Hq, N, d), (B, Hkv, N, d)
+    _expect(where, ("q", q, qs, same), ("k", k, ks, same), ("v", v, ks, same), ("o", o, qs, same),
+            ("lse", lse, (B, Hq, N), (torch.float32,)), ("dout", dout, qs, same),
+            ("dq", dq, qs, same), ("dk", dk, ks, same), ("dv", dv, ks, same),
+            ("workspace", workspace, None, None))
     return B, Hq, Hkv, N, d
 
 
@@ -119,7 +163,7 @@ def fa_status_string(status: int) -> str:
 def fa_fwd(q, k, v, o, lse, scale: float, causal: bool, stream=None) -> None:
     """O and lse (natural log) of exact attention into the given tensors.
     q [B,Hq,N,d], k/v [B,Hkv,N,d] (bf16 or fp16, contiguous, on the GPU)."""
-    B, Hq, Hkv, N, d = _dims(q, k)
+    B, Hq, Hkv, N, d = _expect_attention("fa_fwd", q, k, v, o, lse)
     st = load().fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, N, d,
                        float(scale), int(bool(causal)), _DTYPES[q.dtype], _stream(stream))
     _check(st, "fa_fwd")
@@ -127,7 +171,7 @@ def fa_fwd(q, k, v, o, lse, scale: float, causal: bool, stream=None) -> None:
 
 def fa_fwd_window(q, k, v, o, lse, scale: float, window: int, stream=None) -> None:
     """Causal sliding-window forward: query i sees keys i-window+1 .. i."""
-    B, Hq, Hkv, N, d = _dims(q, k)
+    B, Hq, Hkv, N, d = _expect_attention("fa_fwd_window", q, k, v, o, lse)
     st = load().fa_fwd_window(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, N, d,
                               float(scale), int(window), _DTYPES[q.dtype], _stream(stream))
     _check(st, "fa_fwd_window")
@@ -136,7 +180,7 @@ def fa_fwd_window(q, k, v, o, lse, scale: float, window: int, stream=None) -> No
 def fa_bwd_window(q, k, v, o, dout, lse, dq, dk, dv, scale: float, window: int, workspace,
                   stream=None) -> None:
     """Backward of fa_fwd_window with the same window."""
-    B, Hq, Hkv, N, d = _dims(q, k)
+    B, Hq, Hkv, N, d = _expect_attention("fa_bwd_window", q, k, v, o, lse, dout, dq, dk, dv, workspace)
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     st = load().fa_bwd_window(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq),
                               _ptr(dk), _ptr(dv), B, Hq, Hkv, N, d, float(scale), int(window),
@@ -147,7 +191,7 @@ def fa_bwd_window(q, k, v, o, dout, lse, dq, dk, dv, scale: float, window: int, 
 def fa_fwd_dropout(q, k, v, o, lse, scale: float, causal: bool, p_drop: float, seed: int,
                    stream=None) -> None:
     """Forward with dropout on the probabilities (8-bit threshold round(256 p))."""
-    B, Hq, Hkv, N, d = _dims(q, k)
+    B, Hq, Hkv, N, d = _expect_attention("fa_fwd_dropout", q, k, v, o, lse)
     st = load().fa_fwd_dropout(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, N, d,
                                float(scale), int(bool(causal)), float(p_drop),
                                int(seed) & 0xFFFFFFFFFFFFFFFF, _DTYPES[q.dtype], _stream(stream))
@@ -159,9 +203,11 @@ def fa_fwd_fp8(q8, k8, v8, o, lse, scale: float, descale, causal: bool, stream=N
     float8_e4m3fn tensors on the GPU), descale = (delta_q, delta_k, delta_v);
     O (bf16 or fp16, its dtype picks the output type) and lse fp32."""
     B, Hq, Hkv, N, d = _dims(q8, k8)
-    for t in (q8, k8, v8):
-        if t.element_size() != 1:
-            raise TypeError("fa_fwd_fp8 takes 8-bit E4M3 codes")
+    if o is None or isinstance(o, int) or o.dtype not in _DTYPES:
+        raise TypeError("fa_fwd_fp8: o must be a bfloat16 or float16 tensor (its dtype picks the output type)")
+    _expect("fa_fwd_fp8", ("q8", q8, (B, Hq, N, d), _E4M3), ("k8", k8, (B, Hkv, N, d), _E4M3),
+            ("v8", v8, (B, Hkv, N, d), _E4M3), ("o", o, (B, Hq, N, d), None),
+            ("lse", lse, (B, Hq, N), (torch.float32,)))
     dq, dk, dv = (float(x) for x in descale)
     st = load().fa_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(o), _ptr(lse), B, Hq, Hkv, N, d,
                            float(scale), dq, dk, dv, int(bool(causal)), _DTYPES[o.dtype],
@@ -183,7 +229,7 @@ def attention_fwd_fp8(q8, k8, v8, descale, scale: float | None = None, causal: b
 def fa_bwd_dropout(q, k, v, o, dout, lse, dq, dk, dv, scale: float, causal: bool, p_drop: float,
                    seed: int, workspace, stream=None) -> None:
     """Backward of fa_fwd_dropout with the same p_drop and seed."""
-    B, Hq, Hkv, N, d = _dims(q, k)
+    B, Hq, Hkv, N, d = _expect_attention("fa_bwd_dropout", q, k, v, o, lse, dout, dq, dk, dv, workspace)
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     st = load().fa_bwd_dropout(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq),
                                _ptr(dk), _ptr(dv), B, Hq, Hkv, N, d, float(scale),
@@ -200,7 +246,7 @@ def fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, scale: float, causal: bool, worksp
            stream=None) -> None:
     """dQ, dK, dV into the given tensors; workspace: a uint8 GPU tensor of at
     least fa_bwd_workspace_bytes(...) bytes."""
-    B, Hq, Hkv, N, d = _dims(q, k)
+    B, Hq, Hkv, N, d = _expect_attention("fa_bwd", q, k, v, o, lse, dout, dq, dk, dv, workspace)
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     st = load().fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq),
                        _ptr(dk), _ptr(dv), B, Hq, Hkv, N, d, float(scale), int(bool(causal)),
@@ -249,9 +295,13 @@ def fa_decode_paged(q, k_cache, v_cache, block_table, seq_lens, o, lse, scale: f
         raise ValueError(f"incompatible shapes q{tuple(q.shape)} k_cache{tuple(k_cache.shape)}")
     if block_table.dtype != torch.int32 or seq_lens.dtype != torch.int32:
         raise ValueError("block_table and seq_lens must be int32")
-    for t in (q, k_cache, v_cache, block_table, seq_lens, o, lse):
-        if not t.is_contiguous():
-            raise ValueError("tensors must be contiguous")
+    if q.dtype not in _DTYPES:
+        raise TypeError(f"fa_decode_paged: q has dtype {q.dtype}, expected bfloat16 or float16")
+    same = (q.dtype,)
+    _expect("fa_decode_paged", ("q", q, None, same), ("k_cache", k_cache, None, same),
+            ("v_cache", v_cache, None, same), ("block_table", block_table, (B, block_table.shape[-1]), None),
+            ("seq_lens", seq_lens, (B,), None), ("o", o, (B, Hq, Nq, d), same),
+            ("lse", lse, (B, Hq, Nq), (torch.float32,)), ("workspace", workspace, None, None))
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     st = load().fa_decode_paged(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
                                 _ptr(seq_lens), _ptr(o), _ptr(lse), B, Hq, Hkv, Nq, d, P,
@@ -329,7 +379,7 @@ def fa_bwd_noalloc(q, k, v, o, dout, lse, dq, dk, dv, scale: float, causal: bool
         vp, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
         fn.argtypes = [vp] * 9 + [i, i, i, i, i, f, i, i, vp]
         fn.restype = i
-    B, Hq, Hkv, N, d = _dims(q, k)
+    B, Hq, Hkv, N, d = _expect_attention("fa_bwd_noalloc", q, k, v, o, lse, dout, dq, dk, dv)
     st = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
             _ptr(dv), B, Hq, Hkv, N, d, float(scale), int(bool(causal)), _DTYPES[q.dtype],
             _stream(stream))
