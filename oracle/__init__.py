@@ -25,6 +25,11 @@ Parity status of each function (what pins it, see tests/test_oracle_pins.py):
   fwd_fp8, fwd_fp8_rows  closed form at Q = 0, torch fp64 SDPA on the
                          dequantised values, moving a power of two between
                          the query and key factors changes nothing
+  block_mask= (every     a mask of ones changes nothing, block-diagonal masks
+  attention function)    split into independent problems, pure-Python loops,
+                         torch fp64 SDPA + autograd with the expanded mask,
+                         rows that see no block (O = 0, lse = -inf, no
+                         gradient), row/column/online forms agree
   bwd, bwd_rows,         central finite differences of the forward,
   bwd_cols               closed forms at Q = 0, torch fp64 autograd,
                          gradient invariants, hand-derived golden values
@@ -103,14 +108,39 @@ def _drop(dropout):
     return int(t), seed & 0xFFFFFFFF, seed >> 32
 
 
+def _bmask(block_mask, Hq: int, N: int):
+    """The C arguments (pointer, head stride, bq, bk) of block_mask = None or
+    (mask, bq, bk): mask [Tq, Tk] shared by every head, or [Hq, Tq, Tk], with
+    Tq = ceil(N / bq), Tk = ceil(N / bk); nonzero = the block is computed.
+    Returns (array to keep alive, arguments)."""
+    if block_mask is None:
+        return None, (None, 0, 0, 0)
+    mask, bq, bk = block_mask
+    bq, bk = int(bq), int(bk)
+    if bq <= 0 or bk <= 0:
+        raise ValueError("block sizes must be positive")
+    m = mask.detach().cpu().numpy() if hasattr(mask, "detach") else np.asarray(mask)
+    m = np.ascontiguousarray(m != 0, dtype=np.uint8)
+    Tq, Tk = -(-N // bq), -(-N // bk)
+    if m.shape == (Tq, Tk):
+        hstride = 0
+    elif m.shape == (Hq, Tq, Tk):
+        hstride = Tq * Tk
+    else:
+        raise ValueError(f"block mask of shape {m.shape}: expected ({Tq}, {Tk}) or ({Hq}, {Tq}, {Tk})")
+    return m, (m.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)), hstride, bq, bk)
+
+
 class Oracle:
     """numpy-facing wrapper of one compiled copy of the oracle library."""
 
     def __init__(self, lib_path: str):
         lib = ctypes.CDLL(lib_path)
         u32 = ctypes.c_uint32
-        # B, Hq, Hkv, N, d, scale, causal, window, drop_t, seed_lo, seed_hi
-        common = [_i64, _i64, _i64, _i64, _i64, ctypes.c_double, ctypes.c_int, _i64, ctypes.c_int, u32, u32]
+        # B, Hq, Hkv, N, d, scale, causal, window, drop_t, seed_lo, seed_hi,
+        # block mask, its head stride, block rows, block columns
+        common = [_i64, _i64, _i64, _i64, _i64, ctypes.c_double, ctypes.c_int, _i64, ctypes.c_int, u32, u32,
+                  ctypes.POINTER(ctypes.c_uint8), _i64, _i64, _i64]
         lib.oracle_fwd.argtypes = [_dp, _dp, _dp, _dp, _dp] + common + [ctypes.c_int]
         lib.oracle_fwd_rows.argtypes = [_dp, _dp, _dp, _ip, _i64, _dp, _dp] + common + [ctypes.c_int]
         lib.oracle_fwd_online.argtypes = [_dp, _dp, _dp, _dp, _dp] + common + [_i64, ctypes.c_int]
@@ -165,88 +195,100 @@ class Oracle:
         """Threads the oracle uses for ``nthreads`` (<= 0: every online core)."""
         return self.lib.oracle_num_threads(nthreads)
 
-    def fwd(self, q, k, v, scale: float, causal: bool, nthreads: int = 0, *, window: int = 0, dropout=None):
+    def fwd(self, q, k, v, scale: float, causal: bool, nthreads: int = 0, *, window: int = 0, dropout=None,
+            block_mask=None):
         """O [B,Hq,N,d] and lse [B,Hq,N] (natural log), materialising N x N per head."""
         q, k, v = _f64(q), _f64(k), _f64(v)
         B, Hq, Hkv, N, d = _dims(q, k)
+        keep, margs = _bmask(block_mask, Hq, N)
         o = np.zeros((B, Hq, N, d))
         lse = np.zeros((B, Hq, N))
         rc = self.lib.oracle_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
-                                 B, Hq, Hkv, N, d, float(scale), int(causal), int(window), *_drop(dropout), nthreads)
+                                 B, Hq, Hkv, N, d, float(scale), int(causal), int(window), *_drop(dropout),
+                                 *margs, nthreads)
         if rc:
             raise ValueError(f"oracle_fwd rejected its arguments ({rc})")
         return o, lse
 
     def fwd_rows(self, q, k, v, rows, scale: float, causal: bool, nthreads: int = 0, *,
-                 window: int = 0, dropout=None):
+                 window: int = 0, dropout=None, block_mask=None):
         """O and lse of the query rows ``rows`` of every head: [B,Hq,R,d], [B,Hq,R]."""
         q, k, v = _f64(q), _f64(k), _f64(v)
         B, Hq, Hkv, N, d = _dims(q, k)
+        keep, margs = _bmask(block_mask, Hq, N)
         rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
         R = rows.size
         o = np.zeros((B, Hq, R, d))
         lse = np.zeros((B, Hq, R))
         rc = self.lib.oracle_fwd_rows(_ptr(q), _ptr(k), _ptr(v), rows.ctypes.data_as(_ip), R,
                                       _ptr(o), _ptr(lse), B, Hq, Hkv, N, d, float(scale),
-                                      int(causal), int(window), *_drop(dropout), nthreads)
+                                      int(causal), int(window), *_drop(dropout), *margs, nthreads)
         if rc:
             raise ValueError(f"oracle_fwd_rows rejected its arguments ({rc})")
         return o, lse
 
     def fwd_online(self, q, k, v, scale: float, causal: bool, block: int = 128, nthreads: int = 0,
-                   *, window: int = 0, dropout=None):
+                   *, window: int = 0, dropout=None, block_mask=None):
         """O and lse by the one-pass blocked online softmax (not the definition)."""
         q, k, v = _f64(q), _f64(k), _f64(v)
         B, Hq, Hkv, N, d = _dims(q, k)
+        keep, margs = _bmask(block_mask, Hq, N)
         o = np.zeros((B, Hq, N, d))
         lse = np.zeros((B, Hq, N))
         rc = self.lib.oracle_fwd_online(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
-                                        B, Hq, Hkv, N, d, float(scale), int(causal), int(window), *_drop(dropout), int(block),
-                                        nthreads)
+                                        B, Hq, Hkv, N, d, float(scale), int(causal), int(window), *_drop(dropout),
+                                        *margs, int(block), nthreads)
         if rc:
             raise ValueError(f"oracle_fwd_online rejected its arguments ({rc})")
         return o, lse
 
-    def bwd(self, q, k, v, dout, scale: float, causal: bool, nthreads: int = 0, *, window: int = 0, dropout=None):
+    def bwd(self, q, k, v, dout, scale: float, causal: bool, nthreads: int = 0, *, window: int = 0, dropout=None,
+            block_mask=None):
         """dQ [B,Hq,N,d], dK, dV [B,Hkv,N,d] (dK, dV summed over each query group)."""
         q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
         B, Hq, Hkv, N, d = _dims(q, k)
+        keep, margs = _bmask(block_mask, Hq, N)
         dq = np.zeros((B, Hq, N, d))
         dk = np.zeros((B, Hkv, N, d))
         dv = np.zeros((B, Hkv, N, d))
         rc = self.lib.oracle_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(dq), _ptr(dk),
-                                 _ptr(dv), B, Hq, Hkv, N, d, float(scale), int(causal), int(window), *_drop(dropout), nthreads)
+                                 _ptr(dv), B, Hq, Hkv, N, d, float(scale), int(causal), int(window), *_drop(dropout),
+                                 *margs, nthreads)
         if rc:
             raise ValueError(f"oracle_bwd rejected its arguments ({rc})")
         return dq, dk, dv
 
     def bwd_rows(self, q, k, v, dout, rows, scale: float, causal: bool, nthreads: int = 0, *,
-                 window: int = 0, dropout=None):
+                 window: int = 0, dropout=None, block_mask=None):
         """dQ of the query rows ``rows`` of every head: [B,Hq,R,d]."""
         q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
         B, Hq, Hkv, N, d = _dims(q, k)
+        keep, margs = _bmask(block_mask, Hq, N)
         rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
         R = rows.size
         dq = np.zeros((B, Hq, R, d))
         rc = self.lib.oracle_bwd_rows(_ptr(q), _ptr(k), _ptr(v), _ptr(dout),
                                       rows.ctypes.data_as(_ip), R, _ptr(dq),
-                                      B, Hq, Hkv, N, d, float(scale), int(causal), int(window), *_drop(dropout), nthreads)
+                                      B, Hq, Hkv, N, d, float(scale), int(causal), int(window), *_drop(dropout),
+                                      *margs, nthreads)
         if rc:
             raise ValueError(f"oracle_bwd_rows rejected its arguments ({rc})")
         return dq
 
     def bwd_cols(self, q, k, v, dout, b: int, hkv: int, cols, scale: float, causal: bool,
-                 nthreads: int = 0, *, window: int = 0, dropout=None):
+                 nthreads: int = 0, *, window: int = 0, dropout=None, block_mask=None):
         """dK and dV of key rows ``cols`` of kv head (b, hkv): [C,d] each."""
         q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
         B, Hq, Hkv, N, d = _dims(q, k)
+        keep, margs = _bmask(block_mask, Hq, N)
         cols = np.ascontiguousarray(np.asarray(cols, dtype=np.int64))
         C = cols.size
         dk = np.zeros((C, d))
         dv = np.zeros((C, d))
         rc = self.lib.oracle_bwd_cols(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), int(b), int(hkv),
                                       cols.ctypes.data_as(_ip), C, _ptr(dk), _ptr(dv),
-                                      B, Hq, Hkv, N, d, float(scale), int(causal), int(window), *_drop(dropout), nthreads)
+                                      B, Hq, Hkv, N, d, float(scale), int(causal), int(window), *_drop(dropout),
+                                      *margs, nthreads)
         if rc:
             raise ValueError(f"oracle_bwd_cols rejected its arguments ({rc})")
         return dk, dv

@@ -21,12 +21,18 @@
  *             and, with a sliding window of W keys, -inf for j <= i - W
  *             (query i sees keys i-W+1 .. i: the banded pattern is the
  *             plainest instance of the block-sparse attention that the
- *             "FlashAttention" glossary's block-sparse entry describes)
+ *             "FlashAttention" glossary's block-sparse entry describes),
+ *             and, with a block mask M of blocks of bq query rows by bk
+ *             keys (the general form of that entry: blocks the mask hides
+ *             are skipped), -inf where M[h][i / bq][j / bk] = 0
  *     m_i   = max_j s_ij                                (pass 1)
  *     l_i   = sum_j exp(s_ij - m_i)                     (pass 2)
  *     P_ij  = exp(s_ij - m_i) / l_i
  *     O_i   = sum_j P_ij v_j
  *     lse_i = m_i + ln(l_i)
+ *   A row that sees no key at all (possible only under a block mask) has
+ *   P_i. = 0, O_i = 0 and lse_i = -inf, and contributes nothing to the
+ *   gradients.
  *
  *   Backward (the pages print no formula; this is the calculus of
  *   y = softmax(x) applied to the definition above, summed over the query
@@ -162,7 +168,25 @@ typedef struct {
     i64 b_sel, hkv_sel;
     /* online-softmax block size */
     i64 block;
+    /* block mask (NULL: none): key j visible to query i of query head h only
+     * when bmask[h * bm_hstride + (i / bm_bq) * bm_nbk + j / bm_bk] != 0 */
+    const uint8_t *bmask;
+    i64 bm_hstride, bm_bq, bm_bk, bm_nbk;
 } prob_t;
+
+/* Installs a block mask of bq x bk blocks ([Hq or 1][ceil(N/bq)][ceil(N/bk)]
+ * bytes, head stride hstride: 0 shares one mask among the heads).  P->N must
+ * be set.  Returns nonzero for an invalid description. */
+static int set_block_mask(prob_t *P, const uint8_t *bmask, i64 hstride, i64 bq, i64 bk) {
+    P->bmask = bmask;
+    if (!bmask) return 0;
+    if (bq <= 0 || bk <= 0 || hstride < 0) return 1;
+    P->bm_hstride = hstride;
+    P->bm_bq = bq;
+    P->bm_bk = bk;
+    P->bm_nbk = (P->N + bk - 1) / bk;
+    return 0;
+}
 
 static const double *head_ptr(const double *base, i64 b, i64 h, i64 H, i64 N, i64 d) {
     return base + ((b * H + h) * N) * d;
@@ -213,18 +237,20 @@ static double drop_factor(const prob_t *P, i64 bh, i64 i, i64 j) {
     return u8 >= (uint32_t)P->drop_t ? 256.0 / (256.0 - P->drop_t) : 0.0;
 }
 
-/* Key j is hidden from query i: after it under a causal mask, or W or more
- * keys before it under a sliding window of W keys. */
-static int hidden(const prob_t *P, i64 i, i64 j) {
-    return (P->causal && j > i) || (P->window > 0 && j <= i - P->window);
+/* Key j is hidden from query i of query head h: after it under a causal
+ * mask, W or more keys before it under a sliding window of W keys, or in a
+ * block that the block mask hides. */
+static int hidden(const prob_t *P, i64 h, i64 i, i64 j) {
+    return (P->causal && j > i) || (P->window > 0 && j <= i - P->window) ||
+           (P->bmask && !P->bmask[h * P->bm_hstride + (i / P->bm_bq) * P->bm_nbk + j / P->bm_bk]);
 }
 
 /* Scores of one query row against every key: s[j] = scale * q_i . k_j, with
  * -inf for masked keys.  Returns the number of unmasked keys. */
-static i64 score_row(const prob_t *P, const double *qi, const double *kh, i64 i, double *s) {
+static i64 score_row(const prob_t *P, i64 h, const double *qi, const double *kh, i64 i, double *s) {
     i64 n_valid = 0;
     for (i64 j = 0; j < P->N; ++j) {
-        if (hidden(P, i, j)) {
+        if (hidden(P, h, i, j)) {
             s[j] = -INFINITY;
         } else {
             s[j] = P->scale * dot(qi, kh + j * P->d, P->d);
@@ -234,11 +260,18 @@ static i64 score_row(const prob_t *P, const double *qi, const double *kh, i64 i,
     return n_valid;
 }
 
-/* Two-pass softmax of one row in place: s -> P.  Writes m and l. */
+/* Two-pass softmax of one row in place: s -> P.  Writes m and l.  A row
+ * with every score -inf (no visible key) gives P = 0, m = -inf, l = 0. */
 static void softmax_row_two_pass(double *s, i64 N, double *m_out, double *l_out) {
     double m = -INFINITY;
     for (i64 j = 0; j < N; ++j)
         if (s[j] > m) m = s[j]; /* pass 1: max */
+    if (m == -INFINITY) {
+        for (i64 j = 0; j < N; ++j) s[j] = 0.0;
+        *m_out = m;
+        *l_out = 0.0;
+        return;
+    }
     double l = 0.0;
     for (i64 j = 0; j < N; ++j) l += exp(s[j] - m); /* pass 2: sum */
     for (i64 j = 0; j < N; ++j) s[j] = exp(s[j] - m) / l;
@@ -260,7 +293,7 @@ static void fwd_full_item(void *ctx, i64 item) {
     double *lseh = P->lse + (b * P->Hq + h) * N;
 
     double *S = (double *)malloc(sizeof(double) * (size_t)(N * N));
-    for (i64 i = 0; i < N; ++i) score_row(P, qh + i * d, kh, i, S + i * N);
+    for (i64 i = 0; i < N; ++i) score_row(P, h, qh + i * d, kh, i, S + i * N);
     for (i64 i = 0; i < N; ++i) {
         double m, l;
         softmax_row_two_pass(S + i * N, N, &m, &l);
@@ -281,13 +314,15 @@ static void fwd_full_item(void *ctx, i64 item) {
 
 int oracle_fwd(const double *q, const double *k, const double *v, double *o, double *lse,
                i64 B, i64 Hq, i64 Hkv, i64 N, i64 d, double scale, int causal, i64 window,
-               int drop_t, uint32_t seed_lo, uint32_t seed_hi, int nthreads) {
+               int drop_t, uint32_t seed_lo, uint32_t seed_hi,
+               const uint8_t *bmask, i64 bm_hstride, i64 bm_bq, i64 bm_bk, int nthreads) {
     if (B < 0 || Hq <= 0 || Hkv <= 0 || N < 0 || d <= 0 || Hq % Hkv || window < 0 ||
         drop_t < 0 || drop_t > 255) return 1;
     prob_t P = {0};
     P.window = window; P.drop_t = drop_t; P.seed_lo = seed_lo; P.seed_hi = seed_hi;
     P.q = q; P.k = k; P.v = v; P.o = o; P.lse = lse;
     P.B = B; P.Hq = Hq; P.Hkv = Hkv; P.N = N; P.d = d; P.scale = scale; P.causal = causal;
+    if (set_block_mask(&P, bmask, bm_hstride, bm_bq, bm_bk)) return 1;
     if (N > 0) run_pool(fwd_full_item, &P, B * Hq, nthreads);
     return 0;
 }
@@ -308,7 +343,7 @@ static void fwd_rows_item(void *ctx, i64 item) {
     double *oi = P->o + (bh * P->nrows + r) * d;
 
     double *s = (double *)malloc(sizeof(double) * (size_t)N);
-    score_row(P, qi, kh, i, s);
+    score_row(P, h, qi, kh, i, s);
     double m, l;
     softmax_row_two_pass(s, N, &m, &l);
     P->lse[bh * P->nrows + r] = m + log(l);
@@ -325,7 +360,7 @@ static void fwd_rows_item(void *ctx, i64 item) {
 int oracle_fwd_rows(const double *q, const double *k, const double *v, const i64 *rows, i64 nrows,
                     double *o_rows, double *lse_rows, i64 B, i64 Hq, i64 Hkv, i64 N, i64 d,
                     double scale, int causal, i64 window, int drop_t,
-                    uint32_t seed_lo, uint32_t seed_hi, int nthreads) {
+                    uint32_t seed_lo, uint32_t seed_hi, const uint8_t *bmask, i64 bm_hstride, i64 bm_bq, i64 bm_bk, int nthreads) {
     if (B < 0 || Hq <= 0 || Hkv <= 0 || N < 0 || d <= 0 || Hq % Hkv || nrows < 0 || window < 0 ||
         drop_t < 0 || drop_t > 255)
         return 1;
@@ -335,6 +370,7 @@ int oracle_fwd_rows(const double *q, const double *k, const double *v, const i64
     P.window = window; P.drop_t = drop_t; P.seed_lo = seed_lo; P.seed_hi = seed_hi;
     P.q = q; P.k = k; P.v = v; P.o = o_rows; P.lse = lse_rows; P.rows = rows; P.nrows = nrows;
     P.B = B; P.Hq = Hq; P.Hkv = Hkv; P.N = N; P.d = d; P.scale = scale; P.causal = causal;
+    if (set_block_mask(&P, bmask, bm_hstride, bm_bq, bm_bk)) return 1;
     if (nrows > 0) run_pool(fwd_rows_item, &P, B * Hq * nrows, nthreads);
     return 0;
 }
@@ -367,7 +403,7 @@ static void fwd_online_item(void *ctx, i64 item) {
             double mb = -INFINITY;
             for (i64 t = 0; t < nb; ++t) {
                 const i64 j = j0 + t;
-                s[t] = hidden(P, i, j) ? -INFINITY : P->scale * dot(qh + i * d, kh + j * d, d);
+                s[t] = hidden(P, h, i, j) ? -INFINITY : P->scale * dot(qh + i * d, kh + j * d, d);
                 if (s[t] > mb) mb = s[t];
             }
             if (mb == -INFINITY) continue; /* block fully masked */
@@ -384,6 +420,10 @@ static void fwd_online_item(void *ctx, i64 item) {
             }
             m = m_new;
         }
+        if (l == 0.0) { /* no visible key: O = 0, lse = -inf */
+            lseh[i] = -INFINITY;
+            continue;
+        }
         for (i64 c = 0; c < d; ++c) acc[c] /= l;
         lseh[i] = m + log(l);
     }
@@ -392,7 +432,8 @@ static void fwd_online_item(void *ctx, i64 item) {
 
 int oracle_fwd_online(const double *q, const double *k, const double *v, double *o, double *lse,
                       i64 B, i64 Hq, i64 Hkv, i64 N, i64 d, double scale, int causal, i64 window,
-                      int drop_t, uint32_t seed_lo, uint32_t seed_hi, i64 block, int nthreads) {
+                      int drop_t, uint32_t seed_lo, uint32_t seed_hi, const uint8_t *bmask, i64 bm_hstride, i64 bm_bq, i64 bm_bk, 
+                      i64 block, int nthreads) {
     if (B < 0 || Hq <= 0 || Hkv <= 0 || N < 0 || d <= 0 || Hq % Hkv || block <= 0 || window < 0 ||
         drop_t < 0 || drop_t > 255)
         return 1;
@@ -400,6 +441,7 @@ int oracle_fwd_online(const double *q, const double *k, const double *v, double 
     P.window = window; P.drop_t = drop_t; P.seed_lo = seed_lo; P.seed_hi = seed_hi;
     P.q = q; P.k = k; P.v = v; P.o = o; P.lse = lse; P.block = block;
     P.B = B; P.Hq = Hq; P.Hkv = Hkv; P.N = N; P.d = d; P.scale = scale; P.causal = causal;
+    if (set_block_mask(&P, bmask, bm_hstride, bm_bq, bm_bk)) return 1;
     if (N > 0) run_pool(fwd_online_item, &P, B * Hq, nthreads);
     return 0;
 }
@@ -428,7 +470,7 @@ static void bwd_full_item(void *ctx, i64 item) {
         /* recompute P from the definition */
         for (i64 i = 0; i < N; ++i) {
             double m, l;
-            score_row(P, qh + i * d, kh, i, Pm + i * N);
+            score_row(P, h, qh + i * d, kh, i, Pm + i * N);
             softmax_row_two_pass(Pm + i * N, N, &m, &l);
         }
         /* dP = dO V^T, times the dropout factor (dP of P, not of P') */
@@ -470,13 +512,14 @@ static void bwd_full_item(void *ctx, i64 item) {
 int oracle_bwd(const double *q, const double *k, const double *v, const double *dout, double *dq,
                double *dk, double *dv, i64 B, i64 Hq, i64 Hkv, i64 N, i64 d, double scale,
                int causal, i64 window, int drop_t, uint32_t seed_lo, uint32_t seed_hi,
-               int nthreads) {
+               const uint8_t *bmask, i64 bm_hstride, i64 bm_bq, i64 bm_bk, int nthreads) {
     if (B < 0 || Hq <= 0 || Hkv <= 0 || N < 0 || d <= 0 || Hq % Hkv || window < 0 ||
         drop_t < 0 || drop_t > 255) return 1;
     prob_t P = {0};
     P.window = window; P.drop_t = drop_t; P.seed_lo = seed_lo; P.seed_hi = seed_hi;
     P.q = q; P.k = k; P.v = v; P.dout = dout; P.dq = dq; P.dk = dk; P.dv = dv;
     P.B = B; P.Hq = Hq; P.Hkv = Hkv; P.N = N; P.d = d; P.scale = scale; P.causal = causal;
+    if (set_block_mask(&P, bmask, bm_hstride, bm_bq, bm_bk)) return 1;
     if (N > 0) run_pool(bwd_full_item, &P, B * Hkv, nthreads);
     return 0;
 }
@@ -500,7 +543,7 @@ static void bwd_rows_item(void *ctx, i64 item) {
     double *p = (double *)malloc(sizeof(double) * (size_t)N);
     double *dp = (double *)malloc(sizeof(double) * (size_t)N);
     double m, l;
-    score_row(P, qi, kh, i, p);
+    score_row(P, h, qi, kh, i, p);
     softmax_row_two_pass(p, N, &m, &l);
     double D = 0.0;
     for (i64 j = 0; j < N; ++j) {
@@ -523,7 +566,7 @@ static void bwd_rows_item(void *ctx, i64 item) {
 int oracle_bwd_rows(const double *q, const double *k, const double *v, const double *dout,
                     const i64 *rows, i64 nrows, double *dq_rows, i64 B, i64 Hq, i64 Hkv, i64 N,
                     i64 d, double scale, int causal, i64 window, int drop_t,
-                    uint32_t seed_lo, uint32_t seed_hi, int nthreads) {
+                    uint32_t seed_lo, uint32_t seed_hi, const uint8_t *bmask, i64 bm_hstride, i64 bm_bq, i64 bm_bk, int nthreads) {
     if (B < 0 || Hq <= 0 || Hkv <= 0 || N < 0 || d <= 0 || Hq % Hkv || nrows < 0 || window < 0 ||
         drop_t < 0 || drop_t > 255)
         return 1;
@@ -533,6 +576,7 @@ int oracle_bwd_rows(const double *q, const double *k, const double *v, const dou
     P.window = window; P.drop_t = drop_t; P.seed_lo = seed_lo; P.seed_hi = seed_hi;
     P.q = q; P.k = k; P.v = v; P.dout = dout; P.dq = dq_rows; P.rows = rows; P.nrows = nrows;
     P.B = B; P.Hq = Hq; P.Hkv = Hkv; P.N = N; P.d = d; P.scale = scale; P.causal = causal;
+    if (set_block_mask(&P, bmask, bm_hstride, bm_bq, bm_bk)) return 1;
     if (nrows > 0) run_pool(bwd_rows_item, &P, B * Hq * nrows, nthreads);
     return 0;
 }
@@ -564,7 +608,7 @@ static void col_stats_item(void *ctx, i64 item) {
     const double *vh = head_ptr(P->v, b, g, P->Hkv, N, d);
     double *p = (double *)malloc(sizeof(double) * (size_t)N);
     double m, l;
-    score_row(P, qi, kh, i, p);
+    score_row(P, h, qi, kh, i, p);
     softmax_row_two_pass(p, N, &m, &l);
     double D = 0.0;
     for (i64 j = 0; j < N; ++j)
@@ -596,7 +640,7 @@ static void col_sum_item(void *ctx, i64 r) {
         const double *qh = head_ptr(P->q, b, S->h, P->Hq, N, d);
         const double *doh = head_ptr(P->dout, b, S->h, P->Hq, N, d);
         for (i64 i = S->i_lo; i < N; ++i) {
-            if (hidden(P, i, j)) continue;
+            if (hidden(P, S->h, i, j)) continue;
             const double s = P->scale * dot(qh + i * d, kj, d);
             const double p = exp(s - S->m[i]) / S->l[i];
             const double f = drop_factor(P, b * P->Hq + S->h, i, j);
@@ -615,7 +659,7 @@ int oracle_bwd_cols(const double *q, const double *k, const double *v, const dou
                     i64 b_sel, i64 hkv_sel, const i64 *cols, i64 ncols, double *dk_cols,
                     double *dv_cols, i64 B, i64 Hq, i64 Hkv, i64 N, i64 d, double scale,
                     int causal, i64 window, int drop_t, uint32_t seed_lo, uint32_t seed_hi,
-               int nthreads) {
+                    const uint8_t *bmask, i64 bm_hstride, i64 bm_bq, i64 bm_bk, int nthreads) {
     if (B < 0 || Hq <= 0 || Hkv <= 0 || N < 0 || d <= 0 || Hq % Hkv || ncols < 0 || window < 0 ||
         drop_t < 0 || drop_t > 255)
         return 1;
@@ -631,6 +675,7 @@ int oracle_bwd_cols(const double *q, const double *k, const double *v, const dou
     P.q = q; P.k = k; P.v = v; P.dout = dout; P.dk = dk_cols; P.dv = dv_cols;
     P.rows = cols; P.nrows = ncols; P.b_sel = b_sel; P.hkv_sel = hkv_sel; P.window = window; P.drop_t = drop_t; P.seed_lo = seed_lo; P.seed_hi = seed_hi;
     P.B = B; P.Hq = Hq; P.Hkv = Hkv; P.N = N; P.d = d; P.scale = scale; P.causal = causal;
+    if (set_block_mask(&P, bmask, bm_hstride, bm_bq, bm_bk)) return 1;
 
     const i64 i_lo = causal ? j_min : 0;
     colstat_t *stats = (colstat_t *)calloc((size_t)group, sizeof(colstat_t));

@@ -682,6 +682,156 @@ def pin_fp8_factor_moves(orc):
     _close(lse_r, lse[:, :, rows], 1e-13, "FP8 rows lse")
 
 
+# ----------------------------------------------------------- block-mask pins
+
+def _element_mask(bm, bq, bk, N, causal):
+    """[H or 1, N, N] boolean visibility from a block mask [H?, Tq, Tk]."""
+    bm = np.asarray(bm) != 0
+    if bm.ndim == 2:
+        bm = bm[None]
+    i = np.arange(N)
+    vis = bm[:, i[:, None] // bq, i[None, :] // bk]
+    if causal:
+        vis = vis & (i[None, :] <= i[:, None])[None]
+    return vis
+
+
+def pin_block_mask_all_ones_and_causal(orc):
+    """A mask of ones changes nothing (forward and gradients, causal or not);
+    under a causal mask the blocks above the diagonal may be dropped too."""
+    q, k, v, do = _rand(50, Hq=2, Hkv=1, N=11, d=4)
+    for causal in (False, True):
+        ones = (np.ones((3, 4), dtype=np.uint8), 4, 3)
+        o, lse = orc.fwd(q, k, v, 0.6, causal)
+        g = orc.bwd(q, k, v, do, 0.6, causal)
+        o1, lse1 = orc.fwd(q, k, v, 0.6, causal, block_mask=ones)
+        g1 = orc.bwd(q, k, v, do, 0.6, causal, block_mask=ones)
+        _close(o1, o, 0.0, "mask of ones O")
+        _close(lse1, lse, 0.0, "mask of ones lse")
+        for a, b_, n in zip(g1, g, ("dQ", "dK", "dV")):
+            _close(a, b_, 0.0, f"mask of ones {n}")
+    tri = (np.tril(np.ones((3, 3), dtype=np.uint8)), 4, 4)  # blocks on and below the diagonal
+    o2, lse2 = orc.fwd(q, k, v, 0.6, True, block_mask=tri)
+    o, lse = orc.fwd(q, k, v, 0.6, True)
+    _close(o2, o, 0.0, "causal with lower block triangle")
+    _close(lse2, lse, 0.0, "causal lse with lower block triangle")
+
+
+def pin_block_mask_block_diagonal(orc):
+    """A block-diagonal mask splits the sequence into independent attention
+    problems: each block of rows equals plain attention on its own slice
+    (forward and gradients), with per-head masks that differ."""
+    N, bs = 12, 4
+    q, k, v, do = _rand(51, Hq=2, Hkv=2, N=N, d=3)
+    eye = np.eye(3, dtype=np.uint8)
+    full = np.ones((3, 3), dtype=np.uint8)
+    bm = np.stack([eye, full])  # head 0 block-diagonal, head 1 dense
+    o, lse = orc.fwd(q, k, v, 0.5, False, block_mask=(bm, bs, bs))
+    dq, dk, dv = orc.bwd(q, k, v, do, 0.5, False, block_mask=(bm, bs, bs))
+    od, lsed = orc.fwd(q, k, v, 0.5, False)
+    dqd, dkd, dvd = orc.bwd(q, k, v, do, 0.5, False)
+    _close(o[:, 1], od[:, 1], 1e-15, "dense head under a per-head mask")
+    _close(dk[:, 1], dkd[:, 1], 1e-15, "dense head dK under a per-head mask")
+    for t in range(3):
+        sl = slice(t * bs, (t + 1) * bs)
+        h0 = lambda x: x[:, :1, sl]
+        os_, ls_ = orc.fwd(h0(q), h0(k), h0(v), 0.5, False)
+        gs = orc.bwd(h0(q), h0(k), h0(v), h0(do), 0.5, False)
+        _close(o[:, :1, sl], os_, 1e-14, f"block-diagonal O, block {t}")
+        _close(lse[:, :1, sl], ls_, 1e-14, f"block-diagonal lse, block {t}")
+        for a, b_, n in zip((dq, dk, dv), gs, ("dQ", "dK", "dV")):
+            _close(a[:, :1, sl], b_, 1e-14, f"block-diagonal {n}, block {t}")
+
+
+def pin_block_mask_brute_force_and_torch(orc):
+    """Random block masks with ragged edge blocks, GQA: pure-Python loops for
+    the forward, torch fp64 SDPA with the expanded boolean mask and autograd
+    for the gradients (every row keeps a visible key)."""
+    N, bq, bk = 10, 4, 3
+    q, k, v, do = _rand(52, Hq=2, Hkv=1, N=N, d=3)
+    r = _rng(53)
+    for causal in (False, True):
+        bm = r.integers(0, 2, size=(2, 3, 4)).astype(np.uint8)
+        bm[:, :, 0] = 1  # the first key block keeps every row non-empty
+        vis = _element_mask(bm, bq, bk, N, causal)
+        o, lse = orc.fwd(q, k, v, 0.7, causal, block_mask=(bm, bq, bk))
+        for h in range(2):
+            for i in range(N):
+                s = [0.7 * sum(q[0, h, i, c] * k[0, 0, j, c] for c in range(3)) if vis[h, i, j] else None
+                     for j in range(N)]
+                m = max(x for x in s if x is not None)
+                e = [math.exp(x - m) if x is not None else 0.0 for x in s]
+                ll = sum(e)
+                for c in range(3):
+                    ref = sum(e[j] * v[0, 0, j, c] for j in range(N)) / ll
+                    assert abs(o[0, h, i, c] - ref) < 1e-13, f"brute-force O ({h},{i},{c})"
+                assert abs(lse[0, h, i] - (m + math.log(ll))) < 1e-13, f"brute-force lse ({h},{i})"
+        tq, tk, tv = (torch.tensor(x, dtype=torch.float64, requires_grad=True) for x in (q, k, v))
+        ro = torch.nn.functional.scaled_dot_product_attention(
+            tq, tk.expand(1, 2, N, 3), tv.expand(1, 2, N, 3),
+            attn_mask=torch.from_numpy(vis)[None], scale=0.7)
+        ro.backward(torch.tensor(do))
+        dq, dk, dv = orc.bwd(q, k, v, do, 0.7, causal, block_mask=(bm, bq, bk))
+        _close(o, ro.detach().numpy(), 1e-12, "block mask O vs torch")
+        _close(dq, tq.grad.numpy(), 1e-11, "block mask dQ vs torch")
+        _close(dk, tk.grad.numpy(), 1e-11, "block mask dK vs torch")
+        _close(dv, tv.grad.numpy(), 1e-11, "block mask dV vs torch")
+
+
+def pin_block_mask_empty_rows(orc):
+    """Rows that see no block: O = 0, lse = -inf, dQ = 0, and they add nothing
+    to dK, dV (the same as giving those rows dO = 0 without the mask); the
+    other rows are untouched."""
+    N, bq, bk = 12, 4, 4
+    q, k, v, do = _rand(54, Hq=1, Hkv=1, N=N, d=3)
+    bm = np.ones((3, 3), dtype=np.uint8)
+    bm[1] = 0  # rows 4..7 see nothing
+    o, lse = orc.fwd(q, k, v, 0.4, False, block_mask=(bm, bq, bk))
+    dq, dk, dv = orc.bwd(q, k, v, do, 0.4, False, block_mask=(bm, bq, bk))
+    od, lsed = orc.fwd(q, k, v, 0.4, False)
+    assert np.all(o[0, 0, 4:8] == 0.0) and np.all(np.isneginf(lse[0, 0, 4:8])), "empty rows"
+    assert np.all(dq[0, 0, 4:8] == 0.0), "empty rows dQ"
+    keep = np.r_[0:4, 8:12]
+    _close(o[0, 0, keep], od[0, 0, keep], 0.0, "other rows O")
+    _close(lse[0, 0, keep], lsed[0, 0, keep], 0.0, "other rows lse")
+    do0 = do.copy()
+    do0[:, :, 4:8] = 0.0
+    dqr, dkr, dvr = orc.bwd(q, k, v, do0, 0.4, False)
+    _close(dk, dkr, 1e-15, "empty rows add nothing to dK")
+    _close(dv, dvr, 1e-15, "empty rows add nothing to dV")
+    _close(dq[0, 0, keep], dqr[0, 0, keep], 1e-15, "other rows dQ")
+    o2, lse2 = orc.fwd_online(q, k, v, 0.4, False, block=4, block_mask=(bm, bq, bk))
+    _close(o2, o, 1e-14, "online O with empty rows")
+    assert np.all(np.isneginf(lse2[0, 0, 4:8])), "online lse of empty rows"
+
+
+def pin_block_mask_subsets_and_online(orc):
+    """Row, column and online forms agree with the full form under a block mask."""
+    N = 13
+    q, k, v, do = _rand(55, Hq=4, Hkv=2, N=N, d=3)
+    r = _rng(56)
+    bm = r.integers(0, 2, size=(4, 4, 5)).astype(np.uint8)
+    bm[:, :, 0] = 1
+    mask = (bm, 4, 3)
+    for causal in (False, True):
+        o, lse = orc.fwd(q, k, v, 0.5, causal, block_mask=mask)
+        dq, dk, dv = orc.bwd(q, k, v, do, 0.5, causal, block_mask=mask)
+        rows = np.array([0, 3, 4, 9, 12])
+        o_r, lse_r = orc.fwd_rows(q, k, v, rows, 0.5, causal, block_mask=mask)
+        _close(o_r, o[:, :, rows], 1e-14, "block mask rows O")
+        _close(lse_r, lse[:, :, rows], 1e-14, "block mask rows lse")
+        _close(orc.bwd_rows(q, k, v, do, rows, 0.5, causal, block_mask=mask), dq[:, :, rows], 1e-13,
+               "block mask rows dQ")
+        cols = np.array([1, 5, 6, 12])
+        for g in range(2):
+            dk_c, dv_c = orc.bwd_cols(q, k, v, do, 0, g, cols, 0.5, causal, block_mask=mask)
+            _close(dk_c, dk[0, g, cols], 1e-13, f"block mask cols dK head {g}")
+            _close(dv_c, dv[0, g, cols], 1e-13, f"block mask cols dV head {g}")
+        o2, lse2 = orc.fwd_online(q, k, v, 0.5, causal, block=3, block_mask=mask)
+        _close(o2, o, 1e-13, "block mask online O")
+        _close(lse2, lse, 1e-13, "block mask online lse")
+
+
 ALL_PINS = [
     pin_q_zero_noncausal, pin_q_zero_causal, pin_one_hot, pin_causal_row0,
     pin_rows_sum_to_one, pin_key_shift, pin_golden, pin_brute_force_python,
@@ -693,4 +843,7 @@ ALL_PINS = [
     pin_dropout_torch, pin_dropout_finite_differences, pin_dropout_subsets_and_online,
     pin_decode_equals_contiguous_attention, pin_decode_page_shuffle_and_q_zero,
     pin_e4m3_decode, pin_fp8_q_zero, pin_fp8_torch_sdpa, pin_fp8_factor_moves,
+    pin_block_mask_all_ones_and_causal, pin_block_mask_block_diagonal,
+    pin_block_mask_brute_force_and_torch, pin_block_mask_empty_rows,
+    pin_block_mask_subsets_and_online,
 ]

@@ -33,11 +33,18 @@ MUTANTS = [
     ("dropout_no_rescale", "256.0 / (256.0 - P->drop_t) : 0.0", "1.0 : 0.0"),
     ("dropout_word_byte_swapped", "(x[i & 3] >> (8 * (j & 3)))", "(x[j & 3] >> (8 * (i & 3)))"),
     ("dropout_dV_undropped_in_columns", "dvj[c] += p * f * doh[i * d + c];", "dvj[c] += p * doh[i * d + c];"),
-    ("window_ignored_in_columns", "            if (hidden(P, i, j)) continue;", "            if (P->causal && j > i) continue;"),
+    ("window_ignored_in_columns", "            if (hidden(P, S->h, i, j)) continue;", "            if (P->causal && j > i) continue;"),
     ("e4m3_exponent_bias_8", "ldexp(1.0 + (double)f / 8.0, e - 7)", "ldexp(1.0 + (double)f / 8.0, e - 8)"),
     ("e4m3_subnormal_as_normal", "mag = ldexp((double)f / 8.0, -6);", "mag = ldexp(1.0 + (double)f / 8.0, -6);"),
     ("e4m3_no_nan_code", "if (e == 15 && f == 7)\n        return NAN;", "if (0)\n        return NAN;"),
     ("e4m3_sign_dropped", "return sign ? -mag : mag;", "return mag;"),
+    # block masks (every planted index stays inside the mask array)
+    ("block_mask_of_head_0_for_all", "!P->bmask[h * P->bm_hstride +", "!P->bmask[0 * P->bm_hstride +"),
+    ("block_mask_ignored_in_columns", "            if (hidden(P, S->h, i, j)) continue;",
+     "            if ((P->causal && j > i) || (P->window > 0 && j <= i - P->window)) continue;"),
+    ("empty_row_not_zeroed", "    if (m == -INFINITY) {\n        for (i64 j = 0; j < N; ++j) s[j] = 0.0;",
+     "    if (0) {\n        for (i64 j = 0; j < N; ++j) s[j] = 0.0;"),
+    ("online_empty_row_divides_by_zero", "if (l == 0.0) { /* no visible key", "if (0) { /* no visible key"),
 ]
 
 
