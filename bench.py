@@ -517,6 +517,35 @@ def oracle_sample(w, causal, seconds, rows_hint=None):
     return per_row * n / dt / 1e12, n, dt, threads
 
 
+def oracle_sample_fp8(w, causal, seconds):
+    """Times the fp64 oracle's FP8 forward (E4M3 decode + forward rows) on
+    seeded query rows of the first heads of the workload; returns
+    (TFLOPS-equivalent, rows, s, threads), each row counted at its share of
+    the forward FLOPs."""
+    import oracle
+    from exact_io_aware_bwd_b200.workloads import make_fp8_inputs
+    H = min(w.B * w.Hq, 8)
+    (q8, k8, v8), ds = make_fp8_inputs(w, shape_override=(1, H, H, w.N, w.d))
+    per_row = w.flops_fwd(causal) / (w.B * w.Hq * w.N)
+    g = torch.Generator().manual_seed(w.seed + 5)
+
+    def run(per_head):
+        rows = torch.sort(torch.randperm(w.N, generator=g)[:per_head]).values.numpy()
+        t = time.perf_counter()
+        oracle.fwd_fp8_rows(q8, k8, v8, ds, rows, w.scale, causal)
+        return time.perf_counter() - t, H * per_head
+
+    per_head = 4
+    while True:
+        dt, n = run(per_head)
+        if dt >= 1.0 or per_head >= w.N:
+            break
+        per_head = min(w.N, per_head * 4)
+    per_head = max(1, min(w.N, int(per_head * seconds / max(dt, 1e-6))))
+    dt, n = run(per_head)
+    return per_row * n / dt / 1e12, n, dt, oracle.num_threads()
+
+
 def run_reference(args, w, causal):
     """The oracle arm: each step is a bounded sample of the same workload."""
     budget = 150.0
@@ -596,6 +625,12 @@ def main():
         if args.decode or args.fp8:
             line = (run_decode(args, rank, world, device) if args.decode
                     else run_fp8(args, w, causal, rank, world, device))
+            if rank == 0 and args.fp8 and not args.no_cpu_baseline:
+                v, rows, dt, threads = oracle_sample_fp8(w, causal, args.cpu_seconds)
+                line["cpu_baseline"] = {
+                    "value": round(v, 6), "unit": "TFLOPS", "cores": threads, "kind": "oracle",
+                    "sample": f"{rows} seeded query rows of the FP8 forward (E4M3 decode, fp64 rows), "
+                              f"{dt:.1f} s; each row counted at its share of the forward FLOPs"}
             if rank == 0:
                 print(json.dumps(line), flush=True)
             return
