@@ -32,8 +32,9 @@
  *   - causal != 0 masks key j for query i when j > i.
  *   - q, k, v, dout share one dtype (bf16 or fp16); o, dq, dk, dv are written
  *     in it.  Arithmetic: tensor-core products of the I/O dtype with fp32
- *     accumulation; softmax statistics in fp32.
- *   - d must be 64 or 128; N may be any size >= 0 (a ragged last tile is
+ *     accumulation; softmax statistics in fp32.  (fa_fwd_fp8 alone takes
+ *     8-bit E4M3 inputs and a separate output dtype; see there.)
+ *   - d must be 64 or 128 (128 for fa_fwd_fp8); N may be any size >= 0 (a ragged last tile is
  *     masked); B == 0 or N == 0 is an empty problem and returns FA_OK at once.
  *   - scale must be finite and > 0 (usually 1/sqrt(d)).
  *   - Every tensor pointer must be 16-byte aligned (TMA requirement).
