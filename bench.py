@@ -10,6 +10,7 @@ replica (the path has no exchange step), so scaling is weak.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
   python bench.py --impl reference ...   # the CPU oracle arm
+  python bench.py --window W | --dropout P | --decode | --fp8   # the variants
 
 Timing: W untimed steps, then K steps between a barrier + synchronize on both
 sides, CUDA events on the launching stream, max over ranks.  The inputs
