@@ -71,3 +71,17 @@ def test_fp8_inputs_quantise_the_16bit_draws():
 def test_fp8_flops_follow_the_forward_convention():
     w = WORKLOADS["mha4k"]
     assert w.flops_fwd(True) == 4.0 * 4 * 32 * 4096 * 4096 * 128 / 2
+
+
+def test_profiled_traffic_is_reported_only_for_the_profiled_sources():
+    """The bench reports an ncu traffic figure only while the kernel sources
+    still hash to the digest recorded with it, and only for its workload."""
+    import bench
+    for spec in (bench.PROFILED_TRAFFIC, bench.PROFILED_TRAFFIC_FP8):
+        got = bench.profiled_traffic(spec["workload"], spec)
+        assert got in (None, spec["bytes"])
+        assert bench.profiled_traffic("tiny", spec) is None
+        stale = dict(spec, sources_sha256_16="0" * 16)
+        assert bench.profiled_traffic(spec["workload"], stale) is None
+        missing = dict(spec, sources=("exact_io_aware_bwd_b200/csrc/no_such_file.cuh",))
+        assert bench.profiled_traffic(spec["workload"], missing) is None
