@@ -160,10 +160,13 @@ def rank_seed(w, rank):
     return w.seed + 1000 * rank
 
 
-def run_ours(args, w, causal, rank, world, device):
-    torch.cuda.set_device(device)
-    build()
-    binding.load()
+def kernel_stats(ms):
+    """Mean, median and min of per-launch times (ms)."""
+    return {"mean": statistics.mean(ms), "median": statistics.median(ms), "min": min(ms)}
+
+
+def alloc_problem(w, rank, device):
+    """Device tensors of one replica of workload w (inputs drawn on the device)."""
     B, Hq, Hkv, N, d = w.B, w.Hq, w.Hkv, w.N, w.d
     g = torch.Generator(device=device).manual_seed(rank_seed(w, rank))
     mk = lambda H, s: (torch.randn((B, H, N, d), generator=g, device=device, dtype=torch.float32) * s).to(w.dtype)
@@ -172,52 +175,76 @@ def run_ours(args, w, causal, rank, world, device):
     lse = torch.empty((B, Hq, N), device=device, dtype=torch.float32)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     ws = torch.empty(binding.fa_bwd_workspace_bytes(B, Hq, Hkv, N, d), device=device, dtype=torch.uint8)
+    return dict(q=q, k=k, v=v, do=do, o=o, lse=lse, dq=dq, dk=dk, dv=dv, ws=ws)
+
+
+def make_step(t, w, causal, W, DR, stream, fwd_ev=None, bwd_ev=None):
+    """One pass of the hot path (fa_fwd then fa_bwd) on the tensors t; with
+    events, the i-th call records around each of the two calls on `stream`."""
+    q, k, v, do, o, lse, dq, dk, dv, ws = (t[n] for n in ("q", "k", "v", "do", "o", "lse", "dq", "dk", "dv", "ws"))
     scale = w.scale
-    stream = torch.cuda.current_stream(device)
 
-    W = args.window
-    DR = (args.dropout, 0x5EED0000 + rank) if args.dropout else None
-
-    def step():
+    def step(i=None):
+        if i is not None:
+            fwd_ev[i][0].record(stream)
         if DR:
             binding.fa_fwd_dropout(q, k, v, o, lse, scale, causal, DR[0], DR[1], stream)
-            binding.fa_bwd_dropout(q, k, v, o, do, lse, dq, dk, dv, scale, causal, DR[0], DR[1], ws, stream)
         elif W:
             binding.fa_fwd_window(q, k, v, o, lse, scale, W, stream)
-            binding.fa_bwd_window(q, k, v, o, do, lse, dq, dk, dv, scale, W, ws, stream)
         else:
             binding.fa_fwd(q, k, v, o, lse, scale, causal, stream)
+        if i is not None:
+            fwd_ev[i][1].record(stream)
+            bwd_ev[i][0].record(stream)
+        if DR:
+            binding.fa_bwd_dropout(q, k, v, o, do, lse, dq, dk, dv, scale, causal, DR[0], DR[1], ws, stream)
+        elif W:
+            binding.fa_bwd_window(q, k, v, o, do, lse, dq, dk, dv, scale, W, ws, stream)
+        else:
             binding.fa_bwd(q, k, v, o, do, lse, dq, dk, dv, scale, causal, ws, stream)
+        if i is not None:
+            bwd_ev[i][1].record(stream)
+    return step
+
+
+def time_steps(args, w, causal, rank, world, device, steps, warmup, W=0, DR=None, clocks=None):
+    """W untimed steps, then `steps` timed ones between a barrier and a
+    synchronize on both sides; CUDA events on the launching stream around the
+    whole region, around every fa_fwd and fa_bwd call, and (through the
+    library) around every launch of the forward kernel and of the backward
+    main kernel.  Returns the timings (ms; the total is the max over ranks)."""
+    t = alloc_problem(w, rank, device)
+    stream = torch.cuda.current_stream(device)
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    K = steps
+    fwd_ev = [(ev(), ev()) for _ in range(K)]
+    bwd_ev = [(ev(), ev()) for _ in range(K)]
+    kf_ev = [(ev(), ev()) for _ in range(K)]
+    kb_ev = [(ev(), ev()) for _ in range(K)]
+    for a, b in kf_ev + kb_ev:  # materialise the handles the library records into
+        a.record(stream)
+        b.record(stream)
+    step = make_step(t, w, causal, W, DR, stream, fwd_ev, bwd_ev)
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize(device)
+    assert binding.fa_get_device_status(stream) == binding.FA_OK
 
     def barrier():
         if world > 1:
             torch.distributed.barrier()
 
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize(device)
-    assert binding.fa_get_device_status(stream) == binding.FA_OK
-
-    # per-step events around the whole step and around each kernel of interest
-    K = args.steps
-    ev = lambda: torch.cuda.Event(enable_timing=True)
-    fwd_ev = [(ev(), ev()) for _ in range(K)]
-    bwd_ev = [(ev(), ev()) for _ in range(K)]
-    for a, b in fwd_ev + bwd_ev:  # materialise the handles
-        a.record(stream)
-        b.record(stream)
-    t0, t1 = ev(), ev()
-    clocks = ClockSampler(device) if rank == 0 else None
     if clocks:
         clocks.start()
         time.sleep(0.3)
+    t0, t1 = ev(), ev()
     barrier()
     torch.cuda.synchronize(device)
     t0.record(stream)
     for i in range(K):
-        binding.fa_set_profile_events(binding.KERNEL_FWD, *fwd_ev[i])
-        binding.fa_set_profile_events(binding.KERNEL_BWD_MAIN, *bwd_ev[i])
-        step()
+        binding.fa_set_profile_events(binding.KERNEL_FWD, *kf_ev[i])
+        binding.fa_set_profile_events(binding.KERNEL_BWD_MAIN, *kb_ev[i])
+        step(i)
     t1.record(stream)
     torch.cuda.synchronize(device)
     barrier()
@@ -226,14 +253,56 @@ def run_ours(args, w, causal, rank, world, device):
     clk = clocks.stop() if clocks else None
     status = binding.fa_get_device_status(stream)
     assert status == binding.FA_OK, binding.fa_status_string(status)
+    el = lambda pairs: [a.elapsed_time(b) for a, b in pairs]
+    res = dict(ms_total=max_over_ranks(t0.elapsed_time(t1), world, device),
+               fwd=kernel_stats(el(fwd_ev)), bwd=kernel_stats(el(bwd_ev)),
+               fwd_kernel=kernel_stats(el(kf_ev)), bwd_main=kernel_stats(el(kb_ev)),
+               clocks=clk, tensors=t)
+    return res
 
-    ms_total = t0.elapsed_time(t1)
-    fwd_ms = statistics.mean(a.elapsed_time(b) for a, b in fwd_ev)
-    bwd_main_ms = statistics.mean(a.elapsed_time(b) for a, b in bwd_ev)
-    ms_total = max_over_ranks(ms_total, world, device)
-    ms_step = ms_total / K
+
+def summarize(w, causal, res, K, peak, W=0):
+    """TFLOPS and % of peak of a timed run (medians of per-call times)."""
+    f_fwd, f_bwd = w.flops_fwd(causal, W), w.flops_bwd(causal, W)
+    tf = lambda f, ms: f / (ms * 1e-3) / 1e12
+    fwd, bwd, bm = res["fwd"]["median"], res["bwd"]["median"], res["bwd_main"]["median"]
+    return {
+        "workload": workload_desc(w, causal) + (f" window={W}" if W else ""),
+        "ms_per_step": round(res["ms_total"] / K, 4),
+        "tflops": round(tf(f_fwd + f_bwd, res["ms_total"] / K), 2),
+        "pct_of_peak": round(100 * tf(f_fwd + f_bwd, res["ms_total"] / K) / peak, 2),
+        "fwd_ms": round(fwd, 4), "fwd_ms_min": round(res["fwd"]["min"], 4),
+        "fwd_tflops": round(tf(f_fwd, fwd), 2), "fwd_pct_of_peak": round(100 * tf(f_fwd, fwd) / peak, 2),
+        "bwd_ms": round(bwd, 4), "bwd_ms_min": round(res["bwd"]["min"], 4),
+        "bwd_tflops": round(tf(f_bwd, bwd), 2), "bwd_pct_of_peak": round(100 * tf(f_bwd, bwd) / peak, 2),
+        "bwd_main_ms": round(bm, 4), "bwd_main_ms_min": round(res["bwd_main"]["min"], 4),
+        "bwd_main_tflops": round(tf(f_bwd, bm), 2),
+        "steps": K,
+    }
+
+
+# Configurations of the metric's range besides the headline one, timed after
+# it on the same GPU and reported as sub-results of the same line.
+RANGE_WORKLOADS = ("gqa16k", "long64k")
+
+
+def run_ours(args, w, causal, rank, world, device):
+    torch.cuda.set_device(device)
+    build()
+    binding.load()
+    W = args.window
+    DR = (args.dropout, 0x5EED0000 + rank) if args.dropout else None
+    K = args.steps
+    clocks = ClockSampler(device) if rank == 0 else None
+    res = time_steps(args, w, causal, rank, world, device, K, args.warmup, W, DR, clocks)
+    clk = res["clocks"]
+    t = res.pop("tensors")
+    ms_step = res["ms_total"] / K
     f_fwd, f_bwd = w.flops_fwd(causal, W), w.flops_bwd(causal, W)
     value = job_tflops(world, f_fwd + f_bwd, ms_step)
+    fwd_ms, bwd_ms = res["fwd"]["median"], res["bwd"]["median"]
+    fwd_kern_mean, bwd_main_mean = res["fwd_kernel"]["mean"], res["bwd_main"]["mean"]
+    stream = torch.cuda.current_stream(device)
 
     # end to end through the C ABI with host buffers: every step copies the
     # step's inputs in from pinned host memory, runs fwd + bwd and copies all
@@ -242,43 +311,34 @@ def run_ours(args, w, causal, rank, world, device):
     # directions use separate copy engines) and the kernels.
     e2e = None
     if not args.no_e2e:
-        hin = [t.cpu().pin_memory() for t in (q, k, v, do)]
+        ev = lambda: torch.cuda.Event(enable_timing=True)
+        q, k, v, do, o, lse, dq, dk, dv, ws = (t[n] for n in ("q", "k", "v", "do", "o", "lse", "dq", "dk", "dv", "ws"))
+        hin = [x.cpu().pin_memory() for x in (q, k, v, do)]
         outs_like = (o, lse, dq, dk, dv)
-        sets = [dict(inp=[q, k, v, do], out=[o, lse, dq, dk, dv], ws=ws)]
-        sets.append(dict(inp=[torch.empty_like(t) for t in (q, k, v, do)],
-                         out=[torch.empty_like(t) for t in outs_like],
-                         ws=torch.empty_like(ws)))
-        hout = [[torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs_like] for _ in sets]
+        sets = [dict(q=q, k=k, v=v, do=do, o=o, lse=lse, dq=dq, dk=dk, dv=dv, ws=ws)]
+        sets.append({n: torch.empty_like(x) for n, x in sets[0].items()})
+        hout = [[torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for x in outs_like] for _ in sets]
         streams = [torch.cuda.Stream(device) for _ in sets]
-        h2d = sum(t.numel() * t.element_size() for t in hin)
-        d2h = sum(t.numel() * t.element_size() for t in hout[0])
+        steps_e = [make_step(b, w, causal, W, DR, st) for b, st in zip(sets, streams)]
+        h2d = sum(x.numel() * x.element_size() for x in hin)
+        d2h = sum(x.numel() * x.element_size() for x in hout[0])
 
         def e2e_step(i):
             b, st, ho = sets[i % 2], streams[i % 2], hout[i % 2]
             with torch.cuda.stream(st):
-                for dst, src in zip(b["inp"], hin):
-                    dst.copy_(src, non_blocking=True)
-                bq, bk, bv, bdo = b["inp"]
-                bo, blse, bdq, bdk, bdv = b["out"]
-                if DR:
-                    binding.fa_fwd_dropout(bq, bk, bv, bo, blse, scale, causal, DR[0], DR[1], st)
-                    binding.fa_bwd_dropout(bq, bk, bv, bo, bdo, blse, bdq, bdk, bdv, scale, causal,
-                                           DR[0], DR[1], b["ws"], st)
-                elif W:
-                    binding.fa_fwd_window(bq, bk, bv, bo, blse, scale, W, st)
-                    binding.fa_bwd_window(bq, bk, bv, bo, bdo, blse, bdq, bdk, bdv, scale, W, b["ws"], st)
-                else:
-                    binding.fa_fwd(bq, bk, bv, bo, blse, scale, causal, st)
-                    binding.fa_bwd(bq, bk, bv, bo, bdo, blse, bdq, bdk, bdv, scale, causal, b["ws"], st)
-                for dst, src in zip(ho, b["out"]):
-                    dst.copy_(src, non_blocking=True)
+                for name, src in zip(("q", "k", "v", "do"), hin):
+                    b[name].copy_(src, non_blocking=True)
+                steps_e[i % 2]()
+                for dst, name in zip(ho, ("o", "lse", "dq", "dk", "dv")):
+                    dst.copy_(b[name], non_blocking=True)
 
         for i in range(2):
             e2e_step(i)
         torch.cuda.synchronize(device)
         Ke = max(4, min(K, 10))
         e0, e1 = ev(), ev()
-        barrier()
+        if world > 1:
+            torch.distributed.barrier()
         torch.cuda.synchronize(device)
         e0.record(stream)
         for st in streams:
@@ -291,7 +351,8 @@ def run_ours(args, w, causal, rank, world, device):
             stream.wait_event(done)
         e1.record(stream)
         torch.cuda.synchronize(device)
-        barrier()
+        if world > 1:
+            torch.distributed.barrier()
         status = binding.fa_get_device_status(stream)
         assert status == binding.FA_OK, binding.fa_status_string(status)
         ems = max_over_ranks(e0.elapsed_time(e1) / Ke, world, device)
@@ -299,11 +360,14 @@ def run_ours(args, w, causal, rank, world, device):
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ems,
                "copies": "pinned host buffers; two device buffer sets on two streams, so a "
                          "step's copies back overlap the next step's copies in"}
+        del sets, hin, hout
+    del t
 
     pk, pk_kind = peaks()
     peak = pk["bf16_tflops"]
-    bwd_tflops_main = f_bwd / (bwd_main_ms * 1e-3) / 1e12
-    fwd_tflops = f_fwd / (fwd_ms * 1e-3) / 1e12
+    head = summarize(w, causal, res, K, peak, W)
+    bwd_tflops_main = f_bwd / (bwd_main_mean * 1e-3) / 1e12
+    launches_per_step = 4
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True,
@@ -318,23 +382,43 @@ def run_ours(args, w, causal, rank, world, device):
                    "l2": "inputs larger than L2 (no flush)",
                    "flops_per_step": f_fwd + f_bwd},
         "pct_of_peak": round(100 * value / world / peak, 2),
-        "fwd_ms": round(fwd_ms, 4), "fwd_tflops": round(fwd_tflops, 2),
-        "fwd_pct_of_peak": round(100 * fwd_tflops / peak, 2),
-        "bwd_main_ms": round(bwd_main_ms, 4), "bwd_main_tflops": round(bwd_tflops_main, 2),
-        "bwd_ms": round(ms_step - fwd_ms, 4),
-        "bwd_tflops": round(f_bwd / ((ms_step - fwd_ms) * 1e-3) / 1e12, 2),
-        "bwd_pct_of_peak": round(100 * f_bwd / ((ms_step - fwd_ms) * 1e-3) / 1e12 / peak, 2),
+        "fwd_ms": head["fwd_ms"], "fwd_ms_min": head["fwd_ms_min"],
+        "fwd_tflops": head["fwd_tflops"], "fwd_pct_of_peak": head["fwd_pct_of_peak"],
+        "bwd_ms": head["bwd_ms"], "bwd_ms_min": head["bwd_ms_min"],
+        "bwd_tflops": head["bwd_tflops"], "bwd_pct_of_peak": head["bwd_pct_of_peak"],
+        "bwd_main_ms": head["bwd_main_ms"], "bwd_main_ms_min": head["bwd_main_ms_min"],
+        "bwd_main_tflops": head["bwd_main_tflops"],
+        "timing_stats": "fwd/bwd: median (and min) of per-call CUDA-event times on the launch stream; "
+                        "roofline: mean of the kernel's per-launch times",
         "roofline": {"kernel": "fa_bwd_kernel (main backward pass)", "bound": "tensor",
                      "achieved": round(bwd_tflops_main, 2), "peak": peak, "unit": "TFLOP/s",
                      "frac": round(bwd_tflops_main / peak, 4), "peak_kind": f"{pk_kind} bf16 burst",
-                     "traffic": profiled_traffic(w.name),
+                     "traffic": profiled_traffic(w.name) if not (W or DR) else None,
                      "traffic_unit": "bytes per launch (ncu)",
                      "algorithmic": "2.5 x 4*B*Hq*N^2*d (/2 causal) FLOPs per launch"
                                     + (" (visible pairs under the window)" if W else "")},
-        "gpu_launches": 4 * K,
+        "forward_kernel": {"kernel": "fa_fwd_kernel", "bound": "tensor",
+                           "achieved": round(f_fwd / (fwd_kern_mean * 1e-3) / 1e12, 2), "peak": peak,
+                           "unit": "TFLOP/s",
+                           "frac": round(f_fwd / (fwd_kern_mean * 1e-3) / 1e12 / peak, 4)},
+        "gpu_launches": launches_per_step * K,
         "clocks": clk,
         "e2e": e2e,
     }
+    # the rest of the metric's range (N = 16K GQA, N = 64K fp16), each on
+    # its own inputs, fewer steps (each step is longer)
+    if not (W or DR or args.no_range) and w.name == "mha4k" and causal:
+        subs = []
+        for name in RANGE_WORKLOADS:
+            ws_ = WORKLOADS[name]
+            Ks = max(3, min(K, 10))
+            r = time_steps(args, ws_, True, rank, world, device, Ks, 3)
+            r.pop("tensors")
+            torch.cuda.empty_cache()
+            sub = summarize(ws_, True, r, Ks, peak)
+            sub["gpu_launches"] = launches_per_step * Ks
+            subs.append(sub)
+        line["range"] = subs
     return line
 
 
@@ -480,14 +564,22 @@ def run_fp8(args, w, causal, rank, world, device):
 _ORACLE_INPUTS = {}
 
 
+# Share of the conventional fwd + bwd FLOPs that the oracle's row sample
+# performs: the forward row (S and P V, 2 of the 7 products the convention
+# counts) and the dQ row (S, dP and dQ, 3 more); the key-side products dV and
+# dK are not in the sample.
+ORACLE_ROW_SHARE = 5.0 / 7.0
+
+
 def oracle_sample(w, causal, seconds, rows_hint=None):
     """Times the fp64 oracle (forward rows + dQ rows) on seeded query rows of
     one head of the workload; returns (TFLOPS-equivalent, rows, s, threads).
-    Each row carries its share of the workload's conventional FLOPs."""
+    Each row is credited the FLOPs of the products it computes: 5/7 of its
+    share of the workload's conventional fwd + bwd FLOPs."""
     import oracle
     from exact_io_aware_bwd_b200.workloads import make_inputs
     g = torch.Generator().manual_seed(w.seed + 3)
-    per_row = (w.flops_fwd(causal) + w.flops_bwd(causal)) / (w.B * w.Hq * w.N)
+    per_row = ORACLE_ROW_SHARE * (w.flops_fwd(causal) + w.flops_bwd(causal)) / (w.B * w.Hq * w.N)
     heads_max = min(w.B * w.Hq, 64)
     key = (w.name, heads_max)
     if key not in _ORACLE_INPUTS:
@@ -559,8 +651,8 @@ def run_reference(args, w, causal):
             vals.append((v, dt))
     value = statistics.mean(v for v, _ in vals)
     ms = 1e3 * statistics.mean(dt for _, dt in vals)
-    sample = (f"{rows} seeded query rows per step (forward O/lse rows + dQ rows, fp64), "
-              f"{workload_desc(w, causal)}")
+    sample = (f"{rows} seeded query rows per step (forward O/lse rows + dQ rows, fp64; each row "
+              f"credited the 5 of 7 conventional products it computes), {workload_desc(w, causal)}")
     return {
         "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": 1,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 2),
@@ -592,6 +684,8 @@ def main():
     ap.add_argument("--window", type=int, default=0,
                     help="causal sliding window of this many keys (0: none); FLOPs counted over visible pairs")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-range", action="store_true",
+                    help="skip the 16K GQA and 64K fp16 sub-results of the default line")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     args = ap.parse_args()
@@ -641,7 +735,8 @@ def main():
             line["cpu_baseline"] = {
                 "value": round(v, 6), "unit": UNIT, "cores": threads, "kind": "oracle",
                 "sample": f"{rows} seeded query rows, forward O/lse rows + dQ rows in fp64, "
-                          f"{dt:.1f} s; each row counted at its share of the workload's FLOPs"}
+                          f"{dt:.1f} s; each row credited the 5 of 7 conventional products it "
+                          f"computes (no dK/dV)"}
         if rank == 0:
             print(json.dumps(line), flush=True)
     finally:

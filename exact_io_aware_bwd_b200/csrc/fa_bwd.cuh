@@ -28,8 +28,8 @@
 //               S^T  = K_j Q_i^T        (128 x 64)
 //               dP^T = V_j dO_i^T       (128 x 64)
 //               softmax warps: P^T, dS^T = P^T o (dP^T - D)
-//               dQ_i^T = K_j^T dS^T     (d x 64) -> TMA reduce-add (fp32) into
-//                                        the dQ accumulator in L2
+//               dQ_i^T = K_j^T dS^T     (d x 64) -> registers -> red.global.add.f32
+//                                        into the fp32 dQ accumulator (in L2)
 //               dV  += P^T dO_i         (P^T read from tensor memory)
 //               dK  += dS^T Q_i
 //             dK, dV stay in tensor memory for the whole walk and are written

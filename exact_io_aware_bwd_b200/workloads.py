@@ -144,17 +144,28 @@ def check_rows(w: Workload, N: int | None = None, seed: int | None = None) -> to
     return torch.sort(torch.randperm(N, generator=g)[: w.check_rows]).values
 
 
+# Key rows of the 64K workload's column check drawn from its first 256 keys.
+LONG_LOW_COLS = 4
+
+
 def check_cols(w: Workload, causal: bool, seed: int | None = None):
     """Seeded (b, hkv, kv rows) triples whose dK/dV the oracle recomputes.
 
-    Under a causal mask dK_j and dV_j depend only on query rows i >= j; the
-    kv rows are drawn from the upper half of the sequence for the 64K
-    workload so that the oracle needs the statistics of half the rows."""
+    Under a causal mask dK_j and dV_j depend on the query rows i >= j.  For
+    the 64K workload most checked kv rows come from the upper half of the
+    sequence and LONG_LOW_COLS from its first 256 keys: those are the key
+    rows whose gradients sum over the most queries (up to all 65 536), the
+    longest reductions of the pass; the oracle then needs the statistics of
+    every row of the head once."""
     g = torch.Generator("cpu").manual_seed(w.seed + 11)
     heads = torch.randperm(w.B * w.Hkv, generator=g)[: w.check_col_heads].tolist()
-    lo = w.N // 2 if (causal and w.N >= 65536) else 0
+    long_causal = causal and w.N >= 65536
+    lo = w.N // 2 if long_causal else 0
     out = []
     for bh in heads:
-        cols = lo + torch.randperm(w.N - lo, generator=g)[: w.check_cols]
+        n_hi = w.check_cols - (LONG_LOW_COLS if long_causal else 0)
+        cols = lo + torch.randperm(w.N - lo, generator=g)[:n_hi]
+        if long_causal:
+            cols = torch.cat([torch.randperm(256, generator=g)[:LONG_LOW_COLS], cols])
         out.append((bh // w.Hkv, bh % w.Hkv, torch.sort(cols).values))
     return out

@@ -1,11 +1,14 @@
 """Helpers of the GPU parity tests: run the CUDA path through the C ABI and
 compare it with the fp64 oracle on the same (rounded) inputs.
 
-Tolerances are those stated for this path: max |dO| <= 1e-2, max |dlse| <= 1e-3,
-relative Frobenius error <= 2e-2 on dQ, dK, dV.  An output element of O whose
-error is above 1e-2 passes only if the error is explained by the rounding of
-O to the I/O dtype (at most half an ulp of the output plus 5e-3); such
-elements are counted and reported, never silently absorbed."""
+Tolerances are those stated for this path and are applied as written:
+max |dO| <= 1e-2, max |dlse| <= 1e-3, relative Frobenius error <= 2e-2 on dQ,
+dK, dV.  ``check_o`` reports the largest O error also in units of the output
+ulp (the rounding of O to bf16 alone is half an ulp, 2^-7 |O|).  A case whose
+O error is above 1e-2 because of rounding alone is not absorbed by
+``check_o``: it has its own test, named as a known exceedance, which asserts
+the a-priori rounding bound of ``check_o_rounding_bound`` instead and prints
+how far above 1e-2 it is."""
 
 from __future__ import annotations
 
@@ -41,26 +44,41 @@ def _np(t):
     return t.double().numpy() if hasattr(t, "double") else np.asarray(t, dtype=np.float64)
 
 
-def check_o(o_gpu, o_ref, dtype, o_absv=None, what="O"):
-    """max |O_gpu - O_ref| <= 1e-2.  An element above it passes only if the
-    rounding of the tensor-core operands and of the output explains it:
+def _ulp(x, dtype):
+    """Spacing of the I/O dtype's numbers at |x| (its normal range)."""
+    mant = 8 if dtype == torch.bfloat16 else 11
+    ar = np.maximum(np.abs(x), 1e-30)
+    return np.exp2(np.floor(np.log2(ar)) - (mant - 1))
+
+
+def check_o(o_gpu, o_ref, dtype, what="O"):
+    """max |O_gpu - O_ref| <= 1e-2, every element, no exception."""
+    g, r = _np(o_gpu), _np(o_ref)
+    err = np.abs(g - r)
+    max_err = float(err.max(initial=0.0))
+    info = dict(max_err=max_err,
+                max_err_ulps=float((err / _ulp(r, dtype)).max(initial=0.0)))
+    assert max_err <= TOL_O, f"{what}: {int((err > TOL_O).sum())} elements beyond {TOL_O}, {info}"
+    return info
+
+
+def check_o_rounding_bound(o_gpu, o_ref, dtype, o_absv, what="O"):
+    """The a-priori bound of the 16-bit path, per element:
     |err| <= u * sum_j p_ij |v_jc| + half an ulp of O + 1e-3, where u is the
-    unit roundoff of the I/O dtype (P is rounded to it before the P V
-    product) and ``o_absv`` is the oracle's output with |V| in place of V,
-    i.e. sum_j p_ij |v_jc|.  Such elements are counted in the report."""
+    unit roundoff of the I/O dtype (P is rounded to it before the P V product;
+    ``o_absv`` is the oracle's output with |V| in place of V, i.e.
+    sum_j p_ij |v_jc|), half an ulp is the rounding of O itself, and 1e-3
+    covers fp32 accumulation and the approximate exponential.  Returns the
+    largest error, the number of elements above the stated 1e-2 and the
+    largest error in output ulps, so that a known exceedance is reported."""
     g, r = _np(o_gpu), _np(o_ref)
     err = np.abs(g - r)
     mant = 8 if dtype == torch.bfloat16 else 11
-    u = 2.0 ** -mant
-    ar = np.maximum(np.abs(r), 1e-30)
-    half_ulp = 0.5 * np.exp2(np.floor(np.log2(ar)) - (mant - 1))
-    over = err > TOL_O
-    bound = half_ulp + 1e-3 + (u * _np(o_absv) if o_absv is not None else 0.0)
-    explained = err <= bound
-    bad = over & ~explained
-    info = dict(max_err=float(err.max(initial=0.0)),
-                n_over_tol_explained_by_rounding=int((over & explained).sum()))
-    assert not bad.any(), f"{what}: {int(bad.sum())} elements beyond tolerance, {info}"
+    bound = 2.0 ** -mant * _np(o_absv) + 0.5 * _ulp(r, dtype) + 1e-3
+    bad = err > bound
+    info = dict(max_err=float(err.max(initial=0.0)), n_over_1e_2=int((err > TOL_O).sum()),
+                max_err_ulps=float((err / _ulp(r, dtype)).max(initial=0.0)))
+    assert not bad.any(), f"{what}: {int(bad.sum())} elements beyond the rounding bound, {info}"
     return info
 
 
@@ -94,9 +112,8 @@ def check_full(q, k, v, do, scale, causal, out, window=0, dropout=None):
     """Every output element against the full oracle."""
     dr = oracle_dropout(dropout)
     o_r, lse_r = oracle.fwd(q, k, v, scale, causal, window=window, dropout=dr)
-    o_abs, _ = oracle.fwd(q, k, v.abs(), scale, causal, window=window, dropout=dr)
     dq_r, dk_r, dv_r = oracle.bwd(q, k, v, do, scale, causal, window=window, dropout=dr)
-    rep = dict(o=check_o(out["o"], o_r, q.dtype, o_abs), lse=check_lse(out["lse"], lse_r))
+    rep = dict(o=check_o(out["o"], o_r, q.dtype), lse=check_lse(out["lse"], lse_r))
     rep.update(dq=check_grad(out["dq"], dq_r, "dQ"), dk=check_grad(out["dk"], dk_r, "dK"),
                dv=check_grad(out["dv"], dv_r, "dV"))
     return rep
@@ -108,20 +125,19 @@ def check_rows(q, k, v, do, scale, causal, out, rows, window=0):
     Hkv = k.shape[1]
     G = Hq // Hkv
     rows = np.asarray(rows, dtype=np.int64)
-    o_g, lse_g, dq_g, o_r, lse_r, dq_r, o_a = [], [], [], [], [], [], []
+    o_g, lse_g, dq_g, o_r, lse_r, dq_r = [], [], [], [], [], []
     for b in range(B):
         for g in range(Hkv):
             hs = slice(g * G, (g + 1) * G)
             qq, kk, vv, dd = q[b:b + 1, hs], k[b:b + 1, g:g + 1], v[b:b + 1, g:g + 1], do[b:b + 1, hs]
             o1, l1 = oracle.fwd_rows(qq, kk, vv, rows, scale, causal, window=window)
-            oa, _ = oracle.fwd_rows(qq, kk, vv.abs(), rows, scale, causal, window=window)
             dq1 = oracle.bwd_rows(qq, kk, vv, dd, rows, scale, causal, window=window)
-            o_r.append(o1); lse_r.append(l1); dq_r.append(dq1); o_a.append(oa)
+            o_r.append(o1); lse_r.append(l1); dq_r.append(dq1)
             o_g.append(_np(out["o"][b:b + 1, hs][:, :, rows]))
             lse_g.append(_np(out["lse"][b:b + 1, hs][:, :, rows]))
             dq_g.append(_np(out["dq"][b:b + 1, hs][:, :, rows]))
     cat = lambda xs: np.concatenate([x.reshape(-1) for x in xs])
-    rep = dict(o=check_o(cat(o_g), cat(o_r), q.dtype, cat(o_a)), lse=check_lse(cat(lse_g), cat(lse_r)),
+    rep = dict(o=check_o(cat(o_g), cat(o_r), q.dtype), lse=check_lse(cat(lse_g), cat(lse_r)),
                dq=check_grad(cat(dq_g), cat(dq_r), "dQ rows"))
     return rep
 

@@ -1,6 +1,7 @@
 """The FP8 parity tolerances against a CPU model of the rounding they are
 derived from: scores from E4M3 inputs in fp64, the running maximum moved
-only when a row's maximum grows by more than 8 (log2 units), probabilities
+(for all 32 rows of a warp at once) only when a row's maximum grows by more
+than 8 (log2 units), probabilities
 rounded to E4M3 (torch's round-to-nearest-even cast) before P V, row sums in
 unrounded form, O rounded to bf16.  The model must stay inside the envelope
 the GPU tests use, with margin; a model that skips the rounding of P must
@@ -19,6 +20,10 @@ REL_FROB_TOL = 0.05
 
 
 def _model(q8, k8, v8, ds, scale, causal, round_p=True, value_factor=True):
+    """The kernel's arithmetic in fp64 except for the roundings it models.
+    Rows go in groups of 32 (the 32 rows of one warp): the reference max of
+    all rows of a group moves together, to each row's own larger max,
+    whenever any row of the group has grown by more than 8 (log2 units)."""
     q = oracle.e4m3_decode(q8) * ds[0]
     k = oracle.e4m3_decode(k8) * ds[1]
     v = oracle.e4m3_decode(v8) * (ds[2] if value_factor else 1.0)
@@ -28,23 +33,31 @@ def _model(q8, k8, v8, ds, scale, causal, round_p=True, value_factor=True):
     out = np.zeros((B, Hq, N, d))
     for b in range(B):
         for h in range(Hq):
+            vv = v[b, h // G]
             S = (q[b, h] @ k[b, h // G].T) * scale * c
-            for i in range(N):
-                n_keys = i + 1 if causal else N
-                m_ref, l, acc = -np.inf, 0.0, np.zeros(d)
-                for j0 in range(0, n_keys, 128):
-                    s = S[i, j0:min(j0 + 128, n_keys)]
+            for i0 in range(0, N, 32):
+                rows = np.arange(i0, min(i0 + 32, N))
+                n_keys = rows + 1 if causal else np.full(len(rows), N)
+                m_ref = np.full(len(rows), -np.inf)
+                l = np.zeros(len(rows))
+                acc = np.zeros((len(rows), d))
+                for j0 in range(0, int(n_keys.max()), 128):
+                    j1 = min(j0 + 128, N)
+                    s = S[rows, j0:j1].copy()
+                    s[np.arange(j0, j1)[None, :] >= n_keys[:, None]] = -np.inf
+                    m_new = s.max(axis=1)
                     if j0 == 0:
-                        m_ref = s.max()
-                    elif s.max() > m_ref + 8:
-                        f = 2.0 ** (m_ref - s.max())
-                        acc, l, m_ref = acc * f, l * f, s.max()
-                    p = np.exp2(s - m_ref)
-                    l += p.sum()
+                        m_ref = m_new
+                    elif np.any(m_new > m_ref + 8):
+                        m_upd = np.maximum(m_ref, m_new)
+                        f = np.exp2(m_ref - m_upd)
+                        acc, l, m_ref = acc * f[:, None], l * f, m_upd
+                    p = np.exp2(s - m_ref[:, None])
+                    l += p.sum(axis=1)
                     if round_p:
                         p = torch.from_numpy(p).float().to(torch.float8_e4m3fn).double().numpy()
-                    acc += p @ v[b, h // G, j0:j0 + len(s)]
-                out[b, h, i] = acc / l
+                    acc += p @ vv[j0:j1]
+                out[b, h, rows] = acc / l[:, None]
     return torch.from_numpy(out).to(torch.bfloat16).double().numpy()
 
 

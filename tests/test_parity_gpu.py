@@ -183,9 +183,34 @@ def test_parity_wide_logits_fp16():
 
 
 def test_scale_not_one_over_sqrt_d():
+    # a scale below 1/sqrt(d): flatter rows than the workloads'
+    q, k, v, do = _inputs((1, 2, 1, 300, 64), torch.bfloat16, seed=6)
+    out = ac.run_gpu(q, k, v, do, 0.06, True)
+    ac.check_full(q, k, v, do, 0.06, True, out)
+
+
+def test_peaked_softmax_known_exceedance():
+    """Known exceedance of the O tolerance, reported rather than absorbed.
+
+    scale = 0.3 at d = 64 (2.4 times 1/sqrt(d)) makes the rows peaked: one or
+    two keys carry almost all of a row's weight, so O_i is close to one row of
+    V, and |O| reaches 2-4 in bf16, where half an ulp of the output alone is
+    0.0078-0.0156.  Add the rounding of P to bf16 before the P V product
+    (relative 2^-9 of each weight) and a few elements can end above 1e-2 by
+    rounding alone.  This case is therefore held to the a-priori rounding
+    bound of the 16-bit path, element by element, and prints how many
+    elements are above 1e-2 and the largest error in output ulps; lse and
+    the gradients keep their stated tolerances."""
     q, k, v, do = _inputs((1, 2, 1, 300, 64), torch.bfloat16, seed=5)
     out = ac.run_gpu(q, k, v, do, 0.3, False)
-    ac.check_full(q, k, v, do, 0.3, False, out)
+    o_r, lse_r = oracle.fwd(q, k, v, 0.3, False)
+    o_abs, _ = oracle.fwd(q, k, v.abs(), 0.3, False)
+    info = ac.check_o_rounding_bound(out["o"], o_r, q.dtype, o_abs)
+    print("peaked softmax, O against the rounding bound:", info)
+    ac.check_lse(out["lse"], lse_r)
+    dq_r, dk_r, dv_r = oracle.bwd(q, k, v, do, 0.3, False)
+    for name, r in (("dq", dq_r), ("dk", dk_r), ("dv", dv_r)):
+        ac.check_grad(out[name], r, name)
 
 
 @pytest.mark.parametrize("name", ["tiny", "gpt2", "mha4k", "gqa16k", "long64k"])
@@ -206,6 +231,37 @@ def test_workload(name):
             rep.update(ac.check_invariants(q, k, do, out))
         print(name, causal, rep)
         del out
+
+
+def test_repeated_full_size_runs_are_stable():
+    """The 4K-token MHA workload run many times in a row.  O, lse, dK and dV
+    must be bitwise equal on every run (their reductions have a fixed order;
+    only dQ is reduce-added in a varying order, within 1e-3 relative of the
+    first run); the first run is checked against the oracle on seeded rows.
+    This guards the schedules' reliance on the tensor core reading an MMA's
+    operands before a later MMA of the same thread overwrites them."""
+    w = WORKLOADS["mha4k"]
+    q, k, v, do = make_inputs(w)
+    dev = [t.cuda() for t in (q, k, v, do)]
+    o0, l0 = binding.attention_fwd(dev[0], dev[1], dev[2], w.scale, True)
+    ws = torch.empty(binding.fa_bwd_workspace_bytes(w.B, w.Hq, w.Hkv, w.N, w.d), device="cuda",
+                     dtype=torch.uint8)
+    g0 = binding.attention_bwd(dev[0], dev[1], dev[2], o0, dev[3], l0, w.scale, True, workspace=ws)
+    assert binding.fa_get_device_status() == binding.FA_OK
+    o, lse = torch.empty_like(o0), torch.empty_like(l0)
+    for _ in range(24):
+        binding.fa_fwd(dev[0], dev[1], dev[2], o, lse, w.scale, True)
+        assert torch.equal(o, o0) and torch.equal(lse, l0)
+    dq, dk, dv = (torch.empty_like(t) for t in g0)
+    for _ in range(12):
+        binding.fa_bwd(dev[0], dev[1], dev[2], o0, dev[3], l0, dq, dk, dv, w.scale, True, ws)
+        assert torch.equal(dk, g0[1]) and torch.equal(dv, g0[2])
+        rel = ((dq.float() - g0[0].float()).norm() / g0[0].float().norm()).item()
+        assert rel <= 1e-3, rel
+    assert binding.fa_get_device_status() == binding.FA_OK
+    out = {"o": o0.cpu(), "lse": l0.cpu(), "dq": g0[0].cpu(), "dk": g0[1].cpu(), "dv": g0[2].cpu()}
+    rows = check_rows(w)[::8]
+    print(ac.check_rows(q, k, v, do, w.scale, True, out, rows))
 
 
 def test_forward_is_deterministic():
