@@ -10,7 +10,7 @@ replica (the path has no exchange step), so scaling is weak.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
   python bench.py --impl reference ...   # the CPU oracle arm
-  python bench.py --window W | --dropout P | --decode | --fp8   # the variants
+  python bench.py --window W | --dropout P | --block-mask KIND | --decode | --fp8   # the variants
 
 Timing: W untimed steps, then K steps between a barrier + synchronize on both
 sides, CUDA events on the launching stream, max over ranks.  The inputs
@@ -165,7 +165,46 @@ def kernel_stats(ms):
     return {"mean": statistics.mean(ms), "median": statistics.median(ms), "min": min(ms)}
 
 
-def alloc_problem(w, rank, device):
+def block_mask_for(kind, w):
+    """A block mask over 128 x 128 blocks for workload w, by name:
+    'local': each query block sees itself and the 2 key blocks before it,
+    plus the first key block (global tokens), and the first query block sees
+    all; 'random:RHO': every (head, query block, key block) visible with
+    probability RHO (seeded), the diagonal always."""
+    nb = -(-w.N // 128)
+    if kind == "local":
+        m = torch.zeros((nb, nb), dtype=torch.uint8)
+        for i in range(nb):
+            m[i, max(0, i - 2):i + 1] = 1
+        m[:, 0] = 1
+        m[0, :] = 1
+        return m
+    if kind.startswith("random:"):
+        rho = float(kind.split(":", 1)[1])
+        g = torch.Generator("cpu").manual_seed(w.seed + 13)
+        m = (torch.rand((w.Hq, nb, nb), generator=g) < rho).to(torch.uint8)
+        m[:, torch.arange(nb), torch.arange(nb)] = 1
+        return m
+    raise SystemExit(f"bench.py: unknown block mask {kind!r} (local | random:RHO)")
+
+
+def visible_pairs(mask, w, causal):
+    """(query, key) pairs a block mask (and the causal mask) leaves visible,
+    summed over heads and batch entries."""
+    nb = mask.shape[-1]
+    sizes = torch.tensor([min(128, w.N - 128 * i) for i in range(nb)], dtype=torch.float64)
+    pair = sizes[:, None] * sizes[None, :]
+    if causal:
+        # off-diagonal blocks below the diagonal are whole; a diagonal block
+        # of n rows has n(n+1)/2 visible pairs
+        pair = torch.tril(pair, -1) + torch.diag(sizes * (sizes + 1) / 2)
+    m = mask.to(torch.float64)
+    per_head = (m * pair).sum(dim=(-1, -2))
+    total = per_head.sum() * (w.Hq if m.dim() == 2 else 1)
+    return float(total) * w.B
+
+
+def alloc_problem(w, rank, device, block_mask=False):
     """Device tensors of one replica of workload w (inputs drawn on the device)."""
     B, Hq, Hkv, N, d = w.B, w.Hq, w.Hkv, w.N, w.d
     g = torch.Generator(device=device).manual_seed(rank_seed(w, rank))
@@ -174,11 +213,13 @@ def alloc_problem(w, rank, device):
     o = torch.empty_like(q)
     lse = torch.empty((B, Hq, N), device=device, dtype=torch.float32)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    ws = torch.empty(binding.fa_bwd_workspace_bytes(B, Hq, Hkv, N, d), device=device, dtype=torch.uint8)
+    nbytes = (binding.fa_bwd_blockmask_workspace_bytes if block_mask else binding.fa_bwd_workspace_bytes)(
+        B, Hq, Hkv, N, d)
+    ws = torch.empty(nbytes, device=device, dtype=torch.uint8)
     return dict(q=q, k=k, v=v, do=do, o=o, lse=lse, dq=dq, dk=dk, dv=dv, ws=ws)
 
 
-def make_step(t, w, causal, W, DR, stream, fwd_ev=None, bwd_ev=None):
+def make_step(t, w, causal, W, DR, stream, fwd_ev=None, bwd_ev=None, BM=None):
     """One pass of the hot path (fa_fwd then fa_bwd) on the tensors t; with
     events, the i-th call records around each of the two calls on `stream`."""
     q, k, v, do, o, lse, dq, dk, dv, ws = (t[n] for n in ("q", "k", "v", "do", "o", "lse", "dq", "dk", "dv", "ws"))
@@ -187,7 +228,9 @@ def make_step(t, w, causal, W, DR, stream, fwd_ev=None, bwd_ev=None):
     def step(i=None):
         if i is not None:
             fwd_ev[i][0].record(stream)
-        if DR:
+        if BM is not None:
+            binding.fa_fwd_blockmask(q, k, v, o, lse, scale, causal, BM, stream)
+        elif DR:
             binding.fa_fwd_dropout(q, k, v, o, lse, scale, causal, DR[0], DR[1], stream)
         elif W:
             binding.fa_fwd_window(q, k, v, o, lse, scale, W, stream)
@@ -196,7 +239,9 @@ def make_step(t, w, causal, W, DR, stream, fwd_ev=None, bwd_ev=None):
         if i is not None:
             fwd_ev[i][1].record(stream)
             bwd_ev[i][0].record(stream)
-        if DR:
+        if BM is not None:
+            binding.fa_bwd_blockmask(q, k, v, o, do, lse, dq, dk, dv, scale, causal, BM, ws, stream)
+        elif DR:
             binding.fa_bwd_dropout(q, k, v, o, do, lse, dq, dk, dv, scale, causal, DR[0], DR[1], ws, stream)
         elif W:
             binding.fa_bwd_window(q, k, v, o, do, lse, dq, dk, dv, scale, W, ws, stream)
@@ -207,13 +252,13 @@ def make_step(t, w, causal, W, DR, stream, fwd_ev=None, bwd_ev=None):
     return step
 
 
-def time_steps(args, w, causal, rank, world, device, steps, warmup, W=0, DR=None, clocks=None):
+def time_steps(args, w, causal, rank, world, device, steps, warmup, W=0, DR=None, clocks=None, BM=None):
     """W untimed steps, then `steps` timed ones between a barrier and a
     synchronize on both sides; CUDA events on the launching stream around the
     whole region, around every fa_fwd and fa_bwd call, and (through the
     library) around every launch of the forward kernel and of the backward
     main kernel.  Returns the timings (ms; the total is the max over ranks)."""
-    t = alloc_problem(w, rank, device)
+    t = alloc_problem(w, rank, device, block_mask=BM is not None)
     stream = torch.cuda.current_stream(device)
     ev = lambda: torch.cuda.Event(enable_timing=True)
     K = steps
@@ -224,7 +269,7 @@ def time_steps(args, w, causal, rank, world, device, steps, warmup, W=0, DR=None
     for a, b in kf_ev + kb_ev:  # materialise the handles the library records into
         a.record(stream)
         b.record(stream)
-    step = make_step(t, w, causal, W, DR, stream, fwd_ev, bwd_ev)
+    step = make_step(t, w, causal, W, DR, stream, fwd_ev, bwd_ev, BM)
     for _ in range(warmup):
         step()
     torch.cuda.synchronize(device)
@@ -261,9 +306,9 @@ def time_steps(args, w, causal, rank, world, device, steps, warmup, W=0, DR=None
     return res
 
 
-def summarize(w, causal, res, K, peak, W=0):
+def summarize(w, causal, res, K, peak, W=0, flops=None):
     """TFLOPS and % of peak of a timed run (medians of per-call times)."""
-    f_fwd, f_bwd = w.flops_fwd(causal, W), w.flops_bwd(causal, W)
+    f_fwd, f_bwd = flops if flops else (w.flops_fwd(causal, W), w.flops_bwd(causal, W))
     tf = lambda f, ms: f / (ms * 1e-3) / 1e12
     fwd, bwd, bm = res["fwd"]["median"], res["bwd"]["median"], res["bwd_main"]["median"]
     return {
@@ -292,13 +337,19 @@ def run_ours(args, w, causal, rank, world, device):
     binding.load()
     W = args.window
     DR = (args.dropout, 0x5EED0000 + rank) if args.dropout else None
+    BMh = block_mask_for(args.block_mask, w) if args.block_mask else None
+    BM = BMh.to(device) if BMh is not None else None
     K = args.steps
     clocks = ClockSampler(device) if rank == 0 else None
-    res = time_steps(args, w, causal, rank, world, device, K, args.warmup, W, DR, clocks)
+    res = time_steps(args, w, causal, rank, world, device, K, args.warmup, W, DR, clocks, BM)
     clk = res["clocks"]
     t = res.pop("tensors")
     ms_step = res["ms_total"] / K
     f_fwd, f_bwd = w.flops_fwd(causal, W), w.flops_bwd(causal, W)
+    if BM is not None:
+        # FLOPs over the (query, key) pairs the mask leaves visible
+        f_fwd = 4.0 * w.d * visible_pairs(BMh, w, causal)
+        f_bwd = 2.5 * f_fwd
     value = job_tflops(world, f_fwd + f_bwd, ms_step)
     fwd_ms, bwd_ms = res["fwd"]["median"], res["bwd"]["median"]
     fwd_kern_mean, bwd_main_mean = res["fwd_kernel"]["mean"], res["bwd_main"]["mean"]
@@ -319,7 +370,7 @@ def run_ours(args, w, causal, rank, world, device):
         sets.append({n: torch.empty_like(x) for n, x in sets[0].items()})
         hout = [[torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for x in outs_like] for _ in sets]
         streams = [torch.cuda.Stream(device) for _ in sets]
-        steps_e = [make_step(b, w, causal, W, DR, st) for b, st in zip(sets, streams)]
+        steps_e = [make_step(b, w, causal, W, DR, st, BM=BM) for b, st in zip(sets, streams)]
         h2d = sum(x.numel() * x.element_size() for x in hin)
         d2h = sum(x.numel() * x.element_size() for x in hout[0])
 
@@ -365,16 +416,18 @@ def run_ours(args, w, causal, rank, world, device):
 
     pk, pk_kind = peaks()
     peak = pk["bf16_tflops"]
-    head = summarize(w, causal, res, K, peak, W)
+    head = summarize(w, causal, res, K, peak, W, (f_fwd, f_bwd))
     bwd_tflops_main = f_bwd / (bwd_main_mean * 1e-3) / 1e12
-    launches_per_step = 4
+    launches_per_step = 3  # fa_fwd_kernel, fa_bwd_pre_kernel, fa_bwd_kernel
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": str(w.dtype).replace("torch.", ""),
         "data": "synthetic: seeded normals (per-rank CUDA generator) with the workload's shapes and sigmas",
         "config": {"workload": workload_desc(w, causal) + (f" window={W}" if W else "")
-                   + (f" dropout={args.dropout}" if DR else ""),
+                   + (f" dropout={args.dropout}" if DR else "")
+                   + (f" block_mask={args.block_mask} (visible fraction "
+                      f"{f_fwd / w.flops_fwd(causal):.3f})" if BM is not None else ""),
                    "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv,
                    "seq_len": w.N, "head_dim": w.d, "causal": causal, "window": W,
                    "dropout": args.dropout,
@@ -396,7 +449,8 @@ def run_ours(args, w, causal, rank, world, device):
                      "traffic": profiled_traffic(w.name) if not (W or DR) else None,
                      "traffic_unit": "bytes per launch (ncu)",
                      "algorithmic": "2.5 x 4*B*Hq*N^2*d (/2 causal) FLOPs per launch"
-                                    + (" (visible pairs under the window)" if W else "")},
+                                    + (" (visible pairs under the window)" if W else "")
+                                    + (" (visible pairs under the block mask)" if BM is not None else "")},
         "forward_kernel": {"kernel": "fa_fwd_kernel", "bound": "tensor",
                            "achieved": round(f_fwd / (fwd_kern_mean * 1e-3) / 1e12, 2), "peak": peak,
                            "unit": "TFLOP/s",
@@ -407,7 +461,7 @@ def run_ours(args, w, causal, rank, world, device):
     }
     # the rest of the metric's range (N = 16K GQA, N = 64K fp16), each on
     # its own inputs, fewer steps (each step is longer)
-    if not (W or DR or args.no_range) and w.name == "mha4k" and causal:
+    if not (W or DR or BM is not None or args.no_range) and w.name == "mha4k" and causal:
         subs = []
         for name in RANGE_WORKLOADS:
             ws_ = WORKLOADS[name]
@@ -683,6 +737,9 @@ def main():
                     help="dropout probability on the attention probabilities (0: none)")
     ap.add_argument("--window", type=int, default=0,
                     help="causal sliding window of this many keys (0: none); FLOPs counted over visible pairs")
+    ap.add_argument("--block-mask", default="",
+                    help="block-sparse mask over 128 x 128 blocks: 'local' or 'random:RHO'; FLOPs "
+                         "counted over visible pairs")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-range", action="store_true",
                     help="skip the 16K GQA and 64K fp16 sub-results of the default line")
@@ -693,8 +750,8 @@ def main():
 
     w = WORKLOADS[args.workload]
     causal = (not args.noncausal) and (True in w.causal_modes)
-    if args.window and args.dropout:
-        raise SystemExit("bench.py: --window and --dropout are not combined")
+    if sum(bool(x) for x in (args.window, args.dropout, args.block_mask)) > 1:
+        raise SystemExit("bench.py: --window, --dropout and --block-mask are not combined")
     if args.window:
         assert args.window > 0 and causal, "--window needs a causal workload"
         if args.impl == "reference":
@@ -730,7 +787,7 @@ def main():
                 print(json.dumps(line), flush=True)
             return
         line = run_ours(args, w, causal, rank, world, device)
-        if rank == 0 and not args.no_cpu_baseline and not args.window and not args.dropout:
+        if rank == 0 and not args.no_cpu_baseline and not (args.window or args.dropout or args.block_mask):
             v, rows, dt, threads = oracle_sample(w, causal, args.cpu_seconds)
             line["cpu_baseline"] = {
                 "value": round(v, 6), "unit": UNIT, "cores": threads, "kind": "oracle",

@@ -65,6 +65,12 @@ def load():
             lib.fa_bwd_dropout.restype = i
             lib.fa_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, f, f, f, i, i, vp]
             lib.fa_fwd_fp8.restype = i
+            lib.fa_fwd_blockmask.argtypes = [vp] * 5 + [i] * 5 + [f, i, vp, i, i, vp]
+            lib.fa_fwd_blockmask.restype = i
+            lib.fa_bwd_blockmask_workspace_bytes.argtypes = [i, i, i, i, i]
+            lib.fa_bwd_blockmask_workspace_bytes.restype = ctypes.c_size_t
+            lib.fa_bwd_blockmask.argtypes = ([vp] * 9 + [i] * 5 + [f, i, vp, i, i, vp, ctypes.c_size_t, vp])
+            lib.fa_bwd_blockmask.restype = i
             lib.fa_decode_workspace_bytes.argtypes = [i, i, i, i, i, i]
             lib.fa_decode_workspace_bytes.restype = ctypes.c_size_t
             lib.fa_decode_paged.argtypes = ([vp] * 7 + [i] * 8 + [f, i, vp, ctypes.c_size_t, vp])
@@ -238,6 +244,58 @@ def fa_bwd_dropout(q, k, v, o, dout, lse, dq, dk, dv, scale: float, causal: bool
     _check(st, "fa_bwd_dropout")
 
 
+def _block_mask(where, block_mask, Hq, N, device):
+    """(tensor, mask_per_head) of a block mask over 128 x 128 blocks: a bool
+    or uint8 CUDA tensor [nb, nb] (every head) or [Hq, nb, nb], nb = ceil(N/128)."""
+    nb = -(-N // 128)
+    if block_mask is None or isinstance(block_mask, int):
+        raise ValueError(f"{where}: a block mask tensor is required")
+    if block_mask.dtype not in (torch.uint8, torch.bool):
+        raise TypeError(f"{where}: block_mask has dtype {block_mask.dtype}, expected uint8 or bool")
+    if tuple(block_mask.shape) == (nb, nb):
+        per_head = 0
+    elif tuple(block_mask.shape) == (Hq, nb, nb):
+        per_head = 1
+    else:
+        raise ValueError(f"{where}: block_mask has shape {tuple(block_mask.shape)}, expected "
+                         f"({nb}, {nb}) or ({Hq}, {nb}, {nb})")
+    if not block_mask.is_cuda or block_mask.device != device:
+        raise ValueError(f"{where}: block_mask must be on {device}")
+    if not block_mask.is_contiguous():
+        raise ValueError(f"{where}: block_mask must be contiguous")
+    return block_mask.view(torch.uint8) if block_mask.dtype == torch.bool else block_mask, per_head
+
+
+def fa_fwd_blockmask(q, k, v, o, lse, scale: float, causal: bool, block_mask, stream=None) -> None:
+    """Forward under a block mask over 128-row x 128-key blocks (see
+    _block_mask for its layout); combined with the causal mask when causal."""
+    B, Hq, Hkv, N, d = _expect_attention("fa_fwd_blockmask", q, k, v, o, lse)
+    m, per_head = _block_mask("fa_fwd_blockmask", block_mask, Hq, N, q.device)
+    st = load().fa_fwd_blockmask(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, N, d,
+                                 float(scale), int(bool(causal)), _ptr(m), per_head, _DTYPES[q.dtype],
+                                 _stream(stream))
+    _check(st, "fa_fwd_blockmask")
+
+
+def fa_bwd_blockmask_workspace_bytes(B: int, Hq: int, Hkv: int, N: int, d: int) -> int:
+    return int(load().fa_bwd_blockmask_workspace_bytes(B, Hq, Hkv, N, d))
+
+
+def fa_bwd_blockmask(q, k, v, o, dout, lse, dq, dk, dv, scale: float, causal: bool, block_mask,
+                     workspace, stream=None) -> None:
+    """Backward of fa_fwd_blockmask with the same mask; workspace of at least
+    fa_bwd_blockmask_workspace_bytes(...) bytes."""
+    B, Hq, Hkv, N, d = _expect_attention("fa_bwd_blockmask", q, k, v, o, lse, dout, dq, dk, dv,
+                                         workspace)
+    m, per_head = _block_mask("fa_bwd_blockmask", block_mask, Hq, N, q.device)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = load().fa_bwd_blockmask(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq),
+                                 _ptr(dk), _ptr(dv), B, Hq, Hkv, N, d, float(scale), int(bool(causal)),
+                                 _ptr(m), per_head, _DTYPES[q.dtype], _ptr(workspace), ws_bytes,
+                                 _stream(stream))
+    _check(st, "fa_bwd_blockmask")
+
+
 def fa_bwd_workspace_bytes(B: int, Hq: int, Hkv: int, N: int, d: int) -> int:
     return int(load().fa_bwd_workspace_bytes(B, Hq, Hkv, N, d))
 
@@ -328,17 +386,19 @@ def attention_decode_paged(q, k_cache, v_cache, block_table, seq_lens, scale: fl
 
 
 def attention_fwd(q, k, v, scale: float | None = None, causal: bool = False, stream=None,
-                  window: int = 0, dropout=None):
+                  window: int = 0, dropout=None, block_mask=None):
     """Allocates O and lse with PyTorch and runs fa_fwd (fa_fwd_window when
     window > 0, which implies causal; fa_fwd_dropout when dropout = (p_drop,
-    seed)); returns (O, lse)."""
-    if window and dropout:
-        raise ValueError("a sliding window and dropout are not combined")
+    seed); fa_fwd_blockmask when block_mask is given); returns (O, lse)."""
+    if sum(x is not None and x is not False and x != 0 for x in (window, dropout, block_mask)) > 1:
+        raise ValueError("a sliding window, dropout and a block mask are not combined")
     B, Hq, Hkv, N, d = _dims(q, k)
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     o = torch.empty_like(q)
     lse = torch.empty((B, Hq, N), device=q.device, dtype=torch.float32)
-    if window:
+    if block_mask is not None:
+        fa_fwd_blockmask(q, k, v, o, lse, scale, causal, block_mask, stream)
+    elif window:
         fa_fwd_window(q, k, v, o, lse, scale, window, stream)
     elif dropout:
         fa_fwd_dropout(q, k, v, o, lse, scale, causal, dropout[0], dropout[1], stream)
@@ -348,16 +408,20 @@ def attention_fwd(q, k, v, scale: float | None = None, causal: bool = False, str
 
 
 def attention_bwd(q, k, v, o, dout, lse, scale: float | None = None, causal: bool = False,
-                  workspace=None, stream=None, window: int = 0, dropout=None):
+                  workspace=None, stream=None, window: int = 0, dropout=None, block_mask=None):
     """Allocates dQ, dK, dV (and the workspace if not given) and runs fa_bwd
-    (fa_bwd_window when window > 0)."""
+    (fa_bwd_window when window > 0, fa_bwd_dropout with dropout,
+    fa_bwd_blockmask with a block mask)."""
     B, Hq, Hkv, N, d = _dims(q, k)
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     if workspace is None:
-        workspace = torch.empty(max(fa_bwd_workspace_bytes(B, Hq, Hkv, N, d), 16),
-                                device=q.device, dtype=torch.uint8)
-    if window:
+        nbytes = (fa_bwd_blockmask_workspace_bytes(B, Hq, Hkv, N, d) if block_mask is not None
+                  else fa_bwd_workspace_bytes(B, Hq, Hkv, N, d))
+        workspace = torch.empty(max(nbytes, 16), device=q.device, dtype=torch.uint8)
+    if block_mask is not None:
+        fa_bwd_blockmask(q, k, v, o, dout, lse, dq, dk, dv, scale, causal, block_mask, workspace, stream)
+    elif window:
         fa_bwd_window(q, k, v, o, dout, lse, dq, dk, dv, scale, window, workspace, stream)
     elif dropout:
         fa_bwd_dropout(q, k, v, o, dout, lse, dq, dk, dv, scale, causal, dropout[0], dropout[1],

@@ -149,9 +149,9 @@ fa_status_t opt_in_smem(K kernel, int smem) {
   return FA_OK;
 }
 
-template <int HD, bool BF, bool CA, bool DR>
+template <int HD, bool BF, bool CA, bool DR, bool BM = false>
 fa_status_t launch_fwd(const FwdParams& prm, cudaStream_t st) {
-  auto kern = fa::fa_fwd_kernel<HD, BF, CA, DR>;
+  auto kern = fa::fa_fwd_kernel<HD, BF, CA, DR, BM>;
   const int smem = FwdLayout<HD>::kDynSmem;
   fa_status_t s = opt_in_smem(kern, smem);
   if (s != FA_OK) return s;
@@ -165,6 +165,8 @@ fa_status_t launch_fwd(const FwdParams& prm, cudaStream_t st) {
 
 template <int HD, bool BF>
 fa_status_t launch_fwd_c(const FwdParams& prm, int causal, cudaStream_t st) {
+  if (prm.bmask != nullptr)
+    return causal ? launch_fwd<HD, BF, true, false, true>(prm, st) : launch_fwd<HD, BF, false, false, true>(prm, st);
   if (prm.drop_t > 0)
     return causal ? launch_fwd<HD, BF, true, true>(prm, st) : launch_fwd<HD, BF, false, true>(prm, st);
   return causal ? launch_fwd<HD, BF, true, false>(prm, st) : launch_fwd<HD, BF, false, false>(prm, st);
@@ -186,9 +188,9 @@ fa_status_t launch_fwd_fp8(const fa::Fp8FwdParams& prm, cudaStream_t st) {
   return ok ? FA_OK : FA_ERR_CUDA;
 }
 
-template <int HD, bool BF, bool CA, bool DR>
+template <int HD, bool BF, bool CA, bool DR, bool BM = false>
 fa_status_t launch_bwd_main(const fa::BwdParams& prm, int grid, cudaStream_t st) {
-  auto kern = fa::fa_bwd_kernel<HD, BF, CA, DR>;
+  auto kern = fa::fa_bwd_kernel<HD, BF, CA, DR, BM>;
   const int smem = fa::BwdLayout<HD>::kDynSmem;
   fa_status_t s = opt_in_smem(kern, smem);
   if (s != FA_OK) return s;
@@ -203,19 +205,68 @@ template <int HD, bool BF>
 fa_status_t bwd_run(const void* q, const void* k, const void* v, const void* o, const void* dout,
                     const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N,
                     float scale, int causal, int window, uint32_t drop_t, uint64_t seed,
-                    void* workspace, cudaStream_t st) {
+                    void* workspace, cudaStream_t st, const uint8_t* bmask = nullptr,
+                    long long bm_hstride = 0) {
   const int64_t Np = fa::bwd_padded_rows(N);
   const int64_t BHq = static_cast<int64_t>(B) * Hq, BHkv = static_cast<int64_t>(B) * Hkv;
   float* Dvec = static_cast<float*>(workspace);
   float* lse2 = Dvec + BHq * Np;
   float* dqacc = lse2 + BHq * Np;
   const int64_t rows = BHq * Np;
-  unsigned* work_counter = reinterpret_cast<unsigned*>(dqacc + rows * HD);
+  unsigned* dq_count = reinterpret_cast<unsigned*>(dqacc + rows * HD);
+  unsigned* work_counter = dq_count + rows / 64;
+  const int n_ktiles = (N + 127) / 128;
 
-  // 1. D, lse2, zeroed accumulator and work counter
-  fa::fa_bwd_pre_kernel<HD, BF><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(
-      o, dout, lse, Dvec, lse2, dqacc, work_counter, N, static_cast<int>(Np), rows);
+  // 1. D, lse2, zeroed accumulator, arrival counters and work counter
+  fa::BwdPreParams pre;
+  std::memset(&pre, 0, sizeof(pre));
+  pre.o = o;
+  pre.dout = dout;
+  pre.lse = lse;
+  pre.Dvec = Dvec;
+  pre.lse2 = lse2;
+  pre.dqacc = dqacc;
+  pre.dq_count = dq_count;
+  pre.work_counter = work_counter;
+  pre.dq = dq;
+  pre.bmask = bmask;
+  pre.bm_hstride = bm_hstride;
+  pre.N = N;
+  pre.Np = static_cast<int>(Np);
+  pre.Hq = Hq;
+  pre.n_ktiles = n_ktiles;
+  pre.causal = causal;
+  pre.window = window;
+  pre.total_rows = rows;
+  fa::fa_bwd_pre_kernel<HD, BF><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(pre);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+
+  // 1b. block mask: the walk of every work item
+  uint16_t* plan_list = nullptr;
+  int* plan_steps = nullptr;
+  const int plan_cap = (Hq / Hkv) * n_ktiles;
+  if (bmask != nullptr) {
+    plan_steps = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(workspace) + fa::bwd_workspace_bytes(B, Hq, N, HD));
+    plan_list = reinterpret_cast<uint16_t*>(plan_steps + BHkv * n_ktiles);
+    fa::BwdPlanParams pl;
+    std::memset(&pl, 0, sizeof(pl));
+    pl.bmask = bmask;
+    pl.bm_hstride = bm_hstride;
+    pl.list = plan_list;
+    pl.steps = plan_steps;
+    pl.N = N;
+    pl.Hq = Hq;
+    pl.Hkv = Hkv;
+    pl.group = Hq / Hkv;
+    pl.n_ktiles = n_ktiles;
+    pl.n_qtiles = (N + 63) / 64;
+    pl.causal = causal;
+    pl.window = window;
+    pl.cap = plan_cap;
+    pl.n_items = static_cast<int>(BHkv * n_ktiles);
+    fa::fa_bwd_plan_kernel<<<static_cast<unsigned>((pl.n_items + 7) / 8), 256, 0, st>>>(pl);
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  }
 
   // 2. main pass
   const CUtensorMapDataType dt = BF ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
@@ -229,6 +280,11 @@ fa_status_t bwd_run(const void* q, const void* k, const void* v, const void* o, 
   prm.lse2 = lse2;
   prm.Dvec = Dvec;
   prm.dqacc = dqacc;
+  prm.dq_count = dq_count;
+  prm.dq = dq;
+  prm.plan_list = plan_list;
+  prm.plan_steps = plan_steps;
+  prm.plan_cap = plan_cap;
   prm.dk = dk;
   prm.dv = dv;
   prm.work_counter = work_counter;
@@ -261,19 +317,15 @@ fa_status_t bwd_run(const void* q, const void* k, const void* v, const void* o, 
   if ((n_sm = sm_count()) <= 0) return FA_ERR_CUDA;
   const int cap = g_bwd_max_blocks.load();
   const int grid = std::min(prm.n_items, cap > 0 ? std::min(cap, n_sm) : n_sm);  // persistent
+  if (bmask != nullptr)
+    return causal ? launch_bwd_main<HD, BF, true, false, true>(prm, grid, st)
+                  : launch_bwd_main<HD, BF, false, false, true>(prm, grid, st);
   fa_status_t s = prm.drop_t > 0
                       ? (causal ? launch_bwd_main<HD, BF, true, true>(prm, grid, st)
                                 : launch_bwd_main<HD, BF, false, true>(prm, grid, st))
                       : (causal ? launch_bwd_main<HD, BF, true, false>(prm, grid, st)
                                 : launch_bwd_main<HD, BF, false, false>(prm, grid, st));
-  if (s != FA_OK) return s;
-
-  // 3. dQ = scale * accumulator
-  const int64_t total_vec = BHq * N * (HD / 8);
-  const int64_t blocks = std::min<int64_t>((total_vec + 255) / 256, 148 * 16);
-  fa::fa_bwd_post_kernel<HD, BF><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
-      dqacc, dq, N, static_cast<int>(Np), total_vec, scale);
-  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+  return s;
 }
 
 }  // namespace
@@ -286,7 +338,8 @@ namespace {
 
 fa_status_t fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                      int Hq, int Hkv, int N, int d, float scale, int causal, int window,
-                     uint32_t drop_t, uint64_t seed, fa_dtype_t dtype, void* stream) {
+                     uint32_t drop_t, uint64_t seed, fa_dtype_t dtype, void* stream,
+                     const uint8_t* bmask = nullptr, long long bm_hstride = 0) {
   bool empty = false;
   fa_status_t s = check_common(B, Hq, Hkv, N, d, scale, causal, dtype, &empty);
   if (s != FA_OK) return s;
@@ -320,6 +373,8 @@ fa_status_t fwd_impl(const void* q, const void* k, const void* v, void* o, float
   prm.drop_scale = drop_t ? 256.0f / static_cast<float>(256u - drop_t) : 1.0f;
   prm.seed_lo = static_cast<uint32_t>(seed);
   prm.seed_hi = static_cast<uint32_t>(seed >> 32);
+  prm.bmask = bmask;
+  prm.bm_hstride = bm_hstride;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (d == 128) return bf ? launch_fwd_c<128, true>(prm, causal, st) : launch_fwd_c<128, false>(prm, causal, st);
   return bf ? launch_fwd_c<64, true>(prm, causal, st) : launch_fwd_c<64, false>(prm, causal, st);
@@ -403,17 +458,38 @@ size_t fa_bwd_workspace_bytes(int B, int Hq, int Hkv, int N, int d) {
 
 namespace {
 
+// Block-mask additions to the backward workspace: the step count and the
+// walk of every work item (see fa_bwd_plan_kernel).
+size_t bwd_mask_plan_bytes(int B, int Hq, int Hkv, int N) {
+  const int64_t n_ktiles = (static_cast<int64_t>(N) + 127) / 128;
+  const int64_t items = static_cast<int64_t>(B) * Hkv * n_ktiles;
+  const int64_t cap = static_cast<int64_t>(Hq / Hkv) * n_ktiles;
+  return static_cast<size_t>(items) * 4u + static_cast<size_t>(items * cap) * 2u;
+}
+
+// Sizes a block mask supports: the walk entries hold the group head in 4
+// bits and the query block in 12.
+bool bmask_supported(int Hq, int Hkv, int N) {
+  return Hq / Hkv <= 16 && (static_cast<int64_t>(N) + 127) / 128 <= 4096;
+}
+
 fa_status_t bwd_impl(const void* q, const void* k, const void* v, const void* o, const void* dout,
                      const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N,
                      int d, float scale, int causal, int window, uint32_t drop_t, uint64_t seed,
-                     fa_dtype_t dtype, void* workspace, size_t workspace_bytes, void* stream) {
+                     fa_dtype_t dtype, void* workspace, size_t workspace_bytes, void* stream,
+                     const uint8_t* bmask = nullptr, long long bm_hstride = 0) {
   bool empty = false;
   fa_status_t s = check_common(B, Hq, Hkv, N, d, scale, causal, dtype, &empty);
   if (s != FA_OK) return s;
   if (empty) return FA_OK;
   if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv || !workspace)
     return FA_ERR_INVALID_ARG;
-  if (workspace_bytes < fa::bwd_workspace_bytes(B, Hq, N, d)) return FA_ERR_INVALID_ARG;
+  size_t need = fa::bwd_workspace_bytes(B, Hq, N, d);
+  if (bmask != nullptr) {
+    if (!bmask_supported(Hq, Hkv, N)) return FA_ERR_UNSUPPORTED;
+    need += bwd_mask_plan_bytes(B, Hq, Hkv, N);
+  }
+  if (workspace_bytes < need) return FA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
       !aligned16(lse) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
       !aligned16(workspace))
@@ -422,10 +498,10 @@ fa_status_t bwd_impl(const void* q, const void* k, const void* v, const void* o,
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const bool bf = dtype == FA_BF16;
   if (d == 128)
-    return bf ? bwd_run<128, true>(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, N, scale, causal, window, drop_t, seed, workspace, st)
-              : bwd_run<128, false>(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, N, scale, causal, window, drop_t, seed, workspace, st);
-  return bf ? bwd_run<64, true>(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, N, scale, causal, window, drop_t, seed, workspace, st)
-            : bwd_run<64, false>(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, N, scale, causal, window, drop_t, seed, workspace, st);
+    return bf ? bwd_run<128, true>(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, N, scale, causal, window, drop_t, seed, workspace, st, bmask, bm_hstride)
+              : bwd_run<128, false>(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, N, scale, causal, window, drop_t, seed, workspace, st, bmask, bm_hstride);
+  return bf ? bwd_run<64, true>(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, N, scale, causal, window, drop_t, seed, workspace, st, bmask, bm_hstride)
+            : bwd_run<64, false>(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, N, scale, causal, window, drop_t, seed, workspace, st, bmask, bm_hstride);
 }
 
 }  // namespace
@@ -458,6 +534,33 @@ fa_status_t fa_bwd_dropout(const void* q, const void* k, const void* v, const vo
   if (!drop_threshold(p_drop, &t)) return FA_ERR_INVALID_ARG;
   return bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, N, d, scale, causal, 0,
                   static_cast<uint32_t>(t), seed, dtype, workspace, workspace_bytes, stream);
+}
+
+fa_status_t fa_fwd_blockmask(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                             int Hq, int Hkv, int N, int d, float scale, int causal,
+                             const uint8_t* block_mask, int mask_per_head, fa_dtype_t dtype,
+                             void* stream) {
+  if (block_mask == nullptr || (mask_per_head != 0 && mask_per_head != 1)) return FA_ERR_INVALID_ARG;
+  if (Hq > 0 && Hkv > 0 && Hq % Hkv == 0 && !bmask_supported(Hq, Hkv, N)) return FA_ERR_UNSUPPORTED;
+  const long long nb = (static_cast<long long>(N) + 127) / 128;
+  return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, causal, 0, 0, 0, dtype, stream, block_mask,
+                  mask_per_head ? nb * nb : 0);
+}
+
+size_t fa_bwd_blockmask_workspace_bytes(int B, int Hq, int Hkv, int N, int d) {
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || N <= 0 || d <= 0 || Hq % Hkv != 0) return 0;
+  return fa::bwd_workspace_bytes(B, Hq, N, d) + bwd_mask_plan_bytes(B, Hq, Hkv, N);
+}
+
+fa_status_t fa_bwd_blockmask(const void* q, const void* k, const void* v, const void* o,
+                             const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
+                             int Hq, int Hkv, int N, int d, float scale, int causal,
+                             const uint8_t* block_mask, int mask_per_head, fa_dtype_t dtype,
+                             void* workspace, size_t workspace_bytes, void* stream) {
+  if (block_mask == nullptr || (mask_per_head != 0 && mask_per_head != 1)) return FA_ERR_INVALID_ARG;
+  const long long nb = (static_cast<long long>(N) + 127) / 128;
+  return bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, N, d, scale, causal, 0, 0, 0, dtype,
+                  workspace, workspace_bytes, stream, block_mask, mask_per_head ? nb * nb : 0);
 }
 
 fa_status_t fa_get_device_status(void* stream) {

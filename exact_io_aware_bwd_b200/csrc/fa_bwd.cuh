@@ -15,8 +15,9 @@
 //
 // Three kernels:
 //   bwd_pre   one warp per query row: D_i = dO_i . O_i, lse2_i = lse_i log2(e)
-//             (+inf for padding rows, which makes their P exactly 0), and a
-//             zeroed fp32 dQ accumulator row.
+//             (+inf for padding rows, which makes their P exactly 0), a
+//             zeroed fp32 dQ accumulator row and, per 64-row query block, a
+//             zeroed arrival counter.
 //   bwd_main  persistent: one thread block per SM takes work items (128-row
 //             key block j, kv head) one after another from a counter in the
 //             workspace, head-major and, within a head, the key blocks with
@@ -38,7 +39,11 @@
 //             item's Q / dO loads start while the last steps of the previous
 //             one run, and its dK / dV are written out while the next item's
 //             first steps run.
-//   bwd_post  dQ = scale * accumulator, converted to the I/O dtype.
+//             A query block's dQ is final once every key block that sees it
+//             has added its part: each addition is counted, and the drain
+//             warps of the block that brings the last one convert the query
+//             block (dQ = scale * accumulator, to the I/O dtype) while it is
+//             still in L2.  No separate pass over the accumulator.
 //
 // Warp roles of bwd_main (448 threads):
 //   warps 0-7   softmax-gradient: warp w owns key rows 32(w%4)..+31 (tensor
@@ -65,57 +70,154 @@ namespace fa {
 
 constexpr uint32_t kKernBwdPre = 2;
 constexpr uint32_t kKernBwd = 3;
-constexpr uint32_t kKernBwdPost = 4;
 constexpr uint32_t kKernSelftest = 9;
 
 __host__ __device__ inline int64_t bwd_padded_rows(int N) { return (static_cast<int64_t>(N) + 127) / 128 * 128; }
 
-// Workspace: D [rows], lse2 [rows], dQ accumulator [rows][d] (fp32), then
-// 256 bytes holding the work-item counter of bwd_main.
+// Workspace: D [rows], lse2 [rows], dQ accumulator [rows][d] (fp32), one
+// arrival counter per 64-row query block [rows / 64] (uint32), then 256 bytes
+// holding the work-item counter of bwd_main.
 constexpr size_t kBwdWorkspaceTail = 256;
 
 inline size_t bwd_workspace_bytes(int B, int Hq, int N, int d) {
   const int64_t rows = static_cast<int64_t>(B) * Hq * bwd_padded_rows(N);
-  return static_cast<size_t>(rows) * 4u * static_cast<size_t>(2 + d) + kBwdWorkspaceTail;
+  return static_cast<size_t>(rows) * 4u * static_cast<size_t>(2 + d) + static_cast<size_t>(rows / 64) * 4u +
+         kBwdWorkspaceTail;
 }
 
 // ---------------------------------------------------------------------------
 // bwd_pre
 
+// Number of key blocks whose walk includes 64-row query block qt (of query
+// head hq within its batch): the additions its dQ accumulator receives.  A
+// key block jt walks query blocks [i0, i_end) (bwd_item); under a block
+// mask only those whose 128-row block it sees.  Counted by the whole warp.
+__device__ __forceinline__ unsigned bwd_dq_expected(int qt, int hq, int N, int n_ktiles, int causal,
+                                                    int window, const uint8_t* bmask,
+                                                    long long bm_hstride, int lane) {
+  int jt_lo = 0, jt_hi = n_ktiles - 1;
+  if (causal) {
+    jt_hi = min(qt >> 1, n_ktiles - 1);  // i0 = 2 jt <= qt
+    if (window > 0) {
+      // i_end > qt  <=>  128 jt + 126 + W >= 64 qt
+      const int num = 64 * qt - 126 - window;
+      jt_lo = num > 0 ? (num + 127) / 128 : 0;
+    }
+  }
+  if (jt_hi < jt_lo) return 0u;
+  if (bmask == nullptr) return static_cast<unsigned>(jt_hi - jt_lo + 1);
+  const uint8_t* row = bmask + hq * bm_hstride + static_cast<long long>(qt >> 1) * n_ktiles;
+  unsigned n = 0;
+  for (int j0 = jt_lo; j0 <= jt_hi; j0 += 32) {
+    const int jt = j0 + lane;
+    n += __popc(__ballot_sync(0xffffffffu, jt <= jt_hi && __ldg(row + jt) != 0));
+  }
+  return n;
+}
+
+struct BwdPreParams {
+  const void* o;
+  const void* dout;
+  const float* lse;
+  float* Dvec;            // [B*Hq][Np]
+  float* lse2;            // [B*Hq][Np]
+  float* dqacc;           // [B*Hq][Np][d], zeroed here
+  unsigned* dq_count;     // [B*Hq][Np / 64], set to the additions each query block will receive
+  unsigned* work_counter;
+  void* dq;               // rows of query blocks that no key block sees are zeroed here
+  const uint8_t* bmask;   // block mask or nullptr
+  long long bm_hstride;
+  int N, Np, Hq, n_ktiles, causal, window;
+  long long total_rows;
+};
+
 template <int HD, bool BF16>
-__global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const void* __restrict__ o_,
-                                                         const void* __restrict__ do_,
-                                                         const float* __restrict__ lse,
-                                                         float* __restrict__ Dvec,
-                                                         float* __restrict__ lse2,
-                                                         float* __restrict__ dqacc,
-                                                         unsigned* __restrict__ work_counter, int N,
-                                                         int Np, int64_t total_rows) {
+__global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const __grid_constant__ BwdPreParams p) {
   using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  if (blockIdx.x == 0 && threadIdx.x == 0) *work_counter = 0u;
-  if (row >= total_rows) return;
-  const int64_t bh = row / Np;
-  const int n = static_cast<int>(row % Np);
+  if (blockIdx.x == 0 && threadIdx.x == 0) *p.work_counter = 0u;
+  if (row >= p.total_rows) return;
+  const int64_t bh = row / p.Np;
+  const int n = static_cast<int>(row % p.Np);
+  const int N = p.N;
   constexpr int kPer = HD / 32;  // elements per lane: 2 or 4
   float acc = 0.f;
   if (n < N) {
     const int64_t base = (bh * N + n) * HD + lane * kPer;
-    const T* o = reinterpret_cast<const T*>(o_) + base;
-    const T* d = reinterpret_cast<const T*>(do_) + base;
+    const T* o = reinterpret_cast<const T*>(p.o) + base;
+    const T* d = reinterpret_cast<const T*>(p.dout) + base;
 #pragma unroll
     for (int e = 0; e < kPer; ++e) acc += static_cast<float>(o[e]) * static_cast<float>(d[e]);
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
   if (lane == 0) {
-    Dvec[row] = acc;
-    lse2[row] = n < N ? lse[bh * N + n] * 1.4426950408889634f : INFINITY;
+    p.Dvec[row] = acc;
+    p.lse2[row] = n < N ? p.lse[bh * N + n] * 1.4426950408889634f : INFINITY;
   }
-  float* z = dqacc + row * HD + lane * kPer;
+  if ((n & 63) == 0) {
+    const int qt = n >> 6;
+    const unsigned cnt = n < N ? bwd_dq_expected(qt, static_cast<int>(bh % p.Hq), N, p.n_ktiles, p.causal,
+                                                 p.window, p.bmask, p.bm_hstride, lane)
+                               : 0u;
+    if (lane == 0) p.dq_count[row >> 6] = cnt;
+    if (cnt == 0 && n < N) {
+      // no key block adds to this query block (only under a block mask):
+      // its dQ is zero and no conversion will write it
+      const int rows_here = min(64, N - n);
+      uint4* out = reinterpret_cast<uint4*>(reinterpret_cast<T*>(p.dq) + (bh * N + n) * HD);
+      for (int i = lane; i < rows_here * HD / 8; i += 32) out[i] = make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
+  float* z = p.dqacc + row * HD + lane * kPer;
 #pragma unroll
   for (int e = 0; e < kPer; ++e) z[e] = 0.f;
+}
+
+// ---------------------------------------------------------------------------
+// bwd_plan (block masks only): for every work item (kv head, 128-row key
+// block jt), the (group head, 128-row query block) pairs that see the key
+// block, in walk order, and the number of 64-row steps they make.  One warp
+// per item.  Entry = group head << 12 | query block.
+
+struct BwdPlanParams {
+  const uint8_t* bmask;
+  long long bm_hstride;
+  uint16_t* list;   // [BHkv * n_ktiles][cap]
+  int* steps;       // [BHkv * n_ktiles]
+  int N, Hq, Hkv, group, n_ktiles, n_qtiles, causal, window, cap, n_items;
+};
+
+__global__ void __launch_bounds__(256) fa_bwd_plan_kernel(const __grid_constant__ BwdPlanParams p) {
+  const int item = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (item >= p.n_items) return;
+  const int kvh = item / p.n_ktiles, jt = item % p.n_ktiles;
+  const int g = kvh % p.Hkv;
+  const int i0 = p.causal ? 2 * jt : 0;
+  const int i_end = (p.causal && p.window > 0)
+                        ? min(p.n_qtiles, (min(p.N - 1, jt * 128 + 126 + p.window)) / 64 + 1)
+                        : p.n_qtiles;
+  const int qb_lo = i0 >> 1, qb_hi = (i_end - 1) >> 1;
+  uint16_t* list = p.list + static_cast<long long>(item) * p.cap;
+  int pos = 0, steps = 0;
+  for (int hg = 0; hg < p.group; ++hg) {
+    const uint8_t* col = p.bmask + static_cast<long long>(g * p.group + hg) * p.bm_hstride + jt;
+    for (int qb0 = qb_lo; qb0 <= qb_hi; qb0 += 32) {
+      const int qb = qb0 + lane;
+      const bool vis = qb <= qb_hi && __ldg(col + static_cast<long long>(qb) * p.n_ktiles) != 0;
+      const unsigned m = __ballot_sync(0xffffffffu, vis);
+      if (vis) list[pos + __popc(m & ((1u << lane) - 1u))] = static_cast<uint16_t>((hg << 12) | qb);
+      int mine = 0;
+      if (vis) mine = (2 * qb >= i0 && 2 * qb < i_end) + (2 * qb + 1 >= i0 && 2 * qb + 1 < i_end);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) mine += __shfl_xor_sync(0xffffffffu, mine, off);
+      steps += mine;
+      pos += __popc(m);
+    }
+  }
+  if (lane == 0) p.steps[item] = steps;
 }
 
 // ---------------------------------------------------------------------------
@@ -129,9 +231,15 @@ struct BwdParams {
   const float* lse2;     // [B*Hq][Np]
   const float* Dvec;     // [B*Hq][Np]
   float* dqacc;          // [B*Hq][Np][d] fp32 accumulator
+  unsigned* dq_count;    // [B*Hq][Np / 64] additions received per query block
+  void* dq;              // [B*Hq][N][d]
   void* dk;              // [B*Hkv][N][d]
   void* dv;
   unsigned* work_counter;  // next work item (zeroed by bwd_pre)
+  // block mask (kernels instantiated with BMASK): the walk of each item, from bwd_plan
+  const uint16_t* plan_list;
+  const int* plan_steps;
+  int plan_cap;
   int N, Np, Hq, Hkv, group, n_ktiles, n_qtiles, BHkv, n_items;
   int chunk_heads;         // kv heads per chunk of the item order
   int window;              // causal sliding window of this many keys; 0: none
@@ -165,7 +273,8 @@ struct BwdLayout {
   static constexpr int kOffSched = kOffBar + kNumBars * 8;
   static constexpr int kOffTmemPtr = kOffSched + kSched * 4;
   static constexpr int kOffAbort = kOffTmemPtr + 4;
-  static constexpr int kSmemBytes = kOffAbort + 4;
+  static constexpr int kOffConv = kOffAbort + 4;         // drain warps: convert this block?
+  static constexpr int kSmemBytes = kOffConv + 4;
   // Tiles must sit on 1024-byte boundaries (128-byte swizzle atoms).  The
   // dynamic shared memory of a block without static shared memory starts on
   // such a boundary on sm_100; the d = 64 layout keeps spare bytes for
@@ -176,12 +285,45 @@ struct BwdLayout {
 
 // One work item of bwd_main: key block jt (128 rows) of kv head kvh.
 struct BwdItem {
-  int kvh;  // b * Hkv + kv head
-  int kv0;  // first key row
-  int i0;   // first query block (64 rows) that sees the key block
-  int nq;   // query blocks per query head
-  int T;    // steps: group * nq
-  int bh0;  // first query head of the group (b * Hq + g * group)
+  int kvh;    // b * Hkv + kv head
+  int kv0;    // first key row
+  int i0;     // first query block (64 rows) that sees the key block
+  int i_end;  // one past the last
+  int nq;     // query blocks per query head
+  int T;      // steps: group * nq (block mask: the visible ones)
+  int bh0;    // first query head of the group (b * Hq + g * group)
+  const uint16_t* plan;  // block mask: the item's walk
+};
+
+// The steps of an item in walk order, as (query head, 64-row query block):
+// every query block of every group head, or under a block mask those of
+// the item's plan (each visible 128-row block gives its 64-row halves that
+// lie in [i0, i_end)).  Every role walks the same sequence.
+template <bool BMASK>
+struct BwdWalk {
+  int t = 0, e = 0, half = 0;
+  __device__ __forceinline__ void next(const BwdItem& it, int* bh, int* qt) {
+    if constexpr (!BMASK) {
+      *bh = it.bh0 + t / it.nq;
+      *qt = it.i0 + t % it.nq;
+      ++t;
+    } else {
+      for (;;) {
+        const uint32_t ent = it.plan[e];
+        const int q = 2 * static_cast<int>(ent & 0xFFFu) + half;
+        const int hg = static_cast<int>(ent >> 12);
+        if (++half == 2) {
+          half = 0;
+          ++e;
+        }
+        if (q >= it.i0 && q < it.i_end) {
+          *bh = it.bh0 + hg;
+          *qt = q;
+          return;
+        }
+      }
+    }
+  }
 };
 
 // Item order: kv heads are taken in chunks of chunk_heads (as many as keep
@@ -190,7 +332,7 @@ struct BwdItem {
 // query blocks), each across the chunk's heads.  The blocks running at one
 // time then share few heads, and the items claimed last are short ones, so
 // the blocks finish close together.
-template <bool CAUSAL>
+template <bool CAUSAL, bool BMASK>
 __device__ __forceinline__ BwdItem bwd_item(const BwdParams& p, int item) {
   BwdItem it;
   const int per_chunk = p.chunk_heads * p.n_ktiles;
@@ -208,16 +350,24 @@ __device__ __forceinline__ BwdItem bwd_item(const BwdParams& p, int item) {
   const int i_end = (CAUSAL && p.window > 0)
                         ? min(p.n_qtiles, (min(p.N - 1, it.kv0 + 126 + p.window)) / 64 + 1)
                         : p.n_qtiles;
+  it.i_end = i_end;
   it.nq = i_end - it.i0;
   it.T = p.group * it.nq;
   it.bh0 = b * p.Hq + g * p.group;
+  it.plan = nullptr;
+  if constexpr (BMASK) {
+    const int idx = it.kvh * p.n_ktiles + jt;
+    it.T = __ldg(p.plan_steps + idx);
+    it.plan = p.plan_list + static_cast<long long>(idx) * p.plan_cap;
+  }
   return it;
 }
 
 constexpr int kBwdThreads = 448;
 
-template <int HD, bool BF16, bool CAUSAL, bool DROP>
+template <int HD, bool BF16, bool CAUSAL, bool DROP, bool BMASK>
 __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_constant__ BwdParams p) {
+  static_assert(!(DROP && BMASK), "dropout and block masks are not combined");
   using L = BwdLayout<HD>;
   using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
   extern __shared__ uint8_t smem_raw[];
@@ -248,6 +398,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
   volatile int* sched_item = reinterpret_cast<volatile int*>(sm + L::kOffSched);
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(sm + L::kOffTmemPtr);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::kOffAbort);
+  volatile int* conv_flag = reinterpret_cast<volatile int*>(sm + L::kOffConv);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -326,13 +477,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
         sched_item[slot] = item;
         mbar_arrive(&sched_full[slot]);
         if (item < 0) break;
-        const BwdItem it = bwd_item<CAUSAL>(p, item);
+        const BwdItem it = bwd_item<CAUSAL, BMASK>(p, item);
+        if (it.T == 0) continue;  // no step (block mask): no loads; the epilogue writes zeros
+        BwdWalk<BMASK> walk;
         auto load_step = [&](int t) -> bool {
           const int g = gt + t, s = g % L::kStages;
           if (g >= L::kStages &&
               !mbar_wait(&step_done[s], ((g / L::kStages) - 1) & 1, abort_flag, kKernBwd, 12, 0))
             return false;
-          const int bh = it.bh0 + t / it.nq, qt = it.i0 + t % it.nq;
+          int bh, qt;
+          walk.next(it, &bh, &qt);
           mbar_expect_tx(&q_full[s], 2 * L::kQTile + 512);
           for (int c = 0; c < L::kChunks; ++c) {
             tma_load_3d(sQ + s * L::kQTile + c * L::kQBox, &p.tm_q, &q_full[s], c * 64, qt * 64, bh);
@@ -404,12 +558,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
       umma_commit_w(&sdp_full[g & 1]);
     };
     int gt = 0;
+    int n_loaded = 0;  // items whose K and V were loaded (every item with a step)
     bool ok = true;
     for (int n = 0; ok; ++n) {
       const int item = sched_read(n, true, 13);
       if (item < 0) break;
-      const BwdItem it = bwd_item<CAUSAL>(p, item);
-      if (!wait_all(kv_full, n & 1, 0)) break;
+      const BwdItem it = bwd_item<CAUSAL, BMASK>(p, item);
+      if (it.T == 0) {
+        // nothing to compute (block mask); the epilogue writes zero dK, dV
+        umma_commit_w(acc_done);
+        continue;
+      }
+      if (!wait_all(kv_full, n_loaded & 1, 0)) break;
+      ++n_loaded;
       tc_fence_after();
       // S^T, dP^T of the item's first two steps.  dP^T of step g lands on
       // the columns that held dQ^T of step g-2 (the previous item's): wait
@@ -500,33 +661,40 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
     for (int n = 0;; ++n) {
       const int item = sched_read(n, true, 0);
       if (item < 0) break;
-      const BwdItem it = bwd_item<CAUSAL>(p, item);
+      const BwdItem it = bwd_item<CAUSAL, BMASK>(p, item);
       const int kv_row = it.kv0 + r;
       const bool row_valid = kv_row < p.N;
       bool ok = true;
+      BwdWalk<BMASK> walk;
       for (int t = 0; t < it.T; ++t) {
         const int g = gt + t, buf = g & 1, s = g % L::kStages;
-        const int q_step = (it.i0 + t % it.nq) * 64;   // first query of the step
-        const int bh_step = it.bh0 + t / it.nq;          // query head of the step
+        int bh_step, qt_step;                            // query head and block of the step
+        walk.next(it, &bh_step, &qt_step);
+        const int q_step = qt_step * 64;                 // first query of the step
         if (!__all_sync(0xffffffffu, mbar_wait(&sdp_full[buf], (g >> 1) & 1, abort_flag, kKernBwd, 0, 0))) {
           ok = false;
           break;
         }
         tc_fence_after();
-        // Two passes of 16 query columns keep the live registers low (no
-        // spills).  P^T of columns 16u..16u+15 is packed into the 8
+        // S^T and dP^T of this warp's 32 query columns are read from tensor
+        // memory at once (one wait), then worked in two passes of 16
+        // columns.  P^T of columns 16u..16u+15 is packed into the 8
         // tensor-memory columns at 32(u/2) + 8(u%2) of the S^T buffer, where
         // the dV product reads it; they held S^T of columns 32(u/2) + 8(u%2)
-        // .. +7, which this warp read in this pass or the one before it.
+        // .. +7, which this warp has read already.
+        uint32_t vs[32], vd[32];
+        tmem_ld16(tm_S(buf) + lane_off + 32 * half, vs);
+        tmem_ld16(tm_S(buf) + lane_off + 32 * half + 16, vs + 16);
+        tmem_ld16(tm_dP(buf) + lane_off + 32 * half, vd);
+        tmem_ld16(tm_dP(buf) + lane_off + 32 * half + 16, vd + 16);
+        tmem_ld_wait();
 #pragma unroll
         for (int qq = 2 * half; qq < 2 * half + 2; ++qq) {
           const int q_first = q_step + qq * 16;          // first query of these 16 columns
-          uint32_t v[16];
-          tmem_ld16(tm_S(buf) + lane_off + qq * 16, v);
+          const uint32_t* v = vs + 16 * (qq & 1);
           const float4* lse4 = reinterpret_cast<const float4*>(sLse + s * 64 + qq * 16);
           const float4* d4 = reinterpret_cast<const float4*>(sD + s * 64 + qq * 16);
           float pr[16];
-          tmem_ld_wait();
 #pragma unroll
           for (int c4 = 0; c4 < 4; ++c4) {
             const float4 l4 = lse4[c4];
@@ -585,28 +753,32 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
 #pragma unroll
               for (int u = 0; u < 4; ++u)
                 fd[4 * g + u] = ((cols[g] >> (8 * u)) & 0xFFu) >= p.drop_t ? p.drop_scale : 0.f;
+            // Z P for the dV product: the factor 1/(1-p) of the kept
+            // probabilities is applied to dV once, in its epilogue, rather
+            // than before P is rounded to 16 bits
 #pragma unroll
             for (int i = 0; i < 8; ++i)
-              pk[i] = pack2<BF16>(pr[2 * i] * fd[2 * i], pr[2 * i + 1] * fd[2 * i + 1]);  // P'
+              pk[i] = pack2<BF16>(fd[2 * i] != 0.f ? pr[2 * i] : 0.f, fd[2 * i + 1] != 0.f ? pr[2 * i + 1] : 0.f);
           } else {
 #pragma unroll
             for (int i = 0; i < 8; ++i) pk[i] = pack2<BF16>(pr[2 * i], pr[2 * i + 1]);
           }
           tmem_st8(tm_S(buf) + lane_off + (qq >> 1) * 32 + (qq & 1) * 8, pk);
-          tmem_ld16(tm_dP(buf) + lane_off + qq * 16, v);
-          tmem_ld_wait();
+          float dp[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c) dp[c] = __uint_as_float(vd[16 * (qq & 1) + c]);
           if constexpr (DROP) {
             // dP of P is dP' times the dropout factor
 #pragma unroll
-            for (int c = 0; c < 16; ++c) v[c] = __float_as_uint(__uint_as_float(v[c]) * fd[c]);
+            for (int c = 0; c < 16; ++c) dp[c] *= fd[c];
           }
 #pragma unroll
           for (int c4 = 0; c4 < 4; ++c4) {
             const float4 dd = d4[c4];
-            pr[4 * c4 + 0] *= __uint_as_float(v[4 * c4 + 0]) - dd.x;
-            pr[4 * c4 + 1] *= __uint_as_float(v[4 * c4 + 1]) - dd.y;
-            pr[4 * c4 + 2] *= __uint_as_float(v[4 * c4 + 2]) - dd.z;
-            pr[4 * c4 + 3] *= __uint_as_float(v[4 * c4 + 3]) - dd.w;
+            pr[4 * c4 + 0] *= dp[4 * c4 + 0] - dd.x;
+            pr[4 * c4 + 1] *= dp[4 * c4 + 1] - dd.y;
+            pr[4 * c4 + 2] *= dp[4 * c4 + 2] - dd.z;
+            pr[4 * c4 + 3] *= dp[4 * c4 + 3] - dd.w;
           }
 #pragma unroll
           for (int i = 0; i < 8; ++i) pk[i] = pack2<BF16>(pr[2 * i], pr[2 * i + 1]);
@@ -643,8 +815,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
     for (int n = 0;; ++n) {
       const int item = sched_read(n, true, 8);
       if (item < 0) break;
-      const BwdItem it = bwd_item<CAUSAL>(p, item);
+      const BwdItem it = bwd_item<CAUSAL, BMASK>(p, item);
       bool ok = true;
+      BwdWalk<BMASK> walk;
       for (int t = 0; drains && t < it.T; ++t) {
         const int g = gt + t, buf = g & 1;
         if (!__all_sync(0xffffffffu, mbar_wait(&dq_full[buf], (g >> 1) & 1, abort_flag, kKernBwd, 8, 0))) {
@@ -658,12 +831,45 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
         tmem_ld_wait();
         tc_fence_before();
         mbar_arrive(&dq_drained[buf]);
-        const int bh = it.bh0 + t / it.nq, qt = it.i0 + t % it.nq;
-        float* dst = p.dqacc + (static_cast<size_t>(bh) * p.Np + qt * 64) * HD + dw * 32 + lane;
+        int bh, qt;
+        walk.next(it, &bh, &qt);
+        float* acc_blk = p.dqacc + (static_cast<size_t>(bh) * p.Np + qt * 64) * HD;
+        float* dst = acc_blk + dw * 32 + lane;
 #pragma unroll
         for (int q = 0; q < 32; ++q) atomicAdd(dst + q * HD, __uint_as_float(v0[q]));
 #pragma unroll
         for (int q = 0; q < 32; ++q) atomicAdd(dst + (32 + q) * HD, __uint_as_float(v1[q]));
+        // Count this addition down from the number the query block receives
+        // (set by bwd_pre); the block bringing the last one converts it.
+        // Every drain thread's additions are ordered before the count (fence,
+        // barrier, fence by the counting thread), and the converting threads'
+        // reads after it (fence after the barrier).
+        __threadfence();
+        named_barrier_sync(1, kDrainThreads);
+        if (dw == 0 && lane == 0) {
+          __threadfence();
+          const unsigned old = atomicSub(p.dq_count + static_cast<size_t>(bh) * (p.Np / 64) + qt, 1u);
+          *conv_flag = old == 1u ? 1 : 0;
+        }
+        named_barrier_sync(1, kDrainThreads);
+        if (*conv_flag) {
+          __threadfence();
+          // dQ = scale * accumulator -> I/O dtype, rows of the block below N
+          constexpr int kVec = HD / 4;  // float4 per row
+          T* out = reinterpret_cast<T*>(p.dq) + (static_cast<size_t>(bh) * p.N + qt * 64) * HD;
+          const int rows_here = min(64, p.N - qt * 64);
+          for (int i = dw * 32 + lane; i < rows_here * kVec; i += kDrainThreads) {
+            const int row = i / kVec, c4 = i % kVec;
+            const float4 a = __ldcg(reinterpret_cast<const float4*>(acc_blk + row * HD) + c4);
+            uint2 w;
+            w.x = pack2<BF16>(a.x * p.scale, a.y * p.scale);
+            w.y = pack2<BF16>(a.z * p.scale, a.w * p.scale);
+            *reinterpret_cast<uint2*>(out + row * HD + c4 * 4) = w;
+          }
+        }
+        // the flag is read by every drain thread before the next step's
+        // counting thread may write it: the barrier of the next step comes
+        // after these reads
       }
       if (!ok) break;
       gt += it.T;
@@ -673,16 +879,24 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
       const int r = dw * 32 + lane;
       const int kv_row = it.kv0 + r;
       const size_t row_off = (static_cast<size_t>(it.kvh) * p.N + kv_row) * HD;
+      // an item without steps (block mask: no query sees the key block) has
+      // dK = dV = 0 and never touched the accumulators
+      const bool zero = it.T == 0;
 #pragma unroll
       for (int which = 0; which < 2; ++which) {
         const uint32_t src = (which ? tm_dK : tm_dV) + lane_off;
-        const float mul = which ? p.scale : 1.0f;
+        const float mul = which ? p.scale : (DROP ? p.drop_scale : 1.0f);
         T* dst = reinterpret_cast<T*>(which ? p.dk : p.dv) + row_off;
 #pragma unroll
         for (int c = 0; c < HD; c += 32) {
           uint32_t v[32];
-          tmem_ld32(src + c, v);
-          tmem_ld_wait();
+          if (!zero) {
+            tmem_ld32(src + c, v);
+            tmem_ld_wait();
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = 0u;
+          }
           if (kv_row < p.N) {
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
@@ -706,32 +920,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
   if (warp == 13) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
-  }
-}
-
-// ---------------------------------------------------------------------------
-// bwd_post: dQ = scale * accumulator -> I/O dtype (8 elements per thread)
-
-template <int HD, bool BF16>
-__global__ void __launch_bounds__(256) fa_bwd_post_kernel(const float* __restrict__ dqacc,
-                                                          void* __restrict__ dq_, int N, int Np,
-                                                          int64_t total_vec, float scale) {
-  using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
-  constexpr int kVecPerRow = HD / 8;
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total_vec;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t row = i / kVecPerRow;  // row of the [B*Hq][N] output
-    const int cv = static_cast<int>(i % kVecPerRow);
-    const int64_t bh = row / N;
-    const int64_t n = row % N;
-    const float4* src = reinterpret_cast<const float4*>(dqacc + (bh * Np + n) * HD + cv * 8);
-    const float4 a = src[0], c = src[1];
-    uint4 w;
-    w.x = pack2<BF16>(a.x * scale, a.y * scale);
-    w.y = pack2<BF16>(a.z * scale, a.w * scale);
-    w.z = pack2<BF16>(c.x * scale, c.y * scale);
-    w.w = pack2<BF16>(c.z * scale, c.w * scale);
-    reinterpret_cast<uint4*>(reinterpret_cast<T*>(dq_) + row * HD)[cv] = w;
   }
 }
 

@@ -15,7 +15,7 @@
 // Two query blocks per thread block, each with its own softmax warpgroup, so
 // that the tensor cores work on one block while the softmax warps work on the
 // other (the B200 form of the "two sets of registers" alternation the
-// FlashAttention glossary names for Hopper).  Warp roles (320 threads):
+// FlashAttention glossary names for Hopper).  Warp roles (384 threads):
 //   warps 0-3 / 4-7  softmax of query block 0 / 1: thread r owns row r of its
 //              block and tensor-memory lane r.  Reads S_j, masks, scales,
 //              updates (m, l), writes P_j (16-bit) over S_j, rescales O when
@@ -27,6 +27,8 @@
 //              other block's products.
 //   warp 9     TMA producer: Q0, Q1 once, then K_0, V_0, K_1, V_1, ... through
 //              a ring of kSlots tiles.
+//   warps 10-11 idle (they complete the third warpgroup, which gives its
+//              registers to the softmax warpgroups).
 // Tensor memory (512 columns x 128 lanes x 32 bit): S0 [0,128), S1 [128,256),
 // O0 [256, 256+d), O1 [384, 384+d); P_t packs into the first 64 columns of S_t.
 //
@@ -36,6 +38,8 @@
 // l always share one m_ref, so O / l is exact (a softmax's reference point is
 // arbitrary).
 #pragma once
+
+#include <type_traits>
 
 #include "sm100.cuh"
 
@@ -55,6 +59,44 @@ struct FwdParams {
   uint32_t seed_lo, seed_hi, drop_t;
   float drop_scale;
   float scale_log2;  // scale * log2(e)
+  // block mask (kernels instantiated with BMASK): key block j (128 keys) is
+  // hidden from query block i (128 rows) of query head h when
+  // bmask[h * bm_hstride + i * n_ktiles + j] == 0 (bm_hstride 0: one mask
+  // for every head)
+  const uint8_t* bmask;
+  long long bm_hstride;
+};
+
+// The key blocks a pair of query blocks streams under a block mask: those
+// visible to either block (union), in order.  Block t of the pair sees key
+// block j when j <= jmax[t] (causal) and its mask byte is set.
+struct FwdMaskRows {
+  // mask rows of the pair's query blocks (nullptr: no such block); the
+  // fields are named, not an array, so that a runtime t selects by value
+  const uint8_t* row0;
+  const uint8_t* row1;
+  int jmax0, jmax1;
+
+  __device__ __forceinline__ bool vis(int t, int j) const {
+    const uint8_t* r = t ? row1 : row0;
+    return r != nullptr && j <= (t ? jmax1 : jmax0) && __ldg(r + j) != 0;
+  }
+  __device__ __forceinline__ int jend() const { return max(jmax0, jmax1) + 1; }
+  // first key block >= j that either block sees; jend() if none
+  __device__ __forceinline__ int next(int j) const {
+    const int e = jend();
+    while (j < e && !vis(0, j) && !vis(1, j)) ++j;
+    return j;
+  }
+  // number of key blocks in the union, counted by the whole warp
+  __device__ __forceinline__ int count_warp(int lane) const {
+    int n = 0;
+    for (int j0 = 0; j0 < jend(); j0 += 32) {
+      const int j = j0 + lane;
+      n += __popc(__ballot_sync(0xffffffffu, j < jend() && (vis(0, j) || vis(1, j))));
+    }
+    return n;
+  }
 };
 
 template <int HD>
@@ -66,8 +108,9 @@ struct FwdLayout {
   static constexpr int kOffQ = 0;                    // two query tiles
   static constexpr int kOffRing = 2 * kTileBytes;
   static constexpr int kOffBar = kOffRing + kSlots * kTileBytes;
-  // barriers: q_full, slot_full[kSlots], slot_empty[kSlots], s_full[2], p_full[2], pv_done[2], done
-  static constexpr int kNumBars = 1 + 2 * kSlots + 6 + 1;
+  // barriers: q_full, slot_full[kSlots], slot_empty[kSlots], s_full[2],
+  // p_half[2][2] (keys 0-63 / 64-127 of P_t ready), pv_done[2], done
+  static constexpr int kNumBars = 1 + 2 * kSlots + 8 + 1;
   static constexpr int kOffTmemPtr = kOffBar + kNumBars * 8;
   static constexpr int kOffAbort = kOffTmemPtr + 4;
   static constexpr int kSmemBytes = kOffAbort + 4;
@@ -75,11 +118,27 @@ struct FwdLayout {
   static_assert(kDynSmem <= 232448, "shared memory budget");
 };
 
-constexpr int kFwdThreads = 320;
+// Three warpgroups: two softmax warpgroups and one holding the MMA issuer,
+// the TMA producer and two idle warps.  Launched at 168 registers a thread
+// (384 x 168 of the SM's 65 536), the registers are then moved to the
+// softmax warpgroups: 2 x 128 x 216 + 128 x 72 = 384 x 168.  Per SM
+// sub-partition (16 384 registers, one warp of each warpgroup) that is
+// 32 x (216 + 216 + 72) = 16 128.
+constexpr int kFwdThreads = 384;
+constexpr uint32_t kFwdSoftmaxRegs = 216;
+constexpr uint32_t kFwdOtherRegs = 72;
+static_assert(2 * 128 * kFwdSoftmaxRegs + 128 * kFwdOtherRegs <= kFwdThreads * 168, "register split");
 constexpr uint32_t kKernFwd = 1;
+// Pairs of exponentials of every 8 (per 16 keys) computed on the FMA pipe in
+// unmasked score tiles; the rest go to the MUFU unit.
+#ifndef FA_FWD_POLY_PAIRS
+#define FA_FWD_POLY_PAIRS 0
+#endif
+constexpr int kPolyPairs = FA_FWD_POLY_PAIRS;
 
-template <int HD, bool BF16, bool CAUSAL, bool DROP>
+template <int HD, bool BF16, bool CAUSAL, bool DROP, bool BMASK>
 __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_constant__ FwdParams p) {
+  static_assert(!(DROP && BMASK), "dropout and block masks are not combined");
   using L = FwdLayout<HD>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -91,8 +150,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
   uint64_t* slot_full = bars + 1;
   uint64_t* slot_empty = slot_full + L::kSlots;
   uint64_t* s_full = slot_empty + L::kSlots;
-  uint64_t* p_full = s_full + 2;
-  uint64_t* pv_done = p_full + 2;
+  uint64_t* p_half = s_full + 2;  // [t][half]
+  uint64_t* pv_done = p_half + 4;
   uint64_t* done_bar = pv_done + 2;
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(sm + L::kOffTmemPtr);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::kOffAbort);
@@ -114,8 +173,20 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
   // With a sliding window the key/value stream starts at the first block the
   // pair's first row can see; counts below are of blocks from that one on.
   const int j_start = (CAUSAL && p.window > 0) ? max(0, 2 * pair * 128 - p.window + 1) / 128 : 0;
-  const int n_kv0 = (CAUSAL ? min(2 * pair + 1, p.n_ktiles) : p.n_ktiles) - j_start;
-  const int n_kv1 = (CAUSAL ? min(2 * pair + 2, p.n_ktiles) : p.n_ktiles) - j_start;
+  int n_kv0 = (CAUSAL ? min(2 * pair + 1, p.n_ktiles) : p.n_ktiles) - j_start;
+  int n_kv1 = (CAUSAL ? min(2 * pair + 2, p.n_ktiles) : p.n_ktiles) - j_start;
+  // Under a block mask both blocks walk the union of their visible key
+  // blocks (n_kv0 = n_kv1 = its size, counted by each role's warp); a key
+  // block hidden from one of them is a fully masked tile for it.
+  FwdMaskRows mrows{};
+  if constexpr (BMASK) {
+    const uint8_t* mh = p.bmask + static_cast<long long>(h) * p.bm_hstride;
+    const int qb0 = 2 * pair, qb1 = 2 * pair + 1;
+    mrows.row0 = mh + static_cast<long long>(qb0) * p.n_ktiles;
+    mrows.row1 = qb1 < p.n_ktiles ? mh + static_cast<long long>(qb1) * p.n_ktiles : nullptr;
+    mrows.jmax0 = CAUSAL ? min(qb0, p.n_ktiles - 1) : p.n_ktiles - 1;
+    mrows.jmax1 = CAUSAL ? min(qb1, p.n_ktiles - 1) : p.n_ktiles - 1;
+  }
 
   if (tid == 0) {
     mbar_init(q_full, 1);
@@ -125,7 +196,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], 128);
+      mbar_init(&p_half[2 * i], 128);
+      mbar_init(&p_half[2 * i + 1], 128);
       mbar_init(&pv_done[i], 1);
     }
     mbar_init(done_bar, 1);
@@ -140,9 +212,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_ptr;
-
-  if (warp == 9) {
+  // Each warpgroup changes its register count at one site, all four of its
+  // warps together (the PTX rule for setmaxnreg); the roles branch below it.
+  if (warp >= 8) setmaxnreg_dec<kFwdOtherRegs>();
+  if (warp >= 10) {
+    // idle warps of the third warpgroup
+  } else if (warp == 9) {
     // ------------------------------------------------------------ producer
+    if constexpr (BMASK) n_kv1 = mrows.count_warp(lane);
     if (lane == 0) {
       prefetch_tensormap(&p.tm_q);
       prefetch_tensormap(&p.tm_k);
@@ -153,7 +230,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
           tma_load_3d(sQ + t * L::kTileBytes + c * L::kBoxBytes, &p.tm_q, q_full, c * 64,
                       (2 * pair + t) * 128, bh);
       int n = 0;
-      auto load = [&](const CUtensorMap* map, int tile) -> bool {
+      auto load = [&](const CUtensorMap* map, int kblock) -> bool {
         const int s = n % L::kSlots;
         if (n >= L::kSlots &&
             !mbar_wait(&slot_empty[s], ((n / L::kSlots) - 1) & 1, abort_flag, kKernFwd, 9, 0))
@@ -161,14 +238,16 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
         mbar_expect_tx(&slot_full[s], L::kTileBytes);
         uint8_t* dst = sRing + s * L::kTileBytes;
         for (int c = 0; c < L::kChunks; ++c)
-          tma_load_3d(dst + c * L::kBoxBytes, map, &slot_full[s], c * 64, (j_start + tile) * 128, kvh);
+          tma_load_3d(dst + c * L::kBoxBytes, map, &slot_full[s], c * 64, kblock * 128, kvh);
         ++n;
         return true;
       };
       bool ok = true;
+      int kb = BMASK ? mrows.next(0) : j_start;  // key block of stream position j
       for (int j = 0; ok && j < n_kv1; ++j) {
-        ok = load(&p.tm_k, j);
-        if (ok) ok = load(&p.tm_v, j);
+        ok = load(&p.tm_k, kb);
+        if (ok) ok = load(&p.tm_v, kb);
+        kb = BMASK ? mrows.next(kb + 1) : kb + 1;
       }
     }
   } else if (warp == 8) {
@@ -211,19 +290,26 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
       }
       umma_commit_w(&s_full[t]);
     };
+    // O_t += P_t,j V_j in two halves of 64 keys: the softmax warps hand over
+    // P of keys 0-63 before they compute keys 64-127.
     auto issue_pv = [&](int t, int j, int vslot) -> bool {
-      if (!wait_all(&p_full[t], j & 1, 3)) return false;
-      tc_fence_after();
       const uint32_t vo = vslot * L::kTileBytes;
 #pragma unroll
-      for (int k = 0; k < 8; ++k)
-        umma_ts_w(tmem + 256 + t * 128, tmem + t * 128 + k * 8, sdesc_add(dR_mn, vo + k * 2048),
-                  kIdPV, (j > 0 || k > 0) ? 1u : 0u);
+      for (int half = 0; half < 2; ++half) {
+        if (!wait_all(&p_half[2 * t + half], j & 1, 3)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int k = 4 * half; k < 4 * half + 4; ++k)
+          umma_ts_w(tmem + 256 + t * 128, tmem + t * 128 + k * 8, sdesc_add(dR_mn, vo + k * 2048),
+                    kIdPV, (j > 0 || k > 0) ? 1u : 0u);
+      }
       umma_commit_w(&pv_done[t]);
       return true;
     };
+    if constexpr (BMASK) n_kv0 = n_kv1 = mrows.count_warp(lane);
     int kslot = 0, vslot = 0;
-    if (ok) ok = take(kslot);
+    if (ok && n_kv1 > 0) ok = take(kslot);
+    else ok = false;  // nothing to compute (only under a block mask)
     if (ok) {
       if (n_kv0 > 0) issue_s(0, kslot);
       issue_s(1, kslot);
@@ -248,6 +334,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
     umma_commit_w(done_bar);
     mbar_wait_drain(done_bar, 0, kKernFwd, 8, 4);
   } else {
+    setmaxnreg_inc<kFwdSoftmaxRegs>();
     // ------------------------------------------------------------ softmax
     const int t = warp >> 2;                 // query block of this warpgroup
     const int r = tid & 127;                 // row within the block == TMEM lane
@@ -256,7 +343,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
     const uint32_t tm_O = tmem + 256 + t * 128 + lane_off;
     const int qtile = 2 * pair + t;
     const int q_row = qtile * 128 + r;
+    if constexpr (BMASK) n_kv0 = n_kv1 = mrows.count_warp(lane);
     const int n_kv = t ? n_kv1 : n_kv0;
+    int kb_cur = BMASK ? mrows.next(0) : j_start;  // key block of the current stream position
     const float c_log2 = p.scale_log2;
     const uint64_t c2 = f2pack(c_log2, c_log2);
     float m_ref = -INFINITY;  // in log2 units of the scaled scores
@@ -264,13 +353,20 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
     bool ok = true;
     // Waits are made warp-uniform: tcgen05.ld/st are warp-collective, so a
     // warp either goes on together or leaves together (on abort).
-    for (int j = 0; j < n_kv; ++j) {
-      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[t], j & 1, abort_flag, kKernFwd, t, 0))) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      uint32_t s[128];
+    //
+    // Per key tile: S is read from tensor memory, masked where a block edge
+    // needs it, and the row max taken (three-input max, eight chains).  From
+    // the second tile on, the exponentials of keys 0-63 are computed against
+    // the current reference max while the row max is still being taken (the
+    // two are independent), so that the max costs no time of its own; the
+    // warp then checks whether any of its rows grew by more than 8 (log2).
+    // If none did (the common case) those exponentials stand: P of keys 0-63
+    // goes to tensor memory and is handed to the MMA warp, then keys 64-127.
+    // Otherwise the tile is redone from tensor memory against the moved
+    // reference, after O and l are rescaled.  In unmasked tiles kPolyPairs of
+    // every 8 pairs of exponentials run on the FMA pipe (exp2_poly2), the
+    // rest on the MUFU unit.
+    auto load_s = [&](int kblock, uint32_t* s) {
       tmem_ld32(tm_S + 0, s);
       tmem_ld32(tm_S + 32, s + 32);
       tmem_ld32(tm_S + 64, s + 64);
@@ -278,30 +374,135 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
       tmem_ld_wait();
       // mask: keys past the end of the sequence, and keys after the query
       // inside the diagonal block of a causal problem
-      const int kv0 = (j_start + j) * 128;
-      const bool diag = CAUSAL && (j_start + j == qtile);
+      const int kv0 = kblock * 128;
+      const bool diag = CAUSAL && (kblock == qtile);
       // sliding window: keys below q_row - W + 1 are hidden; some row of the
       // block meets that edge in this key block
       const bool low = CAUSAL && p.window > 0 && kv0 + p.window <= qtile * 128 + 127;
-      if (diag || low || kv0 + 128 > p.N) {
-        const int lim = min(diag ? r : 127, p.N - 1 - kv0);  // last visible column
+      // block mask: a key block of the pair's stream that this query block
+      // does not see is hidden whole
+      const bool hid = BMASK && !mrows.vis(t, kblock);
+      if (diag || low || hid || kv0 + 128 > p.N) {
+        const int lim = hid ? -1 : min(diag ? r : 127, p.N - 1 - kv0);  // last visible column
         const int first = low ? q_row - p.window + 1 - kv0 : 0;  // first visible column
 #pragma unroll
         for (int c = 0; c < 128; ++c)
           if (c > lim || c < first) s[c] = __float_as_uint(-INFINITY);
+        return true;   // masked tile
       }
-      // row max, eight independent chains
-      float mx[8];
+      return false;
+    };
+    // P of the 32 keys 32*q4 .. +31 against the reference -m (nm2), packed to
+    // 16 bits in pk[16]; the unrounded values are summed into acc.
+    auto p_chunk = [&](auto poly_tag, const uint32_t* s, int q4, uint64_t nm2, int kv0, uint32_t* pk,
+                       uint64_t* acc) {
+      constexpr bool kPoly = decltype(poly_tag)::value;
+      [[maybe_unused]] uint32_t kw[4] = {0, 0, 0, 0};  // dropout bytes: keys 4g..4g+3 of 16 in kw[g]
 #pragma unroll
-      for (int i = 0; i < 8; ++i) mx[i] = __uint_as_float(s[i]);
+      for (int i = 0; i < 16; ++i) {
+        const int c = q4 * 32 + 2 * i;
+        const uint64_t x = fma2(f2pack(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), c2, nm2);
+        uint64_t pp;
+        if (!DROP && kPoly && (i & 7) < kPolyPairs)
+          pp = exp2_poly2(x);
+        else
+          pp = f2pack(ex2_approx(f2lo(x)), ex2_approx(f2hi(x)));
+        acc[i & 3] = add2(acc[i & 3], pp);  // l sums the undropped P
+        if constexpr (DROP) {
+          if ((i & 7) == 0) {
+            // The 4 lanes of a quad hold 4 consecutive rows (one Philox
+            // counter row).  Lane g of the quad draws the 4x4 block of keys
+            // 4g..4g+3 of the next 16; four rotations of a shuffle give
+            // each lane its own row's word of all four blocks.
+            const int ql = lane & 3;
+            const uint4 rnd = philox4x32_10(
+                make_uint4(static_cast<uint32_t>((kv0 + c + 4 * ql) >> 2), static_cast<uint32_t>(q_row >> 2),
+                           static_cast<uint32_t>(bh), 0u),
+                p.seed_lo, p.seed_hi);
 #pragma unroll
-      for (int c = 8; c < 128; ++c) mx[c & 7] = fmaxf(mx[c & 7], __uint_as_float(s[c]));
+            for (int rr = 0; rr < 4; ++rr) {
+              const uint32_t got = __shfl_sync(0xffffffffu, uint4_word(rnd, (ql - rr) & 3),
+                                               (lane & ~3) | ((ql + rr) & 3));
+              const int g = (ql + rr) & 3;
+              kw[0] = g == 0 ? got : kw[0];
+              kw[1] = g == 1 ? got : kw[1];
+              kw[2] = g == 2 ? got : kw[2];
+              kw[3] = g == 3 ? got : kw[3];
+            }
+          }
+          const uint32_t keep_word = kw[(i >> 1) & 3];
+          const uint32_t b0 = (keep_word >> (16 * (i & 1))) & 0xFFu;
+          const uint32_t b1 = (keep_word >> (16 * (i & 1) + 8)) & 0xFFu;
+          pk[i] = pack2<BF16>(b0 >= p.drop_t ? f2lo(pp) : 0.f, b1 >= p.drop_t ? f2hi(pp) : 0.f);
+        } else {
+          pk[i] = pack2<BF16>(f2lo(pp), f2hi(pp));
+        }
+      }
+    };
+    auto hand_over = [&](int half) {
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&p_half[2 * t + half]);
+    };
+    auto sum_acc = [&](const uint64_t* acc) {
+      const uint64_t a = add2(add2(acc[0], acc[1]), add2(acc[2], acc[3]));
+      return f2lo(a) + f2hi(a);
+    };
+    for (int j = 0; j < n_kv; ++j) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[t], j & 1, abort_flag, kKernFwd, t, 0))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const int kb = kb_cur;
+      if constexpr (BMASK) kb_cur = mrows.next(kb + 1);
+      else kb_cur = kb + 1;
+      const int kv0 = kb * 128;
+      bool done = false;
+      float m_new;
+      {
+        uint32_t s[128];
+        const bool masked = load_s(kb, s);
+        // row max, eight independent chains of three-input maxima
+        float mx[8];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) mx[i] = fmaxf(mx[i], mx[i + 4]);
-      const float m_new = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * c_log2;
-      if (j == 0) {
-        m_ref = m_new;
-      } else if (__any_sync(0xffffffffu, m_new > m_ref + 8.0f)) {
+        for (int i = 0; i < 8; ++i) mx[i] = max3f(__uint_as_float(s[i]), __uint_as_float(s[8 + i]),
+                                                  __uint_as_float(s[16 + i]));
+#pragma unroll
+        for (int c = 24; c < 128; c += 16)
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            mx[i] = max3f(mx[i], __uint_as_float(s[c + i]), __uint_as_float(s[c + 8 + i]));
+        m_new = max3f(max3f(mx[0], mx[1], mx[2]), max3f(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) * c_log2;
+        if (!DROP && j > 0) {
+          // speculative: keys 0-63 against the current reference
+          const float m_use = m_ref == -INFINITY ? 0.f : m_ref;
+          const uint64_t nm2 = f2pack(-m_use, -m_use);
+          auto spec = [&](auto poly_tag) -> bool {
+            uint32_t pk0[16], pk1[16];
+            uint64_t acc[4] = {0, 0, 0, 0};
+            p_chunk(poly_tag, s, 0, nm2, kv0, pk0, acc);
+            p_chunk(poly_tag, s, 1, nm2, kv0, pk1, acc);
+            if (__any_sync(0xffffffffu, m_new > m_ref + 8.0f)) return false;
+            tmem_st16(tm_S + 0, pk0);
+            tmem_st16(tm_S + 16, pk1);
+            hand_over(0);
+            p_chunk(poly_tag, s, 2, nm2, kv0, pk0, acc);
+            tmem_st16(tm_S + 32, pk0);
+            p_chunk(poly_tag, s, 3, nm2, kv0, pk1, acc);
+            tmem_st16(tm_S + 48, pk1);
+            l_sum += sum_acc(acc);
+            hand_over(1);
+            return true;
+          };
+          // exponentials on the FMA pipe need finite arguments: masked
+          // tiles stay on the MUFU unit
+          done = masked ? spec(std::false_type{}) : spec(std::true_type{});
+        }
+      }
+      if (done) continue;
+      // first tile of the rows, or a reference max that must move
+      if (j > 0) {
         // Move the reference max of every row of this warp (tcgen05.ld/st are
         // warp-wide), rescaling O and l, once O_t += P_t,j-1 V_j-1 is done.
         if (!__all_sync(0xffffffffu, mbar_wait(&pv_done[t], (j - 1) & 1, abort_flag, kKernFwd, t, 1))) {
@@ -328,77 +529,56 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
           }
           tmem_st16(tm_O + c, o);
         }
+      } else {
+        m_ref = m_new;
       }
-      // P = 2^(s c - m_ref), packed to 16 bits over the first 64 columns of S.
-      // A row that has seen no visible key yet (only under a sliding window)
-      // keeps m_ref = -inf; its scores are all -inf and give P = 0 against 0.
-      const float m_use = m_ref == -INFINITY ? 0.f : m_ref;
-      const uint64_t nm2 = f2pack(-m_use, -m_use);
-      uint64_t acc[4] = {0, 0, 0, 0};
+      {
+        // P = 2^(s c - m_ref), packed to 16 bits over the first 64 columns of
+        // S.  A row that has seen no visible key yet (only under a sliding
+        // window) keeps m_ref = -inf; its scores are all -inf and give P = 0
+        // against 0.
+        uint32_t s[128];
+        load_s(kb, s);
+        const float m_use = m_ref == -INFINITY ? 0.f : m_ref;
+        const uint64_t nm2 = f2pack(-m_use, -m_use);
+        uint64_t acc[4] = {0, 0, 0, 0};
 #pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) {
-        uint32_t pk[16];
-        uint32_t kw[4] = {0, 0, 0, 0};  // dropout bytes of this row: keys 4g..4g+3 of 16 in kw[g]
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int c = q4 * 32 + 2 * i;
-          const uint64_t x = fma2(f2pack(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), c2, nm2);
-          const uint64_t pp = f2pack(ex2_approx(f2lo(x)), ex2_approx(f2hi(x)));
-          acc[i & 3] = add2(acc[i & 3], pp);  // l sums the undropped P
-          if constexpr (DROP) {
-            if ((i & 7) == 0) {
-              // The 4 lanes of a quad hold 4 consecutive rows (one Philox
-              // counter row).  Lane g of the quad draws the 4x4 block of keys
-              // 4g..4g+3 of the next 16; four rotations of a shuffle give
-              // each lane its own row's word of all four blocks.
-              const int ql = lane & 3;
-              const uint4 rnd = philox4x32_10(
-                  make_uint4(static_cast<uint32_t>((kv0 + c + 4 * ql) >> 2), static_cast<uint32_t>(q_row >> 2),
-                             static_cast<uint32_t>(bh), 0u),
-                  p.seed_lo, p.seed_hi);
-#pragma unroll
-              for (int rr = 0; rr < 4; ++rr) {
-                const uint32_t got = __shfl_sync(0xffffffffu, uint4_word(rnd, (ql - rr) & 3),
-                                                 (lane & ~3) | ((ql + rr) & 3));
-                const int g = (ql + rr) & 3;
-                kw[0] = g == 0 ? got : kw[0];
-                kw[1] = g == 1 ? got : kw[1];
-                kw[2] = g == 2 ? got : kw[2];
-                kw[3] = g == 3 ? got : kw[3];
-              }
-            }
-            const uint32_t keep_word = kw[(i >> 1) & 3];
-            const uint32_t b0 = (keep_word >> (16 * (i & 1))) & 0xFFu;
-            const uint32_t b1 = (keep_word >> (16 * (i & 1) + 8)) & 0xFFu;
-            pk[i] = pack2<BF16>(b0 >= p.drop_t ? f2lo(pp) * p.drop_scale : 0.f,
-                                b1 >= p.drop_t ? f2hi(pp) * p.drop_scale : 0.f);
-          } else {
-            pk[i] = pack2<BF16>(f2lo(pp), f2hi(pp));
-          }
+        for (int q4 = 0; q4 < 4; ++q4) {
+          uint32_t pk[16];
+          p_chunk(std::false_type{}, s, q4, nm2, kv0, pk, acc);
+          tmem_st16(tm_S + q4 * 16, pk);
+          if (q4 == 1) hand_over(0);
         }
-        tmem_st16(tm_S + q4 * 16, pk);
+        l_sum += sum_acc(acc);
+        hand_over(1);
       }
-      const uint64_t a01 = add2(acc[0], acc[1]), a23 = add2(acc[2], acc[3]);
-      const uint64_t a = add2(a01, a23);
-      l_sum += f2lo(a) + f2hi(a);
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(&p_full[t]);
     }
     // epilogue: O / l -> 16-bit, staged in this block's (now idle) Q tile, TMA store
     uint8_t* sQt = sQ + t * L::kTileBytes;
+    // no key block at all to stream (only under a block mask): O = 0
+    const bool empty_stream = ok && n_kv == 0;
     bool ep_ok = ok && n_kv > 0;
     if (ep_ok) ep_ok = mbar_wait(&pv_done[t], (n_kv - 1) & 1, abort_flag, kKernFwd, t, 2);
     ep_ok = __all_sync(0xffffffffu, ep_ok);
-    if (ep_ok) {
-      tc_fence_after();
-      const float inv_l = 1.0f / l_sum;
+    if (ep_ok || empty_stream) {
+      if (ep_ok) tc_fence_after();
+      // with dropout, the kept probabilities' factor 1/(1-p) is applied here,
+      // once, rather than before P is rounded to 16 bits.  A row that saw
+      // no key (possible only under a block mask) has l = 0: O = 0 and
+      // lse = -inf, the log of an empty sum.
+      const bool seen = l_sum > 0.f;
+      const float inv_l = seen ? (DROP ? p.drop_scale : 1.0f) / l_sum : 0.f;
       const uint64_t inv2 = f2pack(inv_l, inv_l);
 #pragma unroll
       for (int c = 0; c < HD; c += 32) {
         uint32_t o[32];
-        tmem_ld32(tm_O + c, o);
-        tmem_ld_wait();
+        if (ep_ok) {
+          tmem_ld32(tm_O + c, o);
+          tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = 0u;
+        }
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
@@ -415,7 +595,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
         }
       }
       if (q_row < p.N)
-        p.lse[static_cast<size_t>(bh) * p.N + q_row] = (m_ref + __log2f(l_sum)) * 0.69314718055994531f;
+        p.lse[static_cast<size_t>(bh) * p.N + q_row] =
+            seen ? (m_ref + __log2f(l_sum)) * 0.69314718055994531f : -INFINITY;
       fence_proxy_async_smem();
     }
     // every thread of the warpgroup reaches this barrier, whatever happened above

@@ -134,8 +134,10 @@ fa_status_t fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, flo
  * Bytes of device scratch that fa_bwd needs for these sizes (0 for an empty
  * problem).  Linear in N: two fp32 values per query row (D_i = dO_i . O_i and
  * the logsumexp in base 2) plus an fp32 dQ accumulator [B][Hq][Np][d], with N
- * rounded up to a multiple of 128 (Np), plus 256 bytes (the main pass's
- * work-item counter).
+ * rounded up to a multiple of 128 (Np), plus one 32-bit counter per 64 rows
+ * (the additions each query block's accumulator has received), plus 256
+ * bytes (the main pass's work-item counter):
+ * 4 * B * Hq * Np * (2 + d) + 4 * B * Hq * Np / 64 + 256.
  */
 size_t fa_bwd_workspace_bytes(int B, int Hq, int Hkv, int N, int d);
 
@@ -145,11 +147,12 @@ size_t fa_bwd_workspace_bytes(int B, int Hq, int Hkv, int N, int d);
  * scores and probabilities are recomputed from q, k and lse.  workspace is
  * caller-owned device memory of at least fa_bwd_workspace_bytes(...) bytes,
  * 16-byte aligned; its contents on entry do not matter and on exit are
- * unspecified.  Three kernels run on `stream` in order: a row pass (D and the
- * zeroed dQ accumulator), the main pass (persistent, one thread block per
- * SM, each taking work items = (key block of 128 rows, key/value head) in
- * turn: dK, dV in tensor memory, dQ added into the accumulator), and a pass
- * that scales and converts dQ.
+ * unspecified.  Two kernels run on `stream` in order: a row pass (D, the
+ * zeroed dQ accumulator and counters) and the main pass (persistent, one
+ * thread block per SM, each taking work items = (key block of 128 rows,
+ * key/value head) in turn: dK, dV in tensor memory, dQ added into the
+ * accumulator; the block that adds the last part of a 64-row query block's
+ * dQ scales and converts that block to dq).
  */
 fa_status_t fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
                    const float* lse, void* dq, void* dk, void* dv,
@@ -176,6 +179,49 @@ fa_status_t fa_bwd_dropout(const void* q, const void* k, const void* v, const vo
                            int B, int Hq, int Hkv, int N, int d, float scale, int causal,
                            float p_drop, uint64_t seed, fa_dtype_t dtype, void* workspace,
                            size_t workspace_bytes, void* stream);
+
+/*
+ * Block-sparse attention ("FlashAttention" glossary, block-sparse entry:
+ * blocks that a sparsity mask hides are skipped whole; the page gives no
+ * block size or pattern).  block_mask is device memory of bytes over blocks
+ * of 128 query rows x 128 keys, nb = ceil(N / 128) blocks a side:
+ * [Hq][nb][nb] when mask_per_head = 1, or one [nb][nb] mask for every query
+ * head when mask_per_head = 0 (the same mask for every batch entry).  Byte
+ * (h, i, j) nonzero: query block i of query head h sees key block j; zero:
+ * the whole block is hidden, and nothing of it is computed.  Combined with
+ * the causal mask when causal = 1 (a key is seen only if both allow it).  A
+ * query row that sees no key at all gets O = 0 and lse = -inf (the log of an
+ * empty sum) and adds nothing to the gradients.  The mask is read during
+ * the call only.  Limits: Hq / Hkv <= 16 and nb <= 4096, otherwise
+ * FA_ERR_UNSUPPORTED; a null mask or mask_per_head outside {0, 1} is
+ * FA_ERR_INVALID_ARG.  Otherwise as fa_fwd.
+ */
+fa_status_t fa_fwd_blockmask(const void* q, const void* k, const void* v, void* o, float* lse,
+                             int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+                             const uint8_t* block_mask, int mask_per_head, fa_dtype_t dtype,
+                             void* stream);
+
+/*
+ * Workspace of fa_bwd_blockmask: that of fa_bwd plus, per work item (kv head
+ * x key block), its step count and the list of (group head, query block)
+ * pairs that see it: fa_bwd_workspace_bytes(...) + 4 * B * Hkv * nb
+ * + 2 * B * Hkv * nb * (Hq / Hkv) * nb bytes, nb = ceil(N / 128).  0 for an
+ * empty problem or Hq % Hkv != 0.
+ */
+size_t fa_bwd_blockmask_workspace_bytes(int B, int Hq, int Hkv, int N, int d);
+
+/*
+ * Backward pass of fa_fwd_blockmask with the same mask: each key block walks
+ * only the query blocks that see it (a list made by a planning pass at the
+ * start of the call).  o and lse must come from fa_fwd_blockmask; workspace
+ * of at least fa_bwd_blockmask_workspace_bytes(...) bytes.  Otherwise as
+ * fa_bwd.
+ */
+fa_status_t fa_bwd_blockmask(const void* q, const void* k, const void* v, const void* o,
+                             const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                             int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+                             const uint8_t* block_mask, int mask_per_head, fa_dtype_t dtype,
+                             void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * Decode over a paged key/value cache ("Paper digest: FlashAttention",

@@ -55,11 +55,18 @@ def check_o(o_gpu, o_ref, dtype, what="O"):
     """max |O_gpu - O_ref| <= 1e-2, every element, no exception."""
     g, r = _np(o_gpu), _np(o_ref)
     err = np.abs(g - r)
-    max_err = float(err.max(initial=0.0))
-    info = dict(max_err=max_err,
-                max_err_ulps=float((err / _ulp(r, dtype)).max(initial=0.0)))
-    assert max_err <= TOL_O, f"{what}: {int((err > TOL_O).sum())} elements beyond {TOL_O}, {info}"
+    info = _err_info(err, r, dtype)
+    assert info["max_err"] <= TOL_O, f"{what}: {int((err > TOL_O).sum())} elements beyond {TOL_O}, {info}"
     return info
+
+
+def _err_info(err, r, dtype):
+    """Largest error, and the same in ulps of the output value it sits on."""
+    if err.size == 0:
+        return dict(max_err=0.0, max_err_ulps=0.0)
+    i = int(np.argmax(err))
+    return dict(max_err=float(err.flat[i]),
+                max_err_ulps=float(err.flat[i] / _ulp(r.flat[i], dtype)))
 
 
 def check_o_rounding_bound(o_gpu, o_ref, dtype, o_absv, what="O"):
@@ -76,8 +83,7 @@ def check_o_rounding_bound(o_gpu, o_ref, dtype, o_absv, what="O"):
     mant = 8 if dtype == torch.bfloat16 else 11
     bound = 2.0 ** -mant * _np(o_absv) + 0.5 * _ulp(r, dtype) + 1e-3
     bad = err > bound
-    info = dict(max_err=float(err.max(initial=0.0)), n_over_1e_2=int((err > TOL_O).sum()),
-                max_err_ulps=float((err / _ulp(r, dtype)).max(initial=0.0)))
+    info = dict(_err_info(err, r, dtype), n_over_1e_2=int((err > TOL_O).sum()))
     assert not bad.any(), f"{what}: {int(bad.sum())} elements beyond the rounding bound, {info}"
     return info
 
@@ -109,11 +115,20 @@ def oracle_dropout(dropout):
 
 
 def check_full(q, k, v, do, scale, causal, out, window=0, dropout=None):
-    """Every output element against the full oracle."""
+    """Every output element against the full oracle.  With dropout, O is
+    held to the rounding bound of check_o_rounding_bound instead of 1e-2:
+    the kept probabilities carry the factor 1/(1-p), so O reaches magnitudes
+    (4 and above) where half an ulp of a bf16 output alone exceeds 1e-2; the
+    number of elements above 1e-2 is reported."""
     dr = oracle_dropout(dropout)
     o_r, lse_r = oracle.fwd(q, k, v, scale, causal, window=window, dropout=dr)
     dq_r, dk_r, dv_r = oracle.bwd(q, k, v, do, scale, causal, window=window, dropout=dr)
-    rep = dict(o=check_o(out["o"], o_r, q.dtype), lse=check_lse(out["lse"], lse_r))
+    if dr:
+        o_abs, _ = oracle.fwd(q, k, v.abs(), scale, causal, window=window, dropout=dr)
+        o_rep = check_o_rounding_bound(out["o"], o_r, q.dtype, o_abs, what="O (dropout)")
+    else:
+        o_rep = check_o(out["o"], o_r, q.dtype)
+    rep = dict(o=o_rep, lse=check_lse(out["lse"], lse_r))
     rep.update(dq=check_grad(out["dq"], dq_r, "dQ"), dk=check_grad(out["dk"], dk_r, "dK"),
                dv=check_grad(out["dv"], dv_r, "dV"))
     return rep

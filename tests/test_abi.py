@@ -104,16 +104,44 @@ def test_empty_problems_are_no_ops(lib):
 
 def test_workspace_is_linear_in_n():
     # two fp32 row statistics + an fp32 dQ accumulator per (padded) query row,
-    # plus a fixed 256-byte tail (the main pass's work-item counter)
+    # one 32-bit counter per 64 rows, plus a fixed 256-byte tail (the main
+    # pass's work-item counter)
     tail = 256
     for d in (64, 128):
         sizes = [binding.fa_bwd_workspace_bytes(1, 16, 16, n, d) - tail
                  for n in (4096, 8192, 16384, 32768, 65536)]
         for a, b in zip(sizes, sizes[1:]):
             assert b == 2 * a
-        assert sizes[0] == 16 * 4096 * 4 * (2 + d)
+        assert sizes[0] == 16 * 4096 * 4 * (2 + d) + 16 * 4096 // 64 * 4
     # padding to a multiple of 128 rows
-    assert binding.fa_bwd_workspace_bytes(1, 1, 1, 129, 64) == 256 * 4 * 66 + tail
+    assert binding.fa_bwd_workspace_bytes(1, 1, 1, 129, 64) == 256 * 4 * 66 + 256 // 64 * 4 + tail
+
+
+def test_blockmask_workspace_and_argument_errors(lib):
+    vp = ctypes.c_void_p
+    B, Hq, Hkv, N, d = 2, 8, 2, 1000, 128
+    nb = -(-N // 128)
+    plain = binding.fa_bwd_workspace_bytes(B, Hq, Hkv, N, d)
+    # per work item (kv head x key block): a step count and a walk of at most
+    # group x nb two-byte entries
+    assert binding.fa_bwd_blockmask_workspace_bytes(B, Hq, Hkv, N, d) == \
+        plain + 4 * B * Hkv * nb + 2 * B * Hkv * nb * (Hq // Hkv) * nb
+    assert binding.fa_bwd_blockmask_workspace_bytes(1, 3, 2, 256, 64) == 0  # Hq % Hkv
+    fwd = lambda mask, per_head, Hq=2, Hkv=2, N=256: lib.fa_fwd_blockmask(
+        *([vp(FAKE)] * 5 + [1, Hq, Hkv, N, 64, 0.125, 1, mask, per_head, binding.FA_BF16, None]))
+    assert fwd(None, 0) == binding.FA_ERR_INVALID_ARG                 # no mask
+    assert fwd(vp(FAKE), 2) == binding.FA_ERR_INVALID_ARG             # per_head not 0/1
+    assert fwd(vp(FAKE), 0, Hq=34, Hkv=2) == binding.FA_ERR_UNSUPPORTED  # group > 16
+    assert fwd(vp(FAKE), 0, N=4096 * 128 + 1) == binding.FA_ERR_UNSUPPORTED  # nb > 4096
+    ws = binding.fa_bwd_blockmask_workspace_bytes(1, 2, 2, 256, 64)
+    bwd = lambda mask, per_head, ws_bytes=ws: lib.fa_bwd_blockmask(
+        *([vp(FAKE)] * 9 + [1, 2, 2, 256, 64, 0.125, 1, mask, per_head, binding.FA_BF16, vp(FAKE),
+                            ws_bytes, None]))
+    assert bwd(None, 1) == binding.FA_ERR_INVALID_ARG
+    assert bwd(vp(FAKE), 1, binding.fa_bwd_workspace_bytes(1, 2, 2, 256, 64)) == binding.FA_ERR_INVALID_ARG
+    # empty problems are no-ops
+    assert lib.fa_fwd_blockmask(*([vp(0)] * 5 + [0, 2, 2, 256, 64, 0.125, 1, vp(FAKE), 0,
+                                                 binding.FA_BF16, None])) == binding.FA_OK
 
 
 def test_bwd_max_blocks_setting(lib):
