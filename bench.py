@@ -418,7 +418,9 @@ def run_ours(args, w, causal, rank, world, device):
     peak = pk["bf16_tflops"]
     head = summarize(w, causal, res, K, peak, W, (f_fwd, f_bwd))
     bwd_tflops_main = f_bwd / (bwd_main_mean * 1e-3) / 1e12
-    launches_per_step = 3  # fa_fwd_kernel, fa_bwd_pre_kernel, fa_bwd_kernel
+    launches_per_step = 4  # fa_fwd_kernel, fa_bwd_pre_kernel, fa_bwd_kernel, fa_bwd_post_kernel
+    if BM is not None:
+        launches_per_step += 1  # fa_bwd_plan_kernel
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True,

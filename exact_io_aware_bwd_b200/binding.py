@@ -390,7 +390,7 @@ def attention_fwd(q, k, v, scale: float | None = None, causal: bool = False, str
     """Allocates O and lse with PyTorch and runs fa_fwd (fa_fwd_window when
     window > 0, which implies causal; fa_fwd_dropout when dropout = (p_drop,
     seed); fa_fwd_blockmask when block_mask is given); returns (O, lse)."""
-    if sum(x is not None and x is not False and x != 0 for x in (window, dropout, block_mask)) > 1:
+    if sum((bool(window), bool(dropout), block_mask is not None)) > 1:
         raise ValueError("a sliding window, dropout and a block mask are not combined")
     B, Hq, Hkv, N, d = _dims(q, k)
     scale = 1.0 / math.sqrt(d) if scale is None else scale

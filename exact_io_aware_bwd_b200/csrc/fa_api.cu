@@ -213,11 +213,10 @@ fa_status_t bwd_run(const void* q, const void* k, const void* v, const void* o, 
   float* lse2 = Dvec + BHq * Np;
   float* dqacc = lse2 + BHq * Np;
   const int64_t rows = BHq * Np;
-  unsigned* dq_count = reinterpret_cast<unsigned*>(dqacc + rows * HD);
-  unsigned* work_counter = dq_count + rows / 64;
+  unsigned* work_counter = reinterpret_cast<unsigned*>(dqacc + rows * HD);
   const int n_ktiles = (N + 127) / 128;
 
-  // 1. D, lse2, zeroed accumulator, arrival counters and work counter
+  // 1. D, lse2, zeroed accumulator and work counter
   fa::BwdPreParams pre;
   std::memset(&pre, 0, sizeof(pre));
   pre.o = o;
@@ -226,17 +225,9 @@ fa_status_t bwd_run(const void* q, const void* k, const void* v, const void* o, 
   pre.Dvec = Dvec;
   pre.lse2 = lse2;
   pre.dqacc = dqacc;
-  pre.dq_count = dq_count;
   pre.work_counter = work_counter;
-  pre.dq = dq;
-  pre.bmask = bmask;
-  pre.bm_hstride = bm_hstride;
   pre.N = N;
   pre.Np = static_cast<int>(Np);
-  pre.Hq = Hq;
-  pre.n_ktiles = n_ktiles;
-  pre.causal = causal;
-  pre.window = window;
   pre.total_rows = rows;
   fa::fa_bwd_pre_kernel<HD, BF><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(pre);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
@@ -280,8 +271,6 @@ fa_status_t bwd_run(const void* q, const void* k, const void* v, const void* o, 
   prm.lse2 = lse2;
   prm.Dvec = Dvec;
   prm.dqacc = dqacc;
-  prm.dq_count = dq_count;
-  prm.dq = dq;
   prm.plan_list = plan_list;
   prm.plan_steps = plan_steps;
   prm.plan_cap = plan_cap;
@@ -317,15 +306,24 @@ fa_status_t bwd_run(const void* q, const void* k, const void* v, const void* o, 
   if ((n_sm = sm_count()) <= 0) return FA_ERR_CUDA;
   const int cap = g_bwd_max_blocks.load();
   const int grid = std::min(prm.n_items, cap > 0 ? std::min(cap, n_sm) : n_sm);  // persistent
+  fa_status_t s;
   if (bmask != nullptr)
-    return causal ? launch_bwd_main<HD, BF, true, false, true>(prm, grid, st)
-                  : launch_bwd_main<HD, BF, false, false, true>(prm, grid, st);
-  fa_status_t s = prm.drop_t > 0
-                      ? (causal ? launch_bwd_main<HD, BF, true, true>(prm, grid, st)
-                                : launch_bwd_main<HD, BF, false, true>(prm, grid, st))
-                      : (causal ? launch_bwd_main<HD, BF, true, false>(prm, grid, st)
-                                : launch_bwd_main<HD, BF, false, false>(prm, grid, st));
-  return s;
+    s = causal ? launch_bwd_main<HD, BF, true, false, true>(prm, grid, st)
+               : launch_bwd_main<HD, BF, false, false, true>(prm, grid, st);
+  else if (prm.drop_t > 0)
+    s = causal ? launch_bwd_main<HD, BF, true, true>(prm, grid, st)
+               : launch_bwd_main<HD, BF, false, true>(prm, grid, st);
+  else
+    s = causal ? launch_bwd_main<HD, BF, true, false>(prm, grid, st)
+               : launch_bwd_main<HD, BF, false, false>(prm, grid, st);
+  if (s != FA_OK) return s;
+
+  // 3. dQ = scale * accumulator
+  const int64_t total_vec = BHq * N * (HD / 8);
+  const int64_t blocks = std::min<int64_t>((total_vec + 255) / 256, 148 * 16);
+  fa::fa_bwd_post_kernel<HD, BF><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+      dqacc, dq, N, static_cast<int>(Np), total_vec, scale);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 }  // namespace

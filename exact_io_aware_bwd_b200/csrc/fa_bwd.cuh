@@ -15,9 +15,8 @@
 //
 // Three kernels:
 //   bwd_pre   one warp per query row: D_i = dO_i . O_i, lse2_i = lse_i log2(e)
-//             (+inf for padding rows, which makes their P exactly 0), a
-//             zeroed fp32 dQ accumulator row and, per 64-row query block, a
-//             zeroed arrival counter.
+//             (+inf for padding rows, which makes their P exactly 0), and a
+//             zeroed fp32 dQ accumulator row.
 //   bwd_main  persistent: one thread block per SM takes work items (128-row
 //             key block j, kv head) one after another from a counter in the
 //             workspace, head-major and, within a head, the key blocks with
@@ -39,11 +38,9 @@
 //             item's Q / dO loads start while the last steps of the previous
 //             one run, and its dK / dV are written out while the next item's
 //             first steps run.
-//             A query block's dQ is final once every key block that sees it
-//             has added its part: each addition is counted, and the drain
-//             warps of the block that brings the last one convert the query
-//             block (dQ = scale * accumulator, to the I/O dtype) while it is
-//             still in L2.  No separate pass over the accumulator.
+//   bwd_post  dQ = scale * accumulator, converted to the I/O dtype (rows
+//             that no key block reaches, possible under a block mask, keep
+//             their zeroed accumulator: dQ = 0).
 //
 // Warp roles of bwd_main (448 threads):
 //   warps 0-7   softmax-gradient: warp w owns key rows 32(w%4)..+31 (tensor
@@ -70,50 +67,22 @@ namespace fa {
 
 constexpr uint32_t kKernBwdPre = 2;
 constexpr uint32_t kKernBwd = 3;
+constexpr uint32_t kKernBwdPost = 4;
 constexpr uint32_t kKernSelftest = 9;
 
 __host__ __device__ inline int64_t bwd_padded_rows(int N) { return (static_cast<int64_t>(N) + 127) / 128 * 128; }
 
-// Workspace: D [rows], lse2 [rows], dQ accumulator [rows][d] (fp32), one
-// arrival counter per 64-row query block [rows / 64] (uint32), then 256 bytes
-// holding the work-item counter of bwd_main.
+// Workspace: D [rows], lse2 [rows], dQ accumulator [rows][d] (fp32), then
+// 256 bytes holding the work-item counter of bwd_main.
 constexpr size_t kBwdWorkspaceTail = 256;
 
 inline size_t bwd_workspace_bytes(int B, int Hq, int N, int d) {
   const int64_t rows = static_cast<int64_t>(B) * Hq * bwd_padded_rows(N);
-  return static_cast<size_t>(rows) * 4u * static_cast<size_t>(2 + d) + static_cast<size_t>(rows / 64) * 4u +
-         kBwdWorkspaceTail;
+  return static_cast<size_t>(rows) * 4u * static_cast<size_t>(2 + d) + kBwdWorkspaceTail;
 }
 
 // ---------------------------------------------------------------------------
 // bwd_pre
-
-// Number of key blocks whose walk includes 64-row query block qt (of query
-// head hq within its batch): the additions its dQ accumulator receives.  A
-// key block jt walks query blocks [i0, i_end) (bwd_item); under a block
-// mask only those whose 128-row block it sees.  Counted by the whole warp.
-__device__ __forceinline__ unsigned bwd_dq_expected(int qt, int hq, int N, int n_ktiles, int causal,
-                                                    int window, const uint8_t* bmask,
-                                                    long long bm_hstride, int lane) {
-  int jt_lo = 0, jt_hi = n_ktiles - 1;
-  if (causal) {
-    jt_hi = min(qt >> 1, n_ktiles - 1);  // i0 = 2 jt <= qt
-    if (window > 0) {
-      // i_end > qt  <=>  128 jt + 126 + W >= 64 qt
-      const int num = 64 * qt - 126 - window;
-      jt_lo = num > 0 ? (num + 127) / 128 : 0;
-    }
-  }
-  if (jt_hi < jt_lo) return 0u;
-  if (bmask == nullptr) return static_cast<unsigned>(jt_hi - jt_lo + 1);
-  const uint8_t* row = bmask + hq * bm_hstride + static_cast<long long>(qt >> 1) * n_ktiles;
-  unsigned n = 0;
-  for (int j0 = jt_lo; j0 <= jt_hi; j0 += 32) {
-    const int jt = j0 + lane;
-    n += __popc(__ballot_sync(0xffffffffu, jt <= jt_hi && __ldg(row + jt) != 0));
-  }
-  return n;
-}
 
 struct BwdPreParams {
   const void* o;
@@ -122,12 +91,8 @@ struct BwdPreParams {
   float* Dvec;            // [B*Hq][Np]
   float* lse2;            // [B*Hq][Np]
   float* dqacc;           // [B*Hq][Np][d], zeroed here
-  unsigned* dq_count;     // [B*Hq][Np / 64], set to the additions each query block will receive
   unsigned* work_counter;
-  void* dq;               // rows of query blocks that no key block sees are zeroed here
-  const uint8_t* bmask;   // block mask or nullptr
-  long long bm_hstride;
-  int N, Np, Hq, n_ktiles, causal, window;
+  int N, Np;
   long long total_rows;
 };
 
@@ -155,20 +120,6 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const __grid_constant__
   if (lane == 0) {
     p.Dvec[row] = acc;
     p.lse2[row] = n < N ? p.lse[bh * N + n] * 1.4426950408889634f : INFINITY;
-  }
-  if ((n & 63) == 0) {
-    const int qt = n >> 6;
-    const unsigned cnt = n < N ? bwd_dq_expected(qt, static_cast<int>(bh % p.Hq), N, p.n_ktiles, p.causal,
-                                                 p.window, p.bmask, p.bm_hstride, lane)
-                               : 0u;
-    if (lane == 0) p.dq_count[row >> 6] = cnt;
-    if (cnt == 0 && n < N) {
-      // no key block adds to this query block (only under a block mask):
-      // its dQ is zero and no conversion will write it
-      const int rows_here = min(64, N - n);
-      uint4* out = reinterpret_cast<uint4*>(reinterpret_cast<T*>(p.dq) + (bh * N + n) * HD);
-      for (int i = lane; i < rows_here * HD / 8; i += 32) out[i] = make_uint4(0u, 0u, 0u, 0u);
-    }
   }
   float* z = p.dqacc + row * HD + lane * kPer;
 #pragma unroll
@@ -231,8 +182,6 @@ struct BwdParams {
   const float* lse2;     // [B*Hq][Np]
   const float* Dvec;     // [B*Hq][Np]
   float* dqacc;          // [B*Hq][Np][d] fp32 accumulator
-  unsigned* dq_count;    // [B*Hq][Np / 64] additions received per query block
-  void* dq;              // [B*Hq][N][d]
   void* dk;              // [B*Hkv][N][d]
   void* dv;
   unsigned* work_counter;  // next work item (zeroed by bwd_pre)
@@ -273,8 +222,7 @@ struct BwdLayout {
   static constexpr int kOffSched = kOffBar + kNumBars * 8;
   static constexpr int kOffTmemPtr = kOffSched + kSched * 4;
   static constexpr int kOffAbort = kOffTmemPtr + 4;
-  static constexpr int kOffConv = kOffAbort + 4;         // drain warps: convert this block?
-  static constexpr int kSmemBytes = kOffConv + 4;
+  static constexpr int kSmemBytes = kOffAbort + 4;
   // Tiles must sit on 1024-byte boundaries (128-byte swizzle atoms).  The
   // dynamic shared memory of a block without static shared memory starts on
   // such a boundary on sm_100; the d = 64 layout keeps spare bytes for
@@ -398,7 +346,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
   volatile int* sched_item = reinterpret_cast<volatile int*>(sm + L::kOffSched);
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(sm + L::kOffTmemPtr);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::kOffAbort);
-  volatile int* conv_flag = reinterpret_cast<volatile int*>(sm + L::kOffConv);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -478,7 +425,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
         mbar_arrive(&sched_full[slot]);
         if (item < 0) break;
         const BwdItem it = bwd_item<CAUSAL, BMASK>(p, item);
-        if (it.T == 0) continue;  // no step (block mask): no loads; the epilogue writes zeros
+        if (it.T == 0) {
+          // No step (block mask): no loads; the epilogue writes zeros.  The
+          // wait on the previous item's completion is still taken, so that
+          // every wait on acc_done stays within one phase of the barrier
+          // (a parity wait two phases behind would pass at once).
+          if (n > 0 && !mbar_wait(acc_done, (n - 1) & 1, abort_flag, kKernBwd, 12, 2)) break;
+          continue;
+        }
         BwdWalk<BMASK> walk;
         auto load_step = [&](int t) -> bool {
           const int g = gt + t, s = g % L::kStages;
@@ -565,7 +519,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
       if (item < 0) break;
       const BwdItem it = bwd_item<CAUSAL, BMASK>(p, item);
       if (it.T == 0) {
-        // nothing to compute (block mask); the epilogue writes zero dK, dV
+        // Nothing to compute (block mask); the epilogue writes zero dK, dV.
+        // As for every item, acc_done is committed only once the previous
+        // item's epilogue has read its accumulators, which keeps the
+        // epilogue's waits on acc_done within one phase.
+        if (n > 0 && !wait_all(acc_free, (n - 1) & 1, 7)) break;
         umma_commit_w(acc_done);
         continue;
       }
@@ -833,43 +791,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
         mbar_arrive(&dq_drained[buf]);
         int bh, qt;
         walk.next(it, &bh, &qt);
-        float* acc_blk = p.dqacc + (static_cast<size_t>(bh) * p.Np + qt * 64) * HD;
-        float* dst = acc_blk + dw * 32 + lane;
+        float* dst = p.dqacc + (static_cast<size_t>(bh) * p.Np + qt * 64) * HD + dw * 32 + lane;
 #pragma unroll
         for (int q = 0; q < 32; ++q) atomicAdd(dst + q * HD, __uint_as_float(v0[q]));
 #pragma unroll
         for (int q = 0; q < 32; ++q) atomicAdd(dst + (32 + q) * HD, __uint_as_float(v1[q]));
-        // Count this addition down from the number the query block receives
-        // (set by bwd_pre); the block bringing the last one converts it.
-        // Every drain thread's additions are ordered before the count (fence,
-        // barrier, fence by the counting thread), and the converting threads'
-        // reads after it (fence after the barrier).
-        __threadfence();
-        named_barrier_sync(1, kDrainThreads);
-        if (dw == 0 && lane == 0) {
-          __threadfence();
-          const unsigned old = atomicSub(p.dq_count + static_cast<size_t>(bh) * (p.Np / 64) + qt, 1u);
-          *conv_flag = old == 1u ? 1 : 0;
-        }
-        named_barrier_sync(1, kDrainThreads);
-        if (*conv_flag) {
-          __threadfence();
-          // dQ = scale * accumulator -> I/O dtype, rows of the block below N
-          constexpr int kVec = HD / 4;  // float4 per row
-          T* out = reinterpret_cast<T*>(p.dq) + (static_cast<size_t>(bh) * p.N + qt * 64) * HD;
-          const int rows_here = min(64, p.N - qt * 64);
-          for (int i = dw * 32 + lane; i < rows_here * kVec; i += kDrainThreads) {
-            const int row = i / kVec, c4 = i % kVec;
-            const float4 a = __ldcg(reinterpret_cast<const float4*>(acc_blk + row * HD) + c4);
-            uint2 w;
-            w.x = pack2<BF16>(a.x * p.scale, a.y * p.scale);
-            w.y = pack2<BF16>(a.z * p.scale, a.w * p.scale);
-            *reinterpret_cast<uint2*>(out + row * HD + c4 * 4) = w;
-          }
-        }
-        // the flag is read by every drain thread before the next step's
-        // counting thread may write it: the barrier of the next step comes
-        // after these reads
       }
       if (!ok) break;
       gt += it.T;
@@ -920,6 +846,32 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
   if (warp == 13) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// bwd_post: dQ = scale * accumulator -> I/O dtype (8 elements per thread)
+
+template <int HD, bool BF16>
+__global__ void __launch_bounds__(256) fa_bwd_post_kernel(const float* __restrict__ dqacc,
+                                                          void* __restrict__ dq_, int N, int Np,
+                                                          int64_t total_vec, float scale) {
+  using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
+  constexpr int kVecPerRow = HD / 8;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total_vec;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t row = i / kVecPerRow;  // row of the [B*Hq][N] output
+    const int cv = static_cast<int>(i % kVecPerRow);
+    const int64_t bh = row / N;
+    const int64_t n = row % N;
+    const float4* src = reinterpret_cast<const float4*>(dqacc + (bh * Np + n) * HD + cv * 8);
+    const float4 a = src[0], c = src[1];
+    uint4 w;
+    w.x = pack2<BF16>(a.x * scale, a.y * scale);
+    w.y = pack2<BF16>(a.z * scale, a.w * scale);
+    w.z = pack2<BF16>(c.x * scale, c.y * scale);
+    w.w = pack2<BF16>(c.z * scale, c.w * scale);
+    reinterpret_cast<uint4*>(reinterpret_cast<T*>(dq_) + row * HD)[cv] = w;
   }
 }
 

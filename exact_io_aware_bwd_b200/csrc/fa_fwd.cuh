@@ -463,13 +463,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
       {
         uint32_t s[128];
         const bool masked = load_s(kb, s);
-        // row max, eight independent chains of three-input maxima
+        // row max, eight independent chains of three-input maxima: chain i
+        // takes columns i, i + 8, ..., i + 120
         float mx[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) mx[i] = max3f(__uint_as_float(s[i]), __uint_as_float(s[8 + i]),
-                                                  __uint_as_float(s[16 + i]));
+        for (int i = 0; i < 8; ++i) mx[i] = fmaxf(__uint_as_float(s[i]), __uint_as_float(s[8 + i]));
 #pragma unroll
-        for (int c = 24; c < 128; c += 16)
+        for (int c = 16; c < 128; c += 16)
 #pragma unroll
           for (int i = 0; i < 8; ++i)
             mx[i] = max3f(mx[i], __uint_as_float(s[c + i]), __uint_as_float(s[c + 8 + i]));

@@ -134,10 +134,8 @@ fa_status_t fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, flo
  * Bytes of device scratch that fa_bwd needs for these sizes (0 for an empty
  * problem).  Linear in N: two fp32 values per query row (D_i = dO_i . O_i and
  * the logsumexp in base 2) plus an fp32 dQ accumulator [B][Hq][Np][d], with N
- * rounded up to a multiple of 128 (Np), plus one 32-bit counter per 64 rows
- * (the additions each query block's accumulator has received), plus 256
- * bytes (the main pass's work-item counter):
- * 4 * B * Hq * Np * (2 + d) + 4 * B * Hq * Np / 64 + 256.
+ * rounded up to a multiple of 128 (Np), plus 256 bytes (the main pass's
+ * work-item counter): 4 * B * Hq * Np * (2 + d) + 256.
  */
 size_t fa_bwd_workspace_bytes(int B, int Hq, int Hkv, int N, int d);
 
@@ -147,12 +145,11 @@ size_t fa_bwd_workspace_bytes(int B, int Hq, int Hkv, int N, int d);
  * scores and probabilities are recomputed from q, k and lse.  workspace is
  * caller-owned device memory of at least fa_bwd_workspace_bytes(...) bytes,
  * 16-byte aligned; its contents on entry do not matter and on exit are
- * unspecified.  Two kernels run on `stream` in order: a row pass (D, the
- * zeroed dQ accumulator and counters) and the main pass (persistent, one
- * thread block per SM, each taking work items = (key block of 128 rows,
- * key/value head) in turn: dK, dV in tensor memory, dQ added into the
- * accumulator; the block that adds the last part of a 64-row query block's
- * dQ scales and converts that block to dq).
+ * unspecified.  Three kernels run on `stream` in order: a row pass (D and the
+ * zeroed dQ accumulator), the main pass (persistent, one thread block per
+ * SM, each taking work items = (key block of 128 rows, key/value head) in
+ * turn: dK, dV in tensor memory, dQ added into the accumulator), and a pass
+ * that scales and converts dQ.
  */
 fa_status_t fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
                    const float* lse, void* dq, void* dk, void* dv,

@@ -104,17 +104,16 @@ def test_empty_problems_are_no_ops(lib):
 
 def test_workspace_is_linear_in_n():
     # two fp32 row statistics + an fp32 dQ accumulator per (padded) query row,
-    # one 32-bit counter per 64 rows, plus a fixed 256-byte tail (the main
-    # pass's work-item counter)
+    # plus a fixed 256-byte tail (the main pass's work-item counter)
     tail = 256
     for d in (64, 128):
         sizes = [binding.fa_bwd_workspace_bytes(1, 16, 16, n, d) - tail
                  for n in (4096, 8192, 16384, 32768, 65536)]
         for a, b in zip(sizes, sizes[1:]):
             assert b == 2 * a
-        assert sizes[0] == 16 * 4096 * 4 * (2 + d) + 16 * 4096 // 64 * 4
+        assert sizes[0] == 16 * 4096 * 4 * (2 + d)
     # padding to a multiple of 128 rows
-    assert binding.fa_bwd_workspace_bytes(1, 1, 1, 129, 64) == 256 * 4 * 66 + 256 // 64 * 4 + tail
+    assert binding.fa_bwd_workspace_bytes(1, 1, 1, 129, 64) == 256 * 4 * 66 + tail
 
 
 def test_blockmask_workspace_and_argument_errors(lib):
