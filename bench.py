@@ -742,6 +742,8 @@ def main():
     ap.add_argument("--block-mask", default="",
                     help="block-sparse mask over 128 x 128 blocks: 'local' or 'random:RHO'; FLOPs "
                          "counted over visible pairs")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="override the workload's batch size (small cases for profiler captures)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-range", action="store_true",
                     help="skip the 16K GQA and 64K fp16 sub-results of the default line")
@@ -751,6 +753,9 @@ def main():
     assert args.warmup >= 0 and args.steps >= 1
 
     w = WORKLOADS[args.workload]
+    if args.batch:
+        from dataclasses import replace
+        w = replace(w, B=args.batch)
     causal = (not args.noncausal) and (True in w.causal_modes)
     if sum(bool(x) for x in (args.window, args.dropout, args.block_mask)) > 1:
         raise SystemExit("bench.py: --window, --dropout and --block-mask are not combined")

@@ -229,7 +229,15 @@ fa_status_t bwd_run(const void* q, const void* k, const void* v, const void* o, 
   pre.N = N;
   pre.Np = static_cast<int>(Np);
   pre.total_rows = rows;
-  fa::fa_bwd_pre_kernel<HD, BF><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(pre);
+  {
+    // HD / 8 threads a row; a grid of 16 blocks of 256 threads per SM, each
+    // thread taking rows in turn
+    const int64_t groups = rows * (HD / 8);
+    int n_sm = sm_count();
+    if (n_sm <= 0) return FA_ERR_CUDA;
+    const int64_t blocks = std::min<int64_t>((groups + 255) / 256, static_cast<int64_t>(n_sm) * 16);
+    fa::fa_bwd_pre_kernel<HD, BF><<<static_cast<unsigned>(blocks), 256, 0, st>>>(pre);
+  }
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
 
   // 1b. block mask: the walk of every work item

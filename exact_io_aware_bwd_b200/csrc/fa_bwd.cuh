@@ -96,34 +96,44 @@ struct BwdPreParams {
   long long total_rows;
 };
 
+// One group of HD / 8 threads per query row, each thread 8 elements (16
+// bytes) of O and dO and 8 of the zeroed accumulator (two 16-byte stores);
+// the group's partial dot products are summed by shuffles.  Grid-stride over
+// the rows, so that every thread keeps several rows' loads in flight; a
+// warp's lanes take 32 / (HD / 8) consecutive rows and the row count (a
+// multiple of 128) and the stride are multiples of that, so all lanes of a
+// warp run the same iterations and the shuffles see every lane.
 template <int HD, bool BF16>
 __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const __grid_constant__ BwdPreParams p) {
   using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
-  const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (blockIdx.x == 0 && threadIdx.x == 0) *p.work_counter = 0u;
-  if (row >= p.total_rows) return;
-  const int64_t bh = row / p.Np;
-  const int n = static_cast<int>(row % p.Np);
-  const int N = p.N;
-  constexpr int kPer = HD / 32;  // elements per lane: 2 or 4
-  float acc = 0.f;
-  if (n < N) {
-    const int64_t base = (bh * N + n) * HD + lane * kPer;
-    const T* o = reinterpret_cast<const T*>(p.o) + base;
-    const T* d = reinterpret_cast<const T*>(p.dout) + base;
+  constexpr int kTpr = HD / 8;  // threads per row: 16 or 8
+  const int64_t gtid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int c8 = static_cast<int>(gtid % kTpr);
+  if (gtid == 0) *p.work_counter = 0u;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x / kTpr;
+  for (int64_t row = gtid / kTpr; row < p.total_rows; row += stride) {
+    const int64_t bh = row / p.Np;
+    const int n = static_cast<int>(row % p.Np);
+    float acc = 0.f;
+    if (n < p.N) {
+      const int64_t base = (bh * p.N + n) * HD + c8 * 8;
+      const uint4 ov = *reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(p.o) + base);
+      const uint4 dv = *reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(p.dout) + base);
+      const T* o8 = reinterpret_cast<const T*>(&ov);
+      const T* d8 = reinterpret_cast<const T*>(&dv);
 #pragma unroll
-    for (int e = 0; e < kPer; ++e) acc += static_cast<float>(o[e]) * static_cast<float>(d[e]);
+      for (int e = 0; e < 8; ++e) acc = fmaf(static_cast<float>(o8[e]), static_cast<float>(d8[e]), acc);
+    }
+#pragma unroll
+    for (int off = kTpr / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (c8 == 0) {
+      p.Dvec[row] = acc;
+      p.lse2[row] = n < p.N ? p.lse[bh * p.N + n] * 1.4426950408889634f : INFINITY;
+    }
+    float4* z = reinterpret_cast<float4*>(p.dqacc + row * HD + c8 * 8);
+    z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+    z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-  if (lane == 0) {
-    p.Dvec[row] = acc;
-    p.lse2[row] = n < N ? p.lse[bh * N + n] * 1.4426950408889634f : INFINITY;
-  }
-  float* z = p.dqacc + row * HD + lane * kPer;
-#pragma unroll
-  for (int e = 0; e < kPer; ++e) z[e] = 0.f;
 }
 
 // ---------------------------------------------------------------------------

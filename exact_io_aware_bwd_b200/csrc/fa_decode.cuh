@@ -18,13 +18,15 @@
 // second kernel merges the splits: m* = max m_s, l* = sum l_s 2^(m_s - m*),
 // O = sum O_s 2^(m_s - m*) / l*, lse = ln 2 (m* + log2 l*).
 //
-// Inside a block (128 threads) pages are staged in shared memory by
-// asynchronous 16-byte copies (cp.async), double-buffered so that the next
-// page is in flight while the current one is used; K rows are padded by 16
-// bytes so that one thread per key reads its row without bank conflicts.
-// Scores take all 128 threads (128 / P threads per key, combined by
-// shuffles), the softmax update one warp per row, and P V one thread per
-// output column.
+// Inside a block (128 threads) pages are staged in shared memory by bulk
+// copies (cp.async.bulk, the copy engine; completion counted in bytes on an
+// mbarrier) into a ring of kStages page slots, so that several pages are in
+// flight while one is used: warp 0 issues a page's copies (one per K row,
+// into rows padded by 16 bytes so that one thread per key reads its row
+// without bank conflicts, and one for the whole V page) and refills a slot
+// as soon as every thread is done with it.  Scores take all 128 threads
+// (128 / P threads per key, combined by shuffles), the softmax update one
+// warp per row, and P V one thread per output column.
 #pragma once
 
 #include <type_traits>
@@ -54,10 +56,24 @@ struct DecodeParams {
   float scale_log2;
 };
 
+// Page slots of the ring for page size P and row bound RB: as many as fit
+// in about 100 KB (two blocks per SM), at least 2 and at most 8.
+template <int HD>
+__host__ __device__ inline int decode_stages(int P, int rb) {
+  const int slot = P * (HD * 2 + 16) + P * HD * 2;
+  const int fixed = rb * HD * 4 + rb * P * 4 + 3 * kDecodeMaxRows * 4 + 8 * 8;
+  int st = (100 * 1024 - fixed) / slot;
+  return st < 2 ? 2 : (st > 8 ? 8 : st);
+}
+
+// Splits of each (sequence, kv head): enough blocks for four full waves of
+// two blocks per SM of a full B200, at least 4 pages a split.
 __host__ __device__ inline int decode_splits(int B, int Hkv, int max_pages) {
-  // enough blocks for two per SM of a full B200, never more than the pages
-  const int want = (2 * 148 + B * Hkv - 1) / (B * Hkv > 0 ? B * Hkv : 1);
-  return want < 1 ? 1 : (want > max_pages ? (max_pages > 0 ? max_pages : 1) : want);
+  const int bh = B * Hkv > 0 ? B * Hkv : 1;
+  int want = (4 * 2 * 148 + bh - 1) / bh;
+  const int cap = max_pages / 4 > 1 ? max_pages / 4 : 1;
+  want = want > cap ? cap : want;
+  return want < 1 ? 1 : want;
 }
 
 inline size_t decode_workspace_bytes(int B, int Hq, int Hkv, int Nq, int d, int max_pages) {
@@ -66,31 +82,26 @@ inline size_t decode_workspace_bytes(int B, int Hq, int Hkv, int Nq, int d, int 
   return static_cast<size_t>(rows) * 4u * static_cast<size_t>(d + 2);
 }
 
-// Shared memory for page size P and row bound RB (bytes, all offsets
-// multiples of 16): two page buffers (K padded, V), fp32 queries [RB][HD],
-// fp32 scores [RB][P], row state.  Sized by RB so that more blocks fit on an
-// SM when there are few rows.
+// Shared memory for page size P, row bound RB and the ring's slots (bytes,
+// all offsets multiples of 16): the slots' K (padded rows) and V pages,
+// fp32 queries [RB][HD], fp32 scores [RB][P], row state, slot barriers.
+// Sized by RB and P so that two blocks fit on an SM.
 template <int HD>
 struct DecodeLayout {
   static constexpr int kKRow = HD * 2 + 16;  // padded K row, bytes
-  int P, off_k, off_v, off_q, off_s, off_row, bytes;
+  int P, stages, off_k, off_v, off_q, off_s, off_row, off_bar, bytes;
   __host__ __device__ DecodeLayout(int page, int rb) : P(page) {
+    stages = decode_stages<HD>(page, rb);
     const int kbuf = page * kKRow, vbuf = page * HD * 2;
-    off_k = 0;                                   // K buffers 0, 1
-    off_v = 2 * kbuf;                            // V buffers 0, 1
-    off_q = off_v + 2 * vbuf;
+    off_k = 0;                                   // K slots
+    off_v = stages * kbuf;                       // V slots
+    off_q = off_v + stages * vbuf;
     off_s = off_q + rb * HD * 4;
     off_row = off_s + rb * page * 4;
-    bytes = off_row + 3 * kDecodeMaxRows * 4;
+    off_bar = off_row + 3 * kDecodeMaxRows * 4;
+    bytes = off_bar + 8 * 8;
   }
 };
-
-__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 // RB: compile-time bound on the rows (4, 8, 16 or 32, the smallest >= R), so
 // the per-row loops unroll to the rows that exist.
@@ -105,10 +116,12 @@ __global__ void __launch_bounds__(kDecodeThreads) fa_decode_split_kernel(const _
   float* sM = reinterpret_cast<float*>(smem + lay.off_row);
   float* sL = sM + kDecodeMaxRows;
   float* sC = sL + kDecodeMaxRows;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + lay.off_bar);  // [stages]
+  __shared__ int abort_flag;
 
   const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int G = p.Hq / p.Hkv, R = G * p.Nq, P = p.P;
+  const int G = p.Hq / p.Hkv, R = G * p.Nq, P = p.P, NS = lay.stages;
   const int Lb = p.lens[b];
   const bool len_ok = Lb >= p.Nq && Lb <= p.max_pages * P;
   if (!len_ok && split == 0 && g == 0 && tid == 0) record_error(kStatusBadInput, kKernDecode, 0, 0);
@@ -116,6 +129,11 @@ __global__ void __launch_bounds__(kDecodeThreads) fa_decode_split_kernel(const _
   const int pg0 = split * p.pages_per_split;
   const int pg1 = min(n_pages, pg0 + p.pages_per_split);
 
+  if (tid == 0) {
+    for (int i = 0; i < NS; ++i) mbar_init(&full[i], 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
   // queries of the block's rows (row r: head g*G + r / Nq, token r % Nq),
   // fp32 and scaled by scale * log2(e)
   for (int i = tid; i < R * HD; i += kDecodeThreads) {
@@ -133,39 +151,44 @@ __global__ void __launch_bounds__(kDecodeThreads) fa_decode_split_kernel(const _
   for (int r = 0; r < RB; ++r) acc[r] = 0.f;
   __syncthreads();
 
-  // page pg -> buffer (pg - pg0) & 1; a bad page id is recorded and its
-  // keys treated as hidden (nothing is read for it)
+  // page pg -> slot (pg - pg0) % NS; a bad page id is recorded and its keys
+  // treated as hidden: nothing is read for it and the slot's barrier is
+  // completed by a plain arrival.  Issued by warp 0.
   auto page_id = [&](int pg) { return p.table[static_cast<size_t>(b) * p.max_pages + pg]; };
   auto issue = [&](int pg) {
     const int phys = page_id(pg);
-    if (phys < 0 || phys >= p.num_pages) return;
-    const int buf = (pg - pg0) & 1;
-    uint8_t* sKb = smem + lay.off_k + buf * P * kKRow;
-    uint8_t* sVb = smem + lay.off_v + buf * P * HD * 2;
+    const int slot = (pg - pg0) % NS;
+    uint64_t* bar = &full[slot];
+    const bool good = phys >= 0 && phys < p.num_pages;
+    if (lane == 0) {
+      if (good)
+        mbar_expect_tx(bar, static_cast<uint32_t>(2 * P * HD * 2));
+      else
+        mbar_arrive(bar);
+    }
+    __syncwarp();
+    if (!good) return;
+    uint8_t* sKb = smem + lay.off_k + slot * P * kKRow;
+    uint8_t* sVb = smem + lay.off_v + slot * P * HD * 2;
     const size_t base = (static_cast<size_t>(phys) * p.Hkv + g) * P * HD;
     const uint8_t* kg = reinterpret_cast<const uint8_t*>(reinterpret_cast<const T*>(p.kc) + base);
     const uint8_t* vg = reinterpret_cast<const uint8_t*>(reinterpret_cast<const T*>(p.vc) + base);
-    constexpr int kVecRow = HD / 8;  // 16-byte vectors per row
-    for (int i = tid; i < P * kVecRow; i += kDecodeThreads) {
-      const int j = i / kVecRow, c = i % kVecRow;
-      cp_async16(sKb + j * kKRow + c * 16, kg + static_cast<size_t>(i) * 16);
-      cp_async16(sVb + static_cast<size_t>(i) * 16, vg + static_cast<size_t>(i) * 16);
-    }
+    for (int j = lane; j < P; j += 32) bulk_load(sKb + j * kKRow, kg + static_cast<size_t>(j) * HD * 2, HD * 2, bar);
+    if (lane == 0) bulk_load(sVb, vg, static_cast<uint32_t>(P * HD * 2), bar);
   };
-  if (pg0 < pg1) issue(pg0);
-  cp_async_commit();
+  int issued = pg0;  // pages whose copies warp 0 has issued: [pg0, issued)
+  if (warp == 0)
+    for (; issued < pg1 && issued < pg0 + NS; ++issued) issue(issued);
+  int consumed = pg0;  // pages fully used: [pg0, consumed); consumed <= issued
   for (int pg = pg0; pg < pg1; ++pg) {
-    // the next page's copies go out before this page is used
-    if (pg + 1 < pg1) issue(pg + 1);
-    cp_async_commit();
-    cp_async_wait<1>();  // every group but the newest has landed
-    __syncthreads();
+    const int slot = (pg - pg0) % NS;
+    const bool ok = mbar_wait(&full[slot], ((pg - pg0) / NS) & 1, &abort_flag, kKernDecode, 0, 1);
+    if (__syncthreads_or(!ok)) break;
     const int phys = page_id(pg);
     const bool page_ok = phys >= 0 && phys < p.num_pages;
     if (!page_ok && tid == 0) record_error(kStatusBadInput, kKernDecode, 1, 0);
-    const int buf = (pg - pg0) & 1;
-    const uint8_t* sK = smem + lay.off_k + buf * P * kKRow;
-    const T* sV = reinterpret_cast<const T*>(smem + lay.off_v + buf * P * HD * 2);
+    const uint8_t* sK = smem + lay.off_k + slot * P * kKRow;
+    const T* sV = reinterpret_cast<const T*>(smem + lay.off_v + slot * P * HD * 2);
     // scores: tpk = 128 / P threads per key, each over d / tpk features,
     // summed across the key's threads by shuffles; s[r][j] = q_r . k_j (log2
     // units), -inf where hidden (after the query, past the sequence, or a
@@ -258,9 +281,17 @@ __global__ void __launch_bounds__(kDecodeThreads) fa_decode_split_kernel(const _
         }
       }
     }
-    __syncthreads();  // this buffer and the scores are rewritten next
+    __syncthreads();  // every thread is done with this slot and the scores
+    consumed = pg + 1;
+    if (warp == 0 && issued < pg1) issue(issued++);
   }
-  cp_async_wait<0>();
+  // after an abort, copies still in flight land before the block exits:
+  // warp 0 waits (bounded) for every page it issued and no one consumed.
+  // pg0 <= consumed <= issued <= pg1 here (an empty split has all four
+  // equal), so every slot index below is in [0, NS).
+  if (warp == 0 && lane == 0)
+    for (int pg = consumed; pg < issued; ++pg)
+      mbar_wait_drain(&full[(pg - pg0) % NS], ((pg - pg0) / NS) & 1, kKernDecode, 0, 2);
 
   // partial results of this split: unnormalised O, (m, l)
   if (tid < HD) {

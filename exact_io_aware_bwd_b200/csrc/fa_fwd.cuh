@@ -129,13 +129,6 @@ constexpr uint32_t kFwdSoftmaxRegs = 216;
 constexpr uint32_t kFwdOtherRegs = 72;
 static_assert(2 * 128 * kFwdSoftmaxRegs + 128 * kFwdOtherRegs <= kFwdThreads * 168, "register split");
 constexpr uint32_t kKernFwd = 1;
-// Pairs of exponentials of every 8 (per 16 keys) computed on the FMA pipe in
-// unmasked score tiles; the rest go to the MUFU unit.
-#ifndef FA_FWD_POLY_PAIRS
-#define FA_FWD_POLY_PAIRS 0
-#endif
-constexpr int kPolyPairs = FA_FWD_POLY_PAIRS;
-
 template <int HD, bool BF16, bool CAUSAL, bool DROP, bool BMASK>
 __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_constant__ FwdParams p) {
   static_assert(!(DROP && BMASK), "dropout and block masks are not combined");
@@ -363,9 +356,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
     // If none did (the common case) those exponentials stand: P of keys 0-63
     // goes to tensor memory and is handed to the MMA warp, then keys 64-127.
     // Otherwise the tile is redone from tensor memory against the moved
-    // reference, after O and l are rescaled.  In unmasked tiles kPolyPairs of
-    // every 8 pairs of exponentials run on the FMA pipe (exp2_poly2), the
-    // rest on the MUFU unit.
+    // reference, after O and l are rescaled.
     auto load_s = [&](int kblock, uint32_t* s) {
       tmem_ld32(tm_S + 0, s);
       tmem_ld32(tm_S + 32, s + 32);
@@ -394,19 +385,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
     };
     // P of the 32 keys 32*q4 .. +31 against the reference -m (nm2), packed to
     // 16 bits in pk[16]; the unrounded values are summed into acc.
-    auto p_chunk = [&](auto poly_tag, const uint32_t* s, int q4, uint64_t nm2, int kv0, uint32_t* pk,
-                       uint64_t* acc) {
-      constexpr bool kPoly = decltype(poly_tag)::value;
+    auto p_chunk = [&](const uint32_t* s, int q4, uint64_t nm2, int kv0, uint32_t* pk, uint64_t* acc) {
       [[maybe_unused]] uint32_t kw[4] = {0, 0, 0, 0};  // dropout bytes: keys 4g..4g+3 of 16 in kw[g]
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         const int c = q4 * 32 + 2 * i;
         const uint64_t x = fma2(f2pack(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), c2, nm2);
-        uint64_t pp;
-        if (!DROP && kPoly && (i & 7) < kPolyPairs)
-          pp = exp2_poly2(x);
-        else
-          pp = f2pack(ex2_approx(f2lo(x)), ex2_approx(f2hi(x)));
+        const uint64_t pp = f2pack(ex2_approx(f2lo(x)), ex2_approx(f2hi(x)));
         acc[i & 3] = add2(acc[i & 3], pp);  // l sums the undropped P
         if constexpr (DROP) {
           if ((i & 7) == 0) {
@@ -462,7 +447,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
       float m_new;
       {
         uint32_t s[128];
-        const bool masked = load_s(kb, s);
+        load_s(kb, s);
         // row max, eight independent chains of three-input maxima: chain i
         // takes columns i, i + 8, ..., i + 120
         float mx[8];
@@ -478,26 +463,22 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
           // speculative: keys 0-63 against the current reference
           const float m_use = m_ref == -INFINITY ? 0.f : m_ref;
           const uint64_t nm2 = f2pack(-m_use, -m_use);
-          auto spec = [&](auto poly_tag) -> bool {
-            uint32_t pk0[16], pk1[16];
-            uint64_t acc[4] = {0, 0, 0, 0};
-            p_chunk(poly_tag, s, 0, nm2, kv0, pk0, acc);
-            p_chunk(poly_tag, s, 1, nm2, kv0, pk1, acc);
-            if (__any_sync(0xffffffffu, m_new > m_ref + 8.0f)) return false;
+          uint32_t pk0[16], pk1[16];
+          uint64_t acc[4] = {0, 0, 0, 0};
+          p_chunk(s, 0, nm2, kv0, pk0, acc);
+          p_chunk(s, 1, nm2, kv0, pk1, acc);
+          if (!__any_sync(0xffffffffu, m_new > m_ref + 8.0f)) {
             tmem_st16(tm_S + 0, pk0);
             tmem_st16(tm_S + 16, pk1);
             hand_over(0);
-            p_chunk(poly_tag, s, 2, nm2, kv0, pk0, acc);
+            p_chunk(s, 2, nm2, kv0, pk0, acc);
             tmem_st16(tm_S + 32, pk0);
-            p_chunk(poly_tag, s, 3, nm2, kv0, pk1, acc);
+            p_chunk(s, 3, nm2, kv0, pk1, acc);
             tmem_st16(tm_S + 48, pk1);
             l_sum += sum_acc(acc);
             hand_over(1);
-            return true;
-          };
-          // exponentials on the FMA pipe need finite arguments: masked
-          // tiles stay on the MUFU unit
-          done = masked ? spec(std::false_type{}) : spec(std::true_type{});
+            done = true;
+          }
         }
       }
       if (done) continue;
@@ -545,7 +526,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
           uint32_t pk[16];
-          p_chunk(std::false_type{}, s, q4, nm2, kv0, pk, acc);
+          p_chunk(s, q4, nm2, kv0, pk, acc);
           tmem_st16(tm_S + q4 * 16, pk);
           if (q4 == 1) hand_over(0);
         }

@@ -458,32 +458,6 @@ __device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
   return d;
 }
 
-// 2^x for a pair of fp32 values on the FMA and integer pipes instead of the
-// MUFU unit (which computes one exponential per lane every 8 cycles of a
-// sub-partition, as long as the tensor-core work of a 128 x 128 score tile
-// at d = 128).  Method: x = n + f with n = round(x) (the 1.5 * 2^23 shifter:
-// after t = x + 1.5 * 2^23 the integer n sits in the low bits of t) and
-// f = x - n in [-1/2, 1/2], exact; 2^f by a cubic fitted by the Remez
-// exchange for least maximum relative error on [-1/2, 1/2] (7.5e-5, below
-// the 2^-9 / 2^-12 rounding of the probabilities to bf16 / fp16); 2^n is
-// added to the exponent field (t << 23 is n << 23 modulo 2^32, since the
-// shifter's bits end in nine zeros).  x is clamped at -125 so that n + the
-// exponent of 2^f stays above zero; any x up to 127 is exact in range.
-__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x) {
-  const float lo = fmaxf(__uint_as_float(static_cast<uint32_t>(x)), -125.0f);
-  const float hi = fmaxf(__uint_as_float(static_cast<uint32_t>(x >> 32)), -125.0f);
-  const uint64_t xc = f2pack(lo, hi);
-  const uint64_t t = add2(xc, f2pack(12582912.0f, 12582912.0f));  // 1.5 * 2^23 + n
-  const uint64_t n = add2(t, f2pack(-12582912.0f, -12582912.0f));  // n, exact
-  const uint64_t f = fma2(n, f2pack(-1.0f, -1.0f), xc);            // x - n, exact
-  uint64_t p = fma2(f, f2pack(0.0551716685f, 0.0551716685f), f2pack(0.2426111251f, 0.2426111251f));
-  p = fma2(p, f, f2pack(0.6932609677f, 0.6932609677f));
-  p = fma2(p, f, f2pack(0.9999280572f, 0.9999280572f));
-  const uint32_t rlo = static_cast<uint32_t>(p) + (static_cast<uint32_t>(t) << 23);
-  const uint32_t rhi = static_cast<uint32_t>(p >> 32) + (static_cast<uint32_t>(t >> 32) << 23);
-  return (static_cast<uint64_t>(rhi) << 32) | rlo;
-}
-
 // Philox4x32-10 (Salmon, Moraes, Dror and Shaw, "Parallel random numbers: as
 // easy as 1, 2, 3", SC 2011): ten rounds of two 32 x 32 -> 64-bit products of
 // counter words 0 and 2 with the round multipliers, mixed with the other

@@ -27,8 +27,9 @@ def test_window_flops_count_visible_pairs(N, W):
 
 
 def splits(B, Hkv, max_pages):
-    want = math.ceil(2 * 148 / (B * Hkv))
-    return max(1, min(want, max_pages))
+    # four waves of two blocks per SM of a 148-SM B200, at least 4 pages a split
+    want = math.ceil(4 * 2 * 148 / (B * Hkv))
+    return max(1, min(want, max(1, max_pages // 4)))
 
 
 @pytest.mark.parametrize("B,Hq,Hkv,Nq,d,max_pages", [
