@@ -652,8 +652,6 @@ fa_status_t fa_decode_paged(const void* q, const void* k_cache, const void* v_ca
   fa::DecodeParams prm;
   std::memset(&prm, 0, sizeof(prm));
   prm.q = q;
-  prm.kc = k_cache;
-  prm.vc = v_cache;
   prm.table = block_table;
   prm.lens = seq_lens;
   prm.o = o;
@@ -665,8 +663,17 @@ fa_status_t fa_decode_paged(const void* q, const void* k_cache, const void* v_ca
   prm.P = page_size;
   prm.max_pages = max_pages;
   prm.num_pages = num_pages;
-  prm.S = fa::decode_splits(B, Hkv, max_pages);
-  prm.pages_per_split = (max_pages + prm.S - 1) / prm.S;
+  // the caches as [num_pages * Hkv][P][d]: one box = 64 features of the P
+  // rows of one (page, kv head)
+  if (static_cast<int64_t>(num_pages) * Hkv > INT32_MAX) return FA_ERR_UNSUPPORTED;
+  const CUtensorMapDataType tdt = dtype == FA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  if (!make_map(&prm.tm_k, k_cache, tdt, 2, d, page_size, static_cast<uint64_t>(num_pages) * Hkv, 64, page_size) ||
+      !make_map(&prm.tm_v, v_cache, tdt, 2, d, page_size, static_cast<uint64_t>(num_pages) * Hkv, 64, page_size))
+    return FA_ERR_CUDA;
+  prm.S = fa::decode_splits(B, Hkv, d, max_pages);
+  // a split holds whole tiles of 128 keys
+  const int ppt = fa::kDecodeTile / page_size;
+  prm.pages_per_split = ((max_pages + prm.S - 1) / prm.S + ppt - 1) / ppt * ppt;
   prm.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   const int64_t rows = static_cast<int64_t>(B) * Hq * Nq;
   prm.part_o = static_cast<float*>(workspace);
@@ -674,12 +681,8 @@ fa_status_t fa_decode_paged(const void* q, const void* k_cache, const void* v_ca
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const bool bf = dtype == FA_BF16;
   const dim3 grid(static_cast<unsigned>(prm.S), static_cast<unsigned>(Hkv), static_cast<unsigned>(B));
-  // the kernels are opted in once for the largest page size; a launch uses
-  // the bytes of its own page size
-  const int smem_max = d == 128 ? fa::DecodeLayout<128>(fa::kDecodeMaxPage, fa::kDecodeMaxRows).bytes
-                                : fa::DecodeLayout<64>(fa::kDecodeMaxPage, fa::kDecodeMaxRows).bytes;
   auto run = [&](auto split_kern, auto merge_kern, int smem) -> fa_status_t {
-    fa_status_t r = opt_in_smem(split_kern, smem_max);
+    fa_status_t r = opt_in_smem(split_kern, smem);
     if (r != FA_OK) return r;
     split_kern<<<grid, fa::kDecodeThreads, smem, st>>>(prm);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
@@ -688,10 +691,9 @@ fa_status_t fa_decode_paged(const void* q, const void* k_cache, const void* v_ca
   };
   const int R = (Hq / Hkv) * Nq;
   const int rb = R <= 4 ? 4 : R <= 8 ? 8 : R <= 16 ? 16 : 32;
-  const int smem = d == 128 ? fa::DecodeLayout<128>(page_size, rb).bytes
-                            : fa::DecodeLayout<64>(page_size, rb).bytes;
-#define FA_DECODE_RUN(HD, BFV, RBV) \
-  run(fa::fa_decode_split_kernel<HD, BFV, RBV>, fa::fa_decode_merge_kernel<HD, BFV>, smem)
+#define FA_DECODE_RUN(HD, BFV, RBV)                                                                  \
+  run(fa::fa_decode_split_kernel<HD, BFV, RBV>, fa::fa_decode_merge_kernel<HD, BFV>, \
+      fa::DecodeLayout<HD, RBV>::kDynSmem)
 #define FA_DECODE_RB(HD, BFV)                                                        \
   (rb == 4 ? FA_DECODE_RUN(HD, BFV, 4) : rb == 8 ? FA_DECODE_RUN(HD, BFV, 8)        \
              : rb == 16 ? FA_DECODE_RUN(HD, BFV, 16) : FA_DECODE_RUN(HD, BFV, 32))

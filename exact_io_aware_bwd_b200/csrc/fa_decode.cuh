@@ -14,19 +14,25 @@
 // The work is bound by memory (each cached byte is read once, a handful of
 // flops per byte), so it is split along the cache: a block takes one split
 // of the pages of one (sequence, kv head), keeps an online softmax over it
-// and writes its unnormalised O with the row max m and sum l (base 2); a
-// second kernel merges the splits: m* = max m_s, l* = sum l_s 2^(m_s - m*),
-// O = sum O_s 2^(m_s - m*) / l*, lse = ln 2 (m* + log2 l*).
+// and writes its unnormalised O with the row reference max m and sum l
+// (base 2); a second kernel merges the splits: m* = max m_s, l* = sum l_s
+// 2^(m_s - m*), O = sum O_s 2^(m_s - m*) / l*, lse = ln 2 (m* + log2 l*).
 //
-// Inside a block (128 threads) pages are staged in shared memory by bulk
-// copies (cp.async.bulk, the copy engine; completion counted in bytes on an
-// mbarrier) into a ring of kStages page slots, so that several pages are in
-// flight while one is used: warp 0 issues a page's copies (one per K row,
-// into rows padded by 16 bytes so that one thread per key reads its row
-// without bank conflicts, and one for the whole V page) and refills a slot
-// as soon as every thread is done with it.  Scores take all 128 threads
-// (128 / P threads per key, combined by shuffles), the softmax update one
-// warp per row, and P V one thread per output column.
+// Inside a block the cache is walked in tiles of 128 keys (128 / P pages):
+//   warp 4     TMA loads of each page's K and V rows (two 128-byte-swizzled
+//              boxes of 64 features per page at d = 128) into a ring of
+//              tile slots; a page outside the sequence or with a bad table
+//              entry is loaded from outside the tensor (zeros) and hidden;
+//   warp 5     tcgen05.mma, one elected lane: S^T = K Q^T (M = 128 keys,
+//              N = the rows padded to 16 or 32, K = d) into tensor memory,
+//              then O^T += V^T P^T (M = d, N = rows, K = 128 keys), V read
+//              MN-major straight from its [key][d] rows;
+//   warps 0-3  one thread per key (its tensor-memory lane): scores of the R
+//              rows, the online-softmax reference max, the probabilities
+//              written to shared memory as the B operand of the P V product.
+// The reference max of a row moves only when a tile's scores exceed it by
+// more than 8 (log2), so the running O^T is rescaled in tensor memory only
+// then (exact: O and l share the reference).
 #pragma once
 
 #include <type_traits>
@@ -38,14 +44,16 @@ namespace fa {
 constexpr uint32_t kKernDecode = 10;
 constexpr uint32_t kKernDecodeMerge = 11;
 constexpr uint32_t kStatusBadInput = 7;  // a block-table entry or sequence length out of range
-constexpr int kDecodeThreads = 128;
+constexpr int kDecodeThreads = 192;      // softmax warps 0-3, TMA warp 4, MMA warp 5
 constexpr int kDecodeMaxRows = 32;
 constexpr int kDecodeMaxPage = 128;
+constexpr int kDecodeTile = 128;         // keys per tile: the M of S^T = K Q^T
+constexpr int kDecodeSMs = 148;          // B200
 
 struct DecodeParams {
+  CUtensorMap tm_k;       // K cache as [num_pages * Hkv][P][d], box 64 features x P rows
+  CUtensorMap tm_v;       // V cache, the same
   const void* q;          // [B][Hq][Nq][d]
-  const void* kc;         // [num_pages][Hkv][P][d]
-  const void* vc;
   const int* table;       // [B][max_pages]
   const int* lens;        // [B]
   float* part_o;          // [B][Hq][Nq][S][d]   unnormalised partial outputs
@@ -56,259 +64,425 @@ struct DecodeParams {
   float scale_log2;
 };
 
-// Page slots of the ring for page size P and row bound RB: as many as fit
-// in about 100 KB (two blocks per SM), at least 2 and at most 8.
-template <int HD>
-__host__ __device__ inline int decode_stages(int P, int rb) {
-  const int slot = P * (HD * 2 + 16) + P * HD * 2;
-  const int fixed = rb * HD * 4 + rb * P * 4 + 3 * kDecodeMaxRows * 4 + 8 * 8;
-  int st = (100 * 1024 - fixed) / slot;
-  return st < 2 ? 2 : (st > 8 ? 8 : st);
-}
-
-// Splits of each (sequence, kv head): enough blocks for four full waves of
-// two blocks per SM of a full B200, at least 4 pages a split.
-__host__ __device__ inline int decode_splits(int B, int Hkv, int max_pages) {
-  const int bh = B * Hkv > 0 ? B * Hkv : 1;
-  int want = (4 * 2 * 148 + bh - 1) / bh;
-  const int cap = max_pages / 4 > 1 ? max_pages / 4 : 1;
-  want = want > cap ? cap : want;
-  return want < 1 ? 1 : want;
+// Splits of each (sequence, kv head), for a grid of B * Hkv * S blocks: at
+// least four waves of the blocks that fit on a B200 at once (one per SM at
+// d = 128, two at d = 64); among S0 .. 2 S0 the count whose last wave is the
+// fullest; at least 4 pages a split.
+inline int decode_splits(int B, int Hkv, int d, int max_pages) {
+  const int64_t bh = static_cast<int64_t>(B) * Hkv > 0 ? static_cast<int64_t>(B) * Hkv : 1;
+  const int64_t slots = kDecodeSMs * (d == 64 ? 2 : 1);
+  const int64_t s0 = (4 * slots + bh - 1) / bh;
+  const int64_t cap = max_pages / 4 > 1 ? max_pages / 4 : 1;
+  int64_t best = s0 < cap ? s0 : cap;
+  double best_eff = -1.0;
+  for (int64_t s = s0; s <= 2 * s0 && s <= cap; ++s) {
+    const int64_t blocks = bh * s;
+    const int64_t waves = (blocks + slots - 1) / slots;
+    const double eff = static_cast<double>(blocks) / static_cast<double>(waves * slots);
+    if (eff > best_eff + 1e-9) {
+      best = s;
+      best_eff = eff;
+    }
+  }
+  return static_cast<int>(best < 1 ? 1 : best);
 }
 
 inline size_t decode_workspace_bytes(int B, int Hq, int Hkv, int Nq, int d, int max_pages) {
-  const int64_t S = decode_splits(B, Hkv, max_pages);
+  const int64_t S = decode_splits(B, Hkv, d, max_pages);
   const int64_t rows = static_cast<int64_t>(B) * Hq * Nq * S;
   return static_cast<size_t>(rows) * 4u * static_cast<size_t>(d + 2);
 }
 
-// Shared memory for page size P, row bound RB and the ring's slots (bytes,
-// all offsets multiples of 16): the slots' K (padded rows) and V pages,
-// fp32 queries [RB][HD], fp32 scores [RB][P], row state, slot barriers.
-// Sized by RB and P so that two blocks fit on an SM.
-template <int HD>
+// Shared memory of the split kernel for head dimension HD and row bound RB
+// (offsets from a 1024-byte-aligned base).
+template <int HD, int RB>
 struct DecodeLayout {
-  static constexpr int kKRow = HD * 2 + 16;  // padded K row, bytes
-  int P, stages, off_k, off_v, off_q, off_s, off_row, off_bar, bytes;
-  __host__ __device__ DecodeLayout(int page, int rb) : P(page) {
-    stages = decode_stages<HD>(page, rb);
-    const int kbuf = page * kKRow, vbuf = page * HD * 2;
-    off_k = 0;                                   // K slots
-    off_v = stages * kbuf;                       // V slots
-    off_q = off_v + stages * vbuf;
-    off_s = off_q + rb * HD * 4;
-    off_row = off_s + rb * page * 4;
-    off_bar = off_row + 3 * kDecodeMaxRows * 4;
-    bytes = off_bar + 8 * 8;
-  }
+  static constexpr int NP = RB < 16 ? 16 : RB;           // MMA N: rows padded to 16 or 32
+  static constexpr int kChunks = HD / 64;                // 64-feature boxes per row
+  static constexpr int kChunkBytes = kDecodeTile * 128;  // 128 keys x 128 bytes
+  // a slot: the V chunks, then the K chunks (at d = 64 the unused upper half
+  // of the product V^T P^T reads the K chunk that follows: finite data)
+  static constexpr int kSlotBytes = 2 * kChunks * kChunkBytes;
+  static constexpr int kSlots = 3;
+  static constexpr int kQChunk = NP * 128;               // Q rows of one feature box
+  static constexpr int kPChunk = NP * 128;               // P rows of 64 keys
+  static constexpr int kPBytes = 2 * kPChunk;            // one buffer: 128 keys
+  static constexpr int kOffQ = kSlots * kSlotBytes;
+  static constexpr int kOffP = kOffQ + kChunks * kQChunk;
+  static constexpr int kOffFlag = kOffP + 2 * kPBytes;   // int [2][4]
+  static constexpr int kOffMax = kOffFlag + 8 * 4;       // float [2][4][32]
+  static constexpr int kOffSum = kOffMax + 2 * 4 * 32 * 4;  // float [4][32]
+  static constexpr int kOffBar = kOffSum + 4 * 32 * 4;
+  // kv_full[slots], kv_empty[slots], s_full[2], p_full[2], pv_done[2], done
+  static constexpr int kNumBars = 2 * kSlots + 7;
+  static constexpr int kOffTmemPtr = kOffBar + kNumBars * 8;
+  static constexpr int kOffAbort = kOffTmemPtr + 4;
+  static constexpr int kBytes = kOffAbort + 4;
+  static constexpr int kDynSmem = kBytes + 1024;         // room to align the base
+  static_assert(kOffQ % 1024 == 0 && kOffP % 1024 == 0 && kQChunk % 1024 == 0, "swizzle atoms");
+  static_assert(kDynSmem <= 232448, "shared memory budget");
 };
+
+// tensor memory <-> registers, 32 lanes x N 32-bit columns (N = 4 .. 32)
+template <int N>
+__device__ __forceinline__ void tmem_ld_n(uint32_t taddr, uint32_t* r) {
+  if constexpr (N == 4) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(taddr));
+  } else if constexpr (N == 8) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                   "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr));
+  } else if constexpr (N == 16) {
+    tmem_ld16(taddr, r);
+  } else {
+    static_assert(N == 32, "column count");
+    tmem_ld32(taddr, r);
+  }
+}
+
+template <int N>
+__device__ __forceinline__ void tmem_st_n(uint32_t taddr, const uint32_t* r) {
+  if constexpr (N == 4) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1,%2,%3,%4};" ::"r"(taddr),
+                 "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3])
+                 : "memory");
+  } else if constexpr (N == 8) {
+    tmem_st8(taddr, r);
+  } else if constexpr (N == 16) {
+    tmem_st16(taddr, r);
+  } else {
+    static_assert(N == 32, "column count");
+    tmem_st16(taddr, r);
+    tmem_st16(taddr + 16, r + 16);
+  }
+}
 
 // RB: compile-time bound on the rows (4, 8, 16 or 32, the smallest >= R), so
 // the per-row loops unroll to the rows that exist.
 template <int HD, bool BF16, int RB>
-__global__ void __launch_bounds__(kDecodeThreads) fa_decode_split_kernel(const __grid_constant__ DecodeParams p) {
+__global__ void __launch_bounds__(kDecodeThreads, 1) fa_decode_split_kernel(const __grid_constant__ DecodeParams p) {
   using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
-  const DecodeLayout<HD> lay(p.P, RB);
-  constexpr int kKRow = DecodeLayout<HD>::kKRow;
-  extern __shared__ __align__(16) uint8_t smem[];
-  float* sQ = reinterpret_cast<float*>(smem + lay.off_q);
-  float* sS = reinterpret_cast<float*>(smem + lay.off_s);
-  float* sM = reinterpret_cast<float*>(smem + lay.off_row);
-  float* sL = sM + kDecodeMaxRows;
-  float* sC = sL + kDecodeMaxRows;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + lay.off_bar);  // [stages]
-  __shared__ int abort_flag;
+  using L = DecodeLayout<HD, RB>;
+  constexpr int NP = L::NP;
+  constexpr int NS = L::kSlots;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                           ~static_cast<uintptr_t>(1023));
+  uint8_t* sQ = sm + L::kOffQ;
+  uint8_t* sP = sm + L::kOffP;
+  volatile int* sFlag = reinterpret_cast<volatile int*>(sm + L::kOffFlag);
+  float* sMax = reinterpret_cast<float*>(sm + L::kOffMax);
+  float* sSum = reinterpret_cast<float*>(sm + L::kOffSum);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::kOffBar);
+  uint64_t* kv_full = bars;
+  uint64_t* kv_empty = kv_full + NS;
+  uint64_t* s_full = kv_empty + NS;
+  uint64_t* p_full = s_full + 2;
+  uint64_t* pv_done = p_full + 2;
+  uint64_t* done_bar = pv_done + 2;
+  uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(sm + L::kOffTmemPtr);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::kOffAbort);
 
   const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int G = p.Hq / p.Hkv, R = G * p.Nq, P = p.P, NS = lay.stages;
+  const int G = p.Hq / p.Hkv, R = G * p.Nq, P = p.P;
+  const int ppt = kDecodeTile / P;  // pages per tile
   const int Lb = p.lens[b];
   const bool len_ok = Lb >= p.Nq && Lb <= p.max_pages * P;
   if (!len_ok && split == 0 && g == 0 && tid == 0) record_error(kStatusBadInput, kKernDecode, 0, 0);
   const int n_pages = len_ok ? (Lb + P - 1) / P : 0;
-  const int pg0 = split * p.pages_per_split;
+  const int pg0 = split * p.pages_per_split;  // pages_per_split is a multiple of ppt
   const int pg1 = min(n_pages, pg0 + p.pages_per_split);
+  const int n_tiles = pg1 > pg0 ? (pg1 - pg0 + ppt - 1) / ppt : 0;  // tiles of this split
 
   if (tid == 0) {
-    for (int i = 0; i < NS; ++i) mbar_init(&full[i], 1);
-    abort_flag = 0;
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], 128);
+      mbar_init(&pv_done[i], 1);
+    }
+    mbar_init(done_bar, 1);
+    *abort_flag = 0;
     fence_mbar_init();
   }
-  // queries of the block's rows (row r: head g*G + r / Nq, token r % Nq),
-  // fp32 and scaled by scale * log2(e)
-  for (int i = tid; i < R * HD; i += kDecodeThreads) {
-    const int r = i / HD, c = i % HD;
-    const int h = g * G + r / p.Nq, t = r % p.Nq;
-    const T* qr = reinterpret_cast<const T*>(p.q) + ((static_cast<size_t>(b) * p.Hq + h) * p.Nq + t) * HD;
-    sQ[i] = static_cast<float>(qr[c]) * p.scale_log2;
+  if (warp == 0) {
+    tmem_alloc(tmem_ptr, 128);
+    tmem_relinquish();
   }
-  if (tid < kDecodeMaxRows) {
-    sM[tid] = -INFINITY;
-    sL[tid] = 0.f;
+  // Q rows of the block (row r: head g*G + r / Nq, token r % Nq) into the
+  // K-major, 128-byte-swizzled B operand of S^T = K Q^T; padding rows are
+  // zero.
+  for (int i = tid; i < NP * (HD / 8); i += kDecodeThreads) {
+    const int r = i / (HD / 8), c16 = i % (HD / 8);
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (r < R) {
+      const int h = g * G + r / p.Nq, t = r % p.Nq;
+      const T* qr = reinterpret_cast<const T*>(p.q) + ((static_cast<size_t>(b) * p.Hq + h) * p.Nq + t) * HD;
+      v = *reinterpret_cast<const uint4*>(qr + c16 * 8);
+    }
+    *reinterpret_cast<uint4*>(sQ + (c16 >> 3) * L::kQChunk + r * 128 + (((c16 & 7) ^ (r & 7)) << 4)) = v;
   }
-  float acc[RB];  // thread c < HD: output column c of every row
-#pragma unroll
-  for (int r = 0; r < RB; ++r) acc[r] = 0.f;
+  fence_proxy_async_smem();
+  tc_fence_before();
   __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_ptr;
+  const uint32_t tm_O = tmem + 2 * NP;  // O^T: lanes = features, columns = rows
 
-  // page pg -> slot (pg - pg0) % NS; a bad page id is recorded and its keys
-  // treated as hidden: nothing is read for it and the slot's barrier is
-  // completed by a plain arrival.  Issued by warp 0.
-  auto page_id = [&](int pg) { return p.table[static_cast<size_t>(b) * p.max_pages + pg]; };
-  auto issue = [&](int pg) {
-    const int phys = page_id(pg);
-    const int slot = (pg - pg0) % NS;
-    uint64_t* bar = &full[slot];
-    const bool good = phys >= 0 && phys < p.num_pages;
+  if (warp == 4) {
+    // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      if (good)
-        mbar_expect_tx(bar, static_cast<uint32_t>(2 * P * HD * 2));
-      else
-        mbar_arrive(bar);
+      prefetch_tensormap(&p.tm_k);
+      prefetch_tensormap(&p.tm_v);
+      int issued = 0;
+      for (int j = 0; j < n_tiles; ++j) {
+        const int s = j % NS;
+        if (j >= NS && !mbar_wait(&kv_empty[s], ((j / NS) - 1) & 1, abort_flag, kKernDecode, 4, 0)) break;
+        mbar_expect_tx(&kv_full[s], static_cast<uint32_t>(L::kSlotBytes));
+        uint8_t* slot = sm + s * L::kSlotBytes;
+        for (int pp = 0; pp < ppt; ++pp) {
+          const int pg = pg0 + j * ppt + pp;
+          int outer = -1;  // outside the tensor: the box reads as zeros
+          if (pg < pg1) {
+            const int phys = p.table[static_cast<size_t>(b) * p.max_pages + pg];
+            if (phys >= 0 && phys < p.num_pages)
+              outer = phys * p.Hkv + g;
+            else
+              record_error(kStatusBadInput, kKernDecode, 4, 1);
+          }
+#pragma unroll
+          for (int c = 0; c < L::kChunks; ++c) {
+            tma_load_3d(slot + c * L::kChunkBytes + pp * P * 128, &p.tm_v, &kv_full[s], c * 64, 0, outer);
+            tma_load_3d(slot + (L::kChunks + c) * L::kChunkBytes + pp * P * 128, &p.tm_k, &kv_full[s], c * 64,
+                        0, outer);
+          }
+        }
+        issued = j + 1;
+      }
+      // the copies of the last tile issued into each slot land before the
+      // block exits (all earlier ones were waited for by the MMA warp)
+      for (int j = issued > NS ? issued - NS : 0; j < issued; ++j)
+        mbar_wait_drain(&kv_full[j % NS], (j / NS) & 1, kKernDecode, 4, 2);
     }
-    __syncwarp();
-    if (!good) return;
-    uint8_t* sKb = smem + lay.off_k + slot * P * kKRow;
-    uint8_t* sVb = smem + lay.off_v + slot * P * HD * 2;
-    const size_t base = (static_cast<size_t>(phys) * p.Hkv + g) * P * HD;
-    const uint8_t* kg = reinterpret_cast<const uint8_t*>(reinterpret_cast<const T*>(p.kc) + base);
-    const uint8_t* vg = reinterpret_cast<const uint8_t*>(reinterpret_cast<const T*>(p.vc) + base);
-    for (int j = lane; j < P; j += 32) bulk_load(sKb + j * kKRow, kg + static_cast<size_t>(j) * HD * 2, HD * 2, bar);
-    if (lane == 0) bulk_load(sVb, vg, static_cast<uint32_t>(P * HD * 2), bar);
-  };
-  int issued = pg0;  // pages whose copies warp 0 has issued: [pg0, issued)
-  if (warp == 0)
-    for (; issued < pg1 && issued < pg0 + NS; ++issued) issue(issued);
-  int consumed = pg0;  // pages fully used: [pg0, consumed); consumed <= issued
-  for (int pg = pg0; pg < pg1; ++pg) {
-    const int slot = (pg - pg0) % NS;
-    const bool ok = mbar_wait(&full[slot], ((pg - pg0) / NS) & 1, &abort_flag, kKernDecode, 0, 1);
-    if (__syncthreads_or(!ok)) break;
-    const int phys = page_id(pg);
-    const bool page_ok = phys >= 0 && phys < p.num_pages;
-    if (!page_ok && tid == 0) record_error(kStatusBadInput, kKernDecode, 1, 0);
-    const uint8_t* sK = smem + lay.off_k + slot * P * kKRow;
-    const T* sV = reinterpret_cast<const T*>(smem + lay.off_v + slot * P * HD * 2);
-    // scores: tpk = 128 / P threads per key, each over d / tpk features,
-    // summed across the key's threads by shuffles; s[r][j] = q_r . k_j (log2
-    // units), -inf where hidden (after the query, past the sequence, or a
-    // bad page)
-    {
-      const int tpk = kDecodeThreads / P;          // 1, 2, 4 or 8 (P = 128 .. 16)
-      const int j = tid / tpk, part = tid % tpk;   // the threads of a key are adjacent lanes
-      const int n8 = HD / 8 / tpk;                 // 16-byte chunks per thread
-      const int key = pg * P + j;
-      float s[RB];
+  } else if (warp == 5) {
+    // ------------------------------------------------------------ MMA issuer
+    constexpr uint32_t kIdS = idesc_f16(BF16, 128, NP, false, false);  // S^T = K Q^T
+    constexpr uint32_t kIdO = idesc_f16(BF16, 128, NP, true, false);   // O^T += V^T P^T
+    const uint64_t dK = sdesc_sw128(smem_u32(sm) + L::kChunks * L::kChunkBytes, 16, 1024);  // slot 0 K
+    const uint64_t dVt = sdesc_sw128(smem_u32(sm), L::kChunkBytes, 1024);  // slot 0 V, MN-major
+    const uint64_t dQ = sdesc_sw128(smem_u32(sQ), 16, 1024);
+    const uint64_t dP = sdesc_sw128(smem_u32(sP), 16, 1024);
+    auto wait_all = [&](uint64_t* bar, uint32_t parity, uint32_t site) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, kKernDecode, 5, site));
+    };
+    auto issue_pv = [&](int t) -> bool {
+      if (!wait_all(&p_full[t & 1], (t >> 1) & 1, 1)) return false;
+      tc_fence_after();
+      const uint32_t so = (t % NS) * L::kSlotBytes, po = (t & 1) * L::kPBytes;
 #pragma unroll
-      for (int r = 0; r < RB; ++r) s[r] = 0.f;
-      const uint8_t* kr = sK + j * kKRow;
-      for (int c = 0; c < n8; ++c) {
-        const int c8 = part * n8 + c;
-        const uint4 kv = *reinterpret_cast<const uint4*>(kr + c8 * 16);
-        const T* k8 = reinterpret_cast<const T*>(&kv);
-        float kf[8];
+      for (int k = 0; k < kDecodeTile / 16; ++k)
+        umma_ss_w(tm_O, sdesc_add(dVt, so + k * 2048), sdesc_add(dP, po + (k >> 2) * L::kPChunk + (k & 3) * 32),
+                  kIdO, (t > 0 || k > 0) ? 1u : 0u);
+      umma_commit_w(&kv_empty[t % NS]);
+      umma_commit_w(&pv_done[t & 1]);
+      return true;
+    };
+    bool ok = true;
+    for (int j = 0; ok && j < n_tiles; ++j) {
+      const int s = j % NS;
+      if (!(ok = wait_all(&kv_full[s], (j / NS) & 1, 0))) break;
+      tc_fence_after();
+      const uint32_t so = s * L::kSlotBytes;
+      // S^T_j lands in buffer j % 2, last read by the softmax of tile j - 2,
+      // whose P the PV product issued before this one waited for
 #pragma unroll
-        for (int e = 0; e < 8; ++e) kf[e] = static_cast<float>(k8[e]);
+      for (int k = 0; k < HD / 16; ++k)
+        umma_ss_w(tmem + (j & 1) * NP, sdesc_add(dK, so + (k >> 2) * L::kChunkBytes + (k & 3) * 32),
+                  sdesc_add(dQ, (k >> 2) * L::kQChunk + (k & 3) * 32), kIdS, k > 0 ? 1u : 0u);
+      umma_commit_w(&s_full[j & 1]);
+      if (j > 0) ok = issue_pv(j - 1);
+    }
+    if (ok && n_tiles > 0) issue_pv(n_tiles - 1);
+    // every MMA this warp issued completes before tensor memory is freed
+    umma_commit_w(done_bar);
+    mbar_wait_drain(done_bar, 0, kKernDecode, 5, 3);
+  } else {
+    // ------------------------------------------------------------ softmax (warps 0-3)
+    // Thread i owns key i of every tile (tensor-memory lane i of S^T) and,
+    // for the rescales and the epilogue, feature i of O^T.
+    const int i = tid;
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const float c_log2 = p.scale_log2;
+    float ref[RB], lp[RB];
+#pragma unroll
+    for (int r = 0; r < RB; ++r) {
+      ref[r] = -INFINITY;
+      lp[r] = 0.f;
+    }
+    // whether this thread's key of tile jj sits in a page that was loaded
+    auto page_loaded = [&](int jj) -> bool {
+      const int pg = pg0 + jj * ppt + i / P;
+      if (pg >= pg1) return false;
+      const int phys = __ldg(p.table + static_cast<size_t>(b) * p.max_pages + pg);
+      return phys >= 0 && phys < p.num_pages;
+    };
+    bool loaded_next = n_tiles > 0 ? page_loaded(0) : false;
+    bool ok = true;
+    for (int j = 0; j < n_tiles; ++j) {
+      const int buf = j & 1;
+      const bool loaded = loaded_next;
+      if (j + 1 < n_tiles) loaded_next = page_loaded(j + 1);
+      // warp-uniform, as the tensor-memory loads below must be
+      const bool fail = !__all_sync(0xffffffffu, mbar_wait(&s_full[buf], (j >> 1) & 1, abort_flag, kKernDecode, 0, 0));
+      tc_fence_after();
+      uint32_t sv[RB];
+      if (!fail) {
+        tmem_ld_n<RB>(tmem + buf * NP + lane_off, sv);
+        tmem_ld_wait();
+      }
+      const int key = (pg0 + j * ppt) * P + i;
+      float t[RB];
+      bool need = false;
+#pragma unroll
+      for (int r = 0; r < RB; ++r) {
+        t[r] = -INFINITY;
+        if (r < R && !fail) {
+          const bool vis = loaded && key <= Lb - p.Nq + r % p.Nq;
+          t[r] = vis ? __uint_as_float(sv[r]) * c_log2 : -INFINITY;
+          need |= t[r] > ref[r] + 8.f;
+        }
+      }
+      // One decision for all 128 threads: whether a reference max moves (and
+      // whether a wait failed).  Every softmax thread reaches every barrier.
+      const bool wneed = __any_sync(0xffffffffu, need), wfail = __any_sync(0xffffffffu, fail);
+      if (lane == 0) sFlag[buf * 4 + warp] = (wneed ? 1 : 0) | (wfail ? 2 : 0);
+      named_barrier_sync(1, 128);
+      const int f = sFlag[buf * 4 + 0] | sFlag[buf * 4 + 1] | sFlag[buf * 4 + 2] | sFlag[buf * 4 + 3];
+      if (f & 2) {
+        ok = false;
+        break;
+      }
+      if (f & 1) {
+        // per-row maxima of the tile over the 128 keys
 #pragma unroll
         for (int r = 0; r < RB; ++r) {
           if (r < R) {
-            const float4 qa = *reinterpret_cast<const float4*>(sQ + r * HD + c8 * 8);
-            const float4 qb = *reinterpret_cast<const float4*>(sQ + r * HD + c8 * 8 + 4);
-            s[r] = fmaf(qa.x, kf[0], fmaf(qa.y, kf[1], fmaf(qa.z, kf[2], fmaf(qa.w, kf[3],
-                   fmaf(qb.x, kf[4], fmaf(qb.y, kf[5], fmaf(qb.z, kf[6], fmaf(qb.w, kf[7], s[r]))))))));
+            float m = t[r];
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+            if (lane == 0) sMax[(buf * 4 + warp) * 32 + r] = m;
           }
         }
-      }
-      for (int off = 1; off < tpk; off <<= 1) {
-#pragma unroll
-        for (int r = 0; r < RB; ++r) s[r] += __shfl_xor_sync(0xffffffffu, s[r], off);
-      }
-      if (part == 0) {
+        named_barrier_sync(1, 128);
+        float fac[RB];
 #pragma unroll
         for (int r = 0; r < RB; ++r) {
+          fac[r] = 1.f;
           if (r < R) {
-            const int t = r % p.Nq;
-            const bool vis = page_ok && key <= Lb - p.Nq + t;
-            sS[r * P + j] = vis ? s[r] : -INFINITY;
+            const float* mr = sMax + buf * 4 * 32 + r;
+            const float nm = fmaxf(fmaxf(ref[r], fmaxf(mr[0], mr[32])), fmaxf(mr[64], mr[96]));
+            if (nm != ref[r]) fac[r] = ref[r] == -INFINITY ? 0.f : ex2_approx(ref[r] - nm);
+            ref[r] = nm;
+            lp[r] *= fac[r];
+          }
+        }
+        // O^T holds the products of tiles 0 .. j-1: once they are complete,
+        // scale its row columns (this thread: feature lane i)
+        if (j > 0) {
+          if (__all_sync(0xffffffffu, mbar_wait(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, kKernDecode, 0, 1))) {
+            tc_fence_after();
+            uint32_t ov[RB];
+            tmem_ld_n<RB>(tm_O + lane_off, ov);
+            tmem_ld_wait();
+#pragma unroll
+            for (int r = 0; r < RB; ++r) ov[r] = __float_as_uint(__uint_as_float(ov[r]) * fac[r]);
+            tmem_st_n<RB>(tm_O + lane_off, ov);
+            tmem_st_wait();
           }
         }
       }
-    }
-    __syncthreads();
-    // online softmax update, one warp per row: new max, rescale factor, P
-    for (int r = warp; r < R; r += kDecodeThreads / 32) {
-      float* sr = sS + r * P;
-      float mx = -INFINITY;
-      for (int j = lane; j < P; j += 32) mx = fmaxf(mx, sr[j]);
+      // P of this thread's key for every row; buffer `buf` was last read by
+      // the PV product of tile j - 2
+      float pr[RB];
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-      const float m_old = sM[r];
-      const float m_new = fmaxf(m_old, mx);
-      const float m_use = m_new == -INFINITY ? 0.f : m_new;  // no visible key yet: P = 0
-      float sum = 0.f;
-      for (int j = lane; j < P; j += 32) {
-        const float e = ex2_approx(sr[j] - m_use);
-        sr[j] = e;
-        sum += e;
+      for (int r = 0; r < RB; ++r) {
+        pr[r] = 0.f;
+        if (r < R && t[r] != -INFINITY) {
+          pr[r] = ex2_approx(t[r] - ref[r]);
+          lp[r] += pr[r];
+        }
       }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-      __syncwarp();
-      if (lane == 0) {
-        const float corr = m_new == -INFINITY ? 1.f : ex2_approx(m_old - m_new);
-        sC[r] = corr;
-        sL[r] = sL[r] * corr + sum;
-        sM[r] = m_new;
-      }
-    }
-    __syncthreads();
-    // O += P V, one thread per output column
-    if (tid < HD) {
+      if (j >= 2) mbar_wait(&pv_done[buf], ((j - 2) >> 1) & 1, abort_flag, kKernDecode, 0, 2);
+      // P[row][key] in the K-major, 128-byte-swizzled B operand of V^T P^T:
+      // 64 keys (128 bytes) per row and box; the 32 lanes of a warp write 64
+      // consecutive bytes of one row at a time
+      uint8_t* pb = sP + buf * L::kPBytes + (i >> 6) * L::kPChunk + (i & 7) * 2;
 #pragma unroll
       for (int r = 0; r < RB; ++r)
-        if (r < R) acc[r] *= sC[r];
-      for (int j = 0; j < P; j += 4) {
-        const float v0 = static_cast<float>(sV[(j + 0) * HD + tid]);
-        const float v1 = static_cast<float>(sV[(j + 1) * HD + tid]);
-        const float v2 = static_cast<float>(sV[(j + 2) * HD + tid]);
-        const float v3 = static_cast<float>(sV[(j + 3) * HD + tid]);
-#pragma unroll
-        for (int r = 0; r < RB; ++r) {
-          if (r < R) {
-            const float4 pr = *reinterpret_cast<const float4*>(sS + r * P + j);
-            acc[r] = fmaf(pr.x, v0, fmaf(pr.y, v1, fmaf(pr.z, v2, fmaf(pr.w, v3, acc[r]))));
-          }
-        }
-      }
+        if (r < R) *reinterpret_cast<T*>(pb + r * 128 + ((((i & 63) >> 3) ^ (r & 7)) << 4)) = static_cast<T>(pr[r]);
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&p_full[buf]);
     }
-    __syncthreads();  // every thread is done with this slot and the scores
-    consumed = pg + 1;
-    if (warp == 0 && issued < pg1) issue(issued++);
-  }
-  // after an abort, copies still in flight land before the block exits:
-  // warp 0 waits (bounded) for every page it issued and no one consumed.
-  // pg0 <= consumed <= issued <= pg1 here (an empty split has all four
-  // equal), so every slot index below is in [0, NS).
-  if (warp == 0 && lane == 0)
-    for (int pg = consumed; pg < issued; ++pg)
-      mbar_wait_drain(&full[(pg - pg0) % NS], ((pg - pg0) / NS) & 1, kKernDecode, 0, 2);
-
-  // partial results of this split: unnormalised O, (m, l)
-  if (tid < HD) {
+    // ---------------------------------------------------------------- epilogue
+    // l of each row: the sum of the 128 threads' partial sums
 #pragma unroll
     for (int r = 0; r < RB; ++r) {
       if (r < R) {
-        const int h = g * G + r / p.Nq, t = r % p.Nq;
-        const size_t row = ((static_cast<size_t>(b) * p.Hq + h) * p.Nq + t) * p.S + split;
-        p.part_o[row * HD + tid] = acc[r];
+        float s = lp[r];
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+        if (lane == 0) sSum[warp * 32 + r] = s;
       }
     }
+    named_barrier_sync(1, 128);
+    bool have = ok && n_tiles > 0;
+    if (have) {
+      have = mbar_wait(&pv_done[(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1, abort_flag, kKernDecode, 0, 3);
+      tc_fence_after();
+    }
+    uint32_t ov[RB];
+#pragma unroll
+    for (int r = 0; r < RB; ++r) ov[r] = 0u;
+    if (__all_sync(0xffffffffu, have)) {
+      tmem_ld_n<RB>(tm_O + lane_off, ov);
+      tmem_ld_wait();
+    }
+    if (i < HD) {
+#pragma unroll
+      for (int r = 0; r < RB; ++r) {
+        if (r < R) {
+          const int h = g * G + r / p.Nq, t = r % p.Nq;
+          const size_t row = ((static_cast<size_t>(b) * p.Hq + h) * p.Nq + t) * p.S + split;
+          p.part_o[row * HD + i] = __uint_as_float(ov[r]);
+        }
+      }
+    }
+    if (i < R) {
+      float m = -INFINITY;
+#pragma unroll
+      for (int r = 0; r < RB; ++r)
+        if (r == i) m = ref[r];
+      const float l = sSum[i] + sSum[32 + i] + sSum[64 + i] + sSum[96 + i];
+      const int h = g * G + i / p.Nq, t = i % p.Nq;
+      const size_t row = ((static_cast<size_t>(b) * p.Hq + h) * p.Nq + t) * p.S + split;
+      p.part_ml[row * 2 + 0] = l > 0.f ? m : -INFINITY;
+      p.part_ml[row * 2 + 1] = l;
+    }
   }
-  if (tid < R) {
-    const int h = g * G + tid / p.Nq, t = tid % p.Nq;
-    const size_t row = ((static_cast<size_t>(b) * p.Hq + h) * p.Nq + t) * p.S + split;
-    p.part_ml[row * 2 + 0] = sM[tid];
-    p.part_ml[row * 2 + 1] = sL[tid];
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
   }
 }
 

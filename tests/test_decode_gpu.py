@@ -67,6 +67,40 @@ def test_decode_paged_parity(case):
     ac.check_lse(lse.cpu(), lse_r, what="decode lse")
 
 
+def test_decode_long_sequences_many_splits():
+    """The bench shape's heads and GQA group at 16K and 5K cached tokens: many
+    128-key tiles per split, several splits per sequence, a last tile that
+    ends inside a page."""
+    B, Hq, Hkv, Nq, d, P, lens = 2, 32, 8, 1, 128, 64, (16384, 5001)
+    q, kc, vc, table, seq_lens = make_case(77, B, Hq, Hkv, Nq, d, P, lens, torch.bfloat16)
+    dev = "cuda:0"
+    o, lse = binding.attention_decode_paged(q.to(dev), kc.to(dev), vc.to(dev), table.to(dev),
+                                            seq_lens.to(dev))
+    assert binding.fa_get_device_status() == binding.FA_OK
+    o_r, lse_r = oracle.decode_paged(q, kc, vc, table.numpy(), seq_lens.numpy(), 1 / math.sqrt(d))
+    ac.check_o(o.cpu(), o_r, torch.bfloat16, what="decode O")
+    ac.check_lse(lse.cpu(), lse_r, what="decode lse")
+
+
+@pytest.mark.parametrize("d,P,Nq", [(128, 32, 2), (64, 16, 3)])
+def test_decode_peaked_scores_move_the_reference(d, P, Nq):
+    """Scale 0.5 makes a tile's largest score exceed the running reference by
+    more than 8 (log2) again and again, so the running O is rescaled in
+    tensor memory many times.  lse is held to 1e-3; O, whose rows are
+    dominated by a few keys with |O| up to ~3, to the rounding bound of the
+    16-bit P and output (the peaked-softmax class of the O tolerance)."""
+    B, Hq, Hkv, lens = 2, 8, 2, (3000, 777)
+    q, kc, vc, table, seq_lens = make_case(5 + d + P, B, Hq, Hkv, Nq, d, P, lens, torch.bfloat16)
+    dev = "cuda:0"
+    o, lse = binding.attention_decode_paged(q.to(dev), kc.to(dev), vc.to(dev), table.to(dev),
+                                            seq_lens.to(dev), 0.5)
+    assert binding.fa_get_device_status() == binding.FA_OK
+    o_r, lse_r = oracle.decode_paged(q, kc, vc, table.numpy(), seq_lens.numpy(), 0.5)
+    o_abs, _ = oracle.decode_paged(q, kc, vc.abs(), table.numpy(), seq_lens.numpy(), 0.5)
+    ac.check_lse(lse.cpu(), lse_r, what="decode lse")
+    print(ac.check_o_rounding_bound(o.cpu(), o_r, torch.bfloat16, o_abs))
+
+
 @pytest.mark.parametrize("bad", ["page_id", "length"])
 def test_decode_bad_input_is_reported(bad):
     q, kc, vc, table, seq_lens = make_case(9, 2, 4, 2, 1, 64, 16, (40, 20), torch.bfloat16)

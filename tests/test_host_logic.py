@@ -26,16 +26,27 @@ def test_window_flops_count_visible_pairs(N, W):
     assert w.flops_bwd(True, W) == pytest.approx(2.5 * w.flops_fwd(True, W))
 
 
-def splits(B, Hkv, max_pages):
-    # four waves of two blocks per SM of a 148-SM B200, at least 4 pages a split
-    want = math.ceil(4 * 2 * 148 / (B * Hkv))
-    return max(1, min(want, max(1, max_pages // 4)))
+def splits(B, Hkv, d, max_pages):
+    # at least four waves of the blocks a 148-SM B200 holds at once (one per
+    # SM at d = 128, two at d = 64); among S0 .. 2 S0 the count whose last
+    # wave is the fullest; at least 4 pages a split
+    slots = 148 * (2 if d == 64 else 1)
+    bh = max(1, B * Hkv)
+    s0 = -(-4 * slots // bh)
+    cap = max(1, max_pages // 4)
+    best, best_eff = min(s0, cap), -1.0
+    for s in range(s0, min(2 * s0, cap) + 1):
+        blocks = bh * s
+        eff = blocks / (-(-blocks // slots) * slots)
+        if eff > best_eff + 1e-9:
+            best, best_eff = s, eff
+    return max(1, best)
 
 
 @pytest.mark.parametrize("B,Hq,Hkv,Nq,d,max_pages", [
     (32, 32, 8, 1, 128, 256), (1, 8, 8, 3, 64, 1), (2, 16, 1, 2, 128, 19), (300, 4, 4, 1, 64, 10)])
 def test_decode_workspace_bytes(B, Hq, Hkv, Nq, d, max_pages):
-    S = splits(B, Hkv, max_pages)
+    S = splits(B, Hkv, d, max_pages)
     assert binding.fa_decode_workspace_bytes(B, Hq, Hkv, Nq, d, max_pages) == B * Hq * Nq * S * (d + 2) * 4
     assert binding.fa_decode_workspace_bytes(0, Hq, Hkv, Nq, d, max_pages) == 0
 
