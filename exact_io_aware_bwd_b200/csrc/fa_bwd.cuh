@@ -14,7 +14,7 @@
 //   dQ_i  = scale sum_j dS_ij k_j,   dK_j = scale sum_i dS_ij q_i
 //
 // Three kernels:
-//   bwd_pre   one warp per query row: D_i = dO_i . O_i, lse2_i = lse_i log2(e)
+//   bwd_pre   d/8 threads per query row: D_i = dO_i . O_i, lse2_i = lse_i log2(e)
 //             (+inf for padding rows, which makes their P exactly 0), and a
 //             zeroed fp32 dQ accumulator row.
 //   bwd_main  persistent: one thread block per SM takes work items (128-row
@@ -42,21 +42,23 @@
 //             that no key block reaches, possible under a block mask, keep
 //             their zeroed accumulator: dQ = 0).
 //
-// Warp roles of bwd_main (448 threads):
-//   warps 0-7   softmax-gradient: warp w owns key rows 32(w%4)..+31 (tensor
-//               memory lanes) and query columns 32(w/4)..+31 of each step.
-//   warps 8-11  dQ drain (lane = feature index of dQ^T) and, after each
+// Warp roles of bwd_main (768 threads, at most 80 registers each: 24 warps,
+// six per SM sub-partition, share its 16 384 registers):
+//   warps 0-15  softmax-gradient: warp w owns key rows 32(w%4)..+31 (tensor
+//               memory lanes) and query columns 16(w/4)..+15 of each step.
+//   warps 16-19 dQ drain (lane = feature index of dQ^T) and, after each
 //               item, the dK / dV epilogue (lane = key row).
-//   warp 12     TMA producer; it also claims the work items and passes them
+//   warp 20     TMA producer; it also claims the work items and passes them
 //               to the other roles through a small ring in shared memory.
-//   warp 13     MMA issuer (the whole warp runs the loop, one elected lane
+//   warp 21     MMA issuer (the whole warp runs the loop, one elected lane
 //               issues).
+//   warps 22-23 idle (they round the block up to six warps per sub-partition).
 // Tensor memory: dV [0,128), dK [128,256), and two step buffers b = 0, 1:
-// S^T at 256+128b (64 columns; P^T is written over it as 16-bit pairs, each
-// warp half over its own columns) and dP^T at 256+128b+64 (dQ^T is written
-// over it once the softmax warps have read dP^T).  The step buffers let the
-// tensor cores compute step t+1's S^T / dP^T while the softmax warps work on
-// step t.
+// S^T at 256+128b (64 columns; P^T of each 16-query group is written as
+// 16-bit pairs over the first 8 columns of that group) and dP^T at
+// 256+128b+64 (dQ^T is written over it once the softmax warps have read
+// dP^T).  The step buffers let the tensor cores compute step t+1's S^T /
+// dP^T while the softmax warps work on step t.
 #pragma once
 
 #include <type_traits>
@@ -321,7 +323,7 @@ __device__ __forceinline__ BwdItem bwd_item(const BwdParams& p, int item) {
   return it;
 }
 
-constexpr int kBwdThreads = 448;
+constexpr int kBwdThreads = 768;
 
 template <int HD, bool BF16, bool CAUSAL, bool DROP, bool BMASK>
 __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_constant__ BwdParams p) {
@@ -365,7 +367,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
     return;
   }
   constexpr int kDrainThreads = HD == 128 ? 128 : 64;
-  constexpr int kSchedReaders = 1 + 8 + 4;  // MMA warp, softmax warps, drain warps
+  constexpr int kSchedReaders = 1 + 16 + 4;  // MMA warp, softmax warps, drain warps
 
   if (tid == 0) {
     mbar_init(kv_full, 1);
@@ -375,7 +377,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sdp_full[i], 1);
-      mbar_init(&ds_full[i], 256);
+      mbar_init(&ds_full[i], 512);
       mbar_init(&dq_full[i], 1);
       mbar_init(&dq_drained[i], kDrainThreads);
     }
@@ -389,7 +391,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 13) {
+  if (warp == 21) {
     tmem_alloc(tmem_ptr, 512);
     tmem_relinquish();
   }
@@ -416,7 +418,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
 
   // Steps are numbered across the items a block takes (g); the Q / dO ring
   // stage is g % kStages, the tensor-memory step buffer g & 1.
-  if (warp == 12) {
+  if (warp == 20) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       prefetch_tensormap(&p.tm_q);
@@ -481,7 +483,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
         gt += it.T;
       }
     }
-  } else if (warp == 13) {
+  } else if (warp == 21) {
     // ------------------------------------------------------------ MMA issuer
     // The whole warp runs this loop with warp-uniform values; one elected
     // lane issues each MMA and commit.  Descriptors are formed once and
@@ -579,11 +581,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
           }
           tc_fence_after();
         }
-        // dV += P^T dO: P^T from tensor memory (each 32-query half of it sits
-        // at the start of its own 32-column group), dO read MN-major.
+        // dV += P^T dO: P^T from tensor memory (the 16 queries of MMA k sit
+        // in the first 8 columns of their own 16-column group), dO read
+        // MN-major.
 #pragma unroll
         for (int k = 0; k < 4; ++k)
-          umma_ts_w(tm_dV, tm_S(buf) + (k >> 1) * 32 + (k & 1) * 8, sdesc_add(dO_mn, qs + k * 2048),
+          umma_ts_w(tm_dV, tm_S(buf) + k * 16, sdesc_add(dO_mn, qs + k * 2048),
                     kIdAcc, (t > 0 || k > 0) ? 1u : 0u);
         // dK += dS^T Q: dS^T K-major from shared memory, Q read MN-major.
 #pragma unroll
@@ -617,11 +620,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
     // every MMA this warp issued completes before tensor memory is freed
     umma_commit_w(done_bar);
     mbar_wait_drain(done_bar, 0, kKernBwd, 13, 5);
-  } else if (warp < 8) {
+  } else if (warp < 16) {
     // ------------------------------------------------------------ softmax gradient
-    // Every step is shared by the eight warps: warp w takes key rows
-    // 32(w%4)..+31 and query columns 32(w/4)..+31.
-    const int quarter = warp & 3, half = warp >> 2;
+    // Every step is shared by the sixteen warps: warp w takes key rows
+    // 32(w%4)..+31 and query columns 16(w/4)..+15.
+    const int quarter = warp & 3, qq = warp >> 2;
     const int r = quarter * 32 + lane;                 // key row within the block
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const float c_log2 = p.scale_log2;
@@ -644,22 +647,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
           break;
         }
         tc_fence_after();
-        // S^T and dP^T of this warp's 32 query columns are read from tensor
-        // memory at once (one wait), then worked in two passes of 16
-        // columns.  P^T of columns 16u..16u+15 is packed into the 8
-        // tensor-memory columns at 32(u/2) + 8(u%2) of the S^T buffer, where
-        // the dV product reads it; they held S^T of columns 32(u/2) + 8(u%2)
-        // .. +7, which this warp has read already.
-        uint32_t vs[32], vd[32];
-        tmem_ld16(tm_S(buf) + lane_off + 32 * half, vs);
-        tmem_ld16(tm_S(buf) + lane_off + 32 * half + 16, vs + 16);
-        tmem_ld16(tm_dP(buf) + lane_off + 32 * half, vd);
-        tmem_ld16(tm_dP(buf) + lane_off + 32 * half + 16, vd + 16);
+        // S^T and dP^T of this warp's 16 query columns.  P^T of them is
+        // packed into the first 8 of those tensor-memory columns of the S^T
+        // buffer, where the dV product reads it.
+        uint32_t v[16], vd[16];
+        tmem_ld16(tm_S(buf) + lane_off + 16 * qq, v);
+        tmem_ld16(tm_dP(buf) + lane_off + 16 * qq, vd);
         tmem_ld_wait();
-#pragma unroll
-        for (int qq = 2 * half; qq < 2 * half + 2; ++qq) {
+        {
           const int q_first = q_step + qq * 16;          // first query of these 16 columns
-          const uint32_t* v = vs + 16 * (qq & 1);
           const float4* lse4 = reinterpret_cast<const float4*>(sLse + s * 64 + qq * 16);
           const float4* d4 = reinterpret_cast<const float4*>(sD + s * 64 + qq * 16);
           float pr[16];
@@ -731,10 +727,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
 #pragma unroll
             for (int i = 0; i < 8; ++i) pk[i] = pack2<BF16>(pr[2 * i], pr[2 * i + 1]);
           }
-          tmem_st8(tm_S(buf) + lane_off + (qq >> 1) * 32 + (qq & 1) * 8, pk);
+          tmem_st8(tm_S(buf) + lane_off + 16 * qq, pk);
           float dp[16];
 #pragma unroll
-          for (int c = 0; c < 16; ++c) dp[c] = __uint_as_float(vd[16 * (qq & 1) + c]);
+          for (int c = 0; c < 16; ++c) dp[c] = __uint_as_float(vd[c]);
           if constexpr (DROP) {
             // dP of P is dP' times the dropout factor
 #pragma unroll
@@ -770,13 +766,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
       if (!ok) break;
       gt += it.T;
     }
-  } else {
+  } else if (warp < 20) {
     // ------------------------------------------------------------ dQ drain, dK/dV epilogue
     // Lane f of drain warp w holds feature f = 32w + lane of dQ^T: 64 query
     // values.  They are added into the fp32 accumulator straight from
     // registers; for a fixed query the 32 lanes of a warp touch 128
     // consecutive bytes, so every reduction is one coalesced request.
-    const int dw = warp - 8;                           // 0..3 == lane quarter
+    const int dw = warp - 16;                          // 0..3 == lane quarter
     const uint32_t lane_off = static_cast<uint32_t>(dw * 32) << 16;
     const bool drains = dw * 32 < HD;                  // warp holds real dQ^T rows
     int gt = 0;
@@ -853,7 +849,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 13) {
+  if (warp == 21) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
