@@ -47,9 +47,13 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # the backward main kernel on the default workload, from one ncu capture of
 # that kernel, with a digest of the kernel sources it was taken on: reported
 # only while the sources are unchanged.
-PROFILED_TRAFFIC = {"workload": "mha4k", "bytes": 1299325952, "sources_sha256_16": "9752b83a6347c5ae",
+PROFILED_TRAFFIC = {"workload": "mha4k", "bytes": 1296243200, "sources_sha256_16": "47660ecea5a2a1c9",
                     "sources": ("exact_io_aware_bwd_b200/csrc/fa_bwd.cuh",
                                 "exact_io_aware_bwd_b200/csrc/sm100.cuh")}
+# The same for the forward kernel (one launch on the default workload).
+PROFILED_TRAFFIC_FWD = {"workload": "mha4k", "bytes": 520983040, "sources_sha256_16": "97db3872e532d046",
+                        "sources": ("exact_io_aware_bwd_b200/csrc/fa_fwd.cuh",
+                                    "exact_io_aware_bwd_b200/csrc/sm100.cuh")}
 # The same for the FP8 forward kernel (one launch on the 4K-token MHA shape).
 PROFILED_TRAFFIC_FP8 = {"workload": "mha4k", "bytes": 307079936, "sources_sha256_16": "49abecf182bf2acc",
                         "sources": ("exact_io_aware_bwd_b200/csrc/fa_fwd_fp8.cuh",
@@ -448,7 +452,8 @@ def run_ours(args, w, causal, rank, world, device):
         "roofline": {"kernel": "fa_bwd_kernel (main backward pass)", "bound": "tensor",
                      "achieved": round(bwd_tflops_main, 2), "peak": peak, "unit": "TFLOP/s",
                      "frac": round(bwd_tflops_main / peak, 4), "peak_kind": f"{pk_kind} bf16 burst",
-                     "traffic": profiled_traffic(w.name) if not (W or DR) else None,
+                     "traffic": (profiled_traffic(w.name)
+                                 if causal and not (W or DR or BM is not None) else None),
                      "traffic_unit": "bytes per launch (ncu)",
                      "algorithmic": "2.5 x 4*B*Hq*N^2*d (/2 causal) FLOPs per launch"
                                     + (" (visible pairs under the window)" if W else "")
@@ -456,7 +461,9 @@ def run_ours(args, w, causal, rank, world, device):
         "forward_kernel": {"kernel": "fa_fwd_kernel", "bound": "tensor",
                            "achieved": round(f_fwd / (fwd_kern_mean * 1e-3) / 1e12, 2), "peak": peak,
                            "unit": "TFLOP/s",
-                           "frac": round(f_fwd / (fwd_kern_mean * 1e-3) / 1e12 / peak, 4)},
+                           "frac": round(f_fwd / (fwd_kern_mean * 1e-3) / 1e12 / peak, 4),
+                           "traffic": (profiled_traffic(w.name, PROFILED_TRAFFIC_FWD)
+                                       if causal and not (W or DR or BM is not None) else None)},
         "gpu_launches": launches_per_step * K,
         "clocks": clk,
         "e2e": e2e,
