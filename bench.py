@@ -274,6 +274,12 @@ def time_steps(args, w, causal, rank, world, device, steps, warmup, W=0, DR=None
         a.record(stream)
         b.record(stream)
     step = make_step(t, w, causal, W, DR, stream, fwd_ev, bwd_ev, BM)
+    # the clock sampler starts first (it needs a moment), then the warm-up
+    # steps run right before the timed ones, so that the GPU does not idle
+    # (and lower its clock) between the two
+    if clocks:
+        clocks.start()
+        time.sleep(0.3)
     for _ in range(warmup):
         step()
     torch.cuda.synchronize(device)
@@ -283,9 +289,6 @@ def time_steps(args, w, causal, rank, world, device, steps, warmup, W=0, DR=None
         if world > 1:
             torch.distributed.barrier()
 
-    if clocks:
-        clocks.start()
-        time.sleep(0.3)
     t0, t1 = ev(), ev()
     barrier()
     torch.cuda.synchronize(device)
@@ -510,16 +513,16 @@ def run_decode(args, rank, world, device):
     stream = torch.cuda.current_stream(device)
     scale = 1.0 / math.sqrt(d)
     step = lambda: binding.fa_decode_paged(q, kc, vc, table, lens, o, lse, scale, ws, stream)
+    clocks = ClockSampler(device) if rank == 0 else None
+    if clocks:  # started before the warm-up, which then runs right before the timed steps
+        clocks.start()
+        time.sleep(0.3)
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(device)
     assert binding.fa_get_device_status(stream) == binding.FA_OK
     K = args.steps
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    clocks = ClockSampler(device) if rank == 0 else None
-    if clocks:
-        clocks.start()
-        time.sleep(0.3)
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize(device)
@@ -569,19 +572,19 @@ def run_fp8(args, w, causal, rank, world, device):
     lse = torch.empty((B, Hq, N), device=device, dtype=torch.float32)
     stream = torch.cuda.current_stream(device)
     step = lambda: binding.fa_fwd_fp8(q8, k8, v8, o, lse, w.scale, descale, causal, stream)
-    for _ in range(max(args.warmup, 3)):
-        step()
-    torch.cuda.synchronize(device)
-    assert binding.fa_get_device_status(stream) == binding.FA_OK
     K = args.steps
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * K)]
     for e in ev:
         e.record(stream)  # creates the event handle the library records into
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(device) if rank == 0 else None
-    if clocks:
+    if clocks:  # started before the warm-up, which then runs right before the timed steps
         clocks.start()
         time.sleep(0.3)
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize(device)
+    assert binding.fa_get_device_status(stream) == binding.FA_OK
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize(device)

@@ -155,7 +155,8 @@ fa_status_t launch_fwd(const FwdParams& prm, cudaStream_t st) {
   const int smem = FwdLayout<HD>::kDynSmem;
   fa_status_t s = opt_in_smem(kern, smem);
   if (s != FA_OK) return s;
-  const int grid = prm.n_pairs * prm.BH;
+  // one block per (head, couple of query pairs) or per (head, query pair)
+  const int grid = (prm.fold ? (prm.n_pairs + 1) / 2 : prm.n_pairs) * prm.BH;
   prof_begin(fa::kKernFwd, st);
   kern<<<grid, fa::kFwdThreads, smem, st>>>(prm);
   const bool ok = cudaGetLastError() == cudaSuccess;
@@ -362,9 +363,9 @@ fa_status_t fwd_impl(const void* q, const void* k, const void* v, void* o, float
   const uint64_t BHq = static_cast<uint64_t>(B) * Hq, BHkv = static_cast<uint64_t>(B) * Hkv;
   if (!make_map(&prm.tm_q, q, dt, 2, d, N, BHq, 64, 128) ||
       !make_map(&prm.tm_k, k, dt, 2, d, N, BHkv, 64, 128) ||
-      !make_map(&prm.tm_v, v, dt, 2, d, N, BHkv, 64, 128) ||
-      !make_map(&prm.tm_o, o, dt, 2, d, N, BHq, 64, 128))
+      !make_map(&prm.tm_v, v, dt, 2, d, N, BHkv, 64, 128))
     return FA_ERR_CUDA;
+  prm.o = o;
   prm.lse = lse;
   prm.N = N;
   prm.Hq = Hq;
@@ -372,6 +373,9 @@ fa_status_t fwd_impl(const void* q, const void* k, const void* v, void* o, float
   prm.group = Hq / Hkv;
   prm.BH = static_cast<int>(BHq);
   prm.n_pairs = (N + 255) / 256;
+  // fold two query pairs into a block while a pair is short (its fixed costs
+  // then weigh most): up to 64 pairs (N <= 16384)
+  prm.fold = prm.n_pairs <= 64 ? 1 : 0;
   prm.n_ktiles = (N + 127) / 128;
   prm.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   prm.window = window;

@@ -1,5 +1,6 @@
 // Forward pass of exact attention on sm_100a: one thread block per
-// (batch, query head, pair of 128-row query blocks).
+// (batch, query head, couple of query pairs), a query pair being two
+// 128-row query blocks.
 //
 // Method (pages: "FlashAttention" glossary, opening list and online-softmax
 // paragraph; "flash attention io aware", sections "Flash Attention
@@ -19,14 +20,15 @@
 //   warps 0-3 / 4-7  softmax of query block 0 / 1: thread r owns row r of its
 //              block and tensor-memory lane r.  Reads S_j, masks, scales,
 //              updates (m, l), writes P_j (16-bit) over S_j, rescales O when
-//              needed, and at the end normalises O, stores it (TMA) and lse.
+//              needed, and at the end of a pair normalises O and writes it
+//              and lse (each thread its row).
 //   warp 8     MMA issuer (whole warp, one elected lane issues): S_t,j = Q_t K_j^T
 //              and O_t += P_t,j V_j
 //              for t = 0, 1, staggered as S0_j+1, O1 += P1_j V_j, S1_j+1,
 //              O0 += P0_j+1 V_j+1, ... so that one block's softmax overlaps the
 //              other block's products.
-//   warp 9     TMA producer: Q0, Q1 once, then K_0, V_0, K_1, V_1, ... through
-//              a ring of kSlots tiles.
+//   warp 9     TMA producer: Q0, Q1 of a pair, then K_0, V_0, K_1, V_1, ...
+//              through a ring of kSlots tiles; then the next pair's.
 //   warps 10-11 idle (they complete the third warpgroup, which gives its
 //              registers to the softmax warpgroups).
 // Tensor memory (512 columns x 128 lanes x 32 bit): S0 [0,128), S1 [128,256),
@@ -49,9 +51,10 @@ struct FwdParams {
   CUtensorMap tm_q;  // [B*Hq][N][d], box 64 x 128
   CUtensorMap tm_k;  // [B*Hkv][N][d]
   CUtensorMap tm_v;
-  CUtensorMap tm_o;  // [B*Hq][N][d] (store)
+  void* o;           // [B*Hq][N][d], written by the softmax threads
   float* lse;        // [B*Hq][N]
   int N, Hq, Hkv, group, BH, n_pairs, n_ktiles;
+  int fold;          // 1: a block runs query pairs n-1-c and c; 0: one pair
   int window;        // causal sliding window of this many keys (query i sees i-W+1..i); 0: none
   // dropout (kernels instantiated with DROP): key j of query i is dropped
   // when byte j%4 of word i%4 of Philox4x32-10((j/4, i/4, bh, 0), seed) is
@@ -109,8 +112,8 @@ struct FwdLayout {
   static constexpr int kOffRing = 2 * kTileBytes;
   static constexpr int kOffBar = kOffRing + kSlots * kTileBytes;
   // barriers: q_full, slot_full[kSlots], slot_empty[kSlots], s_full[2],
-  // p_half[2][2] (keys 0-63 / 64-127 of P_t ready), pv_done[2], done
-  static constexpr int kNumBars = 1 + 2 * kSlots + 8 + 1;
+  // p_half[2][2] (keys 0-63 / 64-127 of P_t ready), pv_done[2], done, q_free
+  static constexpr int kNumBars = 1 + 2 * kSlots + 8 + 1 + 1;
   static constexpr int kOffTmemPtr = kOffBar + kNumBars * 8;
   static constexpr int kOffAbort = kOffTmemPtr + 4;
   static constexpr int kSmemBytes = kOffAbort + 4;
@@ -129,10 +132,47 @@ constexpr uint32_t kFwdSoftmaxRegs = 216;
 constexpr uint32_t kFwdOtherRegs = 72;
 static_assert(2 * 128 * kFwdSoftmaxRegs + 128 * kFwdOtherRegs <= kFwdThreads * 168, "register split");
 constexpr uint32_t kKernFwd = 1;
+// One query pair of a head: its two 128-row query blocks and the key blocks
+// they stream.
+struct FwdItem {
+  int bh, pair, kvh, j_start, n_kv0, n_kv1;
+  FwdMaskRows mrows;
+};
+
+template <bool CAUSAL, bool BMASK>
+__device__ __forceinline__ FwdItem fwd_item(const FwdParams& p, int bh, int pair) {
+  FwdItem it;
+  it.bh = bh;
+  it.pair = pair;
+  const int h = bh % p.Hq;
+  const int b = bh / p.Hq;
+  it.kvh = b * p.Hkv + h / p.group;
+  // key blocks seen by query block t (t = 0, 1) of the pair.  With a sliding
+  // window the key/value stream starts at the first block the pair's first
+  // row can see; counts are of blocks from that one on.
+  it.j_start = (CAUSAL && p.window > 0) ? max(0, 2 * pair * 128 - p.window + 1) / 128 : 0;
+  it.n_kv0 = (CAUSAL ? min(2 * pair + 1, p.n_ktiles) : p.n_ktiles) - it.j_start;
+  it.n_kv1 = (CAUSAL ? min(2 * pair + 2, p.n_ktiles) : p.n_ktiles) - it.j_start;
+  // Under a block mask both blocks walk the union of their visible key
+  // blocks (n_kv0 = n_kv1 = its size, counted by each role's warp); a key
+  // block hidden from one of them is a fully masked tile for it.
+  it.mrows = FwdMaskRows{};
+  if constexpr (BMASK) {
+    const uint8_t* mh = p.bmask + static_cast<long long>(h) * p.bm_hstride;
+    const int qb0 = 2 * pair, qb1 = 2 * pair + 1;
+    it.mrows.row0 = mh + static_cast<long long>(qb0) * p.n_ktiles;
+    it.mrows.row1 = qb1 < p.n_ktiles ? mh + static_cast<long long>(qb1) * p.n_ktiles : nullptr;
+    it.mrows.jmax0 = CAUSAL ? min(qb0, p.n_ktiles - 1) : p.n_ktiles - 1;
+    it.mrows.jmax1 = CAUSAL ? min(qb1, p.n_ktiles - 1) : p.n_ktiles - 1;
+  }
+  return it;
+}
+
 template <int HD, bool BF16, bool CAUSAL, bool DROP, bool BMASK>
 __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_constant__ FwdParams p) {
   static_assert(!(DROP && BMASK), "dropout and block masks are not combined");
   using L = FwdLayout<HD>;
+  using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
@@ -146,6 +186,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
   uint64_t* p_half = s_full + 2;  // [t][half]
   uint64_t* pv_done = p_half + 4;
   uint64_t* done_bar = pv_done + 2;
+  uint64_t* q_free = done_bar + 1;  // every S product of a pair (the readers of sQ) has completed
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(sm + L::kOffTmemPtr);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::kOffAbort);
 
@@ -153,36 +194,23 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
   const int warp = tid >> 5;
   const int lane = tid & 31;
 
-  // Work item, head-major: the blocks running at the same time mostly share
-  // a head, so its K and V stay in L2; inside a head the query pairs with the
-  // most key blocks (under a causal mask) go first.
-  const int item = blockIdx.x;
-  const int bh = item / p.n_pairs;
-  const int pair = p.n_pairs - 1 - item % p.n_pairs;
-  const int h = bh % p.Hq;
-  const int b = bh / p.Hq;
-  const int kvh = b * p.Hkv + h / p.group;
-  // key blocks seen by query block t (t = 0, 1) of the pair
-  // With a sliding window the key/value stream starts at the first block the
-  // pair's first row can see; counts below are of blocks from that one on.
-  const int j_start = (CAUSAL && p.window > 0) ? max(0, 2 * pair * 128 - p.window + 1) / 128 : 0;
-  int n_kv0 = (CAUSAL ? min(2 * pair + 1, p.n_ktiles) : p.n_ktiles) - j_start;
-  int n_kv1 = (CAUSAL ? min(2 * pair + 2, p.n_ktiles) : p.n_ktiles) - j_start;
-  // Under a block mask both blocks walk the union of their visible key
-  // blocks (n_kv0 = n_kv1 = its size, counted by each role's warp); a key
-  // block hidden from one of them is a fully masked tile for it.
-  FwdMaskRows mrows{};
-  if constexpr (BMASK) {
-    const uint8_t* mh = p.bmask + static_cast<long long>(h) * p.bm_hstride;
-    const int qb0 = 2 * pair, qb1 = 2 * pair + 1;
-    mrows.row0 = mh + static_cast<long long>(qb0) * p.n_ktiles;
-    mrows.row1 = qb1 < p.n_ktiles ? mh + static_cast<long long>(qb1) * p.n_ktiles : nullptr;
-    mrows.jmax0 = CAUSAL ? min(qb0, p.n_ktiles - 1) : p.n_ktiles - 1;
-    mrows.jmax1 = CAUSAL ? min(qb1, p.n_ktiles - 1) : p.n_ktiles - 1;
-  }
+  // The block's work: query pairs n-1-c and c of head bh, back to back (one
+  // pair when they coincide).  Under a causal mask pair i streams 2i + 2 key
+  // blocks, so every couple has the same length and the blocks of a launch
+  // take equal time; the second pair's Q load and first S product overlap
+  // the first pair's last tiles and epilogue.  Head-major order: the blocks
+  // running at the same time mostly share a head, so its K and V stay in L2.
+  // Without folding (long sequences, where a pair's fixed costs are small
+  // next to its key blocks) a block runs one pair, the longest first.
+  const int n_couples = p.fold ? (p.n_pairs + 1) / 2 : p.n_pairs;
+  const int bh = blockIdx.x / n_couples;
+  const int cpl = blockIdx.x % n_couples;
+  const int n_items = (!p.fold || p.n_pairs - 1 - cpl == cpl) ? 1 : 2;
+  auto item_pair = [&](int it) { return it == 0 ? p.n_pairs - 1 - cpl : cpl; };
 
   if (tid == 0) {
     mbar_init(q_full, 1);
+    mbar_init(q_free, 1);
     for (int s = 0; s < L::kSlots; ++s) {
       mbar_init(&slot_full[s], 1);
       mbar_init(&slot_empty[s], 1);
@@ -212,36 +240,48 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
     // idle warps of the third warpgroup
   } else if (warp == 9) {
     // ------------------------------------------------------------ producer
-    if constexpr (BMASK) n_kv1 = mrows.count_warp(lane);
     if (lane == 0) {
       prefetch_tensormap(&p.tm_q);
       prefetch_tensormap(&p.tm_k);
       prefetch_tensormap(&p.tm_v);
-      mbar_expect_tx(q_full, 2 * L::kTileBytes);
-      for (int t = 0; t < 2; ++t)
-        for (int c = 0; c < L::kChunks; ++c)
-          tma_load_3d(sQ + t * L::kTileBytes + c * L::kBoxBytes, &p.tm_q, q_full, c * 64,
-                      (2 * pair + t) * 128, bh);
-      int n = 0;
-      auto load = [&](const CUtensorMap* map, int kblock) -> bool {
-        const int s = n % L::kSlots;
-        if (n >= L::kSlots &&
-            !mbar_wait(&slot_empty[s], ((n / L::kSlots) - 1) & 1, abort_flag, kKernFwd, 9, 0))
-          return false;
-        mbar_expect_tx(&slot_full[s], L::kTileBytes);
-        uint8_t* dst = sRing + s * L::kTileBytes;
-        for (int c = 0; c < L::kChunks; ++c)
-          tma_load_3d(dst + c * L::kBoxBytes, map, &slot_full[s], c * 64, kblock * 128, kvh);
-        ++n;
-        return true;
-      };
-      bool ok = true;
-      int kb = BMASK ? mrows.next(0) : j_start;  // key block of stream position j
-      for (int j = 0; ok && j < n_kv1; ++j) {
-        ok = load(&p.tm_k, kb);
-        if (ok) ok = load(&p.tm_v, kb);
-        kb = BMASK ? mrows.next(kb + 1) : kb + 1;
+    }
+    int n = 0;  // K/V tiles loaded (ring position), over both pairs
+    bool ok = true;
+    for (int it = 0; ok && it < n_items; ++it) {
+      const FwdItem I = fwd_item<CAUSAL, BMASK>(p, bh, item_pair(it));
+      int n_kv1 = I.n_kv1;
+      if constexpr (BMASK) n_kv1 = I.mrows.count_warp(lane);
+      if (lane == 0) {
+        // Q0, Q1 of the pair; the previous pair's S products, the last
+        // readers of sQ, must have completed
+        if (it > 0) ok = mbar_wait(q_free, (it - 1) & 1, abort_flag, kKernFwd, 9, 1);
+        if (ok) {
+          mbar_expect_tx(q_full, 2 * L::kTileBytes);
+          for (int t = 0; t < 2; ++t)
+            for (int c = 0; c < L::kChunks; ++c)
+              tma_load_3d(sQ + t * L::kTileBytes + c * L::kBoxBytes, &p.tm_q, q_full, c * 64,
+                          (2 * I.pair + t) * 128, I.bh);
+        }
+        auto load = [&](const CUtensorMap* map, int kblock) -> bool {
+          const int s = n % L::kSlots;
+          if (n >= L::kSlots &&
+              !mbar_wait(&slot_empty[s], ((n / L::kSlots) - 1) & 1, abort_flag, kKernFwd, 9, 0))
+            return false;
+          mbar_expect_tx(&slot_full[s], L::kTileBytes);
+          uint8_t* dst = sRing + s * L::kTileBytes;
+          for (int c = 0; c < L::kChunks; ++c)
+            tma_load_3d(dst + c * L::kBoxBytes, map, &slot_full[s], c * 64, kblock * 128, I.kvh);
+          ++n;
+          return true;
+        };
+        int kb = BMASK ? I.mrows.next(0) : I.j_start;  // key block of stream position j
+        for (int j = 0; ok && j < n_kv1; ++j) {
+          ok = load(&p.tm_k, kb);
+          if (ok) ok = load(&p.tm_v, kb);
+          kb = BMASK ? I.mrows.next(kb + 1) : kb + 1;
+        }
       }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
     }
   } else if (warp == 8) {
     // ------------------------------------------------------------ MMA issuer
@@ -256,8 +296,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
     auto wait_all = [&](uint64_t* bar, uint32_t parity, uint32_t site) -> bool {
       return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, kKernFwd, 8, site));
     };
-    int n = 0;
-    bool ok = wait_all(q_full, 0, 0);
+    int n = 0;  // K/V tiles taken from the ring, over both pairs
     auto take = [&](int& slot) -> bool {
       slot = n % L::kSlots;
       if (!wait_all(&slot_full[slot], (n / L::kSlots) & 1, 1)) return false;
@@ -273,7 +312,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
     // core runs the MMAs of one thread in issue order, reading an MMA's
     // operands before a later MMA writes its result, so no wait is put
     // between them (waiting for an MMA's completion before issuing the next
-    // costs several hundred cycles of idle tensor core on B200).
+    // costs several hundred cycles of idle tensor core on B200).  The same
+    // holds across the two pairs: the next pair's S_t,0 follows the last
+    // O_t += P_t V.
     auto issue_s = [&](int t, int kslot) {
       const uint32_t qo = t * L::kTileBytes, ko = kslot * L::kTileBytes;
 #pragma unroll
@@ -284,12 +325,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
       umma_commit_w(&s_full[t]);
     };
     // O_t += P_t,j V_j in two halves of 64 keys: the softmax warps hand over
-    // P of keys 0-63 before they compute keys 64-127.
-    auto issue_pv = [&](int t, int j, int vslot) -> bool {
+    // P of keys 0-63 before they compute keys 64-127.  g: the tile's index
+    // over both pairs (barrier phase), j: its index in the pair.
+    auto issue_pv = [&](int t, int g, int j, int vslot) -> bool {
       const uint32_t vo = vslot * L::kTileBytes;
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
-        if (!wait_all(&p_half[2 * t + half], j & 1, 3)) return false;
+        if (!wait_all(&p_half[2 * t + half], g & 1, 3)) return false;
         tc_fence_after();
 #pragma unroll
         for (int k = 4 * half; k < 4 * half + 4; ++k)
@@ -299,29 +341,43 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
       umma_commit_w(&pv_done[t]);
       return true;
     };
-    if constexpr (BMASK) n_kv0 = n_kv1 = mrows.count_warp(lane);
-    int kslot = 0, vslot = 0;
-    if (ok && n_kv1 > 0) ok = take(kslot);
-    else ok = false;  // nothing to compute (only under a block mask)
-    if (ok) {
+    int g0 = 0, g1 = 0;  // tiles of query block 0 / 1 in the pairs before this one
+    bool ok = true;
+    for (int it = 0; ok && it < n_items; ++it) {
+      const FwdItem I = fwd_item<CAUSAL, BMASK>(p, bh, item_pair(it));
+      int n_kv0 = I.n_kv0, n_kv1 = I.n_kv1;
+      if constexpr (BMASK) n_kv0 = n_kv1 = I.mrows.count_warp(lane);
+      if (!(ok = wait_all(q_full, it & 1, 0))) break;
+      tc_fence_after();
+      if (n_kv1 == 0) {
+        // nothing to compute (only under a block mask): sQ is free at once
+        umma_commit_w(q_free);
+        continue;
+      }
+      int kslot = 0, vslot = 0;
+      if (!(ok = take(kslot))) break;
       if (n_kv0 > 0) issue_s(0, kslot);
       issue_s(1, kslot);
       umma_commit_w(&slot_empty[kslot]);
-      ok = take(vslot);
-    }
-    if (ok && n_kv0 > 0) ok = issue_pv(0, 0, vslot);
-    for (int j = 0; ok && j < n_kv1; ++j) {
-      const bool next1 = j + 1 < n_kv1, next0 = j + 1 < n_kv0;
-      if (next1 && !(ok = take(kslot))) break;
-      if (next0) issue_s(0, kslot);
-      if (!(ok = issue_pv(1, j, vslot))) break;
-      umma_commit_w(&slot_empty[vslot]);  // V_j: read by both PV_j
-      if (next1) {
-        issue_s(1, kslot);
-        umma_commit_w(&slot_empty[kslot]);  // K_j+1: read by both S_j+1
-        if (!(ok = take(vslot))) break;
+      if (n_kv1 == 1) umma_commit_w(q_free);  // the pair's last S
+      if (!(ok = take(vslot))) break;
+      if (n_kv0 > 0 && !(ok = issue_pv(0, g0, 0, vslot))) break;
+      for (int j = 0; ok && j < n_kv1; ++j) {
+        const bool next1 = j + 1 < n_kv1, next0 = j + 1 < n_kv0;
+        if (next1 && !(ok = take(kslot))) break;
+        if (next0) issue_s(0, kslot);
+        if (!(ok = issue_pv(1, g1 + j, j, vslot))) break;
+        umma_commit_w(&slot_empty[vslot]);  // V_j: read by both PV_j
+        if (next1) {
+          issue_s(1, kslot);
+          umma_commit_w(&slot_empty[kslot]);  // K_j+1: read by both S_j+1
+          if (j + 2 == n_kv1) umma_commit_w(q_free);  // the pair's last S
+          if (!(ok = take(vslot))) break;
+        }
+        if (next0 && !(ok = issue_pv(0, g0 + j + 1, j + 1, vslot))) break;
       }
-      if (next0 && !(ok = issue_pv(0, j + 1, vslot))) break;
+      g0 += n_kv0;
+      g1 += n_kv1;
     }
     // every MMA this warp issued completes before tensor memory is freed
     umma_commit_w(done_bar);
@@ -334,16 +390,21 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tm_S = tmem + t * 128 + lane_off;
     const uint32_t tm_O = tmem + 256 + t * 128 + lane_off;
-    const int qtile = 2 * pair + t;
+    const float c_log2 = p.scale_log2;
+    const uint64_t c2 = f2pack(c_log2, c_log2);
+    int gt = 0;  // tiles of this query block in the pairs before this one
+    bool ok = true;
+    for (int it = 0; ok && it < n_items; ++it) {
+    const FwdItem I = fwd_item<CAUSAL, BMASK>(p, bh, item_pair(it));
+    const FwdMaskRows& mrows = I.mrows;
+    int n_kv0 = I.n_kv0, n_kv1 = I.n_kv1;
+    const int qtile = 2 * I.pair + t;
     const int q_row = qtile * 128 + r;
     if constexpr (BMASK) n_kv0 = n_kv1 = mrows.count_warp(lane);
     const int n_kv = t ? n_kv1 : n_kv0;
-    int kb_cur = BMASK ? mrows.next(0) : j_start;  // key block of the current stream position
-    const float c_log2 = p.scale_log2;
-    const uint64_t c2 = f2pack(c_log2, c_log2);
+    int kb_cur = BMASK ? mrows.next(0) : I.j_start;  // key block of the current stream position
     float m_ref = -INFINITY;  // in log2 units of the scaled scores
     float l_sum = 0.f;
-    bool ok = true;
     // Waits are made warp-uniform: tcgen05.ld/st are warp-collective, so a
     // warp either goes on together or leaves together (on abort).
     //
@@ -357,189 +418,188 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
     // goes to tensor memory and is handed to the MMA warp, then keys 64-127.
     // Otherwise the tile is redone from tensor memory against the moved
     // reference, after O and l are rescaled.
-    auto load_s = [&](int kblock, uint32_t* s) {
-      tmem_ld32(tm_S + 0, s);
-      tmem_ld32(tm_S + 32, s + 32);
-      tmem_ld32(tm_S + 64, s + 64);
-      tmem_ld32(tm_S + 96, s + 96);
-      tmem_ld_wait();
-      // mask: keys past the end of the sequence, and keys after the query
-      // inside the diagonal block of a causal problem
-      const int kv0 = kblock * 128;
-      const bool diag = CAUSAL && (kblock == qtile);
-      // sliding window: keys below q_row - W + 1 are hidden; some row of the
-      // block meets that edge in this key block
-      const bool low = CAUSAL && p.window > 0 && kv0 + p.window <= qtile * 128 + 127;
-      // block mask: a key block of the pair's stream that this query block
-      // does not see is hidden whole
-      const bool hid = BMASK && !mrows.vis(t, kblock);
-      if (diag || low || hid || kv0 + 128 > p.N) {
-        const int lim = hid ? -1 : min(diag ? r : 127, p.N - 1 - kv0);  // last visible column
-        const int first = low ? q_row - p.window + 1 - kv0 : 0;  // first visible column
-#pragma unroll
-        for (int c = 0; c < 128; ++c)
-          if (c > lim || c < first) s[c] = __float_as_uint(-INFINITY);
-        return true;   // masked tile
-      }
-      return false;
-    };
-    // P of the 32 keys 32*q4 .. +31 against the reference -m (nm2), packed to
-    // 16 bits in pk[16]; the unrounded values are summed into acc.
-    auto p_chunk = [&](const uint32_t* s, int q4, uint64_t nm2, int kv0, uint32_t* pk, uint64_t* acc) {
-      [[maybe_unused]] uint32_t kw[4] = {0, 0, 0, 0};  // dropout bytes: keys 4g..4g+3 of 16 in kw[g]
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const int c = q4 * 32 + 2 * i;
-        const uint64_t x = fma2(f2pack(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), c2, nm2);
-        const uint64_t pp = f2pack(ex2_approx(f2lo(x)), ex2_approx(f2hi(x)));
-        acc[i & 3] = add2(acc[i & 3], pp);  // l sums the undropped P
-        if constexpr (DROP) {
-          if ((i & 7) == 0) {
-            // The 4 lanes of a quad hold 4 consecutive rows (one Philox
-            // counter row).  Lane g of the quad draws the 4x4 block of keys
-            // 4g..4g+3 of the next 16; four rotations of a shuffle give
-            // each lane its own row's word of all four blocks.
-            const int ql = lane & 3;
-            const uint4 rnd = philox4x32_10(
-                make_uint4(static_cast<uint32_t>((kv0 + c + 4 * ql) >> 2), static_cast<uint32_t>(q_row >> 2),
-                           static_cast<uint32_t>(bh), 0u),
-                p.seed_lo, p.seed_hi);
-#pragma unroll
-            for (int rr = 0; rr < 4; ++rr) {
-              const uint32_t got = __shfl_sync(0xffffffffu, uint4_word(rnd, (ql - rr) & 3),
-                                               (lane & ~3) | ((ql + rr) & 3));
-              const int g = (ql + rr) & 3;
-              kw[0] = g == 0 ? got : kw[0];
-              kw[1] = g == 1 ? got : kw[1];
-              kw[2] = g == 2 ? got : kw[2];
-              kw[3] = g == 3 ? got : kw[3];
+      auto load_s = [&](int kblock, uint32_t* s) {
+        tmem_ld32(tm_S + 0, s);
+        tmem_ld32(tm_S + 32, s + 32);
+        tmem_ld32(tm_S + 64, s + 64);
+        tmem_ld32(tm_S + 96, s + 96);
+        tmem_ld_wait();
+        // mask: keys past the end of the sequence, and keys after the query
+        // inside the diagonal block of a causal problem
+        const int kv0 = kblock * 128;
+        const bool diag = CAUSAL && (kblock == qtile);
+        // sliding window: keys below q_row - W + 1 are hidden; some row of the
+        // block meets that edge in this key block
+        const bool low = CAUSAL && p.window > 0 && kv0 + p.window <= qtile * 128 + 127;
+        // block mask: a key block of the pair's stream that this query block
+        // does not see is hidden whole
+        const bool hid = BMASK && !mrows.vis(t, kblock);
+        if (diag || low || hid || kv0 + 128 > p.N) {
+          const int lim = hid ? -1 : min(diag ? r : 127, p.N - 1 - kv0);  // last visible column
+          const int first = low ? q_row - p.window + 1 - kv0 : 0;  // first visible column
+  #pragma unroll
+          for (int c = 0; c < 128; ++c)
+            if (c > lim || c < first) s[c] = __float_as_uint(-INFINITY);
+          return true;   // masked tile
+        }
+        return false;
+      };
+      // P of the 32 keys 32*q4 .. +31 against the reference -m (nm2), packed to
+      // 16 bits in pk[16]; the unrounded values are summed into acc.
+      auto p_chunk = [&](const uint32_t* s, int q4, uint64_t nm2, int kv0, uint32_t* pk, uint64_t* acc) {
+        [[maybe_unused]] uint32_t kw[4] = {0, 0, 0, 0};  // dropout bytes: keys 4g..4g+3 of 16 in kw[g]
+  #pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int c = q4 * 32 + 2 * i;
+          const uint64_t x = fma2(f2pack(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), c2, nm2);
+          const uint64_t pp = f2pack(ex2_approx(f2lo(x)), ex2_approx(f2hi(x)));
+          acc[i & 3] = add2(acc[i & 3], pp);  // l sums the undropped P
+          if constexpr (DROP) {
+            if ((i & 7) == 0) {
+              // The 4 lanes of a quad hold 4 consecutive rows (one Philox
+              // counter row).  Lane g of the quad draws the 4x4 block of keys
+              // 4g..4g+3 of the next 16; four rotations of a shuffle give
+              // each lane its own row's word of all four blocks.
+              const int ql = lane & 3;
+              const uint4 rnd = philox4x32_10(
+                  make_uint4(static_cast<uint32_t>((kv0 + c + 4 * ql) >> 2), static_cast<uint32_t>(q_row >> 2),
+                             static_cast<uint32_t>(bh), 0u),
+                  p.seed_lo, p.seed_hi);
+  #pragma unroll
+              for (int rr = 0; rr < 4; ++rr) {
+                const uint32_t got = __shfl_sync(0xffffffffu, uint4_word(rnd, (ql - rr) & 3),
+                                                 (lane & ~3) | ((ql + rr) & 3));
+                const int g = (ql + rr) & 3;
+                kw[0] = g == 0 ? got : kw[0];
+                kw[1] = g == 1 ? got : kw[1];
+                kw[2] = g == 2 ? got : kw[2];
+                kw[3] = g == 3 ? got : kw[3];
+              }
             }
-          }
-          const uint32_t keep_word = kw[(i >> 1) & 3];
-          const uint32_t b0 = (keep_word >> (16 * (i & 1))) & 0xFFu;
-          const uint32_t b1 = (keep_word >> (16 * (i & 1) + 8)) & 0xFFu;
-          pk[i] = pack2<BF16>(b0 >= p.drop_t ? f2lo(pp) : 0.f, b1 >= p.drop_t ? f2hi(pp) : 0.f);
-        } else {
-          pk[i] = pack2<BF16>(f2lo(pp), f2hi(pp));
-        }
-      }
-    };
-    auto hand_over = [&](int half) {
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(&p_half[2 * t + half]);
-    };
-    auto sum_acc = [&](const uint64_t* acc) {
-      const uint64_t a = add2(add2(acc[0], acc[1]), add2(acc[2], acc[3]));
-      return f2lo(a) + f2hi(a);
-    };
-    for (int j = 0; j < n_kv; ++j) {
-      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[t], j & 1, abort_flag, kKernFwd, t, 0))) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      const int kb = kb_cur;
-      if constexpr (BMASK) kb_cur = mrows.next(kb + 1);
-      else kb_cur = kb + 1;
-      const int kv0 = kb * 128;
-      bool done = false;
-      float m_new;
-      {
-        uint32_t s[128];
-        load_s(kb, s);
-        // row max, eight independent chains of three-input maxima: chain i
-        // takes columns i, i + 8, ..., i + 120
-        float mx[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) mx[i] = fmaxf(__uint_as_float(s[i]), __uint_as_float(s[8 + i]));
-#pragma unroll
-        for (int c = 16; c < 128; c += 16)
-#pragma unroll
-          for (int i = 0; i < 8; ++i)
-            mx[i] = max3f(mx[i], __uint_as_float(s[c + i]), __uint_as_float(s[c + 8 + i]));
-        m_new = max3f(max3f(mx[0], mx[1], mx[2]), max3f(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) * c_log2;
-        if (!DROP && j > 0) {
-          // speculative: keys 0-63 against the current reference
-          const float m_use = m_ref == -INFINITY ? 0.f : m_ref;
-          const uint64_t nm2 = f2pack(-m_use, -m_use);
-          uint32_t pk0[16], pk1[16];
-          uint64_t acc[4] = {0, 0, 0, 0};
-          p_chunk(s, 0, nm2, kv0, pk0, acc);
-          p_chunk(s, 1, nm2, kv0, pk1, acc);
-          if (!__any_sync(0xffffffffu, m_new > m_ref + 8.0f)) {
-            tmem_st16(tm_S + 0, pk0);
-            tmem_st16(tm_S + 16, pk1);
-            hand_over(0);
-            p_chunk(s, 2, nm2, kv0, pk0, acc);
-            tmem_st16(tm_S + 32, pk0);
-            p_chunk(s, 3, nm2, kv0, pk1, acc);
-            tmem_st16(tm_S + 48, pk1);
-            l_sum += sum_acc(acc);
-            hand_over(1);
-            done = true;
+            const uint32_t keep_word = kw[(i >> 1) & 3];
+            const uint32_t b0 = (keep_word >> (16 * (i & 1))) & 0xFFu;
+            const uint32_t b1 = (keep_word >> (16 * (i & 1) + 8)) & 0xFFu;
+            pk[i] = pack2<BF16>(b0 >= p.drop_t ? f2lo(pp) : 0.f, b1 >= p.drop_t ? f2hi(pp) : 0.f);
+          } else {
+            pk[i] = pack2<BF16>(f2lo(pp), f2hi(pp));
           }
         }
-      }
-      if (done) continue;
-      // first tile of the rows, or a reference max that must move
-      if (j > 0) {
-        // Move the reference max of every row of this warp (tcgen05.ld/st are
-        // warp-wide), rescaling O and l, once O_t += P_t,j-1 V_j-1 is done.
-        if (!__all_sync(0xffffffffu, mbar_wait(&pv_done[t], (j - 1) & 1, abort_flag, kKernFwd, t, 1))) {
+      };
+      auto hand_over = [&](int half) {
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&p_half[2 * t + half]);
+      };
+      auto sum_acc = [&](const uint64_t* acc) {
+        const uint64_t a = add2(add2(acc[0], acc[1]), add2(acc[2], acc[3]));
+        return f2lo(a) + f2hi(a);
+      };
+      for (int j = 0; j < n_kv; ++j) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&s_full[t], (gt + j) & 1, abort_flag, kKernFwd, t, 0))) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const float m_upd = fmaxf(m_ref, m_new);
-        // rows still without a visible key (m_upd = -inf) keep their zeros
-        const float corr = m_upd == -INFINITY ? 1.f : ex2_approx(m_ref - m_upd);
-        const uint64_t corr2 = f2pack(corr, corr);
-        m_ref = m_upd;
-        l_sum *= corr;
-#pragma unroll 1
-        for (int c = 0; c < HD; c += 16) {
-          uint32_t o[16];
-          tmem_ld16(tm_O + c, o);
-          tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 16; i += 2) {
-            const uint64_t v = mul2(f2pack(__uint_as_float(o[i]), __uint_as_float(o[i + 1])), corr2);
-            o[i] = __float_as_uint(f2lo(v));
-            o[i + 1] = __float_as_uint(f2hi(v));
+        const int kb = kb_cur;
+        if constexpr (BMASK) kb_cur = mrows.next(kb + 1);
+        else kb_cur = kb + 1;
+        const int kv0 = kb * 128;
+        bool done = false;
+        float m_new;
+        {
+          uint32_t s[128];
+          load_s(kb, s);
+          // row max, eight independent chains of three-input maxima: chain i
+          // takes columns i, i + 8, ..., i + 120
+          float mx[8];
+  #pragma unroll
+          for (int i = 0; i < 8; ++i) mx[i] = fmaxf(__uint_as_float(s[i]), __uint_as_float(s[8 + i]));
+  #pragma unroll
+          for (int c = 16; c < 128; c += 16)
+  #pragma unroll
+            for (int i = 0; i < 8; ++i)
+              mx[i] = max3f(mx[i], __uint_as_float(s[c + i]), __uint_as_float(s[c + 8 + i]));
+          m_new = max3f(max3f(mx[0], mx[1], mx[2]), max3f(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) * c_log2;
+          if (!DROP && j > 0) {
+            // speculative: keys 0-63 against the current reference
+            const float m_use = m_ref == -INFINITY ? 0.f : m_ref;
+            const uint64_t nm2 = f2pack(-m_use, -m_use);
+            uint32_t pk0[16], pk1[16];
+            uint64_t acc[4] = {0, 0, 0, 0};
+            p_chunk(s, 0, nm2, kv0, pk0, acc);
+            p_chunk(s, 1, nm2, kv0, pk1, acc);
+            if (!__any_sync(0xffffffffu, m_new > m_ref + 8.0f)) {
+              tmem_st16(tm_S + 0, pk0);
+              tmem_st16(tm_S + 16, pk1);
+              hand_over(0);
+              p_chunk(s, 2, nm2, kv0, pk0, acc);
+              tmem_st16(tm_S + 32, pk0);
+              p_chunk(s, 3, nm2, kv0, pk1, acc);
+              tmem_st16(tm_S + 48, pk1);
+              l_sum += sum_acc(acc);
+              hand_over(1);
+              done = true;
+            }
           }
-          tmem_st16(tm_O + c, o);
         }
-      } else {
-        m_ref = m_new;
-      }
-      {
-        // P = 2^(s c - m_ref), packed to 16 bits over the first 64 columns of
-        // S.  A row that has seen no visible key yet (only under a sliding
-        // window) keeps m_ref = -inf; its scores are all -inf and give P = 0
-        // against 0.
-        uint32_t s[128];
-        load_s(kb, s);
-        const float m_use = m_ref == -INFINITY ? 0.f : m_ref;
-        const uint64_t nm2 = f2pack(-m_use, -m_use);
-        uint64_t acc[4] = {0, 0, 0, 0};
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          uint32_t pk[16];
-          p_chunk(s, q4, nm2, kv0, pk, acc);
-          tmem_st16(tm_S + q4 * 16, pk);
-          if (q4 == 1) hand_over(0);
+        if (done) continue;
+        // first tile of the rows, or a reference max that must move
+        if (j > 0) {
+          // Move the reference max of every row of this warp (tcgen05.ld/st are
+          // warp-wide), rescaling O and l, once O_t += P_t,j-1 V_j-1 is done.
+          if (!__all_sync(0xffffffffu, mbar_wait(&pv_done[t], (gt + j - 1) & 1, abort_flag, kKernFwd, t, 1))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const float m_upd = fmaxf(m_ref, m_new);
+          // rows still without a visible key (m_upd = -inf) keep their zeros
+          const float corr = m_upd == -INFINITY ? 1.f : ex2_approx(m_ref - m_upd);
+          const uint64_t corr2 = f2pack(corr, corr);
+          m_ref = m_upd;
+          l_sum *= corr;
+  #pragma unroll 1
+          for (int c = 0; c < HD; c += 16) {
+            uint32_t o[16];
+            tmem_ld16(tm_O + c, o);
+            tmem_ld_wait();
+  #pragma unroll
+            for (int i = 0; i < 16; i += 2) {
+              const uint64_t v = mul2(f2pack(__uint_as_float(o[i]), __uint_as_float(o[i + 1])), corr2);
+              o[i] = __float_as_uint(f2lo(v));
+              o[i + 1] = __float_as_uint(f2hi(v));
+            }
+            tmem_st16(tm_O + c, o);
+          }
+        } else {
+          m_ref = m_new;
         }
-        l_sum += sum_acc(acc);
-        hand_over(1);
+        {
+          // P = 2^(s c - m_ref), packed to 16 bits over the first 64 columns of
+          // S.  A row that has seen no visible key yet (only under a sliding
+          // window) keeps m_ref = -inf; its scores are all -inf and give P = 0
+          // against 0.
+          uint32_t s[128];
+          load_s(kb, s);
+          const float m_use = m_ref == -INFINITY ? 0.f : m_ref;
+          const uint64_t nm2 = f2pack(-m_use, -m_use);
+          uint64_t acc[4] = {0, 0, 0, 0};
+  #pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            uint32_t pk[16];
+            p_chunk(s, q4, nm2, kv0, pk, acc);
+            tmem_st16(tm_S + q4 * 16, pk);
+            if (q4 == 1) hand_over(0);
+          }
+          l_sum += sum_acc(acc);
+          hand_over(1);
+        }
       }
-    }
-    // epilogue: O / l -> 16-bit, staged in this block's (now idle) Q tile, TMA store
-    uint8_t* sQt = sQ + t * L::kTileBytes;
+    // epilogue: O / l -> 16-bit, written from registers (each thread its row)
     // no key block at all to stream (only under a block mask): O = 0
     const bool empty_stream = ok && n_kv == 0;
     bool ep_ok = ok && n_kv > 0;
-    if (ep_ok) ep_ok = mbar_wait(&pv_done[t], (n_kv - 1) & 1, abort_flag, kKernFwd, t, 2);
+    if (ep_ok) ep_ok = mbar_wait(&pv_done[t], (gt + n_kv - 1) & 1, abort_flag, kKernFwd, t, 2);
     ep_ok = __all_sync(0xffffffffu, ep_ok);
     if (ep_ok || empty_stream) {
       if (ep_ok) tc_fence_after();
@@ -550,6 +610,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
       const bool seen = l_sum > 0.f;
       const float inv_l = seen ? (DROP ? p.drop_scale : 1.0f) / l_sum : 0.f;
       const uint64_t inv2 = f2pack(inv_l, inv_l);
+      T* orow = reinterpret_cast<T*>(p.o) + (static_cast<size_t>(bh) * p.N + q_row) * HD;
 #pragma unroll
       for (int c = 0; c < HD; c += 32) {
         uint32_t o[32];
@@ -566,27 +627,21 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
           const uint64_t v = mul2(f2pack(__uint_as_float(o[2 * i]), __uint_as_float(o[2 * i + 1])), inv2);
           pk[i] = pack2<BF16>(f2lo(v), f2hi(v));
         }
-        // columns c..c+31 = 4 chunks of 16 B in box c/64, logical chunk (c%64)/8 + u
-        uint8_t* row_base = sQt + (c / 64) * L::kBoxBytes + r * 128;
+        if (q_row < p.N) {
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int chunk = ((c % 64) / 8 + u) ^ (r & 7);
-          *reinterpret_cast<uint4*>(row_base + chunk * 16) =
-              make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+          for (int u = 0; u < 4; ++u)
+            *reinterpret_cast<uint4*>(orow + c + 8 * u) =
+                make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
         }
       }
       if (q_row < p.N)
         p.lse[static_cast<size_t>(bh) * p.N + q_row] =
             seen ? (m_ref + __log2f(l_sum)) * 0.69314718055994531f : -INFINITY;
-      fence_proxy_async_smem();
+      // this pair's O has been read: the next pair's first P V may overwrite it
+      tc_fence_before();
     }
-    // every thread of the warpgroup reaches this barrier, whatever happened above
-    named_barrier_sync(1 + t, 128);
-    if (r == 0 && !*abort_flag) {
-      for (int c = 0; c < L::kChunks; ++c)
-        tma_store_3d(&p.tm_o, sQt + c * L::kBoxBytes, c * 64, qtile * 128, bh);
-      bulk_commit_group();
-      bulk_wait_group_read0();
+    ok = ok && (ep_ok || empty_stream);
+    gt += n_kv;
     }
   }
 
