@@ -258,10 +258,14 @@ def make_step(t, w, causal, W, DR, stream, fwd_ev=None, bwd_ev=None, BM=None):
 
 def time_steps(args, w, causal, rank, world, device, steps, warmup, W=0, DR=None, clocks=None, BM=None):
     """W untimed steps, then `steps` timed ones between a barrier and a
-    synchronize on both sides; CUDA events on the launching stream around the
-    whole region, around every fa_fwd and fa_bwd call, and (through the
-    library) around every launch of the forward kernel and of the backward
-    main kernel.  Returns the timings (ms; the total is the max over ranks)."""
+    synchronize on both sides, with CUDA events on the launching stream
+    around the whole region only (the step time of the headline value); then
+    the same number of steps again with events around every fa_fwd and
+    fa_bwd call and (through the library) around every launch of the forward
+    kernel and of the backward main kernel, for the breakdown (those events
+    add a few microseconds a call to the stream, so they stay out of the
+    first region).  Returns the timings (ms; the total is the max over
+    ranks)."""
     t = alloc_problem(w, rank, device, block_mask=BM is not None)
     stream = torch.cuda.current_stream(device)
     ev = lambda: torch.cuda.Event(enable_timing=True)
@@ -294,10 +298,22 @@ def time_steps(args, w, causal, rank, world, device, steps, warmup, W=0, DR=None
     torch.cuda.synchronize(device)
     t0.record(stream)
     for i in range(K):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize(device)
+    barrier()
+    # a pause, so that the breakdown runs from the same power state as the
+    # timed region (a loop right after it runs under the 1 kW power cap),
+    # then the warm-up steps again
+    time.sleep(1.0)
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize(device)
+    barrier()
+    for i in range(K):
         binding.fa_set_profile_events(binding.KERNEL_FWD, *kf_ev[i])
         binding.fa_set_profile_events(binding.KERNEL_BWD_MAIN, *kb_ev[i])
         step(i)
-    t1.record(stream)
     torch.cuda.synchronize(device)
     barrier()
     binding.fa_set_profile_events(binding.KERNEL_FWD, None, None)
@@ -590,9 +606,21 @@ def run_fp8(args, w, causal, rank, world, device):
     torch.cuda.synchronize(device)
     t0.record(stream)
     for i in range(K):
-        binding.fa_set_profile_events(binding.KERNEL_FWD, ev[2 * i], ev[2 * i + 1])
         step()
     t1.record(stream)
+    torch.cuda.synchronize(device)
+    if world > 1:
+        torch.distributed.barrier()
+    # the same steps again with events around every kernel launch (kept out
+    # of the timed region above: each event adds a little to the stream),
+    # after a pause and the warm-up, from the same power state
+    time.sleep(1.0)
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize(device)
+    for i in range(K):
+        binding.fa_set_profile_events(binding.KERNEL_FWD, ev[2 * i], ev[2 * i + 1])
+        step()
     torch.cuda.synchronize(device)
     binding.fa_set_profile_events(binding.KERNEL_FWD)
     clk = clocks.stop() if clocks else None
