@@ -261,6 +261,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
             for (int c = 0; c < L::kChunks; ++c)
               tma_load_3d(sQ + t * L::kTileBytes + c * L::kBoxBytes, &p.tm_q, q_full, c * 64,
                           (2 * I.pair + t) * 128, I.bh);
+          // the next pair's Q into L2 now, so that its load (which must wait
+          // for this pair's last S product) finds it there
+          if (it + 1 < n_items)
+            for (int t = 0; t < 2; ++t)
+              if ((2 * item_pair(it + 1) + t) * 128 < p.N)
+                for (int c = 0; c < L::kChunks; ++c)
+                  tma_prefetch_3d(&p.tm_q, c * 64, (2 * item_pair(it + 1) + t) * 128, I.bh);
         }
         auto load = [&](const CUtensorMap* map, int kblock) -> bool {
           const int s = n % L::kSlots;
@@ -540,6 +547,23 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
               hand_over(1);
               done = true;
             }
+          } else if (!DROP) {
+            // first tile of the rows: the reference is this tile's max, and
+            // the scores are still in registers
+            m_ref = m_new;
+            const float m_use = m_ref == -INFINITY ? 0.f : m_ref;
+            const uint64_t nm2 = f2pack(-m_use, -m_use);
+            uint64_t acc[4] = {0, 0, 0, 0};
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+              uint32_t pk[16];
+              p_chunk(s, q4, nm2, kv0, pk, acc);
+              tmem_st16(tm_S + q4 * 16, pk);
+              if (q4 == 1) hand_over(0);
+            }
+            l_sum += sum_acc(acc);
+            hand_over(1);
+            done = true;
           }
         }
         if (done) continue;
