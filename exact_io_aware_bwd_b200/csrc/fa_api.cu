@@ -181,7 +181,8 @@ fa_status_t launch_fwd_fp8(const fa::Fp8FwdParams& prm, cudaStream_t st) {
   const int smem = fa::Fp8FwdLayout::kDynSmem;
   fa_status_t s = opt_in_smem(kern, smem);
   if (s != FA_OK) return s;
-  const int grid = prm.n_pairs * prm.BH;
+  // one block per (head, couple of query pairs) or per (head, query pair)
+  const int grid = (prm.fold ? (prm.n_pairs + 1) / 2 : prm.n_pairs) * prm.BH;
   prof_begin(fa::kKernFwd, st);
   kern<<<grid, fa::kFwdFp8Threads, smem, st>>>(prm);
   const bool ok = cudaGetLastError() == cudaSuccess;
@@ -451,6 +452,7 @@ fa_status_t fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, flo
   prm.group = Hq / Hkv;
   prm.BH = static_cast<int>(BHq);
   prm.n_pairs = (N + 255) / 256;
+  prm.fold = prm.n_pairs <= 64 ? 1 : 0;  // as in the 16-bit forward
   prm.n_ktiles = (N + 127) / 128;
   prm.scale_log2 = static_cast<float>(c);
   prm.delta_v = descale_v;

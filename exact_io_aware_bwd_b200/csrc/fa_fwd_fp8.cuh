@@ -12,7 +12,10 @@
 // forward ("flash attention io aware", section "Online Softmax").
 //
 // Structure (the 16-bit forward's, with 8-bit operand tiles): one thread block
-// per (batch, query head, pair of 128-row query blocks), 320 threads:
+// per (batch, query head, pair of 128-row query blocks), or per couple of
+// such pairs (n-1-c, c) of a head run back to back while a head has at most
+// 64 pairs (equal work per block under a causal mask; the second pair's Q
+// load and first products overlap the first pair's tail), 320 threads:
 //   warps 0-3 / 4-7  softmax of query block 0 / 1 (thread r owns row r and
 //              tensor-memory lane r); P goes to E4M3, four keys per 32-bit
 //              tensor-memory column, over the first 32 columns of S_t.
@@ -40,6 +43,7 @@ struct Fp8FwdParams {
   CUtensorMap tm_o;  // [B*Hq][N][128] 16-bit (store), box 64 x 128
   float* lse;        // [B*Hq][N]
   int N, Hq, Hkv, group, BH, n_pairs, n_ktiles;
+  int fold;          // 1: a block runs query pairs n-1-c and c; 0: one pair
   float scale_log2;  // scale * delta_q * delta_k * log2(e)
   float delta_v;
 };
@@ -53,8 +57,9 @@ struct Fp8FwdLayout {
   static constexpr int kOffRing = 2 * kTileBytes;
   static constexpr int kOffOut = kOffRing + kSlots * kTileBytes;  // two output tiles
   static constexpr int kOffBar = kOffOut + 2 * kOutBytes;
-  // barriers: q_full, slot_full[kSlots], slot_empty[kSlots], s_full[2], p_full[2], pv_done[2], done
-  static constexpr int kNumBars = 1 + 2 * kSlots + 6 + 1;
+  // barriers: q_full, slot_full[kSlots], slot_empty[kSlots], s_full[2], p_full[2], pv_done[2], done,
+  // q_free
+  static constexpr int kNumBars = 1 + 2 * kSlots + 6 + 1 + 1;
   static constexpr int kOffTmemPtr = kOffBar + kNumBars * 8;
   static constexpr int kOffAbort = kOffTmemPtr + 4;
   static constexpr int kSmemBytes = kOffAbort + 4;
@@ -125,6 +130,7 @@ __global__ void __launch_bounds__(kFwdFp8Threads, 1) fa_fwd_fp8_kernel(const __g
   uint64_t* p_full = s_full + 2;
   uint64_t* pv_done = p_full + 2;
   uint64_t* done_bar = pv_done + 2;
+  uint64_t* q_free = done_bar + 1;  // every S product of a pair (the readers of sQ) has completed
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(sm + L::kOffTmemPtr);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::kOffAbort);
 
@@ -132,18 +138,23 @@ __global__ void __launch_bounds__(kFwdFp8Threads, 1) fa_fwd_fp8_kernel(const __g
   const int warp = tid >> 5;
   const int lane = tid & 31;
 
-  // head-major work order, query pairs with the most key blocks first
-  const int item = blockIdx.x;
-  const int bh = item / p.n_pairs;
-  const int pair = p.n_pairs - 1 - item % p.n_pairs;
+  // head-major work order, query pairs with the most key blocks first; with
+  // folding, pairs n-1-c and c of a head back to back
+  const int n_couples = p.fold ? (p.n_pairs + 1) / 2 : p.n_pairs;
+  const int bh = blockIdx.x / n_couples;
+  const int cpl = blockIdx.x % n_couples;
+  const int n_items = (!p.fold || p.n_pairs - 1 - cpl == cpl) ? 1 : 2;
+  auto item_pair = [&](int it) { return it == 0 ? p.n_pairs - 1 - cpl : cpl; };
   const int h = bh % p.Hq;
   const int b = bh / p.Hq;
   const int kvh = b * p.Hkv + h / p.group;
-  const int n_kv0 = CAUSAL ? min(2 * pair + 1, p.n_ktiles) : p.n_ktiles;
-  const int n_kv1 = CAUSAL ? min(2 * pair + 2, p.n_ktiles) : p.n_ktiles;
+  auto n_kv_of = [&](int pair, int t) {
+    return CAUSAL ? min(2 * pair + 1 + t, p.n_ktiles) : p.n_ktiles;
+  };
 
   if (tid == 0) {
     mbar_init(q_full, 1);
+    mbar_init(q_free, 1);
     for (int s = 0; s < L::kSlots; ++s) {
       mbar_init(&slot_full[s], 1);
       mbar_init(&slot_empty[s], 1);
@@ -172,10 +183,7 @@ __global__ void __launch_bounds__(kFwdFp8Threads, 1) fa_fwd_fp8_kernel(const __g
       prefetch_tensormap(&p.tm_q);
       prefetch_tensormap(&p.tm_k);
       prefetch_tensormap(&p.tm_v);
-      mbar_expect_tx(q_full, 2 * L::kTileBytes);
-      for (int t = 0; t < 2; ++t)
-        tma_load_3d(sQ + t * L::kTileBytes, &p.tm_q, q_full, 0, (2 * pair + t) * 128, bh);
-      int n = 0;
+      int n = 0;  // K/V tiles loaded (ring position), over both pairs
       auto load = [&](const CUtensorMap* map, int tile) -> bool {
         const int s = n % L::kSlots;
         if (n >= L::kSlots &&
@@ -187,9 +195,19 @@ __global__ void __launch_bounds__(kFwdFp8Threads, 1) fa_fwd_fp8_kernel(const __g
         return true;
       };
       bool ok = true;
-      for (int j = 0; ok && j < n_kv1; ++j) {
-        ok = load(&p.tm_k, j);
-        if (ok) ok = load(&p.tm_v, j);
+      for (int it = 0; ok && it < n_items; ++it) {
+        const int pair = item_pair(it);
+        // Q0, Q1 of the pair once the previous pair's S products (the last
+        // readers of sQ) have completed
+        if (it > 0) ok = mbar_wait(q_free, (it - 1) & 1, abort_flag, kKernFwdFp8, 9, 1);
+        if (!ok) break;
+        mbar_expect_tx(q_full, 2 * L::kTileBytes);
+        for (int t = 0; t < 2; ++t)
+          tma_load_3d(sQ + t * L::kTileBytes, &p.tm_q, q_full, 0, (2 * pair + t) * 128, bh);
+        for (int j = 0; ok && j < n_kv_of(pair, 1); ++j) {
+          ok = load(&p.tm_k, j);
+          if (ok) ok = load(&p.tm_v, j);
+        }
       }
     }
   } else if (warp == 8) {
@@ -205,7 +223,7 @@ __global__ void __launch_bounds__(kFwdFp8Threads, 1) fa_fwd_fp8_kernel(const __g
       return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, kKernFwdFp8, 8, site));
     };
     int n = 0;
-    bool ok = wait_all(q_full, 0, 0);
+    bool ok = true;
     auto take = [&](int& slot) -> bool {
       slot = n % L::kSlots;
       if (!wait_all(&slot_full[slot], (n / L::kSlots) & 1, 1)) return false;
@@ -224,8 +242,9 @@ __global__ void __launch_bounds__(kFwdFp8Threads, 1) fa_fwd_fp8_kernel(const __g
                    k > 0);
       umma_commit_w(&s_full[t]);
     };
-    auto issue_pv = [&](int t, int j, int vslot) -> bool {
-      if (!wait_all(&p_full[t], j & 1, 3)) return false;
+    // g: the tile's index over both pairs (barrier phase), j: its index in the pair
+    auto issue_pv = [&](int t, int g, int j, int vslot) -> bool {
+      if (!wait_all(&p_full[t], g & 1, 3)) return false;
       tc_fence_after();
       const uint32_t vo = vslot * L::kTileBytes;
 #pragma unroll
@@ -235,27 +254,36 @@ __global__ void __launch_bounds__(kFwdFp8Threads, 1) fa_fwd_fp8_kernel(const __g
       umma_commit_w(&pv_done[t]);
       return true;
     };
-    int kslot = 0, vslot = 0;
-    if (ok) ok = take(kslot);
-    if (ok) {
+    int g0 = 0, g1 = 0;  // tiles of query block 0 / 1 in the pairs before this one
+    for (int it = 0; ok && it < n_items; ++it) {
+      const int pair = item_pair(it);
+      const int n_kv0 = n_kv_of(pair, 0), n_kv1 = n_kv_of(pair, 1);
+      if (!(ok = wait_all(q_full, it & 1, 0))) break;
+      tc_fence_after();
+      int kslot = 0, vslot = 0;
+      if (!(ok = take(kslot))) break;
       if (n_kv0 > 0) issue_s(0, kslot);
       issue_s(1, kslot);
       umma_commit_w(&slot_empty[kslot]);
-      ok = take(vslot);
-    }
-    if (ok && n_kv0 > 0) ok = issue_pv(0, 0, vslot);
-    for (int j = 0; ok && j < n_kv1; ++j) {
-      const bool next1 = j + 1 < n_kv1, next0 = j + 1 < n_kv0;
-      if (next1 && !(ok = take(kslot))) break;
-      if (next0) issue_s(0, kslot);
-      if (!(ok = issue_pv(1, j, vslot))) break;
-      umma_commit_w(&slot_empty[vslot]);  // V_j: read by both PV_j
-      if (next1) {
-        issue_s(1, kslot);
-        umma_commit_w(&slot_empty[kslot]);  // K_j+1: read by both S_j+1
-        if (!(ok = take(vslot))) break;
+      if (n_kv1 == 1) umma_commit_w(q_free);  // the pair's last S
+      if (!(ok = take(vslot))) break;
+      if (n_kv0 > 0 && !(ok = issue_pv(0, g0, 0, vslot))) break;
+      for (int j = 0; ok && j < n_kv1; ++j) {
+        const bool next1 = j + 1 < n_kv1, next0 = j + 1 < n_kv0;
+        if (next1 && !(ok = take(kslot))) break;
+        if (next0) issue_s(0, kslot);
+        if (!(ok = issue_pv(1, g1 + j, j, vslot))) break;
+        umma_commit_w(&slot_empty[vslot]);  // V_j: read by both PV_j
+        if (next1) {
+          issue_s(1, kslot);
+          umma_commit_w(&slot_empty[kslot]);  // K_j+1: read by both S_j+1
+          if (j + 2 == n_kv1) umma_commit_w(q_free);  // the pair's last S
+          if (!(ok = take(vslot))) break;
+        }
+        if (next0 && !(ok = issue_pv(0, g0 + j + 1, j + 1, vslot))) break;
       }
-      if (next0 && !(ok = issue_pv(0, j + 1, vslot))) break;
+      g0 += n_kv0;
+      g1 += n_kv1;
     }
     // every MMA this warp issued completes before tensor memory is freed
     umma_commit_w(done_bar);
@@ -267,16 +295,20 @@ __global__ void __launch_bounds__(kFwdFp8Threads, 1) fa_fwd_fp8_kernel(const __g
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tm_S = tmem + t * 128 + lane_off;
     const uint32_t tm_O = tmem + 256 + t * 128 + lane_off;
-    const int qtile = 2 * pair + t;
-    const int q_row = qtile * 128 + r;
-    const int n_kv = t ? n_kv1 : n_kv0;
     const float c_log2 = p.scale_log2;
     const uint64_t c2 = f2pack(c_log2, c_log2);
+    uint8_t* sOt = sOut + t * L::kOutBytes;
+    int gt = 0;  // tiles of this query block in the pairs before this one
+    bool ok = true;
+    for (int it = 0; ok && it < n_items; ++it) {
+    const int pair = item_pair(it);
+    const int qtile = 2 * pair + t;
+    const int q_row = qtile * 128 + r;
+    const int n_kv = n_kv_of(pair, t);
     float m_ref = -INFINITY;  // in log2 units of the scaled scores
     float l_sum = 0.f;
-    bool ok = true;
     for (int j = 0; j < n_kv; ++j) {
-      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[t], j & 1, abort_flag, kKernFwdFp8, t, 0))) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[t], (gt + j) & 1, abort_flag, kKernFwdFp8, t, 0))) {
         ok = false;
         break;
       }
@@ -310,7 +342,7 @@ __global__ void __launch_bounds__(kFwdFp8Threads, 1) fa_fwd_fp8_kernel(const __g
       } else if (__any_sync(0xffffffffu, m_new > m_ref + 8.0f)) {
         // move the reference max of every row of this warp once
         // O_t += P_t,j-1 V_j-1 is done, rescaling O and l
-        if (!__all_sync(0xffffffffu, mbar_wait(&pv_done[t], (j - 1) & 1, abort_flag, kKernFwdFp8, t, 1))) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&pv_done[t], (gt + j - 1) & 1, abort_flag, kKernFwdFp8, t, 1))) {
           ok = false;
           break;
         }
@@ -363,10 +395,12 @@ __global__ void __launch_bounds__(kFwdFp8Threads, 1) fa_fwd_fp8_kernel(const __g
       mbar_arrive(&p_full[t]);
     }
     // epilogue: O * delta_v / l -> 16-bit, staged in this block's output tile, TMA store
-    uint8_t* sOt = sOut + t * L::kOutBytes;
     bool ep_ok = ok && n_kv > 0;
-    if (ep_ok) ep_ok = mbar_wait(&pv_done[t], (n_kv - 1) & 1, abort_flag, kKernFwdFp8, t, 2);
+    if (ep_ok) ep_ok = mbar_wait(&pv_done[t], (gt + n_kv - 1) & 1, abort_flag, kKernFwdFp8, t, 2);
     ep_ok = __all_sync(0xffffffffu, ep_ok);
+    // the previous pair's store has read the staging tile (its storing
+    // thread waited for that before reaching this barrier)
+    if (it > 0) named_barrier_sync(1 + t, 128);
     if (ep_ok) {
       tc_fence_after();
       const float f = p.delta_v / l_sum;
@@ -402,6 +436,9 @@ __global__ void __launch_bounds__(kFwdFp8Threads, 1) fa_fwd_fp8_kernel(const __g
         tma_store_3d(&p.tm_o, sOt + c * L::kOutBoxBytes, c * 64, qtile * 128, bh);
       bulk_commit_group();
       bulk_wait_group_read0();
+    }
+    ok = ok && ep_ok;
+    gt += n_kv;
     }
   }
 
