@@ -47,15 +47,15 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # the backward main kernel on the default workload, from one ncu capture of
 # that kernel, with a digest of the kernel sources it was taken on: reported
 # only while the sources are unchanged.
-PROFILED_TRAFFIC = {"workload": "mha4k", "bytes": 1296243200, "sources_sha256_16": "47660ecea5a2a1c9",
+PROFILED_TRAFFIC = {"workload": "mha4k", "bytes": 1294966784, "sources_sha256_16": "ad6562f226110961",
                     "sources": ("exact_io_aware_bwd_b200/csrc/fa_bwd.cuh",
                                 "exact_io_aware_bwd_b200/csrc/sm100.cuh")}
 # The same for the forward kernel (one launch on the default workload).
-PROFILED_TRAFFIC_FWD = {"workload": "mha4k", "bytes": 520983040, "sources_sha256_16": "97db3872e532d046",
+PROFILED_TRAFFIC_FWD = {"workload": "mha4k", "bytes": 526888448, "sources_sha256_16": "e00471812f442535",
                         "sources": ("exact_io_aware_bwd_b200/csrc/fa_fwd.cuh",
                                     "exact_io_aware_bwd_b200/csrc/sm100.cuh")}
 # The same for the FP8 forward kernel (one launch on the 4K-token MHA shape).
-PROFILED_TRAFFIC_FP8 = {"workload": "mha4k", "bytes": 307079936, "sources_sha256_16": "49abecf182bf2acc",
+PROFILED_TRAFFIC_FP8 = {"workload": "mha4k", "bytes": 305240832, "sources_sha256_16": "481515a16f74b0cd",
                         "sources": ("exact_io_aware_bwd_b200/csrc/fa_fwd_fp8.cuh",
                                     "exact_io_aware_bwd_b200/csrc/sm100.cuh")}
 
