@@ -686,17 +686,32 @@ fa_status_t fa_decode_paged(const void* q, const void* k_cache, const void* v_ca
   prm.part_ml = prm.part_o + rows * prm.S * d;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const bool bf = dtype == FA_BF16;
-  const dim3 grid(static_cast<unsigned>(prm.S), static_cast<unsigned>(Hkv), static_cast<unsigned>(B));
+  const int R = (Hq / Hkv) * Nq;
+  const int rb = R <= 4 ? 4 : R <= 8 ? 8 : R <= 16 ? 16 : 32;
+  // q as [B * Hq * Nq][d]; a box is the NP (rows padded to 16 or 32) rows
+  // that start at an item's first row
+  const int np = rb < 16 ? 16 : rb;
+  if (!make_map(&prm.tm_q, q, tdt, 2, d, static_cast<uint64_t>(B) * Hq * Nq, 1, 64, np)) return FA_ERR_CUDA;
+  const int64_t n_work = static_cast<int64_t>(B) * Hkv * prm.S;
+  if (n_work > INT32_MAX) return FA_ERR_UNSUPPORTED;
+  const int sms = sm_count();
+  if (sms <= 0) return FA_ERR_CUDA;
   auto run = [&](auto split_kern, auto merge_kern, int smem) -> fa_status_t {
     fa_status_t r = opt_in_smem(split_kern, smem);
     if (r != FA_OK) return r;
+    // persistent: as many blocks as fit on the GPU at once, each taking
+    // work items (splits) in turn
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, split_kern, fa::kDecodeThreads, smem) !=
+            cudaSuccess ||
+        per_sm <= 0)
+      return FA_ERR_CUDA;
+    const int grid = static_cast<int>(std::min<int64_t>(n_work, static_cast<int64_t>(sms) * per_sm));
     split_kern<<<grid, fa::kDecodeThreads, smem, st>>>(prm);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
     merge_kern<<<static_cast<unsigned>(rows), d, 0, st>>>(prm);
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
   };
-  const int R = (Hq / Hkv) * Nq;
-  const int rb = R <= 4 ? 4 : R <= 8 ? 8 : R <= 16 ? 16 : 32;
 #define FA_DECODE_RUN(HD, BFV, RBV)                                                                  \
   run(fa::fa_decode_split_kernel<HD, BFV, RBV>, fa::fa_decode_merge_kernel<HD, BFV>, \
       fa::DecodeLayout<HD, RBV>::kDynSmem)

@@ -53,6 +53,7 @@ constexpr int kDecodeSMs = 148;          // B200
 struct DecodeParams {
   CUtensorMap tm_k;       // K cache as [num_pages * Hkv][P][d], box 64 features x P rows
   CUtensorMap tm_v;       // V cache, the same
+  CUtensorMap tm_q;       // q as [B * Hq * Nq][d], box 64 features x NP rows
   const void* q;          // [B][Hq][Nq][d]
   const int* table;       // [B][max_pages]
   const int* lens;        // [B]
@@ -111,10 +112,11 @@ struct DecodeLayout {
   static constexpr int kOffP = kOffQ + kChunks * kQChunk;
   static constexpr int kOffFlag = kOffP + 2 * kPBytes;   // int [2][4]
   static constexpr int kOffMax = kOffFlag + 8 * 4;       // float [2][4][32]
-  static constexpr int kOffSum = kOffMax + 2 * 4 * 32 * 4;  // float [4][32]
-  static constexpr int kOffBar = kOffSum + 4 * 32 * 4;
-  // kv_full[slots], kv_empty[slots], s_full[2], p_full[2], pv_done[2], done
-  static constexpr int kNumBars = 2 * kSlots + 7;
+  static constexpr int kOffSum = kOffMax + 2 * 4 * 32 * 4;  // float [2][4][32]
+  static constexpr int kOffBar = kOffSum + 2 * 4 * 32 * 4;
+  // kv_full[slots], kv_empty[slots], s_full[2], p_full[2], pv_done[2], done,
+  // q_full, q_empty
+  static constexpr int kNumBars = 2 * kSlots + 9;
   static constexpr int kOffTmemPtr = kOffBar + kNumBars * 8;
   static constexpr int kOffAbort = kOffTmemPtr + 4;
   static constexpr int kBytes = kOffAbort + 4;
@@ -160,6 +162,31 @@ __device__ __forceinline__ void tmem_st_n(uint32_t taddr, const uint32_t* r) {
   }
 }
 
+// One work item: a split of the pages of one sequence and kv head.
+struct DecodeItem {
+  int b, g, split, Lb, pg0, pg1, n_tiles;
+  bool len_ok;
+};
+
+__device__ __forceinline__ DecodeItem decode_item(const DecodeParams& p, int w) {
+  DecodeItem it;
+  it.split = w % p.S;
+  it.g = (w / p.S) % p.Hkv;
+  it.b = w / (p.S * p.Hkv);
+  const int P = p.P, ppt = kDecodeTile / P;
+  it.Lb = p.lens[it.b];
+  it.len_ok = it.Lb >= p.Nq && it.Lb <= p.max_pages * P;
+  const int n_pages = it.len_ok ? (it.Lb + P - 1) / P : 0;
+  it.pg0 = it.split * p.pages_per_split;  // pages_per_split is a multiple of ppt
+  it.pg1 = min(n_pages, it.pg0 + p.pages_per_split);
+  it.n_tiles = it.pg1 > it.pg0 ? (it.pg1 - it.pg0 + ppt - 1) / ppt : 0;
+  return it;
+}
+
+// Persistent: a block takes work items blockIdx.x, blockIdx.x + gridDim.x,
+// ...  The tile ring, the tensor-memory buffers and the barrier phases run on
+// across items (tiles are numbered over the block's items), so the fill of
+// the ring and the pipeline's start are paid once per block, not per split.
 // RB: compile-time bound on the rows (4, 8, 16 or 32, the smallest >= R), so
 // the per-row loops unroll to the rows that exist.
 template <int HD, bool BF16, int RB>
@@ -183,20 +210,15 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) fa_decode_split_kernel(cons
   uint64_t* p_full = s_full + 2;
   uint64_t* pv_done = p_full + 2;
   uint64_t* done_bar = pv_done + 2;
+  uint64_t* q_full = done_bar + 1;   // the q rows of an item landed
+  uint64_t* q_empty = q_full + 1;    // the S products of an item (readers of sQ) completed
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(sm + L::kOffTmemPtr);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::kOffAbort);
 
-  const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int G = p.Hq / p.Hkv, R = G * p.Nq, P = p.P;
   const int ppt = kDecodeTile / P;  // pages per tile
-  const int Lb = p.lens[b];
-  const bool len_ok = Lb >= p.Nq && Lb <= p.max_pages * P;
-  if (!len_ok && split == 0 && g == 0 && tid == 0) record_error(kStatusBadInput, kKernDecode, 0, 0);
-  const int n_pages = len_ok ? (Lb + P - 1) / P : 0;
-  const int pg0 = split * p.pages_per_split;  // pages_per_split is a multiple of ppt
-  const int pg1 = min(n_pages, pg0 + p.pages_per_split);
-  const int n_tiles = pg1 > pg0 ? (pg1 - pg0 + ppt - 1) / ppt : 0;  // tiles of this split
+  const int n_work = p.B * p.Hkv * p.S;
 
   if (tid == 0) {
     for (int s = 0; s < NS; ++s) {
@@ -209,6 +231,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) fa_decode_split_kernel(cons
       mbar_init(&pv_done[i], 1);
     }
     mbar_init(done_bar, 1);
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -216,20 +240,6 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) fa_decode_split_kernel(cons
     tmem_alloc(tmem_ptr, 128);
     tmem_relinquish();
   }
-  // Q rows of the block (row r: head g*G + r / Nq, token r % Nq) into the
-  // K-major, 128-byte-swizzled B operand of S^T = K Q^T; padding rows are
-  // zero.
-  for (int i = tid; i < NP * (HD / 8); i += kDecodeThreads) {
-    const int r = i / (HD / 8), c16 = i % (HD / 8);
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (r < R) {
-      const int h = g * G + r / p.Nq, t = r % p.Nq;
-      const T* qr = reinterpret_cast<const T*>(p.q) + ((static_cast<size_t>(b) * p.Hq + h) * p.Nq + t) * HD;
-      v = *reinterpret_cast<const uint4*>(qr + c16 * 8);
-    }
-    *reinterpret_cast<uint4*>(sQ + (c16 >> 3) * L::kQChunk + r * 128 + (((c16 & 7) ^ (r & 7)) << 4)) = v;
-  }
-  fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -241,35 +251,54 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) fa_decode_split_kernel(cons
     if (lane == 0) {
       prefetch_tensormap(&p.tm_k);
       prefetch_tensormap(&p.tm_v);
-      int issued = 0;
-      for (int j = 0; j < n_tiles; ++j) {
-        const int s = j % NS;
-        if (j >= NS && !mbar_wait(&kv_empty[s], ((j / NS) - 1) & 1, abort_flag, kKernDecode, 4, 0)) break;
-        mbar_expect_tx(&kv_full[s], static_cast<uint32_t>(L::kSlotBytes));
-        uint8_t* slot = sm + s * L::kSlotBytes;
-        for (int pp = 0; pp < ppt; ++pp) {
-          const int pg = pg0 + j * ppt + pp;
-          int outer = -1;  // outside the tensor: the box reads as zeros
-          if (pg < pg1) {
-            const int phys = p.table[static_cast<size_t>(b) * p.max_pages + pg];
-            if (phys >= 0 && phys < p.num_pages)
-              outer = phys * p.Hkv + g;
-            else
-              record_error(kStatusBadInput, kKernDecode, 4, 1);
-          }
+      prefetch_tensormap(&p.tm_q);
+      int j = 0;   // tiles issued, over the block's items
+      int qi = 0;  // items with tiles so far
+      bool ok = true;
+      for (int w = blockIdx.x; ok && w < n_work; w += gridDim.x) {
+        const DecodeItem I = decode_item(p, w);
+        if (!I.len_ok && I.split == 0 && I.g == 0) record_error(kStatusBadInput, kKernDecode, 4, 0);
+        if (I.n_tiles == 0) continue;
+        // the item's q rows (row r: head g*G + r / Nq, token r % Nq; rows
+        // past R are the next heads' or zeros, and their columns of S^T and
+        // O^T are never read), once the previous item's S products are done
+        if (qi > 0 && !(ok = mbar_wait(q_empty, (qi - 1) & 1, abort_flag, kKernDecode, 4, 3))) break;
+        mbar_expect_tx(q_full, static_cast<uint32_t>(L::kChunks * L::kQChunk));
+        for (int c = 0; c < L::kChunks; ++c)
+          tma_load_3d(sQ + c * L::kQChunk, &p.tm_q, q_full, c * 64, (I.b * p.Hq + I.g * G) * p.Nq, 0);
+        ++qi;
+        for (int jj = 0; jj < I.n_tiles; ++jj) {
+          const int s = j % NS;
+          if (j >= NS && !(ok = mbar_wait(&kv_empty[s], ((j / NS) - 1) & 1, abort_flag, kKernDecode, 4, 0)))
+            break;
+          mbar_expect_tx(&kv_full[s], static_cast<uint32_t>(L::kSlotBytes));
+          uint8_t* slot = sm + s * L::kSlotBytes;
+          for (int pp = 0; pp < ppt; ++pp) {
+            const int pg = I.pg0 + jj * ppt + pp;
+            int outer = -1;  // outside the tensor: the box reads as zeros
+            if (pg < I.pg1) {
+              const int phys = p.table[static_cast<size_t>(I.b) * p.max_pages + pg];
+              if (phys >= 0 && phys < p.num_pages)
+                outer = phys * p.Hkv + I.g;
+              else
+                record_error(kStatusBadInput, kKernDecode, 4, 1);
+            }
 #pragma unroll
-          for (int c = 0; c < L::kChunks; ++c) {
-            tma_load_3d(slot + c * L::kChunkBytes + pp * P * 128, &p.tm_v, &kv_full[s], c * 64, 0, outer);
-            tma_load_3d(slot + (L::kChunks + c) * L::kChunkBytes + pp * P * 128, &p.tm_k, &kv_full[s], c * 64,
-                        0, outer);
+            for (int c = 0; c < L::kChunks; ++c) {
+              tma_load_3d(slot + c * L::kChunkBytes + pp * P * 128, &p.tm_v, &kv_full[s], c * 64, 0, outer);
+              tma_load_3d(slot + (L::kChunks + c) * L::kChunkBytes + pp * P * 128, &p.tm_k, &kv_full[s],
+                          c * 64, 0, outer);
+            }
           }
+          ++j;
         }
-        issued = j + 1;
       }
-      // the copies of the last tile issued into each slot land before the
-      // block exits (all earlier ones were waited for by the MMA warp)
-      for (int j = issued > NS ? issued - NS : 0; j < issued; ++j)
-        mbar_wait_drain(&kv_full[j % NS], (j / NS) & 1, kKernDecode, 4, 2);
+      // the copies of the last tile issued into each slot, and the last q
+      // rows, land before the block exits (all earlier ones were waited for
+      // by the MMA warp)
+      for (int jx = j > NS ? j - NS : 0; jx < j; ++jx)
+        mbar_wait_drain(&kv_full[jx % NS], (jx / NS) & 1, kKernDecode, 4, 2);
+      if (qi > 0) mbar_wait_drain(q_full, (qi - 1) & 1, kKernDecode, 4, 4);
     }
   } else if (warp == 5) {
     // ------------------------------------------------------------ MMA issuer
@@ -282,34 +311,46 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) fa_decode_split_kernel(cons
     auto wait_all = [&](uint64_t* bar, uint32_t parity, uint32_t site) -> bool {
       return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, kKernDecode, 5, site));
     };
-    auto issue_pv = [&](int t) -> bool {
+    // O^T += V^T P^T of tile t (over the block's items); `first`: the item's
+    // first tile, which starts O^T afresh
+    auto issue_pv = [&](int t, bool first) -> bool {
       if (!wait_all(&p_full[t & 1], (t >> 1) & 1, 1)) return false;
       tc_fence_after();
       const uint32_t so = (t % NS) * L::kSlotBytes, po = (t & 1) * L::kPBytes;
 #pragma unroll
       for (int k = 0; k < kDecodeTile / 16; ++k)
         umma_ss_w(tm_O, sdesc_add(dVt, so + k * 2048), sdesc_add(dP, po + (k >> 2) * L::kPChunk + (k & 3) * 32),
-                  kIdO, (t > 0 || k > 0) ? 1u : 0u);
+                  kIdO, (!first || k > 0) ? 1u : 0u);
       umma_commit_w(&kv_empty[t % NS]);
       umma_commit_w(&pv_done[t & 1]);
       return true;
     };
     bool ok = true;
-    for (int j = 0; ok && j < n_tiles; ++j) {
-      const int s = j % NS;
-      if (!(ok = wait_all(&kv_full[s], (j / NS) & 1, 0))) break;
+    int j = 0;   // tiles, over the block's items
+    int qi = 0;  // items with tiles so far
+    for (int w = blockIdx.x; ok && w < n_work; w += gridDim.x) {
+      const DecodeItem I = decode_item(p, w);
+      if (I.n_tiles == 0) continue;
+      if (!(ok = wait_all(q_full, qi & 1, 2))) break;
       tc_fence_after();
-      const uint32_t so = s * L::kSlotBytes;
-      // S^T_j lands in buffer j % 2, last read by the softmax of tile j - 2,
-      // whose P the PV product issued before this one waited for
+      ++qi;
+      for (int jj = 0; jj < I.n_tiles; ++jj, ++j) {
+        const int s = j % NS;
+        if (!(ok = wait_all(&kv_full[s], (j / NS) & 1, 0))) break;
+        tc_fence_after();
+        const uint32_t so = s * L::kSlotBytes;
+        // S^T_j lands in buffer j % 2, last read by the softmax of tile j - 2,
+        // whose P the PV product issued before this one waited for
 #pragma unroll
-      for (int k = 0; k < HD / 16; ++k)
-        umma_ss_w(tmem + (j & 1) * NP, sdesc_add(dK, so + (k >> 2) * L::kChunkBytes + (k & 3) * 32),
-                  sdesc_add(dQ, (k >> 2) * L::kQChunk + (k & 3) * 32), kIdS, k > 0 ? 1u : 0u);
-      umma_commit_w(&s_full[j & 1]);
-      if (j > 0) ok = issue_pv(j - 1);
+        for (int k = 0; k < HD / 16; ++k)
+          umma_ss_w(tmem + (j & 1) * NP, sdesc_add(dK, so + (k >> 2) * L::kChunkBytes + (k & 3) * 32),
+                    sdesc_add(dQ, (k >> 2) * L::kQChunk + (k & 3) * 32), kIdS, k > 0 ? 1u : 0u);
+        umma_commit_w(&s_full[j & 1]);
+        if (jj + 1 == I.n_tiles) umma_commit_w(q_empty);  // the item's last S: sQ may be refilled
+        if (jj > 0 && !(ok = issue_pv(j - 1, jj == 1))) break;
+      }
+      if (ok) ok = issue_pv(j - 1, I.n_tiles == 1);
     }
-    if (ok && n_tiles > 0) issue_pv(n_tiles - 1);
     // every MMA this warp issued completes before tensor memory is freed
     umma_commit_w(done_bar);
     mbar_wait_drain(done_bar, 0, kKernDecode, 5, 3);
@@ -320,161 +361,171 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) fa_decode_split_kernel(cons
     const int i = tid;
     const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
     const float c_log2 = p.scale_log2;
-    float ref[RB], lp[RB];
-#pragma unroll
-    for (int r = 0; r < RB; ++r) {
-      ref[r] = -INFINITY;
-      lp[r] = 0.f;
-    }
-    // whether this thread's key of tile jj sits in a page that was loaded
-    auto page_loaded = [&](int jj) -> bool {
-      const int pg = pg0 + jj * ppt + i / P;
-      if (pg >= pg1) return false;
-      const int phys = __ldg(p.table + static_cast<size_t>(b) * p.max_pages + pg);
-      return phys >= 0 && phys < p.num_pages;
-    };
-    bool loaded_next = n_tiles > 0 ? page_loaded(0) : false;
     bool ok = true;
-    for (int j = 0; j < n_tiles; ++j) {
-      const int buf = j & 1;
-      const bool loaded = loaded_next;
-      if (j + 1 < n_tiles) loaded_next = page_loaded(j + 1);
-      // warp-uniform, as the tensor-memory loads below must be
-      const bool fail = !__all_sync(0xffffffffu, mbar_wait(&s_full[buf], (j >> 1) & 1, abort_flag, kKernDecode, 0, 0));
-      tc_fence_after();
-      uint32_t sv[RB];
-      if (!fail) {
-        tmem_ld_n<RB>(tmem + buf * NP + lane_off, sv);
-        tmem_ld_wait();
-      }
-      const int key = (pg0 + j * ppt) * P + i;
-      float t[RB];
-      bool need = false;
+    int j = 0;   // tiles, over the block's items
+    int ei = 0;  // items, over the block
+    for (int w = blockIdx.x; ok && w < n_work; w += gridDim.x, ++ei) {
+      const DecodeItem I = decode_item(p, w);
+      float ref[RB], lp[RB];
 #pragma unroll
       for (int r = 0; r < RB; ++r) {
-        t[r] = -INFINITY;
-        if (r < R && !fail) {
-          const bool vis = loaded && key <= Lb - p.Nq + r % p.Nq;
-          t[r] = vis ? __uint_as_float(sv[r]) * c_log2 : -INFINITY;
-          need |= t[r] > ref[r] + 8.f;
+        ref[r] = -INFINITY;
+        lp[r] = 0.f;
+      }
+      // whether this thread's key of the item's tile jj sits in a page that was loaded
+      auto page_loaded = [&](int jj) -> bool {
+        const int pg = I.pg0 + jj * ppt + i / P;
+        if (pg >= I.pg1) return false;
+        const int phys = __ldg(p.table + static_cast<size_t>(I.b) * p.max_pages + pg);
+        return phys >= 0 && phys < p.num_pages;
+      };
+      bool loaded_next = I.n_tiles > 0 ? page_loaded(0) : false;
+      for (int jj = 0; jj < I.n_tiles; ++jj, ++j) {
+        const int buf = j & 1;
+        const bool loaded = loaded_next;
+        if (jj + 1 < I.n_tiles) loaded_next = page_loaded(jj + 1);
+        // warp-uniform, as the tensor-memory loads below must be
+        const bool fail = !__all_sync(0xffffffffu, mbar_wait(&s_full[buf], (j >> 1) & 1, abort_flag, kKernDecode, 0, 0));
+        tc_fence_after();
+        uint32_t sv[RB];
+        if (!fail) {
+          tmem_ld_n<RB>(tmem + buf * NP + lane_off, sv);
+          tmem_ld_wait();
         }
-      }
-      // One decision for all 128 threads: whether a reference max moves (and
-      // whether a wait failed).  Every softmax thread reaches every barrier.
-      const bool wneed = __any_sync(0xffffffffu, need), wfail = __any_sync(0xffffffffu, fail);
-      if (lane == 0) sFlag[buf * 4 + warp] = (wneed ? 1 : 0) | (wfail ? 2 : 0);
-      named_barrier_sync(1, 128);
-      const int f = sFlag[buf * 4 + 0] | sFlag[buf * 4 + 1] | sFlag[buf * 4 + 2] | sFlag[buf * 4 + 3];
-      if (f & 2) {
-        ok = false;
-        break;
-      }
-      if (f & 1) {
-        // per-row maxima of the tile over the 128 keys
+        const int key = (I.pg0 + jj * ppt) * P + i;
+        float t[RB];
+        bool need = false;
 #pragma unroll
         for (int r = 0; r < RB; ++r) {
-          if (r < R) {
-            float m = t[r];
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-            if (lane == 0) sMax[(buf * 4 + warp) * 32 + r] = m;
+          t[r] = -INFINITY;
+          if (r < R && !fail) {
+            const bool vis = loaded && key <= I.Lb - p.Nq + r % p.Nq;
+            t[r] = vis ? __uint_as_float(sv[r]) * c_log2 : -INFINITY;
+            need |= t[r] > ref[r] + 8.f;
           }
         }
+        // One decision for all 128 threads: whether a reference max moves (and
+        // whether a wait failed).  Every softmax thread reaches every barrier.
+        const bool wneed = __any_sync(0xffffffffu, need), wfail = __any_sync(0xffffffffu, fail);
+        if (lane == 0) sFlag[buf * 4 + warp] = (wneed ? 1 : 0) | (wfail ? 2 : 0);
         named_barrier_sync(1, 128);
-        float fac[RB];
+        const int f = sFlag[buf * 4 + 0] | sFlag[buf * 4 + 1] | sFlag[buf * 4 + 2] | sFlag[buf * 4 + 3];
+        if (f & 2) {
+          ok = false;
+          break;
+        }
+        if (f & 1) {
+          // per-row maxima of the tile over the 128 keys
+#pragma unroll
+          for (int r = 0; r < RB; ++r) {
+            if (r < R) {
+              float m = t[r];
+#pragma unroll
+              for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+              if (lane == 0) sMax[(buf * 4 + warp) * 32 + r] = m;
+            }
+          }
+          named_barrier_sync(1, 128);
+          float fac[RB];
+#pragma unroll
+          for (int r = 0; r < RB; ++r) {
+            fac[r] = 1.f;
+            if (r < R) {
+              const float* mr = sMax + buf * 4 * 32 + r;
+              const float nm = fmaxf(fmaxf(ref[r], fmaxf(mr[0], mr[32])), fmaxf(mr[64], mr[96]));
+              if (nm != ref[r]) fac[r] = ref[r] == -INFINITY ? 0.f : ex2_approx(ref[r] - nm);
+              ref[r] = nm;
+              lp[r] *= fac[r];
+            }
+          }
+          // O^T holds the products of the item's tiles before this one: once
+          // they are complete, scale its row columns (this thread: feature lane i)
+          if (jj > 0) {
+            if (__all_sync(0xffffffffu, mbar_wait(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, kKernDecode, 0, 1))) {
+              tc_fence_after();
+              uint32_t ov[RB];
+              tmem_ld_n<RB>(tm_O + lane_off, ov);
+              tmem_ld_wait();
+#pragma unroll
+              for (int r = 0; r < RB; ++r) ov[r] = __float_as_uint(__uint_as_float(ov[r]) * fac[r]);
+              tmem_st_n<RB>(tm_O + lane_off, ov);
+              tmem_st_wait();
+            }
+          }
+        }
+        // P of this thread's key for every row; buffer `buf` was last read by
+        // the PV product of tile j - 2
+        float pr[RB];
 #pragma unroll
         for (int r = 0; r < RB; ++r) {
-          fac[r] = 1.f;
-          if (r < R) {
-            const float* mr = sMax + buf * 4 * 32 + r;
-            const float nm = fmaxf(fmaxf(ref[r], fmaxf(mr[0], mr[32])), fmaxf(mr[64], mr[96]));
-            if (nm != ref[r]) fac[r] = ref[r] == -INFINITY ? 0.f : ex2_approx(ref[r] - nm);
-            ref[r] = nm;
-            lp[r] *= fac[r];
+          pr[r] = 0.f;
+          if (r < R && t[r] != -INFINITY) {
+            pr[r] = ex2_approx(t[r] - ref[r]);
+            lp[r] += pr[r];
           }
         }
-        // O^T holds the products of tiles 0 .. j-1: once they are complete,
-        // scale its row columns (this thread: feature lane i)
-        if (j > 0) {
-          if (__all_sync(0xffffffffu, mbar_wait(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, kKernDecode, 0, 1))) {
-            tc_fence_after();
-            uint32_t ov[RB];
-            tmem_ld_n<RB>(tm_O + lane_off, ov);
-            tmem_ld_wait();
+        if (j >= 2) mbar_wait(&pv_done[buf], ((j - 2) >> 1) & 1, abort_flag, kKernDecode, 0, 2);
+        // P[row][key] in the K-major, 128-byte-swizzled B operand of V^T P^T:
+        // 64 keys (128 bytes) per row and box; the 32 lanes of a warp write 64
+        // consecutive bytes of one row at a time
+        uint8_t* pb = sP + buf * L::kPBytes + (i >> 6) * L::kPChunk + (i & 7) * 2;
 #pragma unroll
-            for (int r = 0; r < RB; ++r) ov[r] = __float_as_uint(__uint_as_float(ov[r]) * fac[r]);
-            tmem_st_n<RB>(tm_O + lane_off, ov);
-            tmem_st_wait();
-          }
-        }
+        for (int r = 0; r < RB; ++r)
+          if (r < R) *reinterpret_cast<T*>(pb + r * 128 + ((((i & 63) >> 3) ^ (r & 7)) << 4)) = static_cast<T>(pr[r]);
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(&p_full[buf]);
       }
-      // P of this thread's key for every row; buffer `buf` was last read by
-      // the PV product of tile j - 2
-      float pr[RB];
-#pragma unroll
-      for (int r = 0; r < RB; ++r) {
-        pr[r] = 0.f;
-        if (r < R && t[r] != -INFINITY) {
-          pr[r] = ex2_approx(t[r] - ref[r]);
-          lp[r] += pr[r];
-        }
-      }
-      if (j >= 2) mbar_wait(&pv_done[buf], ((j - 2) >> 1) & 1, abort_flag, kKernDecode, 0, 2);
-      // P[row][key] in the K-major, 128-byte-swizzled B operand of V^T P^T:
-      // 64 keys (128 bytes) per row and box; the 32 lanes of a warp write 64
-      // consecutive bytes of one row at a time
-      uint8_t* pb = sP + buf * L::kPBytes + (i >> 6) * L::kPChunk + (i & 7) * 2;
-#pragma unroll
-      for (int r = 0; r < RB; ++r)
-        if (r < R) *reinterpret_cast<T*>(pb + r * 128 + ((((i & 63) >> 3) ^ (r & 7)) << 4)) = static_cast<T>(pr[r]);
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(&p_full[buf]);
-    }
-    // ---------------------------------------------------------------- epilogue
-    // l of each row: the sum of the 128 threads' partial sums
-#pragma unroll
-    for (int r = 0; r < RB; ++r) {
-      if (r < R) {
-        float s = lp[r];
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-        if (lane == 0) sSum[warp * 32 + r] = s;
-      }
-    }
-    named_barrier_sync(1, 128);
-    bool have = ok && n_tiles > 0;
-    if (have) {
-      have = mbar_wait(&pv_done[(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1, abort_flag, kKernDecode, 0, 3);
-      tc_fence_after();
-    }
-    uint32_t ov[RB];
-#pragma unroll
-    for (int r = 0; r < RB; ++r) ov[r] = 0u;
-    if (__all_sync(0xffffffffu, have)) {
-      tmem_ld_n<RB>(tm_O + lane_off, ov);
-      tmem_ld_wait();
-    }
-    if (i < HD) {
+      // ---------------------------------------------------------------- epilogue of the item
+      // l of each row: the sum of the 128 threads' partial sums (sSum is
+      // double-buffered by item, so no thread still reads the previous one's)
+      float* ss = sSum + (ei & 1) * 4 * 32;
 #pragma unroll
       for (int r = 0; r < RB; ++r) {
         if (r < R) {
-          const int h = g * G + r / p.Nq, t = r % p.Nq;
-          const size_t row = ((static_cast<size_t>(b) * p.Hq + h) * p.Nq + t) * p.S + split;
-          p.part_o[row * HD + i] = __uint_as_float(ov[r]);
+          float sum = lp[r];
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+          if (lane == 0) ss[warp * 32 + r] = sum;
         }
       }
-    }
-    if (i < R) {
-      float m = -INFINITY;
+      named_barrier_sync(1, 128);
+      bool have = ok && I.n_tiles > 0;
+      if (have) {
+        have = mbar_wait(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, kKernDecode, 0, 3);
+        tc_fence_after();
+      }
+      uint32_t ov[RB];
 #pragma unroll
-      for (int r = 0; r < RB; ++r)
-        if (r == i) m = ref[r];
-      const float l = sSum[i] + sSum[32 + i] + sSum[64 + i] + sSum[96 + i];
-      const int h = g * G + i / p.Nq, t = i % p.Nq;
-      const size_t row = ((static_cast<size_t>(b) * p.Hq + h) * p.Nq + t) * p.S + split;
-      p.part_ml[row * 2 + 0] = l > 0.f ? m : -INFINITY;
-      p.part_ml[row * 2 + 1] = l;
+      for (int r = 0; r < RB; ++r) ov[r] = 0u;
+      if (__all_sync(0xffffffffu, have)) {
+        tmem_ld_n<RB>(tm_O + lane_off, ov);
+        tmem_ld_wait();
+      }
+      if (i < HD) {
+#pragma unroll
+        for (int r = 0; r < RB; ++r) {
+          if (r < R) {
+            const int h = I.g * G + r / p.Nq, tq = r % p.Nq;
+            const size_t row = ((static_cast<size_t>(I.b) * p.Hq + h) * p.Nq + tq) * p.S + I.split;
+            p.part_o[row * HD + i] = __uint_as_float(ov[r]);
+          }
+        }
+      }
+      if (i < R) {
+        float m = -INFINITY;
+#pragma unroll
+        for (int r = 0; r < RB; ++r)
+          if (r == i) m = ref[r];
+        const float l = ss[i] + ss[32 + i] + ss[64 + i] + ss[96 + i];
+        const int h = I.g * G + i / p.Nq, tq = i % p.Nq;
+        const size_t row = ((static_cast<size_t>(I.b) * p.Hq + h) * p.Nq + tq) * p.S + I.split;
+        p.part_ml[row * 2 + 0] = l > 0.f ? m : -INFINITY;
+        p.part_ml[row * 2 + 1] = l;
+      }
+      // this item's O^T has been read: the next item's first P V (after
+      // this thread's next arrival on p_full) may overwrite it
+      tc_fence_before();
     }
   }
 
