@@ -47,16 +47,21 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # the backward main kernel on the default workload, from one ncu capture of
 # that kernel, with a digest of the kernel sources it was taken on: reported
 # only while the sources are unchanged.
-PROFILED_TRAFFIC = {"workload": "mha4k", "bytes": 1294966784, "sources_sha256_16": "ad6562f226110961",
+PROFILED_TRAFFIC = {"workload": "mha4k", "bytes": 1295312384, "sources_sha256_16": "ad6562f226110961",
                     "sources": ("exact_io_aware_bwd_b200/csrc/fa_bwd.cuh",
                                 "exact_io_aware_bwd_b200/csrc/sm100.cuh")}
 # The same for the forward kernel (one launch on the default workload).
-PROFILED_TRAFFIC_FWD = {"workload": "mha4k", "bytes": 526888448, "sources_sha256_16": "e00471812f442535",
+PROFILED_TRAFFIC_FWD = {"workload": "mha4k", "bytes": 520397824, "sources_sha256_16": "ce889865de72d6d5",
                         "sources": ("exact_io_aware_bwd_b200/csrc/fa_fwd.cuh",
                                     "exact_io_aware_bwd_b200/csrc/sm100.cuh")}
 # The same for the FP8 forward kernel (one launch on the 4K-token MHA shape).
 PROFILED_TRAFFIC_FP8 = {"workload": "mha4k", "bytes": 305240832, "sources_sha256_16": "481515a16f74b0cd",
                         "sources": ("exact_io_aware_bwd_b200/csrc/fa_fwd_fp8.cuh",
+                                    "exact_io_aware_bwd_b200/csrc/sm100.cuh")}
+# The same for one decode step (split and merge launch) at 16K cached tokens.
+PROFILED_TRAFFIC_DEC = {"workload": "decode B=32 Hq=32 Hkv=8 Nq=1 d=128 L=16384 page=64", "bytes": 2155432448,
+                        "sources_sha256_16": "028c681ba0cdedd6",
+                        "sources": ("exact_io_aware_bwd_b200/csrc/fa_decode.cuh",
                                     "exact_io_aware_bwd_b200/csrc/sm100.cuh")}
 
 
@@ -554,20 +559,23 @@ def run_decode(args, rank, world, device):
     io_bytes = cache_bytes + 2 * q.numel() * 2 + lse.numel() * 4  # + q read, O and lse written
     gbs = world * io_bytes / (ms * 1e-3) / 1e9
     pk, pk_kind = peaks()
+    workload = f"decode B={B} Hq={Hq} Hkv={Hkv} Nq={Nq} d={d} L={L} page=64"
     return {
         "metric": "paged-KV decode: cache bytes read per second", "value": round(gbs, 1),
         "unit": "GB/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bfloat16",
         "data": "synthetic: seeded normals, pages of 64 tokens in a shuffled pool",
-        "config": {"workload": f"decode B={B} Hq={Hq} Hkv={Hkv} Nq={Nq} d={d} L={L} page=64",
+        "config": {"workload": workload,
                    "parallelism": f"replicas x{world} (no exchange)",
                    "l2": "cache larger than L2 (no flush)" if cache_bytes > 126e6 else "cache fits L2"},
         "tokens_per_s": round(world * B * Nq / (ms * 1e-3), 1),
         "roofline": {"kernel": "fa_decode_split_kernel + fa_decode_merge_kernel", "bound": "hbm",
                      "achieved": round(gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
                      "frac": round(gbs / pk["hbm_gbs"], 4), "peak_kind": f"{pk_kind} copy",
-                     "traffic": None, "algorithmic": "K and V cache read once, q read, O and lse written"},
+                     "traffic": profiled_traffic(workload, PROFILED_TRAFFIC_DEC),
+                     "traffic_unit": "bytes per step, split + merge (ncu)",
+                     "algorithmic": "K and V cache read once, q read, O and lse written"},
         "gpu_launches": 2 * K,
         "clocks": clk,
     }
