@@ -11,6 +11,7 @@
 #include <algorithm>
 #include <atomic>
 #include <mutex>
+#include <utility>
 
 #include "fa.h"
 #include "sm100.cuh"
@@ -147,6 +148,28 @@ fa_status_t opt_in_smem(K kernel, int smem) {
     done_dev[n_done++] = dev;
   }
   return FA_OK;
+}
+
+// Launches `kernel` as a programmatic dependent of the kernel before it on the
+// stream: it may be scheduled while that kernel still runs, and waits
+// (griddepcontrol.wait) before it touches global memory.  Used for the decode
+// pair (split, then merge), whose launch gap is a visible part of a step; on
+// the training path it measured slower and is not used.
+template <typename... Params, typename... Args>
+cudaError_t launch_dependent(void (*kernel)(Params...), unsigned grid, unsigned block, int smem,
+                             cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 template <int HD, bool BF, bool CA, bool DR, bool BM = false>
@@ -707,10 +730,13 @@ fa_status_t fa_decode_paged(const void* q, const void* k_cache, const void* v_ca
         per_sm <= 0)
       return FA_ERR_CUDA;
     const int grid = static_cast<int>(std::min<int64_t>(n_work, static_cast<int64_t>(sms) * per_sm));
-    split_kern<<<grid, fa::kDecodeThreads, smem, st>>>(prm);
-    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
-    merge_kern<<<static_cast<unsigned>(rows), d, 0, st>>>(prm);
-    return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+    if (launch_dependent(split_kern, static_cast<unsigned>(grid), fa::kDecodeThreads, smem, st, prm) !=
+        cudaSuccess)
+      return FA_ERR_CUDA;
+    return launch_dependent(merge_kern, static_cast<unsigned>(rows), static_cast<unsigned>(d), 0, st, prm) ==
+                   cudaSuccess
+               ? FA_OK
+               : FA_ERR_CUDA;
   };
 #define FA_DECODE_RUN(HD, BFV, RBV)                                                                  \
   run(fa::fa_decode_split_kernel<HD, BFV, RBV>, fa::fa_decode_merge_kernel<HD, BFV>, \

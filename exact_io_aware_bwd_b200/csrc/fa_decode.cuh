@@ -189,6 +189,19 @@ __device__ __forceinline__ DecodeItem decode_item(const DecodeParams& p, int w) 
 // the ring and the pipeline's start are paid once per block, not per split.
 // RB: compile-time bound on the rows (4, 8, 16 or 32, the smallest >= R), so
 // the per-row loops unroll to the rows that exist.
+// Programmatic dependent launch: the split and merge kernels are launched as
+// dependents of the kernel before them on the stream, so that each may be
+// scheduled (and run its set-up) while that kernel still runs.
+// Lets the next kernel, if launched as a dependent, be scheduled now.
+__device__ __forceinline__ void grid_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+// Waits until the kernels this one depends on have completed and their
+// memory is visible (returns at once when launched without the dependency).
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 template <int HD, bool BF16, int RB>
 __global__ void __launch_bounds__(kDecodeThreads, 1) fa_decode_split_kernel(const __grid_constant__ DecodeParams p) {
   using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
@@ -240,6 +253,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) fa_decode_split_kernel(cons
     tmem_alloc(tmem_ptr, 128);
     tmem_relinquish();
   }
+  // The set-up above may overlap the previous kernel on the stream; no
+  // global memory is touched before this wait.
+  grid_dependency_wait();
+  grid_launch_dependents();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -544,6 +561,8 @@ __global__ void __launch_bounds__(HD) fa_decode_merge_kernel(const __grid_consta
   using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
   const size_t row = blockIdx.x;  // (b * Hq + h) * Nq + t
   const int c = threadIdx.x;
+  grid_dependency_wait();  // the splits' partial rows are complete and visible
+  grid_launch_dependents();
   const float* ml = p.part_ml + row * p.S * 2;
   float m_star = -INFINITY;
   for (int s = 0; s < p.S; ++s) m_star = fmaxf(m_star, ml[2 * s]);
