@@ -59,8 +59,8 @@ PROFILED_TRAFFIC_FP8 = {"workload": "mha4k", "bytes": 305240832, "sources_sha256
                         "sources": ("exact_io_aware_bwd_b200/csrc/fa_fwd_fp8.cuh",
                                     "exact_io_aware_bwd_b200/csrc/sm100.cuh")}
 # The same for one decode step (split and merge launch) at 16K cached tokens.
-PROFILED_TRAFFIC_DEC = {"workload": "decode B=32 Hq=32 Hkv=8 Nq=1 d=128 L=16384 page=64", "bytes": 2155432448,
-                        "sources_sha256_16": "028c681ba0cdedd6",
+PROFILED_TRAFFIC_DEC = {"workload": "decode B=32 Hq=32 Hkv=8 Nq=1 d=128 L=16384 page=64", "bytes": 2155173376,
+                        "sources_sha256_16": "63499268775b3e64",
                         "sources": ("exact_io_aware_bwd_b200/csrc/fa_decode.cuh",
                                     "exact_io_aware_bwd_b200/csrc/sm100.cuh")}
 
