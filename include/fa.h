@@ -240,6 +240,10 @@ fa_status_t fa_bwd_blockmask(const void* q, const void* k, const void* v, const 
  * seq_lens entry outside [Nq, max_pages * page_size] or a block-table
  * entry outside [0, num_pages) is detected on the device (nothing out of
  * range is read) and reported by fa_get_device_status as FA_ERR_INVALID_ARG.
+ * Two kernels run on `stream`, launched as programmatic dependents of the
+ * work before them: each may be scheduled while the previous kernel on the
+ * stream still runs, and waits for it to complete before reading or writing
+ * any global memory, so stream order holds as for a plain launch.
  */
 size_t fa_decode_workspace_bytes(int B, int Hq, int Hkv, int Nq, int d, int max_pages);
 fa_status_t fa_decode_paged(const void* q, const void* k_cache, const void* v_cache,
