@@ -528,7 +528,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
             for (int i = 0; i < 8; ++i)
               mx[i] = max3f(mx[i], __uint_as_float(s[c + i]), __uint_as_float(s[c + 8 + i]));
           m_new = max3f(max3f(mx[0], mx[1], mx[2]), max3f(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) * c_log2;
-          if (!DROP && j > 0) {
+          if (j > 0) {
             // speculative: keys 0-63 against the current reference
             const float m_use = m_ref == -INFINITY ? 0.f : m_ref;
             const uint64_t nm2 = f2pack(-m_use, -m_use);
@@ -548,7 +548,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
               hand_over(1);
               done = true;
             }
-          } else if (!DROP) {
+          } else {
             // first tile of the rows: the reference is this tile's max, and
             // the scores are still in registers
             m_ref = m_new;
