@@ -89,7 +89,8 @@ def test_profiled_traffic_is_reported_only_for_the_profiled_sources():
     """The bench reports an ncu traffic figure only while the kernel sources
     still hash to the digest recorded with it, and only for its workload."""
     import bench
-    for spec in (bench.PROFILED_TRAFFIC, bench.PROFILED_TRAFFIC_FP8):
+    for spec in (bench.PROFILED_TRAFFIC, bench.PROFILED_TRAFFIC_FWD, bench.PROFILED_TRAFFIC_FP8,
+                 bench.PROFILED_TRAFFIC_DEC):
         got = bench.profiled_traffic(spec["workload"], spec)
         assert got in (None, spec["bytes"])
         assert bench.profiled_traffic("tiny", spec) is None
