@@ -310,3 +310,62 @@ def test_memory_linear_in_n():
     ratios = [b / a for a, b in zip(peaks, peaks[1:])]
     print("peak bytes", peaks, "ratios", ratios)
     assert all(1.9 <= r <= 2.1 for r in ratios), ratios
+
+
+def _random_cases(n, seed):
+    """Seeded shapes across the supported range: tiny and ragged sequence
+    lengths (1, 7, one short of and one past a block), MHA / GQA / MQA, both
+    head dimensions, both 16-bit dtypes, causal or not."""
+    g = np.random.default_rng(seed)
+    lengths = [1, 2, 7, 63, 64, 65, 127, 128, 129, 191, 255, 257, 300, 383, 511, 640]
+    cases = []
+    for _ in range(n):
+        hkv = int(g.integers(1, 4))
+        group = int(g.choice([1, 2, 3, 4]))
+        cases.append(((int(g.integers(1, 4)), hkv * group, hkv, int(g.choice(lengths)),
+                       int(g.choice([64, 128]))),
+                      torch.bfloat16 if g.random() < 0.6 else torch.float16, bool(g.random() < 0.5)))
+    return cases
+
+
+RANDOM_CASES = _random_cases(24, seed=2026)
+
+
+@pytest.mark.parametrize("shape,dtype,causal", RANDOM_CASES,
+                         ids=[f"{'x'.join(map(str, s))}-{str(t)[6:]}-{'c' if c else 'nc'}"
+                              for s, t, c in RANDOM_CASES])
+def test_parity_random_shapes(shape, dtype, causal):
+    """Every output element against the oracle on a seeded sweep of shapes,
+    including sequences shorter than one block and ragged tails."""
+    q, k, v, do = _inputs(shape, dtype, seed=sum(shape) * 31 + causal)
+    scale = 1.0 / math.sqrt(shape[-1])
+    out = ac.run_gpu(q, k, v, do, scale, causal)
+    ac.check_full(q, k, v, do, scale, causal, out)
+
+
+RANDOM_WINDOW_CASES = [(s, t, int(w)) for (s, t, _), w in zip(
+    _random_cases(10, seed=2027), np.random.default_rng(2028).choice([1, 17, 64, 100, 128, 200, 257, 700], 10))]
+
+
+@pytest.mark.parametrize("shape,dtype,window", RANDOM_WINDOW_CASES,
+                         ids=[f"{'x'.join(map(str, s))}-{str(t)[6:]}-w{w}" for s, t, w in RANDOM_WINDOW_CASES])
+def test_parity_random_window(shape, dtype, window):
+    q, k, v, do = _inputs(shape, dtype, seed=sum(shape) * 37 + window)
+    scale = 1.0 / math.sqrt(shape[-1])
+    out = ac.run_gpu(q, k, v, do, scale, True, window=window)
+    ac.check_full(q, k, v, do, scale, True, out, window=window)
+
+
+RANDOM_DROPOUT_CASES = [(s, t, c, float(p_), int(sd)) for (s, t, c), p_, sd in zip(
+    _random_cases(8, seed=2029), np.random.default_rng(2030).choice([0.05, 0.1, 0.3, 0.5], 8),
+    np.random.default_rng(2031).integers(0, 2**62, 8))]
+
+
+@pytest.mark.parametrize("shape,dtype,causal,p_drop,seed", RANDOM_DROPOUT_CASES,
+                         ids=[f"{'x'.join(map(str, s))}-{str(t)[6:]}-{'c' if c else 'nc'}-p{p_}"
+                              for s, t, c, p_, _ in RANDOM_DROPOUT_CASES])
+def test_parity_random_dropout(shape, dtype, causal, p_drop, seed):
+    q, k, v, do = _inputs(shape, dtype, seed=sum(shape) * 41 + int(p_drop * 100))
+    scale = 1.0 / math.sqrt(shape[-1])
+    out = ac.run_gpu(q, k, v, do, scale, causal, dropout=(p_drop, seed))
+    ac.check_full(q, k, v, do, scale, causal, out, dropout=(p_drop, seed))
