@@ -67,6 +67,72 @@ def test_decode_paged_parity(case):
     ac.check_lse(lse.cpu(), lse_r, what="decode lse")
 
 
+LONG_LENGTHS = [16, 17, 63, 64, 65, 127, 128, 129, 255, 500, 1023, 1024, 1025, 3000]
+SHORT_LENGTHS = [1, 2, 3, 5, 8, 15]
+
+
+def _random_decode_cases(n, seed, lengths):
+    """Seeded decode shapes within the supported range: (Hq / Hkv) * Nq <= 32
+    rows a kv head, d 64 or 128, pages of 16 to 128 tokens, sequence lengths
+    drawn from `lengths` (at least Nq)."""
+    g = np.random.default_rng(seed)
+    cases = []
+    while len(cases) < n:
+        Hkv = int(g.choice([1, 2, 4, 8]))
+        G = int(g.choice([1, 2, 4, 8]))
+        Nq = int(g.choice([1, 2, 3, 4]))
+        if G * Nq > 32:
+            continue
+        P = int(g.choice([16, 32, 64, 128]))
+        B = int(g.integers(1, 5))
+        lens = tuple(int(max(Nq, x)) for x in g.choice(lengths, B))
+        cases.append((B, Hkv * G, Hkv, Nq, int(g.choice([64, 128])), P, lens,
+                      torch.bfloat16 if g.random() < 0.6 else torch.float16))
+    return cases
+
+
+RANDOM_CASES = _random_decode_cases(16, seed=3030, lengths=LONG_LENGTHS)
+
+
+@pytest.mark.parametrize("case", RANDOM_CASES,
+                         ids=[f"B{c[0]}-H{c[1]}/{c[2]}-Nq{c[3]}-d{c[4]}-P{c[5]}-{str(c[7])[6:]}-r{i}"
+                              for i, c in enumerate(RANDOM_CASES)])
+def test_decode_random_shapes(case):
+    """Every output of a seeded sweep of decode shapes (sequences of 16 tokens
+    and more) against the oracle, O within 1e-2."""
+    test_decode_paged_parity(case)
+
+
+SHORT_CASES = _random_decode_cases(8, seed=3031, lengths=SHORT_LENGTHS)
+
+
+@pytest.mark.parametrize("case", SHORT_CASES,
+                         ids=[f"B{c[0]}-H{c[1]}/{c[2]}-Nq{c[3]}-d{c[4]}-P{c[5]}-{str(c[7])[6:]}-s{i}"
+                              for i, c in enumerate(SHORT_CASES)])
+def test_decode_short_sequences_known_exceedance(case):
+    """Known exceedance of the O tolerance, reported rather than absorbed.
+
+    A query of a sequence of one to fifteen cached tokens averages a few rows
+    of V, so |O| reaches 2-4, where half an ulp of a bf16 output is
+    0.0078-0.0156; with P rounded to the I/O dtype before the P V product an
+    element can end just above 1e-2 by rounding alone (0.01005 met on a
+    2-token sequence).  These cases are held to the a-priori rounding bound
+    of the 16-bit path, element by element, and print how many elements are
+    above 1e-2; lse keeps its stated tolerance."""
+    B, Hq, Hkv, Nq, d, P, lens, dtype = case
+    q, kc, vc, table, seq_lens = make_case(sum(lens) + d + P + 1, B, Hq, Hkv, Nq, d, P, lens, dtype)
+    scale = 1.0 / math.sqrt(d)
+    dev = "cuda:0"
+    o, lse = binding.attention_decode_paged(q.to(dev), kc.to(dev), vc.to(dev), table.to(dev),
+                                            seq_lens.to(dev), scale)
+    assert binding.fa_get_device_status() == binding.FA_OK
+    o_r, lse_r = oracle.decode_paged(q, kc, vc, table.numpy(), seq_lens.numpy(), scale)
+    o_abs, _ = oracle.decode_paged(q, kc, vc.abs(), table.numpy(), seq_lens.numpy(), scale)
+    info = ac.check_o_rounding_bound(o.cpu(), o_r, dtype, o_abs, what="decode O")
+    print("short sequences, O against the rounding bound:", info)
+    ac.check_lse(lse.cpu(), lse_r, what="decode lse")
+
+
 def test_decode_long_sequences_many_splits():
     """The bench shape's heads and GQA group at 16K and 5K cached tokens: many
     128-key tiles per split, several splits per sequence, a last tile that
