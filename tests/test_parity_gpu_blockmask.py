@@ -203,3 +203,29 @@ def test_blockmask_at_4k_rows_and_columns():
     ac.check_grad(out["dk"][0, 2][cols], dk_r, "dK cols")
     ac.check_grad(out["dv"][0, 2][cols], dv_r, "dV cols")
     ac.check_invariants(q, k, do, out)
+
+
+def _random_mask_cases(n, seed):
+    """Seeded shapes and mask kinds: MHA / GQA / MQA, d 64 or 128, sequences
+    from under one block to several blocks with ragged tails, causal or not."""
+    g = np.random.default_rng(seed)
+    kinds = ["random-head", "random-shared", "sparse-head", "local-global", "dilated"]
+    lengths = [1, 100, 128, 129, 255, 300, 511, 700]
+    cases = []
+    for i in range(n):
+        hkv = int(g.integers(1, 4))
+        cases.append(((int(g.integers(1, 3)), hkv * int(g.choice([1, 2, 4])), hkv, int(g.choice(lengths)),
+                       int(g.choice([64, 128]))),
+                      torch.bfloat16 if g.random() < 0.6 else torch.float16, bool(g.random() < 0.5),
+                      str(g.choice(kinds)), 100 + i))
+    return cases
+
+
+RANDOM_MASK_CASES = _random_mask_cases(10, seed=5050)
+
+
+@pytest.mark.parametrize("shape,dtype,causal,kind,seed", RANDOM_MASK_CASES,
+                         ids=[f"{'x'.join(map(str, s))}-{str(t)[6:]}-{'c' if c else 'nc'}-{k}-r{sd}"
+                              for s, t, c, k, sd in RANDOM_MASK_CASES])
+def test_parity_blockmask_random(shape, dtype, causal, kind, seed):
+    test_parity_blockmask(shape, dtype, causal, kind, seed)

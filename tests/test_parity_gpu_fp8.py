@@ -139,3 +139,26 @@ def test_fp8_forward_4k_workload_rows():
     o, lse = _run(q8, k8, v8, ds, w.scale, True, torch.bfloat16)
     rows = check_rows(w)[::8].numpy()
     print(_check(q8, k8, v8, ds, w.scale, True, o, lse, rows=rows))
+
+
+def _random_fp8_cases(n, seed):
+    """Seeded FP8 forward shapes: d = 128, MHA / GQA / MQA, sequences from one
+    token to several blocks with ragged tails, causal or not, bf16 or fp16 O."""
+    g = np.random.default_rng(seed)
+    lengths = [1, 2, 7, 64, 65, 127, 128, 129, 255, 300, 511, 700]
+    cases = []
+    for _ in range(n):
+        hkv = int(g.integers(1, 4))
+        cases.append(((int(g.integers(1, 4)), hkv * int(g.choice([1, 2, 4])), hkv, int(g.choice(lengths)), 128),
+                      bool(g.random() < 0.5), torch.bfloat16 if g.random() < 0.6 else torch.float16))
+    return cases
+
+
+RANDOM_FP8_CASES = _random_fp8_cases(10, seed=4040)
+
+
+@pytest.mark.parametrize("shape,causal,out_dtype", RANDOM_FP8_CASES,
+                         ids=[f"{'x'.join(map(str, s))}-{'c' if c else 'nc'}-{str(t)[6:]}-r{i}"
+                              for i, (s, c, t) in enumerate(RANDOM_FP8_CASES)])
+def test_fp8_forward_random_shapes(shape, causal, out_dtype):
+    test_fp8_forward_full(shape, causal, out_dtype)
