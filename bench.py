@@ -51,7 +51,7 @@ PROFILED_TRAFFIC = {"workload": "mha4k", "bytes": 1295312384, "sources_sha256_16
                     "sources": ("exact_io_aware_bwd_b200/csrc/fa_bwd.cuh",
                                 "exact_io_aware_bwd_b200/csrc/sm100.cuh")}
 # The same for the forward kernel (one launch on the default workload).
-PROFILED_TRAFFIC_FWD = {"workload": "mha4k", "bytes": 522084864, "sources_sha256_16": "de54dac4b5120482",
+PROFILED_TRAFFIC_FWD = {"workload": "mha4k", "bytes": 516944128, "sources_sha256_16": "404444234fe2e56c",
                         "sources": ("exact_io_aware_bwd_b200/csrc/fa_fwd.cuh",
                                     "exact_io_aware_bwd_b200/csrc/sm100.cuh")}
 # The same for the FP8 forward kernel (one launch on the 4K-token MHA shape).
